@@ -1,0 +1,254 @@
+/*
+ * nvfp4qad.h -- C ABI of libnvfp4qad.so, the B200 (sm_100a) hot path of NVFP4
+ * quantization-aware distillation (QAD).
+ *
+ * What the operations are, and where they are defined:
+ *
+ *  NVFP4 is a 4-bit floating-point element (E2M1: values 0, 0.5, 1, 1.5, 2,
+ *  3, 4, 6 with a sign bit) stored in blocks of 16 consecutive elements, each
+ *  block with an E4M3 (FP8) scale, and one FP32 scale per tensor ("two-level
+ *  scaling") -- Nemotron-3-Nano-30B NVFP4 article, section "NVFP4-Format und
+ *  warum es wichtig ist?" and "Wichtige Erkenntnisse".
+ *
+ *  QAD runs every student forward pass through simulated (fake) quantization
+ *  and trains the student to match a frozen BF16 teacher through a KL
+ *  divergence between their output-token distributions -- Nemotron 3.5
+ *  Lightning NVFP4 article, section "QAD的工作原理"; Nemotron-3-Nano article,
+ *  "Von QAT zu QAD".  Scales are either recomputed from the max every step
+ *  (dynamic-scale QAD) or taken from calibration and held fixed (frozen-scale
+ *  QAD) -- Nemotron 3.5 Lightning article, "量化尺度处理策略".
+ *
+ *  W4A4: weights and activations are both NVFP4, so the linear layer is a
+ *  block-scaled FP4 x FP4 GEMM on the FP4 tensor cores -- Qwen3.6-35B-A3B
+ *  W4A4 NVFP4 tutorial page, "为什么目标是 W4A4".
+ *
+ * Numerical definitions (identical on every entry point):
+ *   per-tensor scale (decode direction)  s_g = amax(|x|) / 2688   (2688 = 6*448)
+ *   per-block scale  (E4M3, RNE, saturating at 448)
+ *                    s_b = E4M3( max_{block}|x| / (6 * s_g) ),  s_b = 0 if s_g = 0
+ *   decode scale     d   = float(s_b) * s_g                     (binary32)
+ *   element code     q   = E2M1( x / d )  RNE, |.| >= 6 -> 6, sign kept;
+ *                    q   = +0 for every element of a block with d = 0
+ *   dequantized      x^  = value(q) * d                         (binary32, then
+ *                                                                 bf16 RNE)
+ *   Each binary32 operation above is rounded once (no fused multiply-add), so
+ *   codes and scales are reproducible bit for bit.
+ *
+ * Conventions:
+ *   - Every function returns nvfp4_status; NVFP4_OK is 0.  Argument checks
+ *     run on the host and fail before anything is launched.
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, unless
+ *     the parameter says "host".  The library never allocates device memory;
+ *     scratch is passed as (workspace, workspace_bytes), sized by the
+ *     *_workspace_size() query of the same operation.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t, passed as
+ *     void*; NULL is the legacy default stream) and never synchronizes,
+ *     except nvfp4_device_error().
+ *   - Matrices are row-major with a row stride `ld` counted in elements of
+ *     their own type (bytes for uint8 code arrays).  Quantization blocks run
+ *     along the last (contiguous) dimension, so `cols` must be a multiple of
+ *     16; base pointers must be 16-byte aligned and ld * element size a
+ *     multiple of 16 bytes.
+ *   - Inputs must be finite; non-finite inputs give NVFP4_OK and unspecified
+ *     outputs.
+ *   - Packed codes: byte j of a row holds element 2j in its low nibble and
+ *     element 2j+1 in its high nibble.
+ */
+#ifndef NVFP4QAD_H
+#define NVFP4QAD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define NVFP4QAD_ABI_VERSION 1
+
+typedef enum nvfp4_status {
+  NVFP4_OK = 0,
+  NVFP4_ERR_ARG = 1,       /* NULL pointer where one is required, bad enum, T <= 0 */
+  NVFP4_ERR_SHAPE = 2,     /* negative or unsupported sizes (e.g. cols % 16 != 0) */
+  NVFP4_ERR_ALIGN = 3,     /* pointer or row stride not 16-byte aligned           */
+  NVFP4_ERR_DTYPE = 4,     /* dtype not supported by this entry point             */
+  NVFP4_ERR_CUDA = 5,      /* a CUDA runtime call or launch failed                */
+  NVFP4_ERR_TIMEOUT = 6,   /* a bounded device-side wait expired                  */
+  NVFP4_ERR_DEVICE = 7,    /* device reported an error word (see nvfp4_device_error) */
+  NVFP4_ERR_WORKSPACE = 8, /* workspace missing or smaller than the size query    */
+  NVFP4_ERR_UNSUPPORTED = 9 /* no kernel for this device / configuration          */
+} nvfp4_status;
+
+typedef enum nvfp4_dtype { NVFP4_BF16 = 0, NVFP4_F32 = 1 } nvfp4_dtype;
+
+/* Scale strategy of the two QAD variants (Nemotron 3.5 Lightning article,
+ * "量化尺度处理策略"):
+ *   DYNAMIC       s_g and every s_b recomputed from the data on each call
+ *                 (dynamic-scale QAD; *tensor_scale is written).
+ *   FROZEN_GLOBAL s_g given (a calibrated activation amax / 2688), s_b derived
+ *                 per block: activations in frozen-scale QAD, whose blocks are
+ *                 per token and cannot be calibrated ahead of time.
+ *   FROZEN_ALL    s_g and s_b both given (frozen-scale QAD weights: "only the
+ *                 weights are updated"). */
+typedef enum nvfp4_scale_mode {
+  NVFP4_DYNAMIC = 0,
+  NVFP4_FROZEN_GLOBAL = 1,
+  NVFP4_FROZEN_ALL = 2
+} nvfp4_scale_mode;
+
+/* Block-scale array layout.
+ *   ROWMAJOR  uint8 [rows][cols/16], row stride cols/16 bytes.
+ *   MMA       the layout the block-scaled tensor-core MMA reads: tiles of 128
+ *             rows x 4 blocks (512 bytes), tiles ordered block-index fastest,
+ *             row r / block kb of a tile at byte (r%32)*16 + (r/32)*4 + kb;
+ *             size nvfp4_mma_scales_bytes(rows, cols); padding bytes (rows
+ *             beyond `rows`, blocks beyond cols/16) are written as 0 by the
+ *             quantizer and never affect a GEMM output that is stored. */
+typedef enum nvfp4_scale_layout { NVFP4_SCALES_ROWMAJOR = 0, NVFP4_SCALES_MMA = 1 } nvfp4_scale_layout;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* nvfp4_status_string(nvfp4_status status);
+
+/* NVFP4QAD_ABI_VERSION of the loaded library. */
+int nvfp4_abi_version(void);
+
+/* Bytes of an MMA-layout block-scale array for a rows x cols tensor:
+ * ceil(rows/128)*128 * ceil(cols/64)*4. */
+size_t nvfp4_mma_scales_bytes(int64_t rows, int64_t cols);
+
+/* Synchronize `stream`, then read and clear the library's device error word.
+ * *code_out (host, may be NULL) receives the raw word: 0 = none, otherwise a
+ * kernel-specific reason (1 = bounded wait expired).  Returns NVFP4_OK,
+ * NVFP4_ERR_TIMEOUT when a bounded wait expired, NVFP4_ERR_DEVICE for other
+ * words, NVFP4_ERR_CUDA if the synchronization failed. */
+nvfp4_status nvfp4_device_error(void* stream, int32_t* code_out);
+
+/* ------------------------------------------------------------------------
+ * Quantize (steps: tensor amax [DYNAMIC] -> block scale -> E2M1 encode and
+ * pack), NVFP4 definition of the Nemotron-3-Nano article, scale modes of the
+ * Nemotron 3.5 Lightning article.
+ *
+ *   x             rows x cols of `dtype` (bf16 or f32), row stride ld_x elements
+ *   mode          see nvfp4_scale_mode
+ *   tensor_scale  one float: written in DYNAMIC mode, read otherwise
+ *   block_scales  read in FROZEN_ALL mode, written otherwise; layout `layout`
+ *                 (FROZEN_ALL requires ROWMAJOR)
+ *   codes         rows x cols/2 bytes, row stride ld_codes bytes (>= cols/2)
+ *   workspace     >= nvfp4_quantize_workspace_size(rows, cols, mode) bytes,
+ *                 16-byte aligned; may be NULL when that size is 0.  Its
+ *                 contents on entry do not matter.
+ * In DYNAMIC mode two kernels run in stream order (a grid-wide amax, then
+ * the encode); no host synchronization and no device-to-host copy happen.
+ * rows == 0 is a no-op (DYNAMIC writes s_g = 0).
+ * ------------------------------------------------------------------------ */
+size_t nvfp4_quantize_workspace_size(int64_t rows, int64_t cols, nvfp4_scale_mode mode);
+
+nvfp4_status nvfp4_quantize(const void* x, nvfp4_dtype dtype, int64_t rows, int64_t cols,
+                            int64_t ld_x, nvfp4_scale_mode mode, float* tensor_scale,
+                            uint8_t* block_scales, nvfp4_scale_layout layout, uint8_t* codes,
+                            int64_t ld_codes, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* Self-test of the encode path's division.  The bf16 encoder divides each
+ * element by its block's decode scale d with a correctly rounded reciprocal
+ * of d and one FMA correction (Markstein) instead of a full IEEE division per
+ * element; this call checks that quotient against IEEE division (CUDA's
+ * __fdiv_rn) for every binary32 significand of d and every bf16 significand
+ * and sign of x, over the exponent offsets that give quotients in
+ * [2^-5, 2^4).  mismatches, first: device, 8 bytes each; on completion
+ * *mismatches holds the number of differing quotients (0 expected) and
+ * *first one of them encoded as (d significand << 16) | ((k + 8) << 8) | x
+ * index, or all ones.  Asynchronous on `stream`. */
+nvfp4_status nvfp4_selftest_division(uint64_t* mismatches, uint64_t* first, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Fake quantization: y = dequantize(quantize(x)) in one pass, the simulated
+ * quantization every student forward pass goes through (Nemotron 3.5
+ * Lightning article, "QAD的工作原理").  Bitwise equal to nvfp4_quantize
+ * followed by nvfp4_dequantize with the same scales.
+ *
+ *   x, y          rows x cols of `dtype`; y may alias x (same ld) -- the amax
+ *                 pass of DYNAMIC mode completes before any element is written
+ *   tensor_scale  written in DYNAMIC mode, read otherwise
+ *   block_scales  ROWMAJOR; read in FROZEN_ALL mode; otherwise written when
+ *                 non-NULL (so a later FROZEN_ALL call can reuse them)
+ * The straight-through estimator makes the backward pass the identity
+ * (dx = dy), so there is no backward entry point.
+ * ------------------------------------------------------------------------ */
+size_t nvfp4_fake_quant_workspace_size(int64_t rows, int64_t cols, nvfp4_scale_mode mode);
+
+nvfp4_status nvfp4_fake_quant(const void* x, nvfp4_dtype dtype, int64_t rows, int64_t cols,
+                              int64_t ld_x, nvfp4_scale_mode mode, float* tensor_scale,
+                              uint8_t* block_scales, void* y, int64_t ld_y, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Dequantize: out = value(q) * (float(s_b) * s_g), rounded to out_dtype.
+ *   codes         rows x cols/2 bytes, row stride ld_codes
+ *   block_scales  layout `layout`
+ *   tensor_scale  one float (device)
+ *   out           rows x cols of out_dtype, row stride ld_out elements
+ * ------------------------------------------------------------------------ */
+nvfp4_status nvfp4_dequantize(const uint8_t* codes, int64_t ld_codes, const uint8_t* block_scales,
+                              nvfp4_scale_layout layout, const float* tensor_scale, int64_t rows,
+                              int64_t cols, void* out, nvfp4_dtype out_dtype, int64_t ld_out,
+                              void* stream);
+
+/* ------------------------------------------------------------------------
+ * W4A4 GEMM: C = (s_gA * s_gB) * A^ * B^T, with A^ (M x K) and B^ (N x K)
+ * the block-scaled NVFP4 operands, FP32 accumulation on the tcgen05
+ * block-scaled FP4 tensor cores, bf16 output (RNE).  Qwen3.6-35B-A3B W4A4
+ * tutorial, "为什么目标是 W4A4" and "吞吐量".
+ *
+ *   a_codes        M x K/2 bytes, contiguous (row stride K/2)
+ *   a_scales_mma   A's block scales in the MMA layout (nvfp4_mma_scales_bytes(M, K))
+ *   a_tensor_scale one float (device)
+ *   b_codes        N x K/2 bytes, contiguous
+ *   b_scales_mma   B's block scales in the MMA layout (nvfp4_mma_scales_bytes(N, K))
+ *   b_tensor_scale one float (device)
+ *   c              M x N bf16, row stride ldc elements (>= N)
+ * Requires M, N >= 1, K >= 64 and K % 64 == 0.  Tails in M and N are
+ * handled (out-of-range rows read as zero, out-of-range outputs not stored).
+ * ------------------------------------------------------------------------ */
+size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+
+nvfp4_status nvfp4_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_scales_mma,
+                             const float* a_tensor_scale, const uint8_t* b_codes,
+                             const uint8_t* b_scales_mma, const float* b_tensor_scale, int64_t M,
+                             int64_t N, int64_t K, void* c, int64_t ldc, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * KL distillation loss, forward and backward in one pass (Nemotron 3.5
+ * Lightning article, "QAD的工作原理"; Nemotron-3-Nano article, "Von QAT zu
+ * QAD"; full-vocabulary form of the loss in the Qwen3.6 tutorial, section 3).
+ * With p = softmax(z / T) per row:
+ *   row_kl[i]   = sum_v p_t[i,v] * (log p_t[i,v] - log p_s[i,v])
+ *   *loss       = (1/rows) * sum_i row_kl[i]       (fixed summation order)
+ *   dlogits[i,v]= grad_scale * (p_s[i,v] - p_t[i,v]) / T
+ * (forward KL(teacher || student), mean over tokens, no T^2 factor).
+ *
+ *   teacher, student  rows x vocab of `dtype`, row stride ld elements
+ *   temperature       T > 0
+ *   loss              one float (device), required
+ *   row_kl            rows floats (device) or NULL
+ *   dlogits           rows x vocab of `dtype`, row stride ld_grad, or NULL
+ *                     (forward only)
+ *   grad_scale        multiplier of the gradient; 1/rows gives the gradient
+ *                     of *loss
+ *   workspace         >= qad_kl_workspace_size(rows, vocab, dtype) bytes
+ * Each logit is read from memory once; probabilities are never stored.
+ * ------------------------------------------------------------------------ */
+size_t qad_kl_workspace_size(int64_t rows, int64_t vocab, nvfp4_dtype dtype);
+
+nvfp4_status qad_kl_fwd_bwd(const void* teacher, const void* student, nvfp4_dtype dtype,
+                            int64_t rows, int64_t vocab, int64_t ld, float temperature,
+                            float* loss, float* row_kl, void* dlogits, int64_t ld_grad,
+                            float grad_scale, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4QAD_H */

@@ -1,0 +1,42 @@
+// api.cu -- library-wide entry points of libnvfp4qad: status strings, ABI
+// version and the device error word that bounded waits report into.
+#include "common.cuh"
+
+namespace nvfp4 {
+__device__ int g_device_error = 0;
+}
+
+extern "C" {
+
+const char* nvfp4_status_string(nvfp4_status status) {
+  switch (status) {
+    case NVFP4_OK: return "NVFP4_OK";
+    case NVFP4_ERR_ARG: return "NVFP4_ERR_ARG: invalid argument";
+    case NVFP4_ERR_SHAPE: return "NVFP4_ERR_SHAPE: unsupported shape";
+    case NVFP4_ERR_ALIGN: return "NVFP4_ERR_ALIGN: pointer or stride not aligned";
+    case NVFP4_ERR_DTYPE: return "NVFP4_ERR_DTYPE: unsupported dtype";
+    case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA: CUDA runtime or launch error";
+    case NVFP4_ERR_TIMEOUT: return "NVFP4_ERR_TIMEOUT: bounded device wait expired";
+    case NVFP4_ERR_DEVICE: return "NVFP4_ERR_DEVICE: device error word set";
+    case NVFP4_ERR_WORKSPACE: return "NVFP4_ERR_WORKSPACE: workspace missing or too small";
+    case NVFP4_ERR_UNSUPPORTED: return "NVFP4_ERR_UNSUPPORTED: no kernel for this device or configuration";
+  }
+  return "NVFP4 unknown status";
+}
+
+int nvfp4_abi_version(void) { return NVFP4QAD_ABI_VERSION; }
+
+nvfp4_status nvfp4_device_error(void* stream, int32_t* code_out) {
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  int word = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&word, nvfp4::g_device_error, sizeof(int)) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (word != 0 && cudaMemcpyToSymbol(nvfp4::g_device_error, &zero, sizeof(int)) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  if (code_out) *code_out = word;
+  if (word == 0) return NVFP4_OK;
+  return word == nvfp4::kErrWaitTimeout ? NVFP4_ERR_TIMEOUT : NVFP4_ERR_DEVICE;
+}
+
+}  // extern "C"

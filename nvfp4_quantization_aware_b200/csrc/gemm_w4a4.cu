@@ -1,0 +1,311 @@
+// gemm_w4a4.cu -- W4A4 block-scaled NVFP4 GEMM on the sm_100a tensor cores.
+//
+// W4A4 quantizes activations as well as weights, so the linear layer is an
+// FP4 x FP4 product that runs on the Blackwell FP4 tensor cores (Qwen3.6-35B-A3B
+// W4A4 NVFP4 tutorial page, "为什么目标是 W4A4" and "吞吐量"):
+//   C[m, n] = (s_gA * s_gB) * sum_k (q_A[m,k] s_bA[m,k/16]) (q_B[n,k] s_bB[n,k/16])
+// with E2M1 codes q, UE4M3 block scales s_b per 16 elements of K and FP32
+// tensor scales s_g (Nemotron-3-Nano-30B NVFP4 article, "NVFP4-Format und warum
+// es wichtig ist?").
+//
+// One CTA computes a 128 x BN output tile.  Warp roles:
+//   warp 0      TMA producer: per K stage (256 elements) the A tile
+//               (128 rows x 128 bytes) and B tile (BN rows x 128 bytes) as 2-D
+//               tiled TMA loads with 128-byte swizzle, and the stage's block
+//               scales as 1-D bulk copies (the MMA scale layout keeps each
+//               128-row x 4-block tile contiguous).  No cluster multicast.
+//   warp 1      allocates tensor memory, then one thread issues per stage:
+//               tcgen05.cp of the scales into tensor memory and four
+//               tcgen05.mma.kind::mxf4nvf4.block_scale (K = 64 each) into an
+//               FP32 accumulator in tensor memory; tcgen05.commit releases the
+//               stage back to the producer.
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator, x (s_gA s_gB), bf16
+//               rounding, stores.
+// STAGES-deep mbarrier ring between producer and MMA; every wait is bounded.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "ptx.cuh"
+
+namespace nvfp4 {
+
+template <int BN_>
+struct GemmCfg {
+  static constexpr int BM = 128;
+  static constexpr int BN = BN_;
+  static constexpr int BK = 256;                 // FP4 elements per stage (128 bytes per row)
+  static constexpr int KB_PER_STAGE = BK / 64;   // MMAs (K = 64) per stage
+  static constexpr int STAGES = 4;
+  static constexpr int A_BYTES = BM * BK / 2;
+  static constexpr int B_BYTES = BN * BK / 2;
+  static constexpr int NB_SFB = BN / 128;        // 128-row scale tiles of B per stage
+  static constexpr int SFA_BYTES = 512 * KB_PER_STAGE;
+  static constexpr int SFB_BYTES = 512 * KB_PER_STAGE * NB_SFB;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  // tensor-memory columns: accumulator, then two sets of scales (alternating
+  // by stage parity)
+  static constexpr int TM_ACC = 0;
+  static constexpr int TM_SFA = BN;                               // 2 x 4*KB columns
+  static constexpr int TM_SFB = BN + 2 * 4 * KB_PER_STAGE;        // 2 x 4*KB*NB_SFB columns
+  static constexpr int TM_COLS_USED = TM_SFB + 2 * 4 * KB_PER_STAGE * NB_SFB;
+  static constexpr int TM_COLS = TM_COLS_USED <= 256 ? 256 : 512;
+  static constexpr int THREADS = 192;
+  // instruction descriptor: E2M1 x E2M1 (format 1), UE4M3 scales, K-major A
+  // and B, N >> 3 in bits 17-22, M >> 4 in bits 24-28, dense K = 64.
+  static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+};
+
+struct GemmParams {
+  const uint8_t* a_sf;   // MMA layout
+  const uint8_t* b_sf;
+  const float* a_ts;
+  const float* b_ts;
+  __nv_bfloat16* c;
+  int64_t ldc;
+  int M, N, K;
+  int kchunks;           // K / 64
+  int b_rowtiles;        // ceil(N / 128): 128-row scale tiles present for B
+  int c_vec16;           // C base 16-byte aligned and ldc % 8 == 0: 16-byte stores
+};
+
+template <int BN>
+__global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
+    gemm_w4a4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
+  using C = GemmCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + C::STAGES * C::A_BYTES;
+  uint8_t* sSFA = sB + C::STAGES * C::B_BYTES;
+  uint8_t* sSFB = sSFA + C::STAGES * C::SFA_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + C::STAGES * C::SFB_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * C::BM;
+  const int n0 = blockIdx.x * C::BN;
+  const int num_kt = (p.kchunks + C::KB_PER_STAGE - 1) / C::KB_PER_STAGE;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_slot, C::TM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const int a_tile = m0 / 128;
+      for (int kt = 0; kt < num_kt; ++kt) {
+        const int s = kt % C::STAGES;
+        const uint32_t ph = (uint32_t)(kt / C::STAGES) & 1u;
+        if (!mbar_wait_bounded(&empty[s], ph ^ 1u)) { *abort_flag = 1; break; }
+        if (*abort_flag) break;
+        int nkc = p.kchunks - kt * C::KB_PER_STAGE;
+        if (nkc > C::KB_PER_STAGE) nkc = C::KB_PER_STAGE;
+        int nsfb = 0;
+        for (int j = 0; j < C::NB_SFB; ++j)
+          if (n0 / 128 + j < p.b_rowtiles) ++nsfb;
+        const uint32_t bytes = C::A_BYTES + C::B_BYTES + (uint32_t)nkc * 512u * (1u + (uint32_t)nsfb);
+        mbar_expect_tx(&full[s], bytes);
+        tma_load_2d(sA + s * C::A_BYTES, &tmA, kt * (C::BK / 2), m0, &full[s]);
+        tma_load_2d(sB + s * C::B_BYTES, &tmB, kt * (C::BK / 2), n0, &full[s]);
+        const int64_t kc0 = (int64_t)kt * C::KB_PER_STAGE;
+        bulk_g2s(sSFA + s * C::SFA_BYTES, p.a_sf + ((int64_t)a_tile * p.kchunks + kc0) * 512, (uint32_t)nkc * 512u,
+                 &full[s]);
+        for (int j = 0; j < nsfb; ++j)
+          bulk_g2s(sSFB + s * C::SFB_BYTES + j * 512 * C::KB_PER_STAGE,
+                   p.b_sf + ((int64_t)(n0 / 128 + j) * p.kchunks + kc0) * 512, (uint32_t)nkc * 512u, &full[s]);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t acc = tmem + C::TM_ACC;
+      for (int kt = 0; kt < num_kt; ++kt) {
+        const int s = kt % C::STAGES;
+        const uint32_t ph = (uint32_t)(kt / C::STAGES) & 1u;
+        if (!mbar_wait_bounded(&full[s], ph)) { *abort_flag = 1; break; }
+        if (*abort_flag) break;
+        tc_fence_after();
+        int nkc = p.kchunks - kt * C::KB_PER_STAGE;
+        if (nkc > C::KB_PER_STAGE) nkc = C::KB_PER_STAGE;
+        const int par = kt & 1;
+        const uint32_t sfa_col = tmem + C::TM_SFA + par * 4 * C::KB_PER_STAGE;
+        const uint32_t sfb_col = tmem + C::TM_SFB + par * 4 * C::KB_PER_STAGE * C::NB_SFB;
+        // scales: each 512-byte (128 rows x 4 blocks) tile -> 4 TMEM columns
+        for (int kb = 0; kb < nkc; ++kb) {
+          tc_cp_32x128b_warpx4(sfa_col + kb * 4, smem_desc(smem_u32(sSFA + s * C::SFA_BYTES + kb * 512), 0, 128, 0));
+#pragma unroll
+          for (int j = 0; j < C::NB_SFB; ++j)
+            tc_cp_32x128b_warpx4(sfb_col + kb * 4 * C::NB_SFB + j * 4,
+                                 smem_desc(smem_u32(sSFB + s * C::SFB_BYTES + j * 512 * C::KB_PER_STAGE + kb * 512), 0,
+                                           128, 0));
+        }
+        const uint32_t a_base = smem_u32(sA + s * C::A_BYTES);
+        const uint32_t b_base = smem_u32(sB + s * C::B_BYTES);
+        for (int kb = 0; kb < nkc; ++kb) {
+          // K = 64 FP4 elements = 32 bytes further along the 128-byte swizzled row
+          const uint64_t ad = smem_desc(a_base + kb * 32, 16, 1024, 2);
+          const uint64_t bd = smem_desc(b_base + kb * 32, 16, 1024, 2);
+          mma_fp4_block16(acc, ad, bd, C::IDESC, sfa_col + kb * 4, sfb_col + kb * 4 * C::NB_SFB,
+                          (kt > 0 || kb > 0) ? 1u : 0u);
+        }
+        tc_commit(&empty[s]);
+      }
+      tc_commit(acc_full);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int sub = warp & 3;                 // TMEM subpartition this warp may read
+    const int row = m0 + sub * 32 + lane;
+    bool ok = mbar_wait_bounded(acc_full, 0);
+    if (!ok) *abort_flag = 1;
+    tc_fence_after();
+    if (ok && !*abort_flag) {
+      const float alpha = __fmul_rn(__ldg(p.a_ts), __ldg(p.b_ts));
+      __nv_bfloat16* crow = p.c + (int64_t)row * p.ldc;
+#pragma unroll 1
+      for (int c0 = 0; c0 < C::BN; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem + C::TM_ACC + ((uint32_t)(sub * 32) << 16) + c0, r);
+        tmem_wait_ld();
+        if (row < p.M) {
+          const int col0 = n0 + c0;
+          uint32_t w[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            w[j] = pack_bf16x2(__uint_as_float(r[2 * j]) * alpha, __uint_as_float(r[2 * j + 1]) * alpha);
+          if (col0 + 32 <= p.N && p.c_vec16) {
+            uint4* dst = reinterpret_cast<uint4*>(crow + col0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          } else {
+            for (int j = 0; j < 32; ++j) {
+              if (col0 + j < p.N) {
+                const uint32_t h = (j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu);
+                crow[col0 + j] = __ushort_as_bfloat16((unsigned short)h);
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host
+
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Row-major uint8 matrix [rows][row_bytes] -> tensor map with a box of
+// box_rows x 128 bytes, 128-byte swizzle, zero fill out of bounds.
+static bool make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN>
+static nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* b, const GemmParams& p, cudaStream_t s) {
+  using C = GemmCfg<BN>;
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, a, p.M, p.K / 2, C::BM) || !make_tmap(&tb, b, p.N, p.K / 2, C::BN)) return NVFP4_ERR_CUDA;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(gemm_w4a4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+        cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    attr_set = true;
+  }
+  dim3 grid((p.N + C::BN - 1) / C::BN, (p.M + C::BM - 1) / C::BM);
+  gemm_w4a4_kernel<BN><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, p);
+  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" {
+
+size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
+  (void)M;
+  (void)N;
+  (void)K;
+  return 0;
+}
+
+nvfp4_status nvfp4_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_scales_mma, const float* a_tensor_scale,
+                             const uint8_t* b_codes, const uint8_t* b_scales_mma, const float* b_tensor_scale,
+                             int64_t M, int64_t N, int64_t K, void* c, int64_t ldc, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (M < 1 || N < 1 || K < 64 || K % 64 != 0 || ldc < N) return NVFP4_ERR_SHAPE;
+  if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return NVFP4_ERR_SHAPE;
+  if (!a_codes || !a_scales_mma || !a_tensor_scale || !b_codes || !b_scales_mma || !b_tensor_scale || !c)
+    return NVFP4_ERR_ARG;
+  auto a16 = [](const void* q) { return ((uintptr_t)q & 15u) == 0; };
+  if (!a16(a_codes) || !a16(b_codes) || !a16(a_scales_mma) || !a16(b_scales_mma) || ((uintptr_t)c & 3u))
+    return NVFP4_ERR_ALIGN;
+  GemmParams p;
+  p.a_sf = a_scales_mma;
+  p.b_sf = b_scales_mma;
+  p.a_ts = a_tensor_scale;
+  p.b_ts = b_tensor_scale;
+  p.c = reinterpret_cast<__nv_bfloat16*>(c);
+  p.ldc = ldc;
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.kchunks = (int)(K / 64);
+  p.b_rowtiles = (int)((N + 127) / 128);
+  p.c_vec16 = (((uintptr_t)c & 15u) == 0 && (ldc % 8) == 0) ? 1 : 0;
+  return launch_gemm<256>(a_codes, b_codes, p, (cudaStream_t)stream);
+}
+
+}  // extern "C"

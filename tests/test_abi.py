@@ -1,0 +1,83 @@
+"""The C-ABI library loads and exports every function declared in
+include/*.h; host-side argument validation returns its status before any
+CUDA call (no GPU needed)."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from nvfp4_quantization_aware_b200 import build
+    build.build()
+    import nvfp4_quantization_aware_b200 as Q
+    return Q.lib()
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"\b([a-z_][a-z0-9_]*)\s*\(", text):
+            name = m.group(1)
+            if name.startswith(("nvfp4_", "qad_")) and not name.endswith("_t"):
+                names.add(name)
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ["nvfp4_quantize", "nvfp4_fake_quant", "nvfp4_dequantize", "nvfp4_gemm_w4a4",
+                     "qad_kl_fwd_bwd", "nvfp4_status_string"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    path = lib._name
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = _declared_functions() - exported
+    assert not missing, missing
+    for name in _declared_functions():
+        assert hasattr(lib, name)
+
+
+def test_status_strings_and_version(lib):
+    assert lib.nvfp4_abi_version() == 1
+    for st in range(10):
+        s = lib.nvfp4_status_string(st)
+        assert s and s.startswith(b"NVFP4")
+
+
+def test_validation_before_launch(lib):
+    # cols not a multiple of 16 -> ERR_SHAPE; bad dtype -> ERR_DTYPE; NULL x -> ERR_ARG.
+    p = ctypes.c_void_p(16)
+    assert lib.nvfp4_quantize(p, 0, 4, 40, 40, 0, p, p, 0, p, 20, p, 4096, None) == 2
+    assert lib.nvfp4_quantize(p, 7, 4, 32, 32, 0, p, p, 0, p, 16, p, 4096, None) == 4
+    assert lib.nvfp4_quantize(None, 0, 4, 32, 32, 0, p, p, 0, p, 16, p, 4096, None) == 1
+    # unaligned x -> ERR_ALIGN; missing workspace in DYNAMIC -> ERR_WORKSPACE
+    assert lib.nvfp4_quantize(ctypes.c_void_p(18), 0, 4, 32, 32, 0, p, p, 0, p, 16, p, 4096, None) == 3
+    assert lib.nvfp4_quantize(p, 0, 4, 32, 32, 0, p, p, 0, p, 16, None, 0, None) == 8
+    # FROZEN_ALL with MMA layout is rejected
+    assert lib.nvfp4_quantize(p, 0, 4, 32, 32, 2, p, p, 1, p, 16, None, 0, None) == 1
+    assert lib.nvfp4_fake_quant(p, 0, 4, 32, 32, 2, p, None, p, 32, None, 0, None) == 1
+    assert lib.nvfp4_dequantize(p, 16, p, 0, p, 4, 33, p, 0, 33, None) == 2
+
+
+def test_mma_scales_bytes(lib):
+    import oracle as O
+    for rows, cols in [(1, 16), (128, 64), (129, 80), (8192, 4096)]:
+        assert lib.nvfp4_mma_scales_bytes(rows, cols) == O.swizzled_scale_bytes(rows, cols)
+
+
+def test_workspace_queries(lib):
+    assert lib.nvfp4_quantize_workspace_size(100, 64, 0) >= 4
+    assert lib.nvfp4_quantize_workspace_size(100, 64, 1) == 0
+    assert lib.nvfp4_quantize_workspace_size(100, 64, 2) == 0

@@ -1,0 +1,261 @@
+"""GPU parity of quantize / fake-quant / dequantize against the CPU oracle.
+
+Codes, block scales (both layouts), tensor scales and fake-quant outputs must
+be bit-exact; inputs come from the seeded generators, the oracle gets exact
+host copies of the same bits.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import nvfp4_quantization_aware_b200 as Q
+from nvfp4_quantization_aware_b200 import synthetic as S
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+MODES = [Q.DYNAMIC, Q.FROZEN_GLOBAL, Q.FROZEN_ALL]
+
+
+def _host_f32(x: torch.Tensor) -> np.ndarray:
+    return x.float().cpu().numpy()
+
+
+def _bits16(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _bits32(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.int32).cpu().numpy().view(np.uint32)
+
+
+def _frozen_inputs(xh):
+    """Scales for the frozen modes: a dynamic oracle pass (as calibration would
+    produce), so frozen calls see realistic s_g / s_b."""
+    codes, sb, sg = O.quantize(xh, O.DYNAMIC)
+    return sg, sb
+
+
+def _run_and_compare(x: torch.Tensor, mode: int, layout: int = Q.SCALES_ROWMAJOR):
+    xh = _host_f32(x)
+    rows, cols = x.shape
+    sg_in, sb_in = _frozen_inputs(xh)
+    if mode == Q.DYNAMIC:
+        ref_codes, ref_sb, ref_sg = O.quantize(xh, O.DYNAMIC)
+        ts = None
+        bs = None
+    elif mode == Q.FROZEN_GLOBAL:
+        ref_codes, ref_sb, ref_sg = O.quantize(xh, O.FROZEN_GLOBAL, s_g=sg_in * 1.25)
+        ts = torch.tensor([np.float32(sg_in * 1.25)], device=DEV)
+        bs = None
+    else:
+        # perturb the frozen block scales so they differ from what the data implies
+        sb_f = np.clip(sb_in.astype(np.int32) + (np.arange(sb_in.size).reshape(sb_in.shape) % 3) - 1, 0, 0x7E).astype(np.uint8)
+        ref_codes, ref_sb, ref_sg = O.quantize(xh, O.FROZEN_ALL, s_g=sg_in, s_b=sb_f)
+        ts = torch.tensor([np.float32(sg_in)], device=DEV)
+        bs = torch.from_numpy(sb_f).to(DEV)
+    codes, sbs, tsg = Q.nvfp4_quantize(x, mode=mode, tensor_scale=ts, block_scales=bs,
+                                       layout=layout if mode != Q.FROZEN_ALL else Q.SCALES_ROWMAJOR)
+    torch.cuda.synchronize()
+    assert np.array_equal(codes.cpu().numpy(), ref_codes), "codes differ"
+    assert _bits32(tsg)[0] == np.float32(ref_sg).view(np.uint32), "tensor scale differs"
+    if layout == Q.SCALES_MMA and mode != Q.FROZEN_ALL:
+        assert np.array_equal(sbs.cpu().numpy(), O.swizzle_scales(ref_sb, cols)), "MMA scales differ"
+    else:
+        assert np.array_equal(sbs.cpu().numpy(), ref_sb), "block scales differ"
+    return ref_codes, ref_sb, ref_sg
+
+
+SHAPES = [(1, 16), (3, 48), (17, 272), (64, 1024), (130, 1040), (5, 4096), (257, 64)]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_quantize_parity(shape, mode, dtype):
+    x = S.weights(*shape, seed=shape[0] * 7 + shape[1], device=DEV, outlier_p=0.01, outlier_mult=40, dtype=dtype)
+    _run_and_compare(x, mode)
+
+
+@pytest.mark.parametrize("shape", [(1, 16), (130, 1040), (300, 80), (128, 256)])
+@pytest.mark.parametrize("mode", [Q.DYNAMIC, Q.FROZEN_GLOBAL])
+def test_quantize_mma_layout_parity(shape, mode):
+    x = S.activations(*shape, seed=11 + shape[0], device=DEV)
+    _run_and_compare(x, mode, layout=Q.SCALES_MMA)
+
+
+def test_quantize_row_stride():
+    big = S.activations(33, 160, seed=3, device=DEV)
+    x = big[:, :96]
+    assert x.stride(0) == 160
+    ref_codes, ref_sb, ref_sg = O.quantize(_host_f32(x), O.DYNAMIC)
+    codes, sb, sg = Q.nvfp4_quantize(x)
+    assert np.array_equal(codes.cpu().numpy(), ref_codes) and np.array_equal(sb.cpu().numpy(), ref_sb)
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_fake_quant_parity(mode, dtype):
+    x = S.weights(96, 1040, seed=5, device=DEV, outlier_p=0.005, outlier_mult=30, dtype=dtype)
+    xh = _host_f32(x)
+    sg_in, sb_in = _frozen_inputs(xh)
+    if mode == Q.DYNAMIC:
+        ref32, ref16, ref_sb, ref_sg = O.fake_quant(xh)
+        y, sb, sg = Q.nvfp4_fake_quant(x, mode, return_scales=True)
+    elif mode == Q.FROZEN_GLOBAL:
+        ref32, ref16, ref_sb, ref_sg = O.fake_quant(xh, O.FROZEN_GLOBAL, s_g=sg_in)
+        y, sb, sg = Q.nvfp4_fake_quant(x, mode, tensor_scale=torch.tensor([sg_in], device=DEV), return_scales=True)
+    else:
+        ref32, ref16, ref_sb, ref_sg = O.fake_quant(xh, O.FROZEN_ALL, s_g=sg_in, s_b=sb_in)
+        sb_t = torch.from_numpy(sb_in).to(DEV)
+        y, sb, sg = Q.nvfp4_fake_quant(x, mode, tensor_scale=torch.tensor([sg_in], device=DEV), block_scales=sb_t,
+                                       return_scales=True)
+    torch.cuda.synchronize()
+    if dtype == torch.bfloat16:
+        assert np.array_equal(_bits16(y), ref16)
+    else:
+        assert np.array_equal(_bits32(y), ref32.view(np.uint32))
+    assert np.array_equal(sb.cpu().numpy(), ref_sb)
+    assert _bits32(sg)[0] == np.float32(ref_sg).view(np.uint32)
+
+
+def test_fake_quant_in_place_alias():
+    x = S.activations(64, 1024, seed=6, device=DEV)
+    ref32, ref16, _, _ = O.fake_quant(_host_f32(x))
+    Q.nvfp4_fake_quant(x, Q.DYNAMIC, out=x)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits16(x), ref16)
+
+
+def test_fake_quant_equals_gpu_dequant_of_quant():
+    x = S.weights(200, 512, seed=7, device=DEV)
+    y = Q.nvfp4_fake_quant(x)
+    codes, sb, sg = Q.nvfp4_quantize(x)
+    z = Q.nvfp4_dequantize(codes, sb, sg, 512)
+    zm = Q.nvfp4_dequantize(*Q.nvfp4_quantize(x, layout=Q.SCALES_MMA)[:2], sg, 512, layout=Q.SCALES_MMA)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), z.view(torch.int16))
+    assert torch.equal(y.view(torch.int16), zm.view(torch.int16))
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_dequantize_parity(out_dtype):
+    x = S.weights(77, 320, seed=8, device=DEV, outlier_p=0.01, outlier_mult=50)
+    codes, sb, sg = Q.nvfp4_quantize(x)
+    out = Q.nvfp4_dequantize(codes, sb, sg, 320, out_dtype=out_dtype)
+    ref32, ref16 = O.dequantize(codes.cpu().numpy(), sb.cpu().numpy(), float(sg.cpu()[0]), 320)
+    if out_dtype == torch.bfloat16:
+        assert np.array_equal(_bits16(out), ref16)
+    else:
+        assert np.array_equal(_bits32(out), ref32.view(np.uint32))
+
+
+def test_every_bf16_value_through_e2m1():
+    # FROZEN_ALL with s_g = 1 and s_b = 1.0 makes d = 1, so each code is the
+    # E2M1 rounding of the bf16 value itself: every finite bf16 pattern once.
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    f = (bits << 16).view(np.float32)
+    f = f[np.isfinite(f)]
+    pad = (-f.size) % 16
+    f = np.concatenate([f, np.zeros(pad, np.float32)]).reshape(-1, 16)
+    x = torch.from_numpy(f).to(torch.bfloat16).to(DEV)
+    sb = np.full((f.shape[0], 1), 0x38, np.uint8)
+    ref_codes, _, _ = O.quantize(f, O.FROZEN_ALL, s_g=1.0, s_b=sb)
+    codes, _, _ = Q.nvfp4_quantize(x, Q.FROZEN_ALL, tensor_scale=torch.ones(1, device=DEV),
+                                   block_scales=torch.from_numpy(sb).to(DEV))
+    assert np.array_equal(codes.cpu().numpy(), ref_codes)
+    # same values as f32 input (the f32 path divides with IEEE division)
+    codes32, _, _ = Q.nvfp4_quantize(x.float(), Q.FROZEN_ALL, tensor_scale=torch.ones(1, device=DEV),
+                                     block_scales=torch.from_numpy(sb).to(DEV))
+    assert np.array_equal(codes32.cpu().numpy(), ref_codes)
+
+
+def test_block_scale_rounding_sweep():
+    # Blocks [m, small...] for a sweep of maxima m: the block scale is
+    # E4M3(m / (6 s_g)), crossing every E4M3 rounding midpoint and saturation.
+    rng = np.random.default_rng(0)
+    table = O.e4m3_table()[:0x7F]
+    mids = (table[1:] + table[:-1]) / 2
+    sg = np.float32(1.0 / 6.0)
+    t = np.concatenate([mids, table, rng.uniform(0, 460, 4000), [448, 460, 470, 1e4]])
+    m = (t * 6.0 * float(sg)).astype(np.float32)
+    m = np.concatenate([m, np.nextafter(m, np.float32(0)), np.nextafter(m, np.float32(1e30))])
+    m = torch.from_numpy(m).to(torch.bfloat16).float().numpy()  # bf16-representable
+    blocks = np.zeros((m.size, 16), np.float32)
+    blocks[:, 0] = m
+    blocks[:, 5] = -m * 0.3
+    blocks[:, 9] = m * 0.77
+    blocks = torch.from_numpy(blocks).to(torch.bfloat16).float().numpy()  # what the kernel sees
+    x = torch.from_numpy(blocks).to(torch.bfloat16).to(DEV)
+    ref_codes, ref_sb, _ = O.quantize(blocks, O.FROZEN_GLOBAL, s_g=float(sg))
+    codes, sb, _ = Q.nvfp4_quantize(x, Q.FROZEN_GLOBAL, tensor_scale=torch.tensor([sg], device=DEV))
+    assert np.array_equal(sb.cpu().numpy(), ref_sb)
+    assert np.array_equal(codes.cpu().numpy(), ref_codes)
+
+
+def test_special_tensors():
+    # all zeros, negative zeros, tiny (subnormal s_g), huge magnitudes
+    cases = [
+        np.zeros((4, 32), np.float32),
+        -np.zeros((4, 32), np.float32),
+        (np.random.default_rng(1).standard_normal((8, 64)) * 1e-38).astype(np.float32),
+        (np.random.default_rng(2).standard_normal((8, 64)) * 1e37).astype(np.float32),
+    ]
+    for c in cases:
+        c = torch.from_numpy(c).to(torch.bfloat16).float().numpy()
+        x = torch.from_numpy(c).to(torch.bfloat16).to(DEV)
+        ref_codes, ref_sb, ref_sg = O.quantize(c, O.DYNAMIC)
+        codes, sb, sg = Q.nvfp4_quantize(x)
+        assert np.array_equal(codes.cpu().numpy(), ref_codes)
+        assert np.array_equal(sb.cpu().numpy(), ref_sb)
+        assert _bits32(sg)[0] == np.float32(ref_sg).view(np.uint32)
+        y32, y16, _, _ = O.fake_quant(c)
+        assert np.array_equal(_bits16(Q.nvfp4_fake_quant(x)), y16)
+
+
+def test_division_selftest_exhaustive():
+    mismatches, first = Q.nvfp4_selftest_division()
+    assert mismatches == 0, hex(first)
+
+
+def test_empty_tensor():
+    x = torch.empty(0, 64, dtype=torch.bfloat16, device=DEV)
+    codes, sb, sg = Q.nvfp4_quantize(x)
+    torch.cuda.synchronize()
+    assert codes.numel() == 0 and float(sg.cpu()[0]) == 0.0
+
+
+def test_bad_arguments_raise():
+    x = torch.zeros(4, 40, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(Q.NVFP4Error):
+        Q.nvfp4_quantize(x)
+    with pytest.raises(ValueError):
+        Q.nvfp4_quantize(torch.zeros(4, 32, dtype=torch.bfloat16))  # CPU tensor
+
+
+def test_weight_sweep_expert_parity():
+    # a slice of the MoE weight sweep at full expert size (2048 x 1024)
+    for i in (0, 77):
+        w = S.weights(2048, 1024, seed=i, device=DEV)
+        for mode in MODES:
+            _run_and_compare(w, mode)
+    _run_and_compare(S.weights(2048, 1024, seed=5, device=DEV), Q.DYNAMIC, layout=Q.SCALES_MMA)
+
+
+@pytest.mark.slow
+def test_weight_sweep_full_size_parity():
+    # The whole 128-expert + lm_head sweep, dynamic then frozen (scales from
+    # the dynamic pass), every code and scale compared.
+    O.set_threads(max(1, O.get_threads()))
+    ws = S.weight_sweep(seed=0, device=DEV)
+    for i, w in enumerate(ws):
+        if i % 16 != 0 and i != len(ws) - 1:
+            continue  # every 16th expert plus the 131072 x 2048 lm_head
+        xh = _host_f32(w)
+        ref_codes, ref_sb, ref_sg = O.quantize(xh, O.DYNAMIC)
+        codes, sb, sg = Q.nvfp4_quantize(w)
+        assert np.array_equal(codes.cpu().numpy(), ref_codes), i
+        assert np.array_equal(sb.cpu().numpy(), ref_sb), i
+        codes_f, _, _ = Q.nvfp4_quantize(w, Q.FROZEN_ALL, tensor_scale=sg, block_scales=sb)
+        assert torch.equal(codes_f, codes), i
