@@ -1,0 +1,498 @@
+#!/usr/bin/env python3
+"""Benchmark of the NVFP4 QAD hot path on B200.
+
+Headline workload (one JSON line on rank 0): the weight quantization sweep --
+128 MoE expert weights 2048 x 1024 plus one 131072 x 2048 lm_head, bf16,
+536,870,912 elements -- quantized to packed E2M1 codes + E4M3 block scales +
+FP32 tensor scales, first with dynamic scales (amax recomputed) and then with
+frozen scales (the dynamic pass's scales passed back in).  One step is both
+passes over all 129 tensors.  value = algorithmic bytes / device time, with
+2.5625 B per element and pass (2 B bf16 in, 0.5 B codes + 0.0625 B scales out;
+the frozen pass reads the 0.0625 B scales instead of writing them).
+
+Also measured in the same run and reported under "gemm" and "kl":
+  * W4A4 GEMM: activations M x 4096 (M = 8192 and 128) quantized on the fly,
+    weights 4096 x 4096 pre-quantized, bf16 out -- TFLOP/s;
+  * KL distillation loss + dLogits over 16384 x 131072 bf16 teacher/student
+    logits -- tokens/s and GB/s (6 B per logit).
+
+Timing: device time with CUDA events on the launching stream; the K timed
+steps are one CUDA-graph replay of K consecutive steps, bracketed by a
+barrier and synchronize; the maximum over ranks is reported.  Inputs are
+larger than L2 (1.07 GB), so no flush is needed between steps; the GEMM
+(25 MB of operands) is timed with an L2 flush before every launch.
+
+--impl reference times the CPU oracle (oracle/, test infrastructure) on the
+host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 quant GB/s & W4A4 GEMM TFLOPS (% of peak); QAD KL loss tokens/s"
+BYTES_PER_ELEM = 2.5625
+WORKLOAD = ("weight quantization sweep: 128 MoE experts 2048x1024 + lm_head 131072x2048 bf16, "
+            "NVFP4 dynamic then frozen (FROZEN_ALL) quantize to packed codes + E4M3 block scales")
+# ncu DRAM bytes (read + write) per launch of the dominant kernel, from the
+# capture summarised in profiles/; valid only while quantize.cu is unchanged.
+TRAFFIC = {"kernel": "group_encode_kernel<bf16,codes> (FROZEN_ALL, whole sweep)", "bytes": None,
+           "source_sha256": None}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def file_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason sampling during the measured region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[4:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [r for r in rows if r[0] > 600] or rows
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i in range(1, 5) if r[2][i].lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(load), "reasons": reasons}
+
+
+# --------------------------------------------------------------------------- distributed
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- our arm
+
+def make_sweep(rank, device):
+    from nvfp4_quantization_aware_b200 import synthetic as S
+    return S.weight_sweep(seed=1000 * rank, device=device)
+
+
+def run_ours(args, world, rank, local):
+    import nvfp4_quantization_aware_b200 as Q
+    dev = torch.device("cuda", local)
+    P = peaks()
+    sampler = ClockSampler(local)
+    xs = make_sweep(rank, dev)
+    n_elem = sum(x.numel() for x in xs)
+    n = len(xs)
+    ts = torch.zeros(n, dtype=torch.float32, device=dev)
+    sbs = [torch.empty(x.shape[0], x.shape[1] // 16, dtype=torch.uint8, device=dev) for x in xs]
+    codes_dyn = [torch.empty(x.shape[0], x.shape[1] // 2, dtype=torch.uint8, device=dev) for x in xs]
+    codes_fro = [torch.empty(x.shape[0], x.shape[1] // 2, dtype=torch.uint8, device=dev) for x in xs]
+    ws = torch.empty(int(Q.lib().nvfp4_grouped_workspace_size(Q.DYNAMIC)), dtype=torch.uint8, device=dev)
+
+    def step():
+        Q.nvfp4_quantize_grouped(xs, Q.DYNAMIC, tensor_scales=ts, block_scales=sbs, codes=codes_dyn, workspace=ws)
+        Q.nvfp4_quantize_grouped(xs, Q.FROZEN_ALL, tensor_scales=ts, block_scales=sbs, codes=codes_fro)
+
+    stream = torch.cuda.Stream(dev)
+    K, W = args.steps, args.warmup
+    sampler.start()
+    with torch.cuda.stream(stream):
+        for _ in range(W):
+            step()
+        stream.synchronize()
+        # capture K consecutive steps, with external timing events between passes
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(K)]
+        g = torch.cuda.CUDAGraph()
+        n0 = Q.nvfp4_launch_count()
+        with torch.cuda.graph(g, stream=stream):
+            for k in range(K):
+                evs[k][0].record(stream)
+                Q.nvfp4_quantize_grouped(xs, Q.DYNAMIC, tensor_scales=ts, block_scales=sbs, codes=codes_dyn,
+                                         workspace=ws)
+                evs[k][1].record(stream)
+                Q.nvfp4_quantize_grouped(xs, Q.FROZEN_ALL, tensor_scales=ts, block_scales=sbs, codes=codes_fro)
+                evs[k][2].record(stream)
+        launches = Q.nvfp4_launch_count() - n0
+        g.replay()  # untimed replay: warms the graph itself
+        stream.synchronize()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        g.replay()
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    total_ms = start.elapsed_time(end)
+    dyn_ms = [evs[k][0].elapsed_time(evs[k][1]) for k in range(K)]
+    fro_ms = [evs[k][1].elapsed_time(evs[k][2]) for k in range(K)]
+    del g
+    t_max = max_over_ranks(total_ms, world)
+    ms_per_step = t_max / K
+    units = sum_over_ranks(float(n_elem), world)
+    value = units * 2 * BYTES_PER_ELEM / (ms_per_step * 1e-3) / 1e9
+
+    # dominant kernel: the frozen pass is one launch of the encode kernel over
+    # the whole sweep (129 tensors <= one group)
+    fro_avg = statistics.mean(fro_ms)
+    dyn_avg = statistics.mean(dyn_ms)
+    achieved = n_elem * BYTES_PER_ELEM / (fro_avg * 1e-3) / 1e9
+    qsrc = os.path.join(ROOT, "nvfp4_quantization_aware_b200", "csrc", "quantize.cu")
+    traffic = TRAFFIC["bytes"] if TRAFFIC["source_sha256"] == file_sha(qsrc) else None
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": P["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / P["hbm_gbs"], 4), "traffic": traffic,
+                "kernel": TRAFFIC["kernel"], "peak_source": P["source"] + " (MEASURED_PEAKS hbm_gbs)",
+                "algorithmic_bytes_per_launch": n_elem * BYTES_PER_ELEM, "avg_launch_ms": round(fro_avg, 5)}
+    phases = {"dynamic_ms": round(dyn_avg, 4), "frozen_ms": round(fro_avg, 4),
+              "dynamic_gbs": round(n_elem * BYTES_PER_ELEM / (dyn_avg * 1e-3) / 1e9, 1),
+              "frozen_gbs": round(achieved, 1)}
+
+    # ---- end to end through the public API, host buffers, copies inside
+    e2e = run_e2e(Q, xs, dev, stream, min(K, 5), world)
+
+    secondary = {}
+    if not args.no_secondary:
+        secondary["gemm"] = bench_gemm(Q, dev, stream, P, max(3, min(K, 20)))
+        secondary["kl"] = bench_kl(Q, dev, stream, P, max(3, min(K, 10)))
+    clocks = sampler.stop()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(xs)
+
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "elements_per_gpu": n_elem, "tensors": n,
+                       "bytes_per_element_per_pass": BYTES_PER_ELEM,
+                       "l2": "inputs larger than L2 (1.07 GB of bf16 per GPU), no flush",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "timing": "CUDA events around one graph replay of K steps"},
+            "phases": phases, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": int(launches), "clocks": clocks}
+    line.update(secondary)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(Q, xs, dev, stream, K, world):
+    """Same metric through the public API with pinned host buffers: per step
+    the inputs are copied host -> device, both passes run, and the frozen
+    codes + block scales + tensor scales are copied back."""
+    hx = [x.cpu().pin_memory() for x in xs]
+    n = len(xs)
+    ts = torch.zeros(n, dtype=torch.float32, device=dev)
+    dx = [torch.empty_like(x) for x in xs]
+    sbs = [torch.empty(x.shape[0], x.shape[1] // 16, dtype=torch.uint8, device=dev) for x in xs]
+    cd = [torch.empty(x.shape[0], x.shape[1] // 2, dtype=torch.uint8, device=dev) for x in xs]
+    cf = [torch.empty_like(c) for c in cd]
+    hc = [torch.empty(c.shape, dtype=torch.uint8).pin_memory() for c in cd]
+    hs = [torch.empty(s.shape, dtype=torch.uint8).pin_memory() for s in sbs]
+    hts = torch.empty(n, dtype=torch.float32).pin_memory()
+    ws = torch.empty(int(Q.lib().nvfp4_grouped_workspace_size(Q.DYNAMIC)), dtype=torch.uint8, device=dev)
+
+    def step():
+        for d, h in zip(dx, hx):
+            d.copy_(h, non_blocking=True)
+        Q.nvfp4_quantize_grouped(dx, Q.DYNAMIC, tensor_scales=ts, block_scales=sbs, codes=cd, workspace=ws)
+        Q.nvfp4_quantize_grouped(dx, Q.FROZEN_ALL, tensor_scales=ts, block_scales=sbs, codes=cf)
+        for h, c in zip(hc, cf):
+            h.copy_(c, non_blocking=True)
+        for h, s in zip(hs, sbs):
+            h.copy_(s, non_blocking=True)
+        hts.copy_(ts, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        step()
+        stream.synchronize()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        for _ in range(K):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    ms = max_over_ranks(start.elapsed_time(end), world) / K
+    n_elem = sum(x.numel() for x in xs)
+    units = sum_over_ranks(float(n_elem), world)
+    h2d = sum(x.numel() * x.element_size() for x in xs)
+    d2h = sum(c.numel() for c in cf) + sum(s.numel() for s in sbs) + 4 * n
+    return {"value": round(units * 2 * BYTES_PER_ELEM / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3), "steps": K}
+
+
+def flush_l2(buf):
+    buf.zero_()
+
+
+def bench_gemm(Q, dev, stream, P, K):
+    from nvfp4_quantization_aware_b200 import synthetic as S
+    out = {}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    fp4_peak = 4.0 * P["bf16_tflops"]  # dense FP4 = 4x dense BF16 (nominal 9 / 2.25 PF)
+    with torch.cuda.stream(stream):
+        w = S.weights(4096, 4096, seed=1, device=dev)
+        wc, wsf, wts = Q.nvfp4_quantize(w, Q.DYNAMIC, layout=Q.SCALES_MMA)
+        for M in (8192, 128):
+            x = S.channel_scaled_activations(M, 4096, seed=0, device=dev)
+            xc = torch.empty(M, 2048, dtype=torch.uint8, device=dev)
+            xsf = torch.empty(Q.mma_scales_bytes(M, 4096), dtype=torch.uint8, device=dev)
+            xts = torch.empty(1, dtype=torch.float32, device=dev)
+            c = torch.empty(M, 4096, dtype=torch.bfloat16, device=dev)
+            qws = torch.empty(1024, dtype=torch.uint8, device=dev)
+            for _ in range(3):
+                Q.nvfp4_quantize(x, Q.DYNAMIC, tensor_scale=xts, block_scales=xsf, layout=Q.SCALES_MMA, codes=xc,
+                                 workspace=qws)
+                Q.nvfp4_gemm_w4a4(xc, xsf, xts, wc, wsf, wts, out=c)
+            tq, tg = [], []
+            for _ in range(K):
+                flush_l2(flush)
+                e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+                e0.record(stream)
+                Q.nvfp4_quantize(x, Q.DYNAMIC, tensor_scale=xts, block_scales=xsf, layout=Q.SCALES_MMA, codes=xc,
+                                 workspace=qws)
+                e1.record(stream)
+                Q.nvfp4_gemm_w4a4(xc, xsf, xts, wc, wsf, wts, out=c)
+                e2.record(stream)
+                tq.append((e0, e1))
+                tg.append((e1, e2))
+            stream.synchronize()
+            q_ms = statistics.mean(a.elapsed_time(b) for a, b in tq)
+            g_ms = statistics.mean(a.elapsed_time(b) for a, b in tg)
+            flops = 2.0 * M * 4096 * 4096
+            tflops = flops / (g_ms * 1e-3) / 1e12
+            gemm_bytes = 4096 * 4096 * 0.5625 + M * 4096 * 0.5625 + M * 4096 * 2
+            out[f"M{M}"] = {"tflops": round(tflops, 1), "gemm_ms": round(g_ms, 5), "x_quant_ms": round(q_ms, 5),
+                            "end_to_end_tflops": round(flops / ((q_ms + g_ms) * 1e-3) / 1e12, 1),
+                            "gemm_gbs": round(gemm_bytes / (g_ms * 1e-3) / 1e9, 1),
+                            "roofline": {"bound": "tensor" if M >= 1024 else "hbm",
+                                         "achieved": round(tflops, 1) if M >= 1024 else round(gemm_bytes / (g_ms * 1e-3) / 1e9, 1),
+                                         "peak": round(fp4_peak, 1) if M >= 1024 else P["hbm_gbs"],
+                                         "unit": "TFLOP/s" if M >= 1024 else "GB/s",
+                                         "frac": round(tflops / fp4_peak, 4) if M >= 1024 else
+                                         round(gemm_bytes / (g_ms * 1e-3) / 1e9 / P["hbm_gbs"], 4),
+                                         "peak_source": "4 x MEASURED_PEAKS bf16_tflops (nominal FP4:BF16 ratio)"
+                                         if M >= 1024 else "MEASURED_PEAKS hbm_gbs"}}
+    out["config"] = "x M x 4096 bf16 N(0,1)*LogNormal(0,1) per channel, dynamic NVFP4 on the fly; w 4096x4096 pre-quantized; L2 flushed before each step"
+    return out
+
+
+def bench_kl(Q, dev, stream, P, K):
+    from nvfp4_quantization_aware_b200 import synthetic as S
+    with torch.cuda.stream(stream):
+        d = S.distill_logits(seed=0, device=dev)
+        t, s = d["teacher"], d["student"]
+        rows, V = t.shape
+        grad = torch.empty_like(s)
+        loss = torch.empty(1, dtype=torch.float32, device=dev)
+        ws = torch.empty(int(Q.lib().qad_kl_workspace_size(rows, V, Q.BF16)), dtype=torch.uint8, device=dev)
+        L = Q.lib()
+        sptr = stream.cuda_stream
+
+        def call():
+            st = L.qad_kl_fwd_bwd(t.data_ptr(), s.data_ptr(), Q.BF16, rows, V, V, 1.0, loss.data_ptr(), None,
+                                  grad.data_ptr(), V, 1.0 / rows, ws.data_ptr(), ws.numel(), sptr)
+            assert st == 0, st
+
+        for _ in range(3):
+            call()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            call()
+        e1.record(stream)
+        stream.synchronize()
+    ms = e0.elapsed_time(e1) / K
+    gbs = 6.0 * rows * V / (ms * 1e-3) / 1e9
+    del t, s, grad, d
+    torch.cuda.empty_cache()
+    return {"tokens_per_s": round(rows / (ms * 1e-3), 1), "ms": round(ms, 4), "gbs": round(gbs, 1),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": P["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / P["hbm_gbs"], 4), "kernel": "kl_row_kernel<bf16>",
+                         "algorithmic_bytes_per_launch": 6 * rows * V},
+            "config": "teacher/student bf16 16384 x 131072, teacher N(0,3) + one +12 entry per row, student = teacher + N(0,1), T=1"}
+
+
+def cpu_baseline(xs):
+    """The oracle (as it stands) on the host cores: dynamic then frozen
+    quantize of the 128 expert weights (268M elements; the lm_head is left out
+    to bound the time)."""
+    import oracle as O
+    cores = len(os.sched_getaffinity(0))
+    O.set_threads(cores)
+    hx = [x.float().cpu().numpy() for x in xs[:128]]
+    t0 = time.perf_counter()
+    for x in hx:
+        c, sb, sg = O.quantize(x, O.DYNAMIC)
+        O.quantize(x, O.FROZEN_ALL, s_g=sg, s_b=sb)
+    dt = time.perf_counter() - t0
+    n_elem = sum(x.size for x in hx)
+    return {"value": round(n_elem * 2 * BYTES_PER_ELEM / dt / 1e9, 4), "unit": "GB/s", "cores": O.get_threads(),
+            "kind": "oracle", "sample": f"128 expert weights 2048x1024 ({n_elem} elements), dynamic + frozen, {dt:.1f} s"}
+
+
+# --------------------------------------------------------------------------- reference arm
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import oracle as O
+    from nvfp4_quantization_aware_b200 import synthetic as S
+    cores = len(os.sched_getaffinity(0))
+    O.set_threads(cores)
+    per_step = 8  # expert weights per step: a bounded sample of the sweep
+    xs = [S.weights(2048, 1024, seed=i).float().numpy() for i in range(per_step)]
+
+    def step():
+        for x in xs:
+            c, sb, sg = O.quantize(x, O.DYNAMIC)
+            O.quantize(x, O.FROZEN_ALL, s_g=sg, s_b=sb)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    n_elem = sum(x.size for x in xs)
+    value = n_elem * 2 * BYTES_PER_ELEM / dt / 1e9
+    sample = f"{per_step} expert weights 2048x1024 per step ({n_elem} elements), dynamic + frozen"
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": sample},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": O.get_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the GEMM and KL measurements")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_init()
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

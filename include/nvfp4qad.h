@@ -116,6 +116,10 @@ int nvfp4_abi_version(void);
  * ceil(rows/128)*128 * ceil(cols/64)*4. */
 size_t nvfp4_mma_scales_bytes(int64_t rows, int64_t cols);
 
+/* Number of kernels this library has launched in this process so far (host
+ * counter, incremented at each launch). */
+uint64_t nvfp4_launch_count(void);
+
 /* Synchronize `stream`, then read and clear the library's device error word.
  * *code_out (host, may be NULL) receives the raw word: 0 = none, otherwise a
  * kernel-specific reason (1 = bounded wait expired).  Returns NVFP4_OK,
@@ -160,6 +164,40 @@ nvfp4_status nvfp4_quantize(const void* x, nvfp4_dtype dtype, int64_t rows, int6
  * *first one of them encoded as (d significand << 16) | ((k + 8) << 8) | x
  * index, or all ones.  Asynchronous on `stream`. */
 nvfp4_status nvfp4_selftest_division(uint64_t* mismatches, uint64_t* first, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Grouped quantize / fake-quant: one call for a list of tensors that share a
+ * dtype and a scale mode, each with its own tensor scale (e.g. the routed and
+ * shared expert weights of a MoE layer; one FP32 scale per expert).  Results
+ * are identical to calling nvfp4_quantize / nvfp4_fake_quant on each tensor.
+ * Kernels are launched per group of tensors (at most 144 tensors per group);
+ * in DYNAMIC mode groups are cut at 48 MiB of input so that the encode pass
+ * re-reads a group's inputs from L2.
+ * ------------------------------------------------------------------------ */
+typedef struct nvfp4_tensor_ref {
+  const void* x;          /* device input, rows x cols of the call's dtype */
+  int64_t rows, cols;     /* cols % 16 == 0 */
+  int64_t ld_x;           /* row stride of x, elements */
+  float* tensor_scale;    /* device, one float: written in DYNAMIC mode, read otherwise */
+  uint8_t* block_scales;  /* device; quantize: as in nvfp4_quantize; fake-quant: ROWMAJOR,
+                             read in FROZEN_ALL, else written when non-NULL */
+  void* out;              /* device; quantize: codes (uint8); fake-quant: y (dtype) */
+  int64_t ld_out;         /* row stride of out: bytes (codes) or elements (y) */
+} nvfp4_tensor_ref;
+
+/* Workspace bytes of a grouped (or single-tensor) call in `mode`; the same
+ * workspace serves every group of the call, in stream order. */
+size_t nvfp4_grouped_workspace_size(nvfp4_scale_mode mode);
+
+/* tensors: HOST array of num_tensors descriptors (read during the call only).
+ * Every descriptor is validated before any launch. */
+nvfp4_status nvfp4_quantize_grouped(int num_tensors, const nvfp4_tensor_ref* tensors, nvfp4_dtype dtype,
+                                    nvfp4_scale_mode mode, nvfp4_scale_layout layout, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+nvfp4_status nvfp4_fake_quant_grouped(int num_tensors, const nvfp4_tensor_ref* tensors, nvfp4_dtype dtype,
+                                      nvfp4_scale_mode mode, void* workspace, size_t workspace_bytes,
+                                      void* stream);
 
 /* ------------------------------------------------------------------------
  * Fake quantization: y = dequantize(quantize(x)) in one pass, the simulated

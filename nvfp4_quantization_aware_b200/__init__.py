@@ -29,6 +29,10 @@ from .binding import (  # noqa: F401
     nvfp4_dequantize,
     nvfp4_device_error,
     nvfp4_fake_quant,
+    nvfp4_fake_quant_grouped,
+    nvfp4_launch_count,
+    nvfp4_quantize_grouped,
+    TensorRef,
     nvfp4_gemm_w4a4,
     nvfp4_quantize,
     nvfp4_selftest_division,

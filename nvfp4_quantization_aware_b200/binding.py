@@ -25,6 +25,13 @@ _STATUS = {0: "OK", 1: "ERR_ARG", 2: "ERR_SHAPE", 3: "ERR_ALIGN", 4: "ERR_DTYPE"
 _lib = None
 
 
+class TensorRef(ctypes.Structure):
+    """nvfp4_tensor_ref of include/nvfp4qad.h."""
+    _fields_ = [("x", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("ld_x", ctypes.c_int64), ("tensor_scale", ctypes.c_void_p), ("block_scales", ctypes.c_void_p),
+                ("out", ctypes.c_void_p), ("ld_out", ctypes.c_int64)]
+
+
 class NVFP4Error(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
@@ -64,6 +71,13 @@ def lib() -> ctypes.CDLL:
     L.nvfp4_fake_quant.restype = i32
     L.nvfp4_dequantize.argtypes = [p, i64, p, i32, p, i64, i64, p, i32, i64, p]
     L.nvfp4_dequantize.restype = i32
+    L.nvfp4_launch_count.restype = ctypes.c_uint64
+    L.nvfp4_grouped_workspace_size.argtypes = [i32]
+    L.nvfp4_grouped_workspace_size.restype = sz
+    L.nvfp4_quantize_grouped.argtypes = [i32, ctypes.POINTER(TensorRef), i32, i32, i32, p, sz, p]
+    L.nvfp4_quantize_grouped.restype = i32
+    L.nvfp4_fake_quant_grouped.argtypes = [i32, ctypes.POINTER(TensorRef), i32, i32, p, sz, p]
+    L.nvfp4_fake_quant_grouped.restype = i32
     L.nvfp4_selftest_division.argtypes = [p, p, p]
     L.nvfp4_selftest_division.restype = i32
     if hasattr(L, "nvfp4_gemm_w4a4"):
@@ -120,6 +134,11 @@ def mma_scales_bytes(rows: int, cols: int) -> int:
     return int(lib().nvfp4_mma_scales_bytes(rows, cols))
 
 
+def nvfp4_launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(lib().nvfp4_launch_count())
+
+
 def nvfp4_device_error() -> tuple[int, int]:
     """Synchronize the current stream and read/clear the device error word.
     Returns (status, word)."""
@@ -163,6 +182,82 @@ def nvfp4_quantize(x: torch.Tensor, mode: int = DYNAMIC, tensor_scale: torch.Ten
                           0 if workspace is None else workspace.numel(), _stream(dev))
     _check(st, "nvfp4_quantize")
     return codes, block_scales, tensor_scale
+
+
+def _refs(xs, tensor_scales, block_scales, outs):
+    arr = (TensorRef * len(xs))()
+    for i, x in enumerate(xs):
+        _cuda2d(x, f"tensor {i}")
+        o = outs[i]
+        arr[i] = TensorRef(x.data_ptr(), x.shape[0], x.shape[1], x.stride(0), tensor_scales[i].data_ptr(),
+                           None if block_scales[i] is None else block_scales[i].data_ptr(), o.data_ptr(),
+                           o.stride(0) if o.dim() == 2 else x.shape[1] // 2)
+    return arr
+
+
+def nvfp4_quantize_grouped(xs, mode: int = DYNAMIC, tensor_scales=None, block_scales=None,
+                           layout: int = SCALES_ROWMAJOR, codes=None, workspace: torch.Tensor | None = None):
+    """Quantize a list of tensors (same dtype, same mode) in grouped launches.
+    Returns (codes list, block_scales list, tensor_scales [n] f32)."""
+    L = lib()
+    n = len(xs)
+    if n == 0:
+        return [], [], None
+    dev = xs[0].device
+    dt = _dtype_code(xs[0])
+    if any(_dtype_code(x) != dt for x in xs):
+        raise TypeError("all tensors of a group must share a dtype")
+    if tensor_scales is None:
+        if mode != DYNAMIC:
+            raise ValueError("frozen modes need tensor_scales")
+        tensor_scales = torch.empty(n, dtype=torch.float32, device=dev)
+    ts_list = [tensor_scales[i:i + 1] for i in range(n)] if isinstance(tensor_scales, torch.Tensor) else list(tensor_scales)
+    if block_scales is None:
+        if mode == FROZEN_ALL:
+            raise ValueError("FROZEN_ALL needs block_scales")
+        block_scales = [(torch.empty(x.shape[0], x.shape[1] // 16, dtype=torch.uint8, device=dev)
+                         if layout == SCALES_ROWMAJOR else
+                         torch.empty(mma_scales_bytes(*x.shape), dtype=torch.uint8, device=dev)) for x in xs]
+    if codes is None:
+        codes = [torch.empty(x.shape[0], x.shape[1] // 2, dtype=torch.uint8, device=dev) for x in xs]
+    arr = _refs(xs, ts_list, block_scales, codes)
+    need = int(L.nvfp4_grouped_workspace_size(mode))
+    if workspace is None:
+        workspace = _workspace(need, dev)
+    st = L.nvfp4_quantize_grouped(n, arr, dt, mode, layout, _ptr(workspace),
+                                  0 if workspace is None else workspace.numel(), _stream(dev))
+    _check(st, "nvfp4_quantize_grouped")
+    return codes, block_scales, tensor_scales
+
+
+def nvfp4_fake_quant_grouped(xs, mode: int = DYNAMIC, tensor_scales=None, block_scales=None, outs=None,
+                             workspace: torch.Tensor | None = None):
+    """Fake-quantize a list of tensors in grouped launches; returns the outputs."""
+    L = lib()
+    n = len(xs)
+    if n == 0:
+        return []
+    dev = xs[0].device
+    dt = _dtype_code(xs[0])
+    if tensor_scales is None:
+        if mode != DYNAMIC:
+            raise ValueError("frozen modes need tensor_scales")
+        tensor_scales = torch.empty(n, dtype=torch.float32, device=dev)
+    ts_list = [tensor_scales[i:i + 1] for i in range(n)] if isinstance(tensor_scales, torch.Tensor) else list(tensor_scales)
+    if block_scales is None:
+        if mode == FROZEN_ALL:
+            raise ValueError("FROZEN_ALL needs block_scales")
+        block_scales = [None] * n
+    if outs is None:
+        outs = [torch.empty_like(x) for x in xs]
+    arr = _refs(xs, ts_list, block_scales, outs)
+    need = int(L.nvfp4_grouped_workspace_size(mode))
+    if workspace is None:
+        workspace = _workspace(need, dev)
+    st = L.nvfp4_fake_quant_grouped(n, arr, dt, mode, _ptr(workspace),
+                                    0 if workspace is None else workspace.numel(), _stream(dev))
+    _check(st, "nvfp4_fake_quant_grouped")
+    return outs
 
 
 def nvfp4_fake_quant(x: torch.Tensor, mode: int = DYNAMIC, tensor_scale: torch.Tensor | None = None,

@@ -2,9 +2,14 @@
 // version and the device error word that bounded waits report into.
 #include "common.cuh"
 
+#include <atomic>
+
 namespace nvfp4 {
 __device__ int g_device_error = 0;
-}
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace nvfp4
 
 extern "C" {
 
@@ -25,6 +30,8 @@ const char* nvfp4_status_string(nvfp4_status status) {
 }
 
 int nvfp4_abi_version(void) { return NVFP4QAD_ABI_VERSION; }
+
+uint64_t nvfp4_launch_count(void) { return nvfp4::g_launches.load(std::memory_order_relaxed); }
 
 nvfp4_status nvfp4_device_error(void* stream, int32_t* code_out) {
   cudaStream_t s = (cudaStream_t)stream;

@@ -21,6 +21,9 @@ constexpr int kErrWaitTimeout = 1;
 
 NVFP4_DEV void report_error(int code) { atomicCAS(&g_device_error, 0, code); }
 
+// Host-side count of kernel launches (nvfp4_launch_count).
+void count_launches(int n);
+
 // ---------------------------------------------------------------- loads/stores
 
 // 16-byte streaming load that bypasses L1 allocation (each byte is read once).

@@ -263,6 +263,7 @@ static nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* b, const GemmPa
   }
   dim3 grid((p.N + C::BN - 1) / C::BN, (p.M + C::BM - 1) / C::BM);
   gemm_w4a4_kernel<BN><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, p);
+  count_launches(1);
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 

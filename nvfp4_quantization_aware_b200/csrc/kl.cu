@@ -393,6 +393,7 @@ nvfp4_status qad_kl_fwd_bwd(const void* teacher, const void* student, nvfp4_dtyp
   cudaError_t e = dtype == NVFP4_BF16 ? launch_kl<__nv_bfloat16>(args, plan, s) : launch_kl<float>(args, plan, s);
   if (e != cudaSuccess) return NVFP4_ERR_CUDA;
   kl_mean_kernel<<<1, 1024, 0, s>>>(args.row_kl, rows, loss, row_kl);
+  count_launches(2);
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 

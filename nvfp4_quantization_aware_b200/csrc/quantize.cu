@@ -15,9 +15,9 @@
 // independent 16-byte loads per lane are in flight.  Grids are persistent:
 // a multiple of the SM count, grid-striding over chunks.
 //
-// Dynamic mode is two launches in stream order: amax_partial_kernel writes one
-// per-CTA partial max into the workspace, and the encode kernel reduces those
-// partials at entry (max is exact, so any order gives the same s_g).
+// Dynamic mode is two launches in stream order: group_amax_kernel folds each
+// tensor's max |x| into a workspace word (max is exact, so any order gives the
+// same s_g), then the encode kernel derives s_g = amax / 2688 from it.
 #include "common.cuh"
 
 namespace nvfp4 {
@@ -26,7 +26,6 @@ constexpr int kThreads = 256;           // 8 warps per CTA
 constexpr int kWarps = kThreads / 32;
 constexpr int kUnroll = 4;              // chunks per warp per iteration
 constexpr int kChunk = 256;             // elements per warp per chunk
-constexpr int kMaxPartials = 1024;      // amax partials (one per amax CTA)
 
 // ------------------------------------------------------------------ input traits
 
@@ -99,41 +98,96 @@ NVFP4_DEV float warp_max(float v) {
   return v;
 }
 
+// ------------------------------------------------------------------ tensor groups
+//
+// One launch processes a group of up to kMaxGroup tensors (e.g. the 128
+// experts of a MoE layer), each with its own FP32 tensor scale.  Their chunks
+// are numbered consecutively: tensor i owns [chunk0_i, chunk0_{i+1}).  The
+// table travels by value as a __grid_constant__ kernel parameter, read with
+// warp-uniform indices.
+
+constexpr int kMaxGroup = 144;
+
+struct GTensor {
+  const void* x;        // input, row stride ld_x elements
+  uint8_t* codes;       // Out::Codes: packed codes, row stride ld_out bytes
+  void* y;              // Out::Fake: output, row stride ld_out elements
+  uint8_t* sb;          // block scales: read (FROZEN_ALL, row-major) or written if non-NULL
+  float* ts;            // tensor scale: written (DYNAMIC) or read
+  int64_t ld_x, ld_out;
+  int64_t cols;
+  int64_t cpr;          // chunks per row = ceil(cols / 256)
+  int64_t chunk0;       // first chunk of this tensor
+  int64_t kchunks;      // ceil(cols / 64), MMA scale layout
+};
+
+struct GroupArgs {
+  GTensor t[kMaxGroup];
+  int n;
+  int mode;             // nvfp4_scale_mode
+  int layout;           // nvfp4_scale_layout of written block scales
+  int64_t total_chunks;
+  unsigned* amax;       // DYNAMIC: n words holding max |x| as float bits (zeroed first)
+};
+
+// Advance `t` to the tensor owning `chunk` (chunks are visited in increasing
+// order by every warp, so the cursor only moves forward).
+NVFP4_DEV int find_tensor(const GroupArgs& a, int64_t chunk, int t) {
+  while (t + 1 < a.n && chunk >= a.t[t + 1].chunk0) ++t;
+  return t;
+}
+
+NVFP4_DEV void chunk_pos(const GTensor& g, int64_t chunk, int lane, int64_t& row, int64_t& col) {
+  const int64_t c = chunk - g.chunk0;
+  row = c / g.cpr;
+  col = (c - row * g.cpr) * kChunk + lane * 8;
+}
+
 // ------------------------------------------------------------------ amax
 
-// One partial max of |x| per CTA.
+// Per-tensor max |x| of a group: each warp reduces the chunks of one
+// iteration and folds them into the tensor's word with atomicMax on the float
+// bits (order-independent: |x| >= 0 compares like its bit pattern).
 template <typename T>
-__global__ void __launch_bounds__(kThreads) amax_partial_kernel(const T* __restrict__ x, Geom g,
-                                                                float* __restrict__ partial) {
+__global__ void __launch_bounds__(kThreads) group_amax_kernel(const __grid_constant__ GroupArgs a) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * kWarps;
-  float m = 0.0f;
-  for (int64_t c0 = warp * kUnroll; c0 < g.total_chunks; c0 += nwarps * kUnroll) {
+  int cur = 0;
+  for (int64_t c0 = warp * kUnroll; c0 < a.total_chunks; c0 += nwarps * kUnroll) {
     Lane8<T> in[kUnroll];
+    int tid[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      int64_t row, col;
-      g.locate(c0 + u, lane, row, col);
-      if (c0 + u < g.total_chunks && col < g.cols) in[u].load(x + row * g.ld + col);
-      else in[u].zero();
+      const int64_t c = c0 + u;
+      in[u].zero();
+      tid[u] = -1;
+      if (c < a.total_chunks) {
+        cur = find_tensor(a, c, cur);
+        const GTensor& g = a.t[cur];
+        int64_t row, col;
+        chunk_pos(g, c, lane, row, col);
+        tid[u] = cur;
+        if (col < g.cols) in[u].load(reinterpret_cast<const T*>(g.x) + row * g.ld_x + col);
+      }
     }
+    float m = 0.0f;
+    int mt = tid[0];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
+      if (tid[u] != mt) {  // chunk of the next tensor: flush the running max
+        const float w = warp_max(m);
+        if (lane == 0 && mt >= 0 && w > 0.0f) atomicMax(a.amax + mt, __float_as_uint(w));
+        m = 0.0f;
+        mt = tid[u];
+      }
       float v[8];
       in[u].to_f32(v);
 #pragma unroll
       for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
     }
-  }
-  m = warp_max(m);
-  __shared__ float s[kWarps];
-  if (lane == 0) s[threadIdx.x >> 5] = m;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    float v = threadIdx.x < kWarps ? s[threadIdx.x] : 0.0f;
-    v = warp_max(v);
-    if (threadIdx.x == 0) partial[blockIdx.x] = v;
+    const float w = warp_max(m);
+    if (lane == 0 && mt >= 0 && w > 0.0f) atomicMax(a.amax + mt, __float_as_uint(w));
   }
 }
 
@@ -141,71 +195,63 @@ __global__ void __launch_bounds__(kThreads) amax_partial_kernel(const T* __restr
 
 enum class Out { Codes, Fake };
 
-struct EncodeArgs {
-  Geom g;
-  int mode;                   // nvfp4_scale_mode
-  const float* partial;       // DYNAMIC: amax partials
-  int npartial;
-  float* tensor_scale;        // DYNAMIC: written by CTA 0; else read
-  uint8_t* block_scales;      // FROZEN_ALL: read (row-major); else written if non-NULL
-  int scale_layout;           // nvfp4_scale_layout of block_scales (written case)
-  int64_t kchunks;            // MMA layout: ceil(cols/64)
-  uint8_t* codes;             // Out::Codes
-  int64_t ld_codes;
-  void* y;                    // Out::Fake
-  int64_t ld_y;
-};
-
-// Resolve s_g at kernel entry (every CTA): reduce the amax partials in DYNAMIC
-// mode, otherwise read the given scale.
-NVFP4_DEV float resolve_tensor_scale(const EncodeArgs& a) {
-  __shared__ float s_sg;
-  if (a.mode == NVFP4_DYNAMIC) {
-    if (threadIdx.x < 32) {
-      float m = 0.0f;
-      for (int i = threadIdx.x; i < a.npartial; i += 32) m = fmaxf(m, a.partial[i]);
-      m = warp_max(m);
-      if (threadIdx.x == 0) {
-        float sg = __fdiv_rn(m, 2688.0f);  // amax / (6 * 448)
-        s_sg = sg;
-        if (blockIdx.x == 0) *a.tensor_scale = sg;
-      }
-    }
-  } else if (threadIdx.x == 0) {
-    s_sg = *a.tensor_scale;
-  }
-  __syncthreads();
-  return s_sg;
+// s_g of tensor t: amax / (6 * 448) in DYNAMIC mode, else the given scale.
+NVFP4_DEV float tensor_scale_of(const GroupArgs& a, int t) {
+  if (a.mode == NVFP4_DYNAMIC) return __fdiv_rn(__uint_as_float(__ldcg(a.amax + t)), 2688.0f);
+  return __ldg(a.t[t].ts);
 }
 
 template <typename T, Out OUT>
-__global__ void __launch_bounds__(kThreads) encode_kernel(const T* __restrict__ x, EncodeArgs a) {
-  const float sg = resolve_tensor_scale(a);
-  const float denom6 = __fmul_rn(6.0f, sg);
+__global__ void __launch_bounds__(kThreads) group_encode_kernel(const __grid_constant__ GroupArgs a) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * kWarps;
-  const Geom& g = a.g;
-  const int64_t nblk = g.cols >> 4;
   const bool frozen_all = a.mode == NVFP4_FROZEN_ALL;
+  if (a.mode == NVFP4_DYNAMIC && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < a.n; i += kThreads) *a.t[i].ts = tensor_scale_of(a, i);
 
-  for (int64_t c0 = warp * kUnroll; c0 < g.total_chunks; c0 += nwarps * kUnroll) {
+  int cur = 0;
+  int sg_t = -1;  // tensor whose scale is cached below
+  float sg = 0.0f, denom6 = 0.0f;
+  for (int64_t c0 = warp * kUnroll; c0 < a.total_chunks; c0 += nwarps * kUnroll) {
     Lane8<T> in[kUnroll];
     uint32_t sb_in[kUnroll];
+    int tid[kUnroll];
+    int64_t rows_[kUnroll], cols_[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      int64_t row, col;
-      g.locate(c0 + u, lane, row, col);
-      const bool ok = (c0 + u < g.total_chunks) && col < g.cols;
-      if (ok) in[u].load(x + row * g.ld + col);
-      else in[u].zero();
-      sb_in[u] = (frozen_all && ok) ? (uint32_t)__ldg(a.block_scales + row * nblk + (col >> 4)) : 0u;
+      const int64_t c = c0 + u;
+      in[u].zero();
+      sb_in[u] = 0u;
+      tid[u] = -1;
+      rows_[u] = 0;
+      cols_[u] = 0;
+      if (c < a.total_chunks) {
+        cur = find_tensor(a, c, cur);
+        const GTensor& g = a.t[cur];
+        int64_t row, col;
+        chunk_pos(g, c, lane, row, col);
+        tid[u] = cur;
+        rows_[u] = row;
+        cols_[u] = col;
+        if (col < g.cols) {
+          in[u].load(reinterpret_cast<const T*>(g.x) + row * g.ld_x + col);
+          if (frozen_all) sb_in[u] = (uint32_t)__ldg(g.sb + row * (g.cols >> 4) + (col >> 4));
+        }
+      }
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      int64_t row, col;
-      g.locate(c0 + u, lane, row, col);
-      const bool ok = (c0 + u < g.total_chunks) && col < g.cols;
+      const int t = tid[u];
+      if (t < 0) continue;  // warp-uniform: the whole chunk is past the end
+      const GTensor& g = a.t[t];
+      const int64_t row = rows_[u], col = cols_[u];
+      const bool ok = col < g.cols;
+      if (t != sg_t) {
+        sg = tensor_scale_of(a, t);
+        denom6 = __fmul_rn(6.0f, sg);
+        sg_t = t;
+      }
       float v[8];
       in[u].to_f32(v);
       // ---- block scale
@@ -237,7 +283,7 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(const T* __restrict__ 
       if (!ok) continue;
       // ---- outputs
       if (OUT == Out::Codes) {
-        st_stream_u32(a.codes + row * a.ld_codes + (col >> 1), word);
+        st_stream_u32(g.codes + row * g.ld_out + (col >> 1), word);
       } else {
         float o[8];
 #pragma unroll
@@ -247,13 +293,13 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(const T* __restrict__ 
           o[2 * j] = __fmul_rn(lo, d);
           o[2 * j + 1] = __fmul_rn(hi, d);
         }
-        store8<T>(reinterpret_cast<T*>(a.y) + row * a.ld_y + col, o);
+        store8<T>(reinterpret_cast<T*>(g.y) + row * g.ld_out + col, o);
       }
-      if (!frozen_all && a.block_scales != nullptr && (lane & 1) == 0) {
+      if (!frozen_all && g.sb != nullptr && (lane & 1) == 0) {
         const int64_t kb = col >> 4;
-        const int64_t off = (a.scale_layout == NVFP4_SCALES_MMA) ? mma_scale_offset(row, kb, a.kchunks)
-                                                                 : row * nblk + kb;
-        a.block_scales[off] = (uint8_t)sb;
+        const int64_t off = (a.layout == NVFP4_SCALES_MMA) ? mma_scale_offset(row, kb, g.kchunks)
+                                                           : row * (g.cols >> 4) + kb;
+        g.sb[off] = (uint8_t)sb;
       }
     }
   }
@@ -378,11 +424,6 @@ static int grid_for(const Geom& g) {
   return need < 1 ? 1 : (int)need;
 }
 
-static int amax_grid(const Geom& g) {
-  int gsz = grid_for(g);
-  return gsz > kMaxPartials ? kMaxPartials : gsz;
-}
-
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 static nvfp4_status check_common(const void* x, nvfp4_dtype dtype, int64_t rows, int64_t cols, int64_t ld_x) {
@@ -401,54 +442,131 @@ static nvfp4_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
-// Shared driver of quantize and fake-quant.
+// In DYNAMIC mode the amax pass and the encode pass of a group run back to
+// back; groups are cut so that their inputs fit in L2 (126 MB on B200) and the
+// encode pass re-reads them from L2 rather than HBM.  A tensor larger than
+// this budget forms a group of its own.
+constexpr int64_t kL2GroupBytes = 48ll << 20;
+constexpr size_t kDynamicWorkspace = 1024;  // >= kMaxGroup amax words
+
+// Validate one tensor of a (possibly grouped) quantize / fake-quant call.
 template <Out OUT>
-static nvfp4_status run_encode(const void* x, nvfp4_dtype dtype, int64_t rows, int64_t cols, int64_t ld_x,
-                               nvfp4_scale_mode mode, float* tensor_scale, uint8_t* block_scales,
-                               nvfp4_scale_layout layout, uint8_t* codes, int64_t ld_codes, void* y,
-                               int64_t ld_y, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  Geom g = make_geom(rows, cols, ld_x);
-  EncodeArgs a;
-  a.g = g;
-  a.mode = (int)mode;
-  a.tensor_scale = tensor_scale;
-  a.block_scales = block_scales;
-  a.scale_layout = (int)layout;
-  a.kchunks = (cols / 16 + 3) / 4;
-  a.codes = codes;
-  a.ld_codes = ld_codes;
-  a.y = y;
-  a.ld_y = ld_y;
-  a.partial = reinterpret_cast<float*>(ws);
-  a.npartial = 0;
-  if (mode == NVFP4_DYNAMIC) {
-    a.npartial = amax_grid(g);
-    if (dtype == NVFP4_BF16)
-      amax_partial_kernel<__nv_bfloat16><<<a.npartial, kThreads, 0, stream>>>(
-          reinterpret_cast<const __nv_bfloat16*>(x), g, reinterpret_cast<float*>(ws));
-    else
-      amax_partial_kernel<float><<<a.npartial, kThreads, 0, stream>>>(reinterpret_cast<const float*>(x), g,
-                                                                      reinterpret_cast<float*>(ws));
+static nvfp4_status check_tensor(const nvfp4_tensor_ref& r, nvfp4_dtype dtype, nvfp4_scale_mode mode,
+                                 nvfp4_scale_layout layout) {
+  nvfp4_status st = check_common(r.x, dtype, r.rows, r.cols, r.ld_x);
+  if (st != NVFP4_OK) return st;
+  if (!r.tensor_scale) return NVFP4_ERR_ARG;
+  if (mode == NVFP4_FROZEN_ALL && layout != NVFP4_SCALES_ROWMAJOR) return NVFP4_ERR_ARG;
+  if (r.rows == 0 || r.cols == 0) return NVFP4_OK;
+  if (mode == NVFP4_FROZEN_ALL && !r.block_scales) return NVFP4_ERR_ARG;
+  if (!r.out) return NVFP4_ERR_ARG;
+  if (OUT == Out::Codes) {
+    if (!r.block_scales) return NVFP4_ERR_ARG;
+    if (r.ld_out < r.cols / 2) return NVFP4_ERR_SHAPE;
+    if ((r.ld_out % 4) != 0 || ((uintptr_t)r.out & 3u) != 0) return NVFP4_ERR_ALIGN;
+  } else {
+    if (r.ld_out < r.cols) return NVFP4_ERR_SHAPE;
+    const int64_t esz = dtype == NVFP4_BF16 ? 2 : 4;
+    if (!aligned16(r.out) || (r.ld_out * esz) % 16 != 0) return NVFP4_ERR_ALIGN;
+  }
+  return NVFP4_OK;
+}
+
+template <Out OUT>
+static nvfp4_status launch_group(GroupArgs& a, nvfp4_dtype dtype, void* ws, cudaStream_t s) {
+  if (a.n == 0 || a.total_chunks == 0) return NVFP4_OK;
+  Geom g;
+  g.total_chunks = a.total_chunks;
+  const int grid = grid_for(g);
+  if (a.mode == NVFP4_DYNAMIC) {
+    a.amax = reinterpret_cast<unsigned*>(ws);
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned) * (size_t)a.n, s) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (dtype == NVFP4_BF16) group_amax_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(a);
+    else group_amax_kernel<float><<<grid, kThreads, 0, s>>>(a);
+    count_launches(1);
     if (launch_status() != NVFP4_OK) return NVFP4_ERR_CUDA;
   }
-  const int grid = grid_for(g);
-  if (dtype == NVFP4_BF16)
-    encode_kernel<__nv_bfloat16, OUT><<<grid, kThreads, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(x), a);
-  else
-    encode_kernel<float, OUT><<<grid, kThreads, 0, stream>>>(reinterpret_cast<const float*>(x), a);
-  if (launch_status() != NVFP4_OK) return NVFP4_ERR_CUDA;
+  if (dtype == NVFP4_BF16) group_encode_kernel<__nv_bfloat16, OUT><<<grid, kThreads, 0, s>>>(a);
+  else group_encode_kernel<float, OUT><<<grid, kThreads, 0, s>>>(a);
+  count_launches(1);
+  return launch_status();
+}
+
+// Quantize or fake-quantize a list of tensors: validation of every tensor
+// first, then one (FROZEN) or two (DYNAMIC) launches per group.
+template <Out OUT>
+static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype dtype, nvfp4_scale_mode mode,
+                                nvfp4_scale_layout layout, void* ws, size_t ws_bytes, cudaStream_t s) {
+  if (n < 0 || (n > 0 && !refs)) return NVFP4_ERR_ARG;
+  if (mode != NVFP4_DYNAMIC && mode != NVFP4_FROZEN_GLOBAL && mode != NVFP4_FROZEN_ALL) return NVFP4_ERR_ARG;
+  if (layout != NVFP4_SCALES_ROWMAJOR && layout != NVFP4_SCALES_MMA) return NVFP4_ERR_ARG;
+  if (OUT == Out::Fake && layout != NVFP4_SCALES_ROWMAJOR) return NVFP4_ERR_ARG;
+  for (int i = 0; i < n; ++i) {
+    nvfp4_status st = check_tensor<OUT>(refs[i], dtype, mode, layout);
+    if (st != NVFP4_OK) return st;
+  }
+  if (mode == NVFP4_DYNAMIC) {
+    if (!ws || ws_bytes < kDynamicWorkspace) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return NVFP4_ERR_ALIGN;
+  }
+  const int64_t esz = dtype == NVFP4_BF16 ? 2 : 4;
+  static GroupArgs a;  // host staging of the kernel parameter (copied at launch)
+  a.n = 0;
+  a.mode = (int)mode;
+  a.layout = (int)layout;
+  a.total_chunks = 0;
+  a.amax = nullptr;
+  int64_t group_bytes = 0;
+  for (int i = 0; i < n; ++i) {
+    const nvfp4_tensor_ref& r = refs[i];
+    if (r.rows == 0 || r.cols == 0) {
+      if (mode == NVFP4_DYNAMIC && cudaMemsetAsync(r.tensor_scale, 0, sizeof(float), s) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+      continue;
+    }
+    const int64_t bytes = r.rows * r.cols * esz;
+    const bool full = a.n == kMaxGroup;
+    const bool over_l2 = mode == NVFP4_DYNAMIC && a.n > 0 && group_bytes + bytes > kL2GroupBytes;
+    if (full || over_l2) {
+      nvfp4_status st = launch_group<OUT>(a, dtype, ws, s);
+      if (st != NVFP4_OK) return st;
+      a.n = 0;
+      a.total_chunks = 0;
+      group_bytes = 0;
+    }
+    GTensor& g = a.t[a.n++];
+    g.x = r.x;
+    g.codes = OUT == Out::Codes ? reinterpret_cast<uint8_t*>(r.out) : nullptr;
+    g.y = OUT == Out::Fake ? r.out : nullptr;
+    g.sb = r.block_scales;
+    g.ts = r.tensor_scale;
+    g.ld_x = r.ld_x;
+    g.ld_out = r.ld_out;
+    g.cols = r.cols;
+    g.cpr = (r.cols + kChunk - 1) / kChunk;
+    g.chunk0 = a.total_chunks;
+    g.kchunks = (r.cols / 16 + 3) / 4;
+    a.total_chunks += r.rows * g.cpr;
+    group_bytes += bytes;
+  }
+  nvfp4_status st = launch_group<OUT>(a, dtype, ws, s);
+  if (st != NVFP4_OK) return st;
+  // zero the padding of MMA-layout scale arrays
   if (OUT == Out::Codes && layout == NVFP4_SCALES_MMA && mode != NVFP4_FROZEN_ALL) {
-    const int64_t rows_pad = (rows + 127) / 128 * 128;
-    if (rows_pad != rows || (cols / 16) % 4 != 0) {
-      const int64_t total = rows_pad * a.kchunks * 4;
+    for (int i = 0; i < n; ++i) {
+      const nvfp4_tensor_ref& r = refs[i];
+      if (r.rows == 0 || r.cols == 0) continue;
+      const int64_t rows_pad = (r.rows + 127) / 128 * 128;
+      const int64_t kchunks = (r.cols / 16 + 3) / 4;
+      if (rows_pad == r.rows && (r.cols / 16) % 4 == 0) continue;
+      const int64_t total = rows_pad * kchunks * 4;
       int64_t blocks = (total + 255) / 256;
       if (blocks > (int64_t)sm_count() * 8) blocks = (int64_t)sm_count() * 8;
-      zero_mma_padding_kernel<<<(int)blocks, 256, 0, stream>>>(block_scales, rows, cols / 16, rows_pad,
-                                                               a.kchunks);
+      zero_mma_padding_kernel<<<(int)blocks, 256, 0, s>>>(r.block_scales, r.rows, r.cols / 16, rows_pad, kchunks);
+      count_launches(1);
       if (launch_status() != NVFP4_OK) return NVFP4_ERR_CUDA;
     }
   }
-  (void)ws_bytes;
   return NVFP4_OK;
 }
 
@@ -466,63 +584,58 @@ size_t nvfp4_mma_scales_bytes(int64_t rows, int64_t cols) {
 size_t nvfp4_quantize_workspace_size(int64_t rows, int64_t cols, nvfp4_scale_mode mode) {
   (void)rows;
   (void)cols;
-  return mode == NVFP4_DYNAMIC ? (size_t)kMaxPartials * sizeof(float) : 0;
+  return mode == NVFP4_DYNAMIC ? kDynamicWorkspace : 0;
 }
 
 size_t nvfp4_fake_quant_workspace_size(int64_t rows, int64_t cols, nvfp4_scale_mode mode) {
   return nvfp4_quantize_workspace_size(rows, cols, mode);
 }
 
+size_t nvfp4_grouped_workspace_size(nvfp4_scale_mode mode) { return mode == NVFP4_DYNAMIC ? kDynamicWorkspace : 0; }
+
 nvfp4_status nvfp4_quantize(const void* x, nvfp4_dtype dtype, int64_t rows, int64_t cols, int64_t ld_x,
                             nvfp4_scale_mode mode, float* tensor_scale, uint8_t* block_scales,
                             nvfp4_scale_layout layout, uint8_t* codes, int64_t ld_codes, void* workspace,
                             size_t workspace_bytes, void* stream) {
-  nvfp4_status st = check_common(x, dtype, rows, cols, ld_x);
-  if (st != NVFP4_OK) return st;
-  if (mode != NVFP4_DYNAMIC && mode != NVFP4_FROZEN_GLOBAL && mode != NVFP4_FROZEN_ALL) return NVFP4_ERR_ARG;
-  if (layout != NVFP4_SCALES_ROWMAJOR && layout != NVFP4_SCALES_MMA) return NVFP4_ERR_ARG;
-  if (mode == NVFP4_FROZEN_ALL && layout != NVFP4_SCALES_ROWMAJOR) return NVFP4_ERR_ARG;
-  if (!tensor_scale) return NVFP4_ERR_ARG;
-  if (ld_codes < cols / 2) return NVFP4_ERR_SHAPE;
-  const size_t need = nvfp4_quantize_workspace_size(rows, cols, mode);
-  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return NVFP4_ERR_WORKSPACE;
-  if (need > 0 && !aligned16(workspace)) return NVFP4_ERR_ALIGN;
-  if (rows == 0 || cols == 0) {
-    if (mode == NVFP4_DYNAMIC)
-      return cudaMemsetAsync(tensor_scale, 0, sizeof(float), (cudaStream_t)stream) == cudaSuccess ? NVFP4_OK
-                                                                                                : NVFP4_ERR_CUDA;
-    return NVFP4_OK;
-  }
-  if (!block_scales || !codes) return NVFP4_ERR_ARG;
-  if ((ld_codes % 4) != 0 || ((uintptr_t)codes & 3u) != 0) return NVFP4_ERR_ALIGN;
-  return run_encode<Out::Codes>(x, dtype, rows, cols, ld_x, mode, tensor_scale, block_scales, layout, codes,
-                                ld_codes, nullptr, 0, workspace, workspace_bytes, (cudaStream_t)stream);
+  nvfp4_tensor_ref r;
+  r.x = x;
+  r.rows = rows;
+  r.cols = cols;
+  r.ld_x = ld_x;
+  r.tensor_scale = tensor_scale;
+  r.block_scales = block_scales;
+  r.out = codes;
+  r.ld_out = ld_codes;
+  return run_tensors<Out::Codes>(1, &r, dtype, mode, layout, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
 nvfp4_status nvfp4_fake_quant(const void* x, nvfp4_dtype dtype, int64_t rows, int64_t cols, int64_t ld_x,
                               nvfp4_scale_mode mode, float* tensor_scale, uint8_t* block_scales, void* y,
                               int64_t ld_y, void* workspace, size_t workspace_bytes, void* stream) {
-  nvfp4_status st = check_common(x, dtype, rows, cols, ld_x);
-  if (st != NVFP4_OK) return st;
-  if (mode != NVFP4_DYNAMIC && mode != NVFP4_FROZEN_GLOBAL && mode != NVFP4_FROZEN_ALL) return NVFP4_ERR_ARG;
-  if (!tensor_scale) return NVFP4_ERR_ARG;
-  if (mode == NVFP4_FROZEN_ALL && !block_scales) return NVFP4_ERR_ARG;
-  if (ld_y < cols) return NVFP4_ERR_SHAPE;
-  const size_t need = nvfp4_fake_quant_workspace_size(rows, cols, mode);
-  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return NVFP4_ERR_WORKSPACE;
-  if (need > 0 && !aligned16(workspace)) return NVFP4_ERR_ALIGN;
-  if (rows == 0 || cols == 0) {
-    if (mode == NVFP4_DYNAMIC)
-      return cudaMemsetAsync(tensor_scale, 0, sizeof(float), (cudaStream_t)stream) == cudaSuccess ? NVFP4_OK
-                                                                                                : NVFP4_ERR_CUDA;
-    return NVFP4_OK;
-  }
-  if (!y) return NVFP4_ERR_ARG;
-  const int64_t esz = dtype == NVFP4_BF16 ? 2 : 4;
-  if (!aligned16(y) || (ld_y * esz) % 16 != 0) return NVFP4_ERR_ALIGN;
-  return run_encode<Out::Fake>(x, dtype, rows, cols, ld_x, mode, tensor_scale, block_scales,
-                               NVFP4_SCALES_ROWMAJOR, nullptr, 0, y, ld_y, workspace, workspace_bytes,
-                               (cudaStream_t)stream);
+  nvfp4_tensor_ref r;
+  r.x = x;
+  r.rows = rows;
+  r.cols = cols;
+  r.ld_x = ld_x;
+  r.tensor_scale = tensor_scale;
+  r.block_scales = block_scales;
+  r.out = y;
+  r.ld_out = ld_y;
+  return run_tensors<Out::Fake>(1, &r, dtype, mode, NVFP4_SCALES_ROWMAJOR, workspace, workspace_bytes,
+                                (cudaStream_t)stream);
+}
+
+nvfp4_status nvfp4_quantize_grouped(int num_tensors, const nvfp4_tensor_ref* tensors, nvfp4_dtype dtype,
+                                    nvfp4_scale_mode mode, nvfp4_scale_layout layout, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  return run_tensors<Out::Codes>(num_tensors, tensors, dtype, mode, layout, workspace, workspace_bytes,
+                                 (cudaStream_t)stream);
+}
+
+nvfp4_status nvfp4_fake_quant_grouped(int num_tensors, const nvfp4_tensor_ref* tensors, nvfp4_dtype dtype,
+                                      nvfp4_scale_mode mode, void* workspace, size_t workspace_bytes, void* stream) {
+  return run_tensors<Out::Fake>(num_tensors, tensors, dtype, mode, NVFP4_SCALES_ROWMAJOR, workspace,
+                                workspace_bytes, (cudaStream_t)stream);
 }
 
 nvfp4_status nvfp4_dequantize(const uint8_t* codes, int64_t ld_codes, const uint8_t* block_scales,
@@ -546,6 +659,7 @@ nvfp4_status nvfp4_dequantize(const uint8_t* codes, int64_t ld_codes, const uint
   else
     dequant_kernel<float><<<grid, kThreads, 0, s>>>(codes, ld_codes, block_scales, (int)layout, kchunks,
                                                     tensor_scale, g, reinterpret_cast<float*>(out), ld_out);
+  count_launches(1);
   return launch_status();
 }
 
@@ -560,6 +674,7 @@ nvfp4_status nvfp4_selftest_division(uint64_t* mismatches, uint64_t* first, void
   if (cudaMemsetAsync(first, 0xFF, sizeof(uint64_t), s) != cudaSuccess) return NVFP4_ERR_CUDA;
   selftest_division_kernel<<<(1 << 23) / 256, 256, 0, s>>>(reinterpret_cast<unsigned long long*>(mismatches),
                                                            reinterpret_cast<unsigned long long*>(first));
+  count_launches(1);
   return launch_status();
 }
 

@@ -259,3 +259,58 @@ def test_weight_sweep_full_size_parity():
         assert np.array_equal(sb.cpu().numpy(), ref_sb), i
         codes_f, _, _ = Q.nvfp4_quantize(w, Q.FROZEN_ALL, tensor_scale=sg, block_scales=sb)
         assert torch.equal(codes_f, codes), i
+
+
+def test_grouped_quantize_matches_oracle_and_single_calls():
+    # mixed shapes, an empty tensor, more tensors than one launch holds and a
+    # tensor larger than one L2-sized group
+    shapes = [(64, 1024), (0, 32), (3, 48), (130, 1040)] + [(40, 256)] * 150 + [(6000, 2048)]
+    xs = [S.weights(r, c, seed=100 + i, device=DEV, outlier_p=0.01, outlier_mult=40) for i, (r, c) in enumerate(shapes)]
+    for mode in [Q.DYNAMIC, Q.FROZEN_GLOBAL, Q.FROZEN_ALL]:
+        if mode == Q.DYNAMIC:
+            codes, sbs, ts = Q.nvfp4_quantize_grouped(xs, mode)
+        else:
+            ref_sg = torch.empty(len(xs), device=DEV)
+            ref_sb = []
+            for i, x in enumerate(xs):
+                c, sb, sg = Q.nvfp4_quantize(x)
+                ref_sg[i] = sg[0] * (1.25 if mode == Q.FROZEN_GLOBAL else 1.0)
+                ref_sb.append(sb)
+            codes, sbs, ts = Q.nvfp4_quantize_grouped(xs, mode, tensor_scales=ref_sg,
+                                                      block_scales=ref_sb if mode == Q.FROZEN_ALL else None)
+        torch.cuda.synchronize()
+        for i, x in enumerate(xs):
+            if i % 7 != 0 and i not in (1, 2, 3, len(xs) - 1):
+                continue
+            xh = _host_f32(x)
+            if mode == Q.DYNAMIC:
+                rc, rsb, rsg = O.quantize(xh, O.DYNAMIC)
+            elif mode == Q.FROZEN_GLOBAL:
+                rc, rsb, rsg = O.quantize(xh, O.FROZEN_GLOBAL, s_g=float(ts[i].cpu()))
+            else:
+                rc, rsb, rsg = O.quantize(xh, O.FROZEN_ALL, s_g=float(ts[i].cpu()), s_b=sbs[i].cpu().numpy())
+            assert np.array_equal(codes[i].cpu().numpy(), rc), (mode, i)
+            assert np.array_equal(sbs[i].cpu().numpy(), rsb), (mode, i)
+            assert _bits32(ts[i:i + 1])[0] == np.float32(rsg).view(np.uint32), (mode, i)
+
+
+def test_grouped_mma_layout_and_fake_quant():
+    xs = [S.activations(r, c, seed=200 + r, device=DEV) for r, c in [(130, 1040), (128, 256), (1, 16)]]
+    codes, sbs, ts = Q.nvfp4_quantize_grouped(xs, Q.DYNAMIC, layout=Q.SCALES_MMA)
+    ys = Q.nvfp4_fake_quant_grouped(xs, Q.DYNAMIC)
+    torch.cuda.synchronize()
+    for i, x in enumerate(xs):
+        xh = _host_f32(x)
+        rc, rsb, rsg = O.quantize(xh, O.DYNAMIC)
+        assert np.array_equal(codes[i].cpu().numpy(), rc)
+        assert np.array_equal(sbs[i].cpu().numpy(), O.swizzle_scales(rsb, x.shape[1]))
+        _, y16, _, _ = O.fake_quant(xh)
+        assert np.array_equal(_bits16(ys[i]), y16)
+
+
+def test_launch_counter_counts_kernels():
+    x = S.activations(64, 256, seed=1, device=DEV)
+    n0 = Q.nvfp4_launch_count()
+    Q.nvfp4_quantize(x)                      # amax + encode
+    Q.nvfp4_quantize(x, Q.FROZEN_GLOBAL, tensor_scale=torch.ones(1, device=DEV))  # encode
+    assert Q.nvfp4_launch_count() - n0 == 3
