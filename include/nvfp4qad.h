@@ -285,6 +285,35 @@ nvfp4_status qad_kl_fwd_bwd(const void* teacher, const void* student, nvfp4_dtyp
                             float grad_scale, void* workspace, size_t workspace_bytes,
                             void* stream);
 
+/* ------------------------------------------------------------------------
+ * qad_kl_fwd_bwd without a workspace argument, for callers that cannot
+ * allocate device memory when they compute the loss (a framework whose
+ * caching allocator holds the device budget, a fixed pre-planned memory
+ * layout, or a path where a possibly synchronizing cudaMalloc is not
+ * acceptable).  The method described on the pages has no counterpart of
+ * this; it is a deployment convenience.
+ *
+ * Same arguments and results as qad_kl_fwd_bwd, minus the workspace.  The
+ * per-row scratch is a static device array inside the library, of
+ * NVFP4_KL_NOALLOC_MAX_ROWS floats (256 KiB), held on every GPU that loads
+ * the library until the process exits; nothing is allocated by the call.
+ *   - rows > NVFP4_KL_NOALLOC_MAX_ROWS returns NVFP4_ERR_SHAPE before any
+ *     launch.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - All calls on a device share the array and each call overwrites it: two
+ *     calls that can run at the same time on the GPU (different streams,
+ *     without ordering between them) race and may return wrong losses.
+ *     Order them on one stream or with events.
+ * ------------------------------------------------------------------------ */
+#define NVFP4_KL_NOALLOC_MAX_ROWS 65536
+
+nvfp4_status qad_kl_fwd_bwd_noalloc(const void* teacher, const void* student, nvfp4_dtype dtype,
+                                    int64_t rows, int64_t vocab, int64_t ld, float temperature,
+                                    float* loss, float* row_kl, void* dlogits, int64_t ld_grad,
+                                    float grad_scale, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

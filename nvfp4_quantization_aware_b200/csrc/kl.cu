@@ -398,3 +398,52 @@ nvfp4_status qad_kl_fwd_bwd(const void* teacher, const void* student, nvfp4_dtyp
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ allocation-free variant
+//
+// Some callers cannot allocate device memory at the point where they need the
+// loss: code running inside a framework whose caching allocator already owns
+// the device memory budget, callers with a fixed, pre-planned memory layout,
+// and code paths where a cudaMalloc (which may synchronize the device) is not
+// acceptable.  qad_kl_fwd_bwd_noalloc serves them: its per-row scratch lives
+// in the file-scope array below, which every GPU that loads this library keeps
+// until the process exits (kKlNoAllocMaxRows floats = 256 KiB per device).
+
+namespace nvfp4 {
+
+constexpr int64_t kKlNoAllocMaxRows = 65536;
+static __device__ __align__(256) float g_kl_noalloc_rows[kKlNoAllocMaxRows];
+
+// Device address of g_kl_noalloc_rows, looked up once per device.  In host
+// code the array's name only stands for the symbol; the address a kernel may
+// use comes from cudaGetSymbolAddress with that device current.
+constexpr int kKlNoAllocMaxDevices = 64;
+static void* g_kl_noalloc_ptr[kKlNoAllocMaxDevices] = {};
+
+static nvfp4_status kl_noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (dev < 0 || dev >= kKlNoAllocMaxDevices) return NVFP4_ERR_UNSUPPORTED;
+  if (g_kl_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_kl_noalloc_rows) != cudaSuccess || p == nullptr) return NVFP4_ERR_CUDA;
+    g_kl_noalloc_ptr[dev] = p;
+  }
+  *out = g_kl_noalloc_ptr[dev];
+  return NVFP4_OK;
+}
+
+}  // namespace nvfp4
+
+extern "C" nvfp4_status qad_kl_fwd_bwd_noalloc(const void* teacher, const void* student, nvfp4_dtype dtype,
+                                               int64_t rows, int64_t vocab, int64_t ld, float temperature,
+                                               float* loss, float* row_kl, void* dlogits, int64_t ld_grad,
+                                               float grad_scale, void* stream) {
+  if (rows > nvfp4::kKlNoAllocMaxRows) return NVFP4_ERR_SHAPE;
+  void* scratch = nullptr;
+  nvfp4_status st = nvfp4::kl_noalloc_scratch(&scratch);
+  if (st != NVFP4_OK) return st;
+  // every row's slot is written before it is read, so nothing needs clearing
+  return qad_kl_fwd_bwd(teacher, student, dtype, rows, vocab, ld, temperature, loss, row_kl, dlogits, ld_grad,
+                        grad_scale, scratch, (size_t)nvfp4::kKlNoAllocMaxRows * sizeof(float), stream);
+}
