@@ -469,6 +469,35 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_case(case: str):
+    """Small single-kernel cases for ncu captures (inputs larger than L2, a
+    few GB on the device at most): each kernel runs 2 warm-up + 3 launches."""
+    import nvfp4_quantization_aware_b200 as Q
+    from nvfp4_quantization_aware_b200 import synthetic as S
+    dev = torch.device("cuda", 0)
+    if case == "quant":
+        xs = S.weight_sweep(seed=0, device=dev, experts=48, lm_head=False)  # 48 x 4 MiB = 201 MB
+        ts = torch.zeros(len(xs), device=dev)
+        sbs = [torch.empty(x.shape[0], x.shape[1] // 16, dtype=torch.uint8, device=dev) for x in xs]
+        cd = [torch.empty(x.shape[0], x.shape[1] // 2, dtype=torch.uint8, device=dev) for x in xs]
+        for _ in range(5):
+            Q.nvfp4_quantize_grouped(xs, Q.DYNAMIC, tensor_scales=ts, block_scales=sbs, codes=cd)
+            Q.nvfp4_quantize_grouped(xs, Q.FROZEN_ALL, tensor_scales=ts, block_scales=sbs, codes=cd)
+    elif case == "gemm":
+        w = S.weights(4096, 4096, seed=1, device=dev)
+        x = S.channel_scaled_activations(8192, 4096, seed=0, device=dev)
+        a = Q.nvfp4_quantize(x, Q.DYNAMIC, layout=Q.SCALES_MMA)
+        b = Q.nvfp4_quantize(w, Q.DYNAMIC, layout=Q.SCALES_MMA)
+        for _ in range(5):
+            Q.nvfp4_gemm_w4a4(*a, *b)
+    elif case == "kl":
+        d = S.distill_logits(seed=0, device=dev, rows=2048)  # 2 x 512 MiB
+        for _ in range(5):
+            Q.qad_kl_fwd_bwd(d["teacher"], d["student"])
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": case, "ok": True}))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -477,7 +506,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-secondary", action="store_true", help="skip the GEMM and KL measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["quant", "gemm", "kl"], default=None,
+                    help="run one small single-kernel case (for ncu captures) and exit")
     args = ap.parse_args()
+    if args.profile:
+        run_profile_case(args.profile)
+        return
     if args.warmup < 3:
         args.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "1"))

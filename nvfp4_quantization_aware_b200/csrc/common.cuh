@@ -119,16 +119,17 @@ NVFP4_DEV void e2m1x2_decode(uint32_t byte, float& lo, float& hi) {
 
 // Correctly rounded quotient x / d for a divisor shared by a whole block,
 // from r = RN(1/d) (computed once per block with __frcp_rn) and Markstein's
-// FMA correction: q0 = RN(x r); e = x - q0 d (exact through the FMA);
-// q = RN(q0 + e r).  The sign of x is copied onto q so that x = -0 gives -0.
-// Used only when d lies in [2^-90, 2^90]; the library's self-test
-// (nvfp4_selftest_division) compares it with __fdiv_rn for every bf16
-// significand of x against every binary32 significand of d.
+// FMA correction: q0 = RN(x r); the remainder x - q0 d is exact through the
+// FMA; q = RN(q0 + (x - q0 d) r).  The remainder is formed as -(q0 d - x) so
+// that both negations are free FMA operand modifiers and x = -0 yields -0
+// (q0 = -0, q0 d - x = +0, -(+0) r + q0 = -0).  Used only when d lies in
+// [2^-90, 2^90]; the library's self-test (nvfp4_selftest_division) compares
+// it with __fdiv_rn for every bf16 significand and sign of x (and +-0)
+// against every binary32 significand of d.
 NVFP4_DEV float div_by_block_scale(float x, float d, float r) {
-  float q0 = __fmul_rn(x, r);
-  float e = __fmaf_rn(-q0, d, x);
-  float q = __fmaf_rn(e, r, q0);
-  return __uint_as_float((__float_as_uint(q) & 0x7FFFFFFFu) | (__float_as_uint(x) & 0x80000000u));
+  const float q0 = __fmul_rn(x, r);
+  const float e = __fmaf_rn(q0, d, -x);
+  return __fmaf_rn(-e, r, q0);
 }
 
 NVFP4_DEV bool block_scale_in_fast_range(float d) {

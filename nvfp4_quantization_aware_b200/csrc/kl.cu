@@ -14,11 +14,17 @@
 //   1. a TMA bulk copy (cp.async.bulk, completion on an mbarrier) brings the
 //      two slices from HBM into shared memory -- the only HBM read of the
 //      logits;
-//   2. slice max of both rows -> exchanged through distributed shared memory;
-//   3. slice sums S_t, S_s and X = sum e_t (w_t - w_s) -> exchanged;
-//   4. dLogits from the on-chip slice, 16-byte stores.
-// Work is in the log2 domain: w = z * log2(e) / T, e = 2^(w - max w).  Per-row
-// KL goes to the workspace; a second one-CTA kernel sums the rows in a fixed
+//   2. one online pass over the slice keeps, per thread, running maxima of
+//      both rows and the sums S_t = sum 2^d_t, S_s = sum 2^d_s and
+//      Y = sum 2^d_t (d_t - d_s) relative to those maxima (rescaled when a
+//      maximum grows), merged across the CTA and then pushed into every peer's
+//      shared memory: one cluster barrier per row;
+//   3. dLogits from the on-chip slice, 16-byte stores.  Of the two
+//      exponentials per logit pair here, one runs on the MUFU unit and one as
+//      a polynomial on the FMA pipe, so that the MUFU unit (16 results per SM
+//      and clock) does not cap the kernel below the HBM rate.
+// Work is in the log2 domain: w = z * log2(e) / T, d = w - max w.  Per-row KL
+// goes to the workspace; a second one-CTA kernel sums the rows in a fixed
 // order (in double) into the mean, so the loss is deterministic.
 #include <cooperative_groups.h>
 
@@ -28,13 +34,80 @@ namespace cg = cooperative_groups;
 
 namespace nvfp4 {
 
-constexpr int kKlThreads = 512;
+constexpr int kKlThreads = 256;
 constexpr int kKlWarps = kKlThreads / 32;
 constexpr int kKlMaxCluster = 8;
 NVFP4_DEV float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x for x <= 0 on the FMA pipe: x = n + f with n = rint(x), f in
+// [-1/2, 1/2]; 2^f by a degree-5 polynomial (least-squares fit of 2^f on 2000
+// Chebyshev nodes of [-1/2, 1/2], coefficients rounded to binary32; maximum
+// relative error 1.8e-7 over the interval); 2^n applied by adding n to the
+// exponent field.  x is clamped at -126 so the result stays normal (2^-126 is
+// below anything the gradient can resolve).
+NVFP4_DEV float exp2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float n = rintf(x);
+  const float f = x - n;
+  float p = 0.0013400432653725147f;
+  p = fmaf(p, f, 0.009676037356257439f);
+  p = fmaf(p, f, 0.05550327152013779f);
+  p = fmaf(p, f, 0.2402210682630539f);
+  p = fmaf(p, f, 0.6931471824645996f);
+  p = fmaf(p, f, 1.0000001192092896f);
+  return __int_as_float(__float_as_int(p) + ((int)n << 23));
+}
+
+// Running softmax statistics of a (teacher, student) pair of rows, in the
+// log2 domain, relative to the running maxima mt and ms:
+//   St = sum 2^(w_t - mt), Ss = sum 2^(w_s - ms),
+//   Y  = sum 2^(w_t - mt) ((w_t - mt) - (w_s - ms)).
+struct KlStats {
+  float mt, ms, St, Ss, Y;
+};
+
+constexpr float kNoMax = -1.0e30f;  // start value of the running maxima
+
+NVFP4_DEV void stats_init(KlStats& a) {
+  a.mt = kNoMax;
+  a.ms = kNoMax;
+  a.St = a.Ss = a.Y = 0.f;
+}
+
+// Re-express `a` relative to new maxima (Mt, Ms) >= (a.mt, a.ms): the terms
+// scale by 2^(m - M) and every d shifts by (M - m).
+NVFP4_DEV void stats_rebase(KlStats& a, float Mt, float Ms) {
+  const float ft = ex2(a.mt - Mt), fs = ex2(a.ms - Ms);
+  const float c = (Mt - a.mt) - (Ms - a.ms);
+  a.Y = ft * fmaf(-c, a.St, a.Y);
+  a.St *= ft;
+  a.Ss *= fs;
+  a.mt = Mt;
+  a.ms = Ms;
+}
+
+NVFP4_DEV KlStats stats_merge(KlStats a, KlStats b) {
+  const float Mt = fmaxf(a.mt, b.mt), Ms = fmaxf(a.ms, b.ms);
+  stats_rebase(a, Mt, Ms);
+  stats_rebase(b, Mt, Ms);
+  a.St += b.St;
+  a.Ss += b.Ss;
+  a.Y += b.Y;
+  return a;
+}
+
+NVFP4_DEV KlStats stats_shfl_xor(const KlStats& a, int o) {
+  KlStats b;
+  b.mt = __shfl_xor_sync(0xFFFFFFFFu, a.mt, o);
+  b.ms = __shfl_xor_sync(0xFFFFFFFFu, a.ms, o);
+  b.St = __shfl_xor_sync(0xFFFFFFFFu, a.St, o);
+  b.Ss = __shfl_xor_sync(0xFFFFFFFFu, a.Ss, o);
+  b.Y = __shfl_xor_sync(0xFFFFFFFFu, a.Y, o);
+  return b;
 }
 
 template <typename T>
@@ -78,31 +151,6 @@ struct KlArgs {
   int64_t ld_grad;
 };
 
-// Block-wide reduction of NV values (sum or max) into warp 0's lane 0..NV-1
-// results broadcast through shared memory.
-template <int NV, bool MAX>
-NVFP4_DEV void block_reduce(float (&v)[NV], float* scratch /* [kKlWarps][NV] */) {
-#pragma unroll
-  for (int i = 0; i < NV; ++i)
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      float w = __shfl_xor_sync(0xFFFFFFFFu, v[i], o);
-      v[i] = MAX ? fmaxf(v[i], w) : v[i] + w;
-    }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0)
-#pragma unroll
-    for (int i = 0; i < NV; ++i) scratch[warp * NV + i] = v[i];
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    float acc = scratch[i];
-    for (int w = 1; w < kKlWarps; ++w) acc = MAX ? fmaxf(acc, scratch[w * NV + i]) : acc + scratch[w * NV + i];
-    v[i] = acc;
-  }
-  __syncthreads();
-}
-
 // Stand-in for positions of the shared-memory slice that hold no logit (the
 // alignment pad before and after the slice): exp underflows to 0 and it never
 // wins the max while the slice holds at least one real logit.
@@ -115,8 +163,8 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
   constexpr int ESZ = (int)sizeof(T);
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ uint64_t bar;
-  __shared__ float red[kKlWarps * 3];
-  __shared__ float xchg[8];  // [0..1] slice max (t, s); [2..4] slice sums (S_t, S_s, Y)
+  __shared__ KlStats warp_stats[kKlWarps];
+  __shared__ KlStats peer_stats[kKlMaxCluster];  // written by every CTA of the cluster
   __shared__ int s_ok;
 
   cg::cluster_group cluster = cg::this_cluster();
@@ -160,10 +208,7 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
   // head, tail and pad slots with plain accesses (disjoint from the bulk copy)
   for (int j = threadIdx.x; j < cap; j += kKlThreads) {
     const int i = j - off;  // logit index inside the slice
-    if (i >= 0 && i < head) {
-      st[j] = gt[i];
-      ss[j] = gs[i];
-    } else if (i >= tail0 && i < n) {
+    if ((i >= 0 && i < head) || (i >= tail0 && i < n)) {
       st[j] = gt[i];
       ss[j] = gs[i];
     } else if (i < 0 || i >= n) {
@@ -177,77 +222,58 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
 
   const uint4* vt = reinterpret_cast<const uint4*>(st);
   const uint4* vs = reinterpret_cast<const uint4*>(ss);
+  const float a = args.a;  // log2(e) / T > 0
 
-  // ---- pass 1: slice max of z_t and z_s
-  float mx[2] = {-INFINITY, -INFINITY};
+  // ---- online statistics over this thread's vectors
+  KlStats my;
+  stats_init(my);
   if (ok) {
     for (int k = threadIdx.x; k < nvec; k += kKlThreads) {
-      float zt[V8], zs[V8];
-      E::unpack(vt[k], zt);
-      E::unpack(vs[k], zs);
+      float wt[V8], ws[V8];
+      E::unpack(vt[k], wt);
+      E::unpack(vs[k], ws);
+      float lt = kNoMax, ls = kNoMax;
 #pragma unroll
       for (int j = 0; j < V8; ++j) {
-        mx[0] = fmaxf(mx[0], zt[j]);
-        mx[1] = fmaxf(mx[1], zs[j]);
+        wt[j] *= a;
+        ws[j] *= a;
+        lt = fmaxf(lt, wt[j]);
+        ls = fmaxf(ls, ws[j]);
       }
-    }
-  }
-  block_reduce<2, true>(mx, red);
-  if (threadIdx.x == 0) {
-    xchg[0] = mx[0];
-    xchg[1] = mx[1];
-  }
-  cluster.sync();
-  float Mt = -INFINITY, Ms = -INFINITY;
-  for (int r = 0; r < csize; ++r) {
-    const float* peer = cluster.map_shared_rank(xchg, r);
-    Mt = fmaxf(Mt, peer[0]);
-    Ms = fmaxf(Ms, peer[1]);
-  }
-  // log2 domain: w = z * a with a = log2(e) / T > 0, so max w = max(z) * a;
-  // d = w - max w <= 0 is formed by one FMA per logit.
-  const float a = args.a;
-  const float Wt = Mt * a, Ws = Ms * a;
-
-  // ---- pass 2: S_t = sum 2^d_t, S_s = sum 2^d_s, Y = sum 2^d_t (d_t - d_s)
-  float sums[3] = {0.f, 0.f, 0.f};
-  if (ok) {
-    for (int k = threadIdx.x; k < nvec; k += kKlThreads) {
-      float zt[V8], zs[V8];
-      E::unpack(vt[k], zt);
-      E::unpack(vs[k], zs);
+      const float Mt = fmaxf(my.mt, lt), Ms = fmaxf(my.ms, ls);
+      if (Mt != my.mt || Ms != my.ms) stats_rebase(my, Mt, Ms);
 #pragma unroll
       for (int j = 0; j < V8; ++j) {
-        const float dt = fmaf(zt[j], a, -Wt), ds = fmaf(zs[j], a, -Ws);
+        const float dt = wt[j] - Mt, ds = ws[j] - Ms;
         const float et = ex2(dt), es = ex2(ds);
-        sums[0] += et;
-        sums[1] += es;
-        sums[2] = fmaf(et, dt - ds, sums[2]);
+        my.St += et;
+        my.Ss += es;
+        my.Y = fmaf(et, dt - ds, my.Y);
       }
     }
   }
-  block_reduce<3, false>(sums, red);
-  if (threadIdx.x == 0) {
-    xchg[2] = sums[0];
-    xchg[3] = sums[1];
-    xchg[4] = sums[2];
+  // ---- merge: warp, CTA, then push to every CTA of the cluster
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) my = stats_merge(my, stats_shfl_xor(my, o));
+  if ((threadIdx.x & 31) == 0) warp_stats[threadIdx.x >> 5] = my;
+  __syncthreads();
+  if (threadIdx.x < csize) {
+    KlStats c = warp_stats[0];
+    for (int w = 1; w < kKlWarps; ++w) c = stats_merge(c, warp_stats[w]);
+    KlStats* dst = cluster.map_shared_rank(peer_stats, (int)threadIdx.x);
+    dst[crank] = c;
   }
-  cluster.sync();
-  float St = 0.f, Ss = 0.f, Y = 0.f;
-  for (int r = 0; r < csize; ++r) {
-    const float* peer = cluster.map_shared_rank(xchg, r);
-    St += peer[2];
-    Ss += peer[3];
-    Y += peer[4];
-  }
+  cluster.sync();  // all pushes visible; no CTA reads a peer after this point
+  KlStats row_stats = peer_stats[0];
+  for (int r = 1; r < csize; ++r) row_stats = stats_merge(row_stats, peer_stats[r]);
+  const float Wt = row_stats.mt, Ws = row_stats.ms, St = row_stats.St, Ss = row_stats.Ss;
   if (crank == 0 && threadIdx.x == 0) {
-    // KL = sum p_t (log p_t - log p_s) = ln2 * (Y / S_t + log2(S_s / S_t)):
-    // the max shifts cancel, so only O(1) terms are combined.
-    const float kl = 0.69314718055994531f * (Y / St + log2f(Ss / St));
+    // KL = sum p_t (log p_t - log p_s) = ln2 * (Y / S_t + log2(S_s / S_t))
+    const float kl = 0.69314718055994531f * (row_stats.Y / St + log2f(Ss / St));
     args.row_kl[row] = ok ? kl : __int_as_float(0x7FC00000);
   }
 
-  // ---- pass 3: dLogits = gscale * (p_s - p_t), p = 2^(w - max w - log2 S)
+  // ---- dLogits = gscale * (p_s - p_t), p = 2^(w - max w - log2 S)
   if (args.dlogits != nullptr && ok) {
     const float g = args.gscale;
     const float Lt = Wt + __log2f(St), Ls = Ws + __log2f(Ss);
@@ -259,7 +285,7 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
       E::unpack(vs[k], zs);
 #pragma unroll
       for (int j = 0; j < V8; ++j) {
-        const float pt = ex2(fmaf(zt[j], a, -Lt));
+        const float pt = exp2_poly(fmaf(zt[j], a, -Lt));
         const float ps = ex2(fmaf(zs[j], a, -Ls));
         o[j] = g * (ps - pt);
       }
@@ -273,8 +299,6 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
       }
     }
   }
-  // keep this CTA's shared memory alive until every peer has read it
-  cluster.sync();
 }
 
 // loss = mean of row_kl in a fixed order (double accumulation); optionally

@@ -7,13 +7,14 @@
 // (recomputed from the max on every call) or frozen (passed in).
 //
 // Work decomposition.  These kernels stream HBM: every input byte is read
-// once per pass with 16-byte non-allocating loads and every output written
-// once.  A lane owns 8 consecutive elements (16 B of bf16), so a lane pair
-// owns one 16-element block and the block max is one shuffle (lane ^ 1).  A
-// warp covers a 256-element chunk of a row; chunks are numbered row-major and
-// each warp takes UNROLL consecutive chunks per iteration so that several
-// independent 16-byte loads per lane are in flight.  Grids are persistent:
-// a multiple of the SM count, grid-striding over chunks.
+// once per pass and every output byte written once.  A lane owns one whole
+// 16-element block (32 bytes of bf16, one 256-bit load), so the block max and
+// the block scale are computed once per block without any shuffle, and a warp
+// covers a 512-element chunk of a row.  Chunks are numbered row-major per
+// tensor; chunk -> (row, column) uses a precomputed multiply-shift divider.
+// Each warp takes kUnroll consecutive chunks per iteration so that several
+// independent loads per lane are in flight.  Grids are persistent: exactly the
+// resident capacity of the GPU (SM count x resident CTAs), grid-striding.
 //
 // Dynamic mode is two launches in stream order: group_amax_kernel folds each
 // tensor's max |x| into a workspace word (max is exact, so any order gives the
@@ -24,8 +25,142 @@ namespace nvfp4 {
 
 constexpr int kThreads = 256;           // 8 warps per CTA
 constexpr int kWarps = kThreads / 32;
-constexpr int kUnroll = 4;              // chunks per warp per iteration
-constexpr int kChunk = 256;             // elements per warp per chunk
+constexpr int kUnroll = 4;              // chunks per warp per iteration (dequantize)
+constexpr int kChunk = 256;             // elements per warp per chunk (dequantize: 8 per lane)
+constexpr int kQUnroll = 2;             // chunks per warp per iteration (amax / encode)
+constexpr int kQChunk = 512;            // elements per warp per chunk (amax / encode: 16 per lane)
+
+// Unsigned 32-bit division by a run-time invariant divisor through one
+// multiply-high and two shifts (Granlund & Montgomery, "Division by Invariant
+// Integers using Multiplication", 1994, section 4): for d >= 1 with
+// l = ceil(log2 d), m = floor(2^32 (2^l - d) / d) + 1,
+//   q = (t + ((n - t) >> min(l, 1))) >> max(l - 1, 0),  t = mulhi(m, n),
+// exact for every 32-bit n.
+struct FastDiv {
+  uint32_t d, m, s1, s2;
+};
+
+static FastDiv make_fastdiv(uint32_t d) {
+  uint32_t l = 0;
+  while (l < 32 && (1ull << l) < d) ++l;
+  FastDiv f;
+  f.d = d;
+  f.m = (uint32_t)((((1ull << l) - d) << 32) / d + 1);
+  f.s1 = l < 1 ? l : 1;
+  f.s2 = l > 0 ? l - 1 : 0;
+  return f;
+}
+
+NVFP4_DEV uint32_t fastdiv(uint32_t n, const FastDiv& f) {
+  const uint32_t t = __umulhi(f.m, n);
+  return (t + ((n - t) >> f.s1)) >> f.s2;
+}
+
+// 32-byte (256-bit) streaming load and store.
+NVFP4_DEV void ld_stream_v8(const void* p, uint32_t (&r)[8]) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "l"(p));
+}
+
+NVFP4_DEV void st_stream_v8(void* p, const uint32_t (&r)[8]) {
+  asm volatile("st.global.cs.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(r[0]), "r"(r[1]), "r"(r[2]),
+               "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
+NVFP4_DEV void st_stream_v2(void* p, uint32_t a, uint32_t b) {
+  asm volatile("st.global.cs.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(a), "r"(b) : "memory");
+}
+
+// One 16-element block held by a lane.
+template <typename T>
+struct Block16;
+
+template <>
+struct Block16<__nv_bfloat16> {
+  uint32_t w[8];
+  // wide: the address is 32-byte aligned (one 256-bit load); else 16-byte
+  NVFP4_DEV void load(const __nv_bfloat16* p, bool wide) {
+    if (wide) {
+      ld_stream_v8(p, w);
+    } else {
+      const uint4 a = ld_stream_v4(p), b = ld_stream_v4(p + 8);
+      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+      w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+    }
+  }
+  NVFP4_DEV void zero() {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = 0u;
+  }
+  NVFP4_DEV void to_f32(float (&v)[16]) const {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[2 * i] = bf16lo_to_f32(w[i]);
+      v[2 * i + 1] = bf16hi_to_f32(w[i]);
+    }
+  }
+  NVFP4_DEV static void store(__nv_bfloat16* p, const float (&v)[16], bool wide) {
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+    if (wide) {
+      st_stream_v8(p, o);
+    } else {
+      st_stream_v4(p, make_uint4(o[0], o[1], o[2], o[3]));
+      st_stream_v4(p + 8, make_uint4(o[4], o[5], o[6], o[7]));
+    }
+  }
+};
+
+template <>
+struct Block16<float> {
+  uint32_t w[16];
+  NVFP4_DEV void load(const float* p, bool wide) {
+    if (wide) {
+      uint32_t a[8], b[8];
+      ld_stream_v8(p, a);
+      ld_stream_v8(p + 8, b);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        w[i] = a[i];
+        w[8 + i] = b[i];
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 a = ld_stream_v4(p + 4 * j);
+        w[4 * j] = a.x; w[4 * j + 1] = a.y; w[4 * j + 2] = a.z; w[4 * j + 3] = a.w;
+      }
+    }
+  }
+  NVFP4_DEV void zero() {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) w[i] = 0u;
+  }
+  NVFP4_DEV void to_f32(float (&v)[16]) const {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(w[i]);
+  }
+  NVFP4_DEV static void store(float* p, const float (&v)[16], bool wide) {
+    uint32_t a[8], b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      a[i] = __float_as_uint(v[i]);
+      b[i] = __float_as_uint(v[8 + i]);
+    }
+    if (wide) {
+      st_stream_v8(p, a);
+      st_stream_v8(p + 8, b);
+    } else {
+      st_stream_v4(p, make_uint4(a[0], a[1], a[2], a[3]));
+      st_stream_v4(p + 4, make_uint4(a[4], a[5], a[6], a[7]));
+      st_stream_v4(p + 8, make_uint4(b[0], b[1], b[2], b[3]));
+      st_stream_v4(p + 12, make_uint4(b[4], b[5], b[6], b[7]));
+    }
+  }
+};
 
 // ------------------------------------------------------------------ input traits
 
@@ -116,9 +251,9 @@ struct GTensor {
   float* ts;            // tensor scale: written (DYNAMIC) or read
   int64_t ld_x, ld_out;
   int64_t cols;
-  int64_t cpr;          // chunks per row = ceil(cols / 256)
-  int64_t chunk0;       // first chunk of this tensor
+  int64_t chunk0;       // first chunk of this tensor in the group
   int64_t kchunks;      // ceil(cols / 64), MMA scale layout
+  FastDiv cpr;          // chunks per row = ceil(cols / 512)
 };
 
 struct GroupArgs {
@@ -128,6 +263,8 @@ struct GroupArgs {
   int layout;           // nvfp4_scale_layout of written block scales
   int64_t total_chunks;
   unsigned* amax;       // DYNAMIC: n words holding max |x| as float bits (zeroed first)
+  int x_wide;           // every input row start is 32-byte aligned: 256-bit loads
+  int out_wide;         // codes rows 8-byte aligned (8-byte stores) / y rows 32-byte aligned
 };
 
 // Advance `t` to the tensor owning `chunk` (chunks are visited in increasing
@@ -137,28 +274,36 @@ NVFP4_DEV int find_tensor(const GroupArgs& a, int64_t chunk, int t) {
   return t;
 }
 
+// Row and first column of this lane's block for a chunk of tensor g.
 NVFP4_DEV void chunk_pos(const GTensor& g, int64_t chunk, int lane, int64_t& row, int64_t& col) {
-  const int64_t c = chunk - g.chunk0;
-  row = c / g.cpr;
-  col = (c - row * g.cpr) * kChunk + lane * 8;
+  const uint32_t c = (uint32_t)(chunk - g.chunk0);
+  const uint32_t r = fastdiv(c, g.cpr);
+  row = r;
+  col = (int64_t)(c - r * g.cpr.d) * kQChunk + lane * 16;
 }
 
 // ------------------------------------------------------------------ amax
 
-// Per-tensor max |x| of a group: each warp reduces the chunks of one
-// iteration and folds them into the tensor's word with atomicMax on the float
-// bits (order-independent: |x| >= 0 compares like its bit pattern).
+// Per-tensor max |x| of a group.  Every warp visits chunks in increasing
+// order, so the tensor it works on only changes forward: it keeps a running
+// max for the current tensor across iterations and folds it into the tensor's
+// word with one atomicMax on the float bits when the tensor changes and at
+// the end (|x| >= 0 compares like its bit pattern; max is exact, so the order
+// of the atomics does not matter).  Same-address atomics stay at about one per
+// warp and tensor.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) group_amax_kernel(const __grid_constant__ GroupArgs a) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * kWarps;
   int cur = 0;
-  for (int64_t c0 = warp * kUnroll; c0 < a.total_chunks; c0 += nwarps * kUnroll) {
-    Lane8<T> in[kUnroll];
-    int tid[kUnroll];
+  int mt = -1;      // tensor of the running max
+  float m = 0.0f;   // running max of this lane
+  for (int64_t c0 = warp * kQUnroll; c0 < a.total_chunks; c0 += nwarps * kQUnroll) {
+    Block16<T> in[kQUnroll];
+    int tid[kQUnroll];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int u = 0; u < kQUnroll; ++u) {
       const int64_t c = c0 + u;
       in[u].zero();
       tid[u] = -1;
@@ -168,27 +313,26 @@ __global__ void __launch_bounds__(kThreads) group_amax_kernel(const __grid_const
         int64_t row, col;
         chunk_pos(g, c, lane, row, col);
         tid[u] = cur;
-        if (col < g.cols) in[u].load(reinterpret_cast<const T*>(g.x) + row * g.ld_x + col);
+        if (col < g.cols) in[u].load(reinterpret_cast<const T*>(g.x) + row * g.ld_x + col, a.x_wide != 0);
       }
     }
-    float m = 0.0f;
-    int mt = tid[0];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      if (tid[u] != mt) {  // chunk of the next tensor: flush the running max
+    for (int u = 0; u < kQUnroll; ++u) {
+      if (tid[u] < 0) continue;  // warp-uniform
+      if (tid[u] != mt) {         // warp-uniform: flush the previous tensor's max
         const float w = warp_max(m);
         if (lane == 0 && mt >= 0 && w > 0.0f) atomicMax(a.amax + mt, __float_as_uint(w));
         m = 0.0f;
         mt = tid[u];
       }
-      float v[8];
+      float v[16];
       in[u].to_f32(v);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
+      for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
     }
-    const float w = warp_max(m);
-    if (lane == 0 && mt >= 0 && w > 0.0f) atomicMax(a.amax + mt, __float_as_uint(w));
   }
+  const float w = warp_max(m);
+  if (lane == 0 && mt >= 0 && w > 0.0f) atomicMax(a.amax + mt, __float_as_uint(w));
 }
 
 // ------------------------------------------------------------------ encode
@@ -213,89 +357,101 @@ __global__ void __launch_bounds__(kThreads) group_encode_kernel(const __grid_con
   int cur = 0;
   int sg_t = -1;  // tensor whose scale is cached below
   float sg = 0.0f, denom6 = 0.0f;
-  for (int64_t c0 = warp * kUnroll; c0 < a.total_chunks; c0 += nwarps * kUnroll) {
-    Lane8<T> in[kUnroll];
-    uint32_t sb_in[kUnroll];
-    int tid[kUnroll];
-    int64_t rows_[kUnroll], cols_[kUnroll];
+  for (int64_t c0 = warp * kQUnroll; c0 < a.total_chunks; c0 += nwarps * kQUnroll) {
+    Block16<T> in[kQUnroll];
+    uint32_t sb_in[kQUnroll];
+    int tid[kQUnroll];
+    int64_t row_[kQUnroll], col_[kQUnroll];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int u = 0; u < kQUnroll; ++u) {
       const int64_t c = c0 + u;
       in[u].zero();
       sb_in[u] = 0u;
       tid[u] = -1;
-      rows_[u] = 0;
-      cols_[u] = 0;
+      row_[u] = 0;
+      col_[u] = 0;
       if (c < a.total_chunks) {
         cur = find_tensor(a, c, cur);
         const GTensor& g = a.t[cur];
         int64_t row, col;
         chunk_pos(g, c, lane, row, col);
         tid[u] = cur;
-        rows_[u] = row;
-        cols_[u] = col;
+        row_[u] = row;
+        col_[u] = col;
         if (col < g.cols) {
-          in[u].load(reinterpret_cast<const T*>(g.x) + row * g.ld_x + col);
+          in[u].load(reinterpret_cast<const T*>(g.x) + row * g.ld_x + col, a.x_wide != 0);
           if (frozen_all) sb_in[u] = (uint32_t)__ldg(g.sb + row * (g.cols >> 4) + (col >> 4));
         }
       }
     }
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int u = 0; u < kQUnroll; ++u) {
       const int t = tid[u];
       if (t < 0) continue;  // warp-uniform: the whole chunk is past the end
       const GTensor& g = a.t[t];
-      const int64_t row = rows_[u], col = cols_[u];
-      const bool ok = col < g.cols;
+      const int64_t row = row_[u], col = col_[u];
+      if (col >= g.cols) continue;  // this lane's block lies past the row end
       if (t != sg_t) {
         sg = tensor_scale_of(a, t);
         denom6 = __fmul_rn(6.0f, sg);
         sg_t = t;
       }
-      float v[8];
+      float v[16];
       in[u].to_f32(v);
-      // ---- block scale
+      // ---- block scale: s_b = E4M3(max|x| / (6 s_g)), d = s_b * s_g
       uint32_t sb;
       if (frozen_all) {
         sb = sb_in[u];
       } else {
         float m = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
-        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+        for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
         sb = (sg == 0.0f) ? 0u : e4m3_encode(__fdiv_rn(m, denom6));
       }
       const float d = __fmul_rn(e4m3_decode(sb), sg);
-      // ---- element codes
-      uint32_t word = 0;
+      // ---- element codes: E2M1(x / d), every code +0 when d = 0
+      uint32_t lo = 0, hi = 0;
       if (d != 0.0f) {
-        float q[8];
+        float q[16];
         if (sizeof(T) == 2 && block_scale_in_fast_range(d)) {
           const float r = __frcp_rn(d);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) q[i] = div_by_block_scale(v[i], d, r);
+          for (int i = 0; i < 16; ++i) q[i] = div_by_block_scale(v[i], d, r);
         } else {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(v[i], d);
+          for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(v[i], d);
         }
-        word = e2m1x8_encode(q);
+        float q0[8], q1[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          q0[i] = q[i];
+          q1[i] = q[8 + i];
+        }
+        lo = e2m1x8_encode(q0);
+        hi = e2m1x8_encode(q1);
       }
-      if (!ok) continue;
       // ---- outputs
       if (OUT == Out::Codes) {
-        st_stream_u32(g.codes + row * g.ld_out + (col >> 1), word);
-      } else {
-        float o[8];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float lo, hi;
-          e2m1x2_decode((word >> (8 * j)) & 0xFF, lo, hi);
-          o[2 * j] = __fmul_rn(lo, d);
-          o[2 * j + 1] = __fmul_rn(hi, d);
+        uint8_t* dst = g.codes + row * g.ld_out + (col >> 1);
+        if (a.out_wide) {
+          st_stream_v2(dst, lo, hi);
+        } else {
+          st_stream_u32(dst, lo);
+          st_stream_u32(dst + 4, hi);
         }
-        store8<T>(reinterpret_cast<T*>(g.y) + row * g.ld_out + col, o);
+      } else {
+        float o[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t word = j < 4 ? lo : hi;
+          float a0, a1;
+          e2m1x2_decode((word >> (8 * (j & 3))) & 0xFF, a0, a1);
+          o[2 * j] = __fmul_rn(a0, d);
+          o[2 * j + 1] = __fmul_rn(a1, d);
+        }
+        Block16<T>::store(reinterpret_cast<T*>(g.y) + row * g.ld_out + col, o, a.out_wide != 0);
       }
-      if (!frozen_all && g.sb != nullptr && (lane & 1) == 0) {
+      if (!frozen_all && g.sb != nullptr) {
         const int64_t kb = col >> 4;
         const int64_t off = (a.layout == NVFP4_SCALES_MMA) ? mma_scale_offset(row, kb, g.kchunks)
                                                            : row * (g.cols >> 4) + kb;
@@ -389,6 +545,14 @@ __global__ void selftest_division_kernel(unsigned long long* mismatches, unsigne
       }
     }
   }
+  // signed zeros
+  for (int sgn = 0; sgn < 2; ++sgn) {
+    const float x = sgn ? -0.0f : 0.0f;
+    if (__float_as_uint(div_by_block_scale(x, d, r)) != __float_as_uint(__fdiv_rn(x, d))) {
+      ++bad;
+      atomicCAS(first, ~0ull, ((unsigned long long)i << 16) | 0xFF00ull | (unsigned long long)sgn);
+    }
+  }
   if (bad) atomicAdd(mismatches, bad);
 }
 
@@ -472,22 +636,40 @@ static nvfp4_status check_tensor(const nvfp4_tensor_ref& r, nvfp4_dtype dtype, n
   return NVFP4_OK;
 }
 
+// Persistent grid for a group: at most the resident capacity of the GPU.
+template <typename K>
+static int resident_grid(K kernel, int64_t total_chunks) {
+  static int per_sm = 0;
+  if (per_sm == 0 && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess ||
+                      per_sm <= 0))
+    per_sm = 4;
+  const int64_t per_cta = (int64_t)kWarps * kQUnroll;
+  int64_t need = (total_chunks + per_cta - 1) / per_cta;
+  const int64_t cap = (int64_t)sm_count() * per_sm;
+  if (need > cap) need = cap;
+  return need < 1 ? 1 : (int)need;
+}
+
 template <Out OUT>
 static nvfp4_status launch_group(GroupArgs& a, nvfp4_dtype dtype, void* ws, cudaStream_t s) {
   if (a.n == 0 || a.total_chunks == 0) return NVFP4_OK;
-  Geom g;
-  g.total_chunks = a.total_chunks;
-  const int grid = grid_for(g);
   if (a.mode == NVFP4_DYNAMIC) {
     a.amax = reinterpret_cast<unsigned*>(ws);
     if (cudaMemsetAsync(ws, 0, sizeof(unsigned) * (size_t)a.n, s) != cudaSuccess) return NVFP4_ERR_CUDA;
-    if (dtype == NVFP4_BF16) group_amax_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(a);
-    else group_amax_kernel<float><<<grid, kThreads, 0, s>>>(a);
+    if (dtype == NVFP4_BF16)
+      group_amax_kernel<__nv_bfloat16>
+          <<<resident_grid(group_amax_kernel<__nv_bfloat16>, a.total_chunks), kThreads, 0, s>>>(a);
+    else
+      group_amax_kernel<float><<<resident_grid(group_amax_kernel<float>, a.total_chunks), kThreads, 0, s>>>(a);
     count_launches(1);
     if (launch_status() != NVFP4_OK) return NVFP4_ERR_CUDA;
   }
-  if (dtype == NVFP4_BF16) group_encode_kernel<__nv_bfloat16, OUT><<<grid, kThreads, 0, s>>>(a);
-  else group_encode_kernel<float, OUT><<<grid, kThreads, 0, s>>>(a);
+  if (dtype == NVFP4_BF16)
+    group_encode_kernel<__nv_bfloat16, OUT>
+        <<<resident_grid(group_encode_kernel<__nv_bfloat16, OUT>, a.total_chunks), kThreads, 0, s>>>(a);
+  else
+    group_encode_kernel<float, OUT>
+        <<<resident_grid(group_encode_kernel<float, OUT>, a.total_chunks), kThreads, 0, s>>>(a);
   count_launches(1);
   return launch_status();
 }
@@ -516,6 +698,8 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
   a.layout = (int)layout;
   a.total_chunks = 0;
   a.amax = nullptr;
+  a.x_wide = 1;
+  a.out_wide = 1;
   int64_t group_bytes = 0;
   for (int i = 0; i < n; ++i) {
     const nvfp4_tensor_ref& r = refs[i];
@@ -525,6 +709,7 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
       continue;
     }
     const int64_t bytes = r.rows * r.cols * esz;
+    if (r.rows * ((r.cols + kQChunk - 1) / kQChunk) > 0xFFFFFFFFll) return NVFP4_ERR_SHAPE;
     const bool full = a.n == kMaxGroup;
     const bool over_l2 = mode == NVFP4_DYNAMIC && a.n > 0 && group_bytes + bytes > kL2GroupBytes;
     if (full || over_l2) {
@@ -532,6 +717,8 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
       if (st != NVFP4_OK) return st;
       a.n = 0;
       a.total_chunks = 0;
+      a.x_wide = 1;
+      a.out_wide = 1;
       group_bytes = 0;
     }
     GTensor& g = a.t[a.n++];
@@ -543,11 +730,19 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
     g.ld_x = r.ld_x;
     g.ld_out = r.ld_out;
     g.cols = r.cols;
-    g.cpr = (r.cols + kChunk - 1) / kChunk;
+    const int64_t cpr = (r.cols + kQChunk - 1) / kQChunk;
+    g.cpr = make_fastdiv((uint32_t)cpr);
     g.chunk0 = a.total_chunks;
     g.kchunks = (r.cols / 16 + 3) / 4;
-    a.total_chunks += r.rows * g.cpr;
+    a.total_chunks += r.rows * cpr;
     group_bytes += bytes;
+    // 32-byte rows for 256-bit input loads; 8-byte code rows / 32-byte y rows
+    if (((uintptr_t)r.x & 31u) || ((r.ld_x * esz) & 31)) a.x_wide = 0;
+    if (OUT == Out::Codes) {
+      if (((uintptr_t)r.out & 7u) || (r.ld_out & 7)) a.out_wide = 0;
+    } else {
+      if (((uintptr_t)r.out & 31u) || ((r.ld_out * esz) & 31)) a.out_wide = 0;
+    }
   }
   nvfp4_status st = launch_group<OUT>(a, dtype, ws, s);
   if (st != NVFP4_OK) return st;

@@ -314,3 +314,30 @@ def test_launch_counter_counts_kernels():
     Q.nvfp4_quantize(x)                      # amax + encode
     Q.nvfp4_quantize(x, Q.FROZEN_GLOBAL, tensor_scale=torch.ones(1, device=DEV))  # encode
     assert Q.nvfp4_launch_count() - n0 == 3
+
+
+def test_unaligned_rows_use_narrow_accesses():
+    # input rows 16-byte but not 32-byte aligned, code rows 4-byte but not
+    # 8-byte aligned, fake-quant output rows 16-byte aligned only
+    big = S.weights(37, 160, seed=21, device=DEV, outlier_p=0.01, outlier_mult=30)
+    x = big[:, 8:104]
+    assert (x.data_ptr() % 32) == 16
+    codes_buf = torch.zeros(37, 52, dtype=torch.uint8, device=DEV)
+    codes = codes_buf[:, 4:52]
+    assert codes.stride(0) == 52 and codes.data_ptr() % 8 == 4
+    ref_codes, ref_sb, ref_sg = O.quantize(_host_f32(x), O.DYNAMIC)
+    c, sb, sg = Q.nvfp4_quantize(x, codes=codes)
+    torch.cuda.synchronize()
+    assert np.array_equal(c.cpu().numpy(), ref_codes) and np.array_equal(sb.cpu().numpy(), ref_sb)
+    assert not codes_buf[:, :4].any()  # nothing written outside the view
+    ybuf = torch.zeros(37, 112, dtype=torch.bfloat16, device=DEV)
+    y = ybuf[:, 8:104]
+    Q.nvfp4_fake_quant(x, out=y)
+    _, y16, _, _ = O.fake_quant(_host_f32(x))
+    assert np.array_equal(_bits16(y), y16)
+    assert not ybuf[:, :8].any() and not ybuf[:, 104:].any()
+    # f32 input with 16-byte aligned rows
+    xf = S.activations(9, 200, seed=22, device=DEV, dtype=torch.float32)[:, 4:196]
+    rc, rsb, rsg = O.quantize(_host_f32(xf), O.DYNAMIC)
+    c2, sb2, _ = Q.nvfp4_quantize(xf)
+    assert np.array_equal(c2.cpu().numpy(), rc) and np.array_equal(sb2.cpu().numpy(), rsb)
