@@ -8,7 +8,8 @@
 // tensor scales s_g (Nemotron-3-Nano-30B NVFP4 article, "NVFP4-Format und warum
 // es wichtig ist?").
 //
-// One CTA computes a 128 x BN output tile.  Warp roles:
+// Persistent kernel: one CTA per SM walks the 128 x BN output tiles
+// (t = blockIdx.x, blockIdx.x + gridDim.x, ...).  Warp roles:
 //   warp 0      TMA producer: per K stage (256 elements) the A tile
 //               (128 rows x 128 bytes) and B tile (BN rows x 128 bytes) as 2-D
 //               tiled TMA loads with 128-byte swizzle, and the stage's block
@@ -19,9 +20,14 @@
 //               tcgen05.mma.kind::mxf4nvf4.block_scale (K = 64 each) into an
 //               FP32 accumulator in tensor memory; tcgen05.commit releases the
 //               stage back to the producer.
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator, x (s_gA s_gB), bf16
-//               rounding, stores.
-// STAGES-deep mbarrier ring between producer and MMA; every wait is bounded.
+//   warps 2-9   epilogue (two per TMEM subpartition, half the columns each): tcgen05.ld of the accumulator, x (s_gA s_gB), bf16
+//               rounding into registers, release of the accumulator to the MMA
+//               warp (acc_empty), then the global stores -- which overlap the
+//               next tile's MMAs.
+// A STAGES-deep mbarrier ring between producer and MMA runs across tile
+// boundaries, so the next tile's operands stream in while the epilogue drains.
+// Tensor memory holds one 128 x BN FP32 accumulator (BN = 256 uses half of the
+// 512 columns) plus two sets of block scales; every wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -50,7 +56,8 @@ struct GemmCfg {
   static constexpr int TM_SFB = BN + 2 * 4 * KB_PER_STAGE;        // 2 x 4*KB*NB_SFB columns
   static constexpr int TM_COLS_USED = TM_SFB + 2 * 4 * KB_PER_STAGE * NB_SFB;
   static constexpr int TM_COLS = TM_COLS_USED <= 256 ? 256 : 512;
-  static constexpr int THREADS = 192;
+  static constexpr int EPI_WARPS = 8;            // two per TMEM subpartition, BN/2 columns each
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   // instruction descriptor: E2M1 x E2M1 (format 1), UE4M3 scales, K-major A
   // and B, N >> 3 in bits 17-22, M >> 4 in bits 24-28, dense K = 64.
   static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
@@ -69,6 +76,14 @@ struct GemmParams {
   int c_vec16;           // C base 16-byte aligned and ldc % 8 == 0: 16-byte stores
 };
 
+// Tile t of the persistent schedule -> (m0, n0); N fastest, so the CTAs that
+// run at the same time share A rows and sweep B (both stay in L2).
+NVFP4_DEV void tile_coords(int t, int num_n, int BM, int BN, int& m0, int& n0) {
+  const int mt = t / num_n;
+  m0 = mt * BM;
+  n0 = (t - mt * num_n) * BN;
+}
+
 template <int BN>
 __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
     gemm_w4a4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
@@ -82,15 +97,16 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
   uint8_t* sSFB = sSFA + C::STAGES * C::SFA_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + C::STAGES * C::SFB_BYTES);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* acc_full = empty + C::STAGES;
-  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* acc_full = empty + C::STAGES;   // MMA -> epilogue: accumulator complete
+  uint64_t* acc_empty = acc_full + 1;       // epilogue -> MMA: accumulator drained
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * C::BM;
-  const int n0 = blockIdx.x * C::BN;
   const int num_kt = (p.kchunks + C::KB_PER_STAGE - 1) / C::KB_PER_STAGE;
+  const int num_n = (p.N + C::BN - 1) / C::BN;
+  const int num_tiles = num_n * ((p.M + C::BM - 1) / C::BM);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -98,6 +114,7 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
+    mbar_init(acc_empty, C::EPI_WARPS);  // one arrival per epilogue warp
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -115,95 +132,131 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const int a_tile = m0 / 128;
-      for (int kt = 0; kt < num_kt; ++kt) {
-        const int s = kt % C::STAGES;
-        const uint32_t ph = (uint32_t)(kt / C::STAGES) & 1u;
-        if (!mbar_wait_bounded(&empty[s], ph ^ 1u)) { *abort_flag = 1; break; }
-        if (*abort_flag) break;
-        int nkc = p.kchunks - kt * C::KB_PER_STAGE;
-        if (nkc > C::KB_PER_STAGE) nkc = C::KB_PER_STAGE;
+      int it = 0;  // k-iteration counter across all tiles (ring position)
+      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+        int m0, n0;
+        tile_coords(t, num_n, C::BM, C::BN, m0, n0);
+        const int a_tile = m0 / 128;
         int nsfb = 0;
         for (int j = 0; j < C::NB_SFB; ++j)
           if (n0 / 128 + j < p.b_rowtiles) ++nsfb;
-        const uint32_t bytes = C::A_BYTES + C::B_BYTES + (uint32_t)nkc * 512u * (1u + (uint32_t)nsfb);
-        mbar_expect_tx(&full[s], bytes);
-        tma_load_2d(sA + s * C::A_BYTES, &tmA, kt * (C::BK / 2), m0, &full[s]);
-        tma_load_2d(sB + s * C::B_BYTES, &tmB, kt * (C::BK / 2), n0, &full[s]);
-        const int64_t kc0 = (int64_t)kt * C::KB_PER_STAGE;
-        bulk_g2s(sSFA + s * C::SFA_BYTES, p.a_sf + ((int64_t)a_tile * p.kchunks + kc0) * 512, (uint32_t)nkc * 512u,
-                 &full[s]);
-        for (int j = 0; j < nsfb; ++j)
-          bulk_g2s(sSFB + s * C::SFB_BYTES + j * 512 * C::KB_PER_STAGE,
-                   p.b_sf + ((int64_t)(n0 / 128 + j) * p.kchunks + kc0) * 512, (uint32_t)nkc * 512u, &full[s]);
+        for (int kt = 0; kt < num_kt; ++kt, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t ph = (uint32_t)(it / C::STAGES) & 1u;
+          if (!mbar_wait_bounded(&empty[s], ph ^ 1u)) { *abort_flag = 1; break; }
+          if (*abort_flag) break;
+          int nkc = p.kchunks - kt * C::KB_PER_STAGE;
+          if (nkc > C::KB_PER_STAGE) nkc = C::KB_PER_STAGE;
+          const uint32_t bytes = C::A_BYTES + C::B_BYTES + (uint32_t)nkc * 512u * (1u + (uint32_t)nsfb);
+          mbar_expect_tx(&full[s], bytes);
+          tma_load_2d(sA + s * C::A_BYTES, &tmA, kt * (C::BK / 2), m0, &full[s]);
+          tma_load_2d(sB + s * C::B_BYTES, &tmB, kt * (C::BK / 2), n0, &full[s]);
+          const int64_t kc0 = (int64_t)kt * C::KB_PER_STAGE;
+          bulk_g2s(sSFA + s * C::SFA_BYTES, p.a_sf + ((int64_t)a_tile * p.kchunks + kc0) * 512,
+                   (uint32_t)nkc * 512u, &full[s]);
+          for (int j = 0; j < nsfb; ++j)
+            bulk_g2s(sSFB + s * C::SFB_BYTES + j * 512 * C::KB_PER_STAGE,
+                     p.b_sf + ((int64_t)(n0 / 128 + j) * p.kchunks + kc0) * 512, (uint32_t)nkc * 512u, &full[s]);
+        }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t acc = tmem + C::TM_ACC;
-      for (int kt = 0; kt < num_kt; ++kt) {
-        const int s = kt % C::STAGES;
-        const uint32_t ph = (uint32_t)(kt / C::STAGES) & 1u;
-        if (!mbar_wait_bounded(&full[s], ph)) { *abort_flag = 1; break; }
-        if (*abort_flag) break;
+      int it = 0;
+      int ti = 0;  // tiles done by this CTA
+      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x, ++ti) {
+        // the epilogue must have drained the previous tile's accumulator
+        if (!mbar_wait_bounded(acc_empty, ((uint32_t)ti & 1u) ^ 1u)) { *abort_flag = 1; break; }
         tc_fence_after();
-        int nkc = p.kchunks - kt * C::KB_PER_STAGE;
-        if (nkc > C::KB_PER_STAGE) nkc = C::KB_PER_STAGE;
-        const int par = kt & 1;
-        const uint32_t sfa_col = tmem + C::TM_SFA + par * 4 * C::KB_PER_STAGE;
-        const uint32_t sfb_col = tmem + C::TM_SFB + par * 4 * C::KB_PER_STAGE * C::NB_SFB;
-        // scales: each 512-byte (128 rows x 4 blocks) tile -> 4 TMEM columns
-        for (int kb = 0; kb < nkc; ++kb) {
-          tc_cp_32x128b_warpx4(sfa_col + kb * 4, smem_desc(smem_u32(sSFA + s * C::SFA_BYTES + kb * 512), 0, 128, 0));
+        for (int kt = 0; kt < num_kt; ++kt, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t ph = (uint32_t)(it / C::STAGES) & 1u;
+          if (!mbar_wait_bounded(&full[s], ph)) { *abort_flag = 1; break; }
+          if (*abort_flag) break;
+          tc_fence_after();
+          int nkc = p.kchunks - kt * C::KB_PER_STAGE;
+          if (nkc > C::KB_PER_STAGE) nkc = C::KB_PER_STAGE;
+          const int par = it & 1;
+          const uint32_t sfa_col = tmem + C::TM_SFA + par * 4 * C::KB_PER_STAGE;
+          const uint32_t sfb_col = tmem + C::TM_SFB + par * 4 * C::KB_PER_STAGE * C::NB_SFB;
+          // scales: each 512-byte (128 rows x 4 blocks) tile -> 4 TMEM columns
+          for (int kb = 0; kb < nkc; ++kb) {
+            tc_cp_32x128b_warpx4(sfa_col + kb * 4,
+                                 smem_desc(smem_u32(sSFA + s * C::SFA_BYTES + kb * 512), 0, 128, 0));
 #pragma unroll
-          for (int j = 0; j < C::NB_SFB; ++j)
-            tc_cp_32x128b_warpx4(sfb_col + kb * 4 * C::NB_SFB + j * 4,
-                                 smem_desc(smem_u32(sSFB + s * C::SFB_BYTES + j * 512 * C::KB_PER_STAGE + kb * 512), 0,
-                                           128, 0));
+            for (int j = 0; j < C::NB_SFB; ++j)
+              tc_cp_32x128b_warpx4(
+                  sfb_col + kb * 4 * C::NB_SFB + j * 4,
+                  smem_desc(smem_u32(sSFB + s * C::SFB_BYTES + j * 512 * C::KB_PER_STAGE + kb * 512), 0, 128, 0));
+          }
+          const uint32_t a_base = smem_u32(sA + s * C::A_BYTES);
+          const uint32_t b_base = smem_u32(sB + s * C::B_BYTES);
+          for (int kb = 0; kb < nkc; ++kb) {
+            // K = 64 FP4 elements = 32 bytes further along the 128-byte swizzled row
+            const uint64_t ad = smem_desc(a_base + kb * 32, 16, 1024, 2);
+            const uint64_t bd = smem_desc(b_base + kb * 32, 16, 1024, 2);
+            mma_fp4_block16(acc, ad, bd, C::IDESC, sfa_col + kb * 4, sfb_col + kb * 4 * C::NB_SFB,
+                            (kt > 0 || kb > 0) ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
         }
-        const uint32_t a_base = smem_u32(sA + s * C::A_BYTES);
-        const uint32_t b_base = smem_u32(sB + s * C::B_BYTES);
-        for (int kb = 0; kb < nkc; ++kb) {
-          // K = 64 FP4 elements = 32 bytes further along the 128-byte swizzled row
-          const uint64_t ad = smem_desc(a_base + kb * 32, 16, 1024, 2);
-          const uint64_t bd = smem_desc(b_base + kb * 32, 16, 1024, 2);
-          mma_fp4_block16(acc, ad, bd, C::IDESC, sfa_col + kb * 4, sfb_col + kb * 4 * C::NB_SFB,
-                          (kt > 0 || kb > 0) ? 1u : 0u);
-        }
-        tc_commit(&empty[s]);
+        tc_commit(acc_full);
       }
-      tc_commit(acc_full);
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int sub = warp & 3;                 // TMEM subpartition this warp may read
-    const int row = m0 + sub * 32 + lane;
-    bool ok = mbar_wait_bounded(acc_full, 0);
-    if (!ok) *abort_flag = 1;
-    tc_fence_after();
-    if (ok && !*abort_flag) {
-      const float alpha = __fmul_rn(__ldg(p.a_ts), __ldg(p.b_ts));
-      __nv_bfloat16* crow = p.c + (int64_t)row * p.ldc;
-#pragma unroll 1
-      for (int c0 = 0; c0 < C::BN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem + C::TM_ACC + ((uint32_t)(sub * 32) << 16) + c0, r);
-        tmem_wait_ld();
-        if (row < p.M) {
-          const int col0 = n0 + c0;
-          uint32_t w[16];
+    const int sub = warp & 3;                      // TMEM subpartition this warp may read
+    const int cbase = ((warp - 2) >> 2) * (C::BN / 2);  // this warp's half of the columns
+    constexpr int HALF = C::BN / 2;
+    const float alpha = __fmul_rn(__ldg(p.a_ts), __ldg(p.b_ts));
+    int ti = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++ti) {
+      int m0, n0;
+      tile_coords(t, num_n, C::BM, C::BN, m0, n0);
+      const bool ok = mbar_wait_bounded(acc_full, (uint32_t)ti & 1u);
+      if (!ok) *abort_flag = 1;
+      if (!ok || *abort_flag) break;
+      tc_fence_after();
+      // drain this warp's part of the accumulator into registers as bf16 pairs ...
+      uint32_t packed[HALF / 2];
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            w[j] = pack_bf16x2(__uint_as_float(r[2 * j]) * alpha, __uint_as_float(r[2 * j + 1]) * alpha);
+      for (int c0 = 0; c0 < HALF; c0 += 64) {  // two loads in flight per wait
+        uint32_t r0[32], r1[32];
+        const uint32_t taddr = tmem + C::TM_ACC + ((uint32_t)(sub * 32) << 16) + cbase + c0;
+        tmem_ld_32x32b_x32(taddr, r0);
+        tmem_ld_32x32b_x32(taddr + 32, r1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          packed[c0 / 2 + j] = pack_bf16x2(__uint_as_float(r0[2 * j]) * alpha, __uint_as_float(r0[2 * j + 1]) * alpha);
+          packed[c0 / 2 + 16 + j] =
+              pack_bf16x2(__uint_as_float(r1[2 * j]) * alpha, __uint_as_float(r1[2 * j + 1]) * alpha);
+        }
+      }
+      // ... hand the accumulator back to the MMA warp ...
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      // ... and store while the next tile accumulates
+      const int row = m0 + sub * 32 + lane;
+      if (row < p.M) {
+        __nv_bfloat16* crow = p.c + (int64_t)row * p.ldc;
+#pragma unroll
+        for (int c0 = 0; c0 < HALF; c0 += 32) {
+          const int col0 = n0 + cbase + c0;
           if (col0 + 32 <= p.N && p.c_vec16) {
             uint4* dst = reinterpret_cast<uint4*>(crow + col0);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_uint4(packed[c0 / 2 + 4 * j], packed[c0 / 2 + 4 * j + 1], packed[c0 / 2 + 4 * j + 2],
+                                  packed[c0 / 2 + 4 * j + 3]);
           } else {
             for (int j = 0; j < 32; ++j) {
               if (col0 + j < p.N) {
-                const uint32_t h = (j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu);
+                const uint32_t w = packed[(c0 + j) >> 1];
+                const uint32_t h = (j & 1) ? (w >> 16) : (w & 0xFFFFu);
                 crow[col0 + j] = __ushort_as_bfloat16((unsigned short)h);
               }
             }
@@ -261,7 +314,14 @@ static nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* b, const GemmPa
       return NVFP4_ERR_CUDA;
     attr_set = true;
   }
-  dim3 grid((p.N + C::BN - 1) / C::BN, (p.M + C::BM - 1) / C::BM);
+  const int tiles = ((p.N + C::BN - 1) / C::BN) * ((p.M + C::BM - 1) / C::BM);
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sms = 148;
+  }
+  const int grid = tiles < sms ? tiles : sms;  // persistent: one CTA per SM
   gemm_w4a4_kernel<BN><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, p);
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
