@@ -49,8 +49,8 @@
  *     along the last (contiguous) dimension, so `cols` must be a multiple of
  *     16; base pointers must be 16-byte aligned and ld * element size a
  *     multiple of 16 bytes.
- *   - Inputs must be finite; non-finite inputs give NVFP4_OK and unspecified
- *     outputs.
+ *   - Inputs must be finite, and logits given to the KL loss above -1e30;
+ *     other inputs give NVFP4_OK and unspecified outputs.
  *   - Packed codes: byte j of a row holds element 2j in its low nibble and
  *     element 2j+1 in its high nibble.
  */

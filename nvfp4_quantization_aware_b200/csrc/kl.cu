@@ -43,23 +43,25 @@ NVFP4_DEV float ex2(float x) {
   return y;
 }
 
-// 2^x for x <= 0 on the FMA pipe: x = n + f with n = rint(x), f in
-// [-1/2, 1/2]; 2^f by a degree-5 polynomial (least-squares fit of 2^f on 2000
-// Chebyshev nodes of [-1/2, 1/2], coefficients rounded to binary32; maximum
-// relative error 1.8e-7 over the interval); 2^n applied by adding n to the
-// exponent field.  x is clamped at -126 so the result stays normal (2^-126 is
-// below anything the gradient can resolve).
+// 2^x for x <= 0 on the FMA and integer pipes only (no conversion
+// instruction, which would share the MUFU/XU pipe): x = n + f with
+// n = rint(x) taken from the low mantissa bits of x + 1.5 * 2^23, f in
+// [-1/2, 1/2]; 2^f by a degree-5 polynomial (least-squares fit of 2^f on
+// 2000 Chebyshev nodes of [-1/2, 1/2], coefficients rounded to binary32;
+// maximum relative error 1.8e-7 over the interval); 2^n applied by adding n
+// to the exponent field (the magic constant's own bits shift out of the
+// 32-bit word).  x is clamped at -126 so that the result stays normal.
 NVFP4_DEV float exp2_poly(float x) {
   x = fmaxf(x, -126.0f);
-  const float n = rintf(x);
-  const float f = x - n;
+  const float t = x + 12582912.0f;      // 1.5 * 2^23: rounds x to an integer in the low bits
+  const float f = x - (t - 12582912.0f);
   float p = 0.0013400432653725147f;
   p = fmaf(p, f, 0.009676037356257439f);
   p = fmaf(p, f, 0.05550327152013779f);
   p = fmaf(p, f, 0.2402210682630539f);
   p = fmaf(p, f, 0.6931471824645996f);
   p = fmaf(p, f, 1.0000001192092896f);
-  return __int_as_float(__float_as_int(p) + ((int)n << 23));
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 // Running softmax statistics of a (teacher, student) pair of rows, in the
@@ -70,12 +72,12 @@ struct KlStats {
   float mt, ms, St, Ss, Y;
 };
 
-constexpr float kNoMax = -1.0e30f;  // start value of the running maxima
-
-NVFP4_DEV void stats_init(KlStats& a) {
-  a.mt = kNoMax;
-  a.ms = kNoMax;
-  a.St = a.Ss = a.Y = 0.f;
+// Empty statistics whose maxima sit at the pad value (scaled by a): merging
+// them into real statistics scales them by 2^(pad a - max) = 0.
+NVFP4_DEV void stats_init(KlStats& s, float pad_w) {
+  s.mt = pad_w;
+  s.ms = pad_w;
+  s.St = s.Ss = s.Y = 0.f;
 }
 
 // Re-express `a` relative to new maxima (Mt, Ms) >= (a.mt, a.ms): the terms
@@ -124,6 +126,15 @@ struct KlElem<__nv_bfloat16> {
                       pack_bf16x2(v[6], v[7]));
   }
   NVFP4_DEV static float load1(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+  // max of the 8 logits of a vector (exact: bf16 max on packed pairs)
+  NVFP4_DEV static float vmax(const uint4& r) {
+    __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&r.x);
+    __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&r.y);
+    __nv_bfloat162 c = *reinterpret_cast<const __nv_bfloat162*>(&r.z);
+    __nv_bfloat162 d = *reinterpret_cast<const __nv_bfloat162*>(&r.w);
+    __nv_bfloat162 m = __hmax2(__hmax2(a, b), __hmax2(c, d));
+    return fmaxf(__low2float(m), __high2float(m));
+  }
   NVFP4_DEV static void store1(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 };
 template <>
@@ -136,6 +147,9 @@ struct KlElem<float> {
     return make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]), __float_as_uint(v[3]));
   }
   NVFP4_DEV static float load1(const float* p) { return *p; }
+  NVFP4_DEV static float vmax(const uint4& r) {
+    return fmaxf(fmaxf(__uint_as_float(r.x), __uint_as_float(r.y)), fmaxf(__uint_as_float(r.z), __uint_as_float(r.w)));
+  }
   NVFP4_DEV static void store1(float* p, float v) { *p = v; }
 };
 
@@ -152,9 +166,12 @@ struct KlArgs {
 };
 
 // Stand-in for positions of the shared-memory slice that hold no logit (the
-// alignment pad before and after the slice): exp underflows to 0 and it never
-// wins the max while the slice holds at least one real logit.
-constexpr float kPadLogit = -1.0e30f;
+// alignment pad before and after the slice).  A power of two, so that its
+// product with a = log2(e) / T is exact and d = fma(pad, a, -pad * a) is 0;
+// it is below every logit the kernel accepts (logits must exceed -1e30), so
+// it never wins a max that a real logit takes part in, and 2^(pad a - max)
+// underflows to 0.
+constexpr float kPadLogit = -0x1p100f;
 
 template <typename T>
 __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
@@ -205,13 +222,24 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
     bulk_g2s(st + off + head, gt + head, (uint32_t)(nint * ESZ), &bar);
     bulk_g2s(ss + off + head, gs + head, (uint32_t)(nint * ESZ), &bar);
   }
-  // head, tail and pad slots with plain accesses (disjoint from the bulk copy)
-  for (int j = threadIdx.x; j < cap; j += kKlThreads) {
-    const int i = j - off;  // logit index inside the slice
-    if ((i >= 0 && i < head) || (i >= tail0 && i < n)) {
+  // head and tail logits with plain loads, pad slots with the pad value; all
+  // disjoint from the bulk-copied interior [off + head, off + tail0)
+  for (int j = threadIdx.x; j < off + head; j += kKlThreads) {  // pad, then head
+    const int i = j - off;
+    if (i < 0) {
+      E::store1(st + j, kPadLogit);
+      E::store1(ss + j, kPadLogit);
+    } else {
       st[j] = gt[i];
       ss[j] = gs[i];
-    } else if (i < 0 || i >= n) {
+    }
+  }
+  for (int j = off + tail0 + threadIdx.x; j < cap; j += kKlThreads) {  // tail, then pad
+    const int i = j - off;
+    if (i < n) {
+      st[j] = gt[i];
+      ss[j] = gs[i];
+    } else {
       E::store1(st + j, kPadLogit);
       E::store1(ss + j, kPadLogit);
     }
@@ -224,27 +252,28 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
   const uint4* vs = reinterpret_cast<const uint4*>(ss);
   const float a = args.a;  // log2(e) / T > 0
 
-  // ---- online statistics over this thread's vectors
+  // ---- online statistics over this thread's vectors; the running maxima are
+  // kept on the raw logits (a > 0, so max w = a * max z) and d = z a - max w
+  // is one FMA
   KlStats my;
-  stats_init(my);
+  stats_init(my, kPadLogit * a);
+  float zmt = kPadLogit, zms = kPadLogit;  // running max of the raw logits
   if (ok) {
     for (int k = threadIdx.x; k < nvec; k += kKlThreads) {
-      float wt[V8], ws[V8];
-      E::unpack(vt[k], wt);
-      E::unpack(vs[k], ws);
-      float lt = kNoMax, ls = kNoMax;
-#pragma unroll
-      for (int j = 0; j < V8; ++j) {
-        wt[j] *= a;
-        ws[j] *= a;
-        lt = fmaxf(lt, wt[j]);
-        ls = fmaxf(ls, ws[j]);
+      const uint4 rt = vt[k], rs = vs[k];
+      const float lt = E::vmax(rt), ls = E::vmax(rs);
+      if (lt > zmt || ls > zms) {
+        zmt = fmaxf(zmt, lt);
+        zms = fmaxf(zms, ls);
+        stats_rebase(my, zmt * a, zms * a);
       }
-      const float Mt = fmaxf(my.mt, lt), Ms = fmaxf(my.ms, ls);
-      if (Mt != my.mt || Ms != my.ms) stats_rebase(my, Mt, Ms);
+      const float nMt = -my.mt, nMs = -my.ms;
+      float zt[V8], zs[V8];
+      E::unpack(rt, zt);
+      E::unpack(rs, zs);
 #pragma unroll
       for (int j = 0; j < V8; ++j) {
-        const float dt = wt[j] - Mt, ds = ws[j] - Ms;
+        const float dt = fmaf(zt[j], a, nMt), ds = fmaf(zs[j], a, nMs);
         const float et = ex2(dt), es = ex2(ds);
         my.St += et;
         my.Ss += es;
@@ -273,12 +302,18 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
     args.row_kl[row] = ok ? kl : __int_as_float(0x7FC00000);
   }
 
-  // ---- dLogits = gscale * (p_s - p_t), p = 2^(w - max w - log2 S)
+  // ---- dLogits = gscale * (p_s - p_t), p = 2^(w - max w - log2 S); for
+  // gscale > 0 the factor goes into the exponent: g p = 2^(w - L + log2 g)
   if (args.dlogits != nullptr && ok) {
     const float g = args.gscale;
-    const float Lt = Wt + __log2f(St), Ls = Ws + __log2f(Ss);
+    const bool fold = g > 0.0f;
+    const float lg = fold ? __log2f(g) : 0.0f;
+    const float Lt = Wt + __log2f(St) - lg, Ls = Ws + __log2f(Ss) - lg;
+    const float gm = fold ? 1.0f : g;
     T* gout = reinterpret_cast<T*>(args.dlogits) + row * args.ld_grad + v0 - off;  // slot j -> gout[j]
     const bool vec_ok = (((uintptr_t)gout) & 15u) == 0;
+    const int kfirst = (off + V8 - 1) / V8;          // first vector with no leading pad
+    const int klast = nslots / V8;                   // vectors [kfirst, klast) are all real
     for (int k = threadIdx.x; k < nvec; k += kKlThreads) {
       float zt[V8], zs[V8], o[V8];
       E::unpack(vt[k], zt);
@@ -287,10 +322,10 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
       for (int j = 0; j < V8; ++j) {
         const float pt = exp2_poly(fmaf(zt[j], a, -Lt));
         const float ps = ex2(fmaf(zs[j], a, -Ls));
-        o[j] = g * (ps - pt);
+        o[j] = fold ? ps - pt : gm * (ps - pt);
       }
       const int j0 = k * V8;
-      if (vec_ok && j0 >= off && j0 + V8 <= nslots) {
+      if (vec_ok && k >= kfirst && k < klast) {
         st_stream_v4(gout + j0, E::pack(o));
       } else {
 #pragma unroll

@@ -284,22 +284,27 @@ NVFP4_DEV void chunk_pos(const GTensor& g, int64_t chunk, int lane, int64_t& row
 
 // ------------------------------------------------------------------ amax
 
-// Per-tensor max |x| of a group.  Every warp visits chunks in increasing
-// order, so the tensor it works on only changes forward: it keeps a running
-// max for the current tensor across iterations and folds it into the tensor's
-// word with one atomicMax on the float bits when the tensor changes and at
-// the end (|x| >= 0 compares like its bit pattern; max is exact, so the order
-// of the atomics does not matter).  Same-address atomics stay at about one per
-// warp and tensor.
+// Per-tensor max |x| of a group.  Each CTA takes one contiguous range of
+// chunks, so it touches one or two tensors; its warps walk the range in
+// increasing order keeping a running max per tensor, fold it into a
+// shared-memory table when the tensor changes, and the CTA finally folds the
+// table into the global words with one atomicMax on the float bits per tensor
+// it touched (|x| >= 0 compares like its bit pattern; max is exact, so the
+// order of the atomics does not matter).
 template <typename T>
 __global__ void __launch_bounds__(kThreads) group_amax_kernel(const __grid_constant__ GroupArgs a) {
+  __shared__ unsigned s_max[kMaxGroup];
+  for (int i = threadIdx.x; i < a.n; i += kThreads) s_max[i] = 0u;
+  __syncthreads();
   const int lane = threadIdx.x & 31;
-  const int64_t warp = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
-  const int64_t nwarps = (int64_t)gridDim.x * kWarps;
+  const int wid = threadIdx.x >> 5;
+  const int64_t per_cta = (a.total_chunks + gridDim.x - 1) / gridDim.x;
+  const int64_t c_begin = (int64_t)blockIdx.x * per_cta;
+  const int64_t c_end = c_begin + per_cta < a.total_chunks ? c_begin + per_cta : a.total_chunks;
   int cur = 0;
   int mt = -1;      // tensor of the running max
   float m = 0.0f;   // running max of this lane
-  for (int64_t c0 = warp * kQUnroll; c0 < a.total_chunks; c0 += nwarps * kQUnroll) {
+  for (int64_t c0 = c_begin + wid * kQUnroll; c0 < c_end; c0 += kWarps * kQUnroll) {
     Block16<T> in[kQUnroll];
     int tid[kQUnroll];
 #pragma unroll
@@ -307,7 +312,7 @@ __global__ void __launch_bounds__(kThreads) group_amax_kernel(const __grid_const
       const int64_t c = c0 + u;
       in[u].zero();
       tid[u] = -1;
-      if (c < a.total_chunks) {
+      if (c < c_end) {
         cur = find_tensor(a, c, cur);
         const GTensor& g = a.t[cur];
         int64_t row, col;
@@ -321,7 +326,7 @@ __global__ void __launch_bounds__(kThreads) group_amax_kernel(const __grid_const
       if (tid[u] < 0) continue;  // warp-uniform
       if (tid[u] != mt) {         // warp-uniform: flush the previous tensor's max
         const float w = warp_max(m);
-        if (lane == 0 && mt >= 0 && w > 0.0f) atomicMax(a.amax + mt, __float_as_uint(w));
+        if (lane == 0 && mt >= 0 && w > 0.0f) atomicMax(s_max + mt, __float_as_uint(w));
         m = 0.0f;
         mt = tid[u];
       }
@@ -332,7 +337,10 @@ __global__ void __launch_bounds__(kThreads) group_amax_kernel(const __grid_const
     }
   }
   const float w = warp_max(m);
-  if (lane == 0 && mt >= 0 && w > 0.0f) atomicMax(a.amax + mt, __float_as_uint(w));
+  if (lane == 0 && mt >= 0 && w > 0.0f) atomicMax(s_max + mt, __float_as_uint(w));
+  __syncthreads();
+  for (int i = threadIdx.x; i < a.n; i += kThreads)
+    if (s_max[i] != 0u) atomicMax(a.amax + i, s_max[i]);
 }
 
 // ------------------------------------------------------------------ encode
@@ -611,7 +619,7 @@ static nvfp4_status launch_status() {
 // encode pass re-reads them from L2 rather than HBM.  A tensor larger than
 // this budget forms a group of its own.
 constexpr int64_t kL2GroupBytes = 48ll << 20;
-constexpr size_t kDynamicWorkspace = 1024;  // >= kMaxGroup amax words
+constexpr size_t kDynamicWorkspace = 1024;  // 256 amax words, >= kMaxGroup
 
 // Validate one tensor of a (possibly grouped) quantize / fake-quant call.
 template <Out OUT>
@@ -636,40 +644,55 @@ static nvfp4_status check_tensor(const nvfp4_tensor_ref& r, nvfp4_dtype dtype, n
   return NVFP4_OK;
 }
 
-// Persistent grid for a group: at most the resident capacity of the GPU.
-template <typename K>
-static int resident_grid(K kernel, int64_t total_chunks) {
-  static int per_sm = 0;
-  if (per_sm == 0 && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess ||
-                      per_sm <= 0))
-    per_sm = 4;
+// Resident CTAs per SM of a kernel (256 threads, no dynamic shared memory),
+// looked up once per kernel and cached by the kernel's address.
+static int resident_per_sm(const void* fn) {
+  static const void* keys[16] = {};
+  static int vals[16] = {};
+  for (int i = 0; i < 16; ++i) {
+    if (keys[i] == fn) return vals[i];
+    if (keys[i] == nullptr) {
+      int v = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, fn, kThreads, 0) != cudaSuccess || v <= 0) v = 1;
+      keys[i] = fn;
+      vals[i] = v;
+      return v;
+    }
+  }
+  return 1;
+}
+
+// Persistent grid for a group: at most the resident capacity of the GPU, so
+// every CTA of the grid-stride loop runs in the same wave.
+static int resident_grid(const void* fn, int64_t total_chunks) {
   const int64_t per_cta = (int64_t)kWarps * kQUnroll;
   int64_t need = (total_chunks + per_cta - 1) / per_cta;
-  const int64_t cap = (int64_t)sm_count() * per_sm;
+  const int64_t cap = (int64_t)sm_count() * resident_per_sm(fn);
   if (need > cap) need = cap;
   return need < 1 ? 1 : (int)need;
 }
 
+// Launch the kernels of one group.  In DYNAMIC mode `amax` points at this
+// group's n zeroed words of the workspace.
 template <Out OUT>
-static nvfp4_status launch_group(GroupArgs& a, nvfp4_dtype dtype, void* ws, cudaStream_t s) {
+static nvfp4_status launch_group(GroupArgs& a, nvfp4_dtype dtype, unsigned* amax, cudaStream_t s) {
   if (a.n == 0 || a.total_chunks == 0) return NVFP4_OK;
   if (a.mode == NVFP4_DYNAMIC) {
-    a.amax = reinterpret_cast<unsigned*>(ws);
-    if (cudaMemsetAsync(ws, 0, sizeof(unsigned) * (size_t)a.n, s) != cudaSuccess) return NVFP4_ERR_CUDA;
+    a.amax = amax;
     if (dtype == NVFP4_BF16)
       group_amax_kernel<__nv_bfloat16>
-          <<<resident_grid(group_amax_kernel<__nv_bfloat16>, a.total_chunks), kThreads, 0, s>>>(a);
+          <<<resident_grid((const void*)group_amax_kernel<__nv_bfloat16>, a.total_chunks), kThreads, 0, s>>>(a);
     else
-      group_amax_kernel<float><<<resident_grid(group_amax_kernel<float>, a.total_chunks), kThreads, 0, s>>>(a);
+      group_amax_kernel<float><<<resident_grid((const void*)group_amax_kernel<float>, a.total_chunks), kThreads, 0, s>>>(a);
     count_launches(1);
     if (launch_status() != NVFP4_OK) return NVFP4_ERR_CUDA;
   }
   if (dtype == NVFP4_BF16)
     group_encode_kernel<__nv_bfloat16, OUT>
-        <<<resident_grid(group_encode_kernel<__nv_bfloat16, OUT>, a.total_chunks), kThreads, 0, s>>>(a);
+        <<<resident_grid((const void*)group_encode_kernel<__nv_bfloat16, OUT>, a.total_chunks), kThreads, 0, s>>>(a);
   else
     group_encode_kernel<float, OUT>
-        <<<resident_grid(group_encode_kernel<float, OUT>, a.total_chunks), kThreads, 0, s>>>(a);
+        <<<resident_grid((const void*)group_encode_kernel<float, OUT>, a.total_chunks), kThreads, 0, s>>>(a);
   count_launches(1);
   return launch_status();
 }
@@ -701,6 +724,21 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
   a.x_wide = 1;
   a.out_wide = 1;
   int64_t group_bytes = 0;
+  // DYNAMIC: every group takes its own amax words from the workspace; the
+  // words are cleared once per call, and again whenever they run out.
+  unsigned* words = reinterpret_cast<unsigned*>(ws);
+  const int nwords = (int)(kDynamicWorkspace / sizeof(unsigned));
+  int word_base = nwords;  // forces a clear before the first group
+  auto flush = [&]() -> nvfp4_status {
+    if (a.n == 0) return NVFP4_OK;
+    if (mode == NVFP4_DYNAMIC && word_base + a.n > nwords) {
+      if (cudaMemsetAsync(ws, 0, kDynamicWorkspace, s) != cudaSuccess) return NVFP4_ERR_CUDA;
+      word_base = 0;
+    }
+    nvfp4_status st = launch_group<OUT>(a, dtype, words + word_base, s);
+    word_base += a.n;
+    return st;
+  };
   for (int i = 0; i < n; ++i) {
     const nvfp4_tensor_ref& r = refs[i];
     if (r.rows == 0 || r.cols == 0) {
@@ -713,7 +751,7 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
     const bool full = a.n == kMaxGroup;
     const bool over_l2 = mode == NVFP4_DYNAMIC && a.n > 0 && group_bytes + bytes > kL2GroupBytes;
     if (full || over_l2) {
-      nvfp4_status st = launch_group<OUT>(a, dtype, ws, s);
+      nvfp4_status st = flush();
       if (st != NVFP4_OK) return st;
       a.n = 0;
       a.total_chunks = 0;
@@ -744,7 +782,7 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
       if (((uintptr_t)r.out & 31u) || ((r.ld_out * esz) & 31)) a.out_wide = 0;
     }
   }
-  nvfp4_status st = launch_group<OUT>(a, dtype, ws, s);
+  nvfp4_status st = flush();
   if (st != NVFP4_OK) return st;
   // zero the padding of MMA-layout scale arrays
   if (OUT == Out::Codes && layout == NVFP4_SCALES_MMA && mode != NVFP4_FROZEN_ALL) {
