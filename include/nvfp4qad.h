@@ -257,6 +257,255 @@ nvfp4_status nvfp4_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_scales_mma
                              size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Grouped W4A4 GEMM for the experts of a MoE layer (Nemotron-3-Nano article,
+ * "Was ist Nemotron-Nano-3-30B-A3B-NVFP4?": 128 routed experts + 1 shared;
+ * Qwen3.6 tutorial, "2. PTQ": experts are NVFP4 W4A4).  For every group g:
+ *   C[rows of g] = (s_gA[g] * s_gB[g]) * A^_g * B^_g^T
+ *
+ *   a_codes         a_rows_total x K/2 bytes: the groups' activation rows, each
+ *                   group in a segment [a_row_offsets[g], a_row_offsets[g] +
+ *                   a_rows[g]) whose start is a multiple of 128 (rows of a
+ *                   segment past a_rows[g] are padding and are not stored)
+ *   a_scales_mma    MMA-layout block scales of the whole a_codes buffer
+ *                   (nvfp4_mma_scales_bytes(a_rows_total, K))
+ *   a_tensor_scales groups floats (device), one per group
+ *   a_row_offsets   groups + 1 int32 (device); a_row_offsets[groups] is the end
+ *                   of the last segment (<= a_rows_total)
+ *   a_rows          groups int32 (device): valid rows of each segment
+ *   b_codes         groups * N x K/2 bytes: B of group g in rows [g N, (g+1) N)
+ *   b_scales_mma    MMA-layout block scales of the stacked B (groups * N rows)
+ *   b_tensor_scales groups floats (device)
+ *   c               a_rows_total x N bf16, row stride ldc; only valid rows written
+ * Requires 1 <= groups <= 256, a_rows_total % 128 == 0, N % 128 == 0,
+ * K % 64 == 0.  The segment table is read on the device, so routing results
+ * never travel to the host.
+ * ------------------------------------------------------------------------ */
+size_t nvfp4_gemm_grouped_workspace_size(int groups, int64_t a_rows_total, int64_t N, int64_t K);
+
+nvfp4_status nvfp4_gemm_w4a4_grouped(int groups, const uint8_t* a_codes, const uint8_t* a_scales_mma,
+                                     const float* a_tensor_scales, int64_t a_rows_total,
+                                     const int32_t* a_row_offsets, const int32_t* a_rows,
+                                     const uint8_t* b_codes, const uint8_t* b_scales_mma,
+                                     const float* b_tensor_scales, int64_t N, int64_t K, void* c,
+                                     int64_t ldc, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Grouped BF16 GEMM on the tcgen05 tensor cores (FP32 accumulation in
+ * tensor memory, bf16 output RNE) for the straight-through backward of the
+ * MoE layer, whose gradients are plain BF16 products with the dequantized
+ * operands (Nemotron 3.5 Lightning article, "QAD的工作原理").  Always
+ * C = A * B^T with A and B row-major and K their contiguous dimension.
+ *
+ *   mode 0 (M-segments)  a: a_rows x a_cols (a_rows % 128 == 0), the groups'
+ *                        rows in segments [seg_off[g], seg_off[g] + seg_len[g])
+ *                        with seg_off[g] % 128 == 0; b: b_rows x K, group g
+ *                        uses rows [g N, (g+1) N); c: a_rows x N (ldc), only
+ *                        the segments' valid rows written.  K % 64 == 0,
+ *                        K <= a_cols, b_rows >= groups * N; M is ignored.
+ *   mode 1 (K-segments)  a: a_rows x a_cols, b: b_rows x a_cols; group g
+ *                        reduces over columns [seg_off[g], seg_off[g] +
+ *                        seg_len[g]) (seg_off[g] % 64 == 0; columns up to the
+ *                        next multiple of 64 are read and must hold zeros
+ *                        or belong to no other term); c: groups * M x N, group
+ *                        g in rows [g M, (g+1) M); M <= a_rows, N <= b_rows,
+ *                        K is ignored.  A group with seg_len 0 writes zeros.
+ *   seg_off, seg_len     device int32 arrays (groups + 1 and groups entries)
+ * 1 <= groups <= 256; a, b 16-byte aligned, lda * 2 and ldb * 2 multiples of
+ * 16; c 4-byte aligned.
+ * ------------------------------------------------------------------------ */
+nvfp4_status nvfp4_gemm_bf16_grouped(int mode, int groups, const void* a, int64_t a_rows, int64_t a_cols,
+                                     int64_t lda, const void* b, int64_t b_rows, int64_t ldb,
+                                     const int32_t* seg_off, const int32_t* seg_len, int64_t M, int64_t N,
+                                     int64_t K, void* c, int64_t ldc, void* stream);
+
+/* ------------------------------------------------------------------------
+ * MoE layer of the QAD student: 128 routed experts plus one shared expert,
+ * top-6 routing (Nemotron-3-Nano-30B NVFP4 article, "Was ist
+ * Nemotron-Nano-3-30B-A3B-NVFP4?"), SwiGLU expert FFNs whose weights and
+ * activations are NVFP4 (W4A4) with frozen scales (Qwen3.6-35B-A3B W4A4
+ * tutorial, "2. PTQ"; Nemotron 3.5 Lightning article, "量化尺度处理策略").
+ * For token t with routed experts e_j and combine weights w_j:
+ *   y_t = sum_j w_j E_{e_j}(x_t) + E_shared(x_t),
+ *   E(x) = Q(a) W^_down^T,  a = silu(Q(x) W^_gate^T) * (Q(x) W^_up^T),
+ * Q = NVFP4 fake quantization (weights FROZEN_ALL, x and a FROZEN_GLOBAL
+ * with one tensor scale per expert), silu(g) = g / (1 + exp(-g)); the gate
+ * and up products are rounded to bf16, a is rounded to bf16 before Q.
+ * Backward: straight-through estimator (dQ(v)/dv = identity), BF16 grads.
+ *
+ * Groups: g < experts is routed expert g; g = experts the shared expert.
+ * Routed (token, slot) pairs are permuted into rows: group g owns rows
+ * [seg_off[g], seg_off[g] + seg_len[g]), seg_off[g] % 128 == 0, rows in
+ * increasing (token, slot) order; rows past seg_len[g] up to the next
+ * segment are padding (row_token -1) and hold zeros in every row buffer.
+ * ------------------------------------------------------------------------ */
+
+/* Rows of the permutation buffers: tokens*topk + 127*experts +
+ * ceil(tokens/128)*128, rounded up to a multiple of 128. */
+int64_t nvfp4_moe_rows_capacity(int tokens, int topk, int experts);
+
+/* Routing.  expert_ids, combine_weights: tokens x topk (device).  Outputs
+ * (device): seg_len [experts+1], seg_off [experts+2] (seg_off[experts+1] =
+ * end of the last segment), row_token / row_weight [rows_cap] (shared rows
+ * have weight 1), slot_row [tokens x topk] = the row of each assignment.
+ * An id outside [0, experts) is routed nowhere: its slot_row is -1 and the
+ * device error word becomes 3.  rows_cap >= nvfp4_moe_rows_capacity(...).
+ * Rows in [seg_off[experts+1], rows_cap) are not written by this call. */
+nvfp4_status nvfp4_moe_route(const int32_t* expert_ids, const float* combine_weights, int tokens, int topk,
+                             int experts, int32_t* seg_len, int32_t* seg_off, int32_t* row_token,
+                             float* row_weight, int32_t* slot_row, int64_t rows_cap, void* stream);
+
+/* Gather + FROZEN_GLOBAL quantize: row r of the permutation holds
+ * x[row_token[r]] (zeros when row_token[r] < 0 or r >= seg_off[groups]),
+ * quantized with tensor scale tensor_scales[group of r].
+ *   x        bf16 tokens x cols, row stride ld_x
+ *   codes    rows_cap x cols/2 bytes; scales_mma: MMA layout of rows_cap x cols
+ *   xhat     bf16 rows_cap x cols, the dequantized rows, or NULL
+ * rows_cap % 128 == 0, cols % 64 == 0, 1 <= groups <= 256. */
+nvfp4_status nvfp4_moe_gather_quantize(const void* x, int64_t ld_x, const int32_t* row_token,
+                                       const int32_t* seg_off, int groups, const float* tensor_scales,
+                                       int64_t rows_cap, int64_t cols, uint8_t* codes, uint8_t* scales_mma,
+                                       void* xhat, void* stream);
+
+/* SwiGLU + FROZEN_GLOBAL quantize: a = bf16(silu(h_gate) * h_up) in binary32
+ * (h_gate, h_up bf16 rows_cap x cols, row stride ld_h; silu through expf),
+ * then quantized per row as above.  ahat: dequantized a or NULL; act: a
+ * itself (bf16 rows_cap x cols) or NULL.  Padding rows give zeros. */
+nvfp4_status nvfp4_moe_swiglu_quantize(const void* h_gate, const void* h_up, int64_t ld_h,
+                                       const int32_t* row_token, const int32_t* seg_off, int groups,
+                                       const float* tensor_scales, int64_t rows_cap, int64_t cols,
+                                       uint8_t* codes, uint8_t* scales_mma, void* ahat, void* act, void* stream);
+
+/* out[t] = bf16( sum_j w[t,j] * y[slot_row[t,j]] + y[seg_off[experts] + t] ),
+ * binary32 sums in the order j = 0..topk-1, then the shared expert; y bf16
+ * rows x cols (cols % 8 == 0), out bf16 tokens x cols. */
+nvfp4_status nvfp4_moe_combine(const void* y, int64_t cols, const int32_t* slot_row, const float* combine_weights,
+                               int tokens, int topk, const int32_t* seg_off, int experts, void* out, void* stream);
+
+/* dyp[r] = bf16(row_weight[r] * dy[row_token[r]]), zeros on padding rows and
+ * rows >= seg_off[groups]; dy tokens x cols, dyp rows_cap x cols (bf16). */
+nvfp4_status nvfp4_moe_scale_rows(const void* dy, int64_t cols, const int32_t* row_token, const float* row_weight,
+                                  const int32_t* seg_off, int groups, int64_t rows_cap, void* dyp, void* stream);
+
+/* SwiGLU backward, binary32: s = 1 / (1 + expf(-g)),
+ *   dG = da * u * s * (1 + g (1 - s)),  dU = da * g * s,
+ * written as dgu[r] = [dG | dU] (bf16 rows_cap x 2 cols); da, h_gate, h_up
+ * bf16 rows_cap x cols contiguous; zeros on padding rows. */
+nvfp4_status nvfp4_moe_swiglu_backward(const void* da, const void* h_gate, const void* h_up, int64_t cols,
+                                       const int32_t* row_token, const int32_t* seg_off, int groups,
+                                       int64_t rows_cap, void* dgu, void* stream);
+
+/* dx[t] = bf16( sum_j dxp[slot_row[t,j]] + dxp[seg_off[experts] + t] ). */
+nvfp4_status nvfp4_moe_gather_sum(const void* dxp, int64_t cols, const int32_t* slot_row, int tokens, int topk,
+                                  const int32_t* seg_off, int experts, void* dx, void* stream);
+
+/* d_combine[t,j] = sum_c dy[t,c] * y[slot_row[t,j], c]  (binary32; 0 for an
+ * assignment routed nowhere): the gradient of the layer w.r.t. its combine
+ * weights. */
+nvfp4_status nvfp4_moe_router_grad(const void* dy, const void* y, int64_t cols, const int32_t* slot_row, int tokens,
+                                   int topk, float* d_combine, void* stream);
+
+/* out[c][r] = in[r][c] for bf16 rows x cols (strides in elements). */
+nvfp4_status nvfp4_transpose_bf16(const void* in, int64_t ld_in, int64_t rows, int64_t cols, void* out,
+                                  int64_t ld_out, void* stream);
+
+/* Dequantized transpose of `groups` stacked NVFP4 tensors of rows_per_group x
+ * cols (codes contiguous, ROWMAJOR block scales, tensor_scales[g]):
+ *   out[g cols + c][col_off + r] = bf16(value(q[g][r][c]) * (s_b * s_g)).
+ * cols % 32 == 0; out bf16 with row stride ld_out >= col_off + rows_per_group. */
+nvfp4_status nvfp4_dequantize_transpose(const uint8_t* codes, const uint8_t* block_scales,
+                                        const float* tensor_scales, int groups, int64_t rows_per_group,
+                                        int64_t cols, void* out, int64_t ld_out, int64_t col_off, void* stream);
+
+/* ROWMAJOR block scales of rows x cols -> the MMA layout (padding 0). */
+nvfp4_status nvfp4_scales_to_mma(const uint8_t* block_scales, int64_t rows, int64_t cols, uint8_t* out,
+                                 void* stream);
+
+/* Shape of one MoE layer step. */
+typedef struct qad_moe_shape {
+  int tokens;    /* T >= 1 */
+  int hidden;    /* H, % 256 == 0 */
+  int ffn;       /* F, % 256 == 0 */
+  int experts;   /* routed experts E (group E is the shared expert), E + 1 <= 256 */
+  int topk;      /* routed experts per token, <= E */
+  int save_act;  /* nonzero: the forward also stores a (pre-quantization) in QAD_MOE_ACT */
+} qad_moe_shape;
+
+/* Parameters of the layer (device pointers; group g's block in rows of g). */
+typedef struct qad_moe_weights {
+  const void* w_gate;          /* bf16 master weights, (E+1) F x H */
+  const void* w_up;            /* bf16 (E+1) F x H */
+  const void* w_down;          /* bf16 (E+1) H x F */
+  const float* gate_ts;        /* frozen tensor scales, E+1 each */
+  const float* up_ts;
+  const float* down_ts;
+  const uint8_t* gate_sb;      /* frozen block scales, ROWMAJOR, of the stacked weights */
+  const uint8_t* up_sb;
+  const uint8_t* down_sb;
+  const uint8_t* gate_sb_mma;  /* the same in the MMA layout (nvfp4_scales_to_mma of the stack) */
+  const uint8_t* up_sb_mma;
+  const uint8_t* down_sb_mma;
+  const float* x_ts;           /* frozen tensor scale of each group's input x, E+1 */
+  const float* a_ts;           /* frozen tensor scale of each group's down-projection input a, E+1 */
+} qad_moe_weights;
+
+/* Buffers inside the step's workspace (offsets from qad_moe_workspace_buffer;
+ * R = qad_moe_rows_capacity).  The forward fills the first group, the
+ * backward reads them and fills the rest; a training step is forward then
+ * backward with the same workspace and no other call in between. */
+enum qad_moe_buffer {
+  QAD_MOE_SEG_LEN = 0,  /* int32 [E+1] */
+  QAD_MOE_SEG_OFF,      /* int32 [E+2] */
+  QAD_MOE_ROW_TOKEN,    /* int32 [R] */
+  QAD_MOE_ROW_WEIGHT,   /* f32 [R] */
+  QAD_MOE_SLOT_ROW,     /* int32 [T x topk] */
+  QAD_MOE_X_CODES,      /* u8 [R x H/2] */
+  QAD_MOE_X_SCALES,     /* u8 MMA layout of R x H */
+  QAD_MOE_X_HAT,        /* bf16 [R x H] */
+  QAD_MOE_WG_CODES,     /* u8 [(E+1) F x H/2] */
+  QAD_MOE_WU_CODES,     /* u8 [(E+1) F x H/2] */
+  QAD_MOE_WD_CODES,     /* u8 [(E+1) H x F/2] */
+  QAD_MOE_H_GATE,       /* bf16 [R x F] */
+  QAD_MOE_H_UP,         /* bf16 [R x F] */
+  QAD_MOE_A_CODES,      /* u8 [R x F/2] */
+  QAD_MOE_A_SCALES,     /* u8 MMA layout of R x F */
+  QAD_MOE_A_HAT,        /* bf16 [R x F] */
+  QAD_MOE_ACT,          /* bf16 [R x F] (0 bytes unless save_act) */
+  QAD_MOE_Y_ROWS,       /* bf16 [R x H] */
+  QAD_MOE_DY_ROWS,      /* bf16 [R x H] */
+  QAD_MOE_WD_T,         /* bf16 [(E+1) F x H] */
+  QAD_MOE_DA,           /* bf16 [R x F] */
+  QAD_MOE_DGU,          /* bf16 [R x 2F] */
+  QAD_MOE_WGU_T,        /* bf16 [(E+1) H x 2F] */
+  QAD_MOE_DX_ROWS,      /* bf16 [R x H] */
+  QAD_MOE_DY_ROWS_T,    /* bf16 [H x R] */
+  QAD_MOE_A_HAT_T,      /* bf16 [F x R] */
+  QAD_MOE_DGU_T,        /* bf16 [2F x R] */
+  QAD_MOE_X_HAT_T,      /* bf16 [H x R] */
+  QAD_MOE_NUM_BUFFERS
+};
+
+/* 0 for an unsupported shape. */
+size_t qad_moe_workspace_size(const qad_moe_shape* shape);
+int64_t qad_moe_rows_capacity(const qad_moe_shape* shape);
+/* Offset (256-byte aligned) and size of one buffer of the workspace (host outputs). */
+nvfp4_status qad_moe_workspace_buffer(const qad_moe_shape* shape, int buffer, size_t* offset, size_t* bytes);
+
+/* Forward.  shape, w: host structs.  x bf16 T x H; expert_ids int32 T x
+ * topk; combine_weights f32 T x topk; y bf16 T x H; workspace 256-byte
+ * aligned, >= qad_moe_workspace_size(shape). */
+nvfp4_status qad_moe_forward(const qad_moe_shape* shape, const qad_moe_weights* w, const void* x,
+                             const int32_t* expert_ids, const float* combine_weights, void* y, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/* Backward of the last forward on this workspace.  dy bf16 T x H; outputs
+ * dx bf16 T x H, dw_gate / dw_up bf16 (E+1) F x H, dw_down bf16 (E+1) H x F
+ * (gradients w.r.t. the master weights through the straight-through
+ * quantizers), d_combine f32 T x topk or NULL. */
+nvfp4_status qad_moe_backward(const qad_moe_shape* shape, const qad_moe_weights* w, const void* dy, void* dx,
+                              void* dw_gate, void* dw_up, void* dw_down, float* d_combine, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * KL distillation loss, forward and backward in one pass (Nemotron 3.5
  * Lightning article, "QAD的工作原理"; Nemotron-3-Nano article, "Von QAT zu
  * QAD"; full-vocabulary form of the loss in the Qwen3.6 tutorial, section 3).

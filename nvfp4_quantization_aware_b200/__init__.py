@@ -5,7 +5,9 @@ The compute lives in ``libnvfp4qad.so`` (hand-written CUDA for sm_100a, C ABI
 declared in ``include/nvfp4qad.h``).  This package is the thin Python side:
 
 * ``nvfp4_quantize``, ``nvfp4_fake_quant``, ``nvfp4_dequantize``,
-  ``nvfp4_gemm_w4a4``, ``qad_kl_fwd_bwd`` -- the C entry points under the
+  ``nvfp4_gemm_w4a4``, ``qad_kl_fwd_bwd``, ``nvfp4_gemm_bf16_grouped`` and the
+  MoE layer step (``MoeLayerStep`` over ``qad_moe_forward`` /
+  ``qad_moe_backward``) -- the C entry points under the
   same names, taking torch tensors and marshalling pointers, sizes and the
   current CUDA stream (nothing is computed in Python);
 * ``FakeQuantSTE`` and ``KLDistillLoss`` -- autograd wiring: straight-through
@@ -34,6 +36,13 @@ from .binding import (  # noqa: F401
     nvfp4_quantize_grouped,
     TensorRef,
     nvfp4_gemm_w4a4,
+    nvfp4_gemm_w4a4_grouped,
+    nvfp4_gemm_bf16_grouped,
+    nvfp4_scales_to_mma,
+    nvfp4_transpose_bf16,
+    nvfp4_dequantize_transpose,
+    MoeLayerStep,
+    MOE_BUFFERS,
     nvfp4_quantize,
     nvfp4_selftest_division,
     qad_kl_fwd_bwd,

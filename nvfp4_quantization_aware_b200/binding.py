@@ -32,6 +32,52 @@ class TensorRef(ctypes.Structure):
                 ("out", ctypes.c_void_p), ("ld_out", ctypes.c_int64)]
 
 
+class MoeShape(ctypes.Structure):
+    """qad_moe_shape of include/nvfp4qad.h."""
+    _fields_ = [("tokens", ctypes.c_int), ("hidden", ctypes.c_int), ("ffn", ctypes.c_int),
+                ("experts", ctypes.c_int), ("topk", ctypes.c_int), ("save_act", ctypes.c_int)]
+
+
+class MoeWeights(ctypes.Structure):
+    """qad_moe_weights of include/nvfp4qad.h."""
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "w_gate", "w_up", "w_down", "gate_ts", "up_ts", "down_ts", "gate_sb", "up_sb", "down_sb",
+        "gate_sb_mma", "up_sb_mma", "down_sb_mma", "x_ts", "a_ts")]
+
+
+# qad_moe_buffer of include/nvfp4qad.h: name -> (index, dtype, shape given (T, H, F, G, k, R))
+MOE_BUFFERS = {
+    "seg_len": (0, torch.int32, lambda T, H, F, G, k, R: (G,)),
+    "seg_off": (1, torch.int32, lambda T, H, F, G, k, R: (G + 1,)),
+    "row_token": (2, torch.int32, lambda T, H, F, G, k, R: (R,)),
+    "row_weight": (3, torch.float32, lambda T, H, F, G, k, R: (R,)),
+    "slot_row": (4, torch.int32, lambda T, H, F, G, k, R: (T, k)),
+    "x_codes": (5, torch.uint8, lambda T, H, F, G, k, R: (R, H // 2)),
+    "x_scales": (6, torch.uint8, lambda T, H, F, G, k, R: (R * H // 16,)),
+    "x_hat": (7, torch.bfloat16, lambda T, H, F, G, k, R: (R, H)),
+    "wg_codes": (8, torch.uint8, lambda T, H, F, G, k, R: (G * F, H // 2)),
+    "wu_codes": (9, torch.uint8, lambda T, H, F, G, k, R: (G * F, H // 2)),
+    "wd_codes": (10, torch.uint8, lambda T, H, F, G, k, R: (G * H, F // 2)),
+    "h_gate": (11, torch.bfloat16, lambda T, H, F, G, k, R: (R, F)),
+    "h_up": (12, torch.bfloat16, lambda T, H, F, G, k, R: (R, F)),
+    "a_codes": (13, torch.uint8, lambda T, H, F, G, k, R: (R, F // 2)),
+    "a_scales": (14, torch.uint8, lambda T, H, F, G, k, R: (R * F // 16,)),
+    "a_hat": (15, torch.bfloat16, lambda T, H, F, G, k, R: (R, F)),
+    "act": (16, torch.bfloat16, lambda T, H, F, G, k, R: (R, F)),
+    "y_rows": (17, torch.bfloat16, lambda T, H, F, G, k, R: (R, H)),
+    "dy_rows": (18, torch.bfloat16, lambda T, H, F, G, k, R: (R, H)),
+    "wd_t": (19, torch.bfloat16, lambda T, H, F, G, k, R: (G * F, H)),
+    "da": (20, torch.bfloat16, lambda T, H, F, G, k, R: (R, F)),
+    "dgu": (21, torch.bfloat16, lambda T, H, F, G, k, R: (R, 2 * F)),
+    "wgu_t": (22, torch.bfloat16, lambda T, H, F, G, k, R: (G * H, 2 * F)),
+    "dx_rows": (23, torch.bfloat16, lambda T, H, F, G, k, R: (R, H)),
+    "dy_rows_t": (24, torch.bfloat16, lambda T, H, F, G, k, R: (H, R)),
+    "a_hat_t": (25, torch.bfloat16, lambda T, H, F, G, k, R: (F, R)),
+    "dgu_t": (26, torch.bfloat16, lambda T, H, F, G, k, R: (2 * F, R)),
+    "x_hat_t": (27, torch.bfloat16, lambda T, H, F, G, k, R: (H, R)),
+}
+
+
 class NVFP4Error(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
@@ -80,16 +126,54 @@ def lib() -> ctypes.CDLL:
     L.nvfp4_fake_quant_grouped.restype = i32
     L.nvfp4_selftest_division.argtypes = [p, p, p]
     L.nvfp4_selftest_division.restype = i32
-    if hasattr(L, "nvfp4_gemm_w4a4"):
-        L.nvfp4_gemm_workspace_size.argtypes = [i64, i64, i64]
-        L.nvfp4_gemm_workspace_size.restype = sz
-        L.nvfp4_gemm_w4a4.argtypes = [p, p, p, p, p, p, i64, i64, i64, p, i64, p, sz, p]
-        L.nvfp4_gemm_w4a4.restype = i32
-    if hasattr(L, "qad_kl_fwd_bwd"):
-        L.qad_kl_workspace_size.argtypes = [i64, i64, i32]
-        L.qad_kl_workspace_size.restype = sz
-        L.qad_kl_fwd_bwd.argtypes = [p, p, i32, i64, i64, i64, f32, p, p, p, i64, f32, p, sz, p]
-        L.qad_kl_fwd_bwd.restype = i32
+    L.nvfp4_gemm_workspace_size.argtypes = [i64, i64, i64]
+    L.nvfp4_gemm_workspace_size.restype = sz
+    L.nvfp4_gemm_w4a4.argtypes = [p, p, p, p, p, p, i64, i64, i64, p, i64, p, sz, p]
+    L.nvfp4_gemm_w4a4.restype = i32
+    L.nvfp4_gemm_w4a4_grouped.argtypes = [i32, p, p, p, i64, p, p, p, p, p, i64, i64, p, i64, p, sz, p]
+    L.nvfp4_gemm_w4a4_grouped.restype = i32
+    L.nvfp4_gemm_bf16_grouped.argtypes = [i32, i32, p, i64, i64, i64, p, i64, i64, p, p, i64, i64, i64, p, i64, p]
+    L.nvfp4_gemm_bf16_grouped.restype = i32
+    L.qad_kl_workspace_size.argtypes = [i64, i64, i32]
+    L.qad_kl_workspace_size.restype = sz
+    L.qad_kl_fwd_bwd.argtypes = [p, p, i32, i64, i64, i64, f32, p, p, p, i64, f32, p, sz, p]
+    L.qad_kl_fwd_bwd.restype = i32
+    # MoE layer step
+    L.nvfp4_moe_rows_capacity.argtypes = [i32, i32, i32]
+    L.nvfp4_moe_rows_capacity.restype = i64
+    L.nvfp4_moe_route.argtypes = [p, p, i32, i32, i32, p, p, p, p, p, i64, p]
+    L.nvfp4_moe_route.restype = i32
+    L.nvfp4_moe_gather_quantize.argtypes = [p, i64, p, p, i32, p, i64, i64, p, p, p, p]
+    L.nvfp4_moe_gather_quantize.restype = i32
+    L.nvfp4_moe_swiglu_quantize.argtypes = [p, p, i64, p, p, i32, p, i64, i64, p, p, p, p, p]
+    L.nvfp4_moe_swiglu_quantize.restype = i32
+    L.nvfp4_moe_combine.argtypes = [p, i64, p, p, i32, i32, p, i32, p, p]
+    L.nvfp4_moe_combine.restype = i32
+    L.nvfp4_moe_scale_rows.argtypes = [p, i64, p, p, p, i32, i64, p, p]
+    L.nvfp4_moe_scale_rows.restype = i32
+    L.nvfp4_moe_swiglu_backward.argtypes = [p, p, p, i64, p, p, i32, i64, p, p]
+    L.nvfp4_moe_swiglu_backward.restype = i32
+    L.nvfp4_moe_gather_sum.argtypes = [p, i64, p, i32, i32, p, i32, p, p]
+    L.nvfp4_moe_gather_sum.restype = i32
+    L.nvfp4_moe_router_grad.argtypes = [p, p, i64, p, i32, i32, p, p]
+    L.nvfp4_moe_router_grad.restype = i32
+    L.nvfp4_transpose_bf16.argtypes = [p, i64, i64, i64, p, i64, p]
+    L.nvfp4_transpose_bf16.restype = i32
+    L.nvfp4_dequantize_transpose.argtypes = [p, p, p, i32, i64, i64, p, i64, i64, p]
+    L.nvfp4_dequantize_transpose.restype = i32
+    L.nvfp4_scales_to_mma.argtypes = [p, i64, i64, p, p]
+    L.nvfp4_scales_to_mma.restype = i32
+    shp, wts = ctypes.POINTER(MoeShape), ctypes.POINTER(MoeWeights)
+    L.qad_moe_workspace_size.argtypes = [shp]
+    L.qad_moe_workspace_size.restype = sz
+    L.qad_moe_rows_capacity.argtypes = [shp]
+    L.qad_moe_rows_capacity.restype = i64
+    L.qad_moe_workspace_buffer.argtypes = [shp, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+    L.qad_moe_workspace_buffer.restype = i32
+    L.qad_moe_forward.argtypes = [shp, wts, p, p, p, p, p, sz, p]
+    L.qad_moe_forward.restype = i32
+    L.qad_moe_backward.argtypes = [shp, wts, p, p, p, p, p, p, p, sz, p]
+    L.qad_moe_backward.restype = i32
     _lib = L
     return L
 
@@ -343,6 +427,28 @@ def nvfp4_gemm_w4a4(a_codes: torch.Tensor, a_scales_mma: torch.Tensor, a_tensor_
     return out
 
 
+def nvfp4_gemm_w4a4_grouped(a_codes: torch.Tensor, a_scales_mma: torch.Tensor, a_tensor_scales: torch.Tensor,
+                            a_row_offsets: torch.Tensor, a_rows: torch.Tensor, b_codes: torch.Tensor,
+                            b_scales_mma: torch.Tensor, b_tensor_scales: torch.Tensor, N: int,
+                            out: torch.Tensor | None = None) -> torch.Tensor:
+    """Grouped W4A4 GEMM: group g multiplies A rows [off[g], off[g] + rows[g]) by
+    B rows [g N, (g+1) N).  a_codes [rows_total, K/2]; b_codes [groups * N, K/2];
+    a_row_offsets int32 [groups + 1], a_rows int32 [groups] (device)."""
+    _cuda2d(a_codes, "a_codes")
+    _cuda2d(b_codes, "b_codes")
+    groups = a_rows.numel()
+    rows_total, K2 = a_codes.shape
+    dev = a_codes.device
+    if out is None:
+        out = torch.empty(rows_total, N, dtype=torch.bfloat16, device=dev)
+    st = lib().nvfp4_gemm_w4a4_grouped(groups, _ptr(a_codes), _ptr(a_scales_mma), _ptr(a_tensor_scales), rows_total,
+                                       _ptr(a_row_offsets), _ptr(a_rows), _ptr(b_codes), _ptr(b_scales_mma),
+                                       _ptr(b_tensor_scales), N, 2 * K2, _ptr(out), out.stride(0), None, 0,
+                                       _stream(dev))
+    _check(st, "nvfp4_gemm_w4a4_grouped")
+    return out
+
+
 # ------------------------------------------------------------------ KL
 
 def qad_kl_fwd_bwd(teacher: torch.Tensor, student: torch.Tensor, temperature: float = 1.0,
@@ -375,3 +481,114 @@ def qad_kl_fwd_bwd(teacher: torch.Tensor, student: torch.Tensor, temperature: fl
                           0 if workspace is None else workspace.numel(), _stream(dev))
     _check(st, "qad_kl_fwd_bwd")
     return loss, row_kl, dlogits
+
+
+# ------------------------------------------------------------------ BF16 grouped GEMM
+
+def nvfp4_gemm_bf16_grouped(mode: int, a: torch.Tensor, b: torch.Tensor, seg_off: torch.Tensor,
+                            seg_len: torch.Tensor, M: int, N: int, K: int, out: torch.Tensor | None = None):
+    """C = A B^T per group, bf16.  mode 0: A rows in 128-aligned segments, B of
+    group g = rows [g N, (g+1) N); mode 1: group g reduces over columns
+    [seg_off[g], seg_off[g] + seg_len[g]), C of group g = rows [g M, (g+1) M)."""
+    _cuda2d(a, "a")
+    _cuda2d(b, "b")
+    groups = seg_len.numel()
+    dev = a.device
+    if out is None:
+        rows = a.shape[0] if mode == 0 else groups * M
+        out = torch.empty(rows, N, dtype=torch.bfloat16, device=dev)
+    st = lib().nvfp4_gemm_bf16_grouped(mode, groups, _ptr(a), a.shape[0], a.shape[1], a.stride(0), _ptr(b),
+                                       b.shape[0], b.stride(0), _ptr(seg_off), _ptr(seg_len), M, N, K, _ptr(out),
+                                       out.stride(0), _stream(dev))
+    _check(st, "nvfp4_gemm_bf16_grouped")
+    return out
+
+
+def nvfp4_scales_to_mma(block_scales: torch.Tensor, rows: int, cols: int) -> torch.Tensor:
+    """ROWMAJOR block scales [rows, cols/16] -> MMA layout (flat uint8)."""
+    out = torch.empty(mma_scales_bytes(rows, cols), dtype=torch.uint8, device=block_scales.device)
+    st = lib().nvfp4_scales_to_mma(_ptr(block_scales), rows, cols, _ptr(out), _stream(block_scales.device))
+    _check(st, "nvfp4_scales_to_mma")
+    return out
+
+
+def nvfp4_transpose_bf16(x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    _cuda2d(x, "x")
+    rows, cols = x.shape
+    if out is None:
+        out = torch.empty(cols, rows, dtype=torch.bfloat16, device=x.device)
+    st = lib().nvfp4_transpose_bf16(_ptr(x), x.stride(0), rows, cols, _ptr(out), out.stride(0), _stream(x.device))
+    _check(st, "nvfp4_transpose_bf16")
+    return out
+
+
+def nvfp4_dequantize_transpose(codes: torch.Tensor, block_scales: torch.Tensor, tensor_scales: torch.Tensor,
+                               groups: int, rows_per_group: int, cols: int, out: torch.Tensor | None = None,
+                               col_off: int = 0) -> torch.Tensor:
+    """out[g cols + c, col_off + r] = bf16 dequantized element (g, r, c) of the stack."""
+    dev = codes.device
+    if out is None:
+        out = torch.empty(groups * cols, rows_per_group, dtype=torch.bfloat16, device=dev)
+    st = lib().nvfp4_dequantize_transpose(_ptr(codes), _ptr(block_scales), _ptr(tensor_scales), groups,
+                                          rows_per_group, cols, _ptr(out), out.stride(0), col_off, _stream(dev))
+    _check(st, "nvfp4_dequantize_transpose")
+    return out
+
+
+# ------------------------------------------------------------------ MoE layer step
+
+class MoeLayerStep:
+    """Holds the C structs and the workspace of qad_moe_forward / qad_moe_backward
+    for one layer shape.  Tensors are kept referenced so the raw pointers in
+    the structs stay valid."""
+
+    def __init__(self, tokens: int, hidden: int, ffn: int, experts: int, topk: int, weights: dict,
+                 save_act: bool = False, device="cuda"):
+        self.shape = MoeShape(tokens, hidden, ffn, experts, topk, 1 if save_act else 0)
+        L = lib()
+        self.ws_bytes = int(L.qad_moe_workspace_size(ctypes.byref(self.shape)))
+        if self.ws_bytes == 0:
+            raise NVFP4Error(2, "qad_moe_workspace_size")
+        self.rows_cap = int(L.qad_moe_rows_capacity(ctypes.byref(self.shape)))
+        self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device)
+        self._keep = dict(weights)
+        self.weights = MoeWeights(**{n: weights[n].data_ptr() for n, _ in MoeWeights._fields_})
+        self.device = torch.device(device)
+
+    def buffer(self, name: str) -> torch.Tensor:
+        """A view of one workspace buffer (see MOE_BUFFERS)."""
+        idx, dtype, shape_fn = MOE_BUFFERS[name]
+        off, nb = ctypes.c_size_t(0), ctypes.c_size_t(0)
+        _check(lib().qad_moe_workspace_buffer(ctypes.byref(self.shape), idx, ctypes.byref(off), ctypes.byref(nb)),
+               "qad_moe_workspace_buffer")
+        s = self.shape
+        shape = shape_fn(s.tokens, s.hidden, s.ffn, s.experts + 1, s.topk, self.rows_cap)
+        raw = self.workspace[off.value:off.value + nb.value]
+        return raw.view(dtype).view(*shape)
+
+    def forward(self, x: torch.Tensor, expert_ids: torch.Tensor, combine_weights: torch.Tensor,
+                y: torch.Tensor | None = None) -> torch.Tensor:
+        if y is None:
+            y = torch.empty_like(x)
+        st = lib().qad_moe_forward(ctypes.byref(self.shape), ctypes.byref(self.weights), _ptr(x), _ptr(expert_ids),
+                                   _ptr(combine_weights), _ptr(y), _ptr(self.workspace), self.ws_bytes,
+                                   _stream(self.device))
+        _check(st, "qad_moe_forward")
+        return y
+
+    def backward(self, dy: torch.Tensor, dx=None, dw_gate=None, dw_up=None, dw_down=None, d_combine=None,
+                 want_combine_grad: bool = True):
+        s = self.shape
+        G, H, F = s.experts + 1, s.hidden, s.ffn
+        dev = self.device
+        dx = torch.empty_like(dy) if dx is None else dx
+        dw_gate = torch.empty(G * F, H, dtype=torch.bfloat16, device=dev) if dw_gate is None else dw_gate
+        dw_up = torch.empty(G * F, H, dtype=torch.bfloat16, device=dev) if dw_up is None else dw_up
+        dw_down = torch.empty(G * H, F, dtype=torch.bfloat16, device=dev) if dw_down is None else dw_down
+        if want_combine_grad and d_combine is None:
+            d_combine = torch.empty(s.tokens, s.topk, dtype=torch.float32, device=dev)
+        st = lib().qad_moe_backward(ctypes.byref(self.shape), ctypes.byref(self.weights), _ptr(dy), _ptr(dx),
+                                    _ptr(dw_gate), _ptr(dw_up), _ptr(dw_down), _ptr(d_combine),
+                                    _ptr(self.workspace), self.ws_bytes, _stream(dev))
+        _check(st, "qad_moe_backward")
+        return dx, dw_gate, dw_up, dw_down, d_combine

@@ -18,6 +18,8 @@ namespace nvfp4 {
 extern __device__ int g_device_error;
 
 constexpr int kErrWaitTimeout = 1;
+constexpr int kErrRowsCapacity = 2;   // routed rows exceed the permutation buffer
+constexpr int kErrExpertId = 3;       // an expert id outside [0, experts)
 
 NVFP4_DEV void report_error(int code) { atomicCAS(&g_device_error, 0, code); }
 

@@ -48,7 +48,9 @@ struct GemmCfg {
   static constexpr int SFA_BYTES = 512 * KB_PER_STAGE;
   static constexpr int SFB_BYTES = 512 * KB_PER_STAGE * NB_SFB;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int MAX_GROUPS = 256;         // grouped problems: segment table in shared memory
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ +
+                                    (2 * MAX_GROUPS + 1) * 4 /*segment table*/;
   // tensor-memory columns: accumulator, then two sets of scales (alternating
   // by stage parity)
   static constexpr int TM_ACC = 0;
@@ -74,14 +76,50 @@ struct GemmParams {
   int kchunks;           // K / 64
   int b_rowtiles;        // ceil(N / 128): 128-row scale tiles present for B
   int c_vec16;           // C base 16-byte aligned and ldc % 8 == 0: 16-byte stores
+  // Grouped problems (groups > 0): group g owns A rows [a_off[g], a_off[g] + a_rows[g]) with
+  // a_off[g] a multiple of 128 (device arrays; a_off[groups] is the padded row total), B rows
+  // [g * N, (g + 1) * N), tensor scales a_ts[g] and b_ts[g].
+  int groups;
+  const int32_t* a_off;
+  const int32_t* a_rows;
 };
 
-// Tile t of the persistent schedule -> (m0, n0); N fastest, so the CTAs that
-// run at the same time share A rows and sweep B (both stay in L2).
-NVFP4_DEV void tile_coords(int t, int num_n, int BM, int BN, int& m0, int& n0) {
+// One output tile of the persistent schedule.
+struct TileInfo {
+  int m0, n0;     // first row of A / C and first column of C
+  int b0;         // first row of B
+  int g;          // group (0 for a dense problem)
+  int row_end;    // rows of A at or beyond this are not part of the problem
+  bool empty;     // no valid row (grouped: padding of a segment)
+};
+
+// Tile t of the persistent schedule; N fastest, so the CTAs that run at the
+// same time share A rows and sweep B (both stay in L2).  For grouped problems
+// the group is found by binary search over the segment table in shared memory.
+NVFP4_DEV TileInfo tile_info(int t, int num_n, int BM, int BN, const GemmParams& p, const int32_t* s_off,
+                             const int32_t* s_rows) {
+  TileInfo ti;
   const int mt = t / num_n;
-  m0 = mt * BM;
-  n0 = (t - mt * num_n) * BN;
+  ti.m0 = mt * BM;
+  ti.n0 = (t - mt * num_n) * BN;
+  if (p.groups == 0) {
+    ti.g = 0;
+    ti.b0 = ti.n0;
+    ti.row_end = p.M;
+    ti.empty = false;
+    return ti;
+  }
+  int lo = 0, hi = p.groups - 1;  // last g with s_off[g] <= m0
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_off[mid] <= ti.m0) lo = mid;
+    else hi = mid - 1;
+  }
+  ti.g = lo;
+  ti.b0 = lo * p.N + ti.n0;
+  ti.row_end = s_off[lo] + s_rows[lo];
+  ti.empty = ti.m0 >= ti.row_end;
+  return ti;
 }
 
 template <int BN>
@@ -101,12 +139,21 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
   uint64_t* acc_empty = acc_full + 1;       // epilogue -> MMA: accumulator drained
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+  int32_t* s_off = reinterpret_cast<int32_t*>(smem + C::STAGES * C::STAGE_BYTES + 256);
+  int32_t* s_rows = s_off + C::MAX_GROUPS + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int num_kt = (p.kchunks + C::KB_PER_STAGE - 1) / C::KB_PER_STAGE;
   const int num_n = (p.N + C::BN - 1) / C::BN;
-  const int num_tiles = num_n * ((p.M + C::BM - 1) / C::BM);
+  for (int i = threadIdx.x; i < p.groups; i += blockDim.x) {
+    s_off[i] = __ldg(p.a_off + i);
+    s_rows[i] = __ldg(p.a_rows + i);
+  }
+  if (threadIdx.x == 0 && p.groups > 0) s_off[p.groups] = __ldg(p.a_off + p.groups);
+  __syncthreads();
+  const int m_total = p.groups > 0 ? s_off[p.groups] : p.M;
+  const int num_tiles = num_n * ((m_total + C::BM - 1) / C::BM);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -134,12 +181,13 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
     if (lane == 0) {
       int it = 0;  // k-iteration counter across all tiles (ring position)
       for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
-        int m0, n0;
-        tile_coords(t, num_n, C::BM, C::BN, m0, n0);
+        const TileInfo tl = tile_info(t, num_n, C::BM, C::BN, p, s_off, s_rows);
+        if (tl.empty) continue;
+        const int m0 = tl.m0;
         const int a_tile = m0 / 128;
         int nsfb = 0;
         for (int j = 0; j < C::NB_SFB; ++j)
-          if (n0 / 128 + j < p.b_rowtiles) ++nsfb;
+          if (tl.b0 / 128 + j < p.b_rowtiles) ++nsfb;
         for (int kt = 0; kt < num_kt; ++kt, ++it) {
           const int s = it % C::STAGES;
           const uint32_t ph = (uint32_t)(it / C::STAGES) & 1u;
@@ -150,13 +198,13 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
           const uint32_t bytes = C::A_BYTES + C::B_BYTES + (uint32_t)nkc * 512u * (1u + (uint32_t)nsfb);
           mbar_expect_tx(&full[s], bytes);
           tma_load_2d(sA + s * C::A_BYTES, &tmA, kt * (C::BK / 2), m0, &full[s]);
-          tma_load_2d(sB + s * C::B_BYTES, &tmB, kt * (C::BK / 2), n0, &full[s]);
+          tma_load_2d(sB + s * C::B_BYTES, &tmB, kt * (C::BK / 2), tl.b0, &full[s]);
           const int64_t kc0 = (int64_t)kt * C::KB_PER_STAGE;
           bulk_g2s(sSFA + s * C::SFA_BYTES, p.a_sf + ((int64_t)a_tile * p.kchunks + kc0) * 512,
                    (uint32_t)nkc * 512u, &full[s]);
           for (int j = 0; j < nsfb; ++j)
             bulk_g2s(sSFB + s * C::SFB_BYTES + j * 512 * C::KB_PER_STAGE,
-                     p.b_sf + ((int64_t)(n0 / 128 + j) * p.kchunks + kc0) * 512, (uint32_t)nkc * 512u, &full[s]);
+                     p.b_sf + ((int64_t)(tl.b0 / 128 + j) * p.kchunks + kc0) * 512, (uint32_t)nkc * 512u, &full[s]);
         }
       }
     }
@@ -166,7 +214,8 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
       const uint32_t acc = tmem + C::TM_ACC;
       int it = 0;
       int ti = 0;  // tiles done by this CTA
-      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x, ++ti) {
+      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+        if (tile_info(t, num_n, C::BM, C::BN, p, s_off, s_rows).empty) continue;
         // the epilogue must have drained the previous tile's accumulator
         if (!mbar_wait_bounded(acc_empty, ((uint32_t)ti & 1u) ^ 1u)) { *abort_flag = 1; break; }
         tc_fence_after();
@@ -203,6 +252,7 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
           tc_commit(&empty[s]);
         }
         tc_commit(acc_full);
+        ++ti;
       }
     }
   } else {
@@ -210,12 +260,14 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
     const int sub = warp & 3;                      // TMEM subpartition this warp may read
     const int cbase = ((warp - 2) >> 2) * (C::BN / 2);  // this warp's half of the columns
     constexpr int HALF = C::BN / 2;
-    const float alpha = __fmul_rn(__ldg(p.a_ts), __ldg(p.b_ts));
     int ti = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++ti) {
-      int m0, n0;
-      tile_coords(t, num_n, C::BM, C::BN, m0, n0);
-      const bool ok = mbar_wait_bounded(acc_full, (uint32_t)ti & 1u);
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      const TileInfo tl = tile_info(t, num_n, C::BM, C::BN, p, s_off, s_rows);
+      if (tl.empty) continue;
+      const int m0 = tl.m0, n0 = tl.n0;
+      const float alpha = __fmul_rn(__ldg(p.a_ts + tl.g), __ldg(p.b_ts + tl.g));
+      const int par_ti = ti++;
+      const bool ok = mbar_wait_bounded(acc_full, (uint32_t)par_ti & 1u);
       if (!ok) *abort_flag = 1;
       if (!ok || *abort_flag) break;
       tc_fence_after();
@@ -241,7 +293,7 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
       if (lane == 0) mbar_arrive(acc_empty);
       // ... and store while the next tile accumulates
       const int row = m0 + sub * 32 + lane;
-      if (row < p.M) {
+      if (row < tl.row_end) {
         __nv_bfloat16* crow = p.c + (int64_t)row * p.ldc;
 #pragma unroll
         for (int c0 = 0; c0 < HALF; c0 += 32) {
@@ -314,7 +366,8 @@ static nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* b, const GemmPa
       return NVFP4_ERR_CUDA;
     attr_set = true;
   }
-  const int tiles = ((p.N + C::BN - 1) / C::BN) * ((p.M + C::BM - 1) / C::BM);
+  // grouped problems: the tile count lives on the device, so one CTA per SM
+  const int tiles = p.groups > 0 ? 1 << 30 : ((p.N + C::BN - 1) / C::BN) * ((p.M + C::BM - 1) / C::BM);
   static int sms = 0;
   if (sms == 0) {
     int dev = 0;
@@ -323,6 +376,22 @@ static nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* b, const GemmPa
   }
   const int grid = tiles < sms ? tiles : sms;  // persistent: one CTA per SM
   gemm_w4a4_kernel<BN><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, p);
+  count_launches(1);
+  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+template <int BN>
+static nvfp4_status launch_gemm_grouped(const uint8_t* a, const uint8_t* b, const GemmParams& p, int64_t b_rows,
+                                        cudaStream_t s) {
+  using C = GemmCfg<BN>;
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, a, p.M, p.K / 2, C::BM) || !make_tmap(&tb, b, b_rows, p.K / 2, C::BN)) return NVFP4_ERR_CUDA;
+  if (cudaFuncSetAttribute(gemm_w4a4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+      cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  gemm_w4a4_kernel<BN><<<sms, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, p);
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
@@ -366,7 +435,54 @@ nvfp4_status nvfp4_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_scales_mma
   p.kchunks = (int)(K / 64);
   p.b_rowtiles = (int)((N + 127) / 128);
   p.c_vec16 = (((uintptr_t)c & 15u) == 0 && (ldc % 8) == 0) ? 1 : 0;
+  p.groups = 0;
+  p.a_off = nullptr;
+  p.a_rows = nullptr;
   return launch_gemm<256>(a_codes, b_codes, p, (cudaStream_t)stream);
+}
+
+size_t nvfp4_gemm_grouped_workspace_size(int groups, int64_t a_rows_total, int64_t N, int64_t K) {
+  (void)groups;
+  (void)a_rows_total;
+  (void)N;
+  (void)K;
+  return 0;
+}
+
+nvfp4_status nvfp4_gemm_w4a4_grouped(int groups, const uint8_t* a_codes, const uint8_t* a_scales_mma,
+                                     const float* a_tensor_scales, int64_t a_rows_total, const int32_t* a_row_offsets,
+                                     const int32_t* a_rows, const uint8_t* b_codes, const uint8_t* b_scales_mma,
+                                     const float* b_tensor_scales, int64_t N, int64_t K, void* c, int64_t ldc,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (groups < 1 || groups > GemmCfg<256>::MAX_GROUPS) return NVFP4_ERR_SHAPE;
+  if (a_rows_total < 128 || a_rows_total % 128 != 0 || N < 128 || N % 128 != 0 || K < 64 || K % 64 != 0 || ldc < N)
+    return NVFP4_ERR_SHAPE;
+  if (a_rows_total > 0x7FFFFFFF || (int64_t)groups * N > 0x7FFFFFFF || K > 0x7FFFFFFF) return NVFP4_ERR_SHAPE;
+  if (!a_codes || !a_scales_mma || !a_tensor_scales || !a_row_offsets || !a_rows || !b_codes || !b_scales_mma ||
+      !b_tensor_scales || !c)
+    return NVFP4_ERR_ARG;
+  auto a16 = [](const void* q) { return ((uintptr_t)q & 15u) == 0; };
+  if (!a16(a_codes) || !a16(b_codes) || !a16(a_scales_mma) || !a16(b_scales_mma) || ((uintptr_t)c & 3u))
+    return NVFP4_ERR_ALIGN;
+  GemmParams p;
+  p.a_sf = a_scales_mma;
+  p.b_sf = b_scales_mma;
+  p.a_ts = a_tensor_scales;
+  p.b_ts = b_tensor_scales;
+  p.c = reinterpret_cast<__nv_bfloat16*>(c);
+  p.ldc = ldc;
+  p.M = (int)a_rows_total;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.kchunks = (int)(K / 64);
+  p.b_rowtiles = (int)((int64_t)groups * N / 128);
+  p.c_vec16 = (((uintptr_t)c & 15u) == 0 && (ldc % 8) == 0) ? 1 : 0;
+  p.groups = groups;
+  p.a_off = a_row_offsets;
+  p.a_rows = a_rows;
+  return launch_gemm_grouped<256>(a_codes, b_codes, p, (int64_t)groups * N, (cudaStream_t)stream);
 }
 
 }  // extern "C"

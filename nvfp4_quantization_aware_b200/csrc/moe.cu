@@ -1,0 +1,607 @@
+// moe.cu -- kernels of the QAD student's MoE layer step around the grouped
+// GEMMs: routing into per-expert segments, NVFP4 quantization of the routed
+// activations and of the SwiGLU output, the weighted combine, and the
+// straight-through backward pieces.
+//
+// The layer is the pages' MoE block: 128 routed experts plus one shared
+// expert, 6 routed experts per token (Nemotron-3-Nano-30B NVFP4 article, "Was
+// ist Nemotron-Nano-3-30B-A3B-NVFP4?"), expert FFNs with down/gate/up
+// projections quantized W4A4 NVFP4 with frozen scales (Qwen3.6-35B-A3B W4A4
+// tutorial, "2. PTQ"; Nemotron 3.5 Lightning NVFP4 article, "量化尺度处理策略").
+//
+// Layout.  Group g < E is routed expert g, group E the shared expert.  The
+// routed (token, slot) pairs are permuted into R rows: group g owns rows
+// [off[g], off[g] + len[g]), off[g] a multiple of 128; rows past len[g] up to
+// the next segment are padding (token -1) and every kernel writes zeros
+// there, which the K-segmented weight-gradient GEMMs rely on.  Within a
+// segment rows are in increasing (token, slot) order, so every result is
+// deterministic.
+#include "quant_common.cuh"
+
+namespace nvfp4 {
+namespace moe {
+
+constexpr int kMaxGroups = 256;
+
+// Group owning permuted row r: last g with off[g] <= r (off in shared memory).
+NVFP4_DEV int group_of_row(const int32_t* s_off, int groups, int r) {
+  int lo = 0, hi = groups - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_off[mid] <= r) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+NVFP4_DEV int pad128(int n) { return (n + 127) & ~127; }
+
+// ------------------------------------------------------------------ routing
+
+// len[e] = number of assignments routed to expert e (one block per expert);
+// len[E] = T for the shared expert.
+// The last block marks assignments with an id outside [0, experts) (slot
+// -1, device error word kErrExpertId); they are routed nowhere.
+__global__ void route_count_kernel(const int32_t* __restrict__ ids, int assignments, int experts, int tokens,
+                                   int32_t* __restrict__ len, int32_t* __restrict__ slot_row) {
+  const int e = blockIdx.x;
+  if (e == experts) {
+    if (threadIdx.x == 0) len[e] = tokens;
+    for (int i = threadIdx.x; i < assignments; i += blockDim.x) {
+      const int id = __ldg(ids + i);
+      if (id < 0 || id >= experts) {
+        slot_row[i] = -1;
+        report_error(kErrExpertId);
+      }
+    }
+    return;
+  }
+  int c = 0;
+  for (int i = threadIdx.x; i < assignments; i += blockDim.x) c += (__ldg(ids + i) == e);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
+  __shared__ int part[32];
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int tot = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += part[w];
+    len[e] = tot;
+  }
+}
+
+// Segment offsets and the permutation (one block of 1024 threads per group).
+// Ranks within a group come from an in-order block scan, so row order is the
+// (token, slot) order.
+__global__ void __launch_bounds__(1024) route_scatter_kernel(
+    const int32_t* __restrict__ ids, const float* __restrict__ weights, int tokens, int topk, int experts,
+    const int32_t* __restrict__ len, int32_t* __restrict__ off, int32_t* __restrict__ row_token,
+    float* __restrict__ row_weight, int32_t* __restrict__ slot_row, int rows_cap) {
+  const int e = blockIdx.x;
+  const int groups = experts + 1;
+  __shared__ int s_off;
+  __shared__ int warp_sum[32];
+  if (threadIdx.x == 0) {
+    int o = 0;
+    for (int g = 0; g < e; ++g) o += pad128(__ldg(len + g));
+    s_off = o;
+    if (e == experts) {
+      // the last block also publishes the whole offset table
+      int q = 0;
+      for (int g = 0; g < groups; ++g) {
+        off[g] = q;
+        q += pad128(__ldg(len + g));
+      }
+      off[groups] = q;
+      if (q > rows_cap) report_error(kErrRowsCapacity);
+    }
+  }
+  __syncthreads();
+  const int base = s_off;
+  const int n = __ldg(len + e);
+  if (base + pad128(n) > rows_cap) return;  // reported above
+  if (e == experts) {
+    for (int t = threadIdx.x; t < tokens; t += blockDim.x) {
+      row_token[base + t] = t;
+      row_weight[base + t] = 1.0f;
+    }
+  } else {
+    const int assignments = tokens * topk;
+    int running = 0;
+    for (int a0 = 0; a0 < assignments; a0 += blockDim.x) {
+      const int a = a0 + threadIdx.x;
+      const bool hit = a < assignments && __ldg(ids + a) == e;
+      const unsigned ballot = __ballot_sync(0xFFFFFFFFu, hit);
+      const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+      if (lane == 0) warp_sum[w] = __popc(ballot);
+      __syncthreads();
+      int before = 0;
+      for (int i = 0; i < w; ++i) before += warp_sum[i];
+      int chunk_total = 0;
+      for (int i = 0; i < (int)(blockDim.x >> 5); ++i) chunk_total += warp_sum[i];
+      if (hit) {
+        const int r = base + running + before + __popc(ballot & ((1u << lane) - 1u));
+        row_token[r] = a / topk;
+        row_weight[r] = __ldg(weights + a);
+        slot_row[a] = r;
+      }
+      running += chunk_total;
+      __syncthreads();
+    }
+  }
+  for (int r = base + n + threadIdx.x; r < base + pad128(n); r += blockDim.x) {
+    row_token[r] = -1;
+    row_weight[r] = 0.0f;
+  }
+}
+
+// ------------------------------------------------------------------ quantize routed rows
+
+struct QuantRowsArgs {
+  const __nv_bfloat16* src;   // gather: x [T][cols]; activation: h_gate [R][cols]
+  const __nv_bfloat16* src2;  // activation: h_up [R][cols]
+  int64_t ld_src;
+  const int32_t* row_token;   // [rows_cap]
+  const int32_t* off;         // [groups + 1]
+  int groups;
+  const float* ts;            // frozen tensor scale per group
+  int rows_cap, cols;
+  uint8_t* codes;             // [rows_cap][cols / 2]
+  uint8_t* scales_mma;        // MMA layout of [rows_cap][cols]
+  __nv_bfloat16* xhat;        // [rows_cap][cols] dequantized (may be NULL)
+  __nv_bfloat16* act;         // activation kernel: the bf16 SwiGLU output before quantization (may be NULL)
+  int64_t kchunks;
+};
+
+// One warp per 512-column chunk of a permuted row, one lane per 16-element
+// block (FROZEN_GLOBAL: the group's tensor scale is given, block scales are
+// computed).  GATHER: the row is x[row_token[r]].  Otherwise the row is the
+// SwiGLU a = silu(h_gate) * h_up, rounded to bf16 before quantization.
+template <bool GATHER>
+__global__ void __launch_bounds__(256) quant_rows_kernel(QuantRowsArgs a) {
+  __shared__ int32_t s_off[kMaxGroups + 1];
+  for (int i = threadIdx.x; i <= a.groups; i += blockDim.x) s_off[i] = __ldg(a.off + i);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int cpr = a.cols / 512 + ((a.cols % 512) ? 1 : 0);
+  const int64_t total = (int64_t)a.rows_cap * cpr;
+  const int end_rows = s_off[a.groups];
+  for (int64_t c = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); c < total; c += (int64_t)gridDim.x * 8) {
+    const int r = (int)(c / cpr);
+    const int col = (int)(c - (int64_t)r * cpr) * 512 + lane * 16;
+    if (col >= a.cols) continue;
+    const int tok = r < end_rows ? __ldg(a.row_token + r) : -1;
+    float v[16];
+    uint32_t lo = 0, hi = 0, sb = 0;
+    float d = 0.f;
+    if (tok >= 0) {
+      const int g = group_of_row(s_off, a.groups, r);
+      const float sg = __ldg(a.ts + g);
+      if (GATHER) {
+        Block16<__nv_bfloat16> in;
+        in.load(a.src + (int64_t)tok * a.ld_src + col, false);
+        in.to_f32(v);
+      } else {
+        Block16<__nv_bfloat16> hg, hu;
+        hg.load(a.src + (int64_t)r * a.ld_src + col, false);
+        hu.load(a.src2 + (int64_t)r * a.ld_src + col, false);
+        float gv[16], uv[16];
+        hg.to_f32(gv);
+        hu.to_f32(uv);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float s = gv[i] / (1.0f + expf(-gv[i]));  // silu
+          v[i] = __bfloat162float(__float2bfloat16_rn(s * uv[i]));
+        }
+        if (a.act) Block16<__nv_bfloat16>::store(a.act + (int64_t)r * a.cols + col, v, false);
+      }
+      sb = encode_block16<true>(v, sg, __fmul_rn(6.0f, sg), false, 0u, lo, hi, d);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = 0.f;
+      if (!GATHER && a.act) Block16<__nv_bfloat16>::store(a.act + (int64_t)r * a.cols + col, v, false);
+    }
+    uint8_t* dst = a.codes + (int64_t)r * (a.cols / 2) + col / 2;
+    st_stream_u32(dst, lo);
+    st_stream_u32(dst + 4, hi);
+    a.scales_mma[mma_scale_offset(r, col >> 4, a.kchunks)] = (uint8_t)sb;
+    if (a.xhat) {
+      float o[16];
+      if (tok >= 0) decode_block16(lo, hi, d, o);
+      else
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o[i] = 0.f;
+      Block16<__nv_bfloat16>::store(a.xhat + (int64_t)r * a.cols + col, o, false);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ combine / gathers
+
+// out[t] = sum_j w[t, j] y[slot_row[t, j]] + y[shared_base + t]   (FP32 sum in
+// the fixed order j = 0..k-1, then the shared expert)
+__global__ void combine_kernel(const __nv_bfloat16* __restrict__ y, int cols, const int32_t* __restrict__ slot_row,
+                               const float* __restrict__ weights, int tokens, int topk,
+                               const int32_t* __restrict__ off, int experts, __nv_bfloat16* __restrict__ out) {
+  const int vpr = cols / 8;
+  const int shared_base = __ldg(off + experts);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)tokens * vpr;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int t = (int)(i / vpr);
+    const int c = (int)(i - (int64_t)t * vpr) * 8;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int j = 0; j < topk; ++j) {
+      const int r = __ldg(slot_row + t * topk + j);
+      if (r < 0) continue;
+      const float w = __ldg(weights + t * topk + j);
+      const uint4 v = *reinterpret_cast<const uint4*>(y + (int64_t)r * cols + c);
+      acc[0] = fmaf(w, bf16lo_to_f32(v.x), acc[0]); acc[1] = fmaf(w, bf16hi_to_f32(v.x), acc[1]);
+      acc[2] = fmaf(w, bf16lo_to_f32(v.y), acc[2]); acc[3] = fmaf(w, bf16hi_to_f32(v.y), acc[3]);
+      acc[4] = fmaf(w, bf16lo_to_f32(v.z), acc[4]); acc[5] = fmaf(w, bf16hi_to_f32(v.z), acc[5]);
+      acc[6] = fmaf(w, bf16lo_to_f32(v.w), acc[6]); acc[7] = fmaf(w, bf16hi_to_f32(v.w), acc[7]);
+    }
+    const uint4 v = *reinterpret_cast<const uint4*>(y + (int64_t)(shared_base + t) * cols + c);
+    acc[0] += bf16lo_to_f32(v.x); acc[1] += bf16hi_to_f32(v.x);
+    acc[2] += bf16lo_to_f32(v.y); acc[3] += bf16hi_to_f32(v.y);
+    acc[4] += bf16lo_to_f32(v.z); acc[5] += bf16hi_to_f32(v.z);
+    acc[6] += bf16lo_to_f32(v.w); acc[7] += bf16hi_to_f32(v.w);
+    *reinterpret_cast<uint4*>(out + (int64_t)t * cols + c) =
+        make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                   pack_bf16x2(acc[6], acc[7]));
+  }
+}
+
+// dyp[r] = row_weight[r] * dy[row_token[r]] (zero on padding rows)
+__global__ void scale_rows_kernel(const __nv_bfloat16* __restrict__ dy, int cols, const int32_t* __restrict__ row_token,
+                                  const float* __restrict__ row_weight, const int32_t* __restrict__ off, int groups,
+                                  int rows_cap, __nv_bfloat16* __restrict__ dyp) {
+  const int vpr = cols / 8;
+  const int end_rows = __ldg(off + groups);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)rows_cap * vpr;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int r = (int)(i / vpr);
+    const int c = (int)(i - (int64_t)r * vpr) * 8;
+    const int t = r < end_rows ? __ldg(row_token + r) : -1;
+    uint4 o = make_uint4(0, 0, 0, 0);
+    if (t >= 0) {
+      const float w = __ldg(row_weight + r);
+      const uint4 v = *reinterpret_cast<const uint4*>(dy + (int64_t)t * cols + c);
+      o = make_uint4(pack_bf16x2(w * bf16lo_to_f32(v.x), w * bf16hi_to_f32(v.x)),
+                     pack_bf16x2(w * bf16lo_to_f32(v.y), w * bf16hi_to_f32(v.y)),
+                     pack_bf16x2(w * bf16lo_to_f32(v.z), w * bf16hi_to_f32(v.z)),
+                     pack_bf16x2(w * bf16lo_to_f32(v.w), w * bf16hi_to_f32(v.w)));
+    }
+    *reinterpret_cast<uint4*>(dyp + (int64_t)r * cols + c) = o;
+  }
+}
+
+// SwiGLU backward: with s = sigmoid(g), silu(g) = g s,
+//   dg = da * u * s * (1 + g (1 - s)),  du = da * silu(g);
+// written as dgu[r] = [dg | du] (zero on padding rows).
+__global__ void swiglu_bwd_kernel(const __nv_bfloat16* __restrict__ da, const __nv_bfloat16* __restrict__ hg,
+                                  const __nv_bfloat16* __restrict__ hu, int cols, const int32_t* __restrict__ row_token,
+                                  const int32_t* __restrict__ off, int groups, int rows_cap,
+                                  __nv_bfloat16* __restrict__ dgu) {
+  const int end_rows = __ldg(off + groups);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)rows_cap * cols;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int r = (int)(i / cols);
+    const int c = (int)(i - (int64_t)r * cols);
+    const int t = r < end_rows ? __ldg(row_token + r) : -1;
+    float dg = 0.f, du = 0.f;
+    if (t >= 0) {
+      const float g = __bfloat162float(hg[i]), u = __bfloat162float(hu[i]), d = __bfloat162float(da[i]);
+      const float s = 1.0f / (1.0f + expf(-g));
+      dg = d * u * s * (1.0f + g * (1.0f - s));
+      du = d * g * s;
+    }
+    dgu[(int64_t)r * 2 * cols + c] = __float2bfloat16_rn(dg);
+    dgu[(int64_t)r * 2 * cols + cols + c] = __float2bfloat16_rn(du);
+  }
+}
+
+// dx[t] = sum_j dxp[slot_row[t, j]] + dxp[shared_base + t]   (fixed order)
+__global__ void gather_sum_kernel(const __nv_bfloat16* __restrict__ dxp, int cols, const int32_t* __restrict__ slot_row,
+                                  int tokens, int topk, const int32_t* __restrict__ off, int experts,
+                                  __nv_bfloat16* __restrict__ dx) {
+  const int vpr = cols / 8;
+  const int shared_base = __ldg(off + experts);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)tokens * vpr;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int t = (int)(i / vpr);
+    const int c = (int)(i - (int64_t)t * vpr) * 8;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int j = 0; j <= topk; ++j) {
+      const int r = j < topk ? __ldg(slot_row + t * topk + j) : shared_base + t;
+      if (r < 0) continue;
+      const uint4 v = *reinterpret_cast<const uint4*>(dxp + (int64_t)r * cols + c);
+      acc[0] += bf16lo_to_f32(v.x); acc[1] += bf16hi_to_f32(v.x);
+      acc[2] += bf16lo_to_f32(v.y); acc[3] += bf16hi_to_f32(v.y);
+      acc[4] += bf16lo_to_f32(v.z); acc[5] += bf16hi_to_f32(v.z);
+      acc[6] += bf16lo_to_f32(v.w); acc[7] += bf16hi_to_f32(v.w);
+    }
+    *reinterpret_cast<uint4*>(dx + (int64_t)t * cols + c) =
+        make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                   pack_bf16x2(acc[6], acc[7]));
+  }
+}
+
+// dw[t, j] = <dy[t], y[slot_row[t, j]]>  (one warp per assignment, FP32)
+__global__ void router_grad_kernel(const __nv_bfloat16* __restrict__ dy, const __nv_bfloat16* __restrict__ y,
+                                   int cols, const int32_t* __restrict__ slot_row, int assignments, int topk,
+                                   float* __restrict__ dw) {
+  const int lane = threadIdx.x & 31;
+  for (int a = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); a < assignments;
+       a += gridDim.x * (blockDim.x >> 5)) {
+    const int t = a / topk;
+    const int r = __ldg(slot_row + a);
+    float acc = 0.f;
+    if (r < 0) {
+      if (lane == 0) dw[a] = 0.f;
+      continue;
+    }
+    for (int c = lane * 8; c < cols; c += 256) {
+      const uint4 p = *reinterpret_cast<const uint4*>(dy + (int64_t)t * cols + c);
+      const uint4 q = *reinterpret_cast<const uint4*>(y + (int64_t)r * cols + c);
+      acc = fmaf(bf16lo_to_f32(p.x), bf16lo_to_f32(q.x), acc); acc = fmaf(bf16hi_to_f32(p.x), bf16hi_to_f32(q.x), acc);
+      acc = fmaf(bf16lo_to_f32(p.y), bf16lo_to_f32(q.y), acc); acc = fmaf(bf16hi_to_f32(p.y), bf16hi_to_f32(q.y), acc);
+      acc = fmaf(bf16lo_to_f32(p.z), bf16lo_to_f32(q.z), acc); acc = fmaf(bf16hi_to_f32(p.z), bf16hi_to_f32(q.z), acc);
+      acc = fmaf(bf16lo_to_f32(p.w), bf16lo_to_f32(q.w), acc); acc = fmaf(bf16hi_to_f32(p.w), bf16hi_to_f32(q.w), acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+    if (lane == 0) dw[a] = acc;
+  }
+}
+
+// ------------------------------------------------------------------ transposes
+
+// out[c][r] = in[r][c] for a bf16 [rows][cols] matrix (32 x 32 tiles through
+// shared memory, padded against bank conflicts).
+__global__ void transpose_bf16_kernel(const __nv_bfloat16* __restrict__ in, int64_t ld_in, int rows, int cols,
+                                      __nv_bfloat16* __restrict__ out, int64_t ld_out) {
+  __shared__ __nv_bfloat16 tile[32][33];
+  const int tiles_c = (cols + 31) / 32;
+  const int64_t ntiles = (int64_t)((rows + 31) / 32) * tiles_c;
+  for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    const int r0 = (int)(t / tiles_c) * 32, c0 = (int)(t % tiles_c) * 32;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+      const int r = r0 + i, c = c0 + threadIdx.x;
+      if (r < rows && c < cols) tile[i][threadIdx.x] = in[(int64_t)r * ld_in + c];
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+      const int c = c0 + i, r = r0 + threadIdx.x;
+      if (r < rows && c < cols) out[(int64_t)c * ld_out + r] = tile[threadIdx.x][i];
+    }
+    __syncthreads();
+  }
+}
+
+// Dequantized transpose of stacked NVFP4 weights: group g is rows
+// [g rows_g, (g+1) rows_g) of codes [*, cols/2] with row-major block scales and
+// tensor scale ts[g]; out[g cols + c][col_off + r] = value(code) * s_b * s_g
+// (bf16).  32 x 32 tiles through shared memory.
+__global__ void dequant_transpose_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sb,
+                                         const float* __restrict__ ts, int groups, int rows_g, int cols,
+                                         __nv_bfloat16* __restrict__ out, int64_t ld_out, int col_off) {
+  __shared__ float tile[32][33];
+  const int tiles_c = cols / 32;
+  const int tiles_r = (rows_g + 31) / 32;
+  const int64_t ntiles = (int64_t)groups * tiles_r * tiles_c;
+  for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    const int g = (int)(t / ((int64_t)tiles_r * tiles_c));
+    const int rem = (int)(t - (int64_t)g * tiles_r * tiles_c);
+    const int r0 = (rem / tiles_c) * 32, c0 = (rem % tiles_c) * 32;
+    const float sg = __ldg(ts + g);
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+      const int r = r0 + i, c = c0 + threadIdx.x;
+      float v = 0.f;
+      if (r < rows_g) {
+        const int64_t row = (int64_t)g * rows_g + r;
+        const uint32_t byte = __ldg(codes + row * (cols / 2) + c / 2);
+        float lo, hi;
+        e2m1x2_decode(byte, lo, hi);
+        const float d = __fmul_rn(e4m3_decode(__ldg(sb + row * (cols / 16) + c / 16)), sg);
+        v = __fmul_rn((c & 1) ? hi : lo, d);
+      }
+      tile[i][threadIdx.x] = v;
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+      const int c = c0 + i, r = r0 + threadIdx.x;
+      if (r < rows_g) out[((int64_t)g * cols + c) * ld_out + col_off + r] = __float2bfloat16_rn(tile[threadIdx.x][i]);
+    }
+    __syncthreads();
+  }
+}
+
+// Row-major block scales [rows][cols/16] -> the MMA scale layout (padding 0).
+__global__ void scales_to_mma_kernel(const uint8_t* __restrict__ sb, int64_t rows, int64_t cols,
+                                     uint8_t* __restrict__ out) {
+  const int64_t nblk = cols / 16;
+  const int64_t kchunks = (nblk + 3) / 4;
+  const int64_t rows_pad = (rows + 127) / 128 * 128;
+  const int64_t total = rows_pad * kchunks * 4;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / (kchunks * 4), kb = i - r * (kchunks * 4);
+    out[mma_scale_offset(r, kb, kchunks)] = (r < rows && kb < nblk) ? __ldg(sb + r * nblk + kb) : (uint8_t)0;
+  }
+}
+
+static int sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      n = 148;
+  }
+  return n;
+}
+
+static nvfp4_status done(int launches) {
+  count_launches(launches);
+  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+}  // namespace moe
+}  // namespace nvfp4
+
+using namespace nvfp4;
+using namespace nvfp4::moe;
+
+extern "C" {
+
+int64_t nvfp4_moe_rows_capacity(int tokens, int topk, int experts) {
+  const int64_t r = (int64_t)tokens * topk + 127ll * experts + ((int64_t)tokens + 127) / 128 * 128;
+  return (r + 127) / 128 * 128;
+}
+
+nvfp4_status nvfp4_moe_route(const int32_t* expert_ids, const float* combine_weights, int tokens, int topk,
+                             int experts, int32_t* seg_len, int32_t* seg_off, int32_t* row_token, float* row_weight,
+                             int32_t* slot_row, int64_t rows_cap, void* stream) {
+  if (tokens < 1 || topk < 1 || experts < 1 || experts + 1 > kMaxGroups) return NVFP4_ERR_SHAPE;
+  if (rows_cap < nvfp4_moe_rows_capacity(tokens, topk, experts) || rows_cap > 0x7FFFFFFF) return NVFP4_ERR_SHAPE;
+  if (!expert_ids || !combine_weights || !seg_len || !seg_off || !row_token || !row_weight || !slot_row)
+    return NVFP4_ERR_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  route_count_kernel<<<experts + 1, 1024, 0, s>>>(expert_ids, tokens * topk, experts, tokens, seg_len, slot_row);
+  route_scatter_kernel<<<experts + 1, 1024, 0, s>>>(expert_ids, combine_weights, tokens, topk, experts, seg_len,
+                                                    seg_off, row_token, row_weight, slot_row, (int)rows_cap);
+  return done(2);
+}
+
+static nvfp4_status quant_rows(bool gather, const void* src, const void* src2, int64_t ld_src, const int32_t* row_token,
+                               const int32_t* seg_off, int groups, const float* ts, int64_t rows_cap, int64_t cols,
+                               uint8_t* codes, uint8_t* scales_mma, void* xhat, void* act, void* stream) {
+  if (groups < 1 || groups > kMaxGroups || rows_cap < 128 || rows_cap % 128 || rows_cap > 0x7FFFFFFF || cols < 64 ||
+      cols % 64 || cols > 0x7FFFFFFF || ld_src < cols)
+    return NVFP4_ERR_SHAPE;
+  if (!src || (!gather && !src2) || !row_token || !seg_off || !ts || !codes || !scales_mma) return NVFP4_ERR_ARG;
+  if (((uintptr_t)src & 15u) || (ld_src * 2) % 16 || ((uintptr_t)codes & 3u) || (cols / 2) % 4 ||
+      (src2 && ((uintptr_t)src2 & 15u)) || (xhat && ((uintptr_t)xhat & 15u)) || (act && ((uintptr_t)act & 15u)))
+    return NVFP4_ERR_ALIGN;
+  QuantRowsArgs a;
+  a.src = reinterpret_cast<const __nv_bfloat16*>(src);
+  a.src2 = reinterpret_cast<const __nv_bfloat16*>(src2);
+  a.ld_src = ld_src;
+  a.row_token = row_token;
+  a.off = seg_off;
+  a.groups = groups;
+  a.ts = ts;
+  a.rows_cap = (int)rows_cap;
+  a.cols = (int)cols;
+  a.codes = codes;
+  a.scales_mma = scales_mma;
+  a.xhat = reinterpret_cast<__nv_bfloat16*>(xhat);
+  a.act = reinterpret_cast<__nv_bfloat16*>(act);
+  a.kchunks = (cols / 16 + 3) / 4;
+  const int grid = sms() * 4;
+  if (gather) quant_rows_kernel<true><<<grid, 256, 0, (cudaStream_t)stream>>>(a);
+  else quant_rows_kernel<false><<<grid, 256, 0, (cudaStream_t)stream>>>(a);
+  return done(1);
+}
+
+nvfp4_status nvfp4_moe_gather_quantize(const void* x, int64_t ld_x, const int32_t* row_token, const int32_t* seg_off,
+                                       int groups, const float* tensor_scales, int64_t rows_cap, int64_t cols,
+                                       uint8_t* codes, uint8_t* scales_mma, void* xhat, void* stream) {
+  return quant_rows(true, x, nullptr, ld_x, row_token, seg_off, groups, tensor_scales, rows_cap, cols, codes,
+                    scales_mma, xhat, nullptr, stream);
+}
+
+nvfp4_status nvfp4_moe_swiglu_quantize(const void* h_gate, const void* h_up, int64_t ld_h, const int32_t* row_token,
+                                       const int32_t* seg_off, int groups, const float* tensor_scales, int64_t rows_cap,
+                                       int64_t cols, uint8_t* codes, uint8_t* scales_mma, void* ahat, void* act,
+                                       void* stream) {
+  return quant_rows(false, h_gate, h_up, ld_h, row_token, seg_off, groups, tensor_scales, rows_cap, cols, codes,
+                    scales_mma, ahat, act, stream);
+}
+
+nvfp4_status nvfp4_moe_combine(const void* y, int64_t cols, const int32_t* slot_row, const float* combine_weights,
+                               int tokens, int topk, const int32_t* seg_off, int experts, void* out, void* stream) {
+  if (cols < 8 || cols % 8 || tokens < 1 || topk < 1) return NVFP4_ERR_SHAPE;
+  if (!y || !slot_row || !combine_weights || !seg_off || !out) return NVFP4_ERR_ARG;
+  if (((uintptr_t)y & 15u) || ((uintptr_t)out & 15u)) return NVFP4_ERR_ALIGN;
+  combine_kernel<<<sms() * 8, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const __nv_bfloat16*>(y), (int)cols,
+                                                              slot_row, combine_weights, tokens, topk, seg_off, experts,
+                                                              reinterpret_cast<__nv_bfloat16*>(out));
+  return done(1);
+}
+
+nvfp4_status nvfp4_moe_scale_rows(const void* dy, int64_t cols, const int32_t* row_token, const float* row_weight,
+                                  const int32_t* seg_off, int groups, int64_t rows_cap, void* dyp, void* stream) {
+  if (cols < 8 || cols % 8 || rows_cap < 1 || groups < 1) return NVFP4_ERR_SHAPE;
+  if (!dy || !row_token || !row_weight || !seg_off || !dyp) return NVFP4_ERR_ARG;
+  if (((uintptr_t)dy & 15u) || ((uintptr_t)dyp & 15u)) return NVFP4_ERR_ALIGN;
+  scale_rows_kernel<<<sms() * 8, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const __nv_bfloat16*>(dy), (int)cols,
+                                                                 row_token, row_weight, seg_off, groups, (int)rows_cap,
+                                                                 reinterpret_cast<__nv_bfloat16*>(dyp));
+  return done(1);
+}
+
+nvfp4_status nvfp4_moe_swiglu_backward(const void* da, const void* h_gate, const void* h_up, int64_t cols,
+                                       const int32_t* row_token, const int32_t* seg_off, int groups, int64_t rows_cap,
+                                       void* dgu, void* stream) {
+  if (cols < 1 || rows_cap < 1 || groups < 1) return NVFP4_ERR_SHAPE;
+  if (!da || !h_gate || !h_up || !row_token || !seg_off || !dgu) return NVFP4_ERR_ARG;
+  swiglu_bwd_kernel<<<sms() * 8, 256, 0, (cudaStream_t)stream>>>(
+      reinterpret_cast<const __nv_bfloat16*>(da), reinterpret_cast<const __nv_bfloat16*>(h_gate),
+      reinterpret_cast<const __nv_bfloat16*>(h_up), (int)cols, row_token, seg_off, groups, (int)rows_cap,
+      reinterpret_cast<__nv_bfloat16*>(dgu));
+  return done(1);
+}
+
+nvfp4_status nvfp4_moe_gather_sum(const void* dxp, int64_t cols, const int32_t* slot_row, int tokens, int topk,
+                                  const int32_t* seg_off, int experts, void* dx, void* stream) {
+  if (cols < 8 || cols % 8 || tokens < 1 || topk < 1) return NVFP4_ERR_SHAPE;
+  if (!dxp || !slot_row || !seg_off || !dx) return NVFP4_ERR_ARG;
+  if (((uintptr_t)dxp & 15u) || ((uintptr_t)dx & 15u)) return NVFP4_ERR_ALIGN;
+  gather_sum_kernel<<<sms() * 8, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const __nv_bfloat16*>(dxp), (int)cols,
+                                                                 slot_row, tokens, topk, seg_off, experts,
+                                                                 reinterpret_cast<__nv_bfloat16*>(dx));
+  return done(1);
+}
+
+nvfp4_status nvfp4_moe_router_grad(const void* dy, const void* y, int64_t cols, const int32_t* slot_row, int tokens,
+                                   int topk, float* dw, void* stream) {
+  if (cols < 8 || cols % 8 || tokens < 1 || topk < 1) return NVFP4_ERR_SHAPE;
+  if (!dy || !y || !slot_row || !dw) return NVFP4_ERR_ARG;
+  if (((uintptr_t)dy & 15u) || ((uintptr_t)y & 15u)) return NVFP4_ERR_ALIGN;
+  router_grad_kernel<<<sms() * 8, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const __nv_bfloat16*>(dy),
+                                                                  reinterpret_cast<const __nv_bfloat16*>(y), (int)cols,
+                                                                  slot_row, tokens * topk, topk, dw);
+  return done(1);
+}
+
+nvfp4_status nvfp4_transpose_bf16(const void* in, int64_t ld_in, int64_t rows, int64_t cols, void* out, int64_t ld_out,
+                                  void* stream) {
+  if (rows < 1 || cols < 1 || ld_in < cols || ld_out < rows || rows > 0x7FFFFFFF || cols > 0x7FFFFFFF)
+    return NVFP4_ERR_SHAPE;
+  if (!in || !out) return NVFP4_ERR_ARG;
+  transpose_bf16_kernel<<<sms() * 16, dim3(32, 8), 0, (cudaStream_t)stream>>>(
+      reinterpret_cast<const __nv_bfloat16*>(in), ld_in, (int)rows, (int)cols, reinterpret_cast<__nv_bfloat16*>(out),
+      ld_out);
+  return done(1);
+}
+
+nvfp4_status nvfp4_dequantize_transpose(const uint8_t* codes, const uint8_t* block_scales, const float* tensor_scales,
+                                        int groups, int64_t rows_per_group, int64_t cols, void* out, int64_t ld_out,
+                                        int64_t col_off, void* stream) {
+  if (groups < 1 || rows_per_group < 1 || cols < 32 || cols % 32 || ld_out < col_off + rows_per_group ||
+      (int64_t)groups * rows_per_group > 0x7FFFFFFF)
+    return NVFP4_ERR_SHAPE;
+  if (!codes || !block_scales || !tensor_scales || !out) return NVFP4_ERR_ARG;
+  dequant_transpose_kernel<<<sms() * 16, dim3(32, 8), 0, (cudaStream_t)stream>>>(
+      codes, block_scales, tensor_scales, groups, (int)rows_per_group, (int)cols, reinterpret_cast<__nv_bfloat16*>(out),
+      ld_out, (int)col_off);
+  return done(1);
+}
+
+nvfp4_status nvfp4_scales_to_mma(const uint8_t* block_scales, int64_t rows, int64_t cols, uint8_t* out, void* stream) {
+  if (rows < 1 || cols < 16 || cols % 16) return NVFP4_ERR_SHAPE;
+  if (!block_scales || !out) return NVFP4_ERR_ARG;
+  scales_to_mma_kernel<<<sms() * 8, 256, 0, (cudaStream_t)stream>>>(block_scales, rows, cols, out);
+  return done(1);
+}
+
+}  // extern "C"

@@ -132,6 +132,16 @@ NVFP4_DEV void mma_fp4_block16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] x B[smem]^T, BF16 operands, FP32 accumulator (K = 16).
+NVFP4_DEV void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Copy 32 rows x 16 bytes of shared memory (described by `sdesc`) into
 // tensor memory at `taddr`, replicated into all four 32-lane subpartitions.
 NVFP4_DEV void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {

@@ -133,15 +133,35 @@ def distill_logits(seed: int = 0, device="cpu", rows: int = 16384, vocab: int = 
 
 
 def moe_layer(seed: int = 0, device="cpu", tokens: int = 4096, hidden: int = 2048, ffn: int = 1024,
-              experts: int = MOE_EXPERTS, topk: int = 6):
-    """One MoE layer: x [tokens, hidden]; per expert e (and the shared expert,
-    index `experts`) gate/up weights [ffn, hidden] and down weight
-    [hidden, ffn]; routing ids/weights; grad of the layer output."""
+              experts: int = MOE_EXPERTS, topk: int = 6, drift: float = 0.1, w_std: float = 0.02):
+    """One MoE layer step: x [tokens, hidden]; for every group g (routed
+    experts 0..experts-1, then the shared expert) gate/up weights
+    [ffn, hidden] and a down weight [hidden, ffn], stacked along dim 0;
+    routing ids/weights; the gradient dy of the layer output.
+
+    Frozen-scale inputs:
+      * w0_gate / w0_up / w0_down: the weights at calibration time (the
+        frozen weight scales are taken from them); the step's master weights
+        are w = w0 + N(0, drift * w_std), i.e. a student that has trained for a
+        while, so a few blocks leave their frozen range;
+      * x_ts, a_ts [experts + 1] fp32: seeded stand-ins for calibrated
+        activation tensor scales.  x_ts ~ U(1.49e-3, 1.86e-3) puts the largest
+        representable magnitude at 4 to 5 standard deviations of x ~ N(0, 1);
+        a_ts ~ U(0.9, 1.1) * 5.36e-3 * hidden * E[w^2], the same for the
+        SwiGLU output (about (4 sigma_h)^2 with sigma_h^2 = hidden * E[w^2])."""
     x = activations(tokens, hidden, seed, device)
     ids, cw = routing(tokens, experts, topk, seed + 1, device)
     n = experts + 1
-    w_gate = torch.stack([weights(ffn, hidden, seed + 10 + 3 * e, device) for e in range(n)])
-    w_up = torch.stack([weights(ffn, hidden, seed + 11 + 3 * e, device) for e in range(n)])
-    w_down = torch.stack([weights(hidden, ffn, seed + 12 + 3 * e, device) for e in range(n)])
-    dy = activations(tokens, hidden, seed + 2, device)
-    return {"x": x, "ids": ids, "combine": cw, "w_gate": w_gate, "w_up": w_up, "w_down": w_down, "dy": dy}
+    out = {"x": x, "ids": ids, "combine": cw, "dy": activations(tokens, hidden, seed + 2, device)}
+    for k, (rows, cols, off) in {"gate": (ffn, hidden, 10), "up": (ffn, hidden, 11),
+                                 "down": (hidden, ffn, 12)}.items():
+        w0 = torch.stack([weights(rows, cols, seed + off + 3 * e, device, std=w_std) for e in range(n)])
+        g = _gen(seed + 7 + off, device)
+        noise = torch.randn(w0.shape, generator=g, device=device, dtype=F32) * (drift * w_std)
+        out["w0_" + k] = w0
+        out["w_" + k] = (w0.to(F32) + noise).to(BF16)
+    g = _gen(seed + 5, device)
+    out["x_ts"] = (torch.rand(n, generator=g, device=device, dtype=F32) * (1.86e-3 - 1.49e-3) + 1.49e-3)
+    ew2 = w_std ** 2 * (1.0 - 0.001 + 0.001 * 50.0 ** 2)
+    out["a_ts"] = (torch.rand(n, generator=g, device=device, dtype=F32) * 0.2 + 0.9) * (5.36e-3 * hidden * ew2)
+    return out

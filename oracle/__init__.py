@@ -49,6 +49,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_e4m3_value.restype = c_d
         L.oracle_bf16_round.argtypes = [c_d]
         L.oracle_bf16_round.restype = ctypes.c_uint16
+        L.oracle_bf16_round_array.argtypes = [c_p, c_i64, c_p]
+        L.oracle_bf16_round_array.restype = None
         L.oracle_tensor_amax.argtypes = [c_p, c_i64, c_i64, c_i64]
         L.oracle_tensor_amax.restype = c_f
         L.oracle_global_scale_from_amax.argtypes = [c_f]
@@ -103,8 +105,14 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
 
 def bf16_round(x: np.ndarray) -> np.ndarray:
     """Round float64/float32 values to bf16 (RNE); returns uint16 bit patterns."""
-    f = np.vectorize(lambda v: lib().oracle_bf16_round(float(v)), otypes=[np.uint16])
-    return f(np.asarray(x, dtype=np.float64))
+    a = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(a.shape, dtype=np.uint16)
+    lib().oracle_bf16_round_array(_ptr(a), a.size, _ptr(out))
+    return out
+
+
+def bf16_round_scalar(v: float) -> int:
+    return int(lib().oracle_bf16_round(float(v)))
 
 
 # --------------------------------------------------------------------------

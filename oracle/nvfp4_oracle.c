@@ -176,6 +176,11 @@ uint16_t oracle_bf16_round(double x) {
   return h;
 }
 
+/* oracle_bf16_round over an array: out[i] = bf16 pattern of x[i]. */
+void oracle_bf16_round_array(const double* x, int64_t n, uint16_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_round(x[i]);
+}
+
 /* ------------------------------------------------------------------------ */
 /* Quantize / dequantize, [FMT] + [MODE].                                    */
 /* ------------------------------------------------------------------------ */

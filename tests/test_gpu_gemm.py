@@ -133,3 +133,51 @@ def test_matches_cublaslt_nvfp4():
     ref = ref * (ats * bts)
     err = float((ours - ref).norm() / ref.norm())
     assert err <= 2 * GEMM_RTOL, err
+
+
+def _grouped_case(rows, N, K, seed):
+    """Builds a grouped problem: segments padded to 128 rows, stacked B."""
+    groups = len(rows)
+    offs = [0]
+    for r in rows:
+        offs.append(offs[-1] + (r + 127) // 128 * 128)
+    total = max(offs[-1], 128)
+    xs = [S.activations(r, K, seed=seed + g, device=DEV) for g, r in enumerate(rows)]
+    ws = [S.weights(N, K, seed=seed + 100 + g, device=DEV) for g in range(groups)]
+    a_codes = torch.zeros(total, K // 2, dtype=torch.uint8, device=DEV)
+    a_sf = torch.zeros(Q.mma_scales_bytes(total, K), dtype=torch.uint8, device=DEV)
+    a_ts = torch.empty(groups, device=DEV)
+    kchunks = K // 64
+    for g, x in enumerate(xs):
+        if rows[g] == 0:
+            a_ts[g] = 1.0
+            continue
+        c, sf, ts = Q.nvfp4_quantize(x, layout=Q.SCALES_MMA)
+        a_codes[offs[g]:offs[g] + rows[g]] = c
+        seg = (offs[g + 1] - offs[g]) // 128 * kchunks * 512
+        a_sf[offs[g] // 128 * kchunks * 512: offs[g] // 128 * kchunks * 512 + sf.numel()] = sf
+        a_ts[g] = ts[0]
+    bc, bsf, bts = Q.nvfp4_quantize_grouped(ws, Q.DYNAMIC, layout=Q.SCALES_MMA)
+    b_codes = torch.cat(bc)
+    b_sf = torch.cat(bsf)
+    off_t = torch.tensor(offs, dtype=torch.int32, device=DEV)
+    rows_t = torch.tensor(rows, dtype=torch.int32, device=DEV)
+    return xs, ws, offs, a_codes, a_sf, a_ts, off_t, rows_t, b_codes, b_sf, bts
+
+
+@pytest.mark.parametrize("rows,N,K", [([200, 0, 128, 1, 300], 384, 512), ([192] * 7 + [4096], 1024, 2048)])
+def test_grouped_gemm_matches_oracle_per_group(rows, N, K):
+    xs, ws, offs, a_codes, a_sf, a_ts, off_t, rows_t, b_codes, b_sf, bts = _grouped_case(rows, N, K, seed=len(rows))
+    c = Q.nvfp4_gemm_w4a4_grouped(a_codes, a_sf, a_ts, off_t, rows_t, b_codes, b_sf, bts, N)
+    torch.cuda.synchronize()
+    assert Q.nvfp4_device_error()[0] == 0
+    for g, r in enumerate(rows):
+        if r == 0:
+            continue
+        ca, sa, ga = _oracle_operand(xs[g])
+        cb, sb, gb = _oracle_operand(ws[g])
+        sel = np.arange(r) if r <= 512 else np.sort(np.random.default_rng(g).choice(r, 256, replace=False))
+        ref = O.gemm_w4a4_rows(ca, sa, ga, cb, sb, gb, K, sel)
+        got = c[offs[g]:offs[g] + r][torch.as_tensor(sel, device=DEV)].double().cpu().numpy()
+        err = _rel_fro(got, _bf16_round(ref))
+        assert err <= GEMM_RTOL, (g, err)
