@@ -14,7 +14,10 @@ Also measured in the same run and reported under "gemm" and "kl":
   * W4A4 GEMM: activations M x 4096 (M = 8192 and 128) quantized on the fly,
     weights 4096 x 4096 pre-quantized, bf16 out -- TFLOP/s;
   * KL distillation loss + dLogits over 16384 x 131072 bf16 teacher/student
-    logits -- tokens/s and GB/s (6 B per logit).
+    logits -- tokens/s and GB/s (6 B per logit);
+  * the MoE layer step (config "moe_step"): 4096 tokens, 128 routed experts
+    + 1 shared, top-6, forward (grouped W4A4) + straight-through backward
+    (BF16) -- tokens/s and per-phase times.
 
 Timing: device time with CUDA events on the launching stream; the K timed
 steps are one CUDA-graph replay of K consecutive steps, bracketed by a
@@ -252,6 +255,7 @@ def run_ours(args, world, rank, local):
     if not args.no_secondary:
         secondary["gemm"] = bench_gemm(Q, dev, stream, P, max(3, min(K, 20)))
         secondary["kl"] = bench_kl(Q, dev, stream, P, max(3, min(K, 10)))
+        secondary["moe_step"] = bench_moe(Q, dev, stream, P, max(3, min(K, 10)))
     clocks = sampler.stop()
 
     cpu = None
@@ -415,6 +419,90 @@ def bench_kl(Q, dev, stream, P, K):
             "config": "teacher/student bf16 16384 x 131072, teacher N(0,3) + one +12 entry per row, student = teacher + N(0,1), T=1"}
 
 
+MOE_CONFIG = ("MoE layer step: 4096 tokens x hidden 2048 bf16 N(0,1), top-6 of 128 experts (uniform) + 1 shared, "
+              "expert FFN 2048->1024->2048 SwiGLU, NVFP4 W4A4 with frozen scales, grouped W4A4 GEMMs forward, "
+              "straight-through BF16 backward (dx, dW_gate/up/down, d combine)")
+
+
+def make_moe_step(Q, dev, tokens=4096, hidden=2048, ffn=1024, experts=128, topk=6, seed=0):
+    """Synthetic config-5 layer on the device with its frozen scales (from a
+    DYNAMIC quantization of the calibration weights) and the step object."""
+    from nvfp4_quantization_aware_b200 import synthetic as S
+    d = S.moe_layer(seed=seed, device=dev, tokens=tokens, hidden=hidden, ffn=ffn, experts=experts, topk=topk)
+    w = {}
+    for k in ("gate", "up", "down"):
+        w0 = d.pop("w0_" + k)
+        G, rows, cols = w0.shape
+        _, sbs, ts = Q.nvfp4_quantize_grouped([w0[g] for g in range(G)], Q.DYNAMIC)
+        sb = torch.cat(sbs).contiguous()
+        del w0, sbs
+        w["w_" + k] = d.pop("w_" + k).reshape(G * rows, cols).contiguous()
+        w[k + "_ts"], w[k + "_sb"] = ts, sb
+        w[k + "_sb_mma"] = Q.nvfp4_scales_to_mma(sb, G * rows, cols)
+    w["x_ts"], w["a_ts"] = d["x_ts"], d["a_ts"]
+    step = Q.MoeLayerStep(tokens, hidden, ffn, experts, topk, w)
+    return d, w, step
+
+
+def bench_moe(Q, dev, stream, P, K):
+    """The config-5 layer step (forward + backward), K steps in one graph
+    replay; per-phase times from events inside the graph."""
+    tokens, hidden, ffn, experts, topk = 4096, 2048, 1024, 128, 6
+    with torch.cuda.stream(stream):
+        d, w, step = make_moe_step(Q, dev, tokens, hidden, ffn, experts, topk)
+        x, ids, cw, dy = d["x"], d["ids"], d["combine"], d["dy"]
+        y = torch.empty_like(x)
+        G = experts + 1
+        dx = torch.empty_like(x)
+        dwg = torch.empty(G * ffn, hidden, dtype=torch.bfloat16, device=dev)
+        dwu = torch.empty_like(dwg)
+        dwd = torch.empty(G * hidden, ffn, dtype=torch.bfloat16, device=dev)
+        dcw = torch.empty(tokens, topk, dtype=torch.float32, device=dev)
+
+        def one():
+            step.forward(x, ids, cw, y=y)
+            step.backward(dy, dx=dx, dw_gate=dwg, dw_up=dwu, dw_down=dwd, d_combine=dcw)
+
+        for _ in range(3):
+            one()
+        stream.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(K)]
+        g = torch.cuda.CUDAGraph()
+        n0 = Q.nvfp4_launch_count()
+        with torch.cuda.graph(g, stream=stream):
+            for k in range(K):
+                evs[k][0].record(stream)
+                step.forward(x, ids, cw, y=y)
+                evs[k][1].record(stream)
+                step.backward(dy, dx=dx, dw_gate=dwg, dw_up=dwu, dw_down=dwd, d_combine=dcw)
+                evs[k][2].record(stream)
+        launches = Q.nvfp4_launch_count() - n0
+        g.replay()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        stream.synchronize()
+        st, word = Q.nvfp4_device_error()
+    del g
+    ms = e0.elapsed_time(e1) / K
+    fwd = statistics.mean(evs[k][0].elapsed_time(evs[k][1]) for k in range(K))
+    bwd = statistics.mean(evs[k][1].elapsed_time(evs[k][2]) for k in range(K))
+    rows = tokens * topk + tokens
+    f_flops = 6.0 * rows * hidden * ffn         # gate, up, down (W4A4)
+    b_flops = 12.0 * rows * hidden * ffn        # dA, dX (2F), dW x3 (BF16)
+    out = {"tokens_per_s": round(tokens / (ms * 1e-3), 1), "ms_per_step": round(ms, 4),
+           "forward_ms": round(fwd, 4), "backward_ms": round(bwd, 4),
+           "forward_fp4_tflops": round(f_flops / (fwd * 1e-3) / 1e12, 1),
+           "backward_bf16_tflops": round(b_flops / (bwd * 1e-3) / 1e12, 1),
+           "gpu_launches_per_step": int(launches // K), "device_error": [int(st), int(word)],
+           "config": MOE_CONFIG + "; inputs larger than L2 (weights 3.2 GB), no flush"}
+    del d, w, step, x, y, dx, dwg, dwu, dwd, dcw
+    torch.cuda.empty_cache()
+    return out
+
+
 def cpu_baseline(xs):
     """The oracle (as it stands) on the host cores: dynamic then frozen
     quantize of the 128 expert weights (268M elements; the lm_head is left out
@@ -490,6 +578,11 @@ def run_profile_case(case: str):
         b = Q.nvfp4_quantize(w, Q.DYNAMIC, layout=Q.SCALES_MMA)
         for _ in range(5):
             Q.nvfp4_gemm_w4a4(*a, *b)
+    elif case == "moe":
+        d, w, step = make_moe_step(Q, dev)
+        for _ in range(3):
+            step.forward(d["x"], d["ids"], d["combine"])
+            step.backward(d["dy"])
     elif case == "kl":
         d = S.distill_logits(seed=0, device=dev, rows=2048)  # 2 x 512 MiB
         for _ in range(5):
@@ -506,7 +599,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-secondary", action="store_true", help="skip the GEMM and KL measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["quant", "gemm", "kl"], default=None,
+    ap.add_argument("--profile", choices=["quant", "gemm", "kl", "moe"], default=None,
                     help="run one small single-kernel case (for ncu captures) and exit")
     args = ap.parse_args()
     if args.profile:

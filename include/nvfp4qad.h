@@ -199,6 +199,17 @@ nvfp4_status nvfp4_fake_quant_grouped(int num_tensors, const nvfp4_tensor_ref* t
                                       nvfp4_scale_mode mode, void* workspace, size_t workspace_bytes,
                                       void* stream);
 
+/* Quantize and fake-quantize in one pass: tensors[i].out receives the codes
+ * (as nvfp4_quantize_grouped) and y[i] the dequantized values (as
+ * nvfp4_fake_quant_grouped, same dtype as the input, row stride ld_y[i]
+ * elements); y and ld_y are HOST arrays of num_tensors entries.  For the
+ * weights of a layer whose forward runs on the codes and whose backward
+ * needs the dequantized weights. */
+nvfp4_status nvfp4_quantize_fake_quant_grouped(int num_tensors, const nvfp4_tensor_ref* tensors, void* const* y,
+                                               const int64_t* ld_y, nvfp4_dtype dtype, nvfp4_scale_mode mode,
+                                               nvfp4_scale_layout layout, void* workspace,
+                                               size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * Fake quantization: y = dequantize(quantize(x)) in one pass, the simulated
  * quantization every student forward pass goes through (Nemotron 3.5
@@ -294,29 +305,36 @@ nvfp4_status nvfp4_gemm_w4a4_grouped(int groups, const uint8_t* a_codes, const u
  * tensor memory, bf16 output RNE) for the straight-through backward of the
  * MoE layer, whose gradients are plain BF16 products with the dequantized
  * operands (Nemotron 3.5 Lightning article, "QAD的工作原理").  Always
- * C = A * B^T with A and B row-major and K their contiguous dimension.
+ * C = A * B^T.
  *
- *   mode 0 (M-segments)  a: a_rows x a_cols (a_rows % 128 == 0), the groups'
- *                        rows in segments [seg_off[g], seg_off[g] + seg_len[g])
- *                        with seg_off[g] % 128 == 0; b: b_rows x K, group g
- *                        uses rows [g N, (g+1) N); c: a_rows x N (ldc), only
- *                        the segments' valid rows written.  K % 64 == 0,
- *                        K <= a_cols, b_rows >= groups * N; M is ignored.
- *   mode 1 (K-segments)  a: a_rows x a_cols, b: b_rows x a_cols; group g
- *                        reduces over columns [seg_off[g], seg_off[g] +
- *                        seg_len[g]) (seg_off[g] % 64 == 0; columns up to the
- *                        next multiple of 64 are read and must hold zeros
- *                        or belong to no other term); c: groups * M x N, group
- *                        g in rows [g M, (g+1) M); M <= a_rows, N <= b_rows,
- *                        K is ignored.  A group with seg_len 0 writes zeros.
+ * Operand storage (row-major, a_rows x a_cols with row stride lda elements;
+ * b likewise):
+ *   *_mn_major = 0  K-major: element (i, k) of the operand at [i][k]
+ *   *_mn_major = 1  MN-major: element (i, k) at [k][i]
+ * (i is the M index for A, the N index for B.)
+ *
+ *   mode 0 (M-segments)  A's M range in segments [seg_off[g], seg_off[g] +
+ *                        seg_len[g]) with seg_off[g] % 128 == 0 and the M
+ *                        extent a multiple of 128; B of group g: N indices
+ *                        [g N, (g+1) N) (K-major) or K indices [g K, (g+1) K)
+ *                        (MN-major); c: M extent x N (ldc), only the
+ *                        segments' valid rows written.  K % 64 == 0; M is
+ *                        ignored.
+ *   mode 1 (K-segments)  group g reduces over K indices [seg_off[g],
+ *                        seg_off[g] + seg_len[g]) of A and B (seg_off[g] % 64
+ *                        == 0; K indices up to the next multiple of 64 are
+ *                        read and must hold zeros); c: groups * M x N, group g
+ *                        in rows [g M, (g+1) M); M <= A's M extent, N <= B's
+ *                        N extent, equal K extents; K is ignored.  A group
+ *                        with seg_len 0 writes zeros.
  *   seg_off, seg_len     device int32 arrays (groups + 1 and groups entries)
  * 1 <= groups <= 256; a, b 16-byte aligned, lda * 2 and ldb * 2 multiples of
  * 16; c 4-byte aligned.
  * ------------------------------------------------------------------------ */
-nvfp4_status nvfp4_gemm_bf16_grouped(int mode, int groups, const void* a, int64_t a_rows, int64_t a_cols,
-                                     int64_t lda, const void* b, int64_t b_rows, int64_t ldb,
-                                     const int32_t* seg_off, const int32_t* seg_len, int64_t M, int64_t N,
-                                     int64_t K, void* c, int64_t ldc, void* stream);
+nvfp4_status nvfp4_gemm_bf16_grouped(int mode, int groups, const void* a, int a_mn_major, int64_t a_rows,
+                                     int64_t a_cols, int64_t lda, const void* b, int b_mn_major, int64_t b_rows,
+                                     int64_t b_cols, int64_t ldb, const int32_t* seg_off, const int32_t* seg_len,
+                                     int64_t M, int64_t N, int64_t K, void* c, int64_t ldc, void* stream);
 
 /* ------------------------------------------------------------------------
  * MoE layer of the QAD student: 128 routed experts plus one shared expert,
@@ -404,18 +422,6 @@ nvfp4_status nvfp4_moe_gather_sum(const void* dxp, int64_t cols, const int32_t* 
 nvfp4_status nvfp4_moe_router_grad(const void* dy, const void* y, int64_t cols, const int32_t* slot_row, int tokens,
                                    int topk, float* d_combine, void* stream);
 
-/* out[c][r] = in[r][c] for bf16 rows x cols (strides in elements). */
-nvfp4_status nvfp4_transpose_bf16(const void* in, int64_t ld_in, int64_t rows, int64_t cols, void* out,
-                                  int64_t ld_out, void* stream);
-
-/* Dequantized transpose of `groups` stacked NVFP4 tensors of rows_per_group x
- * cols (codes contiguous, ROWMAJOR block scales, tensor_scales[g]):
- *   out[g cols + c][col_off + r] = bf16(value(q[g][r][c]) * (s_b * s_g)).
- * cols % 32 == 0; out bf16 with row stride ld_out >= col_off + rows_per_group. */
-nvfp4_status nvfp4_dequantize_transpose(const uint8_t* codes, const uint8_t* block_scales,
-                                        const float* tensor_scales, int groups, int64_t rows_per_group,
-                                        int64_t cols, void* out, int64_t ld_out, int64_t col_off, void* stream);
-
 /* ROWMAJOR block scales of rows x cols -> the MMA layout (padding 0). */
 nvfp4_status nvfp4_scales_to_mma(const uint8_t* block_scales, int64_t rows, int64_t cols, uint8_t* out,
                                  void* stream);
@@ -472,15 +478,11 @@ enum qad_moe_buffer {
   QAD_MOE_ACT,          /* bf16 [R x F] (0 bytes unless save_act) */
   QAD_MOE_Y_ROWS,       /* bf16 [R x H] */
   QAD_MOE_DY_ROWS,      /* bf16 [R x H] */
-  QAD_MOE_WD_T,         /* bf16 [(E+1) F x H] */
+  QAD_MOE_WD_HAT,       /* bf16 [(E+1) H x F]: dequantized W_down (bf16 fake-quant) */
   QAD_MOE_DA,           /* bf16 [R x F] */
   QAD_MOE_DGU,          /* bf16 [R x 2F] */
-  QAD_MOE_WGU_T,        /* bf16 [(E+1) H x 2F] */
+  QAD_MOE_WGU_HAT,      /* bf16 [(E+1) 2F x H]: dequantized W_gate / W_up of group g in rows 2gF.. / 2gF+F.. */
   QAD_MOE_DX_ROWS,      /* bf16 [R x H] */
-  QAD_MOE_DY_ROWS_T,    /* bf16 [H x R] */
-  QAD_MOE_A_HAT_T,      /* bf16 [F x R] */
-  QAD_MOE_DGU_T,        /* bf16 [2F x R] */
-  QAD_MOE_X_HAT_T,      /* bf16 [H x R] */
   QAD_MOE_NUM_BUFFERS
 };
 

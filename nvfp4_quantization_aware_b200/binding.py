@@ -66,15 +66,11 @@ MOE_BUFFERS = {
     "act": (16, torch.bfloat16, lambda T, H, F, G, k, R: (R, F)),
     "y_rows": (17, torch.bfloat16, lambda T, H, F, G, k, R: (R, H)),
     "dy_rows": (18, torch.bfloat16, lambda T, H, F, G, k, R: (R, H)),
-    "wd_t": (19, torch.bfloat16, lambda T, H, F, G, k, R: (G * F, H)),
+    "wd_hat": (19, torch.bfloat16, lambda T, H, F, G, k, R: (G * H, F)),
     "da": (20, torch.bfloat16, lambda T, H, F, G, k, R: (R, F)),
     "dgu": (21, torch.bfloat16, lambda T, H, F, G, k, R: (R, 2 * F)),
-    "wgu_t": (22, torch.bfloat16, lambda T, H, F, G, k, R: (G * H, 2 * F)),
+    "wgu_hat": (22, torch.bfloat16, lambda T, H, F, G, k, R: (G * 2 * F, H)),
     "dx_rows": (23, torch.bfloat16, lambda T, H, F, G, k, R: (R, H)),
-    "dy_rows_t": (24, torch.bfloat16, lambda T, H, F, G, k, R: (H, R)),
-    "a_hat_t": (25, torch.bfloat16, lambda T, H, F, G, k, R: (F, R)),
-    "dgu_t": (26, torch.bfloat16, lambda T, H, F, G, k, R: (2 * F, R)),
-    "x_hat_t": (27, torch.bfloat16, lambda T, H, F, G, k, R: (H, R)),
 }
 
 
@@ -123,6 +119,9 @@ def lib() -> ctypes.CDLL:
     L.nvfp4_quantize_grouped.argtypes = [i32, ctypes.POINTER(TensorRef), i32, i32, i32, p, sz, p]
     L.nvfp4_quantize_grouped.restype = i32
     L.nvfp4_fake_quant_grouped.argtypes = [i32, ctypes.POINTER(TensorRef), i32, i32, p, sz, p]
+    L.nvfp4_quantize_fake_quant_grouped.argtypes = [i32, ctypes.POINTER(TensorRef), ctypes.POINTER(p),
+                                                    ctypes.POINTER(i64), i32, i32, i32, p, sz, p]
+    L.nvfp4_quantize_fake_quant_grouped.restype = i32
     L.nvfp4_fake_quant_grouped.restype = i32
     L.nvfp4_selftest_division.argtypes = [p, p, p]
     L.nvfp4_selftest_division.restype = i32
@@ -132,7 +131,8 @@ def lib() -> ctypes.CDLL:
     L.nvfp4_gemm_w4a4.restype = i32
     L.nvfp4_gemm_w4a4_grouped.argtypes = [i32, p, p, p, i64, p, p, p, p, p, i64, i64, p, i64, p, sz, p]
     L.nvfp4_gemm_w4a4_grouped.restype = i32
-    L.nvfp4_gemm_bf16_grouped.argtypes = [i32, i32, p, i64, i64, i64, p, i64, i64, p, p, i64, i64, i64, p, i64, p]
+    L.nvfp4_gemm_bf16_grouped.argtypes = [i32, i32, p, i32, i64, i64, i64, p, i32, i64, i64, i64, p, p, i64, i64,
+                                          i64, p, i64, p]
     L.nvfp4_gemm_bf16_grouped.restype = i32
     L.qad_kl_workspace_size.argtypes = [i64, i64, i32]
     L.qad_kl_workspace_size.restype = sz
@@ -157,10 +157,6 @@ def lib() -> ctypes.CDLL:
     L.nvfp4_moe_gather_sum.restype = i32
     L.nvfp4_moe_router_grad.argtypes = [p, p, i64, p, i32, i32, p, p]
     L.nvfp4_moe_router_grad.restype = i32
-    L.nvfp4_transpose_bf16.argtypes = [p, i64, i64, i64, p, i64, p]
-    L.nvfp4_transpose_bf16.restype = i32
-    L.nvfp4_dequantize_transpose.argtypes = [p, p, p, i32, i64, i64, p, i64, i64, p]
-    L.nvfp4_dequantize_transpose.restype = i32
     L.nvfp4_scales_to_mma.argtypes = [p, i64, i64, p, p]
     L.nvfp4_scales_to_mma.restype = i32
     shp, wts = ctypes.POINTER(MoeShape), ctypes.POINTER(MoeWeights)
@@ -344,6 +340,31 @@ def nvfp4_fake_quant_grouped(xs, mode: int = DYNAMIC, tensor_scales=None, block_
     return outs
 
 
+def nvfp4_quantize_fake_quant_grouped(xs, mode: int, tensor_scales, block_scales, codes=None, ys=None,
+                                      workspace: torch.Tensor | None = None):
+    """Codes (ROWMAJOR block scales) and fake-quant values of a list of
+    tensors in one pass; returns (codes list, ys list)."""
+    L = lib()
+    n = len(xs)
+    dev = xs[0].device
+    dt = _dtype_code(xs[0])
+    ts_list = [tensor_scales[i:i + 1] for i in range(n)] if isinstance(tensor_scales, torch.Tensor) else list(tensor_scales)
+    if codes is None:
+        codes = [torch.empty(x.shape[0], x.shape[1] // 2, dtype=torch.uint8, device=dev) for x in xs]
+    if ys is None:
+        ys = [torch.empty_like(x) for x in xs]
+    arr = _refs(xs, ts_list, block_scales, codes)
+    yp = (ctypes.c_void_p * n)(*[y.data_ptr() for y in ys])
+    ld = (ctypes.c_int64 * n)(*[y.stride(0) for y in ys])
+    need = int(L.nvfp4_grouped_workspace_size(mode))
+    if workspace is None:
+        workspace = _workspace(need, dev)
+    st = L.nvfp4_quantize_fake_quant_grouped(n, arr, yp, ld, dt, mode, SCALES_ROWMAJOR, _ptr(workspace),
+                                             0 if workspace is None else workspace.numel(), _stream(dev))
+    _check(st, "nvfp4_quantize_fake_quant_grouped")
+    return codes, ys
+
+
 def nvfp4_fake_quant(x: torch.Tensor, mode: int = DYNAMIC, tensor_scale: torch.Tensor | None = None,
                      block_scales: torch.Tensor | None = None, out: torch.Tensor | None = None,
                      return_scales: bool = False, workspace: torch.Tensor | None = None):
@@ -486,20 +507,23 @@ def qad_kl_fwd_bwd(teacher: torch.Tensor, student: torch.Tensor, temperature: fl
 # ------------------------------------------------------------------ BF16 grouped GEMM
 
 def nvfp4_gemm_bf16_grouped(mode: int, a: torch.Tensor, b: torch.Tensor, seg_off: torch.Tensor,
-                            seg_len: torch.Tensor, M: int, N: int, K: int, out: torch.Tensor | None = None):
-    """C = A B^T per group, bf16.  mode 0: A rows in 128-aligned segments, B of
-    group g = rows [g N, (g+1) N); mode 1: group g reduces over columns
+                            seg_len: torch.Tensor, M: int, N: int, K: int, out: torch.Tensor | None = None,
+                            a_mn_major: bool = False, b_mn_major: bool = False):
+    """C = A B^T per group, bf16.  An operand is K-major (stored rows x K) or
+    MN-major (stored K x rows).  mode 0: A's M range in 128-aligned segments,
+    B of group g = N indices [g N, (g+1) N) (K-major) or K indices
+    [g K, (g+1) K) (MN-major); mode 1: group g reduces over K indices
     [seg_off[g], seg_off[g] + seg_len[g]), C of group g = rows [g M, (g+1) M)."""
     _cuda2d(a, "a")
     _cuda2d(b, "b")
     groups = seg_len.numel()
     dev = a.device
     if out is None:
-        rows = a.shape[0] if mode == 0 else groups * M
+        rows = (a.shape[1] if a_mn_major else a.shape[0]) if mode == 0 else groups * M
         out = torch.empty(rows, N, dtype=torch.bfloat16, device=dev)
-    st = lib().nvfp4_gemm_bf16_grouped(mode, groups, _ptr(a), a.shape[0], a.shape[1], a.stride(0), _ptr(b),
-                                       b.shape[0], b.stride(0), _ptr(seg_off), _ptr(seg_len), M, N, K, _ptr(out),
-                                       out.stride(0), _stream(dev))
+    st = lib().nvfp4_gemm_bf16_grouped(mode, groups, _ptr(a), int(a_mn_major), a.shape[0], a.shape[1], a.stride(0),
+                                       _ptr(b), int(b_mn_major), b.shape[0], b.shape[1], b.stride(0), _ptr(seg_off),
+                                       _ptr(seg_len), M, N, K, _ptr(out), out.stride(0), _stream(dev))
     _check(st, "nvfp4_gemm_bf16_grouped")
     return out
 
@@ -509,29 +533,6 @@ def nvfp4_scales_to_mma(block_scales: torch.Tensor, rows: int, cols: int) -> tor
     out = torch.empty(mma_scales_bytes(rows, cols), dtype=torch.uint8, device=block_scales.device)
     st = lib().nvfp4_scales_to_mma(_ptr(block_scales), rows, cols, _ptr(out), _stream(block_scales.device))
     _check(st, "nvfp4_scales_to_mma")
-    return out
-
-
-def nvfp4_transpose_bf16(x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
-    _cuda2d(x, "x")
-    rows, cols = x.shape
-    if out is None:
-        out = torch.empty(cols, rows, dtype=torch.bfloat16, device=x.device)
-    st = lib().nvfp4_transpose_bf16(_ptr(x), x.stride(0), rows, cols, _ptr(out), out.stride(0), _stream(x.device))
-    _check(st, "nvfp4_transpose_bf16")
-    return out
-
-
-def nvfp4_dequantize_transpose(codes: torch.Tensor, block_scales: torch.Tensor, tensor_scales: torch.Tensor,
-                               groups: int, rows_per_group: int, cols: int, out: torch.Tensor | None = None,
-                               col_off: int = 0) -> torch.Tensor:
-    """out[g cols + c, col_off + r] = bf16 dequantized element (g, r, c) of the stack."""
-    dev = codes.device
-    if out is None:
-        out = torch.empty(groups * cols, rows_per_group, dtype=torch.bfloat16, device=dev)
-    st = lib().nvfp4_dequantize_transpose(_ptr(codes), _ptr(block_scales), _ptr(tensor_scales), groups,
-                                          rows_per_group, cols, _ptr(out), out.stride(0), col_off, _stream(dev))
-    _check(st, "nvfp4_dequantize_transpose")
     return out
 
 

@@ -6,17 +6,24 @@
 // "QAD的工作原理": the quantized student is trained through simulated
 // quantization).
 //
-// C = A * B^T with A [rows][K] and B [cols][K] both K-major (the contiguous
-// dimension is the reduction), bf16 in, bf16 out.  Two ways to group:
+// C = A * B^T, bf16 in, bf16 out.  Each operand is either K-major (stored
+// rows x K, K contiguous) or MN-major (stored K x rows, its M or N index
+// contiguous), so that every backward product reads the forward's tensors
+// in the layout they already have: no transposes.
+//
+// Two ways to group:
 //   M-segments  group g owns rows [off[g], off[g] + len[g]) of A and C (off a
-//               multiple of 128), B of group g is rows [g N, (g+1) N) of B.
-//               Used for dA = dY W_down and dX = dGU [W_gate; W_up].
-//   K-segments  group g reduces over columns [off[g], off[g] + len[g]) of A
-//               and B (the group's tokens; off and the padded length are
-//               multiples of 64, padding holds zeros); C of group g is rows
-//               [g M, (g+1) M).  Used for the weight gradients dW = dY^T A.
-// Persistent CTAs, 128 x 256 tiles, 4-stage TMA ring (128-byte swizzle),
-// 8 epilogue warps, every wait bounded.
+//               multiple of 128); B of group g is the g-th block of B along
+//               its N (K-major B: N rows each) or K (MN-major B: K rows each)
+//               dimension.  Used for dA = dY W^_down and
+//               dX = [dG | dU] [W^_gate; W^_up].
+//   K-segments  group g reduces over K indices [off[g], off[g] + len[g]) of A
+//               and B (the group's tokens; off a multiple of 64, padding
+//               holds zeros); C of group g is rows [g M, (g+1) M).  Used for
+//               the weight gradients dW = dY^T A^.
+// Persistent CTAs (one per SM), 128 x 256 tiles, 4-stage TMA ring (128-byte
+// swizzle), two accumulators in tensor memory so that the epilogue of one
+// tile overlaps the MMAs of the next, 8 epilogue warps, every wait bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -27,24 +34,31 @@ namespace nvfp4 {
 namespace bf16gemm {
 
 constexpr int BM = 128, BN = 256;
-constexpr int BK = 64;                    // bf16 elements per stage = 128 bytes per row
+constexpr int BK = 64;                    // K per stage: 64 bf16 = 128 bytes
 constexpr int KB = BK / 16;               // MMAs (K = 16) per stage
 constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;      // 16 KiB
 constexpr int B_BYTES = BN * BK * 2;      // 32 KiB
+constexpr int MN_ATOM_BYTES = BK * 128;   // MN-major: one 64-wide column block of a stage
 constexpr int MAX_GROUPS = 256;
 constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES) + 1024 + 256 + (2 * MAX_GROUPS + 1) * 4;
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
-constexpr int TM_COLS = 256;
-// BF16 x BF16 -> F32 (c_format 1 in bits 4-5, a/b format 1 in bits 7-9 / 10-12),
-// K-major A and B, N >> 3 in bits 17-22, M >> 4 in bits 24-28.
-constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+constexpr int ACC_COLS = BN;              // FP32 accumulator columns per tile
+constexpr int TM_COLS = 2 * ACC_COLS;     // two accumulators
+
+// BF16 x BF16 -> F32: c_format 1 (bits 4-5), a/b format 1 (bits 7-9, 10-12),
+// A / B MN-major flags (bits 15, 16), N >> 3 (bits 17-22), M >> 4 (bits 24-28).
+template <bool A_MN, bool B_MN>
+constexpr uint32_t idesc() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((A_MN ? 1u : 0u) << 15) | ((B_MN ? 1u : 0u) << 16) |
+         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
 
 struct Params {
   __nv_bfloat16* c;
   int64_t ldc;
-  int M, N, K;            // M: rows of A (M-segments: padded total); K: reduction (M-segments)
+  int M, N, K;            // M: rows of C per group (K-segments); K: reduction length (M-segments)
   int mode;               // 0 = M-segments, 1 = K-segments
   int groups;
   const int32_t* off;     // device [groups + 1]
@@ -53,11 +67,14 @@ struct Params {
 };
 
 struct Tile {
-  int g, m0, n0, a_row, b_row, c_row0, row_end;
-  int k0, nk;             // first K column and number of K stages
+  int m0, n0;
+  int a_mn, a_k, b_mn, b_k;   // operand coordinates of the first stage (MN index, K index)
+  int c_row0, row_end;
+  int nk;                     // K stages
   bool empty;
 };
 
+template <bool B_MN>
 NVFP4_DEV Tile tile_of(int t, const Params& p, const int32_t* s_off, const int32_t* s_len, int num_n, int num_m) {
   Tile tl;
   if (p.mode == 0) {
@@ -70,32 +87,55 @@ NVFP4_DEV Tile tile_of(int t, const Params& p, const int32_t* s_off, const int32
       if (s_off[mid] <= tl.m0) lo = mid;
       else hi = mid - 1;
     }
-    tl.g = lo;
-    tl.a_row = tl.m0;
-    tl.b_row = lo * p.N + tl.n0;
+    tl.a_mn = tl.m0;
+    tl.a_k = 0;
+    tl.b_mn = B_MN ? tl.n0 : lo * p.N + tl.n0;
+    tl.b_k = B_MN ? lo * p.K : 0;
     tl.c_row0 = 0;
     tl.row_end = s_off[lo] + s_len[lo];
-    tl.k0 = 0;
     tl.nk = (p.K + BK - 1) / BK;
     tl.empty = tl.m0 >= tl.row_end;
   } else {
     const int per_g = num_m * num_n;
-    tl.g = t / per_g;
-    const int r = t - tl.g * per_g;
+    const int g = t / per_g;
+    const int r = t - g * per_g;
     const int mt = r / num_n;
     tl.m0 = mt * BM;
     tl.n0 = (r - mt * num_n) * BN;
-    tl.a_row = tl.m0;
-    tl.b_row = tl.n0;
-    tl.c_row0 = tl.g * p.M;
+    tl.a_mn = tl.m0;
+    tl.b_mn = tl.n0;
+    tl.a_k = tl.b_k = s_off[g];
+    tl.c_row0 = g * p.M;
     tl.row_end = p.M;
-    tl.k0 = s_off[tl.g];
-    tl.nk = (s_len[tl.g] + BK - 1) / BK;
+    tl.nk = (s_len[g] + BK - 1) / BK;
     tl.empty = false;  // an empty segment still writes its zero gradient
   }
   return tl;
 }
 
+// One stage of one operand: ROWS (M or N) x 64 (K) elements into `dst`.
+template <bool MN, int ROWS>
+NVFP4_DEV void load_operand(uint8_t* dst, const CUtensorMap* map, int mn, int k, uint64_t* bar) {
+  if (MN) {
+#pragma unroll
+    for (int j = 0; j < ROWS / 64; ++j) tma_load_2d(dst + j * MN_ATOM_BYTES, map, mn + 64 * j, k, bar);
+  } else {
+    tma_load_2d(dst, map, k, mn, bar);
+  }
+}
+
+// Shared-memory descriptor of K step kb (16 elements) of one operand stage.
+//   K-major:  rows of 128 bytes (8-row swizzle atoms, 1024 bytes apart); the
+//             K step moves 32 bytes along the swizzled row.
+//   MN-major: 64-wide column blocks of BK rows x 128 bytes (MN_ATOM_BYTES
+//             apart: the leading-dimension offset); 8-row atoms 1024 bytes
+//             apart along K (the stride offset); the K step moves 16 rows.
+template <bool MN>
+NVFP4_DEV uint64_t operand_desc(uint32_t base, int kb) {
+  return MN ? smem_desc(base + kb * 16 * 128, MN_ATOM_BYTES, 1024, 2) : smem_desc(base + kb * 32, 16, 1024, 2);
+}
+
+template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -105,9 +145,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* sB = sA + STAGES * A_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
   uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;
-  uint64_t* acc_empty = acc_full + 1;
-  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  uint64_t* acc_full = empty + STAGES;     // [2]
+  uint64_t* acc_empty = acc_full + 2;      // [2]
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
   int32_t* s_off = reinterpret_cast<int32_t*>(smem + STAGES * (A_BYTES + B_BYTES) + 256);
   int32_t* s_len = s_off + MAX_GROUPS + 1;
@@ -124,8 +164,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, EPI_WARPS);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], EPI_WARPS);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -147,7 +189,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       int it = 0;
       for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
-        const Tile tl = tile_of(t, p, s_off, s_len, num_n, num_m);
+        const Tile tl = tile_of<B_MN>(t, p, s_off, s_len, num_n, num_m);
         if (tl.empty) continue;
         for (int kt = 0; kt < tl.nk; ++kt, ++it) {
           const int s = it % STAGES;
@@ -155,8 +197,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (!mbar_wait_bounded(&empty[s], ph ^ 1u)) { *abort_flag = 1; break; }
           if (*abort_flag) break;
           mbar_expect_tx(&full[s], (uint32_t)(A_BYTES + B_BYTES));
-          tma_load_2d(sA + s * A_BYTES, &tmA, tl.k0 + kt * BK, tl.a_row, &full[s]);
-          tma_load_2d(sB + s * B_BYTES, &tmB, tl.k0 + kt * BK, tl.b_row, &full[s]);
+          load_operand<A_MN, BM>(sA + s * A_BYTES, &tmA, tl.a_mn, tl.a_k + kt * BK, &full[s]);
+          load_operand<B_MN, BN>(sB + s * B_BYTES, &tmB, tl.b_mn, tl.b_k + kt * BK, &full[s]);
         }
       }
     }
@@ -164,10 +206,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       int it = 0, ti = 0;
       for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
-        const Tile tl = tile_of(t, p, s_off, s_len, num_n, num_m);
+        const Tile tl = tile_of<B_MN>(t, p, s_off, s_len, num_n, num_m);
         if (tl.empty) continue;
-        if (!mbar_wait_bounded(acc_empty, ((uint32_t)ti & 1u) ^ 1u)) { *abort_flag = 1; break; }
+        const int buf = ti & 1;
+        if (!mbar_wait_bounded(&acc_empty[buf], ((uint32_t)(ti >> 1) & 1u) ^ 1u)) { *abort_flag = 1; break; }
         tc_fence_after();
+        const uint32_t acc = tmem + (uint32_t)(buf * ACC_COLS);
         for (int kt = 0; kt < tl.nk; ++kt, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -177,28 +221,26 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t a_base = smem_u32(sA + s * A_BYTES);
           const uint32_t b_base = smem_u32(sB + s * B_BYTES);
 #pragma unroll
-          for (int kb = 0; kb < KB; ++kb) {
-            // K = 16 bf16 = 32 bytes further along the 128-byte swizzled row
-            const uint64_t ad = smem_desc(a_base + kb * 32, 16, 1024, 2);
-            const uint64_t bd = smem_desc(b_base + kb * 32, 16, 1024, 2);
-            mma_bf16(tmem, ad, bd, IDESC, (kt > 0 || kb > 0) ? 1u : 0u);
-          }
+          for (int kb = 0; kb < KB; ++kb)
+            mma_bf16(acc, operand_desc<A_MN>(a_base, kb), operand_desc<B_MN>(b_base, kb), idesc<A_MN, B_MN>(),
+                     (kt > 0 || kb > 0) ? 1u : 0u);
           tc_commit(&empty[s]);
         }
-        tc_commit(acc_full);
+        tc_commit(&acc_full[buf]);
         ++ti;
       }
     }
   } else {
-    const int sub = warp & 3;
+    const int sub = warp & 3;                      // TMEM lanes 32 sub .. 32 sub + 31
     const int cbase = ((warp - 2) >> 2) * (BN / 2);
     constexpr int HALF = BN / 2;
     int ti = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-      const Tile tl = tile_of(t, p, s_off, s_len, num_n, num_m);
+      const Tile tl = tile_of<B_MN>(t, p, s_off, s_len, num_n, num_m);
       if (tl.empty) continue;
-      const int par_ti = ti++;
-      const bool ok = mbar_wait_bounded(acc_full, (uint32_t)par_ti & 1u);
+      const int buf = ti & 1;
+      const bool ok = mbar_wait_bounded(&acc_full[buf], (uint32_t)(ti >> 1) & 1u);
+      ++ti;
       if (!ok) *abort_flag = 1;
       if (!ok || *abort_flag) break;
       tc_fence_after();
@@ -206,22 +248,21 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int c0 = 0; c0 < HALF; c0 += 64) {
         uint32_t r0[32], r1[32];
-        const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + cbase + c0;
+        const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + (uint32_t)(buf * ACC_COLS) + cbase + c0;
         tmem_ld_32x32b_x32(taddr, r0);
         tmem_ld_32x32b_x32(taddr + 32, r1);
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           // a K-segment of length 0 issued no MMA: its gradient is zero
-          const float f0 = tl.nk > 0 ? __uint_as_float(r0[2 * j]) : 0.f, f1 = tl.nk > 0 ? __uint_as_float(r0[2 * j + 1]) : 0.f;
-          const float g0 = tl.nk > 0 ? __uint_as_float(r1[2 * j]) : 0.f, g1 = tl.nk > 0 ? __uint_as_float(r1[2 * j + 1]) : 0.f;
-          packed[c0 / 2 + j] = pack_bf16x2(f0, f1);
-          packed[c0 / 2 + 16 + j] = pack_bf16x2(g0, g1);
+          const bool z = tl.nk == 0;
+          packed[c0 / 2 + j] = z ? 0u : pack_bf16x2(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1]));
+          packed[c0 / 2 + 16 + j] = z ? 0u : pack_bf16x2(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1]));
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
       const int row = tl.m0 + sub * 32 + lane;
       if (row < tl.row_end) {
         __nv_bfloat16* crow = p.c + ((int64_t)tl.c_row0 + row) * p.ldc;
@@ -268,7 +309,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // bf16 matrix [rows][cols] with row stride ld elements -> tensor map with a
-// box of box_rows x 64 elements (128 bytes), 128-byte swizzle, zero fill.
+// box of box_rows x 64 columns (128 bytes), 128-byte swizzle, zero fill.
 static bool tmap_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
   auto enc = encode_fn();
   if (!enc) return false;
@@ -281,33 +322,63 @@ static bool tmap_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t co
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <bool A_MN, bool B_MN>
+static nvfp4_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, cudaStream_t s) {
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(gemm_bf16_kernel<A_MN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    attr = true;
+  }
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  gemm_bf16_kernel<A_MN, B_MN><<<sms, THREADS, SMEM_BYTES, s>>>(ta, tb, p);
+  count_launches(1);
+  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
 }  // namespace bf16gemm
 }  // namespace nvfp4
 
 using namespace nvfp4;
 
-extern "C" nvfp4_status nvfp4_gemm_bf16_grouped(int mode, int groups, const void* a, int64_t a_rows, int64_t a_cols,
-                                                int64_t lda, const void* b, int64_t b_rows, int64_t ldb,
-                                                const int32_t* seg_off, const int32_t* seg_len, int64_t M,
-                                                int64_t N, int64_t K, void* c, int64_t ldc, void* stream) {
+extern "C" nvfp4_status nvfp4_gemm_bf16_grouped(int mode, int groups, const void* a, int a_mn_major, int64_t a_rows,
+                                                int64_t a_cols, int64_t lda, const void* b, int b_mn_major,
+                                                int64_t b_rows, int64_t b_cols, int64_t ldb, const int32_t* seg_off,
+                                                const int32_t* seg_len, int64_t M, int64_t N, int64_t K, void* c,
+                                                int64_t ldc, void* stream) {
   using namespace bf16gemm;
   if (mode != 0 && mode != 1) return NVFP4_ERR_ARG;
+  if ((a_mn_major != 0 && a_mn_major != 1) || (b_mn_major != 0 && b_mn_major != 1)) return NVFP4_ERR_ARG;
   if (groups < 1 || groups > MAX_GROUPS) return NVFP4_ERR_SHAPE;
   if (!a || !b || !seg_off || !seg_len || !c) return NVFP4_ERR_ARG;
-  if (a_rows < 1 || a_cols < 1 || b_rows < 1 || lda < a_cols || ldb < a_cols || N < 1 || ldc < N) return NVFP4_ERR_SHAPE;
-  if (mode == 0 && (K < 64 || K % 64 != 0 || K > a_cols || a_rows % 128 != 0 || b_rows < (int64_t)groups * N))
+  if (a_rows < 1 || a_cols < 1 || b_rows < 1 || b_cols < 1 || lda < a_cols || ldb < b_cols || N < 1 || ldc < N)
     return NVFP4_ERR_SHAPE;
-  if (mode == 1 && (M < 1 || M > a_rows || N > b_rows)) return NVFP4_ERR_SHAPE;
-  if (a_rows > 0x7FFFFFFF || b_rows > 0x7FFFFFFF || a_cols > 0x7FFFFFFF || (int64_t)groups * M > 0x7FFFFFFF)
+  if (a_rows > 0x7FFFFFFF || a_cols > 0x7FFFFFFF || b_rows > 0x7FFFFFFF || b_cols > 0x7FFFFFFF)
     return NVFP4_ERR_SHAPE;
+  // stored extents: K-major operands are (rows = M or N index, cols = K), MN-major (rows = K, cols = M or N)
+  const int64_t a_m = a_mn_major ? a_cols : a_rows, a_k = a_mn_major ? a_rows : a_cols;
+  const int64_t b_n = b_mn_major ? b_cols : b_rows, b_k = b_mn_major ? b_rows : b_cols;
+  if (mode == 0) {
+    if (K < 64 || K % 64 != 0 || K > a_k || a_m % 128 != 0) return NVFP4_ERR_SHAPE;
+    if (b_mn_major ? (b_k < (int64_t)groups * K || b_n < N) : (b_n < (int64_t)groups * N || b_k < K))
+      return NVFP4_ERR_SHAPE;
+    if ((int64_t)groups * K > 0x7FFFFFFF || (int64_t)groups * N > 0x7FFFFFFF) return NVFP4_ERR_SHAPE;
+  } else {
+    if (M < 1 || M > a_m || N > b_n || a_k != b_k) return NVFP4_ERR_SHAPE;
+    if ((int64_t)groups * M > 0x7FFFFFFF) return NVFP4_ERR_SHAPE;
+  }
   if (((uintptr_t)a & 15u) || ((uintptr_t)b & 15u) || (lda * 2) % 16 || (ldb * 2) % 16 || ((uintptr_t)c & 3u))
     return NVFP4_ERR_ALIGN;
   CUtensorMap ta, tb;
-  if (!tmap_bf16(&ta, a, a_rows, a_cols, lda, BM) || !tmap_bf16(&tb, b, b_rows, a_cols, ldb, BN)) return NVFP4_ERR_CUDA;
+  if (!tmap_bf16(&ta, a, a_rows, a_cols, lda, a_mn_major ? BK : BM) ||
+      !tmap_bf16(&tb, b, b_rows, b_cols, ldb, b_mn_major ? BK : BN))
+    return NVFP4_ERR_CUDA;
   Params p;
   p.c = reinterpret_cast<__nv_bfloat16*>(c);
   p.ldc = ldc;
-  p.M = (int)(mode == 0 ? a_rows : M);
+  p.M = (int)(mode == 0 ? a_m : M);
   p.N = (int)N;
   p.K = (int)K;
   p.mode = mode;
@@ -315,15 +386,9 @@ extern "C" nvfp4_status nvfp4_gemm_bf16_grouped(int mode, int groups, const void
   p.off = seg_off;
   p.len = seg_len;
   p.c_vec16 = (((uintptr_t)c & 15u) == 0 && (ldc % 8) == 0) ? 1 : 0;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    attr = true;
-  }
-  int sms = 148, dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  gemm_bf16_kernel<<<sms, THREADS, SMEM_BYTES, (cudaStream_t)stream>>>(ta, tb, p);
-  count_launches(1);
-  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (!a_mn_major && !b_mn_major) return launch<false, false>(ta, tb, p, s);
+  if (!a_mn_major && b_mn_major) return launch<false, true>(ta, tb, p, s);
+  if (a_mn_major && !b_mn_major) return launch<true, false>(ta, tb, p, s);
+  return launch<true, true>(ta, tb, p, s);
 }

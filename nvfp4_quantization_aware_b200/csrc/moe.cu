@@ -354,68 +354,6 @@ __global__ void router_grad_kernel(const __nv_bfloat16* __restrict__ dy, const _
   }
 }
 
-// ------------------------------------------------------------------ transposes
-
-// out[c][r] = in[r][c] for a bf16 [rows][cols] matrix (32 x 32 tiles through
-// shared memory, padded against bank conflicts).
-__global__ void transpose_bf16_kernel(const __nv_bfloat16* __restrict__ in, int64_t ld_in, int rows, int cols,
-                                      __nv_bfloat16* __restrict__ out, int64_t ld_out) {
-  __shared__ __nv_bfloat16 tile[32][33];
-  const int tiles_c = (cols + 31) / 32;
-  const int64_t ntiles = (int64_t)((rows + 31) / 32) * tiles_c;
-  for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
-    const int r0 = (int)(t / tiles_c) * 32, c0 = (int)(t % tiles_c) * 32;
-    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-      const int r = r0 + i, c = c0 + threadIdx.x;
-      if (r < rows && c < cols) tile[i][threadIdx.x] = in[(int64_t)r * ld_in + c];
-    }
-    __syncthreads();
-    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-      const int c = c0 + i, r = r0 + threadIdx.x;
-      if (r < rows && c < cols) out[(int64_t)c * ld_out + r] = tile[threadIdx.x][i];
-    }
-    __syncthreads();
-  }
-}
-
-// Dequantized transpose of stacked NVFP4 weights: group g is rows
-// [g rows_g, (g+1) rows_g) of codes [*, cols/2] with row-major block scales and
-// tensor scale ts[g]; out[g cols + c][col_off + r] = value(code) * s_b * s_g
-// (bf16).  32 x 32 tiles through shared memory.
-__global__ void dequant_transpose_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sb,
-                                         const float* __restrict__ ts, int groups, int rows_g, int cols,
-                                         __nv_bfloat16* __restrict__ out, int64_t ld_out, int col_off) {
-  __shared__ float tile[32][33];
-  const int tiles_c = cols / 32;
-  const int tiles_r = (rows_g + 31) / 32;
-  const int64_t ntiles = (int64_t)groups * tiles_r * tiles_c;
-  for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
-    const int g = (int)(t / ((int64_t)tiles_r * tiles_c));
-    const int rem = (int)(t - (int64_t)g * tiles_r * tiles_c);
-    const int r0 = (rem / tiles_c) * 32, c0 = (rem % tiles_c) * 32;
-    const float sg = __ldg(ts + g);
-    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-      const int r = r0 + i, c = c0 + threadIdx.x;
-      float v = 0.f;
-      if (r < rows_g) {
-        const int64_t row = (int64_t)g * rows_g + r;
-        const uint32_t byte = __ldg(codes + row * (cols / 2) + c / 2);
-        float lo, hi;
-        e2m1x2_decode(byte, lo, hi);
-        const float d = __fmul_rn(e4m3_decode(__ldg(sb + row * (cols / 16) + c / 16)), sg);
-        v = __fmul_rn((c & 1) ? hi : lo, d);
-      }
-      tile[i][threadIdx.x] = v;
-    }
-    __syncthreads();
-    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-      const int c = c0 + i, r = r0 + threadIdx.x;
-      if (r < rows_g) out[((int64_t)g * cols + c) * ld_out + col_off + r] = __float2bfloat16_rn(tile[threadIdx.x][i]);
-    }
-    __syncthreads();
-  }
-}
-
 // Row-major block scales [rows][cols/16] -> the MMA scale layout (padding 0).
 __global__ void scales_to_mma_kernel(const uint8_t* __restrict__ sb, int64_t rows, int64_t cols,
                                      uint8_t* __restrict__ out) {
@@ -570,30 +508,6 @@ nvfp4_status nvfp4_moe_router_grad(const void* dy, const void* y, int64_t cols, 
   router_grad_kernel<<<sms() * 8, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const __nv_bfloat16*>(dy),
                                                                   reinterpret_cast<const __nv_bfloat16*>(y), (int)cols,
                                                                   slot_row, tokens * topk, topk, dw);
-  return done(1);
-}
-
-nvfp4_status nvfp4_transpose_bf16(const void* in, int64_t ld_in, int64_t rows, int64_t cols, void* out, int64_t ld_out,
-                                  void* stream) {
-  if (rows < 1 || cols < 1 || ld_in < cols || ld_out < rows || rows > 0x7FFFFFFF || cols > 0x7FFFFFFF)
-    return NVFP4_ERR_SHAPE;
-  if (!in || !out) return NVFP4_ERR_ARG;
-  transpose_bf16_kernel<<<sms() * 16, dim3(32, 8), 0, (cudaStream_t)stream>>>(
-      reinterpret_cast<const __nv_bfloat16*>(in), ld_in, (int)rows, (int)cols, reinterpret_cast<__nv_bfloat16*>(out),
-      ld_out);
-  return done(1);
-}
-
-nvfp4_status nvfp4_dequantize_transpose(const uint8_t* codes, const uint8_t* block_scales, const float* tensor_scales,
-                                        int groups, int64_t rows_per_group, int64_t cols, void* out, int64_t ld_out,
-                                        int64_t col_off, void* stream) {
-  if (groups < 1 || rows_per_group < 1 || cols < 32 || cols % 32 || ld_out < col_off + rows_per_group ||
-      (int64_t)groups * rows_per_group > 0x7FFFFFFF)
-    return NVFP4_ERR_SHAPE;
-  if (!codes || !block_scales || !tensor_scales || !out) return NVFP4_ERR_ARG;
-  dequant_transpose_kernel<<<sms() * 16, dim3(32, 8), 0, (cudaStream_t)stream>>>(
-      codes, block_scales, tensor_scales, groups, (int)rows_per_group, (int)cols, reinterpret_cast<__nv_bfloat16*>(out),
-      ld_out, (int)col_off);
   return done(1);
 }
 

@@ -11,6 +11,8 @@
 // unchanged, so gradients are plain BF16 products with the dequantized
 // operands the forward used):
 //   dY_g = w * dy  ->  dA = dY_g W^_down  ->  SwiGLU backward -> [dG | dU]
+//   (every product reads the forward's buffers in place: the BF16 GEMM takes
+//   MN-major operands, and the forward's weight quantizer also writes W^)
 //   dX_g = [dG | dU] [W^_gate; W^_up]  -> dx = sum over the token's experts
 //   dW_down = dY_g^T A^,  dW_gate = dG^T X^,  dW_up = dU^T X^,
 //   d(combine weight) = <dy, y_expert>.
@@ -58,15 +60,11 @@ Layout layout_of(const qad_moe_shape& s) {
   b[QAD_MOE_ACT] = s.save_act ? 2 * R * F : 0;
   b[QAD_MOE_Y_ROWS] = 2 * R * H;
   b[QAD_MOE_DY_ROWS] = 2 * R * H;
-  b[QAD_MOE_WD_T] = 2 * G * F * H;
+  b[QAD_MOE_WD_HAT] = 2 * G * H * F;
   b[QAD_MOE_DA] = 2 * R * F;
   b[QAD_MOE_DGU] = 2 * R * 2 * F;
-  b[QAD_MOE_WGU_T] = 2 * G * H * 2 * F;
+  b[QAD_MOE_WGU_HAT] = 2 * G * 2 * F * H;
   b[QAD_MOE_DX_ROWS] = 2 * R * H;
-  b[QAD_MOE_DY_ROWS_T] = 2 * H * R;
-  b[QAD_MOE_A_HAT_T] = 2 * F * R;
-  b[QAD_MOE_DGU_T] = 2 * 2 * F * R;
-  b[QAD_MOE_X_HAT_T] = 2 * H * R;
   size_t o = 0;
   for (int i = 0; i < QAD_MOE_NUM_BUFFERS; ++i) {
     L.off[i] = o;
@@ -140,7 +138,10 @@ nvfp4_status qad_moe_forward(const qad_moe_shape* shape, const qad_moe_weights* 
   // 1. routing: segments and the permutation
   QAD_TRY(nvfp4_moe_route(expert_ids, combine_weights, s.tokens, s.topk, s.experts, seg_len, seg_off, row_token,
                           row_weight, slot_row, R, stream));
-  // 2. master weights -> NVFP4 codes with their frozen scales (one call, 3G tensors)
+  // 2. master weights -> NVFP4 codes with their frozen scales, and the bf16
+  //    dequantized weights the backward multiplies with (one call, 3G tensors):
+  //    W^_gate / W^_up of group g interleaved as rows [2gF, 2gF + F) / [2gF + F,
+  //    2(g+1)F) of one stack, W^_down as its own stack
   {
     const __nv_bfloat16* wg = static_cast<const __nv_bfloat16*>(w->w_gate);
     const __nv_bfloat16* wu = static_cast<const __nv_bfloat16*>(w->w_up);
@@ -148,27 +149,34 @@ nvfp4_status qad_moe_forward(const qad_moe_shape* shape, const qad_moe_weights* 
     uint8_t* cg = at<uint8_t>(workspace, L, QAD_MOE_WG_CODES);
     uint8_t* cu = at<uint8_t>(workspace, L, QAD_MOE_WU_CODES);
     uint8_t* cd = at<uint8_t>(workspace, L, QAD_MOE_WD_CODES);
+    __nv_bfloat16* hgu = at<__nv_bfloat16>(workspace, L, QAD_MOE_WGU_HAT);
+    __nv_bfloat16* hd = at<__nv_bfloat16>(workspace, L, QAD_MOE_WD_HAT);
     nvfp4_tensor_ref refs[3 * 256];
+    void* ys[3 * 256];
+    int64_t lds[3 * 256];
     for (int g = 0; g < G; ++g) {
       nvfp4_tensor_ref& a = refs[g];
       a.x = wg + (int64_t)g * F * H; a.rows = F; a.cols = H; a.ld_x = H;
       a.tensor_scale = const_cast<float*>(w->gate_ts + g);
       a.block_scales = const_cast<uint8_t*>(w->gate_sb + (int64_t)g * F * (H / 16));
       a.out = cg + (int64_t)g * F * (H / 2); a.ld_out = H / 2;
+      ys[g] = hgu + (int64_t)g * 2 * F * H; lds[g] = H;
       nvfp4_tensor_ref& b = refs[G + g];
       b = a;
       b.x = wu + (int64_t)g * F * H;
       b.tensor_scale = const_cast<float*>(w->up_ts + g);
       b.block_scales = const_cast<uint8_t*>(w->up_sb + (int64_t)g * F * (H / 16));
       b.out = cu + (int64_t)g * F * (H / 2);
+      ys[G + g] = hgu + (int64_t)g * 2 * F * H + F * H; lds[G + g] = H;
       nvfp4_tensor_ref& d = refs[2 * G + g];
       d.x = wd + (int64_t)g * H * F; d.rows = H; d.cols = F; d.ld_x = F;
       d.tensor_scale = const_cast<float*>(w->down_ts + g);
       d.block_scales = const_cast<uint8_t*>(w->down_sb + (int64_t)g * H * (F / 16));
       d.out = cd + (int64_t)g * H * (F / 2); d.ld_out = F / 2;
+      ys[2 * G + g] = hd + (int64_t)g * H * F; lds[2 * G + g] = F;
     }
-    QAD_TRY(nvfp4_quantize_grouped(3 * G, refs, NVFP4_BF16, NVFP4_FROZEN_ALL, NVFP4_SCALES_ROWMAJOR, nullptr, 0,
-                                   stream));
+    QAD_TRY(nvfp4_quantize_fake_quant_grouped(3 * G, refs, ys, lds, NVFP4_BF16, NVFP4_FROZEN_ALL,
+                                              NVFP4_SCALES_ROWMAJOR, nullptr, 0, stream));
   }
   // 3. gather the routed tokens and quantize them (frozen s_g per expert)
   QAD_TRY(nvfp4_moe_gather_quantize(x, H, row_token, seg_off, G, w->x_ts, R, H,
@@ -219,43 +227,38 @@ nvfp4_status qad_moe_backward(const qad_moe_shape* shape, const qad_moe_weights*
   float* row_weight = at<float>(workspace, L, QAD_MOE_ROW_WEIGHT);
   int32_t* slot_row = at<int32_t>(workspace, L, QAD_MOE_SLOT_ROW);
   void* dyp = at<void>(workspace, L, QAD_MOE_DY_ROWS);
-  void* wdt = at<void>(workspace, L, QAD_MOE_WD_T);
   void* da = at<void>(workspace, L, QAD_MOE_DA);
-  void* dgu = at<void>(workspace, L, QAD_MOE_DGU);
-  void* wgut = at<void>(workspace, L, QAD_MOE_WGU_T);
+  __nv_bfloat16* dgu = at<__nv_bfloat16>(workspace, L, QAD_MOE_DGU);
   void* dxp = at<void>(workspace, L, QAD_MOE_DX_ROWS);
-  __nv_bfloat16* dypt = at<__nv_bfloat16>(workspace, L, QAD_MOE_DY_ROWS_T);
-  __nv_bfloat16* ahatt = at<__nv_bfloat16>(workspace, L, QAD_MOE_A_HAT_T);
-  __nv_bfloat16* dgut = at<__nv_bfloat16>(workspace, L, QAD_MOE_DGU_T);
-  __nv_bfloat16* xhatt = at<__nv_bfloat16>(workspace, L, QAD_MOE_X_HAT_T);
+  const void* xhat = at<void>(workspace, L, QAD_MOE_X_HAT);
+  const void* ahat = at<void>(workspace, L, QAD_MOE_A_HAT);
+  const void* wd_hat = at<void>(workspace, L, QAD_MOE_WD_HAT);    // [G H x F]
+  const void* wgu_hat = at<void>(workspace, L, QAD_MOE_WGU_HAT);  // [G 2F x H]
 
   // dY of each routed row: combine weight times the token's output gradient
   QAD_TRY(nvfp4_moe_scale_rows(dy, H, row_token, row_weight, seg_off, G, R, dyp, stream));
-  // dequantized, transposed weights (the operands the forward used, in bf16)
-  QAD_TRY(nvfp4_dequantize_transpose(at<uint8_t>(workspace, L, QAD_MOE_WD_CODES), w->down_sb, w->down_ts, G, H, F, wdt,
-                                     H, 0, stream));
-  QAD_TRY(nvfp4_dequantize_transpose(at<uint8_t>(workspace, L, QAD_MOE_WG_CODES), w->gate_sb, w->gate_ts, G, F, H, wgut,
-                                     2 * F, 0, stream));
-  QAD_TRY(nvfp4_dequantize_transpose(at<uint8_t>(workspace, L, QAD_MOE_WU_CODES), w->up_sb, w->up_ts, G, F, H, wgut,
-                                     2 * F, F, stream));
-  // dA = dY W^_down   (M-segments: [R x H] x [G F x H]^T per group)
-  QAD_TRY(nvfp4_gemm_bf16_grouped(0, G, dyp, R, H, H, wdt, (int64_t)G * F, H, seg_off, seg_len, R, F, H, da, F, stream));
+  // dA = dY W^_down: A = dY rows (K-major, K = H), B_g[f][h] = W^_down_g[h][f]
+  // (MN-major, the stack's K rows g H .. g H + H - 1)
+  QAD_TRY(nvfp4_gemm_bf16_grouped(0, G, dyp, 0, R, H, H, wd_hat, 1, (int64_t)G * H, F, F, seg_off, seg_len, 0, F, H,
+                                  da, F, stream));
   // SwiGLU backward -> [dG | dU]
   QAD_TRY(nvfp4_moe_swiglu_backward(da, at<void>(workspace, L, QAD_MOE_H_GATE), at<void>(workspace, L, QAD_MOE_H_UP), F,
                                     row_token, seg_off, G, R, dgu, stream));
-  // dX rows = [dG | dU] [W^_gate; W^_up], then the sum over each token's experts
-  QAD_TRY(nvfp4_gemm_bf16_grouped(0, G, dgu, R, 2 * F, 2 * F, wgut, (int64_t)G * H, 2 * F, seg_off, seg_len, R, H,
-                                  2 * F, dxp, H, stream));
+  // dX rows = [dG | dU] [W^_gate; W^_up]: B_g[h][k] = W^_gu_g[k][h] (MN-major,
+  // K rows 2 g F .. 2 (g+1) F - 1), then the sum over each token's experts
+  QAD_TRY(nvfp4_gemm_bf16_grouped(0, G, dgu, 0, R, 2 * F, 2 * F, wgu_hat, 1, (int64_t)G * 2 * F, H, H, seg_off,
+                                  seg_len, 0, H, 2 * F, dxp, H, stream));
   QAD_TRY(nvfp4_moe_gather_sum(dxp, H, slot_row, s.tokens, s.topk, seg_off, s.experts, dx, stream));
-  // weight gradients, reduced over each expert's rows (K-segments)
-  QAD_TRY(nvfp4_transpose_bf16(dyp, H, R, H, dypt, R, stream));
-  QAD_TRY(nvfp4_transpose_bf16(at<void>(workspace, L, QAD_MOE_A_HAT), F, R, F, ahatt, R, stream));
-  QAD_TRY(nvfp4_transpose_bf16(dgu, 2 * F, R, 2 * F, dgut, R, stream));
-  QAD_TRY(nvfp4_transpose_bf16(at<void>(workspace, L, QAD_MOE_X_HAT), H, R, H, xhatt, R, stream));
-  QAD_TRY(nvfp4_gemm_bf16_grouped(1, G, dypt, H, R, R, ahatt, F, R, seg_off, seg_len, H, F, 0, dw_down, F, stream));
-  QAD_TRY(nvfp4_gemm_bf16_grouped(1, G, dgut, F, R, R, xhatt, H, R, seg_off, seg_len, F, H, 0, dw_gate, H, stream));
-  QAD_TRY(nvfp4_gemm_bf16_grouped(1, G, dgut + F * R, F, R, R, xhatt, H, R, seg_off, seg_len, F, H, 0, dw_up, H,
+  // weight gradients, reduced over each expert's rows (K-segments, both
+  // operands MN-major: the row buffers as they are)
+  //   dW_down_g[h][f] = sum_r dY[r][h] A^[r][f]
+  QAD_TRY(nvfp4_gemm_bf16_grouped(1, G, dyp, 1, R, H, H, ahat, 1, R, F, F, seg_off, seg_len, H, F, 0, dw_down, F,
                                   stream));
+  //   dW_gate_g[f][h] = sum_r dG[r][f] X^[r][h],  dW_up_g likewise with dU
+  QAD_TRY(nvfp4_gemm_bf16_grouped(1, G, dgu, 1, R, F, 2 * F, xhat, 1, R, H, H, seg_off, seg_len, F, H, 0, dw_gate, H,
+                                  stream));
+  QAD_TRY(nvfp4_gemm_bf16_grouped(1, G, dgu + F, 1, R, F, 2 * F, xhat, 1, R, H, H, seg_off, seg_len, F, H, 0, dw_up,
+                                  H, stream));
   // gradient of the combine weights
   if (d_combine)
     QAD_TRY(nvfp4_moe_router_grad(dy, at<void>(workspace, L, QAD_MOE_Y_ROWS), H, slot_row, s.tokens, s.topk, d_combine,

@@ -81,10 +81,10 @@ constexpr int kMaxGroup = 144;
 struct GTensor {
   const void* x;        // input, row stride ld_x elements
   uint8_t* codes;       // Out::Codes: packed codes, row stride ld_out bytes
-  void* y;              // Out::Fake: output, row stride ld_out elements
+  void* y;              // Out::Fake / Out::Both: dequantized output, row stride ld_y elements
   uint8_t* sb;          // block scales: read (FROZEN_ALL, row-major) or written if non-NULL
   float* ts;            // tensor scale: written (DYNAMIC) or read
-  int64_t ld_x, ld_out;
+  int64_t ld_x, ld_out, ld_y;
   int64_t cols;
   int64_t chunk0;       // first chunk of this tensor in the group
   int64_t kchunks;      // ceil(cols / 64), MMA scale layout
@@ -99,7 +99,8 @@ struct GroupArgs {
   int64_t total_chunks;
   unsigned* amax;       // DYNAMIC: n words holding max |x| as float bits (zeroed first)
   int x_wide;           // every input row start is 32-byte aligned: 256-bit loads
-  int out_wide;         // codes rows 8-byte aligned (8-byte stores) / y rows 32-byte aligned
+  int out_wide;         // codes rows 8-byte aligned (8-byte stores)
+  int y_wide;           // y rows 32-byte aligned (256-bit stores)
 };
 
 // Advance `t` to the tensor owning `chunk` (chunks are visited in increasing
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(kThreads) group_amax_kernel(const __grid_const
 
 // ------------------------------------------------------------------ encode
 
-enum class Out { Codes, Fake };
+enum class Out { Codes, Fake, Both };  // Both: codes and the fake-quant values
 
 // s_g of tensor t: amax / (6 * 448) in DYNAMIC mode, else the given scale.
 NVFP4_DEV float tensor_scale_of(const GroupArgs& a, int t) {
@@ -246,7 +247,7 @@ __global__ void __launch_bounds__(kThreads) group_encode_kernel(const __grid_con
       float d;
       const uint32_t sb = encode_block16<sizeof(T) == 2>(v, sg, denom6, frozen_all, sb_in[u], lo, hi, d);
       // ---- outputs
-      if (OUT == Out::Codes) {
+      if (OUT != Out::Fake) {
         uint8_t* dst = g.codes + row * g.ld_out + (col >> 1);
         if (a.out_wide) {
           st_stream_v2(dst, lo, hi);
@@ -254,10 +255,11 @@ __global__ void __launch_bounds__(kThreads) group_encode_kernel(const __grid_con
           st_stream_u32(dst, lo);
           st_stream_u32(dst + 4, hi);
         }
-      } else {
+      }
+      if (OUT != Out::Codes) {
         float o[16];
         decode_block16(lo, hi, d, o);
-        Block16<T>::store(reinterpret_cast<T*>(g.y) + row * g.ld_out + col, o, a.out_wide != 0);
+        Block16<T>::store(reinterpret_cast<T*>(g.y) + row * g.ld_y + col, o, a.y_wide != 0);
       }
       if (!frozen_all && g.sb != nullptr) {
         const int64_t kb = col >> 4;
@@ -432,7 +434,7 @@ static nvfp4_status check_tensor(const nvfp4_tensor_ref& r, nvfp4_dtype dtype, n
   if (r.rows == 0 || r.cols == 0) return NVFP4_OK;
   if (mode == NVFP4_FROZEN_ALL && !r.block_scales) return NVFP4_ERR_ARG;
   if (!r.out) return NVFP4_ERR_ARG;
-  if (OUT == Out::Codes) {
+  if (OUT != Out::Fake) {
     if (!r.block_scales) return NVFP4_ERR_ARG;
     if (r.ld_out < r.cols / 2) return NVFP4_ERR_SHAPE;
     if ((r.ld_out % 4) != 0 || ((uintptr_t)r.out & 3u) != 0) return NVFP4_ERR_ALIGN;
@@ -441,6 +443,16 @@ static nvfp4_status check_tensor(const nvfp4_tensor_ref& r, nvfp4_dtype dtype, n
     const int64_t esz = dtype == NVFP4_BF16 ? 2 : 4;
     if (!aligned16(r.out) || (r.ld_out * esz) % 16 != 0) return NVFP4_ERR_ALIGN;
   }
+  return NVFP4_OK;
+}
+
+// The fake-quant output of an Out::Both call (y, ld_y elements of dtype).
+static nvfp4_status check_y(const nvfp4_tensor_ref& r, const void* y, int64_t ld_y, nvfp4_dtype dtype) {
+  if (r.rows == 0 || r.cols == 0) return NVFP4_OK;
+  if (!y) return NVFP4_ERR_ARG;
+  if (ld_y < r.cols) return NVFP4_ERR_SHAPE;
+  const int64_t esz = dtype == NVFP4_BF16 ? 2 : 4;
+  if (!aligned16(y) || (ld_y * esz) % 16 != 0) return NVFP4_ERR_ALIGN;
   return NVFP4_OK;
 }
 
@@ -501,13 +513,16 @@ static nvfp4_status launch_group(GroupArgs& a, nvfp4_dtype dtype, unsigned* amax
 // first, then one (FROZEN) or two (DYNAMIC) launches per group.
 template <Out OUT>
 static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype dtype, nvfp4_scale_mode mode,
-                                nvfp4_scale_layout layout, void* ws, size_t ws_bytes, cudaStream_t s) {
+                                nvfp4_scale_layout layout, void* ws, size_t ws_bytes, cudaStream_t s,
+                                void* const* ys = nullptr, const int64_t* ld_ys = nullptr) {
   if (n < 0 || (n > 0 && !refs)) return NVFP4_ERR_ARG;
+  if (OUT == Out::Both && n > 0 && (!ys || !ld_ys)) return NVFP4_ERR_ARG;
   if (mode != NVFP4_DYNAMIC && mode != NVFP4_FROZEN_GLOBAL && mode != NVFP4_FROZEN_ALL) return NVFP4_ERR_ARG;
   if (layout != NVFP4_SCALES_ROWMAJOR && layout != NVFP4_SCALES_MMA) return NVFP4_ERR_ARG;
   if (OUT == Out::Fake && layout != NVFP4_SCALES_ROWMAJOR) return NVFP4_ERR_ARG;
   for (int i = 0; i < n; ++i) {
     nvfp4_status st = check_tensor<OUT>(refs[i], dtype, mode, layout);
+    if (st == NVFP4_OK && OUT == Out::Both) st = check_y(refs[i], ys[i], ld_ys[i], dtype);
     if (st != NVFP4_OK) return st;
   }
   if (mode == NVFP4_DYNAMIC) {
@@ -523,6 +538,7 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
   a.amax = nullptr;
   a.x_wide = 1;
   a.out_wide = 1;
+  a.y_wide = 1;
   int64_t group_bytes = 0;
   // DYNAMIC: every group takes its own amax words from the workspace; the
   // words are cleared once per call, and again whenever they run out.
@@ -557,12 +573,14 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
       a.total_chunks = 0;
       a.x_wide = 1;
       a.out_wide = 1;
+      a.y_wide = 1;
       group_bytes = 0;
     }
     GTensor& g = a.t[a.n++];
     g.x = r.x;
-    g.codes = OUT == Out::Codes ? reinterpret_cast<uint8_t*>(r.out) : nullptr;
-    g.y = OUT == Out::Fake ? r.out : nullptr;
+    g.codes = OUT != Out::Fake ? reinterpret_cast<uint8_t*>(r.out) : nullptr;
+    g.y = OUT == Out::Fake ? r.out : (OUT == Out::Both ? ys[i] : nullptr);
+    g.ld_y = OUT == Out::Fake ? r.ld_out : (OUT == Out::Both ? ld_ys[i] : 0);
     g.sb = r.block_scales;
     g.ts = r.tensor_scale;
     g.ld_x = r.ld_x;
@@ -576,16 +594,13 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
     group_bytes += bytes;
     // 32-byte rows for 256-bit input loads; 8-byte code rows / 32-byte y rows
     if (((uintptr_t)r.x & 31u) || ((r.ld_x * esz) & 31)) a.x_wide = 0;
-    if (OUT == Out::Codes) {
-      if (((uintptr_t)r.out & 7u) || (r.ld_out & 7)) a.out_wide = 0;
-    } else {
-      if (((uintptr_t)r.out & 31u) || ((r.ld_out * esz) & 31)) a.out_wide = 0;
-    }
+    if (OUT != Out::Fake && (((uintptr_t)r.out & 7u) || (r.ld_out & 7))) a.out_wide = 0;
+    if (OUT != Out::Codes && (((uintptr_t)g.y & 31u) || ((g.ld_y * esz) & 31))) a.y_wide = 0;
   }
   nvfp4_status st = flush();
   if (st != NVFP4_OK) return st;
   // zero the padding of MMA-layout scale arrays
-  if (OUT == Out::Codes && layout == NVFP4_SCALES_MMA && mode != NVFP4_FROZEN_ALL) {
+  if (OUT != Out::Fake && layout == NVFP4_SCALES_MMA && mode != NVFP4_FROZEN_ALL) {
     for (int i = 0; i < n; ++i) {
       const nvfp4_tensor_ref& r = refs[i];
       if (r.rows == 0 || r.cols == 0) continue;
@@ -663,6 +678,14 @@ nvfp4_status nvfp4_quantize_grouped(int num_tensors, const nvfp4_tensor_ref* ten
                                     size_t workspace_bytes, void* stream) {
   return run_tensors<Out::Codes>(num_tensors, tensors, dtype, mode, layout, workspace, workspace_bytes,
                                  (cudaStream_t)stream);
+}
+
+nvfp4_status nvfp4_quantize_fake_quant_grouped(int num_tensors, const nvfp4_tensor_ref* tensors, void* const* y,
+                                               const int64_t* ld_y, nvfp4_dtype dtype, nvfp4_scale_mode mode,
+                                               nvfp4_scale_layout layout, void* workspace, size_t workspace_bytes,
+                                               void* stream) {
+  return run_tensors<Out::Both>(num_tensors, tensors, dtype, mode, layout, workspace, workspace_bytes,
+                                (cudaStream_t)stream, y, ld_y);
 }
 
 nvfp4_status nvfp4_fake_quant_grouped(int num_tensors, const nvfp4_tensor_ref* tensors, nvfp4_dtype dtype,

@@ -117,6 +117,14 @@ def test_moe_step_matches_oracle(case):
         for g in range(G):
             assert np.array_equal(codes[g * rows:(g + 1) * rows], L.weight(kind, g)[0]), (kind, g)
 
+    # dequantized weights the backward uses (exact)
+    wd_hat = step.buffer("wd_hat").view(torch.int16).cpu().numpy().view(np.uint16)
+    wgu_hat = step.buffer("wgu_hat").view(torch.int16).cpu().numpy().view(np.uint16)
+    for g in range(G):
+        assert np.array_equal(wd_hat[g * H:(g + 1) * H], O.bf16_round(L.weight("down", g)[3])), g
+        assert np.array_equal(wgu_hat[2 * g * F:2 * g * F + F], O.bf16_round(L.weight("gate", g)[3])), g
+        assert np.array_equal(wgu_hat[2 * g * F + F:2 * (g + 1) * F], O.bf16_round(L.weight("up", g)[3])), g
+
     # routed rows: codes, MMA scales, dequantized rows (exact); padding zero
     xc = step.buffer("x_codes").cpu().numpy()
     xs = step.buffer("x_scales").cpu().numpy()
@@ -236,28 +244,45 @@ def _segments(lens, align=128):
     return off
 
 
+MAJORS = [(False, False), (False, True), (True, False), (True, True)]
+
+
+def _padded(x: torch.Tensor) -> torch.Tensor:
+    """x on the device in a buffer whose row stride is a multiple of 8 elements."""
+    rows, cols = x.shape
+    buf = torch.zeros(rows, (cols + 7) // 8 * 8, dtype=x.dtype, device=DEV)
+    buf[:, :cols] = x.to(DEV)
+    return buf[:, :cols]
+
+
+@pytest.mark.parametrize("a_mn,b_mn", MAJORS)
 @pytest.mark.parametrize("lens,N,K", [([200, 0, 128, 1, 300], 256, 192), ([192] * 5 + [700], 512, 1024),
                                       ([5], 768, 64)])
-def test_bf16_grouped_gemm_m_segments(lens, N, K):
+def test_bf16_grouped_gemm_m_segments(lens, N, K, a_mn, b_mn):
     g = torch.Generator().manual_seed(len(lens) + N)
     off = _segments(lens)
     R = max(off[-1], 128)
-    a = torch.randn(R, K, generator=g).to(torch.bfloat16)
-    b = (torch.randn(len(lens) * N, K, generator=g) * 0.1).to(torch.bfloat16)
-    c = Q.nvfp4_gemm_bf16_grouped(0, a.to(DEV), b.to(DEV), torch.tensor(off, dtype=torch.int32, device=DEV),
-                                  torch.tensor(lens, dtype=torch.int32, device=DEV), 0, N, K)
+    G = len(lens)
+    a = torch.randn(R, K, generator=g).to(torch.bfloat16)                 # logical A [R x K]
+    b = (torch.randn(G, N, K, generator=g) * 0.1).to(torch.bfloat16)      # logical B_g [N x K]
+    a_st = a.t().contiguous() if a_mn else a
+    b_st = b.transpose(1, 2).reshape(G * K, N).contiguous() if b_mn else b.reshape(G * N, K)
+    c = Q.nvfp4_gemm_bf16_grouped(0, a_st.to(DEV), b_st.to(DEV), torch.tensor(off, dtype=torch.int32, device=DEV),
+                                  torch.tensor(lens, dtype=torch.int32, device=DEV), 0, N, K,
+                                  a_mn_major=a_mn, b_mn_major=b_mn)
     torch.cuda.synchronize()
     assert Q.nvfp4_device_error()[0] == 0
     a64, b64 = a.double(), b.double()
     for i, n in enumerate(lens):
         if n == 0:
             continue
-        want = (a64[off[i]:off[i] + n] @ b64[i * N:(i + 1) * N].T).to(torch.bfloat16).double().numpy()
+        want = (a64[off[i]:off[i] + n] @ b64[i].T).to(torch.bfloat16).double().numpy()
         assert _rel(c[off[i]:off[i] + n].double().cpu().numpy(), want) <= GEMM_RTOL, i
 
 
+@pytest.mark.parametrize("a_mn,b_mn", MAJORS)
 @pytest.mark.parametrize("lens,M,N", [([200, 0, 128, 1, 300], 256, 512), ([192] * 4, 1024, 256), ([64], 130, 260)])
-def test_bf16_grouped_gemm_k_segments(lens, M, N):
+def test_bf16_grouped_gemm_k_segments(lens, M, N, a_mn, b_mn):
     g = torch.Generator().manual_seed(len(lens) + M)
     off = _segments(lens)
     R = max(off[-1], 128)
@@ -267,8 +292,12 @@ def test_bf16_grouped_gemm_k_segments(lens, M, N):
         a[:, off[i]:off[i] + n] = torch.randn(M, n, generator=g)
         b[:, off[i]:off[i] + n] = torch.randn(N, n, generator=g) * 0.1
     a, b = a.to(torch.bfloat16), b.to(torch.bfloat16)
-    c = Q.nvfp4_gemm_bf16_grouped(1, a.to(DEV), b.to(DEV), torch.tensor(off, dtype=torch.int32, device=DEV),
-                                  torch.tensor(lens, dtype=torch.int32, device=DEV), M, N, 0)
+    # MN-major storage: the M / N index contiguous, rows padded to 16 bytes
+    a_st = _padded(a.t()) if a_mn else a.to(DEV)
+    b_st = _padded(b.t()) if b_mn else b.to(DEV)
+    c = Q.nvfp4_gemm_bf16_grouped(1, a_st, b_st, torch.tensor(off, dtype=torch.int32, device=DEV),
+                                  torch.tensor(lens, dtype=torch.int32, device=DEV), M, N, 0,
+                                  a_mn_major=a_mn, b_mn_major=b_mn)
     torch.cuda.synchronize()
     assert Q.nvfp4_device_error()[0] == 0
     a64, b64 = a.double(), b.double()
@@ -281,19 +310,18 @@ def test_bf16_grouped_gemm_k_segments(lens, M, N):
         assert _rel(got, want) <= GEMM_RTOL, i
 
 
-def test_transpose_and_dequantize_transpose_exact():
-    x = torch.randn(300, 200, generator=torch.Generator().manual_seed(0)).to(torch.bfloat16)
-    assert torch.equal(Q.nvfp4_transpose_bf16(x.to(DEV)).cpu(), x.t())
+def test_quantize_fake_quant_grouped_matches_oracle():
     G, rows, cols = 3, 136, 96
-    w = torch.stack([S.weights(rows, cols, seed=g) for g in range(G)])
-    codes, sbs, ts = Q.nvfp4_quantize_grouped([w[g].to(DEV) for g in range(G)], Q.DYNAMIC)
-    out = torch.zeros(G * cols, rows + 8, dtype=torch.bfloat16, device=DEV)
-    Q.nvfp4_dequantize_transpose(torch.cat(codes), torch.cat(sbs), ts, G, rows, cols, out=out, col_off=8)
-    got = out.view(torch.int16).cpu().numpy().view(np.uint16)
-    assert not got[:, :8].any()
+    w = [S.weights(rows, cols, seed=g) for g in range(G)]
+    wd = [x.to(DEV) for x in w]
+    _, sbs, ts = Q.nvfp4_quantize_grouped(wd, Q.DYNAMIC)
+    ys = [torch.zeros(rows, cols + 8, dtype=torch.bfloat16, device=DEV)[:, 8:] for _ in range(G)]
+    codes, ys = Q.nvfp4_quantize_fake_quant_grouped(wd, Q.FROZEN_ALL, ts, sbs, ys=ys)
     for g in range(G):
-        _, bits, _, _ = O.fake_quant(w[g].float().numpy(), O.DYNAMIC)
-        assert np.array_equal(got[g * cols:(g + 1) * cols, 8:], bits.T), g
+        oc, osb, osg = O.quantize(w[g].float().numpy(), O.DYNAMIC)
+        _, bits, _, _ = O.fake_quant(w[g].float().numpy(), O.FROZEN_ALL, s_g=osg, s_b=osb)
+        assert np.array_equal(codes[g].cpu().numpy(), oc), g
+        assert np.array_equal(ys[g].contiguous().view(torch.int16).cpu().numpy().view(np.uint16), bits), g
 
 
 def test_scales_to_mma_matches_oracle_swizzle():
