@@ -317,9 +317,11 @@ nvfp4_status nvfp4_gemm_w4a4_grouped(int groups, const uint8_t* a_codes, const u
  *                        seg_len[g]) with seg_off[g] % 128 == 0 and the M
  *                        extent a multiple of 128; B of group g: N indices
  *                        [g N, (g+1) N) (K-major) or K indices [g K, (g+1) K)
- *                        (MN-major); c: M extent x N (ldc), only the
- *                        segments' valid rows written.  K % 64 == 0; M is
- *                        ignored.
+ *                        (MN-major); c: M extent x N (ldc): the segments'
+ *                        rows are written (when c is 16-byte aligned with
+ *                        ldc % 8 == 0, also the padding rows of each
+ *                        segment's last 128-row tile, with A's padding rows
+ *                        times B).  K % 64 == 0; M is ignored.
  *   mode 1 (K-segments)  group g reduces over K indices [seg_off[g],
  *                        seg_off[g] + seg_len[g]) of A and B (seg_off[g] % 64
  *                        == 0; K indices up to the next multiple of 64 are
@@ -407,7 +409,8 @@ nvfp4_status nvfp4_moe_scale_rows(const void* dy, int64_t cols, const int32_t* r
 /* SwiGLU backward, binary32: s = 1 / (1 + expf(-g)),
  *   dG = da * u * s * (1 + g (1 - s)),  dU = da * g * s,
  * written as dgu[r] = [dG | dU] (bf16 rows_cap x 2 cols); da, h_gate, h_up
- * bf16 rows_cap x cols contiguous; zeros on padding rows. */
+ * bf16 rows_cap x cols contiguous; zeros on padding rows.  cols % 8 == 0,
+ * pointers 16-byte aligned. */
 nvfp4_status nvfp4_moe_swiglu_backward(const void* da, const void* h_gate, const void* h_up, int64_t cols,
                                        const int32_t* row_token, const int32_t* seg_off, int groups,
                                        int64_t rows_cap, void* dgu, void* stream);

@@ -21,11 +21,15 @@
 //               and B (the group's tokens; off a multiple of 64, padding
 //               holds zeros); C of group g is rows [g M, (g+1) M).  Used for
 //               the weight gradients dW = dY^T A^.
-// Persistent CTAs (one per SM), 128 x 256 tiles, 4-stage TMA ring (128-byte
+// Persistent CTAs (one per SM), 128 x 256 tiles, 3-stage TMA ring (128-byte
 // swizzle), two accumulators in tensor memory so that the epilogue of one
-// tile overlaps the MMAs of the next, 8 epilogue warps, every wait bounded.
+// tile overlaps the MMAs of the next, 8 epilogue warps that stage their
+// 32 x 128 part of the tile in shared memory and write it with TMA stores
+// (full 128-byte lines), every wait bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+
+#include <cstring>
 
 #include "ptx.cuh"
 
@@ -36,13 +40,15 @@ namespace bf16gemm {
 constexpr int BM = 128, BN = 256;
 constexpr int BK = 64;                    // K per stage: 64 bf16 = 128 bytes
 constexpr int KB = BK / 16;               // MMAs (K = 16) per stage
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;
 constexpr int A_BYTES = BM * BK * 2;      // 16 KiB
 constexpr int B_BYTES = BN * BK * 2;      // 32 KiB
 constexpr int MN_ATOM_BYTES = BK * 128;   // MN-major: one 64-wide column block of a stage
 constexpr int MAX_GROUPS = 256;
-constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES) + 1024 + 256 + (2 * MAX_GROUPS + 1) * 4;
 constexpr int EPI_WARPS = 8;
+constexpr int STAGE_OUT_BYTES = 32 * 64 * 2;            // one TMA store box: 32 rows x 64 bf16
+constexpr int OUT_BYTES = EPI_WARPS * 2 * STAGE_OUT_BYTES; // two boxes per epilogue warp
+constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES) + OUT_BYTES + 1024 + 256 + (2 * MAX_GROUPS + 1) * 4;
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int ACC_COLS = BN;              // FP32 accumulator columns per tile
 constexpr int TM_COLS = 2 * ACC_COLS;     // two accumulators
@@ -64,10 +70,11 @@ struct Params {
   const int32_t* off;     // device [groups + 1]
   const int32_t* len;     // device [groups]
   int c_vec16;
+  int c_tma;              // write C through the 3-D tensor map (N, rows per group, groups)
 };
 
 struct Tile {
-  int m0, n0;
+  int g, m0, n0;
   int a_mn, a_k, b_mn, b_k;   // operand coordinates of the first stage (MN index, K index)
   int c_row0, row_end;
   int nk;                     // K stages
@@ -87,6 +94,7 @@ NVFP4_DEV Tile tile_of(int t, const Params& p, const int32_t* s_off, const int32
       if (s_off[mid] <= tl.m0) lo = mid;
       else hi = mid - 1;
     }
+    tl.g = lo;
     tl.a_mn = tl.m0;
     tl.a_k = 0;
     tl.b_mn = B_MN ? tl.n0 : lo * p.N + tl.n0;
@@ -100,6 +108,7 @@ NVFP4_DEV Tile tile_of(int t, const Params& p, const int32_t* s_off, const int32
     const int g = t / per_g;
     const int r = t - g * per_g;
     const int mt = r / num_n;
+    tl.g = g;
     tl.m0 = mt * BM;
     tl.n0 = (r - mt * num_n) * BN;
     tl.a_mn = tl.m0;
@@ -137,19 +146,21 @@ NVFP4_DEV uint64_t operand_desc(uint32_t base, int kb) {
 
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(THREADS, 1)
-    gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
+    gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmC, Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+  uint8_t* sOut = sB + STAGES * B_BYTES;   // 1024-byte aligned: 128-byte swizzle of the store boxes
+  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + OUT_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;     // [2]
   uint64_t* acc_empty = acc_full + 2;      // [2]
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
-  int32_t* s_off = reinterpret_cast<int32_t*>(smem + STAGES * (A_BYTES + B_BYTES) + 256);
+  int32_t* s_off = reinterpret_cast<int32_t*>(smem + STAGES * (A_BYTES + B_BYTES) + OUT_BYTES + 256);
   int32_t* s_len = s_off + MAX_GROUPS + 1;
 
   const int warp = threadIdx.x >> 5;
@@ -172,6 +183,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (p.c_tma) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc(tmem_base_slot, TM_COLS);
@@ -263,6 +275,29 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (p.c_tma) {
+        // stage rows sub*32 .. +31, columns cbase .. cbase+127 as two 32 x 64
+        // boxes (row `lane` at 128 bytes per row, 16-byte chunk j at j ^ (row % 8))
+        uint8_t* st = sOut + (warp - 2) * 2 * STAGE_OUT_BYTES;
+        if (lane == 0) bulk_wait_group_read0();  // the previous tile's boxes have been read
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t* v = packed + q * 32 + 4 * j;
+            st_shared_v4(st + q * STAGE_OUT_BYTES + lane * 128 + ((j ^ (lane & 7)) << 4), v[0], v[1], v[2], v[3]);
+          }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int y = tl.m0 + sub * 32, z = p.mode == 0 ? 0 : tl.g;
+          tma_store_3d(&tmC, st, tl.n0 + cbase, y, z);
+          tma_store_3d(&tmC, st + STAGE_OUT_BYTES, tl.n0 + cbase + 64, y, z);
+          bulk_commit_group();
+        }
+        continue;
+      }
       const int row = tl.m0 + sub * 32 + lane;
       if (row < tl.row_end) {
         __nv_bfloat16* crow = p.c + ((int64_t)tl.c_row0 + row) * p.ldc;
@@ -287,6 +322,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
     }
+    if (p.c_tma && lane == 0) bulk_wait_group0();  // stores complete before the CTA's memory goes away
   }
   tc_fence_before();
   __syncthreads();
@@ -322,8 +358,23 @@ static bool tmap_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t co
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// C as a 3-D tensor (N, rows per group, groups), box 64 x 32 x 1, 128-byte
+// swizzle: a store never crosses into the next group's rows.
+static bool tmap_c(CUtensorMap* m, void* base, int64_t n, int64_t rows, int64_t groups, int64_t ldc) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)n, (cuuint64_t)rows, (cuuint64_t)groups};
+  cuuint64_t strides[2] = {(cuuint64_t)(ldc * 2), (cuuint64_t)(ldc * 2 * rows)};
+  cuuint32_t box[3] = {64u, 32u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <bool A_MN, bool B_MN>
-static nvfp4_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, cudaStream_t s) {
+static nvfp4_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const Params& p,
+                           cudaStream_t s) {
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(gemm_bf16_kernel<A_MN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -333,7 +384,7 @@ static nvfp4_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const P
   }
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  gemm_bf16_kernel<A_MN, B_MN><<<sms, THREADS, SMEM_BYTES, s>>>(ta, tb, p);
+  gemm_bf16_kernel<A_MN, B_MN><<<sms, THREADS, SMEM_BYTES, s>>>(ta, tb, tc, p);
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
@@ -386,9 +437,18 @@ extern "C" nvfp4_status nvfp4_gemm_bf16_grouped(int mode, int groups, const void
   p.off = seg_off;
   p.len = seg_len;
   p.c_vec16 = (((uintptr_t)c & 15u) == 0 && (ldc % 8) == 0) ? 1 : 0;
+  // TMA stores need a 16-byte aligned C; in M-segment mode they also write
+  // the padding rows of each segment's last 128-row tile
+  CUtensorMap tc;
+  memset(&tc, 0, sizeof(tc));
+  p.c_tma = 0;
+  if (p.c_vec16) {
+    const bool ok = mode == 0 ? tmap_c(&tc, c, N, a_m, 1, ldc) : tmap_c(&tc, c, N, M, groups, ldc);
+    p.c_tma = ok ? 1 : 0;
+  }
   cudaStream_t s = (cudaStream_t)stream;
-  if (!a_mn_major && !b_mn_major) return launch<false, false>(ta, tb, p, s);
-  if (!a_mn_major && b_mn_major) return launch<false, true>(ta, tb, p, s);
-  if (a_mn_major && !b_mn_major) return launch<true, false>(ta, tb, p, s);
-  return launch<true, true>(ta, tb, p, s);
+  if (!a_mn_major && !b_mn_major) return launch<false, false>(ta, tb, tc, p, s);
+  if (!a_mn_major && b_mn_major) return launch<false, true>(ta, tb, tc, p, s);
+  if (a_mn_major && !b_mn_major) return launch<true, false>(ta, tb, tc, p, s);
+  return launch<true, true>(ta, tb, tc, p, s);
 }

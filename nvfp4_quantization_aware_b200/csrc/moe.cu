@@ -282,21 +282,40 @@ __global__ void swiglu_bwd_kernel(const __nv_bfloat16* __restrict__ da, const __
                                   const __nv_bfloat16* __restrict__ hu, int cols, const int32_t* __restrict__ row_token,
                                   const int32_t* __restrict__ off, int groups, int rows_cap,
                                   __nv_bfloat16* __restrict__ dgu) {
+  // 8 consecutive columns per thread (16-byte loads and stores)
   const int end_rows = __ldg(off + groups);
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)rows_cap * cols;
+  const int vpr = cols / 8;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)rows_cap * vpr;
        i += (int64_t)gridDim.x * blockDim.x) {
-    const int r = (int)(i / cols);
-    const int c = (int)(i - (int64_t)r * cols);
+    const int r = (int)(i / vpr);
+    const int c = (int)(i - (int64_t)r * vpr) * 8;
     const int t = r < end_rows ? __ldg(row_token + r) : -1;
-    float dg = 0.f, du = 0.f;
+    uint4 og = make_uint4(0, 0, 0, 0), ou = make_uint4(0, 0, 0, 0);
     if (t >= 0) {
-      const float g = __bfloat162float(hg[i]), u = __bfloat162float(hu[i]), d = __bfloat162float(da[i]);
-      const float s = 1.0f / (1.0f + expf(-g));
-      dg = d * u * s * (1.0f + g * (1.0f - s));
-      du = d * g * s;
+      const int64_t e = (int64_t)r * cols + c;
+      const uint4 G = ld_stream_v4(hg + e), U = ld_stream_v4(hu + e), D = ld_stream_v4(da + e);
+      const uint32_t gw[4] = {G.x, G.y, G.z, G.w}, uw[4] = {U.x, U.y, U.z, U.w}, dw[4] = {D.x, D.y, D.z, D.w};
+      uint32_t rg[4], ru[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float dg2[2], du2[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float g = h ? bf16hi_to_f32(gw[k]) : bf16lo_to_f32(gw[k]);
+          const float u = h ? bf16hi_to_f32(uw[k]) : bf16lo_to_f32(uw[k]);
+          const float d = h ? bf16hi_to_f32(dw[k]) : bf16lo_to_f32(dw[k]);
+          const float sg = 1.0f / (1.0f + expf(-g));
+          dg2[h] = d * u * sg * (1.0f + g * (1.0f - sg));
+          du2[h] = d * g * sg;
+        }
+        rg[k] = pack_bf16x2(dg2[0], dg2[1]);
+        ru[k] = pack_bf16x2(du2[0], du2[1]);
+      }
+      og = make_uint4(rg[0], rg[1], rg[2], rg[3]);
+      ou = make_uint4(ru[0], ru[1], ru[2], ru[3]);
     }
-    dgu[(int64_t)r * 2 * cols + c] = __float2bfloat16_rn(dg);
-    dgu[(int64_t)r * 2 * cols + cols + c] = __float2bfloat16_rn(du);
+    st_stream_v4(dgu + (int64_t)r * 2 * cols + c, og);
+    st_stream_v4(dgu + (int64_t)r * 2 * cols + cols + c, ou);
   }
 }
 
@@ -480,8 +499,10 @@ nvfp4_status nvfp4_moe_scale_rows(const void* dy, int64_t cols, const int32_t* r
 nvfp4_status nvfp4_moe_swiglu_backward(const void* da, const void* h_gate, const void* h_up, int64_t cols,
                                        const int32_t* row_token, const int32_t* seg_off, int groups, int64_t rows_cap,
                                        void* dgu, void* stream) {
-  if (cols < 1 || rows_cap < 1 || groups < 1) return NVFP4_ERR_SHAPE;
+  if (cols < 8 || cols % 8 || rows_cap < 1 || groups < 1) return NVFP4_ERR_SHAPE;
   if (!da || !h_gate || !h_up || !row_token || !seg_off || !dgu) return NVFP4_ERR_ARG;
+  if (((uintptr_t)da & 15u) || ((uintptr_t)h_gate & 15u) || ((uintptr_t)h_up & 15u) || ((uintptr_t)dgu & 15u))
+    return NVFP4_ERR_ALIGN;
   swiglu_bwd_kernel<<<sms() * 8, 256, 0, (cudaStream_t)stream>>>(
       reinterpret_cast<const __nv_bfloat16*>(da), reinterpret_cast<const __nv_bfloat16*>(h_gate),
       reinterpret_cast<const __nv_bfloat16*>(h_up), (int)cols, row_token, seg_off, groups, (int)rows_cap,

@@ -80,6 +80,33 @@ NVFP4_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* ba
       : "memory");
 }
 
+// 3-D tiled tensor store from this CTA's shared memory (bulk-group
+// completion).  Coordinates must be non-negative; x * element size a
+// multiple of 16 bytes.  Out-of-range parts of the box are not written.
+NVFP4_DEV void tma_store_3d(const void* tmap, const void* src, int32_t x, int32_t y, int32_t z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(tmap),
+               "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
+NVFP4_DEV void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until every committed bulk store of this thread has finished reading
+// its shared-memory source (the buffer may be overwritten afterwards).
+NVFP4_DEV void bulk_wait_group_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// Wait until every committed bulk store of this thread has completed.
+NVFP4_DEV void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Make this thread's generic-proxy shared-memory writes visible to the
+// async proxy (TMA) before a bulk store reads them.
+NVFP4_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+NVFP4_DEV void st_shared_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p)), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05
 
 NVFP4_DEV void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
