@@ -344,7 +344,8 @@ def bench_gemm(Q, dev, stream, P, K):
             xsf = torch.empty(Q.mma_scales_bytes(M, 4096), dtype=torch.uint8, device=dev)
             xts = torch.empty(1, dtype=torch.float32, device=dev)
             c = torch.empty(M, 4096, dtype=torch.bfloat16, device=dev)
-            qws = torch.empty(1024, dtype=torch.uint8, device=dev)
+            qws = torch.empty(int(Q.lib().nvfp4_quantize_workspace_size(M, 4096, Q.DYNAMIC)), dtype=torch.uint8,
+                              device=dev)
             for _ in range(3):
                 Q.nvfp4_quantize(x, Q.DYNAMIC, tensor_scale=xts, block_scales=xsf, layout=Q.SCALES_MMA, codes=xc,
                                  workspace=qws)

@@ -170,9 +170,9 @@ nvfp4_status nvfp4_selftest_division(uint64_t* mismatches, uint64_t* first, void
  * dtype and a scale mode, each with its own tensor scale (e.g. the routed and
  * shared expert weights of a MoE layer; one FP32 scale per expert).  Results
  * are identical to calling nvfp4_quantize / nvfp4_fake_quant on each tensor.
- * Kernels are launched per group of tensors (at most 144 tensors per group);
- * in DYNAMIC mode groups are cut at 48 MiB of input so that the encode pass
- * re-reads a group's inputs from L2.
+ * Kernels are launched per group of tensors (at most 144 tensors per
+ * group): one encode launch per group, preceded in DYNAMIC mode by one
+ * tensor-max launch.
  * ------------------------------------------------------------------------ */
 typedef struct nvfp4_tensor_ref {
   const void* x;          /* device input, rows x cols of the call's dtype */

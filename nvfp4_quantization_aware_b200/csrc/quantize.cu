@@ -16,9 +16,12 @@
 // independent loads per lane are in flight.  Grids are persistent: exactly the
 // resident capacity of the GPU (SM count x resident CTAs), grid-striding.
 //
-// Dynamic mode is two launches in stream order: group_amax_kernel folds each
-// tensor's max |x| into a workspace word (max is exact, so any order gives the
-// same s_g), then the encode kernel derives s_g = amax / 2688 from it.
+// Dynamic mode is two launches per group in stream order: group_amax_kernel
+// folds each tensor's max |x| into a workspace word (max is exact, so any
+// order gives the same s_g), then the encode kernel derives s_g = amax / 2688.
+// The encode is bound by instruction issue rather than by HBM, so re-reading
+// the inputs from L2 instead of HBM gains nothing: groups are cut only by the
+// number of tensors a launch holds.
 #include "quant_common.cuh"
 
 namespace nvfp4 {
@@ -27,7 +30,7 @@ constexpr int kThreads = 256;           // 8 warps per CTA
 constexpr int kWarps = kThreads / 32;
 constexpr int kUnroll = 4;              // chunks per warp per iteration (dequantize)
 constexpr int kChunk = 256;             // elements per warp per chunk (dequantize: 8 per lane)
-constexpr int kQUnroll = 2;             // chunks per warp per iteration (amax / encode)
+constexpr int kQUnroll = 2;             // chunks per warp per iteration (encode)
 constexpr int kQChunk = 512;            // elements per warp per chunk (amax / encode: 16 per lane)
 
 template <typename T>
@@ -86,6 +89,7 @@ struct GTensor {
   float* ts;            // tensor scale: written (DYNAMIC) or read
   int64_t ld_x, ld_out, ld_y;
   int64_t cols;
+  int64_t rows;
   int64_t chunk0;       // first chunk of this tensor in the group
   int64_t kchunks;      // ceil(cols / 64), MMA scale layout
   FastDiv cpr;          // chunks per row = ceil(cols / 512)
@@ -127,6 +131,36 @@ NVFP4_DEV void chunk_pos(const GTensor& g, int64_t chunk, int lane, int64_t& row
 // table into the global words with one atomicMax on the float bits per tensor
 // it touched (|x| >= 0 compares like its bit pattern; max is exact, so the
 // order of the atomics does not matter).
+// Running max |x| of one lane.  bf16: the magnitudes' bit patterns compare
+// like their values, so two 16-bit lanes of a word are folded at once
+// (unsigned 16x2 max of the words with the sign bits cleared).
+template <typename T>
+struct LaneMax;
+
+template <>
+struct LaneMax<__nv_bfloat16> {
+  uint32_t m2 = 0u;
+  NVFP4_DEV void reset() { m2 = 0u; }
+  NVFP4_DEV void add(const Block16<__nv_bfloat16>& b) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m2 = __vmaxu2(m2, b.w[i] & 0x7FFF7FFFu);
+  }
+  NVFP4_DEV float value() const { return fmaxf(bf16lo_to_f32(m2), bf16hi_to_f32(m2)); }
+};
+
+template <>
+struct LaneMax<float> {
+  float m = 0.0f;
+  NVFP4_DEV void reset() { m = 0.0f; }
+  NVFP4_DEV void add(const Block16<float>& b) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(__uint_as_float(b.w[i])));
+  }
+  NVFP4_DEV float value() const { return m; }
+};
+
+constexpr int kAmaxUnroll = 4;  // chunks per warp per iteration (amax)
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) group_amax_kernel(const __grid_constant__ GroupArgs a) {
   __shared__ unsigned s_max[kMaxGroup];
@@ -139,12 +173,12 @@ __global__ void __launch_bounds__(kThreads) group_amax_kernel(const __grid_const
   const int64_t c_end = c_begin + per_cta < a.total_chunks ? c_begin + per_cta : a.total_chunks;
   int cur = 0;
   int mt = -1;      // tensor of the running max
-  float m = 0.0f;   // running max of this lane
-  for (int64_t c0 = c_begin + wid * kQUnroll; c0 < c_end; c0 += kWarps * kQUnroll) {
-    Block16<T> in[kQUnroll];
-    int tid[kQUnroll];
+  LaneMax<T> m;     // running max of this lane
+  for (int64_t c0 = c_begin + wid * kAmaxUnroll; c0 < c_end; c0 += kWarps * kAmaxUnroll) {
+    Block16<T> in[kAmaxUnroll];
+    int tid[kAmaxUnroll];
 #pragma unroll
-    for (int u = 0; u < kQUnroll; ++u) {
+    for (int u = 0; u < kAmaxUnroll; ++u) {
       const int64_t c = c0 + u;
       in[u].zero();
       tid[u] = -1;
@@ -158,21 +192,18 @@ __global__ void __launch_bounds__(kThreads) group_amax_kernel(const __grid_const
       }
     }
 #pragma unroll
-    for (int u = 0; u < kQUnroll; ++u) {
+    for (int u = 0; u < kAmaxUnroll; ++u) {
       if (tid[u] < 0) continue;  // warp-uniform
       if (tid[u] != mt) {         // warp-uniform: flush the previous tensor's max
-        const float w = warp_max(m);
+        const float w = warp_max(m.value());
         if (lane == 0 && mt >= 0 && w > 0.0f) atomicMax(s_max + mt, __float_as_uint(w));
-        m = 0.0f;
+        m.reset();
         mt = tid[u];
       }
-      float v[16];
-      in[u].to_f32(v);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+      m.add(in[u]);
     }
   }
-  const float w = warp_max(m);
+  const float w = warp_max(m.value());
   if (lane == 0 && mt >= 0 && w > 0.0f) atomicMax(s_max + mt, __float_as_uint(w));
   __syncthreads();
   for (int i = threadIdx.x; i < a.n; i += kThreads)
@@ -189,6 +220,42 @@ NVFP4_DEV float tensor_scale_of(const GroupArgs& a, int t) {
   return __ldg(a.t[t].ts);
 }
 
+// Encode one 16-element block of tensor g at (row, col) and write its
+// outputs: block scale s_b = E4M3(max|x| / (6 s_g)) (or the frozen one),
+// d = s_b s_g, codes E2M1(x / d), and per OUT the packed codes and / or the
+// dequantized values.
+template <typename T, Out OUT>
+NVFP4_DEV void emit_block(const GroupArgs& a, const GTensor& g, int64_t row, int64_t col, const float (&v)[16],
+                          float sg, float denom6, bool frozen_all, uint32_t sb_frozen) {
+  uint32_t lo, hi;
+  float d;
+  const uint32_t sb = encode_block16<sizeof(T) == 2>(v, sg, denom6, frozen_all, sb_frozen, lo, hi, d);
+  if (OUT != Out::Fake) {
+    uint8_t* dst = g.codes + row * g.ld_out + (col >> 1);
+    if (a.out_wide) {
+      st_stream_v2(dst, lo, hi);
+    } else {
+      st_stream_u32(dst, lo);
+      st_stream_u32(dst + 4, hi);
+    }
+  }
+  if (OUT != Out::Codes) {
+    float o[16];
+    decode_block16(lo, hi, d, o);
+    Block16<T>::store(reinterpret_cast<T*>(g.y) + row * g.ld_y + col, o, a.y_wide != 0);
+  }
+  if (!frozen_all && g.sb != nullptr) {
+    const int64_t kb = col >> 4;
+    const int64_t off = (a.layout == NVFP4_SCALES_MMA) ? mma_scale_offset(row, kb, g.kchunks)
+                                                       : row * (g.cols >> 4) + kb;
+    g.sb[off] = (uint8_t)sb;
+  }
+}
+
+// Warps take groups of kQUnroll consecutive chunks, grid-striding (the
+// chunks in flight at any time form one dense front through memory).  The
+// position of a group's first chunk costs one division; the rest of the
+// group follows by increments.
 template <typename T, Out OUT>
 __global__ void __launch_bounds__(kThreads) group_encode_kernel(const __grid_constant__ GroupArgs a) {
   const int lane = threadIdx.x & 31;
@@ -202,71 +269,60 @@ __global__ void __launch_bounds__(kThreads) group_encode_kernel(const __grid_con
   int sg_t = -1;  // tensor whose scale is cached below
   float sg = 0.0f, denom6 = 0.0f;
   for (int64_t c0 = warp * kQUnroll; c0 < a.total_chunks; c0 += nwarps * kQUnroll) {
+    cur = find_tensor(a, c0, cur);
+    int t = cur;
+    uint32_t row, ci;
+    {
+      const uint32_t local = (uint32_t)(c0 - a.t[t].chunk0);
+      row = fastdiv(local, a.t[t].cpr);
+      ci = local - row * a.t[t].cpr.d;
+    }
     Block16<T> in[kQUnroll];
     uint32_t sb_in[kQUnroll];
     int tid[kQUnroll];
     int64_t row_[kQUnroll], col_[kQUnroll];
 #pragma unroll
     for (int u = 0; u < kQUnroll; ++u) {
-      const int64_t c = c0 + u;
       in[u].zero();
       sb_in[u] = 0u;
       tid[u] = -1;
       row_[u] = 0;
       col_[u] = 0;
-      if (c < a.total_chunks) {
-        cur = find_tensor(a, c, cur);
-        const GTensor& g = a.t[cur];
-        int64_t row, col;
-        chunk_pos(g, c, lane, row, col);
-        tid[u] = cur;
+      if (c0 + u < a.total_chunks) {
+        const GTensor& g = a.t[t];
+        const int64_t col = (int64_t)ci * kQChunk + lane * 16;
+        tid[u] = t;
         row_[u] = row;
         col_[u] = col;
         if (col < g.cols) {
-          in[u].load(reinterpret_cast<const T*>(g.x) + row * g.ld_x + col, a.x_wide != 0);
-          if (frozen_all) sb_in[u] = (uint32_t)__ldg(g.sb + row * (g.cols >> 4) + (col >> 4));
+          in[u].load(reinterpret_cast<const T*>(g.x) + (int64_t)row * g.ld_x + col, a.x_wide != 0);
+          if (frozen_all) sb_in[u] = (uint32_t)__ldg(g.sb + (int64_t)row * (g.cols >> 4) + (col >> 4));
+        }
+        // next chunk: along the row, then the next row, then the next tensor
+        if (++ci == g.cpr.d) {
+          ci = 0;
+          if (++row == (uint32_t)g.rows) {
+            row = 0;
+            ++t;
+          }
         }
       }
     }
 #pragma unroll
     for (int u = 0; u < kQUnroll; ++u) {
-      const int t = tid[u];
-      if (t < 0) continue;  // warp-uniform: the whole chunk is past the end
-      const GTensor& g = a.t[t];
-      const int64_t row = row_[u], col = col_[u];
+      const int tu = tid[u];
+      if (tu < 0) continue;  // warp-uniform: past the end of the group
+      const GTensor& g = a.t[tu];
+      const int64_t row_u = row_[u], col = col_[u];
       if (col >= g.cols) continue;  // this lane's block lies past the row end
-      if (t != sg_t) {
-        sg = tensor_scale_of(a, t);
+      if (tu != sg_t) {
+        sg = tensor_scale_of(a, tu);
         denom6 = __fmul_rn(6.0f, sg);
-        sg_t = t;
+        sg_t = tu;
       }
       float v[16];
       in[u].to_f32(v);
-      // ---- block scale s_b = E4M3(max|x| / (6 s_g)), d = s_b s_g, codes E2M1(x / d)
-      uint32_t lo, hi;
-      float d;
-      const uint32_t sb = encode_block16<sizeof(T) == 2>(v, sg, denom6, frozen_all, sb_in[u], lo, hi, d);
-      // ---- outputs
-      if (OUT != Out::Fake) {
-        uint8_t* dst = g.codes + row * g.ld_out + (col >> 1);
-        if (a.out_wide) {
-          st_stream_v2(dst, lo, hi);
-        } else {
-          st_stream_u32(dst, lo);
-          st_stream_u32(dst + 4, hi);
-        }
-      }
-      if (OUT != Out::Codes) {
-        float o[16];
-        decode_block16(lo, hi, d, o);
-        Block16<T>::store(reinterpret_cast<T*>(g.y) + row * g.ld_y + col, o, a.y_wide != 0);
-      }
-      if (!frozen_all && g.sb != nullptr) {
-        const int64_t kb = col >> 4;
-        const int64_t off = (a.layout == NVFP4_SCALES_MMA) ? mma_scale_offset(row, kb, g.kchunks)
-                                                           : row * (g.cols >> 4) + kb;
-        g.sb[off] = (uint8_t)sb;
-      }
+      emit_block<T, OUT>(a, g, row_u, col, v, sg, denom6, frozen_all, sb_in[u]);
     }
   }
 }
@@ -416,11 +472,6 @@ static nvfp4_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
-// In DYNAMIC mode the amax pass and the encode pass of a group run back to
-// back; groups are cut so that their inputs fit in L2 (126 MB on B200) and the
-// encode pass re-reads them from L2 rather than HBM.  A tensor larger than
-// this budget forms a group of its own.
-constexpr int64_t kL2GroupBytes = 48ll << 20;
 constexpr size_t kDynamicWorkspace = 1024;  // 256 amax words, >= kMaxGroup
 
 // Validate one tensor of a (possibly grouped) quantize / fake-quant call.
@@ -539,7 +590,6 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
   a.x_wide = 1;
   a.out_wide = 1;
   a.y_wide = 1;
-  int64_t group_bytes = 0;
   // DYNAMIC: every group takes its own amax words from the workspace; the
   // words are cleared once per call, and again whenever they run out.
   unsigned* words = reinterpret_cast<unsigned*>(ws);
@@ -547,12 +597,13 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
   int word_base = nwords;  // forces a clear before the first group
   auto flush = [&]() -> nvfp4_status {
     if (a.n == 0) return NVFP4_OK;
-    if (mode == NVFP4_DYNAMIC && word_base + a.n > nwords) {
+    const int need = a.n;
+    if (mode == NVFP4_DYNAMIC && word_base + need > nwords) {
       if (cudaMemsetAsync(ws, 0, kDynamicWorkspace, s) != cudaSuccess) return NVFP4_ERR_CUDA;
       word_base = 0;
     }
     nvfp4_status st = launch_group<OUT>(a, dtype, words + word_base, s);
-    word_base += a.n;
+    word_base += need;
     return st;
   };
   for (int i = 0; i < n; ++i) {
@@ -562,11 +613,8 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
         return NVFP4_ERR_CUDA;
       continue;
     }
-    const int64_t bytes = r.rows * r.cols * esz;
     if (r.rows * ((r.cols + kQChunk - 1) / kQChunk) > 0xFFFFFFFFll) return NVFP4_ERR_SHAPE;
-    const bool full = a.n == kMaxGroup;
-    const bool over_l2 = mode == NVFP4_DYNAMIC && a.n > 0 && group_bytes + bytes > kL2GroupBytes;
-    if (full || over_l2) {
+    if (a.n == kMaxGroup) {
       nvfp4_status st = flush();
       if (st != NVFP4_OK) return st;
       a.n = 0;
@@ -574,7 +622,6 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
       a.x_wide = 1;
       a.out_wide = 1;
       a.y_wide = 1;
-      group_bytes = 0;
     }
     GTensor& g = a.t[a.n++];
     g.x = r.x;
@@ -588,10 +635,10 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
     g.cols = r.cols;
     const int64_t cpr = (r.cols + kQChunk - 1) / kQChunk;
     g.cpr = make_fastdiv((uint32_t)cpr);
+    g.rows = r.rows;
     g.chunk0 = a.total_chunks;
     g.kchunks = (r.cols / 16 + 3) / 4;
     a.total_chunks += r.rows * cpr;
-    group_bytes += bytes;
     // 32-byte rows for 256-bit input loads; 8-byte code rows / 32-byte y rows
     if (((uintptr_t)r.x & 31u) || ((r.ld_x * esz) & 31)) a.x_wide = 0;
     if (OUT != Out::Fake && (((uintptr_t)r.out & 7u) || (r.ld_out & 7))) a.out_wide = 0;

@@ -262,9 +262,10 @@ def test_weight_sweep_full_size_parity():
 
 
 def test_grouped_quantize_matches_oracle_and_single_calls():
-    # mixed shapes, an empty tensor, more tensors than one launch holds and a
-    # tensor larger than one L2-sized group
-    shapes = [(64, 1024), (0, 32), (3, 48), (130, 1040)] + [(40, 256)] * 150 + [(6000, 2048)]
+    # mixed shapes, an empty tensor, more tensors than one launch holds, and
+    # large tensors among small ones
+    shapes = [(64, 1024), (4001, 272), (2048, 4096), (0, 32), (3, 48), (130, 1040)] + [(40, 256)] * 150 + \
+        [(6000, 2048)]
     xs = [S.weights(r, c, seed=100 + i, device=DEV, outlier_p=0.01, outlier_mult=40) for i, (r, c) in enumerate(shapes)]
     for mode in [Q.DYNAMIC, Q.FROZEN_GLOBAL, Q.FROZEN_ALL]:
         if mode == Q.DYNAMIC:
@@ -280,7 +281,7 @@ def test_grouped_quantize_matches_oracle_and_single_calls():
                                                       block_scales=ref_sb if mode == Q.FROZEN_ALL else None)
         torch.cuda.synchronize()
         for i, x in enumerate(xs):
-            if i % 7 != 0 and i not in (1, 2, 3, len(xs) - 1):
+            if i % 7 != 0 and i not in (1, 2, 3, 4, 5, len(xs) - 1):
                 continue
             xh = _host_f32(x)
             if mode == Q.DYNAMIC:
@@ -314,6 +315,10 @@ def test_launch_counter_counts_kernels():
     Q.nvfp4_quantize(x)                      # amax + encode
     Q.nvfp4_quantize(x, Q.FROZEN_GLOBAL, tensor_scale=torch.ones(1, device=DEV))  # encode
     assert Q.nvfp4_launch_count() - n0 == 3
+    xs = [S.activations(16, 64, seed=3 + i, device=DEV) for i in range(150)]   # two groups
+    n0 = Q.nvfp4_launch_count()
+    Q.nvfp4_quantize_grouped(xs)
+    assert Q.nvfp4_launch_count() - n0 == 4
 
 
 def test_unaligned_rows_use_narrow_accesses():
