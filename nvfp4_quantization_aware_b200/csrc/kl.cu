@@ -19,10 +19,12 @@
 //      Y = sum 2^d_t (d_t - d_s) relative to those maxima (rescaled when a
 //      maximum grows), merged across the CTA and then pushed into every peer's
 //      shared memory: one cluster barrier per row;
-//   3. dLogits from the on-chip slice, 16-byte stores.  Of the two
-//      exponentials per logit pair here, one runs on the MUFU unit and one as
-//      a polynomial on the FMA pipe, so that the MUFU unit (16 results per SM
-//      and clock) does not cap the kernel below the HBM rate.
+//   3. dLogits from the on-chip slice, 16-byte stores.
+// The element arithmetic of the bf16 path uses the paired binary32
+// operations of sm_100 (two logits per instruction) and the MUFU unit for
+// all four exponentials per logit pair: the kernel is bound by instruction
+// issue and the MUFU unit together, and a polynomial exponential on the FMA
+// pipe measured slower than the MUFU one.
 // Work is in the log2 domain: w = z * log2(e) / T, d = w - max w.  Per-row KL
 // goes to the workspace; a second one-CTA kernel sums the rows in a fixed
 // order (in double) into the mean, so the loss is deterministic.
@@ -63,6 +65,37 @@ NVFP4_DEV float exp2_poly(float x) {
   p = fmaf(p, f, 1.0000001192092896f);
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
+
+// ---- paired binary32 arithmetic (sm_100 .f32x2: two lanes per instruction,
+// each rounded like the scalar operation); a pair is a 64-bit register with
+// the first element in the low half.
+typedef unsigned long long f32x2;
+
+NVFP4_DEV f32x2 pair(float lo, float hi) {
+  return ((f32x2)__float_as_uint(hi) << 32) | (f32x2)__float_as_uint(lo);
+}
+NVFP4_DEV float lo_of(f32x2 v) { return __uint_as_float((uint32_t)(v & 0xFFFFFFFFull)); }
+NVFP4_DEV float hi_of(f32x2 v) { return __uint_as_float((uint32_t)(v >> 32)); }
+NVFP4_DEV f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+NVFP4_DEV f32x2 add2(f32x2 a, f32x2 b) {
+  f32x2 r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+NVFP4_DEV f32x2 sub2(f32x2 a, f32x2 b) {
+  f32x2 r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// the two bf16 of a word (element 2i low) as a pair of floats
+NVFP4_DEV f32x2 bf16x2_pair(uint32_t w) {
+  return ((f32x2)(w & 0xFFFF0000u) << 32) | (f32x2)(w << 16);
+}
+NVFP4_DEV f32x2 ex2_pair(f32x2 x) { return pair(ex2(lo_of(x)), ex2(hi_of(x))); }
 
 // Running softmax statistics of a (teacher, student) pair of rows, in the
 // log2 domain, relative to the running maxima mt and ms:
@@ -268,16 +301,35 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
         stats_rebase(my, zmt * a, zms * a);
       }
       const float nMt = -my.mt, nMs = -my.ms;
-      float zt[V8], zs[V8];
-      E::unpack(rt, zt);
-      E::unpack(rs, zs);
+      if constexpr (sizeof(T) == 2) {
+        // two logits of each row per paired operation; the pair sums are
+        // folded into the thread's statistics once per vector
+        const uint32_t wt[4] = {rt.x, rt.y, rt.z, rt.w}, ws[4] = {rs.x, rs.y, rs.z, rs.w};
+        const f32x2 A = pair(a, a), NT = pair(nMt, nMt), NS = pair(nMs, nMs);
+        f32x2 St2 = 0ull, Ss2 = 0ull, Y2 = 0ull;
 #pragma unroll
-      for (int j = 0; j < V8; ++j) {
-        const float dt = fmaf(zt[j], a, nMt), ds = fmaf(zs[j], a, nMs);
-        const float et = ex2(dt), es = ex2(ds);
-        my.St += et;
-        my.Ss += es;
-        my.Y = fmaf(et, dt - ds, my.Y);
+        for (int j = 0; j < 4; ++j) {
+          const f32x2 dt = fma2(bf16x2_pair(wt[j]), A, NT), ds = fma2(bf16x2_pair(ws[j]), A, NS);
+          const f32x2 et = ex2_pair(dt), es = ex2_pair(ds);
+          St2 = add2(St2, et);
+          Ss2 = add2(Ss2, es);
+          Y2 = fma2(et, sub2(dt, ds), Y2);
+        }
+        my.St += lo_of(St2) + hi_of(St2);
+        my.Ss += lo_of(Ss2) + hi_of(Ss2);
+        my.Y += lo_of(Y2) + hi_of(Y2);
+      } else {
+        float zt[V8], zs[V8];
+        E::unpack(rt, zt);
+        E::unpack(rs, zs);
+#pragma unroll
+        for (int j = 0; j < V8; ++j) {
+          const float dt = fmaf(zt[j], a, nMt), ds = fmaf(zs[j], a, nMs);
+          const float et = ex2(dt), es = ex2(ds);
+          my.St += et;
+          my.Ss += es;
+          my.Y = fmaf(et, dt - ds, my.Y);
+        }
       }
     }
   }
@@ -315,14 +367,30 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
     const int kfirst = (off + V8 - 1) / V8;          // first vector with no leading pad
     const int klast = nslots / V8;                   // vectors [kfirst, klast) are all real
     for (int k = threadIdx.x; k < nvec; k += kKlThreads) {
-      float zt[V8], zs[V8], o[V8];
-      E::unpack(vt[k], zt);
-      E::unpack(vs[k], zs);
+      float o[V8];
+      if constexpr (sizeof(T) == 2) {
+        const uint4 rt = vt[k], rs = vs[k];
+        const uint32_t wt[4] = {rt.x, rt.y, rt.z, rt.w}, ws[4] = {rs.x, rs.y, rs.z, rs.w};
+        const f32x2 A = pair(a, a), NLt = pair(-Lt, -Lt), NLs = pair(-Ls, -Ls), G = pair(gm, gm);
 #pragma unroll
-      for (int j = 0; j < V8; ++j) {
-        const float pt = exp2_poly(fmaf(zt[j], a, -Lt));
-        const float ps = ex2(fmaf(zs[j], a, -Ls));
-        o[j] = fold ? ps - pt : gm * (ps - pt);
+        for (int j = 0; j < 4; ++j) {
+          const f32x2 pt = ex2_pair(fma2(bf16x2_pair(wt[j]), A, NLt));
+          const f32x2 ps = ex2_pair(fma2(bf16x2_pair(ws[j]), A, NLs));
+          f32x2 d = sub2(ps, pt);
+          if (!fold) d = fma2(d, G, 0ull);
+          o[2 * j] = lo_of(d);
+          o[2 * j + 1] = hi_of(d);
+        }
+      } else {
+        float zt[V8], zs[V8];
+        E::unpack(vt[k], zt);
+        E::unpack(vs[k], zs);
+#pragma unroll
+        for (int j = 0; j < V8; ++j) {
+          const float pt = exp2_poly(fmaf(zt[j], a, -Lt));
+          const float ps = ex2(fmaf(zs[j], a, -Ls));
+          o[j] = fold ? ps - pt : gm * (ps - pt);
+        }
       }
       const int j0 = k * V8;
       if (vec_ok && k >= kfirst && k < klast) {
