@@ -206,26 +206,25 @@ struct KlArgs {
 // underflows to 0.
 constexpr float kPadLogit = -0x1p100f;
 
+// Geometry of a CTA's slice of one row in shared memory: slot j holds logit
+// v0 + j - off for off <= j < nslots; the other slots of [0, cap) hold the
+// pad value.
+struct KlSliceGeom {
+  int off, nslots, nvec, cap;
+};
+
+// Stages the slice [v0, v0 + n) of row `row` of the teacher and the student
+// into st / ss: the 16-byte-aligned interior by TMA bulk copies (completion
+// on `bar`, bounded wait; *s_ok = 0 if it expired), the head and tail by
+// plain loads.  Called by every thread of the CTA (contains barriers).
 template <typename T>
-__global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
+NVFP4_DEV KlSliceGeom kl_stage_slice(const KlArgs& args, int64_t row, int64_t v0, int n, T* st, T* ss,
+                                     uint64_t* bar_, int* s_ok_) {
   using E = KlElem<T>;
-  constexpr int V8 = E::kVec;        // elements per 16-byte vector
+  constexpr int V8 = E::kVec;
   constexpr int ESZ = (int)sizeof(T);
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  __shared__ uint64_t bar;
-  __shared__ KlStats warp_stats[kKlWarps];
-  __shared__ KlStats peer_stats[kKlMaxCluster];  // written by every CTA of the cluster
-  __shared__ int s_ok;
-
-  cg::cluster_group cluster = cg::this_cluster();
-  const int csize = (int)cluster.num_blocks();
-  const int crank = (int)cluster.block_rank();
-  const int64_t row = blockIdx.x / csize;
-  const int64_t v0 = (int64_t)crank * args.slice;
-  int64_t v1 = v0 + args.slice;
-  if (v1 > args.vocab) v1 = args.vocab;
-  const int n = v1 > v0 ? (int)(v1 - v0) : 0;
-
+  uint64_t& bar = *bar_;
+  int& s_ok = *s_ok_;
   const T* gt = reinterpret_cast<const T*>(args.teacher) + row * args.ld + v0;
   const T* gs = reinterpret_cast<const T*>(args.student) + row * args.ld + v0;
   // Teacher and student rows share one stride, so they share an alignment:
@@ -240,9 +239,6 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
   const int nslots = off + n;
   const int nvec = (nslots + V8 - 1) / V8;    // vectors covering the slice
   const int cap = nvec * V8;                  // slots actually used
-
-  T* st = reinterpret_cast<T*>(smem_raw);
-  T* ss = st + args.slice + 2 * V8;
 
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
@@ -279,6 +275,39 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
   }
   if (nint > 0 && !mbar_wait_bounded(&bar, 0)) s_ok = 0;
   __syncthreads();
+
+  KlSliceGeom g;
+  g.off = off;
+  g.nslots = nslots;
+  g.nvec = nvec;
+  g.cap = cap;
+  return g;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
+  using E = KlElem<T>;
+  constexpr int V8 = E::kVec;        // elements per 16-byte vector
+  constexpr int ESZ = (int)sizeof(T);
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  __shared__ uint64_t bar;
+  __shared__ KlStats warp_stats[kKlWarps];
+  __shared__ KlStats peer_stats[kKlMaxCluster];  // written by every CTA of the cluster
+  __shared__ int s_ok;
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int csize = (int)cluster.num_blocks();
+  const int crank = (int)cluster.block_rank();
+  const int64_t row = blockIdx.x / csize;
+  const int64_t v0 = (int64_t)crank * args.slice;
+  int64_t v1 = v0 + args.slice;
+  if (v1 > args.vocab) v1 = args.vocab;
+  const int n = v1 > v0 ? (int)(v1 - v0) : 0;
+
+  T* st = reinterpret_cast<T*>(smem_raw);
+  T* ss = st + args.slice + 2 * V8;
+  const KlSliceGeom geo = kl_stage_slice<T>(args, row, v0, n, st, ss, &bar, &s_ok);
+  const int off = geo.off, nslots = geo.nslots, nvec = geo.nvec;
   const bool ok = s_ok != 0;
 
   const uint4* vt = reinterpret_cast<const uint4*>(st);
