@@ -540,6 +540,23 @@ nvfp4_status qad_kl_fwd_bwd(const void* teacher, const void* student, nvfp4_dtyp
                             void* stream);
 
 /* ------------------------------------------------------------------------
+ * Top-k KL distillation loss (Qwen3.6-35B-A3B W4A4 tutorial, section "3.
+ * QAD": --logit_kl_topk 4096): per row, S = the teacher's k largest logits
+ * (among equal logits the smaller vocabulary index first; k >= vocab selects
+ * the whole row), both softmaxes renormalised over S:
+ *   row_kl[i]    = sum_{v in S} p_t^S (log p_t^S - log p_s^S)
+ *   *loss        = (1/rows) * sum_i row_kl[i]
+ *   dlogits[i,v] = grad_scale * (p_s^S[v] - p_t^S[v]) / T on S, 0 elsewhere
+ * Arguments as qad_kl_fwd_bwd, plus k >= 1 (NVFP4_ERR_ARG otherwise); same
+ * workspace (qad_kl_workspace_size).  S is found by a radix select over the
+ * teacher logits held on chip; each logit is read from memory once.
+ * ------------------------------------------------------------------------ */
+nvfp4_status qad_kl_topk_fwd_bwd(const void* teacher, const void* student, nvfp4_dtype dtype,
+                                 int64_t rows, int64_t vocab, int64_t ld, int64_t k, float temperature,
+                                 float* loss, float* row_kl, void* dlogits, int64_t ld_grad,
+                                 float grad_scale, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * qad_kl_fwd_bwd without a workspace argument, for callers that cannot
  * allocate device memory when they compute the loss (a framework whose
  * caching allocator holds the device budget, a fixed pre-planned memory

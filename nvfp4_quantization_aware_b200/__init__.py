@@ -45,5 +45,6 @@ from .binding import (  # noqa: F401
     nvfp4_quantize,
     nvfp4_selftest_division,
     qad_kl_fwd_bwd,
+    qad_kl_topk_fwd_bwd,
 )
 from .autograd import FakeQuantSTE, KLDistillLoss, fake_quant_ste, kl_distill_loss  # noqa: F401

@@ -196,6 +196,7 @@ struct KlArgs {
   float* row_kl;          // workspace, rows floats
   void* dlogits;          // may be NULL
   int64_t ld_grad;
+  int64_t topk;           // top-k kernel: entries of the teacher's top set per row
 };
 
 // Stand-in for positions of the shared-memory slice that hold no logit (the
@@ -433,6 +434,303 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
   }
 }
 
+// ------------------------------------------------------------------ top-k KL
+//
+// The distillation loss restricted to the teacher's top-k vocabulary entries
+// of each row (Qwen3.6-35B-A3B W4A4 tutorial, section "3. QAD":
+// --logit_kl_topk 4096), both softmaxes renormalised over that set S, ties
+// broken by the smaller vocabulary index; the gradient is zero outside S.
+// Same cluster-per-row layout as kl_row_kernel.  S is found by a radix
+// select over order-preserving integer keys of the teacher logits held in
+// shared memory: one 8-bit digit per pass (2 passes for bf16, 4 for f32),
+// each pass a CTA histogram (warp-aggregated atomics) summed over the
+// cluster through distributed shared memory; that yields the k-th key tau
+// and how many keys equal to tau belong to S.  When not all of them do, a
+// scan over the slice in index order (and over the cluster's CTAs in rank
+// order) ranks them.  The statistics and the gradient then run over S only.
+
+template <typename T>
+struct KlKey;
+template <>
+struct KlKey<__nv_bfloat16> {
+  static constexpr int kBits = 16;
+  static constexpr int kPerWord = 2;
+  NVFP4_DEV static uint32_t key(uint32_t w, int h) {  // element h of a 32-bit word
+    const uint32_t u = h ? (w >> 16) : (w & 0xFFFFu);
+    return (u & 0x8000u) ? (~u & 0xFFFFu) : (u | 0x8000u);
+  }
+};
+template <>
+struct KlKey<float> {
+  static constexpr int kBits = 32;
+  static constexpr int kPerWord = 1;
+  NVFP4_DEV static uint32_t key(uint32_t w, int) { return (w & 0x80000000u) ? ~w : (w | 0x80000000u); }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
+  using E = KlElem<T>;
+  using Kf = KlKey<T>;
+  constexpr int V8 = E::kVec;
+  constexpr int PASSES = Kf::kBits / 8;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  __shared__ uint64_t bar;
+  __shared__ int s_ok;
+  __shared__ unsigned hist[256];
+  __shared__ unsigned recv[2][kKlMaxCluster][256];  // written by every CTA of the cluster
+  __shared__ unsigned recv_ties[kKlMaxCluster];
+  __shared__ unsigned warp_sum[kKlWarps];
+  __shared__ unsigned s_digit, s_remaining, s_count;
+  __shared__ KlStats warp_stats[kKlWarps];
+  __shared__ KlStats peer_stats[kKlMaxCluster];
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int csize = (int)cluster.num_blocks();
+  const int crank = (int)cluster.block_rank();
+  const int64_t row = blockIdx.x / csize;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t v0 = (int64_t)crank * args.slice;
+  int64_t v1 = v0 + args.slice;
+  if (v1 > args.vocab) v1 = args.vocab;
+  const int n = v1 > v0 ? (int)(v1 - v0) : 0;
+
+  T* st = reinterpret_cast<T*>(smem_raw);
+  T* ss = st + args.slice + 2 * V8;
+  const int nvec_max = (int)((args.slice + 2 * V8) / V8);
+  unsigned* vec_prefix = reinterpret_cast<unsigned*>(ss + args.slice + 2 * V8);
+  uint8_t* sel_mask = reinterpret_cast<uint8_t*>(vec_prefix + nvec_max);
+  const KlSliceGeom geo = kl_stage_slice<T>(args, row, v0, n, st, ss, &bar, &s_ok);
+  const int off = geo.off, nslots = geo.nslots, nvec = geo.nvec;
+  const bool ok = s_ok != 0;
+  const uint32_t* wt = reinterpret_cast<const uint32_t*>(st);  // words of the teacher slice
+  constexpr int WPV = 16 / 4;                                   // words per 16-byte vector
+
+  // ---- radix select of the k-th largest key over the row
+  const uint32_t kk = (uint32_t)(args.topk < args.vocab ? args.topk : args.vocab);
+  uint32_t prefix = 0, remaining = kk, count = 0;
+  for (int p = 0; p < PASSES; ++p) {
+    const int shift = Kf::kBits - 8 * (p + 1);  // digit position
+    hist[threadIdx.x] = 0u;
+    __syncthreads();
+    if (ok) {
+      for (int kb = 0; kb < nvec; kb += kKlThreads) {  // warp-uniform trip count
+        const int k = kb + (int)threadIdx.x;
+#pragma unroll
+        for (int q = 0; q < WPV; ++q) {
+          const uint32_t w = k < nvec ? wt[k * WPV + q] : 0u;
+#pragma unroll
+          for (int h = 0; h < Kf::kPerWord; ++h) {
+            const int j = k * V8 + q * Kf::kPerWord + h;  // slot
+            const uint32_t key = Kf::key(w, h);
+            const bool valid = k < nvec && j >= off && j < nslots &&
+                               (p == 0 || (key >> (shift + 8)) == prefix);
+            const unsigned any = __ballot_sync(0xFFFFFFFFu, valid);
+            if (any == 0u) continue;
+            const uint32_t digit = (key >> shift) & 0xFFu;
+            const unsigned grp = __match_any_sync(0xFFFFFFFFu, valid ? digit : 256u + (uint32_t)lane);
+            if (valid && (__ffs(grp) - 1) == lane) atomicAdd(&hist[digit], (unsigned)__popc(grp));
+          }
+        }
+      }
+    }
+    __syncthreads();
+    {
+      const unsigned v = hist[threadIdx.x];
+      for (int r = 0; r < csize; ++r) cluster.map_shared_rank(&recv[p & 1][0][0], r)[crank * 256 + threadIdx.x] = v;
+    }
+    cluster.sync();
+    {
+      unsigned tot = 0u;
+      for (int r = 0; r < csize; ++r) tot += recv[p & 1][r][threadIdx.x];
+      hist[threadIdx.x] = tot;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      // from the largest digit down: the digit whose bucket holds the remaining-th key
+      unsigned cum = 0u, d = 0u;
+      for (int dd = 255; dd >= 0; --dd) {
+        if (cum + hist[dd] >= remaining) {
+          d = (unsigned)dd;
+          break;
+        }
+        cum += hist[dd];
+      }
+      s_digit = d;
+      s_remaining = remaining - cum;
+      s_count = hist[d];
+    }
+    __syncthreads();
+    prefix = (prefix << 8) | s_digit;
+    remaining = s_remaining;  // keys equal to the prefix so far still to take
+    count = s_count;          // keys equal to the prefix so far
+    __syncthreads();          // hist, s_* are rewritten by the next pass
+  }
+  const uint32_t tau = prefix;
+  const uint32_t m_ties = remaining;          // keys == tau that belong to S
+  const bool rank_ties = m_ties < count;      // uniform across the cluster
+
+  // ---- ranks of the keys equal to tau, in index order (only when not all are taken)
+  unsigned cta_off = 0u;
+  if (rank_ties) {
+    unsigned running = 0u;
+    for (int kb = 0; kb < nvec; kb += kKlThreads) {
+      const int k = kb + (int)threadIdx.x;
+      unsigned c = 0u;
+      if (ok && k < nvec) {
+#pragma unroll
+        for (int q = 0; q < WPV; ++q) {
+          const uint32_t w = wt[k * WPV + q];
+#pragma unroll
+          for (int h = 0; h < Kf::kPerWord; ++h) {
+            const int j = k * V8 + q * Kf::kPerWord + h;
+            c += (j >= off && j < nslots && Kf::key(w, h) == tau) ? 1u : 0u;
+          }
+        }
+      }
+      // exclusive scan of c over the round's threads (index order)
+      unsigned x = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane == 31) warp_sum[wid] = x;
+      __syncthreads();
+      unsigned before = 0u, total = 0u;
+      for (int w = 0; w < kKlWarps; ++w) {
+        if (w < wid) before += warp_sum[w];
+        total += warp_sum[w];
+      }
+      if (k < nvec) vec_prefix[k] = running + before + x - c;
+      running += total;
+      __syncthreads();
+    }
+    for (int r = (int)threadIdx.x; r < csize; r += kKlThreads)
+      cluster.map_shared_rank(recv_ties, r)[crank] = running;
+    cluster.sync();
+    for (int r = 0; r < crank; ++r) cta_off += recv_ties[r];
+  }
+  // ---- selection mask per vector (bit e: element e of the vector is in S)
+  for (int k = (int)threadIdx.x; k < nvec; k += kKlThreads) {
+    unsigned mask = 0u, seen = 0u;
+    if (ok) {
+#pragma unroll
+      for (int q = 0; q < WPV; ++q) {
+        const uint32_t w = wt[k * WPV + q];
+#pragma unroll
+        for (int h = 0; h < Kf::kPerWord; ++h) {
+          const int e = q * Kf::kPerWord + h;
+          const int j = k * V8 + e;
+          if (j < off || j >= nslots) continue;
+          const uint32_t key = Kf::key(w, h);
+          if (key > tau) {
+            mask |= 1u << e;
+          } else if (key == tau) {
+            const bool take = !rank_ties || cta_off + vec_prefix[k] + seen < m_ties;
+            if (take) mask |= 1u << e;
+            ++seen;
+          }
+        }
+      }
+    }
+    sel_mask[k] = (uint8_t)mask;
+  }
+  __syncthreads();
+
+  // ---- online statistics over S (other slots read as the pad value)
+  const uint4* vt = reinterpret_cast<const uint4*>(st);
+  const uint4* vs = reinterpret_cast<const uint4*>(ss);
+  const float a = args.a;
+  KlStats my;
+  stats_init(my, kPadLogit * a);
+  float zmt = kPadLogit, zms = kPadLogit;
+  if (ok) {
+    for (int k = (int)threadIdx.x; k < nvec; k += kKlThreads) {
+      const unsigned mask = sel_mask[k];
+      if (mask == 0u) continue;
+      float zt[V8], zs[V8];
+      E::unpack(vt[k], zt);
+      E::unpack(vs[k], zs);
+      float lt = kPadLogit, ls = kPadLogit;
+#pragma unroll
+      for (int e = 0; e < V8; ++e) {
+        if (!((mask >> e) & 1u)) {
+          zt[e] = kPadLogit;
+          zs[e] = kPadLogit;
+        }
+        lt = fmaxf(lt, zt[e]);
+        ls = fmaxf(ls, zs[e]);
+      }
+      if (lt > zmt || ls > zms) {
+        zmt = fmaxf(zmt, lt);
+        zms = fmaxf(zms, ls);
+        stats_rebase(my, zmt * a, zms * a);
+      }
+      const float nMt = -my.mt, nMs = -my.ms;
+#pragma unroll
+      for (int e = 0; e < V8; ++e) {
+        const float dt = fmaf(zt[e], a, nMt), ds = fmaf(zs[e], a, nMs);
+        const float et = ex2(dt), es = ex2(ds);
+        my.St += et;
+        my.Ss += es;
+        my.Y = fmaf(et, dt - ds, my.Y);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) my = stats_merge(my, stats_shfl_xor(my, o));
+  if (lane == 0) warp_stats[wid] = my;
+  __syncthreads();
+  if (threadIdx.x < csize) {
+    KlStats c = warp_stats[0];
+    for (int w = 1; w < kKlWarps; ++w) c = stats_merge(c, warp_stats[w]);
+    cluster.map_shared_rank(peer_stats, (int)threadIdx.x)[crank] = c;
+  }
+  cluster.sync();  // all pushes visible; no CTA touches a peer after this point
+  KlStats rs_ = peer_stats[0];
+  for (int r = 1; r < csize; ++r) rs_ = stats_merge(rs_, peer_stats[r]);
+  const float Wt = rs_.mt, Ws = rs_.ms, St = rs_.St, Ss = rs_.Ss;
+  if (crank == 0 && threadIdx.x == 0) {
+    const float kl = 0.69314718055994531f * (rs_.Y / St + log2f(Ss / St));
+    args.row_kl[row] = ok ? kl : __int_as_float(0x7FC00000);
+  }
+
+  // ---- dLogits: gscale (p_s^S - p_t^S) on S, 0 elsewhere
+  if (args.dlogits != nullptr && ok) {
+    const float g = args.gscale;
+    const float Lt = Wt + __log2f(St), Ls = Ws + __log2f(Ss);
+    T* gout = reinterpret_cast<T*>(args.dlogits) + row * args.ld_grad + v0 - off;  // slot j -> gout[j]
+    const bool vec_ok = (((uintptr_t)gout) & 15u) == 0;
+    const int kfirst = (off + V8 - 1) / V8;
+    const int klast = nslots / V8;
+    for (int k = (int)threadIdx.x; k < nvec; k += kKlThreads) {
+      const unsigned mask = sel_mask[k];
+      float o[V8];
+      if (mask == 0u) {
+#pragma unroll
+        for (int e = 0; e < V8; ++e) o[e] = 0.0f;
+      } else {
+        float zt[V8], zs[V8];
+        E::unpack(vt[k], zt);
+        E::unpack(vs[k], zs);
+#pragma unroll
+        for (int e = 0; e < V8; ++e) {
+          const float pt = ex2(fmaf(zt[e], a, -Lt)), ps = ex2(fmaf(zs[e], a, -Ls));
+          o[e] = ((mask >> e) & 1u) ? g * (ps - pt) : 0.0f;
+        }
+      }
+      const int j0 = k * V8;
+      if (vec_ok && k >= kfirst && k < klast) {
+        st_stream_v4(gout + j0, E::pack(o));
+      } else {
+#pragma unroll
+        for (int e = 0; e < V8; ++e)
+          if (j0 + e >= off && j0 + e < nslots) E::store1(gout + j0 + e, o[e]);
+      }
+    }
+  }
+}
+
 // loss = mean of row_kl in a fixed order (double accumulation); optionally
 // copies the per-row values to the caller's buffer.
 __global__ void __launch_bounds__(1024) kl_mean_kernel(const float* __restrict__ row_kl, int64_t rows,
@@ -500,6 +798,28 @@ static cudaError_t launch_kl(const KlArgs& a, const KlPlan& p, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, kl_row_kernel<T>, a);
 }
 
+template <typename T>
+static cudaError_t launch_kl_topk(const KlArgs& a, const KlPlan& p, cudaStream_t s) {
+  const int vec = 16 / (int)sizeof(T);
+  const size_t nvec_max = (size_t)((p.slice + 2 * vec) / vec);
+  const size_t smem = p.smem + nvec_max * 5;  // + per-vector tie prefix (u32) and selection mask (u8)
+  cudaError_t e = cudaFuncSetAttribute(kl_topk_row_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(a.rows * p.cluster));
+  cfg.blockDim = dim3(kKlThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kl_topk_row_kernel<T>, a);
+}
+
 }  // namespace nvfp4
 
 using namespace nvfp4;
@@ -546,7 +866,50 @@ nvfp4_status qad_kl_fwd_bwd(const void* teacher, const void* student, nvfp4_dtyp
   args.row_kl = reinterpret_cast<float*>(workspace);
   args.dlogits = dlogits;
   args.ld_grad = ld_grad;
+  args.topk = vocab;
   cudaError_t e = dtype == NVFP4_BF16 ? launch_kl<__nv_bfloat16>(args, plan, s) : launch_kl<float>(args, plan, s);
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  kl_mean_kernel<<<1, 1024, 0, s>>>(args.row_kl, rows, loss, row_kl);
+  count_launches(2);
+  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+nvfp4_status qad_kl_topk_fwd_bwd(const void* teacher, const void* student, nvfp4_dtype dtype, int64_t rows,
+                                 int64_t vocab, int64_t ld, int64_t k, float temperature, float* loss,
+                                 float* row_kl, void* dlogits, int64_t ld_grad, float grad_scale, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (dtype != NVFP4_BF16 && dtype != NVFP4_F32) return NVFP4_ERR_DTYPE;
+  if (!(temperature > 0.0f) || !loss || k < 1) return NVFP4_ERR_ARG;
+  if (rows < 0 || vocab <= 0 || ld < vocab) return NVFP4_ERR_SHAPE;
+  if (dlogits && ld_grad < vocab) return NVFP4_ERR_SHAPE;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (rows == 0) return cudaMemsetAsync(loss, 0, sizeof(float), s) == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+  if (!teacher || !student) return NVFP4_ERR_ARG;
+  if (rows > 0x7FFFFFFFll / kKlMaxCluster) return NVFP4_ERR_SHAPE;
+  const int esz = dtype == NVFP4_BF16 ? 2 : 4;
+  if (((uintptr_t)teacher ^ (uintptr_t)student) & 15u) return NVFP4_ERR_ALIGN;
+  if (((uintptr_t)teacher | (uintptr_t)student) % esz) return NVFP4_ERR_ALIGN;
+  if (dlogits && ((uintptr_t)dlogits % esz)) return NVFP4_ERR_ALIGN;
+  const size_t need = qad_kl_workspace_size(rows, vocab, dtype);
+  if (!workspace || workspace_bytes < need) return NVFP4_ERR_WORKSPACE;
+  if (((uintptr_t)workspace & 15u) != 0) return NVFP4_ERR_ALIGN;
+  KlPlan plan;
+  if (!kl_plan(vocab, esz, plan)) return NVFP4_ERR_UNSUPPORTED;
+  KlArgs args;
+  args.teacher = teacher;
+  args.student = student;
+  args.rows = rows;
+  args.vocab = vocab;
+  args.ld = ld;
+  args.slice = plan.slice;
+  args.a = 1.4426950408889634f / temperature;
+  args.gscale = grad_scale / temperature;
+  args.row_kl = reinterpret_cast<float*>(workspace);
+  args.dlogits = dlogits;
+  args.ld_grad = ld_grad;
+  args.topk = k;
+  cudaError_t e =
+      dtype == NVFP4_BF16 ? launch_kl_topk<__nv_bfloat16>(args, plan, s) : launch_kl_topk<float>(args, plan, s);
   if (e != cudaSuccess) return NVFP4_ERR_CUDA;
   kl_mean_kernel<<<1, 1024, 0, s>>>(args.row_kl, rows, loss, row_kl);
   count_launches(2);
