@@ -14,8 +14,8 @@ and the KL distillation loss (same article, "QAD的工作原理").
 
 Parity status of each function (what pins it is in the tests under
 ``tests/test_oracle_*.py``): e2m1/e4m3 encode and decode, bf16 rounding,
-quantize, dequantize, fake_quant, swizzled_scale_offset, gemm_w4a4 and kl are
-all pinned; none is "parity unpinned".
+quantize, dequantize, fake_quant, swizzled_scale_offset, gemm_w4a4, kl and
+calibrate_mse are all pinned; none is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_gemm_w4a4.restype = ctypes.c_int
         L.oracle_gemm_w4a4_rows.argtypes = [c_p, c_p, c_f, c_p, c_p, c_f, c_i64, c_i64, c_p, c_i64, c_p]
         L.oracle_gemm_w4a4_rows.restype = ctypes.c_int
+        L.oracle_calibrate_mse.argtypes = [c_p, c_i64, c_i64, c_i64, c_f, c_p, c_p]
+        L.oracle_calibrate_mse.restype = ctypes.c_int
         L.oracle_kl.argtypes = [c_p, c_p, c_i64, c_i64, c_i64, c_d, c_d, c_p, c_p, c_p, c_p, ctypes.c_int]
         L.oracle_kl.restype = ctypes.c_int
         L.oracle_set_threads.argtypes = [ctypes.c_int]
@@ -213,6 +215,17 @@ def fake_quant(x: np.ndarray, mode: int = DYNAMIC, s_g: float | None = None,
     _check(lib().oracle_fake_quant(_ptr(x), rows, cols, cols, mode, _ptr(sg), _ptr(sb), _ptr(codes),
                                    _ptr(f32), _ptr(b16)), "fake_quant")
     return f32, b16, sb, float(sg[0])
+
+
+def calibrate_mse(x: np.ndarray, s_g: float):
+    """MSE block-scale calibration with the tensor scale s_g given.
+    Returns (s_b uint8 [rows, cols/16], least squared error float32 per block)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    rows, cols = x.shape
+    sb = np.zeros((rows, cols // 16), dtype=np.uint8)
+    err = np.zeros((rows, cols // 16), dtype=np.float32)
+    _check(lib().oracle_calibrate_mse(_ptr(x), rows, cols, cols, float(s_g), _ptr(sb), _ptr(err)), "calibrate_mse")
+    return sb, err
 
 
 def gemm_w4a4(a_codes, a_sb, a_sg, b_codes, b_sb, b_sg, K: int) -> np.ndarray:

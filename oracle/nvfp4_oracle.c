@@ -290,6 +290,56 @@ int oracle_fake_quant(const float* x, int64_t rows, int64_t cols, int64_t ld, in
 }
 
 /* ------------------------------------------------------------------------ */
+/* MSE block-scale calibration for frozen-scale QAD.                          */
+/* ------------------------------------------------------------------------ */
+
+/* Frozen-scale QAD starts from scales an MSE calibration chose (Nemotron 3.5
+ * Lightning article, "量化尺度处理策略"); the page gives no formula beyond
+ * "MSE".  Reading: with the tensor scale s_g given, every block's E4M3 scale
+ * is the code c (all 127 finite non-negative codes, in increasing order)
+ * whose fake quantization of the block has the least squared error
+ *   err(c) = sum_i (x_i - x^_i)^2,  x^_i = value(q_i) * d,  d = value(c) * s_g,
+ *   q_i = E2M1_RNE_sat(x_i / d)  (q_i = 0 for every i when d == 0),
+ * each operation in binary32 with one rounding, the sum accumulated in
+ * element order as err = fma(diff, diff, err); the smallest code wins a tie.
+ * s_b: rows x cols/16 (output); err_out (may be NULL): the least error per
+ * block. */
+int oracle_calibrate_mse(const float* x, int64_t rows, int64_t cols, int64_t ld, float s_g, uint8_t* s_b,
+                         float* err_out) {
+  if (rows < 0 || cols < 0 || cols % 16 != 0 || ld < cols) return ORACLE_ERR_SHAPE;
+  if (rows > 0 && (!x || !s_b)) return ORACLE_ERR_ARG;
+  const int64_t nblk = cols / 16;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t b = 0; b < nblk; ++b) {
+      const float* xb = x + r * ld + b * 16;
+      int best = 0;
+      float best_err = INFINITY;
+      for (int c = 0; c < 127; ++c) {
+        const float d = (float)oracle_e4m3_value(c) * s_g; /* binary32 product */
+        float err = 0.0f;
+        for (int i = 0; i < 16; ++i) {
+          float xh = 0.0f;
+          if (d != 0.0f) {
+            const float q = xb[i] / d; /* binary32 quotient */
+            xh = (float)oracle_e2m1_value(oracle_e2m1_encode(q)) * d;
+          }
+          const float diff = xb[i] - xh;
+          err = fmaf(diff, diff, err);
+        }
+        if (err < best_err) {
+          best_err = err;
+          best = c;
+        }
+      }
+      s_b[r * nblk + b] = (uint8_t)best;
+      if (err_out) err_out[r * nblk + b] = best_err;
+    }
+  }
+  return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Block-scale layout used by the block-scaled tensor-core MMA.             */
 /* ------------------------------------------------------------------------ */
 
