@@ -15,6 +15,8 @@ Also measured in the same run and reported under "gemm" and "kl":
     weights 4096 x 4096 pre-quantized, bf16 out -- TFLOP/s;
   * KL distillation loss + dLogits over 16384 x 131072 bf16 teacher/student
     logits -- tokens/s and GB/s (6 B per logit);
+  * the top-k KL loss (key "kl_topk"): the same logits, k = 4096 per row;
+  * the MSE block-scale calibration of the 128 expert weights ("calibrate_mse");
   * the MoE layer step (config "moe_step"): 4096 tokens, 128 routed experts
     + 1 shared, top-6, forward (grouped W4A4) + straight-through backward
     (BF16) -- tokens/s and per-phase times.
@@ -255,6 +257,8 @@ def run_ours(args, world, rank, local):
     if not args.no_secondary:
         secondary["gemm"] = bench_gemm(Q, dev, stream, P, max(3, min(K, 20)))
         secondary["kl"] = bench_kl(Q, dev, stream, P, max(3, min(K, 10)))
+        secondary["kl_topk"] = bench_kl_topk(Q, dev, stream, P, max(3, min(K, 10)))
+        secondary["calibrate_mse"] = bench_calibrate(Q, dev, stream, xs, 3)
         secondary["moe_step"] = bench_moe(Q, dev, stream, P, max(3, min(K, 10)))
     clocks = sampler.stop()
 
@@ -502,6 +506,67 @@ def bench_moe(Q, dev, stream, P, K):
     del d, w, step, x, y, dx, dwg, dwu, dwd, dcw
     torch.cuda.empty_cache()
     return out
+
+
+def bench_kl_topk(Q, dev, stream, P, K, k=4096):
+    """Top-k KL over the distillation logits (k = 4096 of 131072): each logit
+    is still read once and every dLogit written (zero outside the set), so the
+    algorithmic bytes are those of the full loss."""
+    from nvfp4_quantization_aware_b200 import synthetic as S
+    with torch.cuda.stream(stream):
+        d = S.distill_logits(seed=0, device=dev)
+        t, s = d["teacher"], d["student"]
+        rows, V = t.shape
+        grad = torch.empty_like(s)
+        loss = torch.empty(1, dtype=torch.float32, device=dev)
+        ws = torch.empty(int(Q.lib().qad_kl_workspace_size(rows, V, Q.BF16)), dtype=torch.uint8, device=dev)
+        L = Q.lib()
+        sptr = stream.cuda_stream
+
+        def call():
+            st = L.qad_kl_topk_fwd_bwd(t.data_ptr(), s.data_ptr(), Q.BF16, rows, V, V, k, 1.0, loss.data_ptr(), None,
+                                       grad.data_ptr(), V, 1.0 / rows, ws.data_ptr(), ws.numel(), sptr)
+            assert st == 0, st
+
+        for _ in range(3):
+            call()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            call()
+        e1.record(stream)
+        stream.synchronize()
+    ms = e0.elapsed_time(e1) / K
+    gbs = 6.0 * rows * V / (ms * 1e-3) / 1e9
+    del t, s, grad, d
+    torch.cuda.empty_cache()
+    return {"tokens_per_s": round(rows / (ms * 1e-3), 1), "ms": round(ms, 4), "gbs": round(gbs, 1), "k": k,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": P["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / P["hbm_gbs"], 4), "kernel": "kl_topk_row_kernel<bf16>",
+                         "algorithmic_bytes_per_launch": 6 * rows * V},
+            "config": "distillation logits 16384 x 131072 bf16 (as kl), KL over the teacher's top-4096 per row"}
+
+
+def bench_calibrate(Q, dev, stream, xs, K):
+    """MSE block-scale calibration of the 128 expert weights (the frozen
+    scales' starting point): elements per second and GB/s of input read."""
+    exp = xs[:128]
+    with torch.cuda.stream(stream):
+        _, _, ts = Q.nvfp4_quantize_grouped(exp, Q.DYNAMIC)
+        sbs = [torch.empty(x.shape[0], x.shape[1] // 16, dtype=torch.uint8, device=dev) for x in exp]
+        Q.nvfp4_calibrate_mse_grouped(exp, ts, block_scales=sbs)
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            Q.nvfp4_calibrate_mse_grouped(exp, ts, block_scales=sbs)
+        e1.record(stream)
+        stream.synchronize()
+    ms = e0.elapsed_time(e1) / K
+    n = sum(x.numel() for x in exp)
+    return {"ms": round(ms, 4), "gelem_per_s": round(n / (ms * 1e-3) / 1e9, 2),
+            "config": "128 expert weights 2048x1024 bf16, s_g from amax, exhaustive search over E4M3 block scales"}
 
 
 def cpu_baseline(xs):

@@ -211,6 +211,32 @@ nvfp4_status nvfp4_quantize_fake_quant_grouped(int num_tensors, const nvfp4_tens
                                                size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * MSE block-scale calibration (the starting scales of frozen-scale QAD,
+ * Nemotron 3.5 Lightning article, "量化尺度处理策略": the page names MSE
+ * calibration only).  With the tensor scale s_g given, each block's E4M3
+ * scale s_b is the code (of the 127 finite non-negative ones) whose fake
+ * quantization of the block has the least squared error
+ *   err = sum_i (x_i - value(q_i) * d)^2,  d = value(s_b) * s_g,
+ *   q_i = E2M1_RNE_sat(x_i / d) (all 0 when d = 0),
+ * binary32 operations rounded once, the sum accumulated in element order
+ * with FMA; a tie goes to the smaller code.  The result is meant for
+ * FROZEN_ALL quantization.
+ *   x             rows x cols (bf16 or f32), row stride ld_x
+ *   tensor_scale  one float (device, read)
+ *   block_scales  rows x cols/16 ROWMAJOR (device, written)
+ *   block_err     rows x cols/16 floats (device), the least error, or NULL
+ * ------------------------------------------------------------------------ */
+nvfp4_status nvfp4_calibrate_mse(const void* x, nvfp4_dtype dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                                 const float* tensor_scale, uint8_t* block_scales, float* block_err,
+                                 void* stream);
+
+/* Grouped form: tensors[i].tensor_scale is read, tensors[i].block_scales
+ * written (ROWMAJOR), .out / .ld_out unused; block_err: HOST array of
+ * num_tensors device pointers (entries may be NULL), or NULL. */
+nvfp4_status nvfp4_calibrate_mse_grouped(int num_tensors, const nvfp4_tensor_ref* tensors, nvfp4_dtype dtype,
+                                         float* const* block_err, void* stream);
+
+/* ------------------------------------------------------------------------
  * Fake quantization: y = dequantize(quantize(x)) in one pass, the simulated
  * quantization every student forward pass goes through (Nemotron 3.5
  * Lightning article, "QAD的工作原理").  Bitwise equal to nvfp4_quantize

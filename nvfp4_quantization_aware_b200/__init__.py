@@ -46,5 +46,7 @@ from .binding import (  # noqa: F401
     nvfp4_selftest_division,
     qad_kl_fwd_bwd,
     qad_kl_topk_fwd_bwd,
+    nvfp4_calibrate_mse,
+    nvfp4_calibrate_mse_grouped,
 )
 from .autograd import FakeQuantSTE, KLDistillLoss, fake_quant_ste, kl_distill_loss  # noqa: F401

@@ -123,6 +123,10 @@ def lib() -> ctypes.CDLL:
                                                     ctypes.POINTER(i64), i32, i32, i32, p, sz, p]
     L.nvfp4_quantize_fake_quant_grouped.restype = i32
     L.nvfp4_fake_quant_grouped.restype = i32
+    L.nvfp4_calibrate_mse.argtypes = [p, i32, i64, i64, i64, p, p, p, p]
+    L.nvfp4_calibrate_mse.restype = i32
+    L.nvfp4_calibrate_mse_grouped.argtypes = [i32, ctypes.POINTER(TensorRef), i32, ctypes.POINTER(p), p]
+    L.nvfp4_calibrate_mse_grouped.restype = i32
     L.nvfp4_selftest_division.argtypes = [p, p, p]
     L.nvfp4_selftest_division.restype = i32
     L.nvfp4_gemm_workspace_size.argtypes = [i64, i64, i64]
@@ -627,3 +631,37 @@ def qad_kl_topk_fwd_bwd(teacher: torch.Tensor, student: torch.Tensor, k: int, te
                                0 if workspace is None else workspace.numel(), _stream(dev))
     _check(st, "qad_kl_topk_fwd_bwd")
     return loss, row_kl, dlogits
+
+
+# ------------------------------------------------------------------ MSE calibration
+
+def nvfp4_calibrate_mse(x: torch.Tensor, tensor_scale: torch.Tensor, want_err: bool = False):
+    """Block scales (ROWMAJOR uint8 [rows, cols/16]) minimising each block's
+    squared fake-quantization error for the given tensor scale; with
+    want_err, also the least error per block (f32)."""
+    _cuda2d(x, "x")
+    rows, cols = x.shape
+    sb = torch.empty(rows, cols // 16, dtype=torch.uint8, device=x.device)
+    err = torch.empty(rows, cols // 16, dtype=torch.float32, device=x.device) if want_err else None
+    st = lib().nvfp4_calibrate_mse(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(tensor_scale), _ptr(sb),
+                                   _ptr(err), _stream(x.device))
+    _check(st, "nvfp4_calibrate_mse")
+    return (sb, err) if want_err else sb
+
+
+def nvfp4_calibrate_mse_grouped(xs, tensor_scales, block_scales=None):
+    """Grouped form over a list of tensors (one tensor scale each)."""
+    n = len(xs)
+    dev = xs[0].device
+    ts_list = [tensor_scales[i:i + 1] for i in range(n)] if isinstance(tensor_scales, torch.Tensor) else list(tensor_scales)
+    if block_scales is None:
+        block_scales = [torch.empty(x.shape[0], x.shape[1] // 16, dtype=torch.uint8, device=dev) for x in xs]
+    dummy = [torch.empty(0, dtype=torch.uint8, device=dev)] * n
+    arr = (TensorRef * n)()
+    for i, x in enumerate(xs):
+        _cuda2d(x, f"tensor {i}")
+        arr[i] = TensorRef(x.data_ptr(), x.shape[0], x.shape[1], x.stride(0), ts_list[i].data_ptr(),
+                           block_scales[i].data_ptr(), None, 0)
+    st = lib().nvfp4_calibrate_mse_grouped(n, arr, _dtype_code(xs[0]), None, _stream(dev))
+    _check(st, "nvfp4_calibrate_mse_grouped")
+    return block_scales

@@ -327,6 +327,83 @@ __global__ void __launch_bounds__(kThreads) group_encode_kernel(const __grid_con
   }
 }
 
+// ------------------------------------------------------------------ MSE calibration
+//
+// Frozen-scale QAD starts from MSE-calibrated scales (Nemotron 3.5 Lightning
+// NVFP4 article, "量化尺度处理策略").  With each tensor's s_g given, a
+// block's E4M3 scale is the code c (all 127 finite non-negative codes) whose
+// fake quantization has the least squared error
+//   err(c) = sum_i (x_i - value(q_i) d)^2,  d = value(c) s_g,  q_i = E2M1(x_i / d),
+// binary32 operations rounded once, accumulated in element order with FMA,
+// ties to the smaller code.  Codes whose d makes every quotient round to 0
+// (max|x| / d <= 1/4) reproduce code 0's error exactly (x - (+-0) = x), so
+// the search stops at the first of them.  One lane per block; the tensor's
+// GTensor.y receives the least error per block (f32, rows x cols/16) when set.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) group_calib_kernel(const __grid_constant__ GroupArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * kWarps;
+  int cur = 0;
+  for (int64_t c = warp; c < a.total_chunks; c += nwarps) {
+    cur = find_tensor(a, c, cur);
+    const GTensor& g = a.t[cur];
+    int64_t row, col;
+    chunk_pos(g, c, lane, row, col);
+    if (col >= g.cols) continue;
+    Block16<T> in;
+    in.load(reinterpret_cast<const T*>(g.x) + row * g.ld_x + col, a.x_wide != 0);
+    float v[16];
+    in.to_f32(v);
+    const float sg = __ldg(g.ts);
+    float amax = 0.0f, err0 = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      amax = fmaxf(amax, fabsf(v[i]));
+      err0 = __fmaf_rn(v[i], v[i], err0);  // code 0 (d = 0): every x^ is 0
+    }
+    uint32_t best = 0u;
+    float best_err = err0;
+    for (uint32_t code = 1; code < 127u; ++code) {
+      const float d = __fmul_rn(e4m3_decode(code), sg);
+      if (d == 0.0f) continue;  // same error as code 0 (a tie: the smaller code stays)
+      const bool fast = sizeof(T) == 2 && block_scale_in_fast_range(d);
+      const float r = fast ? __frcp_rn(d) : 0.0f;
+      const float qmax = fast ? div_by_block_scale(amax, d, r) : __fdiv_rn(amax, d);
+      if (qmax <= 0.25f) break;  // this code and every larger one: all quotients round to 0
+      float q[16];
+      if (fast) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) q[i] = div_by_block_scale(v[i], d, r);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(v[i], d);
+      }
+      float q0[8], q1[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        q0[i] = q[i];
+        q1[i] = q[8 + i];
+      }
+      float xh[16];
+      decode_block16(e2m1x8_encode(q0), e2m1x8_encode(q1), d, xh);
+      float err = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float diff = __fsub_rn(v[i], xh[i]);
+        err = __fmaf_rn(diff, diff, err);
+      }
+      if (err < best_err) {
+        best_err = err;
+        best = code;
+      }
+    }
+    const int64_t kb = col >> 4;
+    g.sb[row * (g.cols >> 4) + kb] = (uint8_t)best;
+    if (g.y) reinterpret_cast<float*>(g.y)[row * (g.cols >> 4) + kb] = best_err;
+  }
+}
+
 // Zero the padding bytes of an MMA-layout scale array (rows beyond `rows`,
 // blocks beyond cols/16).  One thread per padded (row, block) slot.
 __global__ void zero_mma_padding_kernel(uint8_t* __restrict__ s, int64_t rows, int64_t nblk,
@@ -733,6 +810,87 @@ nvfp4_status nvfp4_quantize_fake_quant_grouped(int num_tensors, const nvfp4_tens
                                                void* stream) {
   return run_tensors<Out::Both>(num_tensors, tensors, dtype, mode, layout, workspace, workspace_bytes,
                                 (cudaStream_t)stream, y, ld_y);
+}
+
+nvfp4_status nvfp4_calibrate_mse_grouped(int num_tensors, const nvfp4_tensor_ref* tensors, nvfp4_dtype dtype,
+                                         float* const* block_err, void* stream) {
+  if (num_tensors < 0 || (num_tensors > 0 && !tensors)) return NVFP4_ERR_ARG;
+  if (dtype != NVFP4_BF16 && dtype != NVFP4_F32) return NVFP4_ERR_DTYPE;
+  for (int i = 0; i < num_tensors; ++i) {
+    const nvfp4_tensor_ref& r = tensors[i];
+    nvfp4_status st = check_common(r.x, dtype, r.rows, r.cols, r.ld_x);
+    if (st != NVFP4_OK) return st;
+    if (r.rows == 0 || r.cols == 0) continue;
+    if (!r.tensor_scale || !r.block_scales) return NVFP4_ERR_ARG;
+    if (block_err && block_err[i] && ((uintptr_t)block_err[i] & 3u)) return NVFP4_ERR_ALIGN;
+  }
+  const int64_t esz = dtype == NVFP4_BF16 ? 2 : 4;
+  cudaStream_t s = (cudaStream_t)stream;
+  static GroupArgs a;
+  auto launch = [&]() -> nvfp4_status {
+    if (a.n == 0 || a.total_chunks == 0) return NVFP4_OK;
+    const void* fn = dtype == NVFP4_BF16 ? (const void*)group_calib_kernel<__nv_bfloat16>
+                                         : (const void*)group_calib_kernel<float>;
+    int64_t grid = (a.total_chunks + kWarps - 1) / kWarps;
+    const int64_t cap = (int64_t)sm_count() * resident_per_sm(fn);
+    if (grid > cap) grid = cap;
+    if (dtype == NVFP4_BF16)
+      group_calib_kernel<__nv_bfloat16><<<(int)grid, kThreads, 0, s>>>(a);
+    else
+      group_calib_kernel<float><<<(int)grid, kThreads, 0, s>>>(a);
+    count_launches(1);
+    return launch_status();
+  };
+  a.n = 0;
+  a.total_chunks = 0;
+  a.mode = NVFP4_FROZEN_GLOBAL;
+  a.layout = NVFP4_SCALES_ROWMAJOR;
+  a.x_wide = 1;
+  for (int i = 0; i < num_tensors; ++i) {
+    const nvfp4_tensor_ref& r = tensors[i];
+    if (r.rows == 0 || r.cols == 0) continue;
+    if (r.rows * ((r.cols + kQChunk - 1) / kQChunk) > 0xFFFFFFFFll) return NVFP4_ERR_SHAPE;
+    if (a.n == kMaxGroup) {
+      nvfp4_status st = launch();
+      if (st != NVFP4_OK) return st;
+      a.n = 0;
+      a.total_chunks = 0;
+      a.x_wide = 1;
+    }
+    GTensor& g = a.t[a.n++];
+    g.x = r.x;
+    g.codes = nullptr;
+    g.y = block_err ? block_err[i] : nullptr;
+    g.sb = r.block_scales;
+    g.ts = r.tensor_scale;
+    g.ld_x = r.ld_x;
+    g.ld_out = 0;
+    g.ld_y = 0;
+    g.cols = r.cols;
+    g.rows = r.rows;
+    const int64_t cpr = (r.cols + kQChunk - 1) / kQChunk;
+    g.cpr = make_fastdiv((uint32_t)cpr);
+    g.chunk0 = a.total_chunks;
+    g.kchunks = (r.cols / 16 + 3) / 4;
+    a.total_chunks += r.rows * cpr;
+    if (((uintptr_t)r.x & 31u) || ((r.ld_x * esz) & 31)) a.x_wide = 0;
+  }
+  return launch();
+}
+
+nvfp4_status nvfp4_calibrate_mse(const void* x, nvfp4_dtype dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                                 const float* tensor_scale, uint8_t* block_scales, float* block_err, void* stream) {
+  nvfp4_tensor_ref r;
+  r.x = x;
+  r.rows = rows;
+  r.cols = cols;
+  r.ld_x = ld_x;
+  r.tensor_scale = const_cast<float*>(tensor_scale);
+  r.block_scales = block_scales;
+  r.out = nullptr;
+  r.ld_out = 0;
+  float* errs[1] = {block_err};
+  return nvfp4_calibrate_mse_grouped(1, &r, dtype, errs, stream);
 }
 
 nvfp4_status nvfp4_fake_quant_grouped(int num_tensors, const nvfp4_tensor_ref* tensors, nvfp4_dtype dtype,
