@@ -211,6 +211,22 @@ nvfp4_status nvfp4_quantize_fake_quant_grouped(int num_tensors, const nvfp4_tens
                                                size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Tensor max and tensor scale as separate steps, for a tensor whose rows are
+ * spread over several GPUs: each rank takes the max of its rows, the ranks
+ * combine the maxima with an all-reduce(max), and every rank then derives
+ * the same s_g = amax / 2688 and quantizes its rows in FROZEN_GLOBAL mode --
+ * the same codes and scales as a DYNAMIC call on the whole tensor.
+ *   nvfp4_tensor_amax_grouped: amax[i] = max |x_i| (device, num_tensors floats;
+ *     0 for an empty tensor); tensors[i].tensor_scale / block_scales / out are
+ *     not used.
+ *   nvfp4_global_scale_from_amax: tensor_scale[i] = amax[i] / 2688 (binary32
+ *     division, as in DYNAMIC mode).
+ * ------------------------------------------------------------------------ */
+nvfp4_status nvfp4_tensor_amax_grouped(int num_tensors, const nvfp4_tensor_ref* tensors, nvfp4_dtype dtype,
+                                       float* amax, void* stream);
+nvfp4_status nvfp4_global_scale_from_amax(const float* amax, int n, float* tensor_scale, void* stream);
+
+/* ------------------------------------------------------------------------
  * MSE block-scale calibration (the starting scales of frozen-scale QAD,
  * Nemotron 3.5 Lightning article, "量化尺度处理策略": the page names MSE
  * calibration only).  With the tensor scale s_g given, each block's E4M3

@@ -123,6 +123,10 @@ def lib() -> ctypes.CDLL:
                                                     ctypes.POINTER(i64), i32, i32, i32, p, sz, p]
     L.nvfp4_quantize_fake_quant_grouped.restype = i32
     L.nvfp4_fake_quant_grouped.restype = i32
+    L.nvfp4_tensor_amax_grouped.argtypes = [i32, ctypes.POINTER(TensorRef), i32, p, p]
+    L.nvfp4_tensor_amax_grouped.restype = i32
+    L.nvfp4_global_scale_from_amax.argtypes = [p, i32, p, p]
+    L.nvfp4_global_scale_from_amax.restype = i32
     L.nvfp4_calibrate_mse.argtypes = [p, i32, i64, i64, i64, p, p, p, p]
     L.nvfp4_calibrate_mse.restype = i32
     L.nvfp4_calibrate_mse_grouped.argtypes = [i32, ctypes.POINTER(TensorRef), i32, ctypes.POINTER(p), p]

@@ -404,6 +404,12 @@ __global__ void __launch_bounds__(kThreads) group_calib_kernel(const __grid_cons
   }
 }
 
+// s_g[i] = amax[i] / 2688 (the DYNAMIC tensor scale from a given max).
+__global__ void global_scale_kernel(const float* __restrict__ amax, int n, float* __restrict__ s_g) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    s_g[i] = __fdiv_rn(amax[i], 2688.0f);
+}
+
 // Zero the padding bytes of an MMA-layout scale array (rows beyond `rows`,
 // blocks beyond cols/16).  One thread per padded (row, block) slot.
 __global__ void zero_mma_padding_kernel(uint8_t* __restrict__ s, int64_t rows, int64_t nblk,
@@ -876,6 +882,79 @@ nvfp4_status nvfp4_calibrate_mse_grouped(int num_tensors, const nvfp4_tensor_ref
     if (((uintptr_t)r.x & 31u) || ((r.ld_x * esz) & 31)) a.x_wide = 0;
   }
   return launch();
+}
+
+nvfp4_status nvfp4_tensor_amax_grouped(int num_tensors, const nvfp4_tensor_ref* tensors, nvfp4_dtype dtype,
+                                       float* amax, void* stream) {
+  if (num_tensors < 0 || (num_tensors > 0 && (!tensors || !amax))) return NVFP4_ERR_ARG;
+  if (dtype != NVFP4_BF16 && dtype != NVFP4_F32) return NVFP4_ERR_DTYPE;
+  if ((uintptr_t)amax & 3u) return NVFP4_ERR_ALIGN;
+  for (int i = 0; i < num_tensors; ++i) {
+    nvfp4_status st = check_common(tensors[i].x, dtype, tensors[i].rows, tensors[i].cols, tensors[i].ld_x);
+    if (st != NVFP4_OK) return st;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  if (num_tensors == 0) return NVFP4_OK;
+  // max |x| >= 0 compares like its bit pattern: the words start at 0 (= +0.0f)
+  if (cudaMemsetAsync(amax, 0, (size_t)num_tensors * sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  const int64_t esz = dtype == NVFP4_BF16 ? 2 : 4;
+  static GroupArgs a;
+  int first = 0;  // tensor index of a.t[0]
+  auto launch = [&]() -> nvfp4_status {
+    if (a.n == 0 || a.total_chunks == 0) return NVFP4_OK;
+    a.amax = reinterpret_cast<unsigned*>(amax) + first;
+    const void* fn = dtype == NVFP4_BF16 ? (const void*)group_amax_kernel<__nv_bfloat16>
+                                         : (const void*)group_amax_kernel<float>;
+    if (dtype == NVFP4_BF16)
+      group_amax_kernel<__nv_bfloat16><<<resident_grid(fn, a.total_chunks), kThreads, 0, s>>>(a);
+    else
+      group_amax_kernel<float><<<resident_grid(fn, a.total_chunks), kThreads, 0, s>>>(a);
+    count_launches(1);
+    return launch_status();
+  };
+  a.n = 0;
+  a.total_chunks = 0;
+  a.mode = NVFP4_DYNAMIC;
+  a.x_wide = 1;
+  // tensors map to consecutive words: a group holds consecutive tensors, empty ones included
+  for (int i = 0; i < num_tensors; ++i) {
+    const nvfp4_tensor_ref& r = tensors[i];
+    if (r.rows * ((r.cols + kQChunk - 1) / kQChunk) > 0xFFFFFFFFll) return NVFP4_ERR_SHAPE;
+    if (a.n == kMaxGroup) {
+      nvfp4_status st = launch();
+      if (st != NVFP4_OK) return st;
+      first = i;
+      a.n = 0;
+      a.total_chunks = 0;
+      a.x_wide = 1;
+    }
+    GTensor& g = a.t[a.n++];
+    g.x = r.x;
+    g.codes = nullptr;
+    g.y = nullptr;
+    g.sb = nullptr;
+    g.ts = nullptr;
+    g.ld_x = r.ld_x;
+    g.ld_out = 0;
+    g.ld_y = 0;
+    g.cols = r.cols > 0 ? r.cols : 16;
+    g.rows = r.cols > 0 ? r.rows : 0;
+    const int64_t cpr = (g.cols + kQChunk - 1) / kQChunk;
+    g.cpr = make_fastdiv((uint32_t)cpr);
+    g.chunk0 = a.total_chunks;
+    g.kchunks = (g.cols / 16 + 3) / 4;
+    a.total_chunks += g.rows * cpr;
+    if (((uintptr_t)r.x & 31u) || ((r.ld_x * esz) & 31)) a.x_wide = 0;
+  }
+  return launch();
+}
+
+nvfp4_status nvfp4_global_scale_from_amax(const float* amax, int n, float* tensor_scale, void* stream) {
+  if (n < 0 || (n > 0 && (!amax || !tensor_scale))) return NVFP4_ERR_ARG;
+  if (n == 0) return NVFP4_OK;
+  global_scale_kernel<<<(n + 255) / 256, 256, 0, (cudaStream_t)stream>>>(amax, n, tensor_scale);
+  count_launches(1);
+  return launch_status();
 }
 
 nvfp4_status nvfp4_calibrate_mse(const void* x, nvfp4_dtype dtype, int64_t rows, int64_t cols, int64_t ld_x,
