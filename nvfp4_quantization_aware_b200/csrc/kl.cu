@@ -443,7 +443,7 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
 // Same cluster-per-row layout as kl_row_kernel.  S is found by a radix
 // select over order-preserving integer keys of the teacher logits held in
 // shared memory: one 8-bit digit per pass (2 passes for bf16, 4 for f32),
-// each pass a CTA histogram (warp-aggregated atomics) summed over the
+// each pass a CTA histogram (shared-memory atomics) summed over the
 // cluster through distributed shared memory; that yields the k-th key tau
 // and how many keys equal to tau belong to S.  When not all of them do, a
 // scan over the slice in index order (and over the cluster's CTAs in rank
@@ -524,11 +524,7 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
             const uint32_t key = Kf::key(w, h);
             const bool valid = k < nvec && j >= off && j < nslots &&
                                (p == 0 || (key >> (shift + 8)) == prefix);
-            const unsigned any = __ballot_sync(0xFFFFFFFFu, valid);
-            if (any == 0u) continue;
-            const uint32_t digit = (key >> shift) & 0xFFu;
-            const unsigned grp = __match_any_sync(0xFFFFFFFFu, valid ? digit : 256u + (uint32_t)lane);
-            if (valid && (__ffs(grp) - 1) == lane) atomicAdd(&hist[digit], (unsigned)__popc(grp));
+            if (valid) atomicAdd(&hist[(key >> shift) & 0xFFu], 1u);
           }
         }
       }
