@@ -381,6 +381,30 @@ nvfp4_status nvfp4_gemm_bf16_grouped(int mode, int groups, const void* a, int a_
                                      int64_t M, int64_t N, int64_t K, void* c, int64_t ldc, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Weight-only NVFP4 GEMM (W4A16), the format of the Nemotron 3.5 Lightning
+ * checkpoint; the Qwen3.6-35B-A3B W4A4 tutorial (section "为什么目标是 W4A4
+ * 而不是 W4A16") contrasts it with W4A4: the weights are turned back into
+ * 16-bit values in the GEMM's main loop and the product runs at 16 bits.
+ *   C[M x N] = A[M x K] * W^[N x K]^T,  FP32 accumulation, bf16 output,
+ *   W^[n][k] = bf16(value(q[n][k]) * (value(s_b[n][k/16]) * s_g))
+ * (each product a binary32 multiply rounded once, then rounded to bf16:
+ * exactly the bf16 fake-quant weights of nvfp4_quantize_fake_quant).
+ *   a               bf16, row-major M x K, leading dimension lda (elements)
+ *   b_codes         W's E2M1 codes, N x K/2 bytes, row-major, contiguous
+ *                   (low nibble = even element)
+ *   b_scales        W's E4M3 block scales in NVFP4_SCALES_ROWMAJOR layout
+ *                   (N x K/16, contiguous)
+ *   b_tensor_scale  device pointer to W's FP32 tensor scale s_g
+ *   c               bf16, row-major M x N, leading dimension ldc (elements)
+ * K % 64 == 0; a 16-byte aligned with lda * 2 a multiple of 16; b_codes
+ * 16-byte aligned; b_scales and c 4-byte aligned.  One kernel launch;
+ * NVFP4_ERR_SHAPE / _ARG / _ALIGN on bad arguments (nothing launched).
+ * ------------------------------------------------------------------------ */
+nvfp4_status nvfp4_gemm_w4a16(const void* a, int64_t lda, const uint8_t* b_codes, const uint8_t* b_scales,
+                              const float* b_tensor_scale, int64_t M, int64_t N, int64_t K, void* c, int64_t ldc,
+                              void* stream);
+
+/* ------------------------------------------------------------------------
  * MoE layer of the QAD student: 128 routed experts plus one shared expert,
  * top-6 routing (Nemotron-3-Nano-30B NVFP4 article, "Was ist
  * Nemotron-Nano-3-30B-A3B-NVFP4?"), SwiGLU expert FFNs whose weights and

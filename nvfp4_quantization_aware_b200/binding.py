@@ -142,6 +142,8 @@ def lib() -> ctypes.CDLL:
     L.nvfp4_gemm_bf16_grouped.argtypes = [i32, i32, p, i32, i64, i64, i64, p, i32, i64, i64, i64, p, p, i64, i64,
                                           i64, p, i64, p]
     L.nvfp4_gemm_bf16_grouped.restype = i32
+    L.nvfp4_gemm_w4a16.argtypes = [p, i64, p, p, p, i64, i64, i64, p, i64, p]
+    L.nvfp4_gemm_w4a16.restype = i32
     L.qad_kl_workspace_size.argtypes = [i64, i64, i32]
     L.qad_kl_workspace_size.restype = sz
     L.qad_kl_fwd_bwd.argtypes = [p, p, i32, i64, i64, i64, f32, p, p, p, i64, f32, p, sz, p]
@@ -535,6 +537,28 @@ def nvfp4_gemm_bf16_grouped(mode: int, a: torch.Tensor, b: torch.Tensor, seg_off
                                        _ptr(b), int(b_mn_major), b.shape[0], b.shape[1], b.stride(0), _ptr(seg_off),
                                        _ptr(seg_len), M, N, K, _ptr(out), out.stride(0), _stream(dev))
     _check(st, "nvfp4_gemm_bf16_grouped")
+    return out
+
+
+def nvfp4_gemm_w4a16(a: torch.Tensor, b_codes: torch.Tensor, b_scales: torch.Tensor, b_tensor_scale: torch.Tensor,
+                     out: torch.Tensor | None = None) -> torch.Tensor:
+    """C = A W^T with A bf16 [M, K] and W NVFP4 (codes [N, K/2], ROWMAJOR block
+    scales [N, K/16], tensor scale [1]) dequantized inside the GEMM; bf16 [M, N]."""
+    _cuda2d(a, "a")
+    _cuda2d(b_codes, "b_codes")
+    if a.dtype != torch.bfloat16:
+        raise TypeError("a must be bfloat16")
+    M, K = a.shape
+    N = b_codes.shape[0]
+    if b_codes.shape[1] * 2 != K or not b_codes.is_contiguous() or not b_scales.is_contiguous():
+        raise ValueError("b_codes must be contiguous [N, K/2] and b_scales contiguous [N, K/16]")
+    if b_scales.numel() != N * (K // 16) or b_tensor_scale.dtype != torch.float32:
+        raise ValueError("b_scales must hold N * K/16 bytes and b_tensor_scale be float32")
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=a.device)
+    st = lib().nvfp4_gemm_w4a16(_ptr(a), a.stride(0), _ptr(b_codes), _ptr(b_scales), _ptr(b_tensor_scale), M, N, K,
+                                _ptr(out), out.stride(0), _stream(a.device))
+    _check(st, "nvfp4_gemm_w4a16")
     return out
 
 

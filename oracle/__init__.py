@@ -14,8 +14,8 @@ and the KL distillation loss (same article, "QAD的工作原理").
 
 Parity status of each function (what pins it is in the tests under
 ``tests/test_oracle_*.py``): e2m1/e4m3 encode and decode, bf16 rounding,
-quantize, dequantize, fake_quant, swizzled_scale_offset, gemm_w4a4, kl and
-calibrate_mse are all pinned; none is "parity unpinned".
+quantize, dequantize, fake_quant, swizzled_scale_offset, gemm_w4a4, gemm_w4a16,
+kl and calibrate_mse are all pinned; none is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -239,6 +239,18 @@ def gemm_w4a4(a_codes, a_sb, a_sg, b_codes, b_sb, b_sg, K: int) -> np.ndarray:
     _check(lib().oracle_gemm_w4a4(_ptr(a_codes), _ptr(a_sb), float(a_sg), _ptr(b_codes), _ptr(b_sb),
                                   float(b_sg), M, N, K, _ptr(c)), "gemm_w4a4")
     return c
+
+
+def gemm_w4a16(a: np.ndarray, b_codes, b_sb, b_sg: float, K: int) -> np.ndarray:
+    """Weight-only NVFP4 product in float64: C = A @ W_hat^T with A the bf16
+    activations (given as their exact float32/float64 values, M x K) and
+    W_hat the bf16 dequantized weights (N x K): value(q) * (s_b * s_g) in
+    binary32, rounded to bf16 -- the weights a bf16 fake-quant produces
+    (Qwen3.6-35B-A3B W4A4 tutorial, section "为什么目标是 W4A4 而不是 W4A16":
+    W4A16 multiplies 16-bit activations with weights dequantized to 16 bits)."""
+    _, w_bits = dequantize(b_codes, b_sb, b_sg, K)
+    w_hat = bf16_bits_to_f32(w_bits).astype(np.float64)
+    return np.asarray(a, dtype=np.float64) @ w_hat.T
 
 
 def gemm_w4a4_rows(a_codes, a_sb, a_sg, b_codes, b_sb, b_sg, K: int, rows) -> np.ndarray:
