@@ -16,6 +16,9 @@ Also measured in the same run and reported under "gemm" and "kl":
   * KL distillation loss + dLogits over 16384 x 131072 bf16 teacher/student
     logits -- tokens/s and GB/s (6 B per logit);
   * the top-k KL loss (key "kl_topk"): the same logits, k = 4096 per row;
+  * weight-only NVFP4 (key "w4a16"): the same GEMM shapes with bf16
+    activations, the weights dequantized in the main loop, beside W4A4 and
+    the BF16 GEMM of the dequantized weights;
   * the MSE block-scale calibration of the 128 expert weights ("calibrate_mse");
   * the MoE layer step (config "moe_step"): 4096 tokens, 128 routed experts
     + 1 shared, top-6, forward (grouped W4A4) + straight-through backward
@@ -256,6 +259,7 @@ def run_ours(args, world, rank, local):
     secondary = {}
     if not args.no_secondary:
         secondary["gemm"] = bench_gemm(Q, dev, stream, P, max(3, min(K, 20)))
+        secondary["w4a16"] = bench_w4a16(Q, dev, stream, P, max(3, min(K, 20)))
         secondary["kl"] = bench_kl(Q, dev, stream, P, max(3, min(K, 10)))
         secondary["kl_topk"] = bench_kl_topk(Q, dev, stream, P, max(3, min(K, 10)))
         secondary["calibrate_mse"] = bench_calibrate(Q, dev, stream, xs, 3)
@@ -384,6 +388,53 @@ def bench_gemm(Q, dev, stream, P, K):
                                          "peak_source": "4 x MEASURED_PEAKS bf16_tflops (nominal FP4:BF16 ratio)"
                                          if M >= 1024 else "MEASURED_PEAKS hbm_gbs"}}
     out["config"] = "x M x 4096 bf16 N(0,1)*LogNormal(0,1) per channel, dynamic NVFP4 on the fly; w 4096x4096 pre-quantized; L2 flushed before each step"
+    return out
+
+
+def bench_w4a16(Q, dev, stream, P, K):
+    """Weight-only NVFP4 (W4A16) against W4A4 and BF16 on the same 4096 x 4096
+    weights: W4A16 dequantizes the weights in its main loop and runs the BF16
+    tensor cores; the BF16 product of the already dequantized weights is timed
+    beside it (this package's grouped BF16 GEMM and, as a library reference,
+    torch.matmul / cuBLAS)."""
+    from nvfp4_quantization_aware_b200 import synthetic as S
+    out = {}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(stream):
+        w = S.weights(4096, 4096, seed=1, device=dev)
+        rc, rsf, rts = Q.nvfp4_quantize(w, Q.DYNAMIC)
+        wc, wsf, wts = Q.nvfp4_quantize(w, Q.DYNAMIC, layout=Q.SCALES_MMA)
+        w_hat = Q.nvfp4_fake_quant(w, Q.DYNAMIC)
+        for M in (8192, 128):
+            x = S.channel_scaled_activations(M, 4096, seed=0, device=dev)
+            xc, xsf, xts = Q.nvfp4_quantize(x, Q.DYNAMIC, layout=Q.SCALES_MMA)
+            c = torch.empty(M, 4096, dtype=torch.bfloat16, device=dev)
+            off = torch.tensor([0, M], dtype=torch.int32, device=dev)
+            ln = torch.tensor([M], dtype=torch.int32, device=dev)
+            calls = {"w4a16": lambda: Q.nvfp4_gemm_w4a16(x, rc, rsf, rts, out=c),
+                     "w4a4": lambda: Q.nvfp4_gemm_w4a4(xc, xsf, xts, wc, wsf, wts, out=c),
+                     "bf16": lambda: Q.nvfp4_gemm_bf16_grouped(0, x, w_hat, off, ln, M, 4096, 4096, out=c),
+                     "cublas_bf16": lambda: torch.matmul(x, w_hat.t(), out=c)}
+            res = {}
+            for name, call in calls.items():
+                for _ in range(3):
+                    call()
+                evs = []
+                for _ in range(K):
+                    flush_l2(flush)
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    call()
+                    e1.record(stream)
+                    evs.append((e0, e1))
+                stream.synchronize()
+                ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+                res[name] = {"ms": round(ms, 5), "tflops": round(2.0 * M * 4096 * 4096 / (ms * 1e-3) / 1e12, 1)}
+            res["w4a16_over_bf16_throughput"] = round(res["bf16"]["ms"] / res["w4a16"]["ms"], 3)
+            res["w4a4_over_bf16_throughput"] = round(res["bf16"]["ms"] / res["w4a4"]["ms"], 3)
+            out[f"M{M}"] = res
+    out["config"] = ("x M x 4096 bf16, w 4096 x 4096 NVFP4 (dynamic scales); w4a4 takes x pre-quantized; "
+                     "L2 flushed before each launch")
     return out
 
 

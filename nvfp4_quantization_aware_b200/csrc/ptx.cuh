@@ -95,6 +95,9 @@ NVFP4_DEV void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" 
 // its shared-memory source (the buffer may be overwritten afterwards).
 NVFP4_DEV void bulk_wait_group_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
+// Same, allowing the most recent committed group to still be reading.
+NVFP4_DEV void bulk_wait_group_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+
 // Wait until every committed bulk store of this thread has completed.
 NVFP4_DEV void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
@@ -105,6 +108,37 @@ NVFP4_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared
 NVFP4_DEV void st_shared_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p)), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
+}
+
+// ------------------------------------------------------------------ per-thread async copies
+
+// 16-byte global -> shared copy through L2 only; src_bytes = 0 writes zeros
+// and reads nothing.
+NVFP4_DEV void cp_async_16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+// 4-byte global -> shared copy; src_bytes = 0 writes zeros and reads nothing.
+NVFP4_DEV void cp_async_4(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+NVFP4_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+// Wait until at most N of this thread's committed copy groups are pending.
+template <int N>
+NVFP4_DEV void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Byte permute: byte k of the result is byte (c >> 4k) & 7 of {b:a} (a holds
+// bytes 0-3), or that byte's sign bit replicated when (c >> 4k) & 8 is set.
+NVFP4_DEV uint32_t prmt(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
 }
 
 // ------------------------------------------------------------------ tcgen05
