@@ -15,19 +15,25 @@
 //               tiled TMA loads with 128-byte swizzle, and the stage's block
 //               scales as 1-D bulk copies (the MMA scale layout keeps each
 //               128-row x 4-block tile contiguous).  No cluster multicast.
-//   warp 1      allocates tensor memory, then one thread issues per stage:
-//               tcgen05.cp of the scales into tensor memory and four
-//               tcgen05.mma.kind::mxf4nvf4.block_scale (K = 64 each) into an
-//               FP32 accumulator in tensor memory; tcgen05.commit releases the
-//               stage back to the producer.
-//   warps 2-9   epilogue (two per TMEM subpartition, half the columns each): tcgen05.ld of the accumulator, x (s_gA s_gB), bf16
-//               rounding into registers, release of the accumulator to the MMA
-//               warp (acc_empty), then the global stores -- which overlap the
-//               next tile's MMAs.
+//   warp 1      allocates tensor memory, then one thread issues per stage
+//               four tcgen05.mma.kind::mxf4nvf4.block_scale (K = 64 each) into
+//               an FP32 accumulator in tensor memory; tcgen05.commit releases
+//               the stage back to the producer.
+//   warps 2-9   epilogue (two per TMEM subpartition, half the columns each):
+//               per 32 columns a tcgen05.ld of the accumulator, x (s_gA s_gB),
+//               bf16 rounding and the global stores (which do not wait), then
+//               release of the accumulator to the MMA warp (acc_empty).
+//   warps 10-13 scale writers, one per TMEM lane quadrant: per stage they
+//               move the stage's block scales from shared memory into tensor
+//               memory with tcgen05.st, in the layout the block-scaled MMA
+//               reads, and arrive on sf_full[stage].  Doing this with
+//               tcgen05.cp would put twelve copies per stage in order with
+//               the MMAs on the tensor pipe, about a third of the run time.
 // A STAGES-deep mbarrier ring between producer and MMA runs across tile
 // boundaries, so the next tile's operands stream in while the epilogue drains.
 // Tensor memory holds one 128 x BN FP32 accumulator (BN = 256 uses half of the
-// 512 columns) plus two sets of block scales; every wait is bounded.
+// 512 columns) plus one set of block scales per ring stage; every wait is
+// bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -51,15 +57,17 @@ struct GemmCfg {
   static constexpr int MAX_GROUPS = 256;         // grouped problems: segment table in shared memory
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ +
                                     (2 * MAX_GROUPS + 1) * 4 /*segment table*/;
-  // tensor-memory columns: accumulator, then two sets of scales (alternating
-  // by stage parity)
+  // tensor-memory columns: accumulator, then one set of scales per ring stage
+  // (a set is rewritten only after the producer has seen its stage released,
+  // i.e. after the MMAs that read it have completed)
   static constexpr int TM_ACC = 0;
-  static constexpr int TM_SFA = BN;                               // 2 x 4*KB columns
-  static constexpr int TM_SFB = BN + 2 * 4 * KB_PER_STAGE;        // 2 x 4*KB*NB_SFB columns
-  static constexpr int TM_COLS_USED = TM_SFB + 2 * 4 * KB_PER_STAGE * NB_SFB;
+  static constexpr int TM_SFA = BN;                                    // STAGES x 4*KB columns
+  static constexpr int TM_SFB = BN + STAGES * 4 * KB_PER_STAGE;        // STAGES x 4*KB*NB_SFB columns
+  static constexpr int TM_COLS_USED = TM_SFB + STAGES * 4 * KB_PER_STAGE * NB_SFB;
   static constexpr int TM_COLS = TM_COLS_USED <= 256 ? 256 : 512;
   static constexpr int EPI_WARPS = 8;            // two per TMEM subpartition, BN/2 columns each
-  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int SF_WARPS = 4;             // scale writers, one per TMEM subpartition
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS + 32 * SF_WARPS;
   // instruction descriptor: E2M1 x E2M1 (format 1), UE4M3 scales, K-major A
   // and B, N >> 3 in bits 17-22, M >> 4 in bits 24-28, dense K = 64.
   static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
@@ -137,7 +145,8 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
   uint64_t* empty = full + C::STAGES;
   uint64_t* acc_full = empty + C::STAGES;   // MMA -> epilogue: accumulator complete
   uint64_t* acc_empty = acc_full + 1;       // epilogue -> MMA: accumulator drained
-  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  uint64_t* sf_full = acc_empty + 1;        // scale writers -> MMA: stage's scales in tensor memory
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(sf_full + C::STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
   int32_t* s_off = reinterpret_cast<int32_t*>(smem + C::STAGES * C::STAGE_BYTES + 256);
   int32_t* s_rows = s_off + C::MAX_GROUPS + 1;
@@ -159,6 +168,7 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_full[s], C::SF_WARPS);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, C::EPI_WARPS);  // one arrival per epilogue warp
@@ -222,24 +232,13 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
         for (int kt = 0; kt < num_kt; ++kt, ++it) {
           const int s = it % C::STAGES;
           const uint32_t ph = (uint32_t)(it / C::STAGES) & 1u;
-          if (!mbar_wait_bounded(&full[s], ph)) { *abort_flag = 1; break; }
+          if (!mbar_wait_bounded(&full[s], ph) || !mbar_wait_bounded(&sf_full[s], ph)) { *abort_flag = 1; break; }
           if (*abort_flag) break;
           tc_fence_after();
           int nkc = p.kchunks - kt * C::KB_PER_STAGE;
           if (nkc > C::KB_PER_STAGE) nkc = C::KB_PER_STAGE;
-          const int par = it & 1;
-          const uint32_t sfa_col = tmem + C::TM_SFA + par * 4 * C::KB_PER_STAGE;
-          const uint32_t sfb_col = tmem + C::TM_SFB + par * 4 * C::KB_PER_STAGE * C::NB_SFB;
-          // scales: each 512-byte (128 rows x 4 blocks) tile -> 4 TMEM columns
-          for (int kb = 0; kb < nkc; ++kb) {
-            tc_cp_32x128b_warpx4(sfa_col + kb * 4,
-                                 smem_desc(smem_u32(sSFA + s * C::SFA_BYTES + kb * 512), 0, 128, 0));
-#pragma unroll
-            for (int j = 0; j < C::NB_SFB; ++j)
-              tc_cp_32x128b_warpx4(
-                  sfb_col + kb * 4 * C::NB_SFB + j * 4,
-                  smem_desc(smem_u32(sSFB + s * C::SFB_BYTES + j * 512 * C::KB_PER_STAGE + kb * 512), 0, 128, 0));
-          }
+          const uint32_t sfa_col = tmem + C::TM_SFA + s * 4 * C::KB_PER_STAGE;
+          const uint32_t sfb_col = tmem + C::TM_SFB + s * 4 * C::KB_PER_STAGE * C::NB_SFB;
           const uint32_t a_base = smem_u32(sA + s * C::A_BYTES);
           const uint32_t b_base = smem_u32(sB + s * C::B_BYTES);
           for (int kb = 0; kb < nkc; ++kb) {
@@ -253,6 +252,46 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
         }
         tc_commit(acc_full);
         ++ti;
+      }
+    }
+  } else if (warp >= 2 + C::EPI_WARPS) {
+    // ------------------------------------------------------------ scale writers
+    // Each 512-byte scale tile (128 rows x 4 blocks, MMA layout: row r's 4
+    // bytes at 16 (r % 32) + 4 (r / 32)) becomes 4 TMEM columns in which lane
+    // L holds bytes [16 (L % 32), 16 (L % 32) + 16) of the tile -- on every
+    // subpartition, the image a 32x128b.warpx4 tcgen05.cp would produce.
+    const int q = warp & 3;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+    int it = 0;
+    for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+      if (tile_info(t, num_n, C::BM, C::BN, p, s_off, s_rows).empty) continue;
+      bool ok = true;
+      for (int kt = 0; kt < num_kt; ++kt, ++it) {
+        const int s = it % C::STAGES;
+        const uint32_t ph = (uint32_t)(it / C::STAGES) & 1u;
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[s], ph));  // warp-uniform exit
+        if (!ok) break;
+        int nkc = p.kchunks - kt * C::KB_PER_STAGE;
+        if (nkc > C::KB_PER_STAGE) nkc = C::KB_PER_STAGE;
+        const uint8_t* a_src = sSFA + s * C::SFA_BYTES + lane * 16;
+        const uint8_t* b_src = sSFB + s * C::SFB_BYTES + lane * 16;
+        const uint32_t a_col = lane_base + C::TM_SFA + s * 4 * C::KB_PER_STAGE;
+        const uint32_t b_col = lane_base + C::TM_SFB + s * 4 * C::KB_PER_STAGE * C::NB_SFB;
+        for (int kb = 0; kb < nkc; ++kb) {
+          tmem_st_32x32b_x4(a_col + kb * 4, *reinterpret_cast<const uint4*>(a_src + kb * 512));
+#pragma unroll
+          for (int j = 0; j < C::NB_SFB; ++j)
+            tmem_st_32x32b_x4(b_col + kb * 4 * C::NB_SFB + j * 4,
+                              *reinterpret_cast<const uint4*>(b_src + j * 512 * C::KB_PER_STAGE + kb * 512));
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_full[s]);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        break;
       }
     }
   } else {
@@ -271,50 +310,40 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
       if (!ok) *abort_flag = 1;
       if (!ok || *abort_flag) break;
       tc_fence_after();
-      // drain this warp's part of the accumulator into registers as bf16 pairs ...
-      uint32_t packed[HALF / 2];
+      // drain this warp's part of the accumulator 32 columns at a time: load,
+      // x (s_gA s_gB), round to bf16, store (the stores do not wait) ...
+      const int row = m0 + sub * 32 + lane;
+      __nv_bfloat16* crow = p.c + (int64_t)row * p.ldc;
 #pragma unroll
-      for (int c0 = 0; c0 < HALF; c0 += 64) {  // two loads in flight per wait
-        uint32_t r0[32], r1[32];
-        const uint32_t taddr = tmem + C::TM_ACC + ((uint32_t)(sub * 32) << 16) + cbase + c0;
-        tmem_ld_32x32b_x32(taddr, r0);
-        tmem_ld_32x32b_x32(taddr + 32, r1);
+      for (int c0 = 0; c0 < HALF; c0 += 32) {
+        uint32_t r0[32], packed[16];
+        tmem_ld_32x32b_x32(tmem + C::TM_ACC + ((uint32_t)(sub * 32) << 16) + cbase + c0, r0);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          packed[c0 / 2 + j] = pack_bf16x2(__uint_as_float(r0[2 * j]) * alpha, __uint_as_float(r0[2 * j + 1]) * alpha);
-          packed[c0 / 2 + 16 + j] =
-              pack_bf16x2(__uint_as_float(r1[2 * j]) * alpha, __uint_as_float(r1[2 * j + 1]) * alpha);
-        }
-      }
-      // ... hand the accumulator back to the MMA warp ...
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
-      // ... and store while the next tile accumulates
-      const int row = m0 + sub * 32 + lane;
-      if (row < tl.row_end) {
-        __nv_bfloat16* crow = p.c + (int64_t)row * p.ldc;
-#pragma unroll
-        for (int c0 = 0; c0 < HALF; c0 += 32) {
+        for (int j = 0; j < 16; ++j)
+          packed[j] = pack_bf16x2(__uint_as_float(r0[2 * j]) * alpha, __uint_as_float(r0[2 * j + 1]) * alpha);
+        if (row < tl.row_end) {
           const int col0 = n0 + cbase + c0;
           if (col0 + 32 <= p.N && p.c_vec16) {
             uint4* dst = reinterpret_cast<uint4*>(crow + col0);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(packed[c0 / 2 + 4 * j], packed[c0 / 2 + 4 * j + 1], packed[c0 / 2 + 4 * j + 2],
-                                  packed[c0 / 2 + 4 * j + 3]);
+              dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
           } else {
+#pragma unroll
             for (int j = 0; j < 32; ++j) {
               if (col0 + j < p.N) {
-                const uint32_t w = packed[(c0 + j) >> 1];
-                const uint32_t h = (j & 1) ? (w >> 16) : (w & 0xFFFFu);
-                crow[col0 + j] = __ushort_as_bfloat16((unsigned short)h);
+                const uint32_t w = packed[j >> 1];
+                crow[col0 + j] = __ushort_as_bfloat16((unsigned short)((j & 1) ? (w >> 16) : (w & 0xFFFFu)));
               }
             }
           }
         }
       }
+      // ... and hand the accumulator back to the MMA warp
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
     }
   }
   tc_fence_before();
