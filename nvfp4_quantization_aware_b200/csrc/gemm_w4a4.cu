@@ -20,9 +20,11 @@
 //               an FP32 accumulator in tensor memory; tcgen05.commit releases
 //               the stage back to the producer.
 //   warps 2-9   epilogue (two per TMEM subpartition, half the columns each):
-//               per 32 columns a tcgen05.ld of the accumulator, x (s_gA s_gB),
-//               bf16 rounding and the global stores (which do not wait), then
-//               release of the accumulator to the MMA warp (acc_empty).
+//               tcgen05.ld of the accumulator, x (s_gA s_gB), bf16 rounding
+//               into registers, release of the accumulator to the MMA warp
+//               (acc_empty), then the global stores -- which overlap the next
+//               tile's MMAs.  Ragged tiles store 32 columns at a time and
+//               release at the end.
 //   warps 10-13 scale writers, one per TMEM lane quadrant: per stage they
 //               move the stage's block scales from shared memory into tensor
 //               memory with tcgen05.st, in the layout the block-scaled MMA
@@ -40,6 +42,14 @@
 #include "ptx.cuh"
 
 namespace nvfp4 {
+
+// 32-byte global store of words w[i0 .. i0 + 7] (address 32-byte aligned).
+template <int NW>
+NVFP4_DEV void st_global_v8(void* p, const uint32_t (&w)[NW], int i0) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[i0]), "r"(w[i0 + 1]), "r"(w[i0 + 2]),
+               "r"(w[i0 + 3]), "r"(w[i0 + 4]), "r"(w[i0 + 5]), "r"(w[i0 + 6]), "r"(w[i0 + 7])
+               : "memory");
+}
 
 template <int BN_>
 struct GemmCfg {
@@ -84,6 +94,7 @@ struct GemmParams {
   int kchunks;           // K / 64
   int b_rowtiles;        // ceil(N / 128): 128-row scale tiles present for B
   int c_vec16;           // C base 16-byte aligned and ldc % 8 == 0: 16-byte stores
+  int c_vec32;           // C base 32-byte aligned and ldc % 16 == 0: 32-byte stores
   // Grouped problems (groups > 0): group g owns A rows [a_off[g], a_off[g] + a_rows[g]) with
   // a_off[g] a multiple of 128 (device arrays; a_off[groups] is the padded row total), B rows
   // [g * N, (g + 1) * N), tensor scales a_ts[g] and b_ts[g].
@@ -310,40 +321,74 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
       if (!ok) *abort_flag = 1;
       if (!ok || *abort_flag) break;
       tc_fence_after();
-      // drain this warp's part of the accumulator 32 columns at a time: load,
-      // x (s_gA s_gB), round to bf16, store (the stores do not wait) ...
       const int row = m0 + sub * 32 + lane;
       __nv_bfloat16* crow = p.c + (int64_t)row * p.ldc;
+      const uint32_t tbase = tmem + C::TM_ACC + ((uint32_t)(sub * 32) << 16) + cbase;
+      if (p.c_vec16 && n0 + C::BN <= p.N) {
+        // Full-width tile: drain this warp's part of the accumulator into
+        // registers as bf16 pairs, hand the accumulator back to the MMA warp,
+        // then store while the next tile accumulates.
+        uint32_t packed[HALF / 2];
 #pragma unroll
-      for (int c0 = 0; c0 < HALF; c0 += 32) {
-        uint32_t r0[32], packed[16];
-        tmem_ld_32x32b_x32(tmem + C::TM_ACC + ((uint32_t)(sub * 32) << 16) + cbase + c0, r0);
-        tmem_wait_ld();
+        for (int c0 = 0; c0 < HALF; c0 += 16) {
+          uint32_t r0[16];
+          tmem_ld_32x32b_x16(tbase + c0, r0);
+          tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          packed[j] = pack_bf16x2(__uint_as_float(r0[2 * j]) * alpha, __uint_as_float(r0[2 * j + 1]) * alpha);
+          for (int j = 0; j < 8; ++j)
+            packed[c0 / 2 + j] = pack_bf16x2(__uint_as_float(r0[2 * j]) * alpha, __uint_as_float(r0[2 * j + 1]) * alpha);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
         if (row < tl.row_end) {
-          const int col0 = n0 + cbase + c0;
-          if (col0 + 32 <= p.N && p.c_vec16) {
-            uint4* dst = reinterpret_cast<uint4*>(crow + col0);
+          // 32-byte stores write whole L2 sectors and halve the store
+          // instructions (the uncoalesced row-per-thread stores compete with
+          // the operand traffic in the SM's L1 / shared-memory path)
+          if (p.c_vec32) {
+            uint8_t* dst = reinterpret_cast<uint8_t*>(crow + n0 + cbase);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+            for (int j = 0; j < HALF / 16; ++j) st_global_v8(dst + 32 * j, packed, 8 * j);
           } else {
+            uint4* dst = reinterpret_cast<uint4*>(crow + n0 + cbase);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (col0 + j < p.N) {
-                const uint32_t w = packed[j >> 1];
-                crow[col0 + j] = __ushort_as_bfloat16((unsigned short)((j & 1) ? (w >> 16) : (w & 0xFFFFu)));
+            for (int j = 0; j < HALF / 8; ++j)
+              dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+          }
+        }
+      } else {
+        // Ragged tile (or C without 16-byte alignment): 32 columns at a time
+        // -- load, scale, round, store -- and the hand-back at the end.
+#pragma unroll
+        for (int c0 = 0; c0 < HALF; c0 += 32) {
+          uint32_t r0[32], packed[16];
+          tmem_ld_32x32b_x32(tbase + c0, r0);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            packed[j] = pack_bf16x2(__uint_as_float(r0[2 * j]) * alpha, __uint_as_float(r0[2 * j + 1]) * alpha);
+          const int col0 = n0 + cbase + c0;
+          if (row < tl.row_end && col0 < p.N) {
+            if (col0 + 32 <= p.N && p.c_vec16) {
+              uint4* dst = reinterpret_cast<uint4*>(crow + col0);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+            } else {
+              const int rem = p.N - col0;
+              unsigned short* dst = reinterpret_cast<unsigned short*>(crow + col0);
+#pragma unroll
+              for (int k = 0; k < 16; ++k) {
+                if (2 * k < rem) dst[2 * k] = (unsigned short)(packed[k] & 0xFFFFu);
+                if (2 * k + 1 < rem) dst[2 * k + 1] = (unsigned short)(packed[k] >> 16);
               }
             }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
       }
-      // ... and hand the accumulator back to the MMA warp
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
     }
   }
   tc_fence_before();
@@ -464,6 +509,7 @@ nvfp4_status nvfp4_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_scales_mma
   p.kchunks = (int)(K / 64);
   p.b_rowtiles = (int)((N + 127) / 128);
   p.c_vec16 = (((uintptr_t)c & 15u) == 0 && (ldc % 8) == 0) ? 1 : 0;
+  p.c_vec32 = (((uintptr_t)c & 31u) == 0 && (ldc % 16) == 0) ? 1 : 0;
   p.groups = 0;
   p.a_off = nullptr;
   p.a_rows = nullptr;
@@ -508,6 +554,7 @@ nvfp4_status nvfp4_gemm_w4a4_grouped(int groups, const uint8_t* a_codes, const u
   p.kchunks = (int)(K / 64);
   p.b_rowtiles = (int)((int64_t)groups * N / 128);
   p.c_vec16 = (((uintptr_t)c & 15u) == 0 && (ldc % 8) == 0) ? 1 : 0;
+  p.c_vec32 = (((uintptr_t)c & 31u) == 0 && (ldc % 16) == 0) ? 1 : 0;
   p.groups = groups;
   p.a_off = a_row_offsets;
   p.a_rows = a_rows;
