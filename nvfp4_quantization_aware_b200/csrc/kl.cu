@@ -368,15 +368,22 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
   for (int o = 16; o > 0; o >>= 1) my = stats_merge(my, stats_shfl_xor(my, o));
   if ((threadIdx.x & 31) == 0) warp_stats[threadIdx.x >> 5] = my;
   __syncthreads();
-  if (threadIdx.x < csize) {
-    KlStats c = warp_stats[0];
-    for (int w = 1; w < kKlWarps; ++w) c = stats_merge(c, warp_stats[w]);
-    KlStats* dst = cluster.map_shared_rank(peer_stats, (int)threadIdx.x);
-    dst[crank] = c;
+  if (threadIdx.x < 32) {  // warp 0 merges the warps by the same butterfly, then pushes
+    KlStats c = warp_stats[threadIdx.x & (kKlWarps - 1)];
+    if (threadIdx.x >= kKlWarps) stats_init(c, kPadLogit * a);
+#pragma unroll
+    for (int o = kKlWarps / 2; o > 0; o >>= 1) c = stats_merge(c, stats_shfl_xor(c, o));
+    if ((int)threadIdx.x < csize) cluster.map_shared_rank(peer_stats, (int)threadIdx.x)[crank] = c;
   }
   cluster.sync();  // all pushes visible; no CTA reads a peer after this point
-  KlStats row_stats = peer_stats[0];
-  for (int r = 1; r < csize; ++r) row_stats = stats_merge(row_stats, peer_stats[r]);
+  __shared__ KlStats row_stats_sh;
+  if (threadIdx.x == 0) {  // one thread merges the peers (in rank order) for the whole CTA
+    KlStats m = peer_stats[0];
+    for (int r = 1; r < csize; ++r) m = stats_merge(m, peer_stats[r]);
+    row_stats_sh = m;
+  }
+  __syncthreads();
+  const KlStats row_stats = row_stats_sh;
   const float Wt = row_stats.mt, Ws = row_stats.ms, St = row_stats.St, Ss = row_stats.Ss;
   if (crank == 0 && threadIdx.x == 0) {
     // KL = sum p_t (log p_t - log p_s) = ln2 * (Y / S_t + log2(S_s / S_t))

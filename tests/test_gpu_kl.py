@@ -123,3 +123,27 @@ def test_distill_logits_full_size_sampled():
     rows = np.random.default_rng(0).choice(16384, 48, replace=False)
     rows = np.concatenate([[0, 16383], rows])
     _check(d["teacher"], d["student"], rows_to_check=rows)
+
+
+# The persistent form (aligned bf16 rows, vocabulary a multiple of 8, at least
+# 64 rows, cluster of 2 or more): rows spread over the resident clusters, the
+# shared-memory ring wrapping several times per cluster.
+@pytest.mark.parametrize("rows,V", [(64, 131072), (100, 131072), (70, 40000), (300, 16392), (1000, 32768)])
+def test_persistent_rows(rows, V):
+    t, s = S.logits_pair(rows, V, seed=rows + V, device=DEV, dtype=torch.bfloat16)
+    _check(t, s, T=2.5, grad_scale=0.37)
+
+
+def test_persistent_negative_grad_scale_and_stride():
+    rows, V = 80, 65536
+    t0, s0 = S.logits_pair(rows, V, seed=11, device=DEV, dtype=torch.bfloat16)
+    t = torch.zeros(rows, V + 64, dtype=torch.bfloat16, device=DEV)
+    s = torch.zeros(rows, V + 64, dtype=torch.bfloat16, device=DEV)
+    t[:, :V] = t0
+    s[:, :V] = s0
+    t, s = t[:, :V], s[:, :V]
+    _check(t, s, grad_scale=-0.5)
+    loss, row, g = Q.qad_kl_fwd_bwd(t, s, want_grad=False, want_row_kl=True)
+    assert g is None
+    ref_loss, ref_row, _ = O.kl(t0.double().cpu().numpy(), s0.double().cpu().numpy(), want_grad=False)
+    assert abs(float(loss.cpu()[0]) - ref_loss) <= LOSS_RTOL * ref_loss
