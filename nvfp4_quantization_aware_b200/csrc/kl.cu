@@ -292,7 +292,8 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
   constexpr int ESZ = (int)sizeof(T);
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ uint64_t bar;
-  __shared__ KlStats warp_stats[kKlWarps];
+  __shared__ float warp_max[2][kKlWarps];
+  __shared__ float warp_sum[3][kKlWarps];
   __shared__ KlStats peer_stats[kKlMaxCluster];  // written by every CTA of the cluster
   __shared__ int s_ok;
 
@@ -363,17 +364,56 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
       }
     }
   }
-  // ---- merge: warp, CTA, then push to every CTA of the cluster
+  // ---- merge over the CTA, then push to every CTA of the cluster: the CTA's
+  // maxima first (a max butterfly, no exponentials), then every thread
+  // rebases its sums to them once and the sums are added by a butterfly and
+  // in warp order
+  {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    float Mt = my.mt, Ms = my.ms;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) my = stats_merge(my, stats_shfl_xor(my, o));
-  if ((threadIdx.x & 31) == 0) warp_stats[threadIdx.x >> 5] = my;
-  __syncthreads();
-  if (threadIdx.x < 32) {  // warp 0 merges the warps by the same butterfly, then pushes
-    KlStats c = warp_stats[threadIdx.x & (kKlWarps - 1)];
-    if (threadIdx.x >= kKlWarps) stats_init(c, kPadLogit * a);
+    for (int o = 16; o > 0; o >>= 1) {
+      Mt = fmaxf(Mt, __shfl_xor_sync(0xFFFFFFFFu, Mt, o));
+      Ms = fmaxf(Ms, __shfl_xor_sync(0xFFFFFFFFu, Ms, o));
+    }
+    if (lane == 0) {
+      warp_max[0][wid] = Mt;
+      warp_max[1][wid] = Ms;
+    }
+    __syncthreads();
+    Mt = warp_max[0][0];
+    Ms = warp_max[1][0];
 #pragma unroll
-    for (int o = kKlWarps / 2; o > 0; o >>= 1) c = stats_merge(c, stats_shfl_xor(c, o));
-    if ((int)threadIdx.x < csize) cluster.map_shared_rank(peer_stats, (int)threadIdx.x)[crank] = c;
+    for (int w = 1; w < kKlWarps; ++w) {
+      Mt = fmaxf(Mt, warp_max[0][w]);
+      Ms = fmaxf(Ms, warp_max[1][w]);
+    }
+    stats_rebase(my, Mt, Ms);
+    float sum_t = my.St, sum_s = my.Ss, sum_y = my.Y;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      sum_t += __shfl_xor_sync(0xFFFFFFFFu, sum_t, o);
+      sum_s += __shfl_xor_sync(0xFFFFFFFFu, sum_s, o);
+      sum_y += __shfl_xor_sync(0xFFFFFFFFu, sum_y, o);
+    }
+    if (lane == 0) {
+      warp_sum[0][wid] = sum_t;
+      warp_sum[1][wid] = sum_s;
+      warp_sum[2][wid] = sum_y;
+    }
+    __syncthreads();
+    if ((int)threadIdx.x < csize) {
+      KlStats c;
+      c.mt = Mt;
+      c.ms = Ms;
+      c.St = c.Ss = c.Y = 0.f;
+      for (int w = 0; w < kKlWarps; ++w) {
+        c.St += warp_sum[0][w];
+        c.Ss += warp_sum[1][w];
+        c.Y += warp_sum[2][w];
+      }
+      cluster.map_shared_rank(peer_stats, (int)threadIdx.x)[crank] = c;
+    }
   }
   cluster.sync();  // all pushes visible; no CTA reads a peer after this point
   __shared__ KlStats row_stats_sh;
