@@ -704,6 +704,22 @@ def run_profile_case(case: str):
         d = S.distill_logits(seed=0, device=dev, rows=2048)  # 2 x 512 MiB
         for _ in range(5):
             Q.qad_kl_fwd_bwd(d["teacher"], d["student"])
+    elif case == "kl_topk":
+        d = S.distill_logits(seed=0, device=dev, rows=2048)
+        for _ in range(5):
+            Q.qad_kl_topk_fwd_bwd(d["teacher"], d["student"], 4096)
+    elif case == "w4a16":
+        w = S.weights(4096, 4096, seed=1, device=dev)
+        x = S.channel_scaled_activations(8192, 4096, seed=0, device=dev)
+        codes, sb, ts = Q.nvfp4_quantize(w, Q.DYNAMIC)
+        for _ in range(5):
+            Q.nvfp4_gemm_w4a16(x, codes, sb, ts)
+    elif case == "calibrate":
+        xs = S.weight_sweep(seed=0, device=dev, experts=48, lm_head=False)
+        ts = torch.zeros(len(xs), device=dev)
+        Q.nvfp4_quantize_grouped(xs, Q.DYNAMIC, tensor_scales=ts)
+        for _ in range(5):
+            Q.nvfp4_calibrate_mse_grouped(xs, ts)
     torch.cuda.synchronize()
     print(json.dumps({"profile_case": case, "ok": True}))
 
@@ -716,7 +732,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-secondary", action="store_true", help="skip the GEMM and KL measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["quant", "gemm", "kl", "moe"], default=None,
+    ap.add_argument("--profile", choices=["quant", "gemm", "kl", "kl_topk", "w4a16", "calibrate", "moe"], default=None,
                     help="run one small single-kernel case (for ncu captures) and exit")
     args = ap.parse_args()
     if args.profile:
