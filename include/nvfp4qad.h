@@ -165,6 +165,18 @@ nvfp4_status nvfp4_quantize(const void* x, nvfp4_dtype dtype, int64_t rows, int6
  * index, or all ones.  Asynchronous on `stream`. */
 nvfp4_status nvfp4_selftest_division(uint64_t* mismatches, uint64_t* first, void* stream);
 
+/* Dense FP4 tensor-core throughput probe (measurement support for the W4A4
+ * GEMM's roofline).  Launches `ctas` CTAs (one per SM when ctas <= the SM
+ * count; each takes all 512 tensor-memory columns and enough shared memory to
+ * keep others off its SM), each issuing `iters` x 4 block-scaled FP4 MMAs
+ * (tcgen05.mma.kind::mxf4nvf4, 128 x 256 x 64, UE4M3 scales of 1.0) back to
+ * back on one resident shared-memory stage -- the instruction and tile of
+ * nvfp4_gemm_w4a4 without its operand traffic.  *flop_per_launch (host,
+ * may be NULL) receives 2 * 128 * 256 * 64 * 4 * iters * ctas; the caller
+ * times the launch (CUDA events on `stream`).  1 <= iters <= 2^40,
+ * 1 <= ctas <= 4096, else NVFP4_ERR_ARG. */
+nvfp4_status nvfp4_probe_fp4_mma(int64_t iters, int ctas, double* flop_per_launch, void* stream);
+
 /* ------------------------------------------------------------------------
  * Grouped quantize / fake-quant: one call for a list of tensors that share a
  * dtype and a scale mode, each with its own tensor scale (e.g. the routed and

@@ -39,6 +39,7 @@ from .binding import (  # noqa: F401
     nvfp4_gemm_w4a4_grouped,
     nvfp4_gemm_bf16_grouped,
     nvfp4_gemm_w4a16,
+    nvfp4_probe_fp4_mma,
     nvfp4_scales_to_mma,
     nvfp4_quantize_fake_quant_grouped,
     MoeLayerStep,

@@ -144,6 +144,8 @@ def lib() -> ctypes.CDLL:
     L.nvfp4_gemm_bf16_grouped.restype = i32
     L.nvfp4_gemm_w4a16.argtypes = [p, i64, p, p, p, i64, i64, i64, p, i64, p]
     L.nvfp4_gemm_w4a16.restype = i32
+    L.nvfp4_probe_fp4_mma.argtypes = [i64, i32, ctypes.POINTER(ctypes.c_double), p]
+    L.nvfp4_probe_fp4_mma.restype = i32
     L.qad_kl_workspace_size.argtypes = [i64, i64, i32]
     L.qad_kl_workspace_size.restype = sz
     L.qad_kl_fwd_bwd.argtypes = [p, p, i32, i64, i64, i64, f32, p, p, p, i64, f32, p, sz, p]
@@ -560,6 +562,15 @@ def nvfp4_gemm_w4a16(a: torch.Tensor, b_codes: torch.Tensor, b_scales: torch.Ten
                                 _ptr(out), out.stride(0), _stream(a.device))
     _check(st, "nvfp4_gemm_w4a16")
     return out
+
+
+def nvfp4_probe_fp4_mma(iters: int, ctas: int, stream: torch.cuda.Stream | None = None) -> float:
+    """Launch the dense FP4 MMA throughput probe; returns the flop of the launch
+    (the caller times it with CUDA events on the same stream)."""
+    flop = ctypes.c_double(0.0)
+    s = (stream or torch.cuda.current_stream()).cuda_stream
+    _check(lib().nvfp4_probe_fp4_mma(iters, ctas, ctypes.byref(flop), s), "nvfp4_probe_fp4_mma")
+    return flop.value
 
 
 def nvfp4_scales_to_mma(block_scales: torch.Tensor, rows: int, cols: int) -> torch.Tensor:
