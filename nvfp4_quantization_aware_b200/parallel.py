@@ -15,9 +15,17 @@ rows; the only data exchanged are scalars:
   already those of the global mean, and one all-reduce(sum) of the ranks'
   partial sums gives the loss.
 
+* expert parallelism for the MoE layer (experts owned in contiguous blocks,
+  rank r holding experts [r E/W, (r+1) E/W)): the routed (token, slot) rows
+  travel to the rank that owns their expert and the expert outputs travel
+  back, each way one all_to_all_single of the rows (plus one of the row
+  counts); the backward pass runs the same two exchanges in reverse.  The
+  pages train with expert parallelism (EP 4 and 8).
+
 The device operations are passed in (`ops`), defaulting to this package's
-CUDA entry points; the collectives go through torch.distributed.  No
-arithmetic on tensors happens here beyond the scalar mean.
+CUDA entry points; the collectives go through torch.distributed.  Beyond the
+collectives, only data movement (row gathers and scatters, the weighted sum
+over a token's slots) happens here.
 """
 from __future__ import annotations
 
@@ -93,3 +101,101 @@ def sharded_kl(teacher, student, total_rows: int, T: float = 1.0, ops: ShardOps 
     if dist.is_available() and dist.is_initialized():
         dist.all_reduce(part, op=dist.ReduceOp.SUM, group=group)
     return part / total_rows, row_kl, g
+
+
+# ------------------------------------------------------------------ expert parallelism
+
+
+def _world(group=None) -> int:
+    return dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1
+
+
+@dataclass
+class EpPlan:
+    """Bookkeeping of one expert-parallel dispatch, reused by the combine and
+    by both backward exchanges."""
+    perm: torch.Tensor   # [tokens * topk] int64: (token, slot) pairs in send order
+    send_counts: list    # rows sent to each rank
+    recv_counts: list    # rows received from each rank
+    tokens: int
+    topk: int
+
+
+def _exchange(out_rows: int, rows: torch.Tensor, out_splits, in_splits, group=None) -> torch.Tensor:
+    out = rows.new_empty((out_rows,) + tuple(rows.shape[1:]))
+    if _world(group) > 1:
+        dist.all_to_all_single(out, rows.contiguous(), list(out_splits), list(in_splits), group=group)
+    else:
+        out.copy_(rows)
+    return out
+
+
+def ep_dispatch(x: torch.Tensor, ids: torch.Tensor, experts: int, group=None):
+    """Send this rank's routed rows to the ranks that own their experts.
+
+    x [tokens, H]; ids [tokens, topk] expert of each (token, slot).  Returns
+    (recv_x [R, H], recv_expert [R] int32 -- the expert's index among the
+    receiving rank's experts, plan).  Received rows are grouped by source rank
+    (rank order) and, within a source, in (token, slot) order, so the result
+    does not depend on timing."""
+    world = _world(group)
+    if experts % world:
+        raise ValueError(f"{experts} experts do not split evenly over {world} ranks")
+    per = experts // world
+    tokens, topk = ids.shape
+    flat = ids.reshape(-1).to(torch.int64)
+    if flat.numel() and (int(flat.min()) < 0 or int(flat.max()) >= experts):
+        raise ValueError("expert id out of range")
+    owner = flat // per
+    perm = torch.argsort(owner, stable=True)
+    send_counts = torch.bincount(owner, minlength=world).to(torch.int64)
+    recv_counts = _exchange(world, send_counts.view(world, 1), [1] * world, [1] * world, group).view(world)
+    sc, rc = send_counts.tolist(), recv_counts.tolist()
+    recv_x = _exchange(sum(rc), x[perm // topk], rc, sc, group)
+    local_e = (flat[perm] - owner[perm] * per).to(torch.int32)
+    recv_e = _exchange(sum(rc), local_e, rc, sc, group)
+    return recv_x, recv_e, EpPlan(perm, sc, rc, tokens, topk)
+
+
+def ep_combine(y_recv: torch.Tensor, plan: EpPlan, combine: torch.Tensor, group=None):
+    """Return the expert outputs of the received rows to their tokens and sum
+    them with the combine weights: y[t] = sum_j combine[t, j] * y_slot[t, j]
+    (at least fp32, slots in order).  Returns (y [tokens, H], y_slot [tokens,
+    topk, H] in y_recv's dtype -- kept for the backward pass)."""
+    back = _exchange(plan.tokens * plan.topk, y_recv, plan.send_counts, plan.recv_counts, group)
+    y_slot = torch.empty_like(back)
+    y_slot[plan.perm] = back
+    y_slot = y_slot.view(plan.tokens, plan.topk, -1)
+    acc = torch.promote_types(y_slot.dtype, torch.float32)
+    y = torch.zeros(plan.tokens, y_slot.shape[-1], dtype=acc, device=y_slot.device)
+    for j in range(plan.topk):
+        y += combine[:, j:j + 1].to(acc) * y_slot[:, j].to(acc)
+    return y, y_slot
+
+
+def ep_combine_backward(dy: torch.Tensor, plan: EpPlan, combine: torch.Tensor, y_slot: torch.Tensor, group=None):
+    """Backward of ep_combine: d y_slot[t, j] = combine[t, j] * dy[t] goes to
+    the expert owners (rows in the order the forward received them);
+    d combine[t, j] = <dy[t], y_slot[t, j]> stays here.  Returns
+    (dy_recv [R, H], d_combine [tokens, topk] at least fp32)."""
+    acc = torch.promote_types(dy.dtype, torch.float32)
+    d_slot = (combine.to(acc).unsqueeze(-1) * dy.to(acc).unsqueeze(1)).to(dy.dtype)
+    rows = d_slot.reshape(plan.tokens * plan.topk, -1)[plan.perm]
+    dy_recv = _exchange(sum(plan.recv_counts), rows, plan.recv_counts, plan.send_counts, group)
+    d_combine = (dy.to(acc).unsqueeze(1) * y_slot.to(acc)).sum(-1)
+    return dy_recv, d_combine
+
+
+def ep_dispatch_backward(dx_recv: torch.Tensor, plan: EpPlan, group=None) -> torch.Tensor:
+    """Backward of ep_dispatch: the input gradients of the received rows go
+    back to their tokens and are summed over the token's slots (at least fp32,
+    slots in order).  Returns dx [tokens, H]."""
+    back = _exchange(plan.tokens * plan.topk, dx_recv, plan.send_counts, plan.recv_counts, group)
+    per_slot = torch.empty_like(back)
+    per_slot[plan.perm] = back
+    per_slot = per_slot.view(plan.tokens, plan.topk, -1)
+    acc = torch.promote_types(per_slot.dtype, torch.float32)
+    dx = torch.zeros(plan.tokens, per_slot.shape[-1], dtype=acc, device=per_slot.device)
+    for j in range(plan.topk):
+        dx += per_slot[:, j].to(acc)
+    return dx
