@@ -507,6 +507,14 @@ struct KlKey<__nv_bfloat16> {
     return (u & 0x8000u) ? (~u & 0xFFFFu) : (u | 0x8000u);
   }
 };
+// Both order-preserving keys of a word of two bf16 (element 0 in the low
+// half): positive values get the sign bit set, negative ones all 16 bits
+// flipped -- the same map as KlKey<__nv_bfloat16>::key, two at a time.
+NVFP4_DEV uint32_t bf16x2_keys(uint32_t w) {
+  const uint32_t m = ((w >> 15) & 0x00010001u) * 0xFFFFu;  // 0xFFFF in each half whose sign is set
+  return w ^ (m | 0x80008000u);
+}
+
 template <>
 struct KlKey<float> {
   static constexpr int kBits = 32;
@@ -548,6 +556,8 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
   uint8_t* sel_mask = reinterpret_cast<uint8_t*>(vec_prefix + nvec_max);
   const KlSliceGeom geo = kl_stage_slice<T>(args, row, v0, n, st, ss, &bar, &s_ok);
   const int off = geo.off, nslots = geo.nslots, nvec = geo.nvec;
+  const int kfirst = (off + V8 - 1) / V8;  // vectors [kfirst, klast) hold no pad slot
+  const int klast = nslots / V8;
   const bool ok = s_ok != 0;
   const uint32_t* wt = reinterpret_cast<const uint32_t*>(st);  // words of the teacher slice
   constexpr int WPV = 16 / 4;                                   // words per 16-byte vector
@@ -560,17 +570,39 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
     hist[threadIdx.x] = 0u;
     __syncthreads();
     if (ok) {
-      for (int kb = 0; kb < nvec; kb += kKlThreads) {  // warp-uniform trip count
-        const int k = kb + (int)threadIdx.x;
+      for (int k = (int)threadIdx.x; k < nvec; k += kKlThreads) {
+        if constexpr (sizeof(T) == 2) {
+          if (k >= kfirst && k < klast) {
+            // interior vector of bf16: keys two at a time; one add of 2 when
+            // both keys of a word fall in the same bucket
+#pragma unroll
+            for (int q = 0; q < WPV; ++q) {
+              const uint32_t k2 = bf16x2_keys(wt[k * WPV + q]);
+              const uint32_t k0 = k2 & 0xFFFFu, k1 = k2 >> 16;
+              if (p == 0) {
+                const uint32_t d0 = k0 >> 8, d1 = k1 >> 8;
+                if (d0 == d1) {
+                  atomicAdd(&hist[d0], 2u);
+                } else {
+                  atomicAdd(&hist[d0], 1u);
+                  atomicAdd(&hist[d1], 1u);
+                }
+              } else {
+                if ((k0 >> 8) == prefix) atomicAdd(&hist[k0 & 0xFFu], 1u);
+                if ((k1 >> 8) == prefix) atomicAdd(&hist[k1 & 0xFFu], 1u);
+              }
+            }
+            continue;
+          }
+        }
 #pragma unroll
         for (int q = 0; q < WPV; ++q) {
-          const uint32_t w = k < nvec ? wt[k * WPV + q] : 0u;
+          const uint32_t w = wt[k * WPV + q];
 #pragma unroll
           for (int h = 0; h < Kf::kPerWord; ++h) {
             const int j = k * V8 + q * Kf::kPerWord + h;  // slot
             const uint32_t key = Kf::key(w, h);
-            const bool valid = k < nvec && j >= off && j < nslots &&
-                               (p == 0 || (key >> (shift + 8)) == prefix);
+            const bool valid = j >= off && j < nslots && (p == 0 || (key >> (shift + 8)) == prefix);
             if (valid) atomicAdd(&hist[(key >> shift) & 0xFFu], 1u);
           }
         }
@@ -656,6 +688,18 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
   // ---- selection mask per vector (bit e: element e of the vector is in S)
   for (int k = (int)threadIdx.x; k < nvec; k += kKlThreads) {
     unsigned mask = 0u, seen = 0u;
+    if constexpr (sizeof(T) == 2) {
+      if (ok && !rank_ties && k >= kfirst && k < klast) {  // every key >= tau is in S
+#pragma unroll
+        for (int q = 0; q < WPV; ++q) {
+          const uint32_t k2 = bf16x2_keys(wt[k * WPV + q]);
+          mask |= ((k2 & 0xFFFFu) >= tau ? 1u : 0u) << (2 * q);
+          mask |= ((k2 >> 16) >= tau ? 1u : 0u) << (2 * q + 1);
+        }
+        sel_mask[k] = (uint8_t)mask;
+        continue;
+      }
+    }
     if (ok) {
 #pragma unroll
       for (int q = 0; q < WPV; ++q) {
@@ -744,8 +788,6 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
     const float Lt = Wt + __log2f(St), Ls = Ws + __log2f(Ss);
     T* gout = reinterpret_cast<T*>(args.dlogits) + row * args.ld_grad + v0 - off;  // slot j -> gout[j]
     const bool vec_ok = (((uintptr_t)gout) & 15u) == 0;
-    const int kfirst = (off + V8 - 1) / V8;
-    const int klast = nslots / V8;
     for (int k = (int)threadIdx.x; k < nvec; k += kKlThreads) {
       const unsigned mask = sel_mask[k];
       float o[V8];
