@@ -58,8 +58,13 @@ WORKLOAD = ("weight quantization sweep: 128 MoE experts 2048x1024 + lm_head 1310
             "NVFP4 dynamic then frozen (FROZEN_ALL) quantize to packed codes + E4M3 block scales")
 # ncu DRAM bytes (read + write) per launch of the dominant kernel, from the
 # capture summarised in profiles/; valid only while quantize.cu is unchanged.
-TRAFFIC = {"kernel": "group_encode_kernel<bf16,codes> (FROZEN_ALL, whole sweep)", "bytes": None,
-           "source_sha256": None}
+# DRAM bytes of one launch of the dominant kernel, from the ncu capture in
+# profiles/group_encode_frozen_48experts.md (48 experts, 100.7M elements: read 207.64 MB +
+# write 34.80 MB = 2.407 B per element), scaled by elements to the whole sweep
+# (536,870,912 elements); valid only while quantize.cu is the source that was captured.
+TRAFFIC = {"kernel": "group_encode_kernel<bf16,codes> (FROZEN_ALL, whole sweep)",
+           "bytes": round((207.644928e6 + 34.802944e6) / (48 * 2048 * 1024) * 536870912),
+           "source_sha256": "2fbde53a7929a55538da03608c1a9454a4edff74bb12854c6aac16c8f50ab61c"}
 
 
 def peaks():
@@ -258,6 +263,7 @@ def run_ours(args, world, rank, local):
 
     secondary = {}
     if not args.no_secondary:
+        secondary["tiny"] = bench_tiny(Q, dev, stream)
         secondary["fp4_peak_probe"] = bench_fp4_peak(Q, dev, stream)
         secondary["gemm"] = bench_gemm(Q, dev, stream, P, max(3, min(K, 20)), secondary["fp4_peak_probe"])
         secondary["w4a16"] = bench_w4a16(Q, dev, stream, P, max(3, min(K, 20)))
@@ -337,6 +343,60 @@ def run_e2e(Q, xs, dev, stream, K, world):
 
 def flush_l2(buf):
     buf.zero_()
+
+
+def bench_tiny(Q, dev, stream, reps=50):
+    """The tiny QAD linear (latency-bound): microseconds per call of each step,
+    each timed as one CUDA-graph replay of `reps` back-to-back calls (no L2
+    flush: the whole working set is a few MB)."""
+    from nvfp4_quantization_aware_b200 import synthetic as S
+    d = S.tiny_qad_linear(seed=0, device=dev)
+    x, w, t, s_ = d["x"], d["w"], d["teacher"], d["student"]
+    M, K = x.shape
+    N = w.shape[0]
+    L = Q.lib()
+    ws = torch.empty(int(L.nvfp4_quantize_workspace_size(M, K, Q.DYNAMIC)), dtype=torch.uint8, device=dev)
+    xf, wf = torch.empty_like(x), torch.empty_like(w)
+    xc = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+    xsf = torch.empty(Q.mma_scales_bytes(M, K), dtype=torch.uint8, device=dev)
+    xts = torch.empty(1, dtype=torch.float32, device=dev)
+    wc, wsf, wts = Q.nvfp4_quantize(w, Q.DYNAMIC, layout=Q.SCALES_MMA)
+    c = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    grad = torch.empty_like(s_)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    kws = torch.empty(int(L.qad_kl_workspace_size(t.shape[0], t.shape[1], Q.F32)), dtype=torch.uint8, device=dev)
+    calls = {
+        "fake_quant_x_dynamic": lambda: Q.nvfp4_fake_quant(x, Q.DYNAMIC, tensor_scale=xts, out=xf, workspace=ws),
+        "fake_quant_w_dynamic": lambda: Q.nvfp4_fake_quant(w, Q.DYNAMIC, tensor_scale=xts, out=wf, workspace=ws),
+        "quantize_x_dynamic_mma": lambda: Q.nvfp4_quantize(x, Q.DYNAMIC, tensor_scale=xts, block_scales=xsf,
+                                                           layout=Q.SCALES_MMA, codes=xc, workspace=ws),
+        "gemm_w4a4_64x1024x1024": lambda: Q.nvfp4_gemm_w4a4(xc, xsf, xts, wc, wsf, wts, out=c),
+        "kl_fwd_bwd_64x8192_f32": lambda: L.qad_kl_fwd_bwd(t.data_ptr(), s_.data_ptr(), Q.F32, t.shape[0], t.shape[1],
+                                                           t.shape[1], 1.0, loss.data_ptr(), None, grad.data_ptr(),
+                                                           t.shape[1], 1.0 / t.shape[0], kws.data_ptr(), kws.numel(),
+                                                           stream.cuda_stream),
+    }
+    out = {}
+    with torch.cuda.stream(stream):
+        for name, call in calls.items():
+            call()
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(reps):
+                    call()
+            g.replay()
+            stream.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            stream.synchronize()
+            out[name + "_us"] = round(e0.elapsed_time(e1) * 1e3 / reps, 2)
+            del g
+    out["config"] = ("tiny QAD linear: X 64x1024 bf16, W 1024x1024 bf16 (0.5% outliers x30), KL over 64x8192 fp32; "
+                     "microseconds per call, back-to-back calls in one CUDA graph")
+    return out
 
 
 def bench_fp4_peak(Q, dev, stream):
