@@ -63,8 +63,8 @@ WORKLOAD = ("weight quantization sweep: 128 MoE experts 2048x1024 + lm_head 1310
 # write 34.80 MB = 2.407 B per element), scaled by elements to the whole sweep
 # (536,870,912 elements); valid only while quantize.cu is the source that was captured.
 TRAFFIC = {"kernel": "group_encode_kernel<bf16,codes> (FROZEN_ALL, whole sweep)",
-           "bytes": round((207.644928e6 + 34.802944e6) / (48 * 2048 * 1024) * 536870912),
-           "source_sha256": "2fbde53a7929a55538da03608c1a9454a4edff74bb12854c6aac16c8f50ab61c"}
+           "bytes": round((207.644416e6 + 34.831872e6) / (48 * 2048 * 1024) * 536870912),
+           "source_sha256": "276e49728b85e4d27d225d194f3922cd6738efe7b75cdb26b0abbf91d3e99a31"}
 
 
 def peaks():
@@ -264,13 +264,16 @@ def run_ours(args, world, rank, local):
     secondary = {}
     if not args.no_secondary:
         secondary["tiny"] = bench_tiny(Q, dev, stream)
-        secondary["fp4_peak_probe"] = bench_fp4_peak(Q, dev, stream)
-        secondary["gemm"] = bench_gemm(Q, dev, stream, P, max(3, min(K, 20)), secondary["fp4_peak_probe"])
+        secondary["gemm"] = bench_gemm(Q, dev, stream, P, max(3, min(K, 20)))
         secondary["w4a16"] = bench_w4a16(Q, dev, stream, P, max(3, min(K, 20)))
         secondary["kl"] = bench_kl(Q, dev, stream, P, max(3, min(K, 10)))
         secondary["kl_topk"] = bench_kl_topk(Q, dev, stream, P, max(3, min(K, 10)))
         secondary["calibrate_mse"] = bench_calibrate(Q, dev, stream, xs, 3)
         secondary["moe_step"] = bench_moe(Q, dev, stream, P, max(3, min(K, 10)))
+        # the FP4 probe runs last: its sustained launch (~70 ms at full tensor
+        # power) would lower the clocks of whatever is timed right after it
+        secondary["fp4_peak_probe"] = bench_fp4_peak(Q, dev, stream)
+        apply_fp4_peak(secondary["gemm"], secondary["fp4_peak_probe"])
     clocks = sampler.stop()
 
     cpu = None
@@ -426,6 +429,19 @@ def bench_fp4_peak(Q, dev, stream):
     res["method"] = ("tcgen05.mma.kind::mxf4nvf4.block_scale 128x256x64, UE4M3 scales, operands resident in "
                      "shared memory, one CTA per SM, CUDA events")
     return res
+
+
+def apply_fp4_peak(gemm, probe):
+    """Re-express the tensor-bound GEMM rooflines against the probe's burst peak."""
+    peak = probe.get("burst_tflops") if probe else None
+    if not peak:
+        return
+    for key, res in gemm.items():
+        r = res.get("roofline") if isinstance(res, dict) else None
+        if r and r.get("bound") == "tensor":
+            r["peak"] = peak
+            r["frac"] = round(r["achieved"] / peak, 4)
+            r["peak_source"] = "own tcgen05 FP4 MMA probe, burst (fp4_peak_probe)"
 
 
 def bench_gemm(Q, dev, stream, P, K, probe=None):

@@ -51,8 +51,8 @@ constexpr int MMA_M = 128;
 constexpr int BK = 64;
 constexpr int KB = BK / 16;
 constexpr int STAGES = 3;
-constexpr int A_BYTES = BM * BK * 2;      // 16 KiB
-constexpr int B_BYTES = BN * BK * 2;      // 32 KiB
+constexpr int A_BYTES = BM * BK * 2;      // 32 KiB
+constexpr int B_BYTES = BN * BK * 2;      // 16 KiB
 constexpr int EPI_WARPS = 4;
 constexpr int DQ_WARPS = 8;
 constexpr int DQ_THREADS = 32 * DQ_WARPS;  // == 2 BN: two threads per weight row

@@ -22,7 +22,11 @@
 // The encode is bound by instruction issue rather than by HBM, so re-reading
 // the inputs from L2 instead of HBM gains nothing: groups are cut only by the
 // number of tensors a launch holds.
+#include <cooperative_groups.h>
+
 #include "quant_common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace nvfp4 {
 
@@ -161,16 +165,13 @@ struct LaneMax<float> {
 
 constexpr int kAmaxUnroll = 4;  // chunks per warp per iteration (amax)
 
+// Per-tensor maxima of |x| over chunks [c_begin, c_end) into s_max (shared,
+// one word per tensor of the group, zeroed by the caller): warps take
+// kAmaxUnroll consecutive chunks at a time.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) group_amax_kernel(const __grid_constant__ GroupArgs a) {
-  __shared__ unsigned s_max[kMaxGroup];
-  for (int i = threadIdx.x; i < a.n; i += kThreads) s_max[i] = 0u;
-  __syncthreads();
+NVFP4_DEV void amax_range(const GroupArgs& a, int64_t c_begin, int64_t c_end, unsigned* s_max) {
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
-  const int64_t per_cta = (a.total_chunks + gridDim.x - 1) / gridDim.x;
-  const int64_t c_begin = (int64_t)blockIdx.x * per_cta;
-  const int64_t c_end = c_begin + per_cta < a.total_chunks ? c_begin + per_cta : a.total_chunks;
   int cur = 0;
   int mt = -1;      // tensor of the running max
   LaneMax<T> m;     // running max of this lane
@@ -205,6 +206,17 @@ __global__ void __launch_bounds__(kThreads) group_amax_kernel(const __grid_const
   }
   const float w = warp_max(m.value());
   if (lane == 0 && mt >= 0 && w > 0.0f) atomicMax(s_max + mt, __float_as_uint(w));
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) group_amax_kernel(const __grid_constant__ GroupArgs a) {
+  __shared__ unsigned s_max[kMaxGroup];
+  for (int i = threadIdx.x; i < a.n; i += kThreads) s_max[i] = 0u;
+  __syncthreads();
+  const int64_t per_cta = (a.total_chunks + gridDim.x - 1) / gridDim.x;
+  const int64_t c_begin = (int64_t)blockIdx.x * per_cta;
+  const int64_t c_end = c_begin + per_cta < a.total_chunks ? c_begin + per_cta : a.total_chunks;
+  amax_range<T>(a, c_begin, c_end, s_max);
   __syncthreads();
   for (int i = threadIdx.x; i < a.n; i += kThreads)
     if (s_max[i] != 0u) atomicMax(a.amax + i, s_max[i]);
@@ -256,15 +268,12 @@ NVFP4_DEV void emit_block(const GroupArgs& a, const GTensor& g, int64_t row, int
 // chunks in flight at any time form one dense front through memory).  The
 // position of a group's first chunk costs one division; the rest of the
 // group follows by increments.
-template <typename T, Out OUT>
-__global__ void __launch_bounds__(kThreads) group_encode_kernel(const __grid_constant__ GroupArgs a) {
+// The encode loop over the group's chunks, warps `warp` of `nwarps`
+// striding; SgOf(t) gives tensor t's scale s_g.
+template <typename T, Out OUT, typename SgOf>
+NVFP4_DEV void encode_range(const GroupArgs& a, int64_t warp, int64_t nwarps, SgOf sg_of) {
   const int lane = threadIdx.x & 31;
-  const int64_t warp = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
-  const int64_t nwarps = (int64_t)gridDim.x * kWarps;
   const bool frozen_all = a.mode == NVFP4_FROZEN_ALL;
-  if (a.mode == NVFP4_DYNAMIC && blockIdx.x == 0)
-    for (int i = threadIdx.x; i < a.n; i += kThreads) *a.t[i].ts = tensor_scale_of(a, i);
-
   int cur = 0;
   int sg_t = -1;  // tensor whose scale is cached below
   float sg = 0.0f, denom6 = 0.0f;
@@ -316,7 +325,7 @@ __global__ void __launch_bounds__(kThreads) group_encode_kernel(const __grid_con
       const int64_t row_u = row_[u], col = col_[u];
       if (col >= g.cols) continue;  // this lane's block lies past the row end
       if (tu != sg_t) {
-        sg = tensor_scale_of(a, tu);
+        sg = sg_of(tu);
         denom6 = __fmul_rn(6.0f, sg);
         sg_t = tu;
       }
@@ -325,6 +334,57 @@ __global__ void __launch_bounds__(kThreads) group_encode_kernel(const __grid_con
       emit_block<T, OUT>(a, g, row_u, col, v, sg, denom6, frozen_all, sb_in[u]);
     }
   }
+}
+
+template <typename T, Out OUT>
+__global__ void __launch_bounds__(kThreads) group_encode_kernel(const __grid_constant__ GroupArgs a) {
+  if (a.mode == NVFP4_DYNAMIC && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < a.n; i += kThreads) *a.t[i].ts = tensor_scale_of(a, i);
+  encode_range<T, OUT>(a, (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5), (int64_t)gridDim.x * kWarps,
+                       [&](int t) { return tensor_scale_of(a, t); });
+}
+
+// Dynamic scales for a small group in one launch: one cluster of
+// kSmallCluster CTAs takes each tensor's max |x| over its share of the chunks,
+// pushes the per-tensor maxima into every peer through distributed shared
+// memory, and after one cluster barrier every CTA holds the tensors' amax and
+// encodes its share (the second read of a small group comes from L2).  Same
+// results as the amax + encode launches; no workspace words and no clearing
+// launch.
+constexpr int kSmallCluster = 8;
+// At most 256 chunks (128K elements) take this path: eight CTAs keep too few
+// loads in flight for more (a 1M-element tensor measured 34 us this way and
+// ~12 us as amax + encode launches over the whole GPU; 64K elements: 5 us vs 12).
+constexpr int64_t kSmallChunks = 256;
+
+template <typename T, Out OUT>
+__global__ void __launch_bounds__(kThreads) group_small_dynamic_kernel(const __grid_constant__ GroupArgs a) {
+  __shared__ unsigned s_max[kMaxGroup];
+  __shared__ unsigned peer_max[kSmallCluster][kMaxGroup];  // written by every CTA of the cluster
+  cg::cluster_group cluster = cg::this_cluster();
+  const int csize = (int)cluster.num_blocks();
+  const int crank = (int)cluster.block_rank();
+  for (int i = threadIdx.x; i < a.n; i += kThreads) s_max[i] = 0u;
+  __syncthreads();
+  const int64_t per_cta = (a.total_chunks + csize - 1) / csize;
+  const int64_t c_begin = (int64_t)crank * per_cta;
+  const int64_t c_end = c_begin + per_cta < a.total_chunks ? c_begin + per_cta : a.total_chunks;
+  amax_range<T>(a, c_begin, c_end, s_max);
+  __syncthreads();
+  for (int i = threadIdx.x; i < a.n * csize; i += kThreads) {
+    const int r = i / a.n, t = i - r * a.n;
+    cluster.map_shared_rank(&peer_max[0][0], r)[crank * kMaxGroup + t] = s_max[t];
+  }
+  cluster.sync();  // every peer's maxima are here; no CTA writes a peer after this point
+  for (int i = threadIdx.x; i < a.n; i += kThreads) {
+    unsigned m = peer_max[0][i];
+    for (int r = 1; r < csize; ++r) m = max(m, peer_max[r][i]);
+    s_max[i] = m;
+    if (crank == 0) *a.t[i].ts = __fdiv_rn(__uint_as_float(m), 2688.0f);
+  }
+  __syncthreads();
+  encode_range<T, OUT>(a, (int64_t)crank * kWarps + (threadIdx.x >> 5), (int64_t)csize * kWarps,
+                       [&](int t) { return __fdiv_rn(__uint_as_float(s_max[t]), 2688.0f); });
 }
 
 // ------------------------------------------------------------------ MSE calibration
@@ -620,9 +680,34 @@ static int resident_grid(const void* fn, int64_t total_chunks) {
 
 // Launch the kernels of one group.  In DYNAMIC mode `amax` points at this
 // group's n zeroed words of the workspace.
+// One launch: a single cluster of kSmallCluster CTAs (DYNAMIC, small group).
+template <Out OUT, typename T>
+static nvfp4_status launch_small_dynamic(const GroupArgs& a, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kSmallCluster);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kSmallCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, group_small_dynamic_kernel<T, OUT>, a) != cudaSuccess) return NVFP4_ERR_CUDA;
+  count_launches(1);
+  return launch_status();
+}
+
+// DYNAMIC groups this small take the one-launch cluster path.
+static bool small_dynamic(const GroupArgs& a) { return a.mode == NVFP4_DYNAMIC && a.total_chunks <= kSmallChunks; }
+
 template <Out OUT>
 static nvfp4_status launch_group(GroupArgs& a, nvfp4_dtype dtype, unsigned* amax, cudaStream_t s) {
   if (a.n == 0 || a.total_chunks == 0) return NVFP4_OK;
+  if (small_dynamic(a))
+    return dtype == NVFP4_BF16 ? launch_small_dynamic<OUT, __nv_bfloat16>(a, s) : launch_small_dynamic<OUT, float>(a, s);
   if (a.mode == NVFP4_DYNAMIC) {
     a.amax = amax;
     if (dtype == NVFP4_BF16)
@@ -681,7 +766,7 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
   auto flush = [&]() -> nvfp4_status {
     if (a.n == 0) return NVFP4_OK;
     const int need = a.n;
-    if (mode == NVFP4_DYNAMIC && word_base + need > nwords) {
+    if (mode == NVFP4_DYNAMIC && !small_dynamic(a) && word_base + need > nwords) {
       if (cudaMemsetAsync(ws, 0, kDynamicWorkspace, s) != cudaSuccess) return NVFP4_ERR_CUDA;
       word_base = 0;
     }

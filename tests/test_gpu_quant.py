@@ -312,13 +312,29 @@ def test_grouped_mma_layout_and_fake_quant():
 def test_launch_counter_counts_kernels():
     x = S.activations(64, 256, seed=1, device=DEV)
     n0 = Q.nvfp4_launch_count()
-    Q.nvfp4_quantize(x)                      # amax + encode
+    Q.nvfp4_quantize(x)                      # small dynamic group: one cluster launch
     Q.nvfp4_quantize(x, Q.FROZEN_GLOBAL, tensor_scale=torch.ones(1, device=DEV))  # encode
-    assert Q.nvfp4_launch_count() - n0 == 3
-    xs = [S.activations(16, 64, seed=3 + i, device=DEV) for i in range(150)]   # two groups
+    assert Q.nvfp4_launch_count() - n0 == 2
+    xs = [S.activations(16, 64, seed=3 + i, device=DEV) for i in range(150)]
     n0 = Q.nvfp4_launch_count()
-    Q.nvfp4_quantize_grouped(xs)
-    assert Q.nvfp4_launch_count() - n0 == 4
+    Q.nvfp4_quantize_grouped(xs)  # 144 tensors (2304 chunks): amax + encode; 6 tensors (96 chunks): one launch
+    assert Q.nvfp4_launch_count() - n0 == 3
+    big = S.activations(64, 2064, seed=2, device=DEV)  # 320 chunks: amax + encode
+    n0 = Q.nvfp4_launch_count()
+    Q.nvfp4_quantize(big)
+    assert Q.nvfp4_launch_count() - n0 == 2
+
+
+@pytest.mark.parametrize("rows,cols", [(64, 2048), (64, 2064), (1, 16), (3, 8192), (2048, 2048)])
+def test_dynamic_small_and_large_paths_match_oracle(rows, cols):
+    # 64 x 2048 is the largest group the one-launch cluster path takes (256
+    # chunks of 512 elements); 64 x 2064 (320 chunks) takes amax + encode
+    x = S.weights(rows, cols, seed=rows + cols, device=DEV, outlier_p=0.01, outlier_mult=30)
+    codes, sb, ts = Q.nvfp4_quantize(x, Q.DYNAMIC)
+    ref_codes, ref_sb, ref_sg = O.quantize(_host_f32(x), O.DYNAMIC)
+    assert np.array_equal(codes.cpu().numpy(), ref_codes)
+    assert np.array_equal(sb.cpu().numpy(), ref_sb)
+    assert np.float32(ts.cpu().numpy()[0]).view(np.uint32) == np.float32(ref_sg).view(np.uint32)
 
 
 def test_unaligned_rows_use_narrow_accesses():
