@@ -644,14 +644,21 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
   const uint32_t m_ties = remaining;          // keys == tau that belong to S
   const bool rank_ties = m_ties < count;      // uniform across the cluster
 
+  // Vectors are owned warp-contiguously from here on: warp w takes vectors
+  // [w W, (w + 1) W), lane l the ones at w W + 32 j + l, so index order is
+  // (warp, round, lane) order and the ranking scans stay inside the warp.
+  const int W = ((nvec + kKlWarps - 1) / kKlWarps + 31) / 32 * 32;
+  const int kw0 = wid * W;
+  const unsigned lt_mask = (1u << lane) - 1u;
+
   // ---- ranks of the keys equal to tau, in index order (only when not all are taken)
-  unsigned cta_off = 0u;
+  unsigned cta_off = 0u, warp_base = 0u;
   if (rank_ties) {
-    unsigned running = 0u;
-    for (int kb = 0; kb < nvec; kb += kKlThreads) {
-      const int k = kb + (int)threadIdx.x;
+    unsigned running = 0u;  // ties in this warp's earlier vectors
+    for (int kb = kw0; kb < kw0 + W && kb < nvec; kb += 32) {  // warp-uniform trip count
+      const int k = kb + lane;
       unsigned c = 0u;
-      if (ok && k < nvec) {
+      if (ok && k < nvec && k < kw0 + W) {
 #pragma unroll
         for (int q = 0; q < WPV; ++q) {
           const uint32_t w = wt[k * WPV + q];
@@ -662,65 +669,71 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
           }
         }
       }
-      // exclusive scan of c over the round's threads (index order)
-      unsigned x = c;
+      unsigned x = c;  // inclusive scan over the lanes
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const unsigned y = __shfl_up_sync(0xFFFFFFFFu, x, o);
         if (lane >= o) x += y;
       }
-      if (lane == 31) warp_sum[wid] = x;
-      __syncthreads();
-      unsigned before = 0u, total = 0u;
-      for (int w = 0; w < kKlWarps; ++w) {
-        if (w < wid) before += warp_sum[w];
-        total += warp_sum[w];
-      }
-      if (k < nvec) vec_prefix[k] = running + before + x - c;
-      running += total;
-      __syncthreads();
+      if (k < nvec && k < kw0 + W) vec_prefix[k] = running + x - c;
+      running += __shfl_sync(0xFFFFFFFFu, x, 31);
+    }
+    if (lane == 0) warp_sum[wid] = running;
+    __syncthreads();
+    unsigned total = 0u;
+    for (int w = 0; w < kKlWarps; ++w) {
+      if (w < wid) warp_base += warp_sum[w];
+      total += warp_sum[w];
     }
     for (int r = (int)threadIdx.x; r < csize; r += kKlThreads)
-      cluster.map_shared_rank(recv_ties, r)[crank] = running;
+      cluster.map_shared_rank(recv_ties, r)[crank] = total;
     cluster.sync();
     for (int r = 0; r < crank; ++r) cta_off += recv_ties[r];
   }
-  // ---- selection mask per vector (bit e: element e of the vector is in S)
-  for (int k = (int)threadIdx.x; k < nvec; k += kKlThreads) {
-    unsigned mask = 0u, seen = 0u;
-    if constexpr (sizeof(T) == 2) {
-      if (ok && !rank_ties && k >= kfirst && k < klast) {  // every key >= tau is in S
+  // ---- selection mask per vector (bit e: element e of the vector is in S),
+  // and this warp's list of vectors with a selected element, in index order
+  // (written over the tie prefixes of vectors already read)
+  unsigned* sel_list = vec_prefix;
+  unsigned list_len = 0u;
+  for (int kb = kw0; kb < kw0 + W && kb < nvec; kb += 32) {  // warp-uniform trip count
+    const int k = kb + lane;
+    const bool mine = k < nvec && k < kw0 + W;
+    unsigned mask = 0u;
+    if (mine && ok) {
+      if (sizeof(T) == 2 && !rank_ties && k >= kfirst && k < klast) {  // every key >= tau is in S
 #pragma unroll
         for (int q = 0; q < WPV; ++q) {
           const uint32_t k2 = bf16x2_keys(wt[k * WPV + q]);
           mask |= ((k2 & 0xFFFFu) >= tau ? 1u : 0u) << (2 * q);
           mask |= ((k2 >> 16) >= tau ? 1u : 0u) << (2 * q + 1);
         }
-        sel_mask[k] = (uint8_t)mask;
-        continue;
-      }
-    }
-    if (ok) {
+      } else {
+        unsigned seen = 0u;
+        const unsigned pre = rank_ties ? cta_off + warp_base + vec_prefix[k] : 0u;
 #pragma unroll
-      for (int q = 0; q < WPV; ++q) {
-        const uint32_t w = wt[k * WPV + q];
+        for (int q = 0; q < WPV; ++q) {
+          const uint32_t w = wt[k * WPV + q];
 #pragma unroll
-        for (int h = 0; h < Kf::kPerWord; ++h) {
-          const int e = q * Kf::kPerWord + h;
-          const int j = k * V8 + e;
-          if (j < off || j >= nslots) continue;
-          const uint32_t key = Kf::key(w, h);
-          if (key > tau) {
-            mask |= 1u << e;
-          } else if (key == tau) {
-            const bool take = !rank_ties || cta_off + vec_prefix[k] + seen < m_ties;
-            if (take) mask |= 1u << e;
-            ++seen;
+          for (int h = 0; h < Kf::kPerWord; ++h) {
+            const int e = q * Kf::kPerWord + h;
+            const int j = k * V8 + e;
+            if (j < off || j >= nslots) continue;
+            const uint32_t key = Kf::key(w, h);
+            if (key > tau) {
+              mask |= 1u << e;
+            } else if (key == tau) {
+              const bool take = !rank_ties || pre + seen < m_ties;
+              if (take) mask |= 1u << e;
+              ++seen;
+            }
           }
         }
       }
     }
-    sel_mask[k] = (uint8_t)mask;
+    if (mine) sel_mask[k] = (uint8_t)mask;
+    const unsigned b = __ballot_sync(0xFFFFFFFFu, mask != 0u);  // after every lane read its prefix
+    if (mask != 0u) sel_list[kw0 + list_len + __popc(b & lt_mask)] = (unsigned)k;
+    list_len += __popc(b);
   }
   __syncthreads();
 
@@ -732,9 +745,9 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
   stats_init(my, kPadLogit * a);
   float zmt = kPadLogit, zms = kPadLogit;
   if (ok) {
-    for (int k = (int)threadIdx.x; k < nvec; k += kKlThreads) {
+    for (unsigned i = lane; i < list_len; i += 32) {  // only this warp's vectors with a selected element
+      const int k = (int)sel_list[kw0 + i];
       const unsigned mask = sel_mask[k];
-      if (mask == 0u) continue;
       float zt[V8], zs[V8];
       E::unpack(vt[k], zt);
       E::unpack(vs[k], zs);
@@ -788,22 +801,7 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
     const float Lt = Wt + __log2f(St), Ls = Ws + __log2f(Ss);
     T* gout = reinterpret_cast<T*>(args.dlogits) + row * args.ld_grad + v0 - off;  // slot j -> gout[j]
     const bool vec_ok = (((uintptr_t)gout) & 15u) == 0;
-    for (int k = (int)threadIdx.x; k < nvec; k += kKlThreads) {
-      const unsigned mask = sel_mask[k];
-      float o[V8];
-      if (mask == 0u) {
-#pragma unroll
-        for (int e = 0; e < V8; ++e) o[e] = 0.0f;
-      } else {
-        float zt[V8], zs[V8];
-        E::unpack(vt[k], zt);
-        E::unpack(vs[k], zs);
-#pragma unroll
-        for (int e = 0; e < V8; ++e) {
-          const float pt = ex2(fmaf(zt[e], a, -Lt)), ps = ex2(fmaf(zs[e], a, -Ls));
-          o[e] = ((mask >> e) & 1u) ? g * (ps - pt) : 0.0f;
-        }
-      }
+    auto store_vec = [&](int k, const float (&o)[V8]) {
       const int j0 = k * V8;
       if (vec_ok && k >= kfirst && k < klast) {
         st_stream_v4(gout + j0, E::pack(o));
@@ -812,6 +810,28 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
         for (int e = 0; e < V8; ++e)
           if (j0 + e >= off && j0 + e < nslots) E::store1(gout + j0 + e, o[e]);
       }
+    };
+    // vectors with a selected element: this warp's list
+    for (unsigned i = lane; i < list_len; i += 32) {
+      const int k = (int)sel_list[kw0 + i];
+      const unsigned mask = sel_mask[k];
+      float zt[V8], zs[V8], o[V8];
+      E::unpack(vt[k], zt);
+      E::unpack(vs[k], zs);
+#pragma unroll
+      for (int e = 0; e < V8; ++e) {
+        const float pt = ex2(fmaf(zt[e], a, -Lt)), ps = ex2(fmaf(zs[e], a, -Ls));
+        o[e] = ((mask >> e) & 1u) ? g * (ps - pt) : 0.0f;
+      }
+      store_vec(k, o);
+    }
+    // the rest: zeros
+    for (int k = (int)threadIdx.x; k < nvec; k += kKlThreads) {
+      if (sel_mask[k] != 0u) continue;
+      float o[V8];
+#pragma unroll
+      for (int e = 0; e < V8; ++e) o[e] = 0.0f;
+      store_vec(k, o);
     }
   }
 }
