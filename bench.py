@@ -19,6 +19,10 @@ Also measured in the same run and reported under "gemm" and "kl":
   * weight-only NVFP4 (key "w4a16"): the same GEMM shapes with bf16
     activations, the weights dequantized in the main loop, beside W4A4 and
     the BF16 GEMM of the dequantized weights;
+  * the tiny QAD linear (key "tiny"): microseconds per call of its dynamic
+    fake-quant, quantize, GEMM and KL steps;
+  * the dense FP4 MMA peak measured by the library's own probe (key
+    "fp4_peak_probe", run last), which the GEMM's roofline takes as its peak;
   * the MSE block-scale calibration of the 128 expert weights ("calibrate_mse");
   * the MoE layer step (config "moe_step"): 4096 tokens, 128 routed experts
     + 1 shared, top-6, forward (grouped W4A4) + straight-through backward

@@ -35,7 +35,7 @@ __global__ void __launch_bounds__(THREADS, 1) fp4_mma_probe_kernel(int64_t iters
   uint8_t* sB = sA + A_BYTES;
   __shared__ uint64_t done;
   __shared__ uint32_t tmem_slot;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
 
   // operands: a fixed pseudo-random byte pattern (a multiplicative hash of the
   // byte index), so the MMAs see mixed codes rather than zeros
@@ -81,7 +81,6 @@ __global__ void __launch_bounds__(THREADS, 1) fp4_mma_probe_kernel(int64_t iters
     tc_fence_after();
     tmem_dealloc(tmem, TM_COLS);
   }
-  (void)lane;
 }
 
 }  // namespace probe
