@@ -475,7 +475,7 @@ nvfp4_status nvfp4_moe_swiglu_quantize(const void* h_gate, const void* h_up, int
 
 /* out[t] = bf16( sum_j w[t,j] * y[slot_row[t,j]] + y[seg_off[experts] + t] ),
  * binary32 sums in the order j = 0..topk-1, then the shared expert; y bf16
- * rows x cols (cols % 8 == 0), out bf16 tokens x cols. */
+ * rows x cols (cols % 8 == 0), out bf16 tokens x cols; 1 <= topk <= 32. */
 nvfp4_status nvfp4_moe_combine(const void* y, int64_t cols, const int32_t* slot_row, const float* combine_weights,
                                int tokens, int topk, const int32_t* seg_off, int experts, void* out, void* stream);
 
@@ -484,7 +484,8 @@ nvfp4_status nvfp4_moe_combine(const void* y, int64_t cols, const int32_t* slot_
 nvfp4_status nvfp4_moe_scale_rows(const void* dy, int64_t cols, const int32_t* row_token, const float* row_weight,
                                   const int32_t* seg_off, int groups, int64_t rows_cap, void* dyp, void* stream);
 
-/* SwiGLU backward, binary32: s = 1 / (1 + expf(-g)),
+/* SwiGLU backward, binary32 with the hardware exponential and a fast
+ * reciprocal for s = 1 / (1 + exp(-g)) (relative error ~1e-6),
  *   dG = da * u * s * (1 + g (1 - s)),  dU = da * g * s,
  * written as dgu[r] = [dG | dU] (bf16 rows_cap x 2 cols); da, h_gate, h_up
  * bf16 rows_cap x cols contiguous; zeros on padding rows.  cols % 8 == 0,
@@ -493,7 +494,8 @@ nvfp4_status nvfp4_moe_swiglu_backward(const void* da, const void* h_gate, const
                                        const int32_t* row_token, const int32_t* seg_off, int groups,
                                        int64_t rows_cap, void* dgu, void* stream);
 
-/* dx[t] = bf16( sum_j dxp[slot_row[t,j]] + dxp[seg_off[experts] + t] ). */
+/* dx[t] = bf16( sum_j dxp[slot_row[t,j]] + dxp[seg_off[experts] + t] ), slots in order
+ * j = 0..topk-1 then the shared expert; 1 <= topk <= 32. */
 nvfp4_status nvfp4_moe_gather_sum(const void* dxp, int64_t cols, const int32_t* slot_row, int tokens, int topk,
                                   const int32_t* seg_off, int experts, void* dx, void* stream);
 
@@ -513,7 +515,7 @@ typedef struct qad_moe_shape {
   int hidden;    /* H, % 256 == 0 */
   int ffn;       /* F, % 256 == 0 */
   int experts;   /* routed experts E (group E is the shared expert), E + 1 <= 256 */
-  int topk;      /* routed experts per token, <= E */
+  int topk;      /* routed experts per token, <= E and <= 32 */
   int save_act;  /* nonzero: the forward also stores a (pre-quantization) in QAD_MOE_ACT */
 } qad_moe_shape;
 

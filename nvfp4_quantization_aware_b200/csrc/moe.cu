@@ -223,31 +223,37 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantRowsArgs a) {
 __global__ void combine_kernel(const __nv_bfloat16* __restrict__ y, int cols, const int32_t* __restrict__ slot_row,
                                const float* __restrict__ weights, int tokens, int topk,
                                const int32_t* __restrict__ off, int experts, __nv_bfloat16* __restrict__ out) {
+  // one warp per token: its slot rows and weights are read once, the lanes
+  // stride over the row's 16-byte vectors
+  const int lane = threadIdx.x & 31;
   const int vpr = cols / 8;
   const int shared_base = __ldg(off + experts);
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)tokens * vpr;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int t = (int)(i / vpr);
-    const int c = (int)(i - (int64_t)t * vpr) * 8;
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int j = 0; j < topk; ++j) {
-      const int r = __ldg(slot_row + t * topk + j);
-      if (r < 0) continue;
-      const float w = __ldg(weights + t * topk + j);
-      const uint4 v = *reinterpret_cast<const uint4*>(y + (int64_t)r * cols + c);
-      acc[0] = fmaf(w, bf16lo_to_f32(v.x), acc[0]); acc[1] = fmaf(w, bf16hi_to_f32(v.x), acc[1]);
-      acc[2] = fmaf(w, bf16lo_to_f32(v.y), acc[2]); acc[3] = fmaf(w, bf16hi_to_f32(v.y), acc[3]);
-      acc[4] = fmaf(w, bf16lo_to_f32(v.z), acc[4]); acc[5] = fmaf(w, bf16hi_to_f32(v.z), acc[5]);
-      acc[6] = fmaf(w, bf16lo_to_f32(v.w), acc[6]); acc[7] = fmaf(w, bf16hi_to_f32(v.w), acc[7]);
+  const int warps = (int)(gridDim.x * blockDim.x / 32);
+  for (int t = (int)((blockIdx.x * blockDim.x + threadIdx.x) / 32); t < tokens; t += warps) {
+    const int my_r = lane < topk ? __ldg(slot_row + (int64_t)t * topk + lane) : -1;
+    const float my_w = lane < topk ? __ldg(weights + (int64_t)t * topk + lane) : 0.0f;
+    for (int vc = lane; vc < vpr; vc += 32) {
+      const int c = vc * 8;
+      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int j = 0; j < topk; ++j) {
+        const int r = __shfl_sync(0xFFFFFFFFu, my_r, j);
+        const float w = __shfl_sync(0xFFFFFFFFu, my_w, j);
+        if (r < 0) continue;
+        const uint4 v = *reinterpret_cast<const uint4*>(y + (int64_t)r * cols + c);
+        acc[0] = fmaf(w, bf16lo_to_f32(v.x), acc[0]); acc[1] = fmaf(w, bf16hi_to_f32(v.x), acc[1]);
+        acc[2] = fmaf(w, bf16lo_to_f32(v.y), acc[2]); acc[3] = fmaf(w, bf16hi_to_f32(v.y), acc[3]);
+        acc[4] = fmaf(w, bf16lo_to_f32(v.z), acc[4]); acc[5] = fmaf(w, bf16hi_to_f32(v.z), acc[5]);
+        acc[6] = fmaf(w, bf16lo_to_f32(v.w), acc[6]); acc[7] = fmaf(w, bf16hi_to_f32(v.w), acc[7]);
+      }
+      const uint4 v = *reinterpret_cast<const uint4*>(y + (int64_t)(shared_base + t) * cols + c);
+      acc[0] += bf16lo_to_f32(v.x); acc[1] += bf16hi_to_f32(v.x);
+      acc[2] += bf16lo_to_f32(v.y); acc[3] += bf16hi_to_f32(v.y);
+      acc[4] += bf16lo_to_f32(v.z); acc[5] += bf16hi_to_f32(v.z);
+      acc[6] += bf16lo_to_f32(v.w); acc[7] += bf16hi_to_f32(v.w);
+      *reinterpret_cast<uint4*>(out + (int64_t)t * cols + c) =
+          make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                     pack_bf16x2(acc[6], acc[7]));
     }
-    const uint4 v = *reinterpret_cast<const uint4*>(y + (int64_t)(shared_base + t) * cols + c);
-    acc[0] += bf16lo_to_f32(v.x); acc[1] += bf16hi_to_f32(v.x);
-    acc[2] += bf16lo_to_f32(v.y); acc[3] += bf16hi_to_f32(v.y);
-    acc[4] += bf16lo_to_f32(v.z); acc[5] += bf16hi_to_f32(v.z);
-    acc[6] += bf16lo_to_f32(v.w); acc[7] += bf16hi_to_f32(v.w);
-    *reinterpret_cast<uint4*>(out + (int64_t)t * cols + c) =
-        make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
-                   pack_bf16x2(acc[6], acc[7]));
   }
 }
 
@@ -255,67 +261,75 @@ __global__ void combine_kernel(const __nv_bfloat16* __restrict__ y, int cols, co
 __global__ void scale_rows_kernel(const __nv_bfloat16* __restrict__ dy, int cols, const int32_t* __restrict__ row_token,
                                   const float* __restrict__ row_weight, const int32_t* __restrict__ off, int groups,
                                   int rows_cap, __nv_bfloat16* __restrict__ dyp) {
+  // one warp per row: its token and weight are read once, the lanes stride
+  // over the row's 16-byte vectors
+  const int lane = threadIdx.x & 31;
   const int vpr = cols / 8;
   const int end_rows = __ldg(off + groups);
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)rows_cap * vpr;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int r = (int)(i / vpr);
-    const int c = (int)(i - (int64_t)r * vpr) * 8;
+  const int warps = (int)(gridDim.x * blockDim.x / 32);
+  for (int r = (int)((blockIdx.x * blockDim.x + threadIdx.x) / 32); r < rows_cap; r += warps) {
     const int t = r < end_rows ? __ldg(row_token + r) : -1;
-    uint4 o = make_uint4(0, 0, 0, 0);
-    if (t >= 0) {
-      const float w = __ldg(row_weight + r);
-      const uint4 v = *reinterpret_cast<const uint4*>(dy + (int64_t)t * cols + c);
-      o = make_uint4(pack_bf16x2(w * bf16lo_to_f32(v.x), w * bf16hi_to_f32(v.x)),
-                     pack_bf16x2(w * bf16lo_to_f32(v.y), w * bf16hi_to_f32(v.y)),
-                     pack_bf16x2(w * bf16lo_to_f32(v.z), w * bf16hi_to_f32(v.z)),
-                     pack_bf16x2(w * bf16lo_to_f32(v.w), w * bf16hi_to_f32(v.w)));
+    const float w = t >= 0 ? __ldg(row_weight + r) : 0.0f;
+    __nv_bfloat16* drow = dyp + (int64_t)r * cols;
+    const __nv_bfloat16* srow = dy + (int64_t)(t >= 0 ? t : 0) * cols;
+    for (int vc = lane; vc < vpr; vc += 32) {
+      uint4 o = make_uint4(0, 0, 0, 0);
+      if (t >= 0) {
+        const uint4 v = *reinterpret_cast<const uint4*>(srow + vc * 8);
+        o = make_uint4(pack_bf16x2(w * bf16lo_to_f32(v.x), w * bf16hi_to_f32(v.x)),
+                       pack_bf16x2(w * bf16lo_to_f32(v.y), w * bf16hi_to_f32(v.y)),
+                       pack_bf16x2(w * bf16lo_to_f32(v.z), w * bf16hi_to_f32(v.z)),
+                       pack_bf16x2(w * bf16lo_to_f32(v.w), w * bf16hi_to_f32(v.w)));
+      }
+      *reinterpret_cast<uint4*>(drow + vc * 8) = o;
     }
-    *reinterpret_cast<uint4*>(dyp + (int64_t)r * cols + c) = o;
   }
 }
 
 // SwiGLU backward: with s = sigmoid(g), silu(g) = g s,
 //   dg = da * u * s * (1 + g (1 - s)),  du = da * silu(g);
-// written as dgu[r] = [dg | du] (zero on padding rows).
+// written as dgu[r] = [dg | du] (zero on padding rows).  s comes from the
+// hardware exponential and a fast reciprocal (relative error ~1e-6; these
+// gradients feed no rounding decision), one warp per row.
 __global__ void swiglu_bwd_kernel(const __nv_bfloat16* __restrict__ da, const __nv_bfloat16* __restrict__ hg,
                                   const __nv_bfloat16* __restrict__ hu, int cols, const int32_t* __restrict__ row_token,
                                   const int32_t* __restrict__ off, int groups, int rows_cap,
                                   __nv_bfloat16* __restrict__ dgu) {
-  // 8 consecutive columns per thread (16-byte loads and stores)
+  const int lane = threadIdx.x & 31;
   const int end_rows = __ldg(off + groups);
   const int vpr = cols / 8;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)rows_cap * vpr;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int r = (int)(i / vpr);
-    const int c = (int)(i - (int64_t)r * vpr) * 8;
+  const int warps = (int)(gridDim.x * blockDim.x / 32);
+  for (int r = (int)((blockIdx.x * blockDim.x + threadIdx.x) / 32); r < rows_cap; r += warps) {
     const int t = r < end_rows ? __ldg(row_token + r) : -1;
-    uint4 og = make_uint4(0, 0, 0, 0), ou = make_uint4(0, 0, 0, 0);
-    if (t >= 0) {
-      const int64_t e = (int64_t)r * cols + c;
-      const uint4 G = ld_stream_v4(hg + e), U = ld_stream_v4(hu + e), D = ld_stream_v4(da + e);
-      const uint32_t gw[4] = {G.x, G.y, G.z, G.w}, uw[4] = {U.x, U.y, U.z, U.w}, dw[4] = {D.x, D.y, D.z, D.w};
-      uint32_t rg[4], ru[4];
+    for (int vc = lane; vc < vpr; vc += 32) {
+      const int c = vc * 8;
+      uint4 og = make_uint4(0, 0, 0, 0), ou = make_uint4(0, 0, 0, 0);
+      if (t >= 0) {
+        const int64_t e = (int64_t)r * cols + c;
+        const uint4 G = ld_stream_v4(hg + e), U = ld_stream_v4(hu + e), D = ld_stream_v4(da + e);
+        const uint32_t gw[4] = {G.x, G.y, G.z, G.w}, uw[4] = {U.x, U.y, U.z, U.w}, dw[4] = {D.x, D.y, D.z, D.w};
+        uint32_t rg[4], ru[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        float dg2[2], du2[2];
+        for (int k = 0; k < 4; ++k) {
+          float dg2[2], du2[2];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float g = h ? bf16hi_to_f32(gw[k]) : bf16lo_to_f32(gw[k]);
-          const float u = h ? bf16hi_to_f32(uw[k]) : bf16lo_to_f32(uw[k]);
-          const float d = h ? bf16hi_to_f32(dw[k]) : bf16lo_to_f32(dw[k]);
-          const float sg = 1.0f / (1.0f + expf(-g));
-          dg2[h] = d * u * sg * (1.0f + g * (1.0f - sg));
-          du2[h] = d * g * sg;
+          for (int h = 0; h < 2; ++h) {
+            const float g = h ? bf16hi_to_f32(gw[k]) : bf16lo_to_f32(gw[k]);
+            const float u = h ? bf16hi_to_f32(uw[k]) : bf16lo_to_f32(uw[k]);
+            const float d = h ? bf16hi_to_f32(dw[k]) : bf16lo_to_f32(dw[k]);
+            const float sg = __fdividef(1.0f, 1.0f + __expf(-g));
+            dg2[h] = d * u * sg * (1.0f + g * (1.0f - sg));
+            du2[h] = d * g * sg;
+          }
+          rg[k] = pack_bf16x2(dg2[0], dg2[1]);
+          ru[k] = pack_bf16x2(du2[0], du2[1]);
         }
-        rg[k] = pack_bf16x2(dg2[0], dg2[1]);
-        ru[k] = pack_bf16x2(du2[0], du2[1]);
+        og = make_uint4(rg[0], rg[1], rg[2], rg[3]);
+        ou = make_uint4(ru[0], ru[1], ru[2], ru[3]);
       }
-      og = make_uint4(rg[0], rg[1], rg[2], rg[3]);
-      ou = make_uint4(ru[0], ru[1], ru[2], ru[3]);
+      st_stream_v4(dgu + (int64_t)r * 2 * cols + c, og);
+      st_stream_v4(dgu + (int64_t)r * 2 * cols + cols + c, ou);
     }
-    st_stream_v4(dgu + (int64_t)r * 2 * cols + c, og);
-    st_stream_v4(dgu + (int64_t)r * 2 * cols + cols + c, ou);
   }
 }
 
@@ -323,25 +337,30 @@ __global__ void swiglu_bwd_kernel(const __nv_bfloat16* __restrict__ da, const __
 __global__ void gather_sum_kernel(const __nv_bfloat16* __restrict__ dxp, int cols, const int32_t* __restrict__ slot_row,
                                   int tokens, int topk, const int32_t* __restrict__ off, int experts,
                                   __nv_bfloat16* __restrict__ dx) {
+  // one warp per token (its slot rows read once), lanes over 16-byte vectors
+  const int lane = threadIdx.x & 31;
   const int vpr = cols / 8;
   const int shared_base = __ldg(off + experts);
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)tokens * vpr;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int t = (int)(i / vpr);
-    const int c = (int)(i - (int64_t)t * vpr) * 8;
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int j = 0; j <= topk; ++j) {
-      const int r = j < topk ? __ldg(slot_row + t * topk + j) : shared_base + t;
-      if (r < 0) continue;
-      const uint4 v = *reinterpret_cast<const uint4*>(dxp + (int64_t)r * cols + c);
-      acc[0] += bf16lo_to_f32(v.x); acc[1] += bf16hi_to_f32(v.x);
-      acc[2] += bf16lo_to_f32(v.y); acc[3] += bf16hi_to_f32(v.y);
-      acc[4] += bf16lo_to_f32(v.z); acc[5] += bf16hi_to_f32(v.z);
-      acc[6] += bf16lo_to_f32(v.w); acc[7] += bf16hi_to_f32(v.w);
+  const int warps = (int)(gridDim.x * blockDim.x / 32);
+  for (int t = (int)((blockIdx.x * blockDim.x + threadIdx.x) / 32); t < tokens; t += warps) {
+    const int my_r = lane < topk ? __ldg(slot_row + (int64_t)t * topk + lane) : -1;
+    for (int vc = lane; vc < vpr; vc += 32) {
+      const int c = vc * 8;
+      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int j = 0; j <= topk; ++j) {
+        const int rj = __shfl_sync(0xFFFFFFFFu, my_r, j < topk ? j : 0);
+        const int r = j < topk ? rj : shared_base + t;
+        if (r < 0) continue;
+        const uint4 v = *reinterpret_cast<const uint4*>(dxp + (int64_t)r * cols + c);
+        acc[0] += bf16lo_to_f32(v.x); acc[1] += bf16hi_to_f32(v.x);
+        acc[2] += bf16lo_to_f32(v.y); acc[3] += bf16hi_to_f32(v.y);
+        acc[4] += bf16lo_to_f32(v.z); acc[5] += bf16hi_to_f32(v.z);
+        acc[6] += bf16lo_to_f32(v.w); acc[7] += bf16hi_to_f32(v.w);
+      }
+      *reinterpret_cast<uint4*>(dx + (int64_t)t * cols + c) =
+          make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                     pack_bf16x2(acc[6], acc[7]));
     }
-    *reinterpret_cast<uint4*>(dx + (int64_t)t * cols + c) =
-        make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
-                   pack_bf16x2(acc[6], acc[7]));
   }
 }
 
@@ -476,7 +495,7 @@ nvfp4_status nvfp4_moe_swiglu_quantize(const void* h_gate, const void* h_up, int
 
 nvfp4_status nvfp4_moe_combine(const void* y, int64_t cols, const int32_t* slot_row, const float* combine_weights,
                                int tokens, int topk, const int32_t* seg_off, int experts, void* out, void* stream) {
-  if (cols < 8 || cols % 8 || tokens < 1 || topk < 1) return NVFP4_ERR_SHAPE;
+  if (cols < 8 || cols % 8 || tokens < 1 || topk < 1 || topk > 32) return NVFP4_ERR_SHAPE;
   if (!y || !slot_row || !combine_weights || !seg_off || !out) return NVFP4_ERR_ARG;
   if (((uintptr_t)y & 15u) || ((uintptr_t)out & 15u)) return NVFP4_ERR_ALIGN;
   combine_kernel<<<sms() * 8, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const __nv_bfloat16*>(y), (int)cols,
@@ -512,7 +531,7 @@ nvfp4_status nvfp4_moe_swiglu_backward(const void* da, const void* h_gate, const
 
 nvfp4_status nvfp4_moe_gather_sum(const void* dxp, int64_t cols, const int32_t* slot_row, int tokens, int topk,
                                   const int32_t* seg_off, int experts, void* dx, void* stream) {
-  if (cols < 8 || cols % 8 || tokens < 1 || topk < 1) return NVFP4_ERR_SHAPE;
+  if (cols < 8 || cols % 8 || tokens < 1 || topk < 1 || topk > 32) return NVFP4_ERR_SHAPE;
   if (!dxp || !slot_row || !seg_off || !dx) return NVFP4_ERR_ARG;
   if (((uintptr_t)dxp & 15u) || ((uintptr_t)dx & 15u)) return NVFP4_ERR_ALIGN;
   gather_sum_kernel<<<sms() * 8, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const __nv_bfloat16*>(dxp), (int)cols,

@@ -31,7 +31,7 @@ struct Layout {
 
 bool shape_ok(const qad_moe_shape* s) {
   return s && s->tokens >= 1 && s->topk >= 1 && s->experts >= 1 && s->experts + 1 <= 256 && s->hidden >= 256 &&
-         s->hidden % 256 == 0 && s->ffn >= 256 && s->ffn % 256 == 0 && s->topk <= s->experts &&
+         s->hidden % 256 == 0 && s->ffn >= 256 && s->ffn % 256 == 0 && s->topk <= s->experts && s->topk <= 32 &&
          (int64_t)s->tokens * s->topk <= (1 << 26) && (int64_t)(s->experts + 1) * s->hidden * s->ffn * 2 < (1ll << 40);
 }
 
