@@ -1,7 +1,8 @@
 // ptx.cuh -- thin wrappers over the sm_100a PTX used by the TMA / tcgen05
 // kernels: mbarriers (all waits bounded), TMA tensor and bulk copies (no
 // cluster multicast anywhere), tcgen05 TMEM allocation, block-scaled MMA,
-// shared->tensor-memory copies and tensor-memory loads.
+// shared->tensor-memory copies and tensor-memory loads, and the CTA-pair
+// (tcgen05 .cta_group::2) forms used by two-SM MMA kernels.
 #pragma once
 
 #include "common.cuh"
@@ -247,5 +248,97 @@ NVFP4_DEV void tmem_st_32x32b_x4(uint32_t taddr, uint4 v) {
 
 // Wait until this thread's tcgen05.st have completed.
 NVFP4_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// ------------------------------------------------------------------ CTA pairs
+//
+// A cluster of two CTAs (ranks 0 and 1, one TPC) whose tensor cores execute
+// one M = 256 MMA together (tcgen05 .cta_group::2): rank 0 issues the MMAs,
+// each CTA holds its own operand rows at the same shared-memory offsets and
+// its own rows of the accumulator in its tensor memory.  Every tcgen05
+// allocation, MMA and commit of such a kernel uses .cta_group::2.
+
+NVFP4_DEV uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Shared::cluster address of the object at `p` in CTA `rank` of this cluster.
+NVFP4_DEV uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+
+// Every thread of both CTAs (may be called from diverged warps).
+NVFP4_DEV void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// Barriers of a pair kernel are waited on and arrived at with the default
+// (CTA-scope) semantics: what they order is tcgen05 work made complete by
+// tcgen05.wait / commit and the tcgen05 thread-sync fences, and TMA bytes
+// counted by complete_tx, not plain memory traffic.  Cluster-scope acquire /
+// release forms put a memory fence on the MMA thread's path every stage.
+
+// Arrive on a barrier given by its shared::cluster address (either CTA).
+NVFP4_DEV void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
+// 2-D tiled tensor load into this CTA's shared memory whose completion is
+// counted on a barrier of either CTA of the pair (no multicast).
+NVFP4_DEV void tma_load_2d_pair(void* dst, const void* tmap, int32_t x, int32_t y, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+
+// One warp of each CTA of the pair, same warp index and same `dst_smem` offset.
+NVFP4_DEV void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+
+NVFP4_DEV void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+NVFP4_DEV void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Arrive on the barrier at shared::cluster address `bar_cluster` (this CTA's
+// or the peer's) once the pair MMAs issued so far by this thread completed.
+NVFP4_DEV void tc_commit_pair(uint32_t bar_cluster) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cluster)
+               : "memory");
+}
+
+// Pair form of mma_fp4_block16: M = 256 split as 128 rows per CTA; B's N
+// columns split as N/2 rows of B per CTA; each CTA's tensor memory holds the
+// scales of its own A rows and of all N rows of B.
+NVFP4_DEV void mma_fp4_block16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                    uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Pair form of mma_bf16 (kind::f16, M = 256).
+NVFP4_DEV void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
 }  // namespace nvfp4

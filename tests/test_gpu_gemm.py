@@ -63,7 +63,9 @@ def test_tiny_qad_linear():
 
 @pytest.mark.parametrize("M,N,K", [(1, 8, 64), (127, 100, 192), (129, 256, 320), (200, 300, 1024),
                                    (64, 520, 256), (256, 512, 576), (3, 1000, 2048), (5, 1002, 1024),
-                                   (130, 4096, 4096), (1, 256, 8192)])
+                                   (130, 4096, 4096), (1, 256, 8192),
+                                   # CTA-pair path: more 256 x 256 tiles than resident pairs, long K
+                                   (2304, 2560, 576), (300, 520, 4096)])
 def test_ragged_shapes(M, N, K):
     x = S.activations(M, K, seed=M + K, device=DEV)
     w = S.weights(N, K, seed=N + K, device=DEV)
