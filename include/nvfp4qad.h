@@ -652,7 +652,9 @@ nvfp4_status qad_kl_topk_fwd_bwd(const void* teacher, const void* student, nvfp4
  *     launch.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture.
+ *     that first call before any stream capture.  Calls made outside a
+ *     capture look the address up again, so after a cudaDeviceReset the
+ *     first call must again come before any capture.
  *   - All calls on a device share the array and each call overwrites it: two
  *     calls that can run at the same time on the GPU (different streams,
  *     without ordering between them) race and may return wrong losses.

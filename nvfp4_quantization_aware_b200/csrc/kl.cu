@@ -30,6 +30,8 @@
 // order (in double) into the mean, so the loss is deterministic.
 #include <cooperative_groups.h>
 
+#include <atomic>
+
 #include "ptx.cuh"
 
 namespace cg = cooperative_groups;
@@ -1038,22 +1040,29 @@ namespace nvfp4 {
 constexpr int64_t kKlNoAllocMaxRows = 65536;
 static __device__ __align__(256) float g_kl_noalloc_rows[kKlNoAllocMaxRows];
 
-// Device address of g_kl_noalloc_rows, looked up once per device.  In host
-// code the array's name only stands for the symbol; the address a kernel may
-// use comes from cudaGetSymbolAddress with that device current.
+// Device address of g_kl_noalloc_rows per device.  In host code the array's
+// name only stands for the symbol; the address a kernel may use comes from
+// cudaGetSymbolAddress with that device current.  The first call on a device
+// looks it up; later calls outside a stream capture look it up again (cheap,
+// and correct after a cudaDeviceReset reloaded the module), calls inside a
+// capture use the cached value.
 constexpr int kKlNoAllocMaxDevices = 64;
-static void* g_kl_noalloc_ptr[kKlNoAllocMaxDevices] = {};
+static std::atomic<void*> g_kl_noalloc_ptr[kKlNoAllocMaxDevices];
 
-static nvfp4_status kl_noalloc_scratch(void** out) {
+static nvfp4_status kl_noalloc_scratch(cudaStream_t stream, void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
   if (dev < 0 || dev >= kKlNoAllocMaxDevices) return NVFP4_ERR_UNSUPPORTED;
-  if (g_kl_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_kl_noalloc_rows) != cudaSuccess || p == nullptr) return NVFP4_ERR_CUDA;
-    g_kl_noalloc_ptr[dev] = p;
+  void* p = g_kl_noalloc_ptr[dev].load(std::memory_order_acquire);
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusActive;
+  const bool capturing = cudaStreamIsCapturing(stream, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone;
+  if (p == nullptr || !capturing) {
+    void* q = nullptr;
+    if (cudaGetSymbolAddress(&q, g_kl_noalloc_rows) != cudaSuccess || q == nullptr) return NVFP4_ERR_CUDA;
+    g_kl_noalloc_ptr[dev].store(q, std::memory_order_release);
+    p = q;
   }
-  *out = g_kl_noalloc_ptr[dev];
+  *out = p;
   return NVFP4_OK;
 }
 
@@ -1065,7 +1074,7 @@ extern "C" nvfp4_status qad_kl_fwd_bwd_noalloc(const void* teacher, const void* 
                                                float grad_scale, void* stream) {
   if (rows > nvfp4::kKlNoAllocMaxRows) return NVFP4_ERR_SHAPE;
   void* scratch = nullptr;
-  nvfp4_status st = nvfp4::kl_noalloc_scratch(&scratch);
+  nvfp4_status st = nvfp4::kl_noalloc_scratch((cudaStream_t)stream, &scratch);
   if (st != NVFP4_OK) return st;
   // every row's slot is written before it is read, so nothing needs clearing
   return qad_kl_fwd_bwd(teacher, student, dtype, rows, vocab, ld, temperature, loss, row_kl, dlogits, ld_grad,

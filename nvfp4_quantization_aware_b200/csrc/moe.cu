@@ -232,19 +232,24 @@ __global__ void combine_kernel(const __nv_bfloat16* __restrict__ y, int cols, co
   for (int t = (int)((blockIdx.x * blockDim.x + threadIdx.x) / 32); t < tokens; t += warps) {
     const int my_r = lane < topk ? __ldg(slot_row + (int64_t)t * topk + lane) : -1;
     const float my_w = lane < topk ? __ldg(weights + (int64_t)t * topk + lane) : 0.0f;
-    for (int vc = lane; vc < vpr; vc += 32) {
+    // warp-uniform trip count: every lane takes part in every shuffle; only
+    // the loads and the store are predicated on the lane's vector
+    for (int vb = 0; vb < vpr; vb += 32) {
+      const int vc = vb + lane;
+      const bool act = vc < vpr;
       const int c = vc * 8;
       float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       for (int j = 0; j < topk; ++j) {
         const int r = __shfl_sync(0xFFFFFFFFu, my_r, j);
         const float w = __shfl_sync(0xFFFFFFFFu, my_w, j);
-        if (r < 0) continue;
+        if (r < 0 || !act) continue;
         const uint4 v = *reinterpret_cast<const uint4*>(y + (int64_t)r * cols + c);
         acc[0] = fmaf(w, bf16lo_to_f32(v.x), acc[0]); acc[1] = fmaf(w, bf16hi_to_f32(v.x), acc[1]);
         acc[2] = fmaf(w, bf16lo_to_f32(v.y), acc[2]); acc[3] = fmaf(w, bf16hi_to_f32(v.y), acc[3]);
         acc[4] = fmaf(w, bf16lo_to_f32(v.z), acc[4]); acc[5] = fmaf(w, bf16hi_to_f32(v.z), acc[5]);
         acc[6] = fmaf(w, bf16lo_to_f32(v.w), acc[6]); acc[7] = fmaf(w, bf16hi_to_f32(v.w), acc[7]);
       }
+      if (!act) continue;
       const uint4 v = *reinterpret_cast<const uint4*>(y + (int64_t)(shared_base + t) * cols + c);
       acc[0] += bf16lo_to_f32(v.x); acc[1] += bf16hi_to_f32(v.x);
       acc[2] += bf16lo_to_f32(v.y); acc[3] += bf16hi_to_f32(v.y);
@@ -344,19 +349,23 @@ __global__ void gather_sum_kernel(const __nv_bfloat16* __restrict__ dxp, int col
   const int warps = (int)(gridDim.x * blockDim.x / 32);
   for (int t = (int)((blockIdx.x * blockDim.x + threadIdx.x) / 32); t < tokens; t += warps) {
     const int my_r = lane < topk ? __ldg(slot_row + (int64_t)t * topk + lane) : -1;
-    for (int vc = lane; vc < vpr; vc += 32) {
+    // warp-uniform trip count (all lanes shuffle); loads and store predicated
+    for (int vb = 0; vb < vpr; vb += 32) {
+      const int vc = vb + lane;
+      const bool act = vc < vpr;
       const int c = vc * 8;
       float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       for (int j = 0; j <= topk; ++j) {
         const int rj = __shfl_sync(0xFFFFFFFFu, my_r, j < topk ? j : 0);
         const int r = j < topk ? rj : shared_base + t;
-        if (r < 0) continue;
+        if (r < 0 || !act) continue;
         const uint4 v = *reinterpret_cast<const uint4*>(dxp + (int64_t)r * cols + c);
         acc[0] += bf16lo_to_f32(v.x); acc[1] += bf16hi_to_f32(v.x);
         acc[2] += bf16lo_to_f32(v.y); acc[3] += bf16hi_to_f32(v.y);
         acc[4] += bf16lo_to_f32(v.z); acc[5] += bf16hi_to_f32(v.z);
         acc[6] += bf16lo_to_f32(v.w); acc[7] += bf16hi_to_f32(v.w);
       }
+      if (!act) continue;
       *reinterpret_cast<uint4*>(dx + (int64_t)t * cols + c) =
           make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
                      pack_bf16x2(acc[6], acc[7]));

@@ -208,3 +208,26 @@ def layer_step(L: Layer, dy: np.ndarray | None, quantized: bool = True, rounded:
         out["dx"] = rnd(dx_acc)
         out["d_combine"] = d_cw
     return out
+
+
+def combine_rows(y: np.ndarray, slot_row: np.ndarray, weights: np.ndarray, shared_base: int) -> np.ndarray:
+    """The layer output from its permuted expert rows: token t's output is
+    sum_j w[t, j] y[slot_row[t, j]] + y[shared_base + t] (a slot routed
+    nowhere, slot_row -1, contributes nothing), summed in float64 and
+    rounded to bf16 once -- the combine of y_t = sum_j w_tj E_{e_tj}(x_t) +
+    E_shared(x_t) written over the row buffer of the expert outputs."""
+    T, k = slot_row.shape
+    out = np.zeros((T, y.shape[1]))
+    for t in range(T):
+        for j in range(k):
+            r = int(slot_row[t, j])
+            if r >= 0:
+                out[t] += float(weights[t, j]) * y[r]
+        out[t] += y[shared_base + t]
+    return to_bf16(out)
+
+
+def gather_sum_rows(dxp: np.ndarray, slot_row: np.ndarray, shared_base: int) -> np.ndarray:
+    """dx of each token from the permuted rows' input gradients:
+    sum_j dxp[slot_row[t, j]] + dxp[shared_base + t], float64, rounded to bf16."""
+    return combine_rows(dxp, slot_row, np.ones(slot_row.shape), shared_base)

@@ -11,8 +11,8 @@ Bars:
     what remains is the FP32 accumulation of the GPU GEMMs (~1e-6 relative)
     turning into occasional one-ulp bf16 differences (2^-8 relative) and,
     downstream of those, rare one-step E2M1 differences in the quantized
-    SwiGLU output; 2e-3 bounds that with a factor of about 5 at the
-    measured rates (the design doc derives it).
+    SwiGLU output.  The largest error measured on the layer shapes below is
+    3.3e-4 (dx), so the bar is the GEMM's 1e-3.
   * BF16 grouped GEMM: relative Frobenius error <= 1e-3 against float64
     products rounded to bf16.
 """
@@ -28,7 +28,7 @@ from moe_cases import f64, oracle_layer, remap_unused
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
-MOE_RTOL = 2e-3
+MOE_RTOL = 1e-3
 GEMM_RTOL = 1e-3
 
 
@@ -145,7 +145,8 @@ def test_moe_step_matches_oracle(case):
     assert np.array_equal(xh, want_h)
 
     # gate / up products, SwiGLU output (tolerance), its codes (exact where the inputs agree)
-    hg, hu, act = _bf(step.buffer("h_gate")), _bf(step.buffer("h_up")), step.buffer("act")
+    # rows past the last segment are never written: only segment rows are read
+    hg, hu, act = step.buffer("h_gate"), step.buffer("h_up"), step.buffer("act")
     act_bits = act.view(torch.int16).cpu().numpy().view(np.uint16)
     ac = step.buffer("a_codes").cpu().numpy()
     compared = total = 0
@@ -154,8 +155,8 @@ def test_moe_step_matches_oracle(case):
         if st is None:
             continue
         o, n = seg_off[g], seg_len[g]
-        assert _rel(hg[o:o + n], st["h_gate"]) <= MOE_RTOL
-        assert _rel(hu[o:o + n], st["h_up"]) <= MOE_RTOL
+        assert _rel(_bf(hg[o:o + n]), st["h_gate"]) <= MOE_RTOL
+        assert _rel(_bf(hu[o:o + n]), st["h_up"]) <= MOE_RTOL
         a_ref_bits = O.bf16_round(st["a"])
         assert _rel(O.bf16_bits_to_f32(act_bits[o:o + n]).astype(np.float64), st["a"]) <= MOE_RTOL
         same = np.all((act_bits[o:o + n] == a_ref_bits).reshape(n, F // 16, 16), axis=2)
@@ -351,3 +352,53 @@ def test_route_marks_out_of_range_ids():
     s = slot_row.cpu().numpy()
     assert s[1, 0] == -1 and s[2, 1] == -1
     assert s[0, 0] == 0 and s[0, 1] == 128 and s[1, 1] == 129 and s[2, 0] == 256
+
+
+# ------------------------------------------------------------------ combine / gather-sum at any width
+
+def _combine_case(tokens, topk, cols, experts, seed, dyadic):
+    """A row buffer of expert outputs, each token's slot rows (distinct rows,
+    some slots routed nowhere) and the shared rows after the routed ones."""
+    g = torch.Generator().manual_seed(seed)
+    shared_base = tokens * topk + 5
+    rows = shared_base + tokens
+    if dyadic:
+        # small multiples of 1/8 and power-of-two weights: every binary32 sum is exact
+        y = (torch.randint(-64, 65, (rows, cols), generator=g).float() / 8).to(torch.bfloat16)
+        w = 2.0 ** torch.randint(-3, 2, (tokens, topk), generator=g).float()
+    else:
+        y = torch.randn(rows, cols, generator=g).to(torch.bfloat16)
+        w = torch.rand(tokens, topk, generator=g)
+    slot = torch.randperm(shared_base, generator=g)[:tokens * topk].reshape(tokens, topk).to(torch.int32)
+    slot[torch.rand(tokens, topk, generator=g) < 0.1] = -1
+    seg_off = torch.zeros(experts + 2, dtype=torch.int32)
+    seg_off[experts:] = shared_base
+    return y, w, slot, seg_off, shared_base
+
+
+@pytest.mark.parametrize("cols", [8, 40, 264, 2048])
+@pytest.mark.parametrize("dyadic", [True, False])
+def test_combine_and_gather_sum_any_width(cols, dyadic):
+    """cols need only be a multiple of 8; widths whose 16-byte vectors do not
+    fill whole warps exercise the lanes with no vector."""
+    tokens, topk, experts = 37, 6, 4
+    y, w, slot, seg_off, base = _combine_case(tokens, topk, cols, experts, seed=cols, dyadic=dyadic)
+    yd, wd, sd, od = y.to(DEV), w.to(DEV), slot.to(DEV), seg_off.to(DEV)
+    out = torch.empty(tokens, cols, dtype=torch.bfloat16, device=DEV)
+    dx = torch.empty(tokens, cols, dtype=torch.bfloat16, device=DEV)
+    stream = torch.cuda.current_stream().cuda_stream
+    assert Q.lib().nvfp4_moe_combine(yd.data_ptr(), cols, sd.data_ptr(), wd.data_ptr(), tokens, topk, od.data_ptr(),
+                                     experts, out.data_ptr(), stream) == 0
+    assert Q.lib().nvfp4_moe_gather_sum(yd.data_ptr(), cols, sd.data_ptr(), tokens, topk, od.data_ptr(), experts,
+                                        dx.data_ptr(), stream) == 0
+    torch.cuda.synchronize()
+    assert Q.nvfp4_device_error() == (0, 0)
+    y64, s_np = _bf(y), slot.numpy()
+    want_out = OM.combine_rows(y64, s_np, w.double().numpy(), base)
+    want_dx = OM.gather_sum_rows(y64, s_np, base)
+    if dyadic:
+        assert np.array_equal(_bf(out), want_out)
+        assert np.array_equal(_bf(dx), want_dx)
+    else:
+        assert _rel(_bf(out), want_out) <= MOE_RTOL
+        assert _rel(_bf(dx), want_dx) <= MOE_RTOL

@@ -137,3 +137,42 @@ def test_shared_expert_alone_when_routed_weights_vanish():
     out = OM.layer_step(L, None)
     st = OM.expert_forward(L, L.experts, L.x)
     assert np.array_equal(out["y"], st["y"])
+
+
+def test_combine_rows_reproduces_the_layer_output():
+    """combine_rows over the per-expert output rows (laid out as a row
+    buffer, shared expert last) gives the layer_step output bit for bit, and
+    gather_sum_rows of the per-expert dX rows gives the layer's dx."""
+    d = _small(tokens=30, experts=5, topk=3)
+    L = oracle_layer(d)
+    dy = d["dy"].double().numpy()
+    ref = OM.layer_step(L, dy)
+    T, H = L.x.shape
+    E = L.experts
+    rows_y, rows_dx, base = [], [], 0
+    slot_row = -np.ones(L.ids.shape, dtype=np.int64)
+    for g, (t, j) in enumerate(ref["segments"]):
+        per = ref["groups"][g]
+        if len(t) == 0:
+            continue
+        if g < E:
+            slot_row[t, j] = base + np.arange(len(t))
+        else:
+            shared_base = base
+        rows_y.append(per["fwd"]["y"])
+        rows_dx.append(per["bwd"]["dX"])
+        base += len(t)
+    y = np.concatenate(rows_y)
+    dxp = np.concatenate(rows_dx)
+    assert np.array_equal(OM.combine_rows(y, slot_row, L.cw, shared_base), ref["y"])
+    assert np.array_equal(OM.gather_sum_rows(dxp, slot_row, shared_base), ref["dx"])
+
+
+def test_combine_rows_hand_case():
+    y = np.array([[1.0, 2.0], [3.0, -1.0], [0.5, 0.5], [10.0, 20.0], [-4.0, 8.0]])
+    slot_row = np.array([[0, 2], [-1, 1]])
+    w = np.array([[0.25, 2.0], [7.0, 0.5]])
+    out = OM.combine_rows(y, slot_row, w, shared_base=3)
+    # token 0: 0.25*[1,2] + 2*[0.5,0.5] + [10,20]; token 1: 0.5*[3,-1] + [-4,8]
+    assert np.array_equal(out, [[11.25, 21.5], [-2.5, 7.5]])
+    assert np.array_equal(OM.gather_sum_rows(y, slot_row, 3), [[11.5, 22.5], [-1.0, 7.0]])

@@ -59,13 +59,15 @@ def _compare(t, s, T=1.0):
 
 
 def test_noalloc_matches_workspace_entry_point_twice():
-    # two calls in a row on different inputs: the shared scratch keeps the
-    # previous call's contents, which must not leak into the next result
-    t1, s1 = S.logits_pair(48, 131072, seed=11, device=DEV, dtype=torch.bfloat16)
-    _compare(t1, s1)
-    t2, s2 = S.logits_pair(100, 8192, seed=12, device=DEV, dtype=torch.float32, boost=None, teacher_std=4.0,
+    # two calls in a row on different inputs, the larger first: the shared
+    # scratch keeps the first call's 100 row values, so a second call that
+    # read a slot at or beyond its own 48 rows, or left one of its rows
+    # unwritten, would return a different loss or per-row KL
+    t1, s1 = S.logits_pair(100, 8192, seed=12, device=DEV, dtype=torch.float32, boost=None, teacher_std=4.0,
                            noise_std=0.5)
-    _compare(t2, s2, T=1.5)
+    _compare(t1, s1, T=1.5)
+    t2, s2 = S.logits_pair(48, 131072, seed=11, device=DEV, dtype=torch.bfloat16)
+    _compare(t2, s2)
 
 
 def test_noalloc_rejects_rows_beyond_the_maximum():
