@@ -60,12 +60,11 @@ METRIC = "NVFP4 quant GB/s & W4A4 GEMM TFLOPS (% of peak); QAD KL loss tokens/s"
 BYTES_PER_ELEM = 2.5625
 WORKLOAD = ("weight quantization sweep: 128 MoE experts 2048x1024 + lm_head 131072x2048 bf16, "
             "NVFP4 dynamic then frozen (FROZEN_ALL) quantize to packed codes + E4M3 block scales")
-# ncu DRAM bytes (read + write) per launch of the dominant kernel, from the
-# capture summarised in profiles/; valid only while quantize.cu is unchanged.
-# DRAM bytes of one launch of the dominant kernel, from the ncu capture in
-# profiles/group_encode_frozen_48experts.md (48 experts, 100.7M elements: read 207.64 MB +
-# write 34.80 MB = 2.407 B per element), scaled by elements to the whole sweep
-# (536,870,912 elements); valid only while quantize.cu is the source that was captured.
+# DRAM bytes of one launch of the dominant kernel, from an ncu capture of the
+# same kernel on 48 expert weights (100.7M elements: read 207.64 MB + write
+# 34.80 MB = 2.407 B per element), scaled by elements to the whole sweep
+# (536,870,912 elements); reported only while quantize.cu is the source that
+# was captured (its SHA-256 below).
 TRAFFIC = {"kernel": "group_encode_kernel<bf16,codes> (FROZEN_ALL, whole sweep)",
            "bytes": round((207.644416e6 + 34.831872e6) / (48 * 2048 * 1024) * 536870912),
            "source_sha256": "276e49728b85e4d27d225d194f3922cd6738efe7b75cdb26b0abbf91d3e99a31"}
@@ -278,6 +277,12 @@ def run_ours(args, world, rank, local):
         # power) would lower the clocks of whatever is timed right after it
         secondary["fp4_peak_probe"] = bench_fp4_peak(Q, dev, stream)
         apply_fp4_peak(secondary["gemm"], secondary["fp4_peak_probe"])
+        peak = (secondary["fp4_peak_probe"] or {}).get("burst_tflops")
+        gf = secondary["moe_step"]["phases"]["w4a4_gemms_forward"]
+        if peak:
+            gf["peak"] = peak
+            gf["frac"] = round(gf["tflops"] / peak, 4)
+            gf["peak_source"] = "own tcgen05 FP4 MMA probe, burst (fp4_peak_probe)"
     clocks = sampler.stop()
 
     cpu = None
@@ -473,21 +478,25 @@ def bench_gemm(Q, dev, stream, P, K, probe=None):
                 Q.nvfp4_quantize(x, Q.DYNAMIC, tensor_scale=xts, block_scales=xsf, layout=Q.SCALES_MMA, codes=xc,
                                  workspace=qws)
                 Q.nvfp4_gemm_w4a4(xc, xsf, xts, wc, wsf, wts, out=c)
-            tq, tg = [], []
-            for _ in range(K):
-                flush_l2(flush)
-                e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-                e0.record(stream)
-                Q.nvfp4_quantize(x, Q.DYNAMIC, tensor_scale=xts, block_scales=xsf, layout=Q.SCALES_MMA, codes=xc,
-                                 workspace=qws)
-                e1.record(stream)
-                Q.nvfp4_gemm_w4a4(xc, xsf, xts, wc, wsf, wts, out=c)
-                e2.record(stream)
-                tq.append((e0, e1))
-                tg.append((e1, e2))
             stream.synchronize()
-            q_ms = statistics.mean(a.elapsed_time(b) for a, b in tq)
-            g_ms = statistics.mean(a.elapsed_time(b) for a, b in tg)
+            # K steps in one CUDA graph (no host launch time inside the timed
+            # intervals): L2 flush, X quantize, GEMM, with events between them
+            evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(K)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for k in range(K):
+                    flush_l2(flush)
+                    evs[k][0].record(stream)
+                    Q.nvfp4_quantize(x, Q.DYNAMIC, tensor_scale=xts, block_scales=xsf, layout=Q.SCALES_MMA,
+                                     codes=xc, workspace=qws)
+                    evs[k][1].record(stream)
+                    Q.nvfp4_gemm_w4a4(xc, xsf, xts, wc, wsf, wts, out=c)
+                    evs[k][2].record(stream)
+            g.replay()
+            stream.synchronize()
+            q_ms = statistics.mean(evs[k][0].elapsed_time(evs[k][1]) for k in range(K))
+            g_ms = statistics.mean(evs[k][1].elapsed_time(evs[k][2]) for k in range(K))
+            del g
             flops = 2.0 * M * 4096 * 4096
             tflops = flops / (g_ms * 1e-3) / 1e12
             gemm_bytes = 4096 * 4096 * 0.5625 + M * 4096 * 0.5625 + M * 4096 * 2
@@ -657,22 +666,101 @@ def bench_moe(Q, dev, stream, P, K):
         e1.record(stream)
         stream.synchronize()
         st, word = Q.nvfp4_device_error()
-    del g
+        del g
+        phases = moe_phases(Q, stream, step, w, tokens, hidden, ffn, experts, K)
     ms = e0.elapsed_time(e1) / K
     fwd = statistics.mean(evs[k][0].elapsed_time(evs[k][1]) for k in range(K))
     bwd = statistics.mean(evs[k][1].elapsed_time(evs[k][2]) for k in range(K))
     rows = tokens * topk + tokens
     f_flops = 6.0 * rows * hidden * ffn         # gate, up, down (W4A4)
     b_flops = 12.0 * rows * hidden * ffn        # dA, dX (2F), dW x3 (BF16)
+    wp = phases["weight_pass"]
+    gf = phases["w4a4_gemms"]
+    bf = {"ms": round(bwd, 4), "tflops": round(b_flops / (bwd * 1e-3) / 1e12, 1)}
+    bf["frac"] = round(bf["tflops"] / P["bf16_tflops_sustained"], 4)
+    bf["peak"] = P["bf16_tflops_sustained"]
+    bf["peak_source"] = "MEASURED_PEAKS bf16_tflops_sustained (the backward runs inside a seconds-long step)"
+    bf["what"] = "whole backward: 5 BF16 grouped GEMMs (dA, dX, dW x3) and the elementwise steps, 1.16e12 flop"
+    fp4_peak = (P.get("fp4_probe") or {}).get("burst_tflops") or 4.0 * P["bf16_tflops"]
+    gf["peak"] = fp4_peak
+    gf["frac"] = round(gf["tflops"] / fp4_peak, 4)
+    gf["peak_source"] = ("own tcgen05 FP4 MMA probe, burst" if (P.get("fp4_probe") or {}).get("burst_tflops")
+                         else "4 x MEASURED_PEAKS bf16_tflops")
     out = {"tokens_per_s": round(tokens / (ms * 1e-3), 1), "ms_per_step": round(ms, 4),
            "forward_ms": round(fwd, 4), "backward_ms": round(bwd, 4),
            "forward_fp4_tflops": round(f_flops / (fwd * 1e-3) / 1e12, 1),
            "backward_bf16_tflops": round(b_flops / (bwd * 1e-3) / 1e12, 1),
+           # dominant kernel of the step: the per-step weight pass (group_encode_kernel<bf16, Both>,
+           # 3 launches over the 387 expert weights: master weight in, codes + bf16 W^ out)
+           "roofline": {"bound": "hbm", "achieved": wp["gbs"], "peak": P["hbm_gbs"], "unit": "GB/s",
+                        "frac": round(wp["gbs"] / P["hbm_gbs"], 4),
+                        "kernel": "group_encode_kernel<bf16,Both> (FROZEN_ALL weight pass, 3 launches)",
+                        "algorithmic_bytes_per_step": wp["bytes"], "avg_step_ms": wp["ms"],
+                        "share_of_step": round(wp["ms"] / ms, 4), "peak_source": "measured (MEASURED_PEAKS hbm_gbs)"},
+           "phases": {"weight_pass": wp, "w4a4_gemms_forward": gf, "bf16_backward": bf},
            "gpu_launches_per_step": int(launches // K), "device_error": [int(st), int(word)],
            "config": MOE_CONFIG + "; inputs larger than L2 (weights 3.2 GB), no flush"}
     del d, w, step, x, y, dx, dwg, dwu, dwd, dcw
     torch.cuda.empty_cache()
     return out
+
+
+def _graph_ms(stream, fn, K):
+    """Mean device time of fn() over K calls captured in one CUDA graph."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(K):
+            fn()
+    g.replay()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    stream.synchronize()
+    del g
+    return e0.elapsed_time(e1) / K
+
+
+def moe_phases(Q, stream, step, w, tokens, hidden, ffn, experts, K):
+    """Two phases of the layer step timed on their own, with the step's own
+    buffers (after a forward): the weight pass (FROZEN_ALL quantize of the 3 G
+    master weights to codes + bf16 W^, exactly the step's first call) and the
+    three grouped W4A4 GEMMs of the forward."""
+    G, H, F = experts + 1, hidden, ffn
+    wg, wu, wd = w["w_gate"], w["w_up"], w["w_down"]
+    cg, cu, cd = step.buffer("wg_codes"), step.buffer("wu_codes"), step.buffer("wd_codes")
+    hgu, hd = step.buffer("wgu_hat"), step.buffer("wd_hat")
+    xs = ([wg[g * F:(g + 1) * F] for g in range(G)] + [wu[g * F:(g + 1) * F] for g in range(G)] +
+          [wd[g * H:(g + 1) * H] for g in range(G)])
+    ts = ([w["gate_ts"][g:g + 1] for g in range(G)] + [w["up_ts"][g:g + 1] for g in range(G)] +
+          [w["down_ts"][g:g + 1] for g in range(G)])
+    sbs = ([w["gate_sb"][g * F:(g + 1) * F] for g in range(G)] + [w["up_sb"][g * F:(g + 1) * F] for g in range(G)] +
+           [w["down_sb"][g * H:(g + 1) * H] for g in range(G)])
+    codes = ([cg[g * F:(g + 1) * F] for g in range(G)] + [cu[g * F:(g + 1) * F] for g in range(G)] +
+             [cd[g * H:(g + 1) * H] for g in range(G)])
+    ys = ([hgu[2 * g * F:2 * g * F + F] for g in range(G)] + [hgu[2 * g * F + F:2 * (g + 1) * F] for g in range(G)] +
+          [hd[g * H:(g + 1) * H] for g in range(G)])
+    wp_ms = _graph_ms(stream, lambda: Q.nvfp4_quantize_fake_quant_grouped(xs, Q.FROZEN_ALL, ts, sbs, codes=codes,
+                                                                           ys=ys), K)
+    n = sum(x.numel() for x in xs)
+    wp_bytes = n * (2.0 + 0.0625 + 0.5 + 2.0)  # bf16 in, block scales in, codes + bf16 W^ out
+    seg_off, seg_len = step.buffer("seg_off"), step.buffer("seg_len")
+    xc, xsf, ac, asf = step.buffer("x_codes"), step.buffer("x_scales"), step.buffer("a_codes"), step.buffer("a_scales")
+    hg, hu, yr = step.buffer("h_gate"), step.buffer("h_up"), step.buffer("y_rows")
+
+    def gemms():
+        Q.nvfp4_gemm_w4a4_grouped(xc, xsf, w["x_ts"], seg_off, seg_len, cg, w["gate_sb_mma"], w["gate_ts"], F, out=hg)
+        Q.nvfp4_gemm_w4a4_grouped(xc, xsf, w["x_ts"], seg_off, seg_len, cu, w["up_sb_mma"], w["up_ts"], F, out=hu)
+        Q.nvfp4_gemm_w4a4_grouped(ac, asf, w["a_ts"], seg_off, seg_len, cd, w["down_sb_mma"], w["down_ts"], H, out=yr)
+
+    g_ms = _graph_ms(stream, gemms, K)
+    rows = tokens * 6 + tokens
+    g_flops = 6.0 * rows * H * F
+    return {"weight_pass": {"ms": round(wp_ms, 4), "bytes": int(wp_bytes), "gbs": round(wp_bytes / (wp_ms * 1e-3) / 1e9, 1),
+                            "what": "FROZEN_ALL quantize of the 3 x 129 master weights to codes + bf16 W^ (811.6M elements, 4.5625 B each)"},
+            "w4a4_gemms": {"ms": round(g_ms, 4), "tflops": round(g_flops / (g_ms * 1e-3) / 1e12, 1),
+                           "what": "grouped W4A4 gate, up and down over the 28672 routed + shared rows (useful flop, padding excluded)"}}
 
 
 def bench_kl_topk(Q, dev, stream, P, K, k=4096):
@@ -856,7 +944,18 @@ def main():
         return
     if args.warmup < 3:
         args.warmup = 3
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: start the ranks under torch.distributed.run (NCCL)
+        # and return its status; the bound on the whole job is well above the
+        # process group's own timeout
+        port = os.environ.get("MASTER_PORT", "29517")
+        cmd = ["timeout", "-k", "60", "1800", sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+               f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1", f"--master-port={port}",
+               os.path.abspath(__file__), *sys.argv[1:]]
+        sys.exit(subprocess.call(cmd))
     world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != args.gpus and args.gpus > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":
         run_reference(args, world, rank)

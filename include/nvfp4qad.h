@@ -127,6 +127,24 @@ uint64_t nvfp4_launch_count(void);
  * words, NVFP4_ERR_CUDA if the synchronization failed. */
 nvfp4_status nvfp4_device_error(void* stream, int32_t* code_out);
 
+/* Host-side fault injection (failure-detection tests; the pages' QAD runs are
+ * long multi-job trainings, Qwen3.6-35B-A3B W4A4 tutorial, "成本").  After
+ * nvfp4_fault_inject(n) with n >= 1, the n-th outermost call of an exported
+ * operation from now returns NVFP4_ERR_CUDA before it validates its arguments
+ * or launches anything; one failure per arming; n = 0 disarms.  Setting
+ * NVFP4QAD_FAIL_AT=n in the environment arms it when the library loads.
+ * Operations called by another exported operation (the MoE step's parts) are
+ * not counted on their own.  Every exported operation also opens an NVTX
+ * range named after itself for the duration of the call. */
+void nvfp4_fault_inject(int64_t nth);
+
+/* Self-test of the bounded device waits: one thread waits on an mbarrier that
+ * nothing arrives at for limit_cycles SM clock cycles (1 .. 2^32), then sets
+ * the device error word to 1, as every expired wait of this library does; the
+ * next nvfp4_device_error returns NVFP4_ERR_TIMEOUT and the context stays
+ * usable.  NVFP4_ERR_ARG for a limit outside the range. */
+nvfp4_status nvfp4_selftest_timeout(int64_t limit_cycles, void* stream);
+
 /* ------------------------------------------------------------------------
  * Quantize (steps: tensor amax [DYNAMIC] -> block scale -> E2M1 encode and
  * pack), NVFP4 definition of the Nemotron-3-Nano article, scale modes of the
@@ -589,6 +607,37 @@ nvfp4_status qad_moe_forward(const qad_moe_shape* shape, const qad_moe_weights* 
 nvfp4_status qad_moe_backward(const qad_moe_shape* shape, const qad_moe_weights* w, const void* dy, void* dx,
                               void* dw_gate, void* dw_up, void* dw_down, float* d_combine, void* workspace,
                               size_t workspace_bytes, void* stream);
+
+/* Expert-parallel form: the expert FFNs of this rank's experts on the rows it
+ * received from every rank (expert parallelism with EP 4 / 8: Nemotron 3.5
+ * Lightning NVFP4 article, training set-up; Qwen3.6-35B-A3B W4A4 tutorial,
+ * "3. QAD").  Each received row is one (token, slot) assignment, so
+ *   shape->tokens  rows received (>= 1), shape->topk must be 1,
+ *   shape->experts this rank's experts E_r; there is no shared expert (it
+ *                  runs on each token's home rank: call this with experts = 1
+ *                  and every id 0 for it);
+ *   expert_ids     [rows] the expert of each row among this rank's experts;
+ *   w              the E_r experts' weights and scales as in qad_moe_forward
+ *                  (no shared group: gate/up/down, the tensor scales and
+ *                  x_ts / a_ts have E_r entries);
+ *   y              [rows x hidden] bf16: y[r] = E_{id[r]}(x[r]), not combined
+ *                  (the home rank weights and sums the returned rows).
+ * Workspace: qad_moe_workspace_size(shape) bytes, as for qad_moe_forward.
+ * The results of a row equal those qad_moe_forward computes for the same
+ * (token, expert) pair, bit for bit (rows are independent in every step). */
+nvfp4_status qad_moe_expert_forward(const qad_moe_shape* shape, const qad_moe_weights* w, const void* x,
+                                    const int32_t* expert_ids, void* y, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
+/* Backward of qad_moe_expert_forward (after it, same workspace): dy [rows x
+ * hidden] is each received row's output gradient, already multiplied by its
+ * combine weight on the home rank; dx [rows x hidden] the rows' input
+ * gradients; dw_gate / dw_up [E_r F x H], dw_down [E_r H x F] the weight
+ * gradients of this rank's experts, reduced over the received rows in row
+ * order (sources in rank order keep the single-process order). */
+nvfp4_status qad_moe_expert_backward(const qad_moe_shape* shape, const qad_moe_weights* w, const void* dy, void* dx,
+                                     void* dw_gate, void* dw_up, void* dw_down, void* workspace,
+                                     size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * KL distillation loss, forward and backward in one pass (Nemotron 3.5

@@ -30,6 +30,8 @@ from .binding import (  # noqa: F401
     mma_scales_bytes,
     nvfp4_dequantize,
     nvfp4_device_error,
+    nvfp4_fault_inject,
+    nvfp4_selftest_timeout,
     nvfp4_fake_quant,
     nvfp4_fake_quant_grouped,
     nvfp4_launch_count,
@@ -43,6 +45,7 @@ from .binding import (  # noqa: F401
     nvfp4_scales_to_mma,
     nvfp4_quantize_fake_quant_grouped,
     MoeLayerStep,
+    MoeExpertStep,
     MOE_BUFFERS,
     nvfp4_quantize,
     nvfp4_selftest_division,

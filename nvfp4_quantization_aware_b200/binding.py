@@ -103,6 +103,10 @@ def lib() -> ctypes.CDLL:
     L.nvfp4_mma_scales_bytes.restype = sz
     L.nvfp4_device_error.argtypes = [p, ctypes.POINTER(ctypes.c_int32)]
     L.nvfp4_device_error.restype = i32
+    L.nvfp4_fault_inject.argtypes = [i64]
+    L.nvfp4_fault_inject.restype = None
+    L.nvfp4_selftest_timeout.argtypes = [i64, p]
+    L.nvfp4_selftest_timeout.restype = i32
     L.nvfp4_quantize_workspace_size.argtypes = [i64, i64, i32]
     L.nvfp4_quantize_workspace_size.restype = sz
     L.nvfp4_fake_quant_workspace_size.argtypes = [i64, i64, i32]
@@ -184,6 +188,10 @@ def lib() -> ctypes.CDLL:
     L.qad_moe_forward.restype = i32
     L.qad_moe_backward.argtypes = [shp, wts, p, p, p, p, p, p, p, sz, p]
     L.qad_moe_backward.restype = i32
+    L.qad_moe_expert_forward.argtypes = [shp, wts, p, p, p, p, sz, p]
+    L.qad_moe_expert_forward.restype = i32
+    L.qad_moe_expert_backward.argtypes = [shp, wts, p, p, p, p, p, p, sz, p]
+    L.qad_moe_expert_backward.restype = i32
     _lib = L
     return L
 
@@ -231,6 +239,19 @@ def mma_scales_bytes(rows: int, cols: int) -> int:
 def nvfp4_launch_count() -> int:
     """Kernels launched by the library so far in this process."""
     return int(lib().nvfp4_launch_count())
+
+
+def nvfp4_fault_inject(nth: int) -> None:
+    """Arm the library's host-side fault injection: the nth outermost call of
+    an exported operation from now fails with NVFP4_ERR_CUDA before launching
+    (0 disarms)."""
+    lib().nvfp4_fault_inject(int(nth))
+
+
+def nvfp4_selftest_timeout(limit_cycles: int, device="cuda") -> None:
+    """Launch the bounded-wait self-test kernel (a wait that nothing ends,
+    expiring after limit_cycles); nvfp4_device_error() then reports it."""
+    _check(lib().nvfp4_selftest_timeout(int(limit_cycles), _stream(torch.device(device))), "nvfp4_selftest_timeout")
 
 
 def nvfp4_device_error() -> tuple[int, int]:
@@ -638,6 +659,66 @@ class MoeLayerStep:
                                     _ptr(self.workspace), self.ws_bytes, _stream(dev))
         _check(st, "qad_moe_backward")
         return dx, dw_gate, dw_up, dw_down, d_combine
+
+
+class MoeExpertStep:
+    """qad_moe_expert_forward / qad_moe_expert_backward: the expert FFNs of
+    `experts` experts (one expert-parallel rank's, or the shared expert alone
+    with experts = 1) on a set of rows, each row routed to one of them.  The
+    number of rows may change from call to call; the workspace grows when it
+    must."""
+
+    def __init__(self, hidden: int, ffn: int, experts: int, weights: dict, device="cuda"):
+        self.hidden, self.ffn, self.experts = hidden, ffn, experts
+        self._keep = dict(weights)
+        self.weights = MoeWeights(**{n: weights[n].data_ptr() for n, _ in MoeWeights._fields_})
+        self.device = torch.device(device)
+        self.workspace = torch.empty(0, dtype=torch.uint8, device=self.device)
+        self.shape = None
+
+    def _shape(self, rows: int) -> MoeShape:
+        shape = MoeShape(rows, self.hidden, self.ffn, self.experts, 1, 0)
+        need = int(lib().qad_moe_workspace_size(ctypes.byref(shape)))
+        if need == 0:
+            raise NVFP4Error(2, "qad_moe_workspace_size")
+        if self.workspace.numel() < need:
+            self.workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+        self.shape = shape
+        return shape
+
+    def forward(self, x: torch.Tensor, expert_ids: torch.Tensor, y: torch.Tensor | None = None) -> torch.Tensor:
+        """y[r] = E_{expert_ids[r]}(x[r]) for the rows x [n, hidden] (bf16)."""
+        if y is None:
+            y = torch.empty_like(x)
+        if x.shape[0] == 0:
+            self.shape = None
+            return y
+        shape = self._shape(x.shape[0])
+        st = lib().qad_moe_expert_forward(ctypes.byref(shape), ctypes.byref(self.weights), _ptr(x), _ptr(expert_ids),
+                                          _ptr(y), _ptr(self.workspace), self.workspace.numel(), _stream(self.device))
+        _check(st, "qad_moe_expert_forward")
+        return y
+
+    def backward(self, dy: torch.Tensor, dx=None, dw_gate=None, dw_up=None, dw_down=None):
+        """After forward on the same rows: dy [n, hidden] the rows' output
+        gradients (combine weight applied).  Returns (dx, dw_gate, dw_up, dw_down)."""
+        E, H, F = self.experts, self.hidden, self.ffn
+        dev = self.device
+        dx = torch.empty_like(dy) if dx is None else dx
+        dw_gate = torch.empty(E * F, H, dtype=torch.bfloat16, device=dev) if dw_gate is None else dw_gate
+        dw_up = torch.empty(E * F, H, dtype=torch.bfloat16, device=dev) if dw_up is None else dw_up
+        dw_down = torch.empty(E * H, F, dtype=torch.bfloat16, device=dev) if dw_down is None else dw_down
+        if dy.shape[0] == 0:
+            for t in (dw_gate, dw_up, dw_down):
+                t.zero_()
+            return dx, dw_gate, dw_up, dw_down
+        if self.shape is None or self.shape.tokens != dy.shape[0]:
+            raise ValueError("backward needs the forward of the same rows first")
+        st = lib().qad_moe_expert_backward(ctypes.byref(self.shape), ctypes.byref(self.weights), _ptr(dy), _ptr(dx),
+                                           _ptr(dw_gate), _ptr(dw_up), _ptr(dw_down), _ptr(self.workspace),
+                                           self.workspace.numel(), _stream(dev))
+        _check(st, "qad_moe_expert_backward")
+        return dx, dw_gate, dw_up, dw_down
 
 
 def qad_kl_topk_fwd_bwd(teacher: torch.Tensor, student: torch.Tensor, k: int, temperature: float = 1.0,

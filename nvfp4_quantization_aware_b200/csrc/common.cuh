@@ -23,8 +23,28 @@ constexpr int kErrExpertId = 3;       // an expert id outside [0, experts)
 
 NVFP4_DEV void report_error(int code) { atomicCAS(&g_device_error, 0, code); }
 
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream serialization attribute may start while the previous kernel of the
+// stream is finishing; it must execute this before it reads or writes any
+// global memory that kernel may touch (a no-op for a normal launch).
+NVFP4_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Host-side count of kernel launches (nvfp4_launch_count).
 void count_launches(int n);
+
+// Entry of an exported operation: an NVTX range named after it for the
+// duration of the call (nested calls nest), and the host-side fault-injection
+// point -- when armed (nvfp4_fault_inject, or NVFP4QAD_FAIL_AT=n in the
+// environment at load time) the n-th outermost entry returns NVFP4_ERR_CUDA
+// before it validates or launches anything.
+struct EntryScope {
+  explicit EntryScope(const char* name);
+  ~EntryScope();
+  bool inject;  // this entry is the armed one
+};
+#define NVFP4_ENTRY(name)                         \
+  ::nvfp4::EntryScope nvfp4_entry_scope_(name);   \
+  if (nvfp4_entry_scope_.inject) return NVFP4_ERR_CUDA
 
 // ---------------------------------------------------------------- loads/stores
 

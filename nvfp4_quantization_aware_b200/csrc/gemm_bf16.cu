@@ -375,13 +375,9 @@ static bool tmap_c(CUtensorMap* m, void* base, int64_t n, int64_t rows, int64_t 
 template <bool A_MN, bool B_MN>
 static nvfp4_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const Params& p,
                            cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(gemm_bf16_kernel<A_MN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    attr = true;
-  }
+  // the attribute is per device: set it on every call (cheap)
+  if (cudaFuncSetAttribute(gemm_bf16_kernel<A_MN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   gemm_bf16_kernel<A_MN, B_MN><<<sms, THREADS, SMEM_BYTES, s>>>(ta, tb, tc, p);
@@ -399,6 +395,7 @@ extern "C" nvfp4_status nvfp4_gemm_bf16_grouped(int mode, int groups, const void
                                                 int64_t b_rows, int64_t b_cols, int64_t ldb, const int32_t* seg_off,
                                                 const int32_t* seg_len, int64_t M, int64_t N, int64_t K, void* c,
                                                 int64_t ldc, void* stream) {
+  NVFP4_ENTRY("nvfp4_gemm_bf16_grouped");
   using namespace bf16gemm;
   if (mode != 0 && mode != 1) return NVFP4_ERR_ARG;
   if ((a_mn_major != 0 && a_mn_major != 1) || (b_mn_major != 0 && b_mn_major != 1)) return NVFP4_ERR_ARG;

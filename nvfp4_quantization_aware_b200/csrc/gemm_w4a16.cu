@@ -363,6 +363,7 @@ using namespace nvfp4;
 extern "C" nvfp4_status nvfp4_gemm_w4a16(const void* a, int64_t lda, const uint8_t* b_codes, const uint8_t* b_scales,
                                          const float* b_tensor_scale, int64_t M, int64_t N, int64_t K, void* c,
                                          int64_t ldc, void* stream) {
+  NVFP4_ENTRY("nvfp4_gemm_w4a16");
   using namespace w4a16;
   if (M < 1 || N < 1 || K < 64 || K % 64 != 0 || lda < K || ldc < N) return NVFP4_ERR_SHAPE;
   if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return NVFP4_ERR_SHAPE;
@@ -404,12 +405,9 @@ extern "C" nvfp4_status nvfp4_gemm_w4a16(const void* a, int64_t lda, const uint8
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
   }
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(gemm_w4a16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    attr = true;
-  }
+  // the attribute is per device: set it on every call (cheap)
+  if (cudaFuncSetAttribute(gemm_w4a16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int tiles = (int)(((M + BM - 1) / BM) * ((N + BN - 1) / BN));

@@ -39,7 +39,11 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cooperative_groups.h>
+
 #include "ptx.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace nvfp4 {
 
@@ -95,6 +99,7 @@ struct GemmParams {
   int b_rowtiles;        // ceil(N / 128): 128-row scale tiles present for B
   int c_vec16;           // C base 16-byte aligned and ldc % 8 == 0: 16-byte stores
   int c_vec32;           // C base 32-byte aligned and ldc % 16 == 0: 32-byte stores
+  int c_vec8;            // C base 8-byte aligned and ldc % 4 == 0: 8-byte stores
   // Grouped problems (groups > 0): group g owns A rows [a_off[g], a_off[g] + a_rows[g]) with
   // a_off[g] a multiple of 128 (device arrays; a_off[groups] is the padded row total), B rows
   // [g * N, (g + 1) * N), tensor scales a_ts[g] and b_ts[g].
@@ -241,14 +246,6 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
   const int lane = threadIdx.x & 31;
   const int num_kt = (p.kchunks + C::KB_PER_STAGE - 1) / C::KB_PER_STAGE;
   const int num_n = (p.N + C::BN - 1) / C::BN;
-  for (int i = threadIdx.x; i < p.groups; i += blockDim.x) {
-    s_off[i] = __ldg(p.a_off + i);
-    s_rows[i] = __ldg(p.a_rows + i);
-  }
-  if (threadIdx.x == 0 && p.groups > 0) s_off[p.groups] = __ldg(p.a_off + p.groups);
-  __syncthreads();
-  const int m_total = p.groups > 0 ? s_off[p.groups] : p.M;
-  const int num_tiles = num_n * ((m_total + C::BM - 1) / C::BM);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -267,10 +264,20 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
     tmem_alloc(tmem_base_slot, C::TM_COLS);
     tmem_relinquish();
   }
+  // the set-up above overlaps the previous kernel of the stream under a
+  // programmatic dependent launch; global memory only after this point
+  griddep_wait();
+  for (int i = threadIdx.x; i < p.groups; i += blockDim.x) {
+    s_off[i] = __ldg(p.a_off + i);
+    s_rows[i] = __ldg(p.a_rows + i);
+  }
+  if (threadIdx.x == 0 && p.groups > 0) s_off[p.groups] = __ldg(p.a_off + p.groups);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_base_slot;
+  const int m_total = p.groups > 0 ? s_off[p.groups] : p.M;
+  const int num_tiles = num_n * ((m_total + C::BM - 1) / C::BM);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -646,6 +653,246 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
   }
 }
 
+// ------------------------------------------------------------------ split-K kernel (few output tiles)
+//
+// When the output has few tiles -- a decode-sized batch: M of one or two
+// 128-row tiles against a large weight -- the persistent kernel leaves most
+// SMs idle and each busy SM walks the whole K serially (the per-call FP4
+// overhead the Qwen3.6-35B-A3B W4A4 tutorial measures at batch 1, section
+// "吞吐量").  Here each 128 x 128 output tile is computed by a cluster of S
+// CTAs that split K into S contiguous ranges: every CTA streams its range of
+// A and B through a ring with the same producer / MMA / scale-writer roles
+// as the persistent kernel, accumulating an FP32 partial tile in tensor
+// memory.  CTA r reduces rows [r 128/S, (r+1) 128/S) of the tile: every CTA
+// stores its partial of those rows from tensor memory straight into slot
+// `rank` of CTA r's receive buffer (distributed shared memory stores, which
+// need no reply), and after one cluster barrier CTA r adds the S partials in
+// rank order 0..S-1 from its own shared memory, scales by s_gA s_gB and
+// stores bf16.  The sum order is fixed, so the result is deterministic; no
+// workspace and no second launch.
+namespace splitk {
+constexpr int BM = 128, BN = 128;
+constexpr int BK = 256;                  // FP4 elements per stage (128 bytes per row)
+constexpr int KB = BK / 64;              // MMAs (K = 64) per stage
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK / 2;     // 16 KiB
+constexpr int B_BYTES = BN * BK / 2;     // 16 KiB
+constexpr int SF_BYTES = 512 * KB;       // one 128-row scale tile per operand
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + 2 * SF_BYTES;
+constexpr int PART_STRIDE = BN + 4;      // floats per partial-tile row in shared memory
+constexpr int PART_BYTES = BM * PART_STRIDE * 4;  // receive buffer: S partials of this CTA's BM / S rows
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + PART_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int TM_ACC = 0;                        // 128 lanes x 128 FP32 columns
+constexpr int TM_SFA = BN;                       // STAGES x 4 KB columns
+constexpr int TM_SFB = BN + STAGES * 4 * KB;     // STAGES x 4 KB columns
+constexpr int TM_COLS = 256;
+constexpr int EPI_WARPS = 4;                     // one per TMEM subpartition, all 128 columns
+constexpr int SF_WARPS = 4;
+constexpr int THREADS = 64 + 32 * (EPI_WARPS + SF_WARPS);
+constexpr int MAX_SPLIT = 8;                     // portable cluster size
+constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+static_assert(TM_SFB + STAGES * 4 * KB <= TM_COLS, "tensor memory");
+}  // namespace splitk
+
+__global__ void __launch_bounds__(splitk::THREADS, 1)
+    gemm_w4a4_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                            GemmParams p) {
+  using namespace splitk;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + STAGES * A_BYTES;
+  uint8_t* sSFA = sB + STAGES * B_BYTES;
+  uint8_t* sSFB = sSFA + STAGES * SF_BYTES;
+  float* recv = reinterpret_cast<float*>(sSFB + STAGES * SF_BYTES);  // [S][BM / S][PART_STRIDE]
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(recv) + PART_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* sf_full = empty + STAGES;
+  uint64_t* acc_full = sf_full + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int split = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int tile = blockIdx.x / split;
+  const int num_n = (p.N + BN - 1) / BN;
+  const int mt = tile / num_n;
+  const int m0 = mt * BM, n0 = (tile - mt * num_n) * BN;
+  const int num_kt = (p.kchunks + KB - 1) / KB;
+  // contiguous K-stage range of this CTA; split <= num_kt, so none is empty
+  const int kt0 = (int)((int64_t)num_kt * rank / split);
+  const int kt1 = (int)((int64_t)num_kt * (rank + 1) / split);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&sf_full[s], SF_WARPS);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TM_COLS);
+    tmem_relinquish();
+  }
+  griddep_wait();  // global memory only after this point (programmatic dependent launch)
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      for (int kt = kt0; kt < kt1; ++kt) {
+        const int it = kt - kt0, s = it % STAGES;
+        const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+        if (!mbar_wait_bounded(&empty[s], ph ^ 1u)) { *abort_flag = 1; break; }
+        if (*abort_flag) break;
+        int nkc = p.kchunks - kt * KB;
+        if (nkc > KB) nkc = KB;
+        mbar_expect_tx(&full[s], (uint32_t)(A_BYTES + B_BYTES) + 2u * (uint32_t)nkc * 512u);
+        tma_load_2d(sA + s * A_BYTES, &tmA, kt * (BK / 2), m0, &full[s]);
+        tma_load_2d(sB + s * B_BYTES, &tmB, kt * (BK / 2), n0, &full[s]);
+        const int64_t kc0 = (int64_t)kt * KB;
+        bulk_g2s(sSFA + s * SF_BYTES, p.a_sf + ((int64_t)(m0 / 128) * p.kchunks + kc0) * 512, (uint32_t)nkc * 512u,
+                 &full[s]);
+        bulk_g2s(sSFB + s * SF_BYTES, p.b_sf + ((int64_t)(n0 / 128) * p.kchunks + kc0) * 512, (uint32_t)nkc * 512u,
+                 &full[s]);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      for (int kt = kt0; kt < kt1 && ok; ++kt) {
+        const int it = kt - kt0, s = it % STAGES;
+        const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+        if (!mbar_wait_bounded(&full[s], ph) || !mbar_wait_bounded(&sf_full[s], ph) || *abort_flag) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        int nkc = p.kchunks - kt * KB;
+        if (nkc > KB) nkc = KB;
+        const uint32_t a_base = smem_u32(sA + s * A_BYTES);
+        const uint32_t b_base = smem_u32(sB + s * B_BYTES);
+        for (int kb = 0; kb < nkc; ++kb)
+          mma_fp4_block16(tmem + TM_ACC, smem_desc(a_base + kb * 32, 16, 1024, 2), smem_desc(b_base + kb * 32, 16, 1024, 2),
+                          IDESC, tmem + TM_SFA + s * 4 * KB + kb * 4, tmem + TM_SFB + s * 4 * KB + kb * 4,
+                          (it > 0 || kb > 0) ? 1u : 0u);
+        tc_commit(&empty[s]);
+      }
+      if (ok) tc_commit(acc_full);
+      else *abort_flag = 1;
+    }
+  } else if (warp >= 2 + EPI_WARPS) {
+    // ------------------------------------------------------------ scale writers
+    // the persistent kernel's image: per 512-byte scale tile, 4 TMEM columns in
+    // which lane L holds bytes [16 (L % 32), +16) on every subpartition
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    for (int kt = kt0; kt < kt1; ++kt) {
+      const int it = kt - kt0, s = it % STAGES;
+      const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[s], ph))) {  // warp-uniform exit
+        *abort_flag = 1;
+        break;
+      }
+      int nkc = p.kchunks - kt * KB;
+      if (nkc > KB) nkc = KB;
+      const uint8_t* a_src = sSFA + s * SF_BYTES + lane * 16;
+      const uint8_t* b_src = sSFB + s * SF_BYTES + lane * 16;
+      for (int kb = 0; kb < nkc; ++kb) {
+        tmem_st_32x32b_x4(lane_base + TM_SFA + s * 4 * KB + kb * 4, *reinterpret_cast<const uint4*>(a_src + kb * 512));
+        tmem_st_32x32b_x4(lane_base + TM_SFB + s * 4 * KB + kb * 4, *reinterpret_cast<const uint4*>(b_src + kb * 512));
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sf_full[s]);
+    }
+  } else {
+    // ------------------------------------------------------------ partial tile -> its rows' owners
+    // Row `row` of the tile is reduced by CTA row / rows_per; this CTA's
+    // partial of the row goes straight from tensor memory into slot `rank`
+    // of that CTA's receive buffer (distributed shared memory stores, which
+    // do not wait for a reply).  The receive buffer is not part of the ring,
+    // so a peer still computing is not disturbed.
+    const int sub = warp & 3;
+    const bool ok = mbar_wait_bounded(acc_full, 0u);
+    if (!ok) *abort_flag = 1;
+    if (ok) {
+      tc_fence_after();
+      const int rows_per = BM / split;  // split divides BM (a power of two up to 8)
+      const int row = sub * 32 + lane;
+      const int owner = row / rows_per;
+      const uint32_t dst = cluster_addr(recv + ((size_t)rank * rows_per + (row - owner * rows_per)) * PART_STRIDE,
+                                        (uint32_t)owner);
+      const uint32_t tbase = tmem + TM_ACC + ((uint32_t)(sub * 32) << 16);
+#pragma unroll
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tbase + c0, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 4u * (c0 + j)), "r"(r[j]),
+                       "r"(r[j + 1]), "r"(r[j + 2]), "r"(r[j + 3])
+                       : "memory");
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();  // every partial row is in its owner's receive buffer
+  // ---- reduction of this CTA's rows [rank * rows_per, +rows_per): per row 32
+  // groups of 4 columns, each the sum of the S partials in rank order 0..S-1
+  {
+    const int rows_per = BM / split;
+    const int r0 = rank * rows_per;
+    const float alpha = __fmul_rn(__ldg(p.a_ts), __ldg(p.b_ts));
+    const bool bad = *abort_flag != 0;
+    for (int item = threadIdx.x; item < rows_per * (BN / 4); item += THREADS) {
+      const int lrow = item / (BN / 4);
+      const int col = (item % (BN / 4)) * 4;
+      const int grow = m0 + r0 + lrow, gcol = n0 + col;
+      if (grow >= p.M || gcol >= p.N) continue;
+      float4 acc = *reinterpret_cast<const float4*>(recv + (size_t)lrow * PART_STRIDE + col);
+      for (int q = 1; q < split; ++q) {
+        const float4 v = *reinterpret_cast<const float4*>(recv + ((size_t)q * rows_per + lrow) * PART_STRIDE + col);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      if (bad) acc = make_float4(__int_as_float(0x7FC00000), __int_as_float(0x7FC00000),
+                                 __int_as_float(0x7FC00000), __int_as_float(0x7FC00000));
+      const uint32_t lo = pack_bf16x2(acc.x * alpha, acc.y * alpha), hi = pack_bf16x2(acc.z * alpha, acc.w * alpha);
+      __nv_bfloat16* dst = p.c + (int64_t)grow * p.ldc + gcol;
+      if (gcol + 4 <= p.N && p.c_vec8) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
+      } else {
+        const uint32_t w[2] = {lo, hi};
+        unsigned short* d16 = reinterpret_cast<unsigned short*>(dst);
+        for (int j = 0; j < 4 && gcol + j < p.N; ++j) d16[j] = (unsigned short)(w[j >> 1] >> (16 * (j & 1)));
+      }
+    }
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ host
 
 static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
@@ -658,6 +905,31 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   }
   return fn;
+}
+
+// Launch as a programmatic dependent launch (the kernel's set-up may overlap
+// the previous kernel of the stream; the kernel waits with griddepcontrol.wait
+// before it touches global memory), in clusters of `cluster` CTAs.
+template <typename K>
+static nvfp4_status launch_pdl(K kernel, int grid, int threads, int smem, int cluster, const CUtensorMap& ta,
+                               const CUtensorMap& tb, const GemmParams& p, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3((unsigned)threads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)cluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = cluster > 1 ? 2 : 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, ta, tb, p);
+  count_launches(1);
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
 // Row-major uint8 matrix [rows][row_bytes] -> tensor map with a box of
@@ -680,25 +952,15 @@ static nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* b, const GemmPa
   using C = GemmCfg<BN>;
   CUtensorMap ta, tb;
   if (!make_tmap(&ta, a, p.M, p.K / 2, C::BM) || !make_tmap(&tb, b, p.N, p.K / 2, C::BN)) return NVFP4_ERR_CUDA;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(gemm_w4a4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-        cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    attr_set = true;
-  }
-  // grouped problems: the tile count lives on the device, so one CTA per SM
-  const int tiles = p.groups > 0 ? 1 << 30 : ((p.N + C::BN - 1) / C::BN) * ((p.M + C::BM - 1) / C::BM);
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      sms = 148;
-  }
+  // the attribute is per device: set it on every call (cheap)
+  if (cudaFuncSetAttribute(gemm_w4a4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+      cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  const int tiles = ((p.N + C::BN - 1) / C::BN) * ((p.M + C::BM - 1) / C::BM);
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = tiles < sms ? tiles : sms;  // persistent: one CTA per SM
-  gemm_w4a4_kernel<BN><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, p);
-  count_launches(1);
-  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+  return launch_pdl(gemm_w4a4_kernel<BN>, grid, C::THREADS, C::SMEM_BYTES, 1, ta, tb, p, s);
 }
 
 // Dense problem on CTA pairs: one cluster of two CTAs per TPC, persistent
@@ -732,6 +994,32 @@ static nvfp4_status launch_gemm_pair(const uint8_t* a, const uint8_t* b, const G
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+// Split-K dispatch: the output has few 128 x 128 tiles.  S CTAs per tile
+// (one cluster), S = the SMs per tile rounded down, at most 8 and at most the
+// K stages; S = 1 means the split does not pay and the persistent kernel runs.
+static int splitk_factor(const GemmParams& p, int sms) {
+  const int tiles = ((p.M + splitk::BM - 1) / splitk::BM) * ((p.N + splitk::BN - 1) / splitk::BN);
+  const int num_kt = (p.kchunks + splitk::KB - 1) / splitk::KB;
+  if (tiles * 2 > sms) return 1;  // the persistent kernel fills the GPU at least as well
+  int sk = sms / tiles;
+  if (sk > splitk::MAX_SPLIT) sk = splitk::MAX_SPLIT;
+  if (sk > num_kt) sk = num_kt;
+  while (sk & (sk - 1)) --sk;  // a power of two, so that it divides the tile's 128 rows
+  return sk;
+}
+
+static nvfp4_status launch_gemm_splitk(const uint8_t* a, const uint8_t* b, const GemmParams& p, int split,
+                                       cudaStream_t s) {
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, a, p.M, p.K / 2, splitk::BM) || !make_tmap(&tb, b, p.N, p.K / 2, splitk::BN))
+    return NVFP4_ERR_CUDA;
+  if (cudaFuncSetAttribute(gemm_w4a4_splitk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           splitk::SMEM_BYTES) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  const int tiles = ((p.M + splitk::BM - 1) / splitk::BM) * ((p.N + splitk::BN - 1) / splitk::BN);
+  return launch_pdl(gemm_w4a4_splitk_kernel, tiles * split, splitk::THREADS, splitk::SMEM_BYTES, split, ta, tb, p, s);
+}
+
 template <int BN>
 static nvfp4_status launch_gemm_grouped(const uint8_t* a, const uint8_t* b, const GemmParams& p, int64_t b_rows,
                                         cudaStream_t s) {
@@ -743,9 +1031,7 @@ static nvfp4_status launch_gemm_grouped(const uint8_t* a, const uint8_t* b, cons
     return NVFP4_ERR_CUDA;
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  gemm_w4a4_kernel<BN><<<sms, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, p);
-  count_launches(1);
-  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+  return launch_pdl(gemm_w4a4_kernel<BN>, sms, C::THREADS, C::SMEM_BYTES, 1, ta, tb, p, s);
 }
 
 }  // namespace nvfp4
@@ -765,6 +1051,7 @@ nvfp4_status nvfp4_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_scales_mma
                              const uint8_t* b_codes, const uint8_t* b_scales_mma, const float* b_tensor_scale,
                              int64_t M, int64_t N, int64_t K, void* c, int64_t ldc, void* workspace,
                              size_t workspace_bytes, void* stream) {
+  NVFP4_ENTRY("nvfp4_gemm_w4a4");
   (void)workspace;
   (void)workspace_bytes;
   if (M < 1 || N < 1 || K < 64 || K % 64 != 0 || ldc < N) return NVFP4_ERR_SHAPE;
@@ -788,6 +1075,7 @@ nvfp4_status nvfp4_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_scales_mma
   p.b_rowtiles = (int)((N + 127) / 128);
   p.c_vec16 = (((uintptr_t)c & 15u) == 0 && (ldc % 8) == 0) ? 1 : 0;
   p.c_vec32 = (((uintptr_t)c & 31u) == 0 && (ldc % 16) == 0) ? 1 : 0;
+  p.c_vec8 = (((uintptr_t)c & 7u) == 0 && (ldc % 4) == 0) ? 1 : 0;
   p.groups = 0;
   p.a_off = nullptr;
   p.a_rows = nullptr;
@@ -795,6 +1083,10 @@ nvfp4_status nvfp4_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_scales_mma
   // against 80 us for the single-CTA kernel at 8192 x 4096 x 4096 (tensor pipe
   // 40% active, one accumulator drained between tiles); it is not dispatched.
   (void)launch_gemm_pair;
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int split = splitk_factor(p, sms);
+  if (split > 1) return launch_gemm_splitk(a_codes, b_codes, p, split, (cudaStream_t)stream);
   return launch_gemm<256>(a_codes, b_codes, p, (cudaStream_t)stream);
 }
 
@@ -811,6 +1103,7 @@ nvfp4_status nvfp4_gemm_w4a4_grouped(int groups, const uint8_t* a_codes, const u
                                      const int32_t* a_rows, const uint8_t* b_codes, const uint8_t* b_scales_mma,
                                      const float* b_tensor_scales, int64_t N, int64_t K, void* c, int64_t ldc,
                                      void* workspace, size_t workspace_bytes, void* stream) {
+  NVFP4_ENTRY("nvfp4_gemm_w4a4_grouped");
   (void)workspace;
   (void)workspace_bytes;
   if (groups < 1 || groups > GemmCfg<256>::MAX_GROUPS) return NVFP4_ERR_SHAPE;
@@ -837,6 +1130,7 @@ nvfp4_status nvfp4_gemm_w4a4_grouped(int groups, const uint8_t* a_codes, const u
   p.b_rowtiles = (int)((int64_t)groups * N / 128);
   p.c_vec16 = (((uintptr_t)c & 15u) == 0 && (ldc % 8) == 0) ? 1 : 0;
   p.c_vec32 = (((uintptr_t)c & 31u) == 0 && (ldc % 16) == 0) ? 1 : 0;
+  p.c_vec8 = (((uintptr_t)c & 7u) == 0 && (ldc % 4) == 0) ? 1 : 0;
   p.groups = groups;
   p.a_off = a_row_offsets;
   p.a_rows = a_rows;

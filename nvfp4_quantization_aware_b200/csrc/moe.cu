@@ -16,6 +16,7 @@
 // there, which the K-segmented weight-gradient GEMMs rely on.  Within a
 // segment rows are in increasing (token, slot) order, so every result is
 // deterministic.
+#include "moe_internal.cuh"
 #include "quant_common.cuh"
 
 namespace nvfp4 {
@@ -42,11 +43,13 @@ NVFP4_DEV int pad128(int n) { return (n + 127) & ~127; }
 // len[E] = T for the shared expert.
 // The last block marks assignments with an id outside [0, experts) (slot
 // -1, device error word kErrExpertId); they are routed nowhere.
-__global__ void route_count_kernel(const int32_t* __restrict__ ids, int assignments, int experts, int tokens,
+// shared_rows: rows of the shared expert's segment (tokens, or 0 when the
+// layer has no shared expert, e.g. the rows an expert-parallel rank received).
+__global__ void route_count_kernel(const int32_t* __restrict__ ids, int assignments, int experts, int shared_rows,
                                    int32_t* __restrict__ len, int32_t* __restrict__ slot_row) {
   const int e = blockIdx.x;
   if (e == experts) {
-    if (threadIdx.x == 0) len[e] = tokens;
+    if (threadIdx.x == 0) len[e] = shared_rows;
     for (int i = threadIdx.x; i < assignments; i += blockDim.x) {
       const int id = __ldg(ids + i);
       if (id < 0 || id >= experts) {
@@ -101,7 +104,7 @@ __global__ void __launch_bounds__(1024) route_scatter_kernel(
   const int n = __ldg(len + e);
   if (base + pad128(n) > rows_cap) return;  // reported above
   if (e == experts) {
-    for (int t = threadIdx.x; t < tokens; t += blockDim.x) {
+    for (int t = threadIdx.x; t < n; t += blockDim.x) {  // n = tokens, or 0 without a shared expert
       row_token[base + t] = t;
       row_weight[base + t] = 1.0f;
     }
@@ -122,7 +125,7 @@ __global__ void __launch_bounds__(1024) route_scatter_kernel(
       if (hit) {
         const int r = base + running + before + __popc(ballot & ((1u << lane) - 1u));
         row_token[r] = a / topk;
-        row_weight[r] = __ldg(weights + a);
+        row_weight[r] = weights ? __ldg(weights + a) : 1.0f;
         slot_row[a] = r;
       }
       running += chunk_total;
@@ -220,9 +223,11 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantRowsArgs a) {
 
 // out[t] = sum_j w[t, j] y[slot_row[t, j]] + y[shared_base + t]   (FP32 sum in
 // the fixed order j = 0..k-1, then the shared expert)
+// (without `shared` the shared expert's term is left out; NULL weights are 1)
 __global__ void combine_kernel(const __nv_bfloat16* __restrict__ y, int cols, const int32_t* __restrict__ slot_row,
                                const float* __restrict__ weights, int tokens, int topk,
-                               const int32_t* __restrict__ off, int experts, __nv_bfloat16* __restrict__ out) {
+                               const int32_t* __restrict__ off, int experts, int shared,
+                               __nv_bfloat16* __restrict__ out) {
   // one warp per token: its slot rows and weights are read once, the lanes
   // stride over the row's 16-byte vectors
   const int lane = threadIdx.x & 31;
@@ -231,7 +236,7 @@ __global__ void combine_kernel(const __nv_bfloat16* __restrict__ y, int cols, co
   const int warps = (int)(gridDim.x * blockDim.x / 32);
   for (int t = (int)((blockIdx.x * blockDim.x + threadIdx.x) / 32); t < tokens; t += warps) {
     const int my_r = lane < topk ? __ldg(slot_row + (int64_t)t * topk + lane) : -1;
-    const float my_w = lane < topk ? __ldg(weights + (int64_t)t * topk + lane) : 0.0f;
+    const float my_w = lane < topk ? (weights ? __ldg(weights + (int64_t)t * topk + lane) : 1.0f) : 0.0f;
     // warp-uniform trip count: every lane takes part in every shuffle; only
     // the loads and the store are predicated on the lane's vector
     for (int vb = 0; vb < vpr; vb += 32) {
@@ -250,11 +255,13 @@ __global__ void combine_kernel(const __nv_bfloat16* __restrict__ y, int cols, co
         acc[6] = fmaf(w, bf16lo_to_f32(v.w), acc[6]); acc[7] = fmaf(w, bf16hi_to_f32(v.w), acc[7]);
       }
       if (!act) continue;
-      const uint4 v = *reinterpret_cast<const uint4*>(y + (int64_t)(shared_base + t) * cols + c);
-      acc[0] += bf16lo_to_f32(v.x); acc[1] += bf16hi_to_f32(v.x);
-      acc[2] += bf16lo_to_f32(v.y); acc[3] += bf16hi_to_f32(v.y);
-      acc[4] += bf16lo_to_f32(v.z); acc[5] += bf16hi_to_f32(v.z);
-      acc[6] += bf16lo_to_f32(v.w); acc[7] += bf16hi_to_f32(v.w);
+      if (shared) {
+        const uint4 v = *reinterpret_cast<const uint4*>(y + (int64_t)(shared_base + t) * cols + c);
+        acc[0] += bf16lo_to_f32(v.x); acc[1] += bf16hi_to_f32(v.x);
+        acc[2] += bf16lo_to_f32(v.y); acc[3] += bf16hi_to_f32(v.y);
+        acc[4] += bf16lo_to_f32(v.z); acc[5] += bf16hi_to_f32(v.z);
+        acc[6] += bf16lo_to_f32(v.w); acc[7] += bf16hi_to_f32(v.w);
+      }
       *reinterpret_cast<uint4*>(out + (int64_t)t * cols + c) =
           make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
                      pack_bf16x2(acc[6], acc[7]));
@@ -340,7 +347,7 @@ __global__ void swiglu_bwd_kernel(const __nv_bfloat16* __restrict__ da, const __
 
 // dx[t] = sum_j dxp[slot_row[t, j]] + dxp[shared_base + t]   (fixed order)
 __global__ void gather_sum_kernel(const __nv_bfloat16* __restrict__ dxp, int cols, const int32_t* __restrict__ slot_row,
-                                  int tokens, int topk, const int32_t* __restrict__ off, int experts,
+                                  int tokens, int topk, const int32_t* __restrict__ off, int experts, int shared,
                                   __nv_bfloat16* __restrict__ dx) {
   // one warp per token (its slot rows read once), lanes over 16-byte vectors
   const int lane = threadIdx.x & 31;
@@ -355,7 +362,7 @@ __global__ void gather_sum_kernel(const __nv_bfloat16* __restrict__ dxp, int col
       const bool act = vc < vpr;
       const int c = vc * 8;
       float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      for (int j = 0; j <= topk; ++j) {
+      for (int j = 0; j < topk + shared; ++j) {
         const int rj = __shfl_sync(0xFFFFFFFFu, my_r, j < topk ? j : 0);
         const int r = j < topk ? rj : shared_base + t;
         if (r < 0 || !act) continue;
@@ -442,18 +449,59 @@ int64_t nvfp4_moe_rows_capacity(int tokens, int topk, int experts) {
   return (r + 127) / 128 * 128;
 }
 
-nvfp4_status nvfp4_moe_route(const int32_t* expert_ids, const float* combine_weights, int tokens, int topk,
-                             int experts, int32_t* seg_len, int32_t* seg_off, int32_t* row_token, float* row_weight,
-                             int32_t* slot_row, int64_t rows_cap, void* stream) {
+}  // extern "C"
+
+namespace nvfp4 {
+namespace moe {
+
+nvfp4_status route(const int32_t* expert_ids, const float* combine_weights, int tokens, int topk, int experts,
+                   bool shared, int32_t* seg_len, int32_t* seg_off, int32_t* row_token, float* row_weight,
+                   int32_t* slot_row, int64_t rows_cap, void* stream) {
   if (tokens < 1 || topk < 1 || experts < 1 || experts + 1 > kMaxGroups) return NVFP4_ERR_SHAPE;
   if (rows_cap < nvfp4_moe_rows_capacity(tokens, topk, experts) || rows_cap > 0x7FFFFFFF) return NVFP4_ERR_SHAPE;
-  if (!expert_ids || !combine_weights || !seg_len || !seg_off || !row_token || !row_weight || !slot_row)
+  if (!expert_ids || (shared && !combine_weights) || !seg_len || !seg_off || !row_token || !row_weight || !slot_row)
     return NVFP4_ERR_ARG;
   cudaStream_t s = (cudaStream_t)stream;
-  route_count_kernel<<<experts + 1, 1024, 0, s>>>(expert_ids, tokens * topk, experts, tokens, seg_len, slot_row);
+  route_count_kernel<<<experts + 1, 1024, 0, s>>>(expert_ids, tokens * topk, experts, shared ? tokens : 0, seg_len,
+                                                  slot_row);
   route_scatter_kernel<<<experts + 1, 1024, 0, s>>>(expert_ids, combine_weights, tokens, topk, experts, seg_len,
                                                     seg_off, row_token, row_weight, slot_row, (int)rows_cap);
   return done(2);
+}
+
+nvfp4_status combine(const void* y, int64_t cols, const int32_t* slot_row, const float* combine_weights, int tokens,
+                     int topk, const int32_t* seg_off, int experts, bool shared, void* out, void* stream) {
+  if (cols < 8 || cols % 8 || tokens < 1 || topk < 1 || topk > 32) return NVFP4_ERR_SHAPE;
+  if (!y || !slot_row || (shared && !combine_weights) || !seg_off || !out) return NVFP4_ERR_ARG;
+  if (((uintptr_t)y & 15u) || ((uintptr_t)out & 15u)) return NVFP4_ERR_ALIGN;
+  combine_kernel<<<sms() * 8, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const __nv_bfloat16*>(y), (int)cols,
+                                                              slot_row, combine_weights, tokens, topk, seg_off, experts,
+                                                              shared ? 1 : 0, reinterpret_cast<__nv_bfloat16*>(out));
+  return done(1);
+}
+
+nvfp4_status gather_sum(const void* dxp, int64_t cols, const int32_t* slot_row, int tokens, int topk,
+                        const int32_t* seg_off, int experts, bool shared, void* dx, void* stream) {
+  if (cols < 8 || cols % 8 || tokens < 1 || topk < 1 || topk > 32) return NVFP4_ERR_SHAPE;
+  if (!dxp || !slot_row || !seg_off || !dx) return NVFP4_ERR_ARG;
+  if (((uintptr_t)dxp & 15u) || ((uintptr_t)dx & 15u)) return NVFP4_ERR_ALIGN;
+  gather_sum_kernel<<<sms() * 8, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const __nv_bfloat16*>(dxp), (int)cols,
+                                                                 slot_row, tokens, topk, seg_off, experts,
+                                                                 shared ? 1 : 0, reinterpret_cast<__nv_bfloat16*>(dx));
+  return done(1);
+}
+
+}  // namespace moe
+}  // namespace nvfp4
+
+extern "C" {
+
+nvfp4_status nvfp4_moe_route(const int32_t* expert_ids, const float* combine_weights, int tokens, int topk,
+                             int experts, int32_t* seg_len, int32_t* seg_off, int32_t* row_token, float* row_weight,
+                             int32_t* slot_row, int64_t rows_cap, void* stream) {
+  NVFP4_ENTRY("nvfp4_moe_route");
+  return moe::route(expert_ids, combine_weights, tokens, topk, experts, true, seg_len, seg_off, row_token, row_weight,
+                    slot_row, rows_cap, stream);
 }
 
 static nvfp4_status quant_rows(bool gather, const void* src, const void* src2, int64_t ld_src, const int32_t* row_token,
@@ -490,6 +538,7 @@ static nvfp4_status quant_rows(bool gather, const void* src, const void* src2, i
 nvfp4_status nvfp4_moe_gather_quantize(const void* x, int64_t ld_x, const int32_t* row_token, const int32_t* seg_off,
                                        int groups, const float* tensor_scales, int64_t rows_cap, int64_t cols,
                                        uint8_t* codes, uint8_t* scales_mma, void* xhat, void* stream) {
+  NVFP4_ENTRY("nvfp4_moe_gather_quantize");
   return quant_rows(true, x, nullptr, ld_x, row_token, seg_off, groups, tensor_scales, rows_cap, cols, codes,
                     scales_mma, xhat, nullptr, stream);
 }
@@ -498,23 +547,21 @@ nvfp4_status nvfp4_moe_swiglu_quantize(const void* h_gate, const void* h_up, int
                                        const int32_t* seg_off, int groups, const float* tensor_scales, int64_t rows_cap,
                                        int64_t cols, uint8_t* codes, uint8_t* scales_mma, void* ahat, void* act,
                                        void* stream) {
+  NVFP4_ENTRY("nvfp4_moe_swiglu_quantize");
   return quant_rows(false, h_gate, h_up, ld_h, row_token, seg_off, groups, tensor_scales, rows_cap, cols, codes,
                     scales_mma, ahat, act, stream);
 }
 
 nvfp4_status nvfp4_moe_combine(const void* y, int64_t cols, const int32_t* slot_row, const float* combine_weights,
                                int tokens, int topk, const int32_t* seg_off, int experts, void* out, void* stream) {
-  if (cols < 8 || cols % 8 || tokens < 1 || topk < 1 || topk > 32) return NVFP4_ERR_SHAPE;
-  if (!y || !slot_row || !combine_weights || !seg_off || !out) return NVFP4_ERR_ARG;
-  if (((uintptr_t)y & 15u) || ((uintptr_t)out & 15u)) return NVFP4_ERR_ALIGN;
-  combine_kernel<<<sms() * 8, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const __nv_bfloat16*>(y), (int)cols,
-                                                              slot_row, combine_weights, tokens, topk, seg_off, experts,
-                                                              reinterpret_cast<__nv_bfloat16*>(out));
-  return done(1);
+  NVFP4_ENTRY("nvfp4_moe_combine");
+  if (!combine_weights) return NVFP4_ERR_ARG;
+  return moe::combine(y, cols, slot_row, combine_weights, tokens, topk, seg_off, experts, true, out, stream);
 }
 
 nvfp4_status nvfp4_moe_scale_rows(const void* dy, int64_t cols, const int32_t* row_token, const float* row_weight,
                                   const int32_t* seg_off, int groups, int64_t rows_cap, void* dyp, void* stream) {
+  NVFP4_ENTRY("nvfp4_moe_scale_rows");
   if (cols < 8 || cols % 8 || rows_cap < 1 || groups < 1) return NVFP4_ERR_SHAPE;
   if (!dy || !row_token || !row_weight || !seg_off || !dyp) return NVFP4_ERR_ARG;
   if (((uintptr_t)dy & 15u) || ((uintptr_t)dyp & 15u)) return NVFP4_ERR_ALIGN;
@@ -527,6 +574,7 @@ nvfp4_status nvfp4_moe_scale_rows(const void* dy, int64_t cols, const int32_t* r
 nvfp4_status nvfp4_moe_swiglu_backward(const void* da, const void* h_gate, const void* h_up, int64_t cols,
                                        const int32_t* row_token, const int32_t* seg_off, int groups, int64_t rows_cap,
                                        void* dgu, void* stream) {
+  NVFP4_ENTRY("nvfp4_moe_swiglu_backward");
   if (cols < 8 || cols % 8 || rows_cap < 1 || groups < 1) return NVFP4_ERR_SHAPE;
   if (!da || !h_gate || !h_up || !row_token || !seg_off || !dgu) return NVFP4_ERR_ARG;
   if (((uintptr_t)da & 15u) || ((uintptr_t)h_gate & 15u) || ((uintptr_t)h_up & 15u) || ((uintptr_t)dgu & 15u))
@@ -540,17 +588,13 @@ nvfp4_status nvfp4_moe_swiglu_backward(const void* da, const void* h_gate, const
 
 nvfp4_status nvfp4_moe_gather_sum(const void* dxp, int64_t cols, const int32_t* slot_row, int tokens, int topk,
                                   const int32_t* seg_off, int experts, void* dx, void* stream) {
-  if (cols < 8 || cols % 8 || tokens < 1 || topk < 1 || topk > 32) return NVFP4_ERR_SHAPE;
-  if (!dxp || !slot_row || !seg_off || !dx) return NVFP4_ERR_ARG;
-  if (((uintptr_t)dxp & 15u) || ((uintptr_t)dx & 15u)) return NVFP4_ERR_ALIGN;
-  gather_sum_kernel<<<sms() * 8, 256, 0, (cudaStream_t)stream>>>(reinterpret_cast<const __nv_bfloat16*>(dxp), (int)cols,
-                                                                 slot_row, tokens, topk, seg_off, experts,
-                                                                 reinterpret_cast<__nv_bfloat16*>(dx));
-  return done(1);
+  NVFP4_ENTRY("nvfp4_moe_gather_sum");
+  return moe::gather_sum(dxp, cols, slot_row, tokens, topk, seg_off, experts, true, dx, stream);
 }
 
 nvfp4_status nvfp4_moe_router_grad(const void* dy, const void* y, int64_t cols, const int32_t* slot_row, int tokens,
                                    int topk, float* dw, void* stream) {
+  NVFP4_ENTRY("nvfp4_moe_router_grad");
   if (cols < 8 || cols % 8 || tokens < 1 || topk < 1) return NVFP4_ERR_SHAPE;
   if (!dy || !y || !slot_row || !dw) return NVFP4_ERR_ARG;
   if (((uintptr_t)dy & 15u) || ((uintptr_t)y & 15u)) return NVFP4_ERR_ALIGN;
@@ -561,6 +605,7 @@ nvfp4_status nvfp4_moe_router_grad(const void* dy, const void* y, int64_t cols, 
 }
 
 nvfp4_status nvfp4_scales_to_mma(const uint8_t* block_scales, int64_t rows, int64_t cols, uint8_t* out, void* stream) {
+  NVFP4_ENTRY("nvfp4_scales_to_mma");
   if (rows < 1 || cols < 16 || cols % 16) return NVFP4_ERR_SHAPE;
   if (!block_scales || !out) return NVFP4_ERR_ARG;
   scales_to_mma_kernel<<<sms() * 8, 256, 0, (cudaStream_t)stream>>>(block_scales, rows, cols, out);

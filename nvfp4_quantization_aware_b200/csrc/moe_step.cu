@@ -18,7 +18,7 @@
 //   d(combine weight) = <dy, y_expert>.
 #include <cstring>
 
-#include "common.cuh"
+#include "moe_internal.cuh"
 
 namespace {
 
@@ -115,19 +115,26 @@ int64_t qad_moe_rows_capacity(const qad_moe_shape* shape) {
   return layout_of(*shape).rows_cap;
 }
 
-nvfp4_status qad_moe_forward(const qad_moe_shape* shape, const qad_moe_weights* w, const void* x,
-                             const int32_t* expert_ids, const float* combine_weights, void* y, void* workspace,
-                             size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The layer step; without `shared` there is no shared expert (group E holds
+// no rows and its weights are not read), combine_weights may be NULL (weight
+// 1), and G below counts the routed experts only.
+nvfp4_status moe_forward(const qad_moe_shape* shape, const qad_moe_weights* w, const void* x,
+                         const int32_t* expert_ids, const float* combine_weights, void* y, void* workspace,
+                         size_t workspace_bytes, void* stream, bool shared) {
   if (!shape_ok(shape)) return NVFP4_ERR_SHAPE;
   QAD_TRY(weights_ok(w));
-  if (!x || !expert_ids || !combine_weights || !y) return NVFP4_ERR_ARG;
+  if (!x || !expert_ids || (shared && !combine_weights) || !y) return NVFP4_ERR_ARG;
   const qad_moe_shape& s = *shape;
   const Layout L = layout_of(s);
   if (!workspace || workspace_bytes < L.total) return NVFP4_ERR_WORKSPACE;
   if (((uintptr_t)workspace & 255u) || ((uintptr_t)x & 15u) || ((uintptr_t)y & 15u) || ((uintptr_t)w->w_gate & 15u) ||
       ((uintptr_t)w->w_up & 15u) || ((uintptr_t)w->w_down & 15u))
     return NVFP4_ERR_ALIGN;
-  const int G = s.experts + 1;
+  const int G = s.experts + (shared ? 1 : 0);
   const int64_t H = s.hidden, F = s.ffn, R = L.rows_cap;
   int32_t* seg_len = at<int32_t>(workspace, L, QAD_MOE_SEG_LEN);
   int32_t* seg_off = at<int32_t>(workspace, L, QAD_MOE_SEG_OFF);
@@ -136,8 +143,8 @@ nvfp4_status qad_moe_forward(const qad_moe_shape* shape, const qad_moe_weights* 
   int32_t* slot_row = at<int32_t>(workspace, L, QAD_MOE_SLOT_ROW);
 
   // 1. routing: segments and the permutation
-  QAD_TRY(nvfp4_moe_route(expert_ids, combine_weights, s.tokens, s.topk, s.experts, seg_len, seg_off, row_token,
-                          row_weight, slot_row, R, stream));
+  QAD_TRY(nvfp4::moe::route(expert_ids, combine_weights, s.tokens, s.topk, s.experts, shared, seg_len, seg_off,
+                            row_token, row_weight, slot_row, R, stream));
   // 2. master weights -> NVFP4 codes with their frozen scales, and the bf16
   //    dequantized weights the backward multiplies with (one call, 3G tensors):
   //    W^_gate / W^_up of group g interleaved as rows [2gF, 2gF + F) / [2gF + F,
@@ -203,13 +210,13 @@ nvfp4_status qad_moe_forward(const qad_moe_shape* shape, const qad_moe_weights* 
                                   at<uint8_t>(workspace, L, QAD_MOE_WD_CODES), w->down_sb_mma, w->down_ts, H, F,
                                   at<void>(workspace, L, QAD_MOE_Y_ROWS), H, nullptr, 0, stream));
   // 7. combine
-  return nvfp4_moe_combine(at<void>(workspace, L, QAD_MOE_Y_ROWS), H, slot_row, combine_weights, s.tokens, s.topk,
-                           seg_off, s.experts, y, stream);
+  return nvfp4::moe::combine(at<void>(workspace, L, QAD_MOE_Y_ROWS), H, slot_row, combine_weights, s.tokens, s.topk,
+                             seg_off, s.experts, shared, y, stream);
 }
 
-nvfp4_status qad_moe_backward(const qad_moe_shape* shape, const qad_moe_weights* w, const void* dy, void* dx,
-                              void* dw_gate, void* dw_up, void* dw_down, float* d_combine, void* workspace,
-                              size_t workspace_bytes, void* stream) {
+nvfp4_status moe_backward(const qad_moe_shape* shape, const qad_moe_weights* w, const void* dy, void* dx,
+                          void* dw_gate, void* dw_up, void* dw_down, float* d_combine, void* workspace,
+                          size_t workspace_bytes, void* stream, bool shared) {
   if (!shape_ok(shape)) return NVFP4_ERR_SHAPE;
   QAD_TRY(weights_ok(w));
   if (!dy || !dx || !dw_gate || !dw_up || !dw_down) return NVFP4_ERR_ARG;
@@ -219,7 +226,7 @@ nvfp4_status qad_moe_backward(const qad_moe_shape* shape, const qad_moe_weights*
   if (((uintptr_t)workspace & 255u) || ((uintptr_t)dy & 15u) || ((uintptr_t)dx & 15u) || ((uintptr_t)dw_gate & 15u) ||
       ((uintptr_t)dw_up & 15u) || ((uintptr_t)dw_down & 15u))
     return NVFP4_ERR_ALIGN;
-  const int G = s.experts + 1;
+  const int G = s.experts + (shared ? 1 : 0);
   const int64_t H = s.hidden, F = s.ffn, R = L.rows_cap;
   int32_t* seg_len = at<int32_t>(workspace, L, QAD_MOE_SEG_LEN);
   int32_t* seg_off = at<int32_t>(workspace, L, QAD_MOE_SEG_OFF);
@@ -248,7 +255,7 @@ nvfp4_status qad_moe_backward(const qad_moe_shape* shape, const qad_moe_weights*
   // K rows 2 g F .. 2 (g+1) F - 1), then the sum over each token's experts
   QAD_TRY(nvfp4_gemm_bf16_grouped(0, G, dgu, 0, R, 2 * F, 2 * F, wgu_hat, 1, (int64_t)G * 2 * F, H, H, seg_off,
                                   seg_len, 0, H, 2 * F, dxp, H, stream));
-  QAD_TRY(nvfp4_moe_gather_sum(dxp, H, slot_row, s.tokens, s.topk, seg_off, s.experts, dx, stream));
+  QAD_TRY(nvfp4::moe::gather_sum(dxp, H, slot_row, s.tokens, s.topk, seg_off, s.experts, shared, dx, stream));
   // weight gradients, reduced over each expert's rows (K-segments, both
   // operands MN-major: the row buffers as they are)
   //   dW_down_g[h][f] = sum_r dY[r][h] A^[r][f]
@@ -264,6 +271,40 @@ nvfp4_status qad_moe_backward(const qad_moe_shape* shape, const qad_moe_weights*
     QAD_TRY(nvfp4_moe_router_grad(dy, at<void>(workspace, L, QAD_MOE_Y_ROWS), H, slot_row, s.tokens, s.topk, d_combine,
                                   stream));
   return NVFP4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+nvfp4_status qad_moe_forward(const qad_moe_shape* shape, const qad_moe_weights* w, const void* x,
+                             const int32_t* expert_ids, const float* combine_weights, void* y, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  NVFP4_ENTRY("qad_moe_forward");
+  return moe_forward(shape, w, x, expert_ids, combine_weights, y, workspace, workspace_bytes, stream, true);
+}
+
+nvfp4_status qad_moe_backward(const qad_moe_shape* shape, const qad_moe_weights* w, const void* dy, void* dx,
+                              void* dw_gate, void* dw_up, void* dw_down, float* d_combine, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  NVFP4_ENTRY("qad_moe_backward");
+  return moe_backward(shape, w, dy, dx, dw_gate, dw_up, dw_down, d_combine, workspace, workspace_bytes, stream, true);
+}
+
+nvfp4_status qad_moe_expert_forward(const qad_moe_shape* shape, const qad_moe_weights* w, const void* x,
+                                    const int32_t* expert_ids, void* y, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  NVFP4_ENTRY("qad_moe_expert_forward");
+  if (!shape || shape->topk != 1) return NVFP4_ERR_SHAPE;
+  return moe_forward(shape, w, x, expert_ids, nullptr, y, workspace, workspace_bytes, stream, false);
+}
+
+nvfp4_status qad_moe_expert_backward(const qad_moe_shape* shape, const qad_moe_weights* w, const void* dy, void* dx,
+                                     void* dw_gate, void* dw_up, void* dw_down, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  NVFP4_ENTRY("qad_moe_expert_backward");
+  if (!shape || shape->topk != 1) return NVFP4_ERR_SHAPE;
+  return moe_backward(shape, w, dy, dx, dw_gate, dw_up, dw_down, nullptr, workspace, workspace_bytes, stream, false);
 }
 
 }  // extern "C"

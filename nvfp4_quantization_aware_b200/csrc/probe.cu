@@ -89,17 +89,49 @@ __global__ void __launch_bounds__(THREADS, 1) fp4_mma_probe_kernel(int64_t iters
 using namespace nvfp4;
 
 extern "C" nvfp4_status nvfp4_probe_fp4_mma(int64_t iters, int ctas, double* flop_per_launch, void* stream) {
+  NVFP4_ENTRY("nvfp4_probe_fp4_mma");
   if (iters < 1 || iters > ((int64_t)1 << 40) || ctas < 1 || ctas > 4096) return NVFP4_ERR_ARG;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(probe::fp4_mma_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             probe::SMEM_BYTES) != cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    attr = true;
-  }
+  // the attribute is per device: set it on every call (cheap)
+  if (cudaFuncSetAttribute(probe::fp4_mma_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, probe::SMEM_BYTES) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
   probe::fp4_mma_probe_kernel<<<ctas, probe::THREADS, probe::SMEM_BYTES, (cudaStream_t)stream>>>(iters);
   count_launches(1);
   if (flop_per_launch)
     *flop_per_launch = 2.0 * probe::BM * probe::BN * 64.0 * probe::KB * (double)iters * (double)ctas;
+  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ bounded-wait self-test
+//
+// Every wait of this library's kernels (on an mbarrier, a TMA transaction, a
+// peer) is bounded: when it expires the kernel sets the device error word
+// and returns instead of hanging.  This kernel exercises exactly that path:
+// one thread waits on an mbarrier that nothing arrives at, with a caller-given
+// cycle limit, then reports the expiry the way every other wait does.
+namespace nvfp4 {
+__global__ void timeout_selftest_kernel(long long limit_cycles) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(&bar, 0)) {
+      if (clock64() - t0 > limit_cycles) {
+        report_error(kErrWaitTimeout);
+        break;
+      }
+    }
+  }
+}
+}  // namespace nvfp4
+
+extern "C" nvfp4_status nvfp4_selftest_timeout(int64_t limit_cycles, void* stream) {
+  NVFP4_ENTRY("nvfp4_selftest_timeout");
+  if (limit_cycles < 1 || limit_cycles > (1ll << 32)) return NVFP4_ERR_ARG;
+  nvfp4::timeout_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((long long)limit_cycles);
+  nvfp4::count_launches(1);
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }

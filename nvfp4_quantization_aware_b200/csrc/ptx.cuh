@@ -281,6 +281,51 @@ NVFP4_DEV void cluster_sync_all() {
 // counted by complete_tx, not plain memory traffic.  Cluster-scope acquire /
 // release forms put a memory fence on the MMA thread's path every stage.
 
+// Arrive on a barrier given by its shared::cluster address, releasing this
+// thread's earlier memory operations (e.g. distributed shared memory stores
+// into the barrier owner's CTA) at cluster scope.
+NVFP4_DEV void mbar_arrive_release_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
+// Bounded wait on a barrier of this CTA with cluster-scope acquire (what the
+// arrivals released becomes visible).  On expiry it sets the device error word
+// and returns false.
+NVFP4_DEV bool mbar_wait_acquire_cluster(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  for (;;) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      report_error(kErrWaitTimeout);
+      return false;
+    }
+  }
+}
+
+// Asynchronous stores into another CTA's shared memory (shared::cluster
+// addresses) whose bytes complete a transaction on that CTA's mbarrier: the
+// receiver's phase completes only once the data is there, with no fence on
+// the sender's side.
+NVFP4_DEV void st_async_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t bar_cluster) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+               "r"(a), "r"(b), "r"(c), "r"(d), "r"(bar_cluster)
+               : "memory");
+}
+
+NVFP4_DEV void st_async_b32(uint32_t addr, uint32_t v, uint32_t bar_cluster) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(addr), "r"(v),
+               "r"(bar_cluster)
+               : "memory");
+}
+
 // Arrive on a barrier given by its shared::cluster address (either CTA).
 NVFP4_DEV void mbar_arrive_cluster(uint32_t bar_cluster) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");

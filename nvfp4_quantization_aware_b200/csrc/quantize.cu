@@ -106,6 +106,8 @@ struct GroupArgs {
   int layout;           // nvfp4_scale_layout of written block scales
   int64_t total_chunks;
   unsigned* amax;       // DYNAMIC: n words holding max |x| as float bits (zeroed first)
+  unsigned* amax_part;  // DYNAMIC, one tensor: per-CTA maxima of the amax launch (or NULL)
+  int amax_grid;        // CTAs of that launch (entries of amax_part)
   int x_wide;           // every input row start is 32-byte aligned: 256-bit loads
   int out_wide;         // codes rows 8-byte aligned (8-byte stores)
   int y_wide;           // y rows 32-byte aligned (256-bit stores)
@@ -208,16 +210,24 @@ NVFP4_DEV void amax_range(const GroupArgs& a, int64_t c_begin, int64_t c_end, un
   if (lane == 0 && mt >= 0 && w > 0.0f) atomicMax(s_max + mt, __float_as_uint(w));
 }
 
+// With amax_part (a single tensor) every CTA writes its maximum to its own
+// entry instead, so nothing has to be cleared before the launch; the encode
+// kernel folds the entries.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) group_amax_kernel(const __grid_constant__ GroupArgs a) {
   __shared__ unsigned s_max[kMaxGroup];
   for (int i = threadIdx.x; i < a.n; i += kThreads) s_max[i] = 0u;
   __syncthreads();
+  griddep_wait();
   const int64_t per_cta = (a.total_chunks + gridDim.x - 1) / gridDim.x;
   const int64_t c_begin = (int64_t)blockIdx.x * per_cta;
   const int64_t c_end = c_begin + per_cta < a.total_chunks ? c_begin + per_cta : a.total_chunks;
   amax_range<T>(a, c_begin, c_end, s_max);
   __syncthreads();
+  if (a.amax_part != nullptr) {
+    if (threadIdx.x == 0) a.amax_part[blockIdx.x] = s_max[0];
+    return;
+  }
   for (int i = threadIdx.x; i < a.n; i += kThreads)
     if (s_max[i] != 0u) atomicMax(a.amax + i, s_max[i]);
 }
@@ -338,6 +348,24 @@ NVFP4_DEV void encode_range(const GroupArgs& a, int64_t warp, int64_t nwarps, Sg
 
 template <typename T, Out OUT>
 __global__ void __launch_bounds__(kThreads) group_encode_kernel(const __grid_constant__ GroupArgs a) {
+  griddep_wait();
+  if (a.mode == NVFP4_DYNAMIC && a.amax_part != nullptr) {
+    // one tensor: its max is the max of the amax launch's per-CTA entries
+    __shared__ unsigned s_warp[kWarps];
+    unsigned m = 0u;
+    for (int i = threadIdx.x; i < a.amax_grid; i += kThreads) m = max(m, __ldcg(a.amax_part + i));
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    if ((threadIdx.x & 31) == 0) s_warp[threadIdx.x >> 5] = m;
+    __syncthreads();
+    m = s_warp[0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) m = max(m, s_warp[w]);
+    const float sg = __fdiv_rn(__uint_as_float(m), 2688.0f);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *a.t[0].ts = sg;
+    encode_range<T, OUT>(a, (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5), (int64_t)gridDim.x * kWarps,
+                         [&](int) { return sg; });
+    return;
+  }
   if (a.mode == NVFP4_DYNAMIC && blockIdx.x == 0)
     for (int i = threadIdx.x; i < a.n; i += kThreads) *a.t[i].ts = tensor_scale_of(a, i);
   encode_range<T, OUT>(a, (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5), (int64_t)gridDim.x * kWarps,
@@ -616,6 +644,11 @@ static nvfp4_status launch_status() {
 }
 
 constexpr size_t kDynamicWorkspace = 1024;  // 256 amax words, >= kMaxGroup
+// What the size queries ask for: the amax words, then one word per CTA of a
+// single tensor's amax launch (that path needs no clearing launch).  A
+// workspace of only kDynamicWorkspace bytes still works (clear + atomics).
+constexpr size_t kDynamicWorkspacePart = 8192;
+constexpr int kMaxAmaxGrid = (int)((kDynamicWorkspacePart - kDynamicWorkspace) / sizeof(unsigned));
 
 // Validate one tensor of a (possibly grouped) quantize / fake-quant call.
 template <Out OUT>
@@ -703,20 +736,53 @@ static nvfp4_status launch_small_dynamic(const GroupArgs& a, cudaStream_t s) {
 // DYNAMIC groups this small take the one-launch cluster path.
 static bool small_dynamic(const GroupArgs& a) { return a.mode == NVFP4_DYNAMIC && a.total_chunks <= kSmallChunks; }
 
+// The encode launch of a DYNAMIC group follows its amax launch as a
+// programmatic dependent launch: it may be scheduled while the amax launch
+// drains and waits (griddepcontrol.wait) before touching memory.
+template <typename K>
+static nvfp4_status launch_dependent(K kernel, int grid, const GroupArgs& a, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, a) != cudaSuccess) return NVFP4_ERR_CUDA;
+  count_launches(1);
+  return launch_status();
+}
+
 template <Out OUT>
-static nvfp4_status launch_group(GroupArgs& a, nvfp4_dtype dtype, unsigned* amax, cudaStream_t s) {
+static nvfp4_status launch_group(GroupArgs& a, nvfp4_dtype dtype, unsigned* amax, unsigned* amax_part,
+                                 cudaStream_t s) {
   if (a.n == 0 || a.total_chunks == 0) return NVFP4_OK;
   if (small_dynamic(a))
     return dtype == NVFP4_BF16 ? launch_small_dynamic<OUT, __nv_bfloat16>(a, s) : launch_small_dynamic<OUT, float>(a, s);
+  a.amax_part = nullptr;
+  a.amax_grid = 0;
   if (a.mode == NVFP4_DYNAMIC) {
     a.amax = amax;
+    const void* fn = dtype == NVFP4_BF16 ? (const void*)group_amax_kernel<__nv_bfloat16> : (const void*)group_amax_kernel<float>;
+    const int grid = resident_grid(fn, a.total_chunks);
+    if (a.n == 1 && amax_part != nullptr && grid <= kMaxAmaxGrid) {
+      a.amax_part = amax_part;
+      a.amax_grid = grid;
+    }
     if (dtype == NVFP4_BF16)
-      group_amax_kernel<__nv_bfloat16>
-          <<<resident_grid((const void*)group_amax_kernel<__nv_bfloat16>, a.total_chunks), kThreads, 0, s>>>(a);
+      group_amax_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(a);
     else
-      group_amax_kernel<float><<<resident_grid((const void*)group_amax_kernel<float>, a.total_chunks), kThreads, 0, s>>>(a);
+      group_amax_kernel<float><<<grid, kThreads, 0, s>>>(a);
     count_launches(1);
     if (launch_status() != NVFP4_OK) return NVFP4_ERR_CUDA;
+    if (dtype == NVFP4_BF16)
+      return launch_dependent(group_encode_kernel<__nv_bfloat16, OUT>,
+                              resident_grid((const void*)group_encode_kernel<__nv_bfloat16, OUT>, a.total_chunks), a, s);
+    return launch_dependent(group_encode_kernel<float, OUT>,
+                            resident_grid((const void*)group_encode_kernel<float, OUT>, a.total_chunks), a, s);
   }
   if (dtype == NVFP4_BF16)
     group_encode_kernel<__nv_bfloat16, OUT>
@@ -749,8 +815,10 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
     if (!aligned16(ws)) return NVFP4_ERR_ALIGN;
   }
   const int64_t esz = dtype == NVFP4_BF16 ? 2 : 4;
-  static GroupArgs a;  // host staging of the kernel parameter (copied at launch)
+  GroupArgs a;  // host staging of the kernel parameter (copied at launch)
   a.n = 0;
+  a.amax_part = nullptr;
+  a.amax_grid = 0;
   a.mode = (int)mode;
   a.layout = (int)layout;
   a.total_chunks = 0;
@@ -763,14 +831,18 @@ static nvfp4_status run_tensors(int n, const nvfp4_tensor_ref* refs, nvfp4_dtype
   unsigned* words = reinterpret_cast<unsigned*>(ws);
   const int nwords = (int)(kDynamicWorkspace / sizeof(unsigned));
   int word_base = nwords;  // forces a clear before the first group
+  // A single-tensor group takes per-CTA maxima in the rest of a workspace of
+  // kDynamicWorkspacePart bytes instead (no clear needed).
+  unsigned* part = ws_bytes >= kDynamicWorkspacePart ? words + nwords : nullptr;
   auto flush = [&]() -> nvfp4_status {
     if (a.n == 0) return NVFP4_OK;
     const int need = a.n;
-    if (mode == NVFP4_DYNAMIC && !small_dynamic(a) && word_base + need > nwords) {
+    const bool use_part = a.n == 1 && part != nullptr;
+    if (mode == NVFP4_DYNAMIC && !small_dynamic(a) && !use_part && word_base + need > nwords) {
       if (cudaMemsetAsync(ws, 0, kDynamicWorkspace, s) != cudaSuccess) return NVFP4_ERR_CUDA;
       word_base = 0;
     }
-    nvfp4_status st = launch_group<OUT>(a, dtype, words + word_base, s);
+    nvfp4_status st = launch_group<OUT>(a, dtype, words + word_base, use_part ? part : nullptr, s);
     word_base += need;
     return st;
   };
@@ -847,19 +919,20 @@ size_t nvfp4_mma_scales_bytes(int64_t rows, int64_t cols) {
 size_t nvfp4_quantize_workspace_size(int64_t rows, int64_t cols, nvfp4_scale_mode mode) {
   (void)rows;
   (void)cols;
-  return mode == NVFP4_DYNAMIC ? kDynamicWorkspace : 0;
+  return mode == NVFP4_DYNAMIC ? kDynamicWorkspacePart : 0;
 }
 
 size_t nvfp4_fake_quant_workspace_size(int64_t rows, int64_t cols, nvfp4_scale_mode mode) {
   return nvfp4_quantize_workspace_size(rows, cols, mode);
 }
 
-size_t nvfp4_grouped_workspace_size(nvfp4_scale_mode mode) { return mode == NVFP4_DYNAMIC ? kDynamicWorkspace : 0; }
+size_t nvfp4_grouped_workspace_size(nvfp4_scale_mode mode) { return mode == NVFP4_DYNAMIC ? kDynamicWorkspacePart : 0; }
 
 nvfp4_status nvfp4_quantize(const void* x, nvfp4_dtype dtype, int64_t rows, int64_t cols, int64_t ld_x,
                             nvfp4_scale_mode mode, float* tensor_scale, uint8_t* block_scales,
                             nvfp4_scale_layout layout, uint8_t* codes, int64_t ld_codes, void* workspace,
                             size_t workspace_bytes, void* stream) {
+  NVFP4_ENTRY("nvfp4_quantize");
   nvfp4_tensor_ref r;
   r.x = x;
   r.rows = rows;
@@ -875,6 +948,7 @@ nvfp4_status nvfp4_quantize(const void* x, nvfp4_dtype dtype, int64_t rows, int6
 nvfp4_status nvfp4_fake_quant(const void* x, nvfp4_dtype dtype, int64_t rows, int64_t cols, int64_t ld_x,
                               nvfp4_scale_mode mode, float* tensor_scale, uint8_t* block_scales, void* y,
                               int64_t ld_y, void* workspace, size_t workspace_bytes, void* stream) {
+  NVFP4_ENTRY("nvfp4_fake_quant");
   nvfp4_tensor_ref r;
   r.x = x;
   r.rows = rows;
@@ -891,6 +965,7 @@ nvfp4_status nvfp4_fake_quant(const void* x, nvfp4_dtype dtype, int64_t rows, in
 nvfp4_status nvfp4_quantize_grouped(int num_tensors, const nvfp4_tensor_ref* tensors, nvfp4_dtype dtype,
                                     nvfp4_scale_mode mode, nvfp4_scale_layout layout, void* workspace,
                                     size_t workspace_bytes, void* stream) {
+  NVFP4_ENTRY("nvfp4_quantize_grouped");
   return run_tensors<Out::Codes>(num_tensors, tensors, dtype, mode, layout, workspace, workspace_bytes,
                                  (cudaStream_t)stream);
 }
@@ -899,12 +974,14 @@ nvfp4_status nvfp4_quantize_fake_quant_grouped(int num_tensors, const nvfp4_tens
                                                const int64_t* ld_y, nvfp4_dtype dtype, nvfp4_scale_mode mode,
                                                nvfp4_scale_layout layout, void* workspace, size_t workspace_bytes,
                                                void* stream) {
+  NVFP4_ENTRY("nvfp4_quantize_fake_quant_grouped");
   return run_tensors<Out::Both>(num_tensors, tensors, dtype, mode, layout, workspace, workspace_bytes,
                                 (cudaStream_t)stream, y, ld_y);
 }
 
 nvfp4_status nvfp4_calibrate_mse_grouped(int num_tensors, const nvfp4_tensor_ref* tensors, nvfp4_dtype dtype,
                                          float* const* block_err, void* stream) {
+  NVFP4_ENTRY("nvfp4_calibrate_mse_grouped");
   if (num_tensors < 0 || (num_tensors > 0 && !tensors)) return NVFP4_ERR_ARG;
   if (dtype != NVFP4_BF16 && dtype != NVFP4_F32) return NVFP4_ERR_DTYPE;
   for (int i = 0; i < num_tensors; ++i) {
@@ -971,6 +1048,7 @@ nvfp4_status nvfp4_calibrate_mse_grouped(int num_tensors, const nvfp4_tensor_ref
 
 nvfp4_status nvfp4_tensor_amax_grouped(int num_tensors, const nvfp4_tensor_ref* tensors, nvfp4_dtype dtype,
                                        float* amax, void* stream) {
+  NVFP4_ENTRY("nvfp4_tensor_amax_grouped");
   if (num_tensors < 0 || (num_tensors > 0 && (!tensors || !amax))) return NVFP4_ERR_ARG;
   if (dtype != NVFP4_BF16 && dtype != NVFP4_F32) return NVFP4_ERR_DTYPE;
   if ((uintptr_t)amax & 3u) return NVFP4_ERR_ALIGN;
@@ -1035,6 +1113,7 @@ nvfp4_status nvfp4_tensor_amax_grouped(int num_tensors, const nvfp4_tensor_ref* 
 }
 
 nvfp4_status nvfp4_global_scale_from_amax(const float* amax, int n, float* tensor_scale, void* stream) {
+  NVFP4_ENTRY("nvfp4_global_scale_from_amax");
   if (n < 0 || (n > 0 && (!amax || !tensor_scale))) return NVFP4_ERR_ARG;
   if (n == 0) return NVFP4_OK;
   global_scale_kernel<<<(n + 255) / 256, 256, 0, (cudaStream_t)stream>>>(amax, n, tensor_scale);
@@ -1044,6 +1123,7 @@ nvfp4_status nvfp4_global_scale_from_amax(const float* amax, int n, float* tenso
 
 nvfp4_status nvfp4_calibrate_mse(const void* x, nvfp4_dtype dtype, int64_t rows, int64_t cols, int64_t ld_x,
                                  const float* tensor_scale, uint8_t* block_scales, float* block_err, void* stream) {
+  NVFP4_ENTRY("nvfp4_calibrate_mse");
   nvfp4_tensor_ref r;
   r.x = x;
   r.rows = rows;
@@ -1059,6 +1139,7 @@ nvfp4_status nvfp4_calibrate_mse(const void* x, nvfp4_dtype dtype, int64_t rows,
 
 nvfp4_status nvfp4_fake_quant_grouped(int num_tensors, const nvfp4_tensor_ref* tensors, nvfp4_dtype dtype,
                                       nvfp4_scale_mode mode, void* workspace, size_t workspace_bytes, void* stream) {
+  NVFP4_ENTRY("nvfp4_fake_quant_grouped");
   return run_tensors<Out::Fake>(num_tensors, tensors, dtype, mode, NVFP4_SCALES_ROWMAJOR, workspace,
                                 workspace_bytes, (cudaStream_t)stream);
 }
@@ -1066,6 +1147,7 @@ nvfp4_status nvfp4_fake_quant_grouped(int num_tensors, const nvfp4_tensor_ref* t
 nvfp4_status nvfp4_dequantize(const uint8_t* codes, int64_t ld_codes, const uint8_t* block_scales,
                               nvfp4_scale_layout layout, const float* tensor_scale, int64_t rows, int64_t cols,
                               void* out, nvfp4_dtype out_dtype, int64_t ld_out, void* stream) {
+  NVFP4_ENTRY("nvfp4_dequantize");
   if (out_dtype != NVFP4_BF16 && out_dtype != NVFP4_F32) return NVFP4_ERR_DTYPE;
   if (rows < 0 || cols < 0 || cols % 16 != 0 || ld_codes < cols / 2 || ld_out < cols) return NVFP4_ERR_SHAPE;
   if (layout != NVFP4_SCALES_ROWMAJOR && layout != NVFP4_SCALES_MMA) return NVFP4_ERR_ARG;
@@ -1093,6 +1175,7 @@ nvfp4_status nvfp4_dequantize(const uint8_t* codes, int64_t ld_codes, const uint
 // 8 bytes, initialised here: the mismatch count, and one mismatch (or
 // all ones when there is none).
 nvfp4_status nvfp4_selftest_division(uint64_t* mismatches, uint64_t* first, void* stream) {
+  NVFP4_ENTRY("nvfp4_selftest_division");
   if (!mismatches || !first) return NVFP4_ERR_ARG;
   cudaStream_t s = (cudaStream_t)stream;
   if (cudaMemsetAsync(mismatches, 0, sizeof(uint64_t), s) != cudaSuccess) return NVFP4_ERR_CUDA;

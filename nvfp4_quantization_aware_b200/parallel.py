@@ -20,7 +20,9 @@ rows; the only data exchanged are scalars:
   travel to the rank that owns their expert and the expert outputs travel
   back, each way one all_to_all_single of the rows (plus one of the row
   counts); the backward pass runs the same two exchanges in reverse.  The
-  pages train with expert parallelism (EP 4 and 8).
+  pages train with expert parallelism (EP 4 and 8).  ExpertParallelMoE runs
+  the whole layer step: the exchanges here, the experts' FFNs on the device
+  (qad_moe_expert_forward / qad_moe_expert_backward).
 
 The device operations are passed in (`ops`), defaulting to this package's
 CUDA entry points; the collectives go through torch.distributed.  Beyond the
@@ -124,7 +126,13 @@ class EpPlan:
 def _exchange(out_rows: int, rows: torch.Tensor, out_splits, in_splits, group=None) -> torch.Tensor:
     out = rows.new_empty((out_rows,) + tuple(rows.shape[1:]))
     if _world(group) > 1:
-        dist.all_to_all_single(out, rows.contiguous(), list(out_splits), list(in_splits), group=group)
+        if rows.is_cuda and dist.get_backend(group) == "gloo":
+            # gloo moves host memory only: stage the rows through the host
+            host = torch.empty(out.shape, dtype=out.dtype)
+            dist.all_to_all_single(host, rows.contiguous().cpu(), list(out_splits), list(in_splits), group=group)
+            out.copy_(host)
+        else:
+            dist.all_to_all_single(out, rows.contiguous(), list(out_splits), list(in_splits), group=group)
     else:
         out.copy_(rows)
     return out
@@ -199,3 +207,72 @@ def ep_dispatch_backward(dx_recv: torch.Tensor, plan: EpPlan, group=None) -> tor
     for j in range(plan.topk):
         dx += per_slot[:, j].to(acc)
     return dx
+
+
+class ExpertParallelMoE:
+    """The QAD student's MoE layer step with expert parallelism over the ranks
+    of `group` (EP 4 / 8 on the pages): rank r owns experts [r E/W, (r+1) E/W).
+
+    forward: ep_dispatch sends each routed (token, slot) row to its expert's
+    owner; the owner runs its experts' FFNs on the received rows on the device
+    (qad_moe_expert_forward: grouped W4A4 with frozen scales, as in the
+    single-GPU step); ep_combine returns the rows and sums them with the
+    combine weights; the shared expert runs on each rank's own tokens (the
+    same device path with one expert).  backward: the combine-weighted output
+    gradients travel to the owners (ep_combine_backward), the owners run the
+    straight-through backward of their experts (qad_moe_expert_backward: the
+    rows' input gradients and their experts' weight gradients), the input
+    gradients return and are summed over the token's slots
+    (ep_dispatch_backward); the shared expert's weight gradient is summed over
+    the ranks (all-reduce), since every rank computed it on its own tokens.
+
+    local_weights / shared_weights: the qad_moe_weights tensors (as for
+    MoeLayerStep) of this rank's E/W experts and of the shared expert alone.
+    """
+
+    def __init__(self, hidden: int, ffn: int, experts: int, local_weights: dict, shared_weights: dict, group=None,
+                 device="cuda"):
+        from .binding import MoeExpertStep
+
+        self.group = group
+        self.experts = experts
+        self.hidden, self.ffn = hidden, ffn
+        world = _world(group)
+        if experts % world:
+            raise ValueError(f"{experts} experts do not split evenly over {world} ranks")
+        self.local = MoeExpertStep(hidden, ffn, experts // world, local_weights, device)
+        self.shared = MoeExpertStep(hidden, ffn, 1, shared_weights, device)
+        self._ctx = None
+
+    def forward(self, x: torch.Tensor, ids: torch.Tensor, combine: torch.Tensor) -> torch.Tensor:
+        """x [tokens, H] bf16 (this rank's tokens), ids / combine [tokens, topk]."""
+        recv_x, recv_e, plan = ep_dispatch(x, ids, self.experts, self.group)
+        y_recv = self.local.forward(recv_x, recv_e)
+        y_routed, y_slot = ep_combine(y_recv, plan, combine, self.group)
+        zero = torch.zeros(x.shape[0], dtype=torch.int32, device=x.device)
+        y_shared = self.shared.forward(x, zero)
+        self._ctx = (plan, combine, y_slot)
+        return (y_routed + y_shared.to(y_routed.dtype)).to(x.dtype)
+
+    def backward(self, dy: torch.Tensor):
+        """Returns (dx [tokens, H], (dw_gate, dw_up, dw_down) of this rank's
+        experts, (dw_gate, dw_up, dw_down) of the shared expert summed over the
+        ranks, d_combine [tokens, topk])."""
+        plan, combine, y_slot = self._ctx
+        dy_recv, d_combine = ep_combine_backward(dy, plan, combine, y_slot, self.group)
+        dx_recv, dwg, dwu, dwd = self.local.backward(dy_recv)
+        dx_routed = ep_dispatch_backward(dx_recv, plan, self.group)
+        dx_sh, sg, su, sd = self.shared.backward(dy)
+        dx = (dx_routed + dx_sh.to(dx_routed.dtype)).to(dy.dtype)
+        shared_dw = []
+        for t in (sg, su, sd):
+            acc = t.float()
+            if _world(self.group) > 1:
+                if acc.is_cuda and dist.get_backend(self.group) == "gloo":
+                    host = acc.cpu()
+                    dist.all_reduce(host, op=dist.ReduceOp.SUM, group=self.group)
+                    acc.copy_(host)
+                else:
+                    dist.all_reduce(acc, op=dist.ReduceOp.SUM, group=self.group)
+            shared_dw.append(acc.to(t.dtype))
+        return dx, (dwg, dwu, dwd), tuple(shared_dw), d_combine

@@ -81,3 +81,38 @@ def test_workspace_queries(lib):
     assert lib.nvfp4_quantize_workspace_size(100, 64, 0) >= 4
     assert lib.nvfp4_quantize_workspace_size(100, 64, 1) == 0
     assert lib.nvfp4_quantize_workspace_size(100, 64, 2) == 0
+
+
+def test_fault_injection_fails_the_nth_call_before_launch(lib):
+    """Armed with n = 2, the second outermost call returns NVFP4_ERR_CUDA (5)
+    without validating or launching; the calls around it are unaffected and
+    the arming is spent after one failure."""
+    p = ctypes.c_void_p(16)
+    bad_cols = lambda: lib.nvfp4_quantize(p, 0, 4, 40, 40, 0, p, p, 0, p, 20, p, 4096, None)
+    lib.nvfp4_fault_inject.argtypes = [ctypes.c_int64]
+    lib.nvfp4_fault_inject(2)
+    try:
+        assert bad_cols() == 2          # 1st: validated as usual (ERR_SHAPE)
+        assert bad_cols() == 5          # 2nd: injected ERR_CUDA before validation
+        assert bad_cols() == 2          # disarmed again
+        lib.nvfp4_fault_inject(1)
+        assert lib.nvfp4_dequantize(p, 16, p, 0, p, 4, 33, p, 0, 33, None) == 5  # any exported operation
+        assert lib.nvfp4_dequantize(p, 16, p, 0, p, 4, 33, p, 0, 33, None) == 2
+    finally:
+        lib.nvfp4_fault_inject(0)
+    assert bad_cols() == 2
+
+
+def test_fault_injection_from_the_environment():
+    """NVFP4QAD_FAIL_AT=n arms the injection when the library loads."""
+    code = ("import ctypes, nvfp4_quantization_aware_b200 as Q; L = Q.lib(); p = ctypes.c_void_p(16); "
+            "r = [L.nvfp4_quantize(p, 0, 4, 40, 40, 0, p, p, 0, p, 20, p, 4096, None) for _ in range(4)]; print(r)")
+    env = dict(os.environ, NVFP4QAD_FAIL_AT="3", PYTHONPATH=ROOT)
+    out = subprocess.run(["python", "-c", code], capture_output=True, text=True, env=env, check=True).stdout
+    assert out.strip() == "[2, 2, 5, 2]"
+
+
+def test_timeout_selftest_rejects_unbounded_limits(lib):
+    lib.nvfp4_selftest_timeout.argtypes = [ctypes.c_int64, ctypes.c_void_p]
+    assert lib.nvfp4_selftest_timeout(0, None) == 1
+    assert lib.nvfp4_selftest_timeout((1 << 32) + 1, None) == 1

@@ -64,7 +64,7 @@ def test_tiny_qad_linear():
 @pytest.mark.parametrize("M,N,K", [(1, 8, 64), (127, 100, 192), (129, 256, 320), (200, 300, 1024),
                                    (64, 520, 256), (256, 512, 576), (3, 1000, 2048), (5, 1002, 1024),
                                    (130, 4096, 4096), (1, 256, 8192),
-                                   # CTA-pair path: more 256 x 256 tiles than resident pairs, long K
+                                   # more tiles than resident CTAs (several per CTA), long K
                                    (2304, 2560, 576), (300, 520, 4096)])
 def test_ragged_shapes(M, N, K):
     x = S.activations(M, K, seed=M + K, device=DEV)
@@ -106,6 +106,21 @@ def test_integer_operands_exact():
 def test_w4a4_gemm_decode_shape():
     d = S.w4a4_gemm(128, seed=0, device=DEV)
     _run(d["x"], d["w"])
+
+
+@pytest.mark.parametrize("M", [1, 127, 128, 129, 256])
+def test_w4a4_gemm_small_m_split_k(M):
+    """Decode-sized batches against a 4096 x 4096 weight run the split-K
+    kernel (clusters of CTAs along K, partials added in rank order through
+    distributed shared memory); parity as for every other shape."""
+    d = S.w4a4_gemm(M, seed=M, device=DEV)
+    rows = None if M <= 129 else np.concatenate([[0, 127, 128, 255], np.arange(1, 255, 9)])
+    c1, _ = _run(d["x"], d["w"], rows=rows)
+    # deterministic: the fixed rank order of the partial sums gives the same bits every call
+    a = _gpu_operand(d["x"])
+    b = _gpu_operand(d["w"])
+    c2 = Q.nvfp4_gemm_w4a4(*a, *b)
+    assert torch.equal(c1.view(torch.int16), c2.view(torch.int16))
 
 
 def test_w4a4_gemm_prefill_shape_sampled():
