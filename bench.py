@@ -899,6 +899,15 @@ def run_profile_case(case: str):
         b = Q.nvfp4_quantize(w, Q.DYNAMIC, layout=Q.SCALES_MMA)
         for _ in range(5):
             Q.nvfp4_gemm_w4a4(*a, *b)
+    elif case == "gemm_small":
+        w = S.weights(4096, 4096, seed=1, device=dev)
+        x = S.channel_scaled_activations(128, 4096, seed=0, device=dev)
+        a = Q.nvfp4_quantize(x, Q.DYNAMIC, layout=Q.SCALES_MMA)
+        b = Q.nvfp4_quantize(w, Q.DYNAMIC, layout=Q.SCALES_MMA)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        for _ in range(5):
+            flush_l2(flush)
+            Q.nvfp4_gemm_w4a4(*a, *b)
     elif case == "moe":
         d, w, step = make_moe_step(Q, dev)
         for _ in range(3):
@@ -936,7 +945,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-secondary", action="store_true", help="skip the GEMM and KL measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["quant", "gemm", "kl", "kl_topk", "w4a16", "calibrate", "moe"], default=None,
+    ap.add_argument("--profile", choices=["quant", "gemm", "gemm_small", "kl", "kl_topk", "w4a16", "calibrate", "moe"],
+                    default=None,
                     help="run one small single-kernel case (for ncu captures) and exit")
     args = ap.parse_args()
     if args.profile:

@@ -417,242 +417,6 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
   }
 }
 
-// ------------------------------------------------------------------ CTA-pair kernel
-//
-// The single-CTA kernel above is bound by its operand feed: every 512-cycle
-// stage moves a 128-row A and a 256-row B tile through the SM's shared memory
-// (TMA writes, MMA reads).  Here a cluster of two CTAs on one TPC computes a
-// 256 x 256 output tile with tcgen05.mma.cta_group::2: each CTA stages its
-// own 128 rows of A and its own 128 of the tile's 256 rows of B, the pair's
-// tensor cores share the B halves, and each SM moves 32 KiB of operands per
-// 256-deep stage instead of 48 KiB for the same MMA work.  Block scales: each
-// CTA writes the scales of its A rows and of all 256 B rows into its own
-// tensor memory (the image the single-CTA 128 x 256 MMA reads).
-// Roles per CTA as in the single-CTA kernel (producer, MMA, 8 epilogue warps,
-// 4 scale writers); only rank 0 issues MMAs.  Barriers:
-//   full[s]     rank 0: both CTAs' A and B tiles of stage s landed (the TMA
-//               loads of both CTAs count their bytes on rank 0's barrier)
-//   sfl[s]      each CTA: its own stage-s block scales are in shared memory
-//   sf_full[s]  rank 0: both CTAs' scale writers finished stage s
-//   empty[s]    each CTA: the MMAs reading stage s completed (rank 0 commits
-//               to its own barrier and to its peer's)
-//   acc_full    each CTA: the tile's MMAs completed
-//   acc_empty   rank 0: both CTAs' epilogues drained the accumulator
-namespace pair {
-constexpr int BM = 256, BN = 256;       // output tile of the pair
-constexpr int HM = 128, HN = 128;       // A rows and B rows staged per CTA
-constexpr int BK = 256;                 // FP4 elements per stage (128 bytes per row)
-constexpr int KB = BK / 64;             // MMAs (K = 64) per stage
-constexpr int STAGES = 5;
-constexpr int A_BYTES = HM * BK / 2;    // 16 KiB
-constexpr int B_BYTES = HN * BK / 2;    // 16 KiB
-constexpr int SFA_BYTES = 512 * KB;     // one 128-row scale tile
-constexpr int SFB_BYTES = 512 * KB * 2; // both 128-row scale tiles of B
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-constexpr int TM_ACC = 0;                         // 128 lanes x 256 FP32 columns
-constexpr int TM_SFA = BN;                        // STAGES x 4 KB columns
-constexpr int TM_SFB = BN + STAGES * 4 * KB;      // STAGES x 8 KB columns
-constexpr int TM_COLS = 512;
-static_assert(TM_SFB + STAGES * 8 * KB <= TM_COLS, "tensor memory");
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-constexpr int EPI_WARPS = 8;
-constexpr int SF_WARPS = 4;
-constexpr int THREADS = 64 + 32 * (EPI_WARPS + SF_WARPS);
-// E2M1 x E2M1, UE4M3 scales, K-major A and B, N = 256, M = 256 (the pair)
-constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-}  // namespace pair
-
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::THREADS, 1)
-    gemm_w4a4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                          GemmParams p) {
-  using namespace pair;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw_addr = smem_u32(smem_raw);
-  // same offset in both CTAs: the MMA descriptors of rank 0 address the peer's
-  // operands at the offsets of its own
-  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-  uint8_t* sA = smem;
-  uint8_t* sB = sA + STAGES * A_BYTES;
-  uint8_t* sSFA = sB + STAGES * B_BYTES;
-  uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_BYTES);
-  uint64_t* sfl = full + STAGES;
-  uint64_t* empty = sfl + STAGES;
-  uint64_t* sf_full = empty + STAGES;
-  uint64_t* acc_full = sf_full + STAGES;
-  uint64_t* acc_empty = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
-  const int num_kt = (p.kchunks + KB - 1) / KB;
-  const int num_n = (p.N + BN - 1) / BN;
-  const int num_tiles = num_n * ((p.M + BM - 1) / BM);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&sfl[s], 1);
-      mbar_init(&empty[s], 1);
-      mbar_init(&sf_full[s], 2 * SF_WARPS);
-    }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 2 * EPI_WARPS);
-    *abort_flag = 0;
-    fence_mbar_init();
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(tmem_slot, TM_COLS);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  cluster_sync_all();  // both CTAs' barriers initialised and tensor memory allocated
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t full0 = cluster_addr(full, 0);           // rank 0's barriers
-  const uint32_t sf_full0 = cluster_addr(sf_full, 0);
-  const uint32_t acc_empty0 = cluster_addr(acc_empty, 0);
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer (both CTAs)
-    if (lane == 0) {
-      int it = 0;
-      for (int t = cid; t < num_tiles && !*abort_flag; t += ncl) {
-        const int mt = t / num_n;
-        const int m0 = mt * BM + (int)rank * HM;  // this CTA's A rows
-        const int n0 = (t - mt * num_n) * BN;
-        const bool has_a = m0 < p.M;              // rows past M: zero-filled codes, no scale tile
-        int nsfb = 0;
-        for (int j = 0; j < 2; ++j)
-          if (n0 / 128 + j < p.b_rowtiles) ++nsfb;
-        for (int kt = 0; kt < num_kt; ++kt, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!mbar_wait_bounded(&empty[s], ph ^ 1u)) { *abort_flag = 1; break; }
-          if (*abort_flag) break;
-          int nkc = p.kchunks - kt * KB;
-          if (nkc > KB) nkc = KB;
-          if (rank == 0) mbar_expect_tx(&full[s], 2u * (uint32_t)(A_BYTES + B_BYTES));
-          mbar_expect_tx(&sfl[s], (uint32_t)nkc * 512u * ((has_a ? 1u : 0u) + (uint32_t)nsfb));
-          tma_load_2d_pair(sA + s * A_BYTES, &tmA, kt * (BK / 2), m0, full0 + 8u * s);
-          tma_load_2d_pair(sB + s * B_BYTES, &tmB, kt * (BK / 2), n0 + (int)rank * HN, full0 + 8u * s);
-          const int64_t kc0 = (int64_t)kt * KB;
-          if (has_a)
-            bulk_g2s(sSFA + s * SFA_BYTES, p.a_sf + ((int64_t)(m0 / 128) * p.kchunks + kc0) * 512, (uint32_t)nkc * 512u,
-                     &sfl[s]);
-          for (int j = 0; j < nsfb; ++j)
-            bulk_g2s(sSFB + s * SFB_BYTES + j * 512 * KB, p.b_sf + ((int64_t)(n0 / 128 + j) * p.kchunks + kc0) * 512,
-                     (uint32_t)nkc * 512u, &sfl[s]);
-        }
-      }
-      // drain: every stage this CTA filled has been released by the MMAs, so
-      // no commit from rank 0 arrives here after the CTA has exited
-      for (int i = 0; i < STAGES && !*abort_flag; ++i, ++it)
-        if (!mbar_wait_bounded(&empty[it % STAGES], (((uint32_t)(it / STAGES)) & 1u) ^ 1u)) *abort_flag = 1;
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (rank 0)
-    if (rank == 0 && lane == 0) {
-      const uint32_t empty1 = cluster_addr(empty, 1);
-      const uint32_t acc_full1 = cluster_addr(acc_full, 1);
-      int it = 0, ti = 0;
-      for (int t = cid; t < num_tiles && !*abort_flag; t += ncl, ++ti) {
-        if (!mbar_wait_bounded(acc_empty, ((uint32_t)ti & 1u) ^ 1u)) { *abort_flag = 1; break; }
-        tc_fence_after();
-        for (int kt = 0; kt < num_kt; ++kt, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!mbar_wait_bounded(&full[s], ph) || !mbar_wait_bounded(&sf_full[s], ph)) {
-            *abort_flag = 1;
-            break;
-          }
-          if (*abort_flag) break;
-          tc_fence_after();
-          int nkc = p.kchunks - kt * KB;
-          if (nkc > KB) nkc = KB;
-          const uint32_t sfa_col = tmem + TM_SFA + s * 4 * KB;
-          const uint32_t sfb_col = tmem + TM_SFB + s * 8 * KB;
-          const uint32_t a_base = smem_u32(sA + s * A_BYTES);
-          const uint32_t b_base = smem_u32(sB + s * B_BYTES);
-          for (int kb = 0; kb < nkc; ++kb)
-            mma_fp4_block16_pair(tmem + TM_ACC, smem_desc(a_base + kb * 32, 16, 1024, 2),
-                                 smem_desc(b_base + kb * 32, 16, 1024, 2), IDESC, sfa_col + kb * 4, sfb_col + kb * 8,
-                                 (kt > 0 || kb > 0) ? 1u : 0u);
-          tc_commit_pair(smem_u32(&empty[s]));
-          tc_commit_pair(empty1 + 8u * s);
-        }
-        tc_commit_pair(smem_u32(acc_full));
-        tc_commit_pair(acc_full1);
-      }
-    }
-  } else if (warp >= 2 + EPI_WARPS) {
-    // ------------------------------------------------------------ scale writers (both CTAs)
-    // the single-CTA kernel's image: per 512-byte scale tile, 4 TMEM columns
-    // in which lane L holds bytes [16 (L % 32), +16) on every subpartition
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-    int it = 0;
-    bool ok = true;
-    for (int t = cid; t < num_tiles && ok && !*abort_flag; t += ncl) {
-      for (int kt = 0; kt < num_kt; ++kt, ++it) {
-        const int s = it % STAGES;
-        const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&sfl[s], ph));  // warp-uniform exit
-        if (!ok) break;
-        int nkc = p.kchunks - kt * KB;
-        if (nkc > KB) nkc = KB;
-        const uint8_t* a_src = sSFA + s * SFA_BYTES + lane * 16;
-        const uint8_t* b_src = sSFB + s * SFB_BYTES + lane * 16;
-        const uint32_t a_col = lane_base + TM_SFA + s * 4 * KB;
-        const uint32_t b_col = lane_base + TM_SFB + s * 8 * KB;
-        for (int kb = 0; kb < nkc; ++kb) {
-          tmem_st_32x32b_x4(a_col + kb * 4, *reinterpret_cast<const uint4*>(a_src + kb * 512));
-          tmem_st_32x32b_x4(b_col + kb * 8, *reinterpret_cast<const uint4*>(b_src + kb * 512));
-          tmem_st_32x32b_x4(b_col + kb * 8 + 4, *reinterpret_cast<const uint4*>(b_src + 512 * KB + kb * 512));
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(sf_full0 + 8u * s);
-      }
-    }
-    if (!ok) *abort_flag = 1;
-  } else {
-    // ------------------------------------------------------------ epilogue (both CTAs)
-    const int sub = warp & 3;
-    const int cbase = ((warp - 2) >> 2) * (BN / 2);
-    const float alpha = __fmul_rn(__ldg(p.a_ts), __ldg(p.b_ts));
-    int ti = 0;
-    for (int t = cid; t < num_tiles; t += ncl) {
-      const int mt = t / num_n;
-      const int m0 = mt * BM + (int)rank * HM;
-      const int n0 = (t - mt * num_n) * BN;
-      const bool ok = mbar_wait_bounded(acc_full, (uint32_t)(ti++) & 1u);
-      if (!ok) *abort_flag = 1;
-      if (!ok || *abort_flag) break;
-      tc_fence_after();
-      const uint32_t tbase = tmem + TM_ACC + ((uint32_t)(sub * 32) << 16) + cbase;
-      epilogue_rows<BN>(tbase, m0 + sub * 32 + lane, p.M, n0, cbase, p, alpha, [&] {
-        if (lane == 0) mbar_arrive_cluster(acc_empty0);
-      });
-    }
-  }
-  __syncwarp();
-  tc_fence_before();
-  // neither CTA leaves while its peer may still signal its barriers or its
-  // tensor memory is in use
-  cluster_sync_all();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc_pair(tmem, TM_COLS);
-  }
-}
-
 // ------------------------------------------------------------------ split-K kernel (few output tiles)
 //
 // When the output has few tiles -- a decode-sized batch: M of one or two
@@ -711,8 +475,10 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* sf_full = empty + STAGES;
   uint64_t* acc_full = sf_full + STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* recv_full = acc_full + 1;  // every CTA's partial rows have arrived (transaction bytes)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* stage = reinterpret_cast<float*>(smem);  // [BM][PART_STRIDE]: this CTA's partial, over the drained ring
 
   cg::cluster_group cluster = cg::this_cluster();
   const int split = (int)cluster.num_blocks();
@@ -735,8 +501,11 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
       mbar_init(&sf_full[s], SF_WARPS);
     }
     mbar_init(acc_full, 1);
+    mbar_init(recv_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // the S partial-row blocks this CTA will receive, (BM / S) rows each
+    mbar_expect_tx(recv_full, (uint32_t)(BM * PART_STRIDE * 4));
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
@@ -744,7 +513,11 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
     tmem_alloc(tmem_slot, TM_COLS);
     tmem_relinquish();
   }
+  // first half of a cluster barrier: the peers' receive barriers are
+  // initialised before any partial is sent (the wait comes just before)
+  cluster_arrive();
   griddep_wait();  // global memory only after this point (programmatic dependent launch)
+  const float alpha = __fmul_rn(__ldg(p.a_ts), __ldg(p.b_ts));
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -821,22 +594,15 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
       if (lane == 0) mbar_arrive(&sf_full[s]);
     }
   } else {
-    // ------------------------------------------------------------ partial tile -> its rows' owners
-    // Row `row` of the tile is reduced by CTA row / rows_per; this CTA's
-    // partial of the row goes straight from tensor memory into slot `rank`
-    // of that CTA's receive buffer (distributed shared memory stores, which
-    // do not wait for a reply).  The receive buffer is not part of the ring,
-    // so a peer still computing is not disturbed.
+    // ------------------------------------------------------------ partial tile -> shared memory
+    // After acc_full every MMA of this CTA has completed, so every TMA load
+    // has landed and been read and the ring can be overwritten.
     const int sub = warp & 3;
     const bool ok = mbar_wait_bounded(acc_full, 0u);
     if (!ok) *abort_flag = 1;
     if (ok) {
       tc_fence_after();
-      const int rows_per = BM / split;  // split divides BM (a power of two up to 8)
-      const int row = sub * 32 + lane;
-      const int owner = row / rows_per;
-      const uint32_t dst = cluster_addr(recv + ((size_t)rank * rows_per + (row - owner * rows_per)) * PART_STRIDE,
-                                        (uint32_t)owner);
+      float* prow = stage + (sub * 32 + lane) * PART_STRIDE;
       const uint32_t tbase = tmem + TM_ACC + ((uint32_t)(sub * 32) << 16);
 #pragma unroll
       for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -844,22 +610,30 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
         tmem_ld_32x32b_x32(tbase + c0, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 4u * (c0 + j)), "r"(r[j]),
-                       "r"(r[j + 1]), "r"(r[j + 2]), "r"(r[j + 3])
-                       : "memory");
+        for (int j = 0; j < 32; j += 4) st_shared_v4(prow + c0 + j, r[j], r[j + 1], r[j + 2], r[j + 3]);
       }
     }
+    fence_proxy_async_smem();  // the bulk copies below read these writes
   }
   __syncwarp();
   tc_fence_before();
-  cluster_sync_all();  // every partial row is in its owner's receive buffer
+  __syncthreads();
+  // ---- exchange: rows [q 128/S, (q+1) 128/S) of this CTA's partial go to slot
+  // `rank` of CTA q's receive buffer, one bulk shared-to-shared copy per CTA
+  const int rows_per = BM / split;  // split divides BM (a power of two up to 8)
+  cluster_wait();                   // every CTA's receive barrier is initialised
+  if (threadIdx.x == 0) {
+    const uint32_t bytes = (uint32_t)(rows_per * PART_STRIDE * 4);
+    for (int q = 0; q < split; ++q)
+      bulk_s2cluster(cluster_addr(recv + (size_t)rank * rows_per * PART_STRIDE, (uint32_t)q),
+                     stage + (size_t)q * rows_per * PART_STRIDE, bytes, cluster_addr(recv_full, (uint32_t)q));
+  }
   // ---- reduction of this CTA's rows [rank * rows_per, +rows_per): per row 32
   // groups of 4 columns, each the sum of the S partials in rank order 0..S-1
   {
-    const int rows_per = BM / split;
+    const bool arrived = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(recv_full, 0u));
+    if (!arrived) *abort_flag = 1;
     const int r0 = rank * rows_per;
-    const float alpha = __fmul_rn(__ldg(p.a_ts), __ldg(p.b_ts));
     const bool bad = *abort_flag != 0;
     for (int item = threadIdx.x; item < rows_per * (BN / 4); item += THREADS) {
       const int lrow = item / (BN / 4);
@@ -887,6 +661,9 @@ __global__ void __launch_bounds__(splitk::THREADS, 1)
       }
     }
   }
+  // every CTA has received all its rows, so every copy out of this CTA's
+  // shared memory has completed: now it may exit
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, TM_COLS);
@@ -961,37 +738,6 @@ static nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* b, const GemmPa
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = tiles < sms ? tiles : sms;  // persistent: one CTA per SM
   return launch_pdl(gemm_w4a4_kernel<BN>, grid, C::THREADS, C::SMEM_BYTES, 1, ta, tb, p, s);
-}
-
-// Dense problem on CTA pairs: one cluster of two CTAs per TPC, persistent
-// over the 256 x 256 tiles.  The number of pairs that can be resident at once
-// comes from the occupancy query (a TPC with a disabled SM holds no pair).
-static nvfp4_status launch_gemm_pair(const uint8_t* a, const uint8_t* b, const GemmParams& p, cudaStream_t s) {
-  CUtensorMap ta, tb;
-  if (!make_tmap(&ta, a, p.M, p.K / 2, pair::HM) || !make_tmap(&tb, b, p.N, p.K / 2, pair::HN)) return NVFP4_ERR_CUDA;
-  static int max_pairs = 0;
-  if (max_pairs == 0) {
-    if (cudaFuncSetAttribute(gemm_w4a4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pair::SMEM_BYTES) !=
-        cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    int sms = 148, dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
-    cfg.blockDim = dim3(pair::THREADS, 1, 1);
-    cfg.dynamicSmemBytes = pair::SMEM_BYTES;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_w4a4_pair_kernel, &cfg) != cudaSuccess || n < 1) {
-      (void)cudaGetLastError();  // a failed query is not a launch error
-      n = sms / 2;
-    }
-    max_pairs = n;
-  }
-  const int tiles = ((p.N + pair::BN - 1) / pair::BN) * ((p.M + pair::BM - 1) / pair::BM);
-  const int pairs = tiles < max_pairs ? tiles : max_pairs;
-  gemm_w4a4_pair_kernel<<<2 * pairs, pair::THREADS, pair::SMEM_BYTES, s>>>(ta, tb, p);
-  count_launches(1);
-  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
 // Split-K dispatch: the output has few 128 x 128 tiles.  S CTAs per tile
@@ -1079,10 +825,6 @@ nvfp4_status nvfp4_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_scales_mma
   p.groups = 0;
   p.a_off = nullptr;
   p.a_rows = nullptr;
-  // The CTA-pair kernel (launch_gemm_pair) is parity-green but measured 87 us
-  // against 80 us for the single-CTA kernel at 8192 x 4096 x 4096 (tensor pipe
-  // 40% active, one accumulator drained between tiles); it is not dispatched.
-  (void)launch_gemm_pair;
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int split = splitk_factor(p, sms);

@@ -256,7 +256,7 @@ NVFP4_DEV KlSliceGeom kl_stage_slice(const KlArgs& args, int64_t row, int64_t v0
   }
   // head and tail logits with plain loads, pad slots with the pad value; all
   // disjoint from the bulk-copied interior [off + head, off + tail0)
-  for (int j = threadIdx.x; j < off + head; j += blockDim.x) {  // pad, then head
+  for (int j = threadIdx.x; j < off + head; j += kKlThreads) {  // pad, then head
     const int i = j - off;
     if (i < 0) {
       E::store1(st + j, kPadLogit);
@@ -266,7 +266,7 @@ NVFP4_DEV KlSliceGeom kl_stage_slice(const KlArgs& args, int64_t row, int64_t v0
       ss[j] = gs[i];
     }
   }
-  for (int j = off + tail0 + threadIdx.x; j < cap; j += blockDim.x) {  // tail, then pad
+  for (int j = off + tail0 + threadIdx.x; j < cap; j += kKlThreads) {  // tail, then pad
     const int i = j - off;
     if (i < n) {
       st[j] = gt[i];
@@ -481,536 +481,6 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
       }
     }
   }
-}
-
-#ifndef KL_IMPL
-#define KL_IMPL 1
-#endif
-#ifndef KL_NT
-#define KL_NT 256
-#endif
-#ifndef KL_UNROLL
-#define KL_UNROLL 2
-#endif
-// bf16 form with the slice maxima taken first.  Pass 0: every thread takes
-// the max of the teacher and of the student logits over its own vectors
-// (packed bf16 max, two logits per instruction, exact).  Pass 1: the sums
-// relative to those maxima, with no rescaling and no branch, two vectors per
-// iteration with independent accumulators.  The thread statistics then merge
-// over the CTA and the cluster exactly as in kl_row_kernel.
-#ifndef KL_MINB
-#define KL_MINB 3
-#endif
-template <int NT>
-__global__ void __launch_bounds__(NT, KL_MINB) kl_row_bf16_kernel(KlArgs args) {
-  using T = __nv_bfloat16;
-  constexpr int V8 = 8;
-  constexpr int NW = NT / 32;
-  constexpr int U = KL_UNROLL;
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  __shared__ uint64_t bar;
-  __shared__ float warp_max[2][NW];
-  __shared__ float warp_sum[3][NW];
-  __shared__ KlStats peer_stats[kKlMaxCluster];
-  __shared__ int s_ok;
-
-  cg::cluster_group cluster = cg::this_cluster();
-  const int csize = (int)cluster.num_blocks();
-  const int crank = (int)cluster.block_rank();
-  const int64_t row = blockIdx.x / csize;
-  const int64_t v0 = (int64_t)crank * args.slice;
-  int64_t v1 = v0 + args.slice;
-  if (v1 > args.vocab) v1 = args.vocab;
-  const int n = v1 > v0 ? (int)(v1 - v0) : 0;
-
-  T* st = reinterpret_cast<T*>(smem_raw);
-  T* ss = st + args.slice + 2 * V8;
-  const KlSliceGeom geo = kl_stage_slice<T>(args, row, v0, n, st, ss, &bar, &s_ok);
-  const int off = geo.off, nslots = geo.nslots, nvec = geo.nvec;
-  const bool ok = s_ok != 0;
-  const uint4* vt = reinterpret_cast<const uint4*>(st);
-  const uint4* vs = reinterpret_cast<const uint4*>(ss);
-  const float a = args.a;  // log2(e) / T > 0
-
-  // ---- pass 0: this thread's maxima (pad slots hold kPadLogit, below every logit)
-  __nv_bfloat162 mt2 = __float2bfloat162_rn(kPadLogit), ms2 = mt2;
-  if (ok) {
-    for (int k = threadIdx.x; k < nvec; k += NT) {
-      const uint4 rt = vt[k], rs = vs[k];
-      mt2 = __hmax2(mt2, __hmax2(__hmax2(*reinterpret_cast<const __nv_bfloat162*>(&rt.x),
-                                         *reinterpret_cast<const __nv_bfloat162*>(&rt.y)),
-                                 __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&rt.z),
-                                         *reinterpret_cast<const __nv_bfloat162*>(&rt.w))));
-      ms2 = __hmax2(ms2, __hmax2(__hmax2(*reinterpret_cast<const __nv_bfloat162*>(&rs.x),
-                                         *reinterpret_cast<const __nv_bfloat162*>(&rs.y)),
-                                 __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&rs.z),
-                                         *reinterpret_cast<const __nv_bfloat162*>(&rs.w))));
-    }
-  }
-  KlStats my;
-  my.mt = fmaxf(__low2float(mt2), __high2float(mt2)) * a;  // exact: a power-of-two pad times a, or a logit times a
-  my.ms = fmaxf(__low2float(ms2), __high2float(ms2)) * a;
-  my.St = my.Ss = my.Y = 0.f;
-
-  // ---- pass 1: sums relative to the thread's maxima, d = z a - max w (one FMA)
-  if (ok) {
-    const f32x2 A = pair(a, a), NT2 = pair(-my.mt, -my.mt), NS2 = pair(-my.ms, -my.ms);
-    f32x2 St2[U], Ss2[U], Y2[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) St2[u] = Ss2[u] = Y2[u] = 0ull;
-    int k = threadIdx.x;
-    for (; k + (U - 1) * NT < nvec; k += U * NT) {
-      uint4 rt[U], rs[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        rt[u] = vt[k + u * NT];
-        rs[u] = vs[k + u * NT];
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const uint32_t wt[4] = {rt[u].x, rt[u].y, rt[u].z, rt[u].w}, ws[4] = {rs[u].x, rs[u].y, rs[u].z, rs[u].w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const f32x2 dt = fma2(bf16x2_pair(wt[j]), A, NT2), ds = fma2(bf16x2_pair(ws[j]), A, NS2);
-          const f32x2 et = ex2_pair(dt), es = ex2_pair(ds);
-          St2[u] = add2(St2[u], et);
-          Ss2[u] = add2(Ss2[u], es);
-          Y2[u] = fma2(et, sub2(dt, ds), Y2[u]);
-        }
-      }
-    }
-    for (; k < nvec; k += NT) {
-      const uint4 rt = vt[k], rs = vs[k];
-      const uint32_t wt[4] = {rt.x, rt.y, rt.z, rt.w}, ws[4] = {rs.x, rs.y, rs.z, rs.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const f32x2 dt = fma2(bf16x2_pair(wt[j]), A, NT2), ds = fma2(bf16x2_pair(ws[j]), A, NS2);
-        const f32x2 et = ex2_pair(dt), es = ex2_pair(ds);
-        St2[0] = add2(St2[0], et);
-        Ss2[0] = add2(Ss2[0], es);
-        Y2[0] = fma2(et, sub2(dt, ds), Y2[0]);
-      }
-    }
-#pragma unroll
-    for (int u = 1; u < U; ++u) {
-      St2[0] = add2(St2[0], St2[u]);
-      Ss2[0] = add2(Ss2[0], Ss2[u]);
-      Y2[0] = add2(Y2[0], Y2[u]);
-    }
-    my.St = lo_of(St2[0]) + hi_of(St2[0]);
-    my.Ss = lo_of(Ss2[0]) + hi_of(Ss2[0]);
-    my.Y = lo_of(Y2[0]) + hi_of(Y2[0]);
-  }
-  // ---- merge over the CTA (max butterfly, one rebase, sum butterfly), push to the cluster
-  {
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    float Mt = my.mt, Ms = my.ms;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      Mt = fmaxf(Mt, __shfl_xor_sync(0xFFFFFFFFu, Mt, o));
-      Ms = fmaxf(Ms, __shfl_xor_sync(0xFFFFFFFFu, Ms, o));
-    }
-    if (lane == 0) {
-      warp_max[0][wid] = Mt;
-      warp_max[1][wid] = Ms;
-    }
-    __syncthreads();
-    Mt = warp_max[0][0];
-    Ms = warp_max[1][0];
-#pragma unroll
-    for (int w = 1; w < NW; ++w) {
-      Mt = fmaxf(Mt, warp_max[0][w]);
-      Ms = fmaxf(Ms, warp_max[1][w]);
-    }
-    stats_rebase(my, Mt, Ms);
-    float sum_t = my.St, sum_s = my.Ss, sum_y = my.Y;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      sum_t += __shfl_xor_sync(0xFFFFFFFFu, sum_t, o);
-      sum_s += __shfl_xor_sync(0xFFFFFFFFu, sum_s, o);
-      sum_y += __shfl_xor_sync(0xFFFFFFFFu, sum_y, o);
-    }
-    if (lane == 0) {
-      warp_sum[0][wid] = sum_t;
-      warp_sum[1][wid] = sum_s;
-      warp_sum[2][wid] = sum_y;
-    }
-    __syncthreads();
-    if ((int)threadIdx.x < csize) {
-      KlStats c;
-      c.mt = Mt;
-      c.ms = Ms;
-      c.St = c.Ss = c.Y = 0.f;
-      for (int w = 0; w < NW; ++w) {
-        c.St += warp_sum[0][w];
-        c.Ss += warp_sum[1][w];
-        c.Y += warp_sum[2][w];
-      }
-      cluster.map_shared_rank(peer_stats, (int)threadIdx.x)[crank] = c;
-    }
-  }
-  cluster.sync();
-  __shared__ KlStats row_stats_sh;
-  if (threadIdx.x == 0) {
-    KlStats m = peer_stats[0];
-    for (int r = 1; r < csize; ++r) m = stats_merge(m, peer_stats[r]);
-    row_stats_sh = m;
-  }
-  __syncthreads();
-  const KlStats row_stats = row_stats_sh;
-  if (crank == 0 && threadIdx.x == 0) {
-    const float kl = 0.69314718055994531f * (row_stats.Y / row_stats.St + log2f(row_stats.Ss / row_stats.St));
-    args.row_kl[row] = ok ? kl : __int_as_float(0x7FC00000);
-  }
-  // ---- dLogits = gscale (p_s - p_t), g p = 2^(w - L + log2 g) for gscale > 0
-  if (args.dlogits != nullptr && ok) {
-    const float g = args.gscale;
-    const bool fold = g > 0.0f;
-    const float lg = fold ? __log2f(g) : 0.0f;
-    const float Lt = row_stats.mt + __log2f(row_stats.St) - lg, Ls = row_stats.ms + __log2f(row_stats.Ss) - lg;
-    const float gm = fold ? 1.0f : g;
-    T* gout = reinterpret_cast<T*>(args.dlogits) + row * args.ld_grad + v0 - off;
-    const bool vec_ok = (((uintptr_t)gout) & 15u) == 0;
-    const int kfirst = (off + V8 - 1) / V8;
-    const int klast = nslots / V8;
-    const f32x2 A = pair(a, a), NLt = pair(-Lt, -Lt), NLs = pair(-Ls, -Ls), G = pair(gm, gm);
-    for (int k0 = threadIdx.x; k0 < nvec; k0 += U * NT) {
-      uint4 rt[U], rs[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int k = k0 + u * NT;
-        if (k < nvec) {
-          rt[u] = vt[k];
-          rs[u] = vs[k];
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int k = k0 + u * NT;
-        if (k >= nvec) break;
-        const uint32_t wt[4] = {rt[u].x, rt[u].y, rt[u].z, rt[u].w}, ws[4] = {rs[u].x, rs[u].y, rs[u].z, rs[u].w};
-        uint32_t o2[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const f32x2 pt = ex2_pair(fma2(bf16x2_pair(wt[j]), A, NLt));
-          const f32x2 ps = ex2_pair(fma2(bf16x2_pair(ws[j]), A, NLs));
-          f32x2 d = sub2(ps, pt);
-          if (!fold) d = fma2(d, G, 0ull);
-          o2[j] = pack_bf16x2(lo_of(d), hi_of(d));
-        }
-        const int j0 = k * V8;
-        if (vec_ok && k >= kfirst && k < klast) {
-          st_stream_v4(gout + j0, make_uint4(o2[0], o2[1], o2[2], o2[3]));
-        } else {
-#pragma unroll
-          for (int j = 0; j < V8; ++j)
-            if (j0 + j >= off && j0 + j < nslots)
-              reinterpret_cast<unsigned short*>(gout)[j0 + j] = (unsigned short)(o2[j >> 1] >> (16 * (j & 1)));
-        }
-      }
-    }
-  }
-}
-
-// ------------------------------------------------------------------ persistent pipelined form (bf16)
-//
-// In the one-row-per-cluster kernels above a CTA loads its slice, then
-// computes, then exits, and the CTAs resident on an SM tend to move through
-// those phases together, so the SM alternates between waiting for HBM and
-// computing.  Here clusters are persistent: cluster c takes rows c, c + NC,
-// c + 2 NC, ... (NC clusters resident), and every CTA keeps its slices of
-// three rows in a ring of shared-memory slots.  While it computes on row i,
-// the TMA copies of rows i + 1 and i + 2 are in flight.  The cluster-wide
-// merge of a row's statistics does not stall the CTA either: iteration i
-// computes the statistics of row i and pushes them into every peer (stores to
-// distributed shared memory, then a remote arrive with release semantics on
-// the peer's exchange barrier for that slot), then waits for the exchange of
-// row i - 1, which completed while row i was being computed, and writes row
-// i - 1's gradient.  A slot is refilled (row i + 2) as soon as the gradient
-// of the row it held is written.  The arithmetic per row is that of
-// kl_row_bf16_kernel.
-struct KlPersistGeom {
-  int head, off, nint, nslots, nvec;
-};
-
-NVFP4_DEV KlPersistGeom kl_persist_geom(const KlArgs& args, int64_t row, int64_t v0, int n) {
-  constexpr int V8 = 8, ESZ = 2;
-  const __nv_bfloat16* gt = reinterpret_cast<const __nv_bfloat16*>(args.teacher) + row * args.ld + v0;
-  KlPersistGeom g;
-  g.head = (int)(((16u - ((uint32_t)(uintptr_t)gt & 15u)) & 15u) / ESZ);
-  if (g.head > n) g.head = n;
-  g.off = (V8 - g.head % V8) % V8;
-  g.nint = (n - g.head) / V8 * V8;
-  g.nslots = g.off + n;
-  g.nvec = (g.nslots + V8 - 1) / V8;
-  return g;
-}
-
-template <int NT>
-__global__ void __launch_bounds__(NT, 1) kl_row_persistent_kernel(KlArgs args) {
-  using T = __nv_bfloat16;
-  constexpr int V8 = 8;
-  constexpr int NW = NT / 32;
-  constexpr int SLOTS = 3;
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  __shared__ uint64_t load_bar[SLOTS];   // TMA copies of a slot landed
-  // exchange ring of XSLOTS rows: a CTA pushes row i only after every peer
-  // pushed row i - 2, i.e. after every peer finished iteration i - 3 and with
-  // it its read of row i - 4, the slot's previous row
-  constexpr int XSLOTS = 4;
-  __shared__ uint64_t xbar[XSLOTS];      // all CTAs' statistics of the slot's row arrived (transaction bytes)
-  __shared__ __align__(16) float xstats[XSLOTS][kKlMaxCluster][8];  // mt, ms, St, Ss, Y: written by every CTA
-  __shared__ float warp_max[2][NW];
-  __shared__ float warp_sum[3][NW];
-  __shared__ KlStats cta_stats, row_stats_sh;
-  __shared__ int s_bad;
-
-  cg::cluster_group cluster = cg::this_cluster();
-  const int csize = (int)cluster.num_blocks();
-  const int crank = (int)cluster.block_rank();
-  const int64_t ncl = (int64_t)gridDim.x / csize;
-  const int64_t cid = (int64_t)blockIdx.x / csize;
-  const int64_t nrows = cid < args.rows ? (args.rows - cid + ncl - 1) / ncl : 0;  // rows of this cluster
-  const int64_t v0 = (int64_t)crank * args.slice;
-  int64_t v1 = v0 + args.slice;
-  if (v1 > args.vocab) v1 = args.vocab;
-  const int n = v1 > v0 ? (int)(v1 - v0) : 0;
-  const int64_t slot_elems = args.slice + 2 * V8;  // per tensor
-  T* slot_base = reinterpret_cast<T*>(smem_raw);
-  auto slot_t = [&](int k) { return slot_base + (int64_t)k * 2 * slot_elems; };
-  auto slot_s = [&](int k) { return slot_base + (int64_t)k * 2 * slot_elems + slot_elems; };
-  auto row_of = [&](int64_t i) { return cid + i * ncl; };
-  const float a = args.a;
-
-  constexpr uint32_t kXBytes = 20;  // bytes of one CTA's statistics
-  if (threadIdx.x == 0) {
-    for (int k = 0; k < SLOTS; ++k) mbar_init(&load_bar[k], 1);
-    for (int k = 0; k < XSLOTS; ++k) mbar_init(&xbar[k], 1);
-    s_bad = 0;
-    fence_mbar_init();
-    // arm the exchange of the first rows: one arrival (ours) and the bytes of
-    // every CTA's statistics
-    for (int64_t i = 0; i < XSLOTS && i < nrows; ++i) mbar_expect_tx(&xbar[i], kXBytes * (uint32_t)csize);
-  }
-  // every CTA's barriers are initialised before any peer arrives on them
-  cluster.sync();
-
-  // thread 0: bulk copies of the 16-byte-aligned interior of row i's slice into slot i % 3
-  auto issue_load = [&](int64_t i) {
-    const int k = (int)(i % SLOTS);
-    const int64_t row = row_of(i);
-    const KlPersistGeom g = kl_persist_geom(args, row, v0, n);
-    if (g.nint > 0) {
-      const T* gt = reinterpret_cast<const T*>(args.teacher) + row * args.ld + v0;
-      const T* gs = reinterpret_cast<const T*>(args.student) + row * args.ld + v0;
-      mbar_expect_tx(&load_bar[k], (uint32_t)(2 * g.nint * 2));
-      bulk_g2s(slot_t(k) + g.off + g.head, gt + g.head, (uint32_t)(g.nint * 2), &load_bar[k]);
-      bulk_g2s(slot_s(k) + g.off + g.head, gs + g.head, (uint32_t)(g.nint * 2), &load_bar[k]);
-    } else {
-      mbar_arrive(&load_bar[k]);
-    }
-  };
-  if (threadIdx.x == 0)
-    for (int64_t i = 0; i < SLOTS && i < nrows; ++i) issue_load(i);
-
-  for (int64_t i = 0; i <= nrows; ++i) {
-    // ------------------------------------------------ statistics of row i
-    if (i < nrows) {
-      const int k = (int)(i % SLOTS);
-      const int64_t row = row_of(i);
-      const KlPersistGeom g = kl_persist_geom(args, row, v0, n);
-      T* st = slot_t(k);
-      T* ss = slot_s(k);
-      if (!mbar_wait_bounded(&load_bar[k], (uint32_t)((i / SLOTS) & 1))) s_bad = 1;
-      // head and tail by plain loads, pad slots with the pad value (disjoint
-      // from the copied interior [off + head, off + head + nint))
-      {
-        const T* gt = reinterpret_cast<const T*>(args.teacher) + row * args.ld + v0;
-        const T* gs = reinterpret_cast<const T*>(args.student) + row * args.ld + v0;
-        const int cap = g.nvec * V8;
-        const int tail0 = g.head + g.nint;
-        for (int j = threadIdx.x; j < g.off + g.head; j += NT) {
-          const int e = j - g.off;
-          st[j] = e < 0 ? __float2bfloat16_rn(kPadLogit) : gt[e];
-          ss[j] = e < 0 ? __float2bfloat16_rn(kPadLogit) : gs[e];
-        }
-        for (int j = g.off + tail0 + threadIdx.x; j < cap; j += NT) {
-          const int e = j - g.off;
-          st[j] = e < n ? gt[e] : __float2bfloat16_rn(kPadLogit);
-          ss[j] = e < n ? gs[e] : __float2bfloat16_rn(kPadLogit);
-        }
-      }
-      __syncthreads();
-      const uint4* vt = reinterpret_cast<const uint4*>(st);
-      const uint4* vs = reinterpret_cast<const uint4*>(ss);
-      __nv_bfloat162 mt2 = __float2bfloat162_rn(kPadLogit), ms2 = mt2;
-      for (int q = threadIdx.x; q < g.nvec; q += NT) {
-        const uint4 rt = vt[q], rs = vs[q];
-        mt2 = __hmax2(mt2, __hmax2(__hmax2(*reinterpret_cast<const __nv_bfloat162*>(&rt.x),
-                                           *reinterpret_cast<const __nv_bfloat162*>(&rt.y)),
-                                   __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&rt.z),
-                                           *reinterpret_cast<const __nv_bfloat162*>(&rt.w))));
-        ms2 = __hmax2(ms2, __hmax2(__hmax2(*reinterpret_cast<const __nv_bfloat162*>(&rs.x),
-                                           *reinterpret_cast<const __nv_bfloat162*>(&rs.y)),
-                                   __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&rs.z),
-                                           *reinterpret_cast<const __nv_bfloat162*>(&rs.w))));
-      }
-      KlStats my;
-      my.mt = fmaxf(__low2float(mt2), __high2float(mt2)) * a;
-      my.ms = fmaxf(__low2float(ms2), __high2float(ms2)) * a;
-      {
-        const f32x2 A = pair(a, a), NT2 = pair(-my.mt, -my.mt), NS2 = pair(-my.ms, -my.ms);
-        f32x2 St2 = 0ull, Ss2 = 0ull, Y2 = 0ull;
-        for (int q = threadIdx.x; q < g.nvec; q += NT) {
-          const uint4 rt = vt[q], rs = vs[q];
-          const uint32_t wt[4] = {rt.x, rt.y, rt.z, rt.w}, ws[4] = {rs.x, rs.y, rs.z, rs.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const f32x2 dt = fma2(bf16x2_pair(wt[j]), A, NT2), ds = fma2(bf16x2_pair(ws[j]), A, NS2);
-            const f32x2 et = ex2_pair(dt), es = ex2_pair(ds);
-            St2 = add2(St2, et);
-            Ss2 = add2(Ss2, es);
-            Y2 = fma2(et, sub2(dt, ds), Y2);
-          }
-        }
-        my.St = lo_of(St2) + hi_of(St2);
-        my.Ss = lo_of(Ss2) + hi_of(Ss2);
-        my.Y = lo_of(Y2) + hi_of(Y2);
-      }
-      // CTA merge: max butterfly, one rebase per thread, sum butterfly
-      const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-      float Mt = my.mt, Ms = my.ms;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        Mt = fmaxf(Mt, __shfl_xor_sync(0xFFFFFFFFu, Mt, o));
-        Ms = fmaxf(Ms, __shfl_xor_sync(0xFFFFFFFFu, Ms, o));
-      }
-      if (lane == 0) {
-        warp_max[0][wid] = Mt;
-        warp_max[1][wid] = Ms;
-      }
-      __syncthreads();
-      Mt = warp_max[0][0];
-      Ms = warp_max[1][0];
-#pragma unroll
-      for (int w = 1; w < NW; ++w) {
-        Mt = fmaxf(Mt, warp_max[0][w]);
-        Ms = fmaxf(Ms, warp_max[1][w]);
-      }
-      stats_rebase(my, Mt, Ms);
-      float sum_t = my.St, sum_s = my.Ss, sum_y = my.Y;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        sum_t += __shfl_xor_sync(0xFFFFFFFFu, sum_t, o);
-        sum_s += __shfl_xor_sync(0xFFFFFFFFu, sum_s, o);
-        sum_y += __shfl_xor_sync(0xFFFFFFFFu, sum_y, o);
-      }
-      if (lane == 0) {
-        warp_sum[0][wid] = sum_t;
-        warp_sum[1][wid] = sum_s;
-        warp_sum[2][wid] = sum_y;
-      }
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        KlStats c;
-        c.mt = Mt;
-        c.ms = Ms;
-        c.St = c.Ss = c.Y = 0.f;
-        for (int w = 0; w < NW; ++w) {
-          c.St += warp_sum[0][w];
-          c.Ss += warp_sum[1][w];
-          c.Y += warp_sum[2][w];
-        }
-        cta_stats = c;
-      }
-      __syncthreads();
-      // push to every CTA of the cluster (this one included): asynchronous
-      // stores that complete their bytes on the receiver's exchange barrier
-      if ((int)threadIdx.x < csize) {
-        const KlStats c = cta_stats;
-        const int x = (int)(i % XSLOTS);
-        const uint32_t dst = cluster_addr(&xstats[x][crank][0], (uint32_t)threadIdx.x);
-        const uint32_t bar = cluster_addr(&xbar[x], (uint32_t)threadIdx.x);
-        st_async_v4(dst, __float_as_uint(c.mt), __float_as_uint(c.ms), __float_as_uint(c.St), __float_as_uint(c.Ss), bar);
-        st_async_b32(dst + 16, __float_as_uint(c.Y), bar);
-      }
-    }
-    // ------------------------------------------------ gradient of row i - 1
-    if (i >= 1) {
-      const int64_t j = i - 1;
-      const int k = (int)(j % SLOTS);
-      const int64_t row = row_of(j);
-      const KlPersistGeom g = kl_persist_geom(args, row, v0, n);
-      if (threadIdx.x == 0) {
-        const int x = (int)(j % XSLOTS);
-        if (!mbar_wait_bounded(&xbar[x], (uint32_t)((j / XSLOTS) & 1))) s_bad = 1;
-        auto peer = [&](int r) {
-          KlStats q;
-          q.mt = xstats[x][r][0];
-          q.ms = xstats[x][r][1];
-          q.St = xstats[x][r][2];
-          q.Ss = xstats[x][r][3];
-          q.Y = xstats[x][r][4];
-          return q;
-        };
-        KlStats m = peer(0);
-        for (int r = 1; r < csize; ++r) m = stats_merge(m, peer(r));
-        // the slot's statistics are read: arm its barrier for row j + XSLOTS
-        if (j + XSLOTS < nrows) mbar_expect_tx(&xbar[x], kXBytes * (uint32_t)csize);
-        row_stats_sh = m;
-        if (crank == 0) {
-          const float kl = 0.69314718055994531f * (m.Y / m.St + log2f(m.Ss / m.St));
-          args.row_kl[row] = s_bad ? __int_as_float(0x7FC00000) : kl;
-        }
-      }
-      __syncthreads();
-      const KlStats rs = row_stats_sh;
-      if (args.dlogits != nullptr) {
-        const uint4* vt = reinterpret_cast<const uint4*>(slot_t(k));
-        const uint4* vs = reinterpret_cast<const uint4*>(slot_s(k));
-        const float gsc = args.gscale;
-        const bool fold = gsc > 0.0f;
-        const float lg = fold ? __log2f(gsc) : 0.0f;
-        const float Lt = rs.mt + __log2f(rs.St) - lg, Ls = rs.ms + __log2f(rs.Ss) - lg;
-        const float gm = fold ? 1.0f : gsc;
-        T* gout = reinterpret_cast<T*>(args.dlogits) + row * args.ld_grad + v0 - g.off;
-        const bool vec_ok = (((uintptr_t)gout) & 15u) == 0;
-        const int kfirst = (g.off + V8 - 1) / V8;
-        const int klast = g.nslots / V8;
-        const f32x2 A = pair(a, a), NLt = pair(-Lt, -Lt), NLs = pair(-Ls, -Ls), G = pair(gm, gm);
-        for (int q = threadIdx.x; q < g.nvec; q += NT) {
-          const uint4 rt = vt[q], rsv = vs[q];
-          const uint32_t wt[4] = {rt.x, rt.y, rt.z, rt.w}, ws[4] = {rsv.x, rsv.y, rsv.z, rsv.w};
-          uint32_t o2[4];
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            const f32x2 pt = ex2_pair(fma2(bf16x2_pair(wt[jj]), A, NLt));
-            const f32x2 ps = ex2_pair(fma2(bf16x2_pair(ws[jj]), A, NLs));
-            f32x2 d = sub2(ps, pt);
-            if (!fold) d = fma2(d, G, 0ull);
-            o2[jj] = pack_bf16x2(lo_of(d), hi_of(d));
-          }
-          const int j0 = q * V8;
-          if (vec_ok && q >= kfirst && q < klast) {
-            st_stream_v4(gout + j0, make_uint4(o2[0], o2[1], o2[2], o2[3]));
-          } else {
-#pragma unroll
-            for (int e = 0; e < V8; ++e)
-              if (j0 + e >= g.off && j0 + e < g.nslots)
-                reinterpret_cast<unsigned short*>(gout)[j0 + e] = (unsigned short)(o2[e >> 1] >> (16 * (e & 1)));
-          }
-        }
-      }
-      // every read of slot k is done: refill it with row j + 3
-      __syncthreads();
-      if (threadIdx.x == 0 && j + SLOTS < nrows) {
-        fence_proxy_async_smem();
-        issue_load(j + SLOTS);
-      }
-    }
-  }
-  // no CTA leaves while a peer may still push into its shared memory
-  cluster.sync();
 }
 
 // ------------------------------------------------------------------ top-k KL
@@ -1416,59 +886,13 @@ static bool kl_plan(int64_t vocab, int esz, KlPlan& p) {
   return false;
 }
 
-#ifndef KL_PNT
-#define KL_PNT 1024
-#endif
-// Persistent pipelined form (bf16, three slots of the plan's slice in shared memory).
-static bool launch_kl_persistent(const KlArgs& a, const KlPlan& p, cudaStream_t s, cudaError_t* err) {
-  const size_t smem = 3 * (size_t)(p.slice + 16) * 2 * 2;
-  if (smem > 200 * 1024) return false;
-  auto fn = kl_row_persistent_kernel<KL_PNT>;
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) {
-    *err = e;
-    return true;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(KL_PNT);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = p.cluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int sms = 148, dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cfg.gridDim = dim3((unsigned)((sms / p.cluster) * p.cluster));
-  int ncl = 0;
-  if (cudaOccupancyMaxActiveClusters(&ncl, fn, &cfg) != cudaSuccess || ncl < 1) {
-    (void)cudaGetLastError();  // a failed query is not a launch error
-    ncl = sms / p.cluster;
-  }
-  if ((int64_t)ncl > a.rows) ncl = (int)a.rows;
-  cfg.gridDim = dim3((unsigned)(ncl * p.cluster));
-  *err = cudaLaunchKernelEx(&cfg, fn, a);
-  return true;
-}
-
 template <typename T>
 static cudaError_t launch_kl(const KlArgs& a, const KlPlan& p, cudaStream_t s) {
-#if KL_IMPL == 3
-  if (sizeof(T) == 2) {
-    cudaError_t e = cudaSuccess;
-    if (launch_kl_persistent(a, p, s, &e)) return e;
-  }
-#endif
-  const bool v2 = KL_IMPL == 2 && sizeof(T) == 2;
-  const void* fn = v2 ? (const void*)kl_row_bf16_kernel<KL_NT> : (const void*)kl_row_kernel<T>;
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+  cudaError_t e = cudaFuncSetAttribute(kl_row_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(a.rows * p.cluster));
-  cfg.blockDim = dim3(v2 ? KL_NT : kKlThreads);
+  cfg.blockDim = dim3(kKlThreads);
   cfg.dynamicSmemBytes = p.smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -1478,7 +902,6 @@ static cudaError_t launch_kl(const KlArgs& a, const KlPlan& p, cudaStream_t s) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (v2) return cudaLaunchKernelEx(&cfg, kl_row_bf16_kernel<KL_NT>, a);
   return cudaLaunchKernelEx(&cfg, kl_row_kernel<T>, a);
 }
 

@@ -1,8 +1,8 @@
 // ptx.cuh -- thin wrappers over the sm_100a PTX used by the TMA / tcgen05
 // kernels: mbarriers (all waits bounded), TMA tensor and bulk copies (no
-// cluster multicast anywhere), tcgen05 TMEM allocation, block-scaled MMA,
-// shared->tensor-memory copies and tensor-memory loads, and the CTA-pair
-// (tcgen05 .cta_group::2) forms used by two-SM MMA kernels.
+// cluster multicast anywhere), tcgen05 TMEM allocation, block-scaled and BF16
+// MMA, tensor-memory loads and stores, and cluster (distributed shared
+// memory) addressing and barriers.
 #pragma once
 
 #include "common.cuh"
@@ -204,12 +204,6 @@ NVFP4_DEV void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint3
       : "memory");
 }
 
-// Copy 32 rows x 16 bytes of shared memory (described by `sdesc`) into
-// tensor memory at `taddr`, replicated into all four 32-lane subpartitions.
-NVFP4_DEV void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
 // Load 32 consecutive 32-bit columns of this warp's 32 lanes.
 NVFP4_DEV void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -249,19 +243,7 @@ NVFP4_DEV void tmem_st_32x32b_x4(uint32_t taddr, uint4 v) {
 // Wait until this thread's tcgen05.st have completed.
 NVFP4_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// ------------------------------------------------------------------ CTA pairs
-//
-// A cluster of two CTAs (ranks 0 and 1, one TPC) whose tensor cores execute
-// one M = 256 MMA together (tcgen05 .cta_group::2): rank 0 issues the MMAs,
-// each CTA holds its own operand rows at the same shared-memory offsets and
-// its own rows of the accumulator in its tensor memory.  Every tcgen05
-// allocation, MMA and commit of such a kernel uses .cta_group::2.
-
-NVFP4_DEV uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
+// ------------------------------------------------------------------ clusters
 
 // Shared::cluster address of the object at `p` in CTA `rank` of this cluster.
 NVFP4_DEV uint32_t cluster_addr(const void* p, uint32_t rank) {
@@ -270,120 +252,24 @@ NVFP4_DEV uint32_t cluster_addr(const void* p, uint32_t rank) {
   return r;
 }
 
-// Every thread of both CTAs (may be called from diverged warps).
+// Every thread of every CTA of the cluster (may be called from diverged warps):
+// the writes of each before the barrier are visible to all after it.
 NVFP4_DEV void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
 
-// Barriers of a pair kernel are waited on and arrived at with the default
-// (CTA-scope) semantics: what they order is tcgen05 work made complete by
-// tcgen05.wait / commit and the tcgen05 thread-sync fences, and TMA bytes
-// counted by complete_tx, not plain memory traffic.  Cluster-scope acquire /
-// release forms put a memory fence on the MMA thread's path every stage.
+// The two halves of cluster_sync_all, for work in between.
+NVFP4_DEV void cluster_arrive() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
+NVFP4_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
 
-// Arrive on a barrier given by its shared::cluster address, releasing this
-// thread's earlier memory operations (e.g. distributed shared memory stores
-// into the barrier owner's CTA) at cluster scope.
-NVFP4_DEV void mbar_arrive_release_cluster(uint32_t bar_cluster) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
-}
-
-// Bounded wait on a barrier of this CTA with cluster-scope acquire (what the
-// arrivals released becomes visible).  On expiry it sets the device error word
-// and returns false.
-NVFP4_DEV bool mbar_wait_acquire_cluster(uint64_t* bar, uint32_t parity) {
-  const long long t0 = clock64();
-  for (;;) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    if (ok) return true;
-    if (clock64() - t0 > kWaitLimitCycles) {
-      report_error(kErrWaitTimeout);
-      return false;
-    }
-  }
-}
-
-// Asynchronous stores into another CTA's shared memory (shared::cluster
-// addresses) whose bytes complete a transaction on that CTA's mbarrier: the
-// receiver's phase completes only once the data is there, with no fence on
-// the sender's side.
-NVFP4_DEV void st_async_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t bar_cluster) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
-               "r"(a), "r"(b), "r"(c), "r"(d), "r"(bar_cluster)
+// Bulk copy from this CTA's shared memory into a CTA of the cluster
+// (dst and bar are shared::cluster addresses, bar in the destination CTA);
+// the bytes complete a transaction on that barrier.  Both addresses 16-byte
+// aligned, size a multiple of 16.
+NVFP4_DEV void bulk_s2cluster(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "r"(smem_u32(src)), "r"(bytes), "r"(bar)
                : "memory");
-}
-
-NVFP4_DEV void st_async_b32(uint32_t addr, uint32_t v, uint32_t bar_cluster) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(addr), "r"(v),
-               "r"(bar_cluster)
-               : "memory");
-}
-
-// Arrive on a barrier given by its shared::cluster address (either CTA).
-NVFP4_DEV void mbar_arrive_cluster(uint32_t bar_cluster) {
-  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
-}
-
-// 2-D tiled tensor load into this CTA's shared memory whose completion is
-// counted on a barrier of either CTA of the pair (no multicast).
-NVFP4_DEV void tma_load_2d_pair(void* dst, const void* tmap, int32_t x, int32_t y, uint32_t bar_cluster) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-      "[%4];" ::"r"(smem_u32(dst)),
-      "l"(tmap), "r"(x), "r"(y), "r"(bar_cluster)
-      : "memory");
-}
-
-// One warp of each CTA of the pair, same warp index and same `dst_smem` offset.
-NVFP4_DEV void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
-               "r"(ncols)
-               : "memory");
-}
-
-NVFP4_DEV void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-
-NVFP4_DEV void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-// Arrive on the barrier at shared::cluster address `bar_cluster` (this CTA's
-// or the peer's) once the pair MMAs issued so far by this thread completed.
-NVFP4_DEV void tc_commit_pair(uint32_t bar_cluster) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cluster)
-               : "memory");
-}
-
-// Pair form of mma_fp4_block16: M = 256 split as 128 rows per CTA; B's N
-// columns split as N/2 rows of B per CTA; each CTA's tensor memory holds the
-// scales of its own A rows and of all N rows of B.
-NVFP4_DEV void mma_fp4_block16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                    uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-      : "memory");
-}
-
-// Pair form of mma_bf16 (kind::f16, M = 256).
-NVFP4_DEV void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
 }
 
 }  // namespace nvfp4
