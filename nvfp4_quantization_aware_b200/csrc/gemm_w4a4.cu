@@ -740,13 +740,15 @@ static nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* b, const GemmPa
   return launch_pdl(gemm_w4a4_kernel<BN>, grid, C::THREADS, C::SMEM_BYTES, 1, ta, tb, p, s);
 }
 
-// Split-K dispatch: the output has few 128 x 128 tiles.  S CTAs per tile
-// (one cluster), S = the SMs per tile rounded down, at most 8 and at most the
-// K stages; S = 1 means the split does not pay and the persistent kernel runs.
+// Split-K dispatch: the output has few 128 x 128 tiles and K is long.  S CTAs
+// per tile (one cluster), S = the SMs per tile rounded down to a power of two,
+// at most 8 and at most the K stages; S = 1 means the split does not pay and
+// the persistent kernel runs.
 static int splitk_factor(const GemmParams& p, int sms) {
   const int tiles = ((p.M + splitk::BM - 1) / splitk::BM) * ((p.N + splitk::BN - 1) / splitk::BN);
   const int num_kt = (p.kchunks + splitk::KB - 1) / splitk::KB;
   if (tiles * 2 > sms) return 1;  // the persistent kernel fills the GPU at least as well
+  if (num_kt < 8) return 1;       // short K (< 2048): the exchange costs more than the split saves
   int sk = sms / tiles;
   if (sk > splitk::MAX_SPLIT) sk = splitk::MAX_SPLIT;
   if (sk > num_kt) sk = num_kt;

@@ -266,7 +266,7 @@ class ExpertParallelMoE:
         dx = (dx_routed + dx_sh.to(dx_routed.dtype)).to(dy.dtype)
         shared_dw = []
         for t in (sg, su, sd):
-            acc = t.float()
+            acc = t.to(torch.promote_types(t.dtype, torch.float32))  # summed in at least fp32
             if _world(self.group) > 1:
                 if acc.is_cuda and dist.get_backend(self.group) == "gloo":
                     host = acc.cpu()

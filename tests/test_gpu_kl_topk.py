@@ -56,12 +56,13 @@ def test_topk_vocab_sizes(V, k, dtype):
     _check(t, s, k)
 
 
-@pytest.mark.parametrize("V,k", [(40000, 3000), (1003, 500), (131072, 4096)])
-def test_topk_ties_split_across_the_cluster(V, k):
-    # integer-valued logits: large groups of equal teacher logits, the k-th
-    # falls inside one, whose members span several CTAs of the row's cluster
-    g = torch.Generator().manual_seed(V)
-    t = torch.randint(-3, 4, (4, V), generator=g).to(torch.bfloat16)
+@pytest.mark.parametrize("V,k,span", [(40000, 3000, 3), (1003, 500, 3), (131072, 4096, 3), (131072, 4096, 60)])
+def test_topk_ties_split_across_the_cluster(V, k, span):
+    # integer-valued logits in [-span, span]: groups of equal teacher logits,
+    # the k-th falls inside one, whose members span several CTAs of the row's
+    # cluster (a few hundred ties per CTA with span 60, thousands with 3)
+    g = torch.Generator().manual_seed(V + span)
+    t = torch.randint(-span, span + 1, (4, V), generator=g).to(torch.bfloat16)
     s = (t.float() + torch.randn(4, V, generator=g)).to(torch.bfloat16)
     _check(t.to(DEV), s.to(DEV), k)
 
