@@ -491,7 +491,7 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
 // broken by the smaller vocabulary index; the gradient is zero outside S.
 // Same cluster-per-row layout as kl_row_kernel.  S is found by a radix
 // select over order-preserving integer keys of the teacher logits held in
-// shared memory: one 8-bit digit per pass (2 passes for bf16, 4 for f32),
+// shared memory: one digit per pass (9 + 7 bits for bf16, 4 x 8 for f32),
 // each pass a CTA histogram (shared-memory atomics) summed over the
 // cluster through distributed shared memory; that yields the k-th key tau
 // and how many keys equal to tau belong to S.  When not all of them do, a
@@ -524,20 +524,76 @@ struct KlKey<float> {
   NVFP4_DEV static uint32_t key(uint32_t w, int) { return (w & 0x80000000u) ? ~w : (w | 0x80000000u); }
 };
 
+// bf16 keys are selected in two digits of 9 and 7 bits: the first digit is
+// the sign and exponent, so its bucket at the k-th key holds one binade; the
+// keys in that bucket (the candidates) are collected once (up to
+// kTopkCand per CTA, else the second digit scans the whole slice), and the
+// second digit's histogram and the ranking of the ties (keys equal to the
+// k-th key; up to kTopkTies per CTA among the candidates, else a scan of
+// the whole slice) read only them.  f32 keys take four 8-bit digits over the
+// whole slice.
+constexpr int kTopkCand = 4096;
+constexpr int kTopkTies = 512;
+
+// The digit whose bucket holds the remaining-th largest key of a histogram
+// of `bins` counts (cluster totals in hist): an inclusive scan of the
+// bucket counts from the largest digit down over the CTA's threads
+// (kKlThreads, each owning bins / kKlThreads or one bucket).  Every thread
+// returns (digit, keys to take from its bucket, keys in its bucket).
+NVFP4_DEV void topk_find_digit(const unsigned* hist, int bins, unsigned remaining, unsigned* warp_tot,
+                               unsigned* s_digit, unsigned* s_remaining, unsigned* s_count) {
+  const int t = (int)threadIdx.x, lane = t & 31, wid = t >> 5;
+  const int per = bins > kKlThreads ? bins / kKlThreads : 1;
+  const int b_hi = bins - 1 - t * per;  // this thread's buckets: b_hi, b_hi - 1, ..., b_hi - per + 1
+  unsigned mine = 0u;
+  if (b_hi >= 0)
+    for (int i = 0; i < per; ++i) mine += hist[b_hi - i];
+  unsigned x = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[wid] = x;
+  __syncthreads();
+  unsigned before = x - mine;
+  for (int w = 0; w < wid; ++w) before += warp_tot[w];
+  if (b_hi >= 0 && before < remaining && remaining <= before + mine) {
+    unsigned cum = before;
+    for (int i = 0; i < per; ++i) {
+      const int b = b_hi - i;
+      if (cum + hist[b] >= remaining) {
+        *s_digit = (unsigned)b;
+        *s_remaining = remaining - cum;
+        *s_count = hist[b];
+        break;
+      }
+      cum += hist[b];
+    }
+  }
+  __syncthreads();
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
   using E = KlElem<T>;
   using Kf = KlKey<T>;
   constexpr int V8 = E::kVec;
-  constexpr int PASSES = Kf::kBits / 8;
+  constexpr bool BF = sizeof(T) == 2;
+  constexpr int PASSES = BF ? 2 : 4;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ uint64_t bar;
   __shared__ int s_ok;
-  __shared__ unsigned hist[256];
-  __shared__ unsigned recv[2][kKlMaxCluster][256];  // written by every CTA of the cluster
+  __shared__ unsigned hist[512];
+  // cluster exchange of the histograms: one buffer per pass parity (f32) or
+  // per digit (bf16), written by every CTA of the cluster; the even passes'
+  // buffer (512 counts per CTA) lies over the tie prefixes, selection mask
+  // and candidate list, none of which is in use before the second digit
+  __shared__ unsigned recv_b[kKlMaxCluster][256];
   __shared__ unsigned recv_ties[kKlMaxCluster];
   __shared__ unsigned warp_sum[kKlWarps];
-  __shared__ unsigned s_digit, s_remaining, s_count;
+  __shared__ unsigned s_digit, s_remaining, s_count, s_ncand, s_ntie;
+  __shared__ int s_thr;
   __shared__ KlStats warp_stats[kKlWarps];
   __shared__ KlStats peer_stats[kKlMaxCluster];
 
@@ -556,6 +612,14 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
   const int nvec_max = (int)((args.slice + 2 * V8) / V8);
   unsigned* vec_prefix = reinterpret_cast<unsigned*>(ss + args.slice + 2 * V8);
   uint8_t* sel_mask = reinterpret_cast<uint8_t*>(vec_prefix + nvec_max);
+  uint16_t* cand = reinterpret_cast<uint16_t*>(sel_mask + (nvec_max + 3) / 4 * 4);  // kTopkCand slot indices
+  int* ties = reinterpret_cast<int*>(cand + kTopkCand);                            // kTopkTies slot indices
+  unsigned* recv_a = vec_prefix;  // [csize][512]
+  const uint16_t* t16 = reinterpret_cast<const uint16_t*>(st);
+  auto key16 = [&](int j) {  // order-preserving key of the bf16 teacher logit in slot j
+    const uint32_t u = t16[j];
+    return (u & 0x8000u) ? (~u & 0xFFFFu) : (u | 0x8000u);
+  };
   const KlSliceGeom geo = kl_stage_slice<T>(args, row, v0, n, st, ss, &bar, &s_ok);
   const int off = geo.off, nslots = geo.nslots, nvec = geo.nvec;
   const int kfirst = (off + V8 - 1) / V8;  // vectors [kfirst, klast) hold no pad slot
@@ -567,22 +631,71 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
   // ---- radix select of the k-th largest key over the row
   const uint32_t kk = (uint32_t)(args.topk < args.vocab ? args.topk : args.vocab);
   uint32_t prefix = 0, remaining = kk, count = 0;
+  bool use_cand = false;  // bf16: the second digit and the ties read the candidate list (CTA-uniform)
   for (int p = 0; p < PASSES; ++p) {
-    const int shift = Kf::kBits - 8 * (p + 1);  // digit position
-    hist[threadIdx.x] = 0u;
+    // digit p: bf16 bits [15:7] then [6:0]; f32 8 bits at a time from the top
+    const int dbits = BF ? (p == 0 ? 9 : 7) : 8;
+    const int shift = BF ? (p == 0 ? 7 : 0) : Kf::kBits - 8 * (p + 1);
+    const int bins = 1 << dbits;
+    for (int b = (int)threadIdx.x; b < bins; b += kKlThreads) hist[b] = 0u;
+    if constexpr (BF) {
+      if (p == 1) {
+        // the candidates: slots whose key's first digit is `prefix`, appended
+        // per warp (a count per lane, an inclusive scan, one atomic per round)
+        if (threadIdx.x == 0) s_ncand = 0u;
+        __syncthreads();
+        if (ok) {
+          for (int kb = wid * 32; kb < nvec; kb += kKlThreads) {  // warp-uniform trip count
+            const int k = kb + lane;
+            unsigned m = 0u;  // bit e: element e of vector k is a candidate
+            if (k < nvec) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const uint32_t k2 = bf16x2_keys(wt[k * 4 + q]);
+                const int j0 = k * V8 + 2 * q;
+                if (j0 >= off && j0 < nslots && ((k2 & 0xFFFFu) >> 7) == prefix) m |= 1u << (2 * q);
+                if (j0 + 1 >= off && j0 + 1 < nslots && ((k2 >> 16) >> 7) == prefix) m |= 2u << (2 * q);
+              }
+            }
+            const unsigned c = (unsigned)__popc(m);
+            unsigned x = c;  // inclusive scan over the lanes
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const unsigned y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+              if (lane >= o) x += y;
+            }
+            unsigned base = 0u;
+            if (lane == 31 && x != 0u) base = atomicAdd(&s_ncand, x);
+            base = __shfl_sync(0xFFFFFFFFu, base, 31);
+            unsigned pos = base + x - c;
+            while (m != 0u) {
+              const int e = __ffs((int)m) - 1;
+              m &= m - 1u;
+              if (pos < (unsigned)kTopkCand) cand[pos] = (uint16_t)(k * V8 + e);
+              ++pos;
+            }
+          }
+        }
+        __syncthreads();
+        use_cand = ok && s_ncand <= (unsigned)kTopkCand;
+      }
+    }
     __syncthreads();
-    if (ok) {
+    if (ok && use_cand) {
+      const int nc = (int)s_ncand;
+      for (int i = (int)threadIdx.x; i < nc; i += kKlThreads) atomicAdd(&hist[key16(cand[i]) & 0x7Fu], 1u);
+    } else if (ok) {
       for (int k = (int)threadIdx.x; k < nvec; k += kKlThreads) {
-        if constexpr (sizeof(T) == 2) {
+        if constexpr (BF) {
           if (k >= kfirst && k < klast) {
             // interior vector of bf16: keys two at a time; one add of 2 when
             // both keys of a word fall in the same bucket
 #pragma unroll
-            for (int q = 0; q < WPV; ++q) {
-              const uint32_t k2 = bf16x2_keys(wt[k * WPV + q]);
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t k2 = bf16x2_keys(wt[k * 4 + q]);
               const uint32_t k0 = k2 & 0xFFFFu, k1 = k2 >> 16;
               if (p == 0) {
-                const uint32_t d0 = k0 >> 8, d1 = k1 >> 8;
+                const uint32_t d0 = k0 >> 7, d1 = k1 >> 7;
                 if (d0 == d1) {
                   atomicAdd(&hist[d0], 2u);
                 } else {
@@ -590,13 +703,14 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
                   atomicAdd(&hist[d1], 1u);
                 }
               } else {
-                if ((k0 >> 8) == prefix) atomicAdd(&hist[k0 & 0xFFu], 1u);
-                if ((k1 >> 8) == prefix) atomicAdd(&hist[k1 & 0xFFu], 1u);
+                if ((k0 >> 7) == prefix) atomicAdd(&hist[k0 & 0x7Fu], 1u);
+                if ((k1 >> 7) == prefix) atomicAdd(&hist[k1 & 0x7Fu], 1u);
               }
             }
             continue;
           }
         }
+        // edge vectors (and f32): one key at a time
 #pragma unroll
         for (int q = 0; q < WPV; ++q) {
           const uint32_t w = wt[k * WPV + q];
@@ -604,40 +718,32 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
           for (int h = 0; h < Kf::kPerWord; ++h) {
             const int j = k * V8 + q * Kf::kPerWord + h;  // slot
             const uint32_t key = Kf::key(w, h);
-            const bool valid = j >= off && j < nslots && (p == 0 || (key >> (shift + 8)) == prefix);
-            if (valid) atomicAdd(&hist[(key >> shift) & 0xFFu], 1u);
+            const bool valid = j >= off && j < nslots && (p == 0 || (key >> (shift + dbits)) == prefix);
+            if (valid) atomicAdd(&hist[(key >> shift) & (uint32_t)(bins - 1)], 1u);
           }
         }
       }
     }
     __syncthreads();
     {
-      const unsigned v = hist[threadIdx.x];
-      for (int r = 0; r < csize; ++r) cluster.map_shared_rank(&recv[p & 1][0][0], r)[crank * 256 + threadIdx.x] = v;
-    }
-    cluster.sync();
-    {
-      unsigned tot = 0u;
-      for (int r = 0; r < csize; ++r) tot += recv[p & 1][r][threadIdx.x];
-      hist[threadIdx.x] = tot;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      // from the largest digit down: the digit whose bucket holds the remaining-th key
-      unsigned cum = 0u, d = 0u;
-      for (int dd = 255; dd >= 0; --dd) {
-        if (cum + hist[dd] >= remaining) {
-          d = (unsigned)dd;
-          break;
-        }
-        cum += hist[dd];
+      // the cluster's totals (the buffers alternate, so that no CTA writes a
+      // peer's buffer of the previous digit while that peer still reads it)
+      unsigned* rbuf = (p & 1) ? &recv_b[0][0] : recv_a;
+      const int rstride = (p & 1) ? 256 : 512;
+      for (int b = (int)threadIdx.x; b < bins; b += kKlThreads) {
+        const unsigned v = hist[b];
+        for (int r = 0; r < csize; ++r) cluster.map_shared_rank(rbuf, r)[crank * rstride + b] = v;
       }
-      s_digit = d;
-      s_remaining = remaining - cum;
-      s_count = hist[d];
+      cluster.sync();
+      for (int b = (int)threadIdx.x; b < bins; b += kKlThreads) {
+        unsigned tot = 0u;
+        for (int r = 0; r < csize; ++r) tot += rbuf[r * rstride + b];
+        hist[b] = tot;
+      }
     }
     __syncthreads();
-    prefix = (prefix << 8) | s_digit;
+    topk_find_digit(hist, bins, remaining, warp_sum, &s_digit, &s_remaining, &s_count);
+    prefix = (prefix << dbits) | s_digit;
     remaining = s_remaining;  // keys equal to the prefix so far still to take
     count = s_count;          // keys equal to the prefix so far
     __syncthreads();          // hist, s_* are rewritten by the next pass
@@ -655,7 +761,22 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
 
   // ---- ranks of the keys equal to tau, in index order (only when not all are taken)
   unsigned cta_off = 0u, warp_base = 0u;
-  if (rank_ties) {
+  bool fast_ties = false;  // CTA-uniform: the ties are ranked among the candidates
+  if (rank_ties && use_cand) {
+    if (threadIdx.x == 0) s_ntie = 0u;
+    __syncthreads();
+    const int nc = (int)s_ncand;
+    for (int i = (int)threadIdx.x; i < nc; i += kKlThreads) {
+      const int j = cand[i];
+      if (key16(j) == tau) {
+        const unsigned pos = atomicAdd(&s_ntie, 1u);
+        if (pos < (unsigned)kTopkTies) ties[pos] = j;
+      }
+    }
+    __syncthreads();
+    fast_ties = s_ntie <= (unsigned)kTopkTies;
+  }
+  if (rank_ties && !fast_ties) {
     unsigned running = 0u;  // ties in this warp's earlier vectors
     for (int kb = kw0; kb < kw0 + W && kb < nvec; kb += 32) {  // warp-uniform trip count
       const int k = kb + lane;
@@ -682,16 +803,38 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
     }
     if (lane == 0) warp_sum[wid] = running;
     __syncthreads();
+  }
+  if (rank_ties) {
+    // ties per CTA, exchanged in rank order (the same steps on both paths)
     unsigned total = 0u;
-    for (int w = 0; w < kKlWarps; ++w) {
-      if (w < wid) warp_base += warp_sum[w];
-      total += warp_sum[w];
+    if (fast_ties) {
+      total = s_ntie;
+    } else {
+      for (int w = 0; w < kKlWarps; ++w) {
+        if (w < wid) warp_base += warp_sum[w];
+        total += warp_sum[w];
+      }
     }
     for (int r = (int)threadIdx.x; r < csize; r += kKlThreads)
       cluster.map_shared_rank(recv_ties, r)[crank] = total;
     cluster.sync();
     for (int r = 0; r < crank; ++r) cta_off += recv_ties[r];
+    if (fast_ties) {
+      // this CTA's `take` ties with the smallest slot indices are in S:
+      // s_thr = the largest of them (-1: none)
+      const int nt = (int)s_ntie;
+      const int take = m_ties > cta_off ? (int)min(m_ties - cta_off, (unsigned)nt) : 0;
+      if (threadIdx.x == 0) s_thr = -1;
+      __syncthreads();
+      for (int i = (int)threadIdx.x; i < nt; i += kKlThreads) {
+        int smaller = 0;
+        for (int q = 0; q < nt; ++q) smaller += ties[q] < ties[i] ? 1 : 0;
+        if (smaller == take - 1) s_thr = ties[i];
+      }
+      __syncthreads();
+    }
   }
+  const int thr = fast_ties ? s_thr : -1;
   // ---- selection mask per vector (bit e: element e of the vector is in S),
   // and this warp's list of vectors with a selected element, in index order
   // (written over the tie prefixes of vectors already read)
@@ -702,16 +845,22 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
     const bool mine = k < nvec && k < kw0 + W;
     unsigned mask = 0u;
     if (mine && ok) {
-      if (sizeof(T) == 2 && !rank_ties && k >= kfirst && k < klast) {  // every key >= tau is in S
+      if (sizeof(T) == 2 && (!rank_ties || fast_ties) && k >= kfirst && k < klast) {
+        // every key > tau is in S; a key == tau unless the ties are ranked
+        // and its slot lies beyond this CTA's threshold
 #pragma unroll
         for (int q = 0; q < WPV; ++q) {
           const uint32_t k2 = bf16x2_keys(wt[k * WPV + q]);
-          mask |= ((k2 & 0xFFFFu) >= tau ? 1u : 0u) << (2 * q);
-          mask |= ((k2 >> 16) >= tau ? 1u : 0u) << (2 * q + 1);
+          const int j0 = k * V8 + 2 * q;
+          const uint32_t k0 = k2 & 0xFFFFu, k1 = k2 >> 16;
+          const bool s0 = k0 > tau || (k0 == tau && (!rank_ties || j0 <= thr));
+          const bool s1 = k1 > tau || (k1 == tau && (!rank_ties || j0 + 1 <= thr));
+          mask |= (s0 ? 1u : 0u) << (2 * q);
+          mask |= (s1 ? 1u : 0u) << (2 * q + 1);
         }
       } else {
         unsigned seen = 0u;
-        const unsigned pre = rank_ties ? cta_off + warp_base + vec_prefix[k] : 0u;
+        const unsigned pre = (rank_ties && !fast_ties) ? cta_off + warp_base + vec_prefix[k] : 0u;
 #pragma unroll
         for (int q = 0; q < WPV; ++q) {
           const uint32_t w = wt[k * WPV + q];
@@ -724,7 +873,7 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
             if (key > tau) {
               mask |= 1u << e;
             } else if (key == tau) {
-              const bool take = !rank_ties || pre + seen < m_ties;
+              const bool take = !rank_ties || (fast_ties ? j <= thr : pre + seen < m_ties);
               if (take) mask |= 1u << e;
               ++seen;
             }
@@ -909,7 +1058,11 @@ template <typename T>
 static cudaError_t launch_kl_topk(const KlArgs& a, const KlPlan& p, cudaStream_t s) {
   const int vec = 16 / (int)sizeof(T);
   const size_t nvec_max = (size_t)((p.slice + 2 * vec) / vec);
-  const size_t smem = p.smem + nvec_max * 5;  // + per-vector tie prefix (u32) and selection mask (u8)
+  // + per-vector tie prefix (u32) and selection mask (u8), the candidate and
+  // tie lists; at least the cluster's 512-count histograms, which lie over them
+  size_t tail = nvec_max * 4 + (nvec_max + 3) / 4 * 4 + kTopkCand * 2 + kTopkTies * 4;
+  if (tail < (size_t)p.cluster * 512 * 4) tail = (size_t)p.cluster * 512 * 4;
+  const size_t smem = p.smem + tail;
   cudaError_t e = cudaFuncSetAttribute(kl_topk_row_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
