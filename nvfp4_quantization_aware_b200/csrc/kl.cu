@@ -220,7 +220,7 @@ struct KlSliceGeom {
 // into st / ss: the 16-byte-aligned interior by TMA bulk copies (completion
 // on `bar`, bounded wait; *s_ok = 0 if it expired), the head and tail by
 // plain loads.  Called by every thread of the CTA (contains barriers).
-template <typename T>
+template <typename T, int NT = kKlThreads>
 NVFP4_DEV KlSliceGeom kl_stage_slice(const KlArgs& args, int64_t row, int64_t v0, int n, T* st, T* ss,
                                      uint64_t* bar_, int* s_ok_) {
   using E = KlElem<T>;
@@ -256,7 +256,7 @@ NVFP4_DEV KlSliceGeom kl_stage_slice(const KlArgs& args, int64_t row, int64_t v0
   }
   // head and tail logits with plain loads, pad slots with the pad value; all
   // disjoint from the bulk-copied interior [off + head, off + tail0)
-  for (int j = threadIdx.x; j < off + head; j += kKlThreads) {  // pad, then head
+  for (int j = threadIdx.x; j < off + head; j += NT) {  // pad, then head
     const int i = j - off;
     if (i < 0) {
       E::store1(st + j, kPadLogit);
@@ -266,7 +266,7 @@ NVFP4_DEV KlSliceGeom kl_stage_slice(const KlArgs& args, int64_t row, int64_t v0
       ss[j] = gs[i];
     }
   }
-  for (int j = off + tail0 + threadIdx.x; j < cap; j += kKlThreads) {  // tail, then pad
+  for (int j = off + tail0 + threadIdx.x; j < cap; j += NT) {  // tail, then pad
     const int i = j - off;
     if (i < n) {
       st[j] = gt[i];
@@ -291,7 +291,6 @@ template <typename T>
 __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
   using E = KlElem<T>;
   constexpr int V8 = E::kVec;        // elements per 16-byte vector
-  constexpr int ESZ = (int)sizeof(T);
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ uint64_t bar;
   __shared__ float warp_max[2][kKlWarps];
@@ -494,9 +493,11 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
 // shared memory: one digit per pass (9 + 7 bits for bf16, 4 x 8 for f32),
 // each pass a CTA histogram (shared-memory atomics) summed over the
 // cluster through distributed shared memory; that yields the k-th key tau
-// and how many keys equal to tau belong to S.  When not all of them do, a
-// scan over the slice in index order (and over the cluster's CTAs in rank
-// order) ranks them.  The statistics and the gradient then run over S only.
+// and how many keys equal to tau belong to S.  The last pass's per-CTA
+// counts of keys equal to tau give, in rank order, how many of them each
+// CTA contributes; the one CTA where that number is neither none nor all
+// ranks its own in index order.  The statistics and the gradient then run
+// over S only.
 
 template <typename T>
 struct KlKey;
@@ -524,26 +525,25 @@ struct KlKey<float> {
   NVFP4_DEV static uint32_t key(uint32_t w, int) { return (w & 0x80000000u) ? ~w : (w | 0x80000000u); }
 };
 
-// bf16 keys are selected in two digits of 9 and 7 bits: the first digit is
-// the sign and exponent, so its bucket at the k-th key holds one binade; the
-// keys in that bucket (the candidates) are collected once (up to
-// kTopkCand per CTA, else the second digit scans the whole slice), and the
-// second digit's histogram and the ranking of the ties (keys equal to the
-// k-th key; up to kTopkTies per CTA among the candidates, else a scan of
-// the whole slice) read only them.  f32 keys take four 8-bit digits over the
-// whole slice.
-constexpr int kTopkCand = 4096;
-constexpr int kTopkTies = 512;
+// bf16 keys are selected in two digits of 9 and 7 bits; the first digit is
+// the sign and exponent, so its bucket at the k-th key holds one binade.  The
+// first pass also keeps each 16-byte vector's largest key, so that the
+// second digit and the final selection read only the vectors that can hold a
+// key of the bucket (or of S): each warp lists those of its vectors with a
+// ballot and works through the list with all lanes.  f32 keys take four
+// 8-bit digits over the whole slice.
+constexpr int kTopkThreads = 512;  // more warps than kl_row_kernel: the select phases are latency-bound
+constexpr int kTopkWarps = kTopkThreads / 32;
 
 // The digit whose bucket holds the remaining-th largest key of a histogram
 // of `bins` counts (cluster totals in hist): an inclusive scan of the
 // bucket counts from the largest digit down over the CTA's threads
-// (kKlThreads, each owning bins / kKlThreads or one bucket).  Every thread
-// returns (digit, keys to take from its bucket, keys in its bucket).
+// (kTopkThreads, each owning bins / kTopkThreads or one bucket).  Every
+// thread returns (digit, keys to take from its bucket, keys in its bucket).
 NVFP4_DEV void topk_find_digit(const unsigned* hist, int bins, unsigned remaining, unsigned* warp_tot,
                                unsigned* s_digit, unsigned* s_remaining, unsigned* s_count) {
   const int t = (int)threadIdx.x, lane = t & 31, wid = t >> 5;
-  const int per = bins > kKlThreads ? bins / kKlThreads : 1;
+  const int per = bins > kTopkThreads ? bins / kTopkThreads : 1;
   const int b_hi = bins - 1 - t * per;  // this thread's buckets: b_hi, b_hi - 1, ..., b_hi - per + 1
   unsigned mine = 0u;
   if (b_hi >= 0)
@@ -574,8 +574,101 @@ NVFP4_DEV void topk_find_digit(const unsigned* hist, int bins, unsigned remainin
   __syncthreads();
 }
 
+// Sums the CTA histograms (hist[0..bins)) over the cluster: every CTA pushes
+// its counts into slot crank of each peer's rbuf ([csize][stride], 16-byte
+// vectors), then, after the cluster barrier, adds the csize rows into hist.
+// rbuf keeps the per-CTA rows.
+NVFP4_DEV void topk_cluster_hist(cg::cluster_group& cluster, unsigned* hist, unsigned* rbuf, int stride, int bins,
+                                 int csize, int crank) {
+  const int q4 = bins / 4;
+  const uint4* h4 = reinterpret_cast<const uint4*>(hist);
+  for (int i = (int)threadIdx.x; i < csize * q4; i += kTopkThreads) {
+    const int r = i / q4, b4 = i - r * q4;
+    reinterpret_cast<uint4*>(cluster.map_shared_rank(rbuf, r) + crank * stride)[b4] = h4[b4];
+  }
+  cluster.sync();
+  for (int b = (int)threadIdx.x; b < bins; b += kTopkThreads) {
+    unsigned tot = 0u;
+    for (int r = 0; r < csize; ++r) tot += rbuf[r * stride + b];
+    hist[b] = tot;
+  }
+  __syncthreads();
+}
+
+// Appends to this warp's list (list[kw0 ...], in index order) its vectors k
+// in [kw0, kw0 + W) with pred(k); returns the list length.  Warp-uniform.
+template <typename P>
+NVFP4_DEV unsigned topk_warp_list(unsigned* list, int kw0, int W, int nvec, P pred) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  unsigned len = 0u;
+  for (int kb = kw0; kb < kw0 + W && kb < nvec; kb += 32) {
+    const int k = kb + lane;
+    const bool in = k < nvec && k < kw0 + W && pred(k);
+    const unsigned b = __ballot_sync(0xFFFFFFFFu, in);
+    if (in) list[kw0 + len + __popc(b & lt_mask)] = (unsigned)k;
+    len += __popc(b);
+  }
+  __syncwarp();
+  return len;
+}
+
+// The largest slot index among the first `take` (in index order) keys equal
+// to tau of this CTA's slice, 0 < take < the CTA's count, where every such
+// key lies in a vector of the warps' lists (each list in index order, the
+// warps' ranges in index order): lanes own contiguous runs of their warp's
+// list, count their ties, scan the counts over the CTA, and the lane holding
+// the take-th tie finds its slot.  Writes *s_thr.
 template <typename T>
-__global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
+NVFP4_DEV void topk_rank_ties(const uint32_t* wt, const unsigned* list, unsigned len, int kw0, int off, int nslots,
+                              uint32_t tau, unsigned take, unsigned* warp_tot, int* s_thr) {
+  using Kf = KlKey<T>;
+  constexpr int V8 = KlElem<T>::kVec;
+  constexpr int WPV = 4;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const unsigned run = (len + 31u) / 32u;
+  const unsigned i0 = min((unsigned)lane * run, len), i1 = min(i0 + run, len);
+  unsigned c = 0u;
+  for (unsigned i = i0; i < i1; ++i) {
+    const int k = (int)list[kw0 + i];
+#pragma unroll
+    for (int q = 0; q < WPV; ++q) {
+      const uint32_t w = wt[k * WPV + q];
+#pragma unroll
+      for (int h = 0; h < Kf::kPerWord; ++h) {
+        const int j = k * V8 + q * Kf::kPerWord + h;
+        c += (j >= off && j < nslots && Kf::key(w, h) == tau) ? 1u : 0u;
+      }
+    }
+  }
+  unsigned x = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[wid] = x;
+  __syncthreads();
+  unsigned before = x - c;
+  for (int w = 0; w < wid; ++w) before += warp_tot[w];
+  if (before < take && take <= before + c) {
+    unsigned seen = before;
+    for (unsigned i = i0; i < i1; ++i) {
+      const int k = (int)list[kw0 + i];
+      for (int q = 0; q < WPV; ++q) {
+        const uint32_t w = wt[k * WPV + q];
+        for (int h = 0; h < Kf::kPerWord; ++h) {
+          const int j = k * V8 + q * Kf::kPerWord + h;
+          if (j >= off && j < nslots && Kf::key(w, h) == tau && ++seen == take) *s_thr = j;
+        }
+      }
+    }
+  }
+  __syncthreads();
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kTopkThreads) kl_topk_row_kernel(KlArgs args) {
   using E = KlElem<T>;
   using Kf = KlKey<T>;
   constexpr int V8 = E::kVec;
@@ -584,17 +677,16 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ uint64_t bar;
   __shared__ int s_ok;
-  __shared__ unsigned hist[512];
-  // cluster exchange of the histograms: one buffer per pass parity (f32) or
-  // per digit (bf16), written by every CTA of the cluster; the even passes'
-  // buffer (512 counts per CTA) lies over the tie prefixes, selection mask
-  // and candidate list, none of which is in use before the second digit
-  __shared__ unsigned recv_b[kKlMaxCluster][256];
-  __shared__ unsigned recv_ties[kKlMaxCluster];
-  __shared__ unsigned warp_sum[kKlWarps];
-  __shared__ unsigned s_digit, s_remaining, s_count, s_ncand, s_ntie;
+  __shared__ __align__(16) unsigned hist[512];
+  // cluster exchange of the histograms: one buffer per pass parity, written
+  // by every CTA of the cluster; the even passes' buffer (512 counts per
+  // CTA) lies over the vector lists and the selection mask, which are not in
+  // use before the second digit
+  __shared__ __align__(16) unsigned recv_b[kKlMaxCluster][256];
+  __shared__ unsigned warp_sum[kTopkWarps];
+  __shared__ unsigned s_digit, s_remaining, s_count;
   __shared__ int s_thr;
-  __shared__ KlStats warp_stats[kKlWarps];
+  __shared__ KlStats warp_stats[kTopkWarps];
   __shared__ KlStats peer_stats[kKlMaxCluster];
 
   cg::cluster_group cluster = cg::this_cluster();
@@ -610,107 +702,76 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
   T* st = reinterpret_cast<T*>(smem_raw);
   T* ss = st + args.slice + 2 * V8;
   const int nvec_max = (int)((args.slice + 2 * V8) / V8);
-  unsigned* vec_prefix = reinterpret_cast<unsigned*>(ss + args.slice + 2 * V8);
-  uint8_t* sel_mask = reinterpret_cast<uint8_t*>(vec_prefix + nvec_max);
-  uint16_t* cand = reinterpret_cast<uint16_t*>(sel_mask + (nvec_max + 3) / 4 * 4);  // kTopkCand slot indices
-  int* ties = reinterpret_cast<int*>(cand + kTopkCand);                            // kTopkTies slot indices
-  unsigned* recv_a = vec_prefix;  // [csize][512]
-  const uint16_t* t16 = reinterpret_cast<const uint16_t*>(st);
-  auto key16 = [&](int j) {  // order-preserving key of the bf16 teacher logit in slot j
-    const uint32_t u = t16[j];
-    return (u & 0x8000u) ? (~u & 0xFFFFu) : (u | 0x8000u);
-  };
-  const KlSliceGeom geo = kl_stage_slice<T>(args, row, v0, n, st, ss, &bar, &s_ok);
+  // bf16: largest valid key of each vector (0 when it has none)
+  uint16_t* vmax = reinterpret_cast<uint16_t*>(ss + args.slice + 2 * V8);
+  unsigned* vlist = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(vmax) + (nvec_max * 2 + 15) / 16 * 16);
+  uint8_t* sel_mask = reinterpret_cast<uint8_t*>(vlist + nvec_max);  // bit e: element e of the vector is in S
+  unsigned* recv_a = vlist;                                          // [csize][512], first digit only
+  const KlSliceGeom geo = kl_stage_slice<T, kTopkThreads>(args, row, v0, n, st, ss, &bar, &s_ok);
   const int off = geo.off, nslots = geo.nslots, nvec = geo.nvec;
   const int kfirst = (off + V8 - 1) / V8;  // vectors [kfirst, klast) hold no pad slot
   const int klast = nslots / V8;
   const bool ok = s_ok != 0;
   const uint32_t* wt = reinterpret_cast<const uint32_t*>(st);  // words of the teacher slice
+  const uint4* vt = reinterpret_cast<const uint4*>(st);
   constexpr int WPV = 16 / 4;                                   // words per 16-byte vector
+  // Warp w owns vectors [w W, (w + 1) W) for its lists, so that index order
+  // is (warp, list position) order.
+  const int W = ((nvec + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;
+  const int kw0 = wid * W;
 
   // ---- radix select of the k-th largest key over the row
   const uint32_t kk = (uint32_t)(args.topk < args.vocab ? args.topk : args.vocab);
-  uint32_t prefix = 0, remaining = kk, count = 0;
-  bool use_cand = false;  // bf16: the second digit and the ties read the candidate list (CTA-uniform)
+  uint32_t prefix = 0, remaining = kk;
   for (int p = 0; p < PASSES; ++p) {
     // digit p: bf16 bits [15:7] then [6:0]; f32 8 bits at a time from the top
     const int dbits = BF ? (p == 0 ? 9 : 7) : 8;
     const int shift = BF ? (p == 0 ? 7 : 0) : Kf::kBits - 8 * (p + 1);
     const int bins = 1 << dbits;
-    for (int b = (int)threadIdx.x; b < bins; b += kKlThreads) hist[b] = 0u;
-    if constexpr (BF) {
-      if (p == 1) {
-        // the candidates: slots whose key's first digit is `prefix`, appended
-        // per warp (a count per lane, an inclusive scan, one atomic per round)
-        if (threadIdx.x == 0) s_ncand = 0u;
-        __syncthreads();
-        if (ok) {
-          for (int kb = wid * 32; kb < nvec; kb += kKlThreads) {  // warp-uniform trip count
-            const int k = kb + lane;
-            unsigned m = 0u;  // bit e: element e of vector k is a candidate
-            if (k < nvec) {
+    for (int b = (int)threadIdx.x; b < bins; b += kTopkThreads) hist[b] = 0u;
+    __syncthreads();
+    if (BF && p == 1) {
+      // the vectors whose largest key reaches bucket `prefix`; keys outside
+      // the bucket are counted in a lane's own spare bin (128 + lane), so
+      // that every lane adds and no two lanes collide there
+      const uint32_t base = prefix << 7;
+      const unsigned len =
+          topk_warp_list(vlist, kw0, W, nvec, [&](int k) { return ok && (uint32_t)vmax[k] >= base; });
+      for (unsigned i = lane; i < len; i += 32) {
+        const int k = (int)vlist[kw0 + i];
+        const uint4 v = vt[k];
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        const bool interior = k >= kfirst && k < klast;
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const uint32_t k2 = bf16x2_keys(wt[k * 4 + q]);
-                const int j0 = k * V8 + 2 * q;
-                if (j0 >= off && j0 < nslots && ((k2 & 0xFFFFu) >> 7) == prefix) m |= 1u << (2 * q);
-                if (j0 + 1 >= off && j0 + 1 < nslots && ((k2 >> 16) >> 7) == prefix) m |= 2u << (2 * q);
-              }
-            }
-            const unsigned c = (unsigned)__popc(m);
-            unsigned x = c;  // inclusive scan over the lanes
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t k2 = bf16x2_keys(w4[q]);
+          const int j0 = k * V8 + 2 * q;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const unsigned y = __shfl_up_sync(0xFFFFFFFFu, x, o);
-              if (lane >= o) x += y;
-            }
-            unsigned base = 0u;
-            if (lane == 31 && x != 0u) base = atomicAdd(&s_ncand, x);
-            base = __shfl_sync(0xFFFFFFFFu, base, 31);
-            unsigned pos = base + x - c;
-            while (m != 0u) {
-              const int e = __ffs((int)m) - 1;
-              m &= m - 1u;
-              if (pos < (unsigned)kTopkCand) cand[pos] = (uint16_t)(k * V8 + e);
-              ++pos;
-            }
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t key = h ? (k2 >> 16) : (k2 & 0xFFFFu);
+            const bool in = (key >> 7) == prefix && (interior || (j0 + h >= off && j0 + h < nslots));
+            atomicAdd(&hist[in ? (key & 0x7Fu) : 128u + (unsigned)lane], 1u);
           }
         }
-        __syncthreads();
-        use_cand = ok && s_ncand <= (unsigned)kTopkCand;
       }
-    }
-    __syncthreads();
-    if (ok && use_cand) {
-      const int nc = (int)s_ncand;
-      for (int i = (int)threadIdx.x; i < nc; i += kKlThreads) atomicAdd(&hist[key16(cand[i]) & 0x7Fu], 1u);
     } else if (ok) {
-      for (int k = (int)threadIdx.x; k < nvec; k += kKlThreads) {
-        if constexpr (BF) {
-          if (k >= kfirst && k < klast) {
-            // interior vector of bf16: keys two at a time; one add of 2 when
-            // both keys of a word fall in the same bucket
+      for (int k = (int)threadIdx.x; k < nvec; k += kTopkThreads) {
+        if (BF && k >= kfirst && k < klast) {  // interior bf16 vector, first digit: every key counts
+          const uint4 v = vt[k];
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint32_t k2 = bf16x2_keys(wt[k * 4 + q]);
-              const uint32_t k0 = k2 & 0xFFFFu, k1 = k2 >> 16;
-              if (p == 0) {
-                const uint32_t d0 = k0 >> 7, d1 = k1 >> 7;
-                if (d0 == d1) {
-                  atomicAdd(&hist[d0], 2u);
-                } else {
-                  atomicAdd(&hist[d0], 1u);
-                  atomicAdd(&hist[d1], 1u);
-                }
-              } else {
-                if ((k0 >> 7) == prefix) atomicAdd(&hist[k0 & 0x7Fu], 1u);
-                if ((k1 >> 7) == prefix) atomicAdd(&hist[k1 & 0x7Fu], 1u);
-              }
-            }
-            continue;
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t k2 = bf16x2_keys(w4[q]);
+            atomicAdd(&hist[(k2 & 0xFFFFu) >> 7], 1u);
+            atomicAdd(&hist[k2 >> 23], 1u);
           }
+          const uint32_t m = __vmaxu2(__vmaxu2(bf16x2_keys(w4[0]), bf16x2_keys(w4[1])),
+                                      __vmaxu2(bf16x2_keys(w4[2]), bf16x2_keys(w4[3])));
+          vmax[k] = (uint16_t)max(m & 0xFFFFu, m >> 16);
+          continue;
         }
         // edge vectors (and f32): one key at a time
+        uint32_t vm = 0u;
 #pragma unroll
         for (int q = 0; q < WPV; ++q) {
           const uint32_t w = wt[k * WPV + q];
@@ -718,178 +779,90 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
           for (int h = 0; h < Kf::kPerWord; ++h) {
             const int j = k * V8 + q * Kf::kPerWord + h;  // slot
             const uint32_t key = Kf::key(w, h);
-            const bool valid = j >= off && j < nslots && (p == 0 || (key >> (shift + dbits)) == prefix);
-            if (valid) atomicAdd(&hist[(key >> shift) & (uint32_t)(bins - 1)], 1u);
+            const bool in_slice = j >= off && j < nslots;
+            if (in_slice) vm = max(vm, key);
+            if (in_slice && (p == 0 || (key >> (shift + dbits)) == prefix))
+              atomicAdd(&hist[(key >> shift) & (uint32_t)(bins - 1)], 1u);
           }
         }
+        if (BF && p == 0) vmax[k] = (uint16_t)vm;
       }
     }
     __syncthreads();
-    {
-      // the cluster's totals (the buffers alternate, so that no CTA writes a
-      // peer's buffer of the previous digit while that peer still reads it)
-      unsigned* rbuf = (p & 1) ? &recv_b[0][0] : recv_a;
-      const int rstride = (p & 1) ? 256 : 512;
-      for (int b = (int)threadIdx.x; b < bins; b += kKlThreads) {
-        const unsigned v = hist[b];
-        for (int r = 0; r < csize; ++r) cluster.map_shared_rank(rbuf, r)[crank * rstride + b] = v;
-      }
-      cluster.sync();
-      for (int b = (int)threadIdx.x; b < bins; b += kKlThreads) {
-        unsigned tot = 0u;
-        for (int r = 0; r < csize; ++r) tot += rbuf[r * rstride + b];
-        hist[b] = tot;
-      }
-    }
-    __syncthreads();
+    // the cluster's totals (the buffers alternate, so that no CTA writes a
+    // peer's buffer of the previous digit while that peer still reads it)
+    if (p & 1)
+      topk_cluster_hist(cluster, hist, &recv_b[0][0], 256, bins, csize, crank);
+    else
+      topk_cluster_hist(cluster, hist, recv_a, 512, bins, csize, crank);
     topk_find_digit(hist, bins, remaining, warp_sum, &s_digit, &s_remaining, &s_count);
     prefix = (prefix << dbits) | s_digit;
     remaining = s_remaining;  // keys equal to the prefix so far still to take
-    count = s_count;          // keys equal to the prefix so far
     __syncthreads();          // hist, s_* are rewritten by the next pass
   }
   const uint32_t tau = prefix;
-  const uint32_t m_ties = remaining;          // keys == tau that belong to S
-  const bool rank_ties = m_ties < count;      // uniform across the cluster
+  const uint32_t m_ties = remaining;  // keys == tau that belong to S
 
-  // Vectors are owned warp-contiguously from here on: warp w takes vectors
-  // [w W, (w + 1) W), lane l the ones at w W + 32 j + l, so index order is
-  // (warp, round, lane) order and the ranking scans stay inside the warp.
-  const int W = ((nvec + kKlWarps - 1) / kKlWarps + 31) / 32 * 32;
-  const int kw0 = wid * W;
+  // ---- this CTA's share of the ties: the last digit's per-CTA counts (the
+  // odd passes' buffer, last written in the final pass) in rank order
+  const unsigned last_digit = BF ? (tau & 0x7Fu) : (tau & 0xFFu);
+  unsigned cta_off = 0u;
+  for (int r = 0; r < crank; ++r) cta_off += recv_b[r][last_digit];
+  const unsigned n_mine = recv_b[crank][last_digit];
+  const unsigned take = m_ties > cta_off ? min(m_ties - cta_off, n_mine) : 0u;
+
+  // ---- the vectors that can hold a key of S (bf16: largest key >= tau)
+  unsigned len = topk_warp_list(vlist, kw0, W, nvec, [&](int k) {
+    sel_mask[k] = 0u;
+    return ok && (!BF || (uint32_t)vmax[k] >= tau);
+  });
+  // slots j with key == tau belong to S iff j <= thr
+  int thr = take == n_mine ? 0x7FFFFFFF : -1;
+  if (take != 0u && take != n_mine) {  // CTA-uniform: this CTA holds the boundary among the ties
+    topk_rank_ties<T>(wt, vlist, len, kw0, off, nslots, tau, take, warp_sum, &s_thr);
+    thr = s_thr;
+  }
+  // ---- their selection masks; the list keeps (in place, in order) the
+  // vectors with a selected element
   const unsigned lt_mask = (1u << lane) - 1u;
-
-  // ---- ranks of the keys equal to tau, in index order (only when not all are taken)
-  unsigned cta_off = 0u, warp_base = 0u;
-  bool fast_ties = false;  // CTA-uniform: the ties are ranked among the candidates
-  if (rank_ties && use_cand) {
-    if (threadIdx.x == 0) s_ntie = 0u;
-    __syncthreads();
-    const int nc = (int)s_ncand;
-    for (int i = (int)threadIdx.x; i < nc; i += kKlThreads) {
-      const int j = cand[i];
-      if (key16(j) == tau) {
-        const unsigned pos = atomicAdd(&s_ntie, 1u);
-        if (pos < (unsigned)kTopkTies) ties[pos] = j;
-      }
-    }
-    __syncthreads();
-    fast_ties = s_ntie <= (unsigned)kTopkTies;
-  }
-  if (rank_ties && !fast_ties) {
-    unsigned running = 0u;  // ties in this warp's earlier vectors
-    for (int kb = kw0; kb < kw0 + W && kb < nvec; kb += 32) {  // warp-uniform trip count
-      const int k = kb + lane;
-      unsigned c = 0u;
-      if (ok && k < nvec && k < kw0 + W) {
-#pragma unroll
-        for (int q = 0; q < WPV; ++q) {
-          const uint32_t w = wt[k * WPV + q];
-#pragma unroll
-          for (int h = 0; h < Kf::kPerWord; ++h) {
-            const int j = k * V8 + q * Kf::kPerWord + h;
-            c += (j >= off && j < nslots && Kf::key(w, h) == tau) ? 1u : 0u;
-          }
-        }
-      }
-      unsigned x = c;  // inclusive scan over the lanes
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const unsigned y = __shfl_up_sync(0xFFFFFFFFu, x, o);
-        if (lane >= o) x += y;
-      }
-      if (k < nvec && k < kw0 + W) vec_prefix[k] = running + x - c;
-      running += __shfl_sync(0xFFFFFFFFu, x, 31);
-    }
-    if (lane == 0) warp_sum[wid] = running;
-    __syncthreads();
-  }
-  if (rank_ties) {
-    // ties per CTA, exchanged in rank order (the same steps on both paths)
-    unsigned total = 0u;
-    if (fast_ties) {
-      total = s_ntie;
-    } else {
-      for (int w = 0; w < kKlWarps; ++w) {
-        if (w < wid) warp_base += warp_sum[w];
-        total += warp_sum[w];
-      }
-    }
-    for (int r = (int)threadIdx.x; r < csize; r += kKlThreads)
-      cluster.map_shared_rank(recv_ties, r)[crank] = total;
-    cluster.sync();
-    for (int r = 0; r < crank; ++r) cta_off += recv_ties[r];
-    if (fast_ties) {
-      // this CTA's `take` ties with the smallest slot indices are in S:
-      // s_thr = the largest of them (-1: none)
-      const int nt = (int)s_ntie;
-      const int take = m_ties > cta_off ? (int)min(m_ties - cta_off, (unsigned)nt) : 0;
-      if (threadIdx.x == 0) s_thr = -1;
-      __syncthreads();
-      for (int i = (int)threadIdx.x; i < nt; i += kKlThreads) {
-        int smaller = 0;
-        for (int q = 0; q < nt; ++q) smaller += ties[q] < ties[i] ? 1 : 0;
-        if (smaller == take - 1) s_thr = ties[i];
-      }
-      __syncthreads();
-    }
-  }
-  const int thr = fast_ties ? s_thr : -1;
-  // ---- selection mask per vector (bit e: element e of the vector is in S),
-  // and this warp's list of vectors with a selected element, in index order
-  // (written over the tie prefixes of vectors already read)
-  unsigned* sel_list = vec_prefix;
   unsigned list_len = 0u;
-  for (int kb = kw0; kb < kw0 + W && kb < nvec; kb += 32) {  // warp-uniform trip count
-    const int k = kb + lane;
-    const bool mine = k < nvec && k < kw0 + W;
+  for (unsigned ib = 0; ib < len; ib += 32) {  // warp-uniform trip count
+    const unsigned i = ib + lane;
+    const int k = i < len ? (int)vlist[kw0 + i] : -1;
     unsigned mask = 0u;
-    if (mine && ok) {
-      if (sizeof(T) == 2 && (!rank_ties || fast_ties) && k >= kfirst && k < klast) {
-        // every key > tau is in S; a key == tau unless the ties are ranked
-        // and its slot lies beyond this CTA's threshold
+    if (k >= 0) {
+      const uint4 v = vt[k];
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      if (BF && k >= kfirst && k < klast) {
 #pragma unroll
         for (int q = 0; q < WPV; ++q) {
-          const uint32_t k2 = bf16x2_keys(wt[k * WPV + q]);
+          const uint32_t k2 = bf16x2_keys(w4[q]);
           const int j0 = k * V8 + 2 * q;
           const uint32_t k0 = k2 & 0xFFFFu, k1 = k2 >> 16;
-          const bool s0 = k0 > tau || (k0 == tau && (!rank_ties || j0 <= thr));
-          const bool s1 = k1 > tau || (k1 == tau && (!rank_ties || j0 + 1 <= thr));
-          mask |= (s0 ? 1u : 0u) << (2 * q);
-          mask |= (s1 ? 1u : 0u) << (2 * q + 1);
+          mask |= (k0 > tau || (k0 == tau && j0 <= thr) ? 1u : 0u) << (2 * q);
+          mask |= (k1 > tau || (k1 == tau && j0 + 1 <= thr) ? 1u : 0u) << (2 * q + 1);
         }
       } else {
-        unsigned seen = 0u;
-        const unsigned pre = (rank_ties && !fast_ties) ? cta_off + warp_base + vec_prefix[k] : 0u;
 #pragma unroll
-        for (int q = 0; q < WPV; ++q) {
-          const uint32_t w = wt[k * WPV + q];
+        for (int q = 0; q < WPV; ++q)
 #pragma unroll
           for (int h = 0; h < Kf::kPerWord; ++h) {
             const int e = q * Kf::kPerWord + h;
             const int j = k * V8 + e;
-            if (j < off || j >= nslots) continue;
-            const uint32_t key = Kf::key(w, h);
-            if (key > tau) {
-              mask |= 1u << e;
-            } else if (key == tau) {
-              const bool take = !rank_ties || (fast_ties ? j <= thr : pre + seen < m_ties);
-              if (take) mask |= 1u << e;
-              ++seen;
-            }
+            const uint32_t key = Kf::key(w4[q], h);
+            const bool in = j >= off && j < nslots && (key > tau || (key == tau && j <= thr));
+            mask |= (in ? 1u : 0u) << e;
           }
-        }
       }
+      sel_mask[k] = (uint8_t)mask;
     }
-    if (mine) sel_mask[k] = (uint8_t)mask;
-    const unsigned b = __ballot_sync(0xFFFFFFFFu, mask != 0u);  // after every lane read its prefix
-    if (mask != 0u) sel_list[kw0 + list_len + __popc(b & lt_mask)] = (unsigned)k;
+    const unsigned b = __ballot_sync(0xFFFFFFFFu, mask != 0u);  // every lane has read its entry
+    if (mask != 0u) vlist[kw0 + list_len + __popc(b & lt_mask)] = (unsigned)k;
     list_len += __popc(b);
   }
+  unsigned* sel_list = vlist;
   __syncthreads();
-
   // ---- online statistics over S (other slots read as the pad value)
-  const uint4* vt = reinterpret_cast<const uint4*>(st);
   const uint4* vs = reinterpret_cast<const uint4*>(ss);
   const float a = args.a;
   KlStats my;
@@ -934,7 +907,7 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
   __syncthreads();
   if (threadIdx.x < csize) {
     KlStats c = warp_stats[0];
-    for (int w = 1; w < kKlWarps; ++w) c = stats_merge(c, warp_stats[w]);
+    for (int w = 1; w < kTopkWarps; ++w) c = stats_merge(c, warp_stats[w]);
     cluster.map_shared_rank(peer_stats, (int)threadIdx.x)[crank] = c;
   }
   cluster.sync();  // all pushes visible; no CTA touches a peer after this point
@@ -977,7 +950,7 @@ __global__ void __launch_bounds__(kKlThreads) kl_topk_row_kernel(KlArgs args) {
       store_vec(k, o);
     }
     // the rest: zeros
-    for (int k = (int)threadIdx.x; k < nvec; k += kKlThreads) {
+    for (int k = (int)threadIdx.x; k < nvec; k += kTopkThreads) {
       if (sel_mask[k] != 0u) continue;
       float o[V8];
 #pragma unroll
@@ -1058,16 +1031,16 @@ template <typename T>
 static cudaError_t launch_kl_topk(const KlArgs& a, const KlPlan& p, cudaStream_t s) {
   const int vec = 16 / (int)sizeof(T);
   const size_t nvec_max = (size_t)((p.slice + 2 * vec) / vec);
-  // + per-vector tie prefix (u32) and selection mask (u8), the candidate and
-  // tie lists; at least the cluster's 512-count histograms, which lie over them
-  size_t tail = nvec_max * 4 + (nvec_max + 3) / 4 * 4 + kTopkCand * 2 + kTopkTies * 4;
+  // + per-vector largest key (u16), then the vector lists (u32) and the
+  // selection mask (u8), or, over them, the cluster's 512-count histograms
+  size_t tail = nvec_max * 4 + (nvec_max + 3) / 4 * 4;
   if (tail < (size_t)p.cluster * 512 * 4) tail = (size_t)p.cluster * 512 * 4;
-  const size_t smem = p.smem + tail;
+  const size_t smem = p.smem + (nvec_max * 2 + 15) / 16 * 16 + tail;
   cudaError_t e = cudaFuncSetAttribute(kl_topk_row_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(a.rows * p.cluster));
-  cfg.blockDim = dim3(kKlThreads);
+  cfg.blockDim = dim3(kTopkThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
