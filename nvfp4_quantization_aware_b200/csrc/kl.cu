@@ -217,9 +217,10 @@ struct KlSliceGeom {
 };
 
 // Stages the slice [v0, v0 + n) of row `row` of the teacher and the student
-// into st / ss: the 16-byte-aligned interior by TMA bulk copies (completion
-// on `bar`, bounded wait; *s_ok = 0 if it expired), the head and tail by
-// plain loads.  Called by every thread of the CTA (contains barriers).
+// into st / ss (the teacher only when ss is null): the 16-byte-aligned
+// interior by TMA bulk copies (completion on `bar`, bounded wait; *s_ok = 0
+// if it expired), the head and tail by plain loads.  Called by every thread
+// of the CTA (contains barriers).
 template <typename T, int NT = kKlThreads>
 NVFP4_DEV KlSliceGeom kl_stage_slice(const KlArgs& args, int64_t row, int64_t v0, int n, T* st, T* ss,
                                      uint64_t* bar_, int* s_ok_) {
@@ -250,9 +251,9 @@ NVFP4_DEV KlSliceGeom kl_stage_slice(const KlArgs& args, int64_t row, int64_t v0
   }
   __syncthreads();
   if (threadIdx.x == 0 && nint > 0) {
-    mbar_expect_tx(&bar, (uint32_t)(2 * nint * ESZ));
+    mbar_expect_tx(&bar, (uint32_t)((ss != nullptr ? 2 : 1) * nint * ESZ));
     bulk_g2s(st + off + head, gt + head, (uint32_t)(nint * ESZ), &bar);
-    bulk_g2s(ss + off + head, gs + head, (uint32_t)(nint * ESZ), &bar);
+    if (ss != nullptr) bulk_g2s(ss + off + head, gs + head, (uint32_t)(nint * ESZ), &bar);
   }
   // head and tail logits with plain loads, pad slots with the pad value; all
   // disjoint from the bulk-copied interior [off + head, off + tail0)
@@ -260,20 +261,20 @@ NVFP4_DEV KlSliceGeom kl_stage_slice(const KlArgs& args, int64_t row, int64_t v0
     const int i = j - off;
     if (i < 0) {
       E::store1(st + j, kPadLogit);
-      E::store1(ss + j, kPadLogit);
+      if (ss != nullptr) E::store1(ss + j, kPadLogit);
     } else {
       st[j] = gt[i];
-      ss[j] = gs[i];
+      if (ss != nullptr) ss[j] = gs[i];
     }
   }
   for (int j = off + tail0 + threadIdx.x; j < cap; j += NT) {  // tail, then pad
     const int i = j - off;
     if (i < n) {
       st[j] = gt[i];
-      ss[j] = gs[i];
+      if (ss != nullptr) ss[j] = gs[i];
     } else {
       E::store1(st + j, kPadLogit);
-      E::store1(ss + j, kPadLogit);
+      if (ss != nullptr) E::store1(ss + j, kPadLogit);
     }
   }
   if (nint > 0 && !mbar_wait_bounded(&bar, 0)) s_ok = 0;
@@ -532,7 +533,7 @@ struct KlKey<float> {
 // key of the bucket (or of S): each warp lists those of its vectors with a
 // ballot and works through the list with all lanes.  f32 keys take four
 // 8-bit digits over the whole slice.
-constexpr int kTopkThreads = 512;  // more warps than kl_row_kernel: the select phases are latency-bound
+constexpr int kTopkThreads = 256;
 constexpr int kTopkWarps = kTopkThreads / 32;
 
 // The digit whose bucket holds the remaining-th largest key of a histogram
@@ -699,15 +700,17 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topk_row_kernel(KlArgs args) 
   if (v1 > args.vocab) v1 = args.vocab;
   const int n = v1 > v0 ? (int)(v1 - v0) : 0;
 
+  // Only the teacher slice is staged; the few student logits of S are read
+  // from global memory (slot j holds logit v0 + j - off of the row).
   T* st = reinterpret_cast<T*>(smem_raw);
-  T* ss = st + args.slice + 2 * V8;
+  const T* gs = reinterpret_cast<const T*>(args.student) + row * args.ld + v0;
   const int nvec_max = (int)((args.slice + 2 * V8) / V8);
   // bf16: largest valid key of each vector (0 when it has none)
-  uint16_t* vmax = reinterpret_cast<uint16_t*>(ss + args.slice + 2 * V8);
+  uint16_t* vmax = reinterpret_cast<uint16_t*>(st + args.slice + 2 * V8);
   unsigned* vlist = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(vmax) + (nvec_max * 2 + 15) / 16 * 16);
   uint8_t* sel_mask = reinterpret_cast<uint8_t*>(vlist + nvec_max);  // bit e: element e of the vector is in S
   unsigned* recv_a = vlist;                                          // [csize][512], first digit only
-  const KlSliceGeom geo = kl_stage_slice<T, kTopkThreads>(args, row, v0, n, st, ss, &bar, &s_ok);
+  const KlSliceGeom geo = kl_stage_slice<T, kTopkThreads>(args, row, v0, n, st, nullptr, &bar, &s_ok);
   const int off = geo.off, nslots = geo.nslots, nvec = geo.nvec;
   const int kfirst = (off + V8 - 1) / V8;  // vectors [kfirst, klast) hold no pad slot
   const int klast = nslots / V8;
@@ -863,7 +866,19 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topk_row_kernel(KlArgs args) 
   unsigned* sel_list = vlist;
   __syncthreads();
   // ---- online statistics over S (other slots read as the pad value)
-  const uint4* vs = reinterpret_cast<const uint4*>(ss);
+  // the student's vector k (pad value outside the slice); interior vectors
+  // are 16-byte aligned in global memory as in shared memory
+  auto student_vec = [&](int k, float (&zs)[V8]) {
+    if (k >= kfirst && k < klast) {
+      E::unpack(__ldg(reinterpret_cast<const uint4*>(gs + (k * V8 - off))), zs);
+    } else {
+#pragma unroll
+      for (int e = 0; e < V8; ++e) {
+        const int j = k * V8 + e;
+        zs[e] = (j >= off && j < nslots) ? E::load1(gs + (j - off)) : kPadLogit;
+      }
+    }
+  };
   const float a = args.a;
   KlStats my;
   stats_init(my, kPadLogit * a);
@@ -874,7 +889,7 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topk_row_kernel(KlArgs args) 
       const unsigned mask = sel_mask[k];
       float zt[V8], zs[V8];
       E::unpack(vt[k], zt);
-      E::unpack(vs[k], zs);
+      student_vec(k, zs);
       float lt = kPadLogit, ls = kPadLogit;
 #pragma unroll
       for (int e = 0; e < V8; ++e) {
@@ -941,7 +956,7 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topk_row_kernel(KlArgs args) 
       const unsigned mask = sel_mask[k];
       float zt[V8], zs[V8], o[V8];
       E::unpack(vt[k], zt);
-      E::unpack(vs[k], zs);
+      student_vec(k, zs);
 #pragma unroll
       for (int e = 0; e < V8; ++e) {
         const float pt = ex2(fmaf(zt[e], a, -Lt)), ps = ex2(fmaf(zs[e], a, -Ls));
@@ -1031,11 +1046,12 @@ template <typename T>
 static cudaError_t launch_kl_topk(const KlArgs& a, const KlPlan& p, cudaStream_t s) {
   const int vec = 16 / (int)sizeof(T);
   const size_t nvec_max = (size_t)((p.slice + 2 * vec) / vec);
-  // + per-vector largest key (u16), then the vector lists (u32) and the
-  // selection mask (u8), or, over them, the cluster's 512-count histograms
+  // the teacher slice, the per-vector largest key (u16), then the vector
+  // lists (u32) and the selection mask (u8), or, over them, the cluster's
+  // 512-count histograms
   size_t tail = nvec_max * 4 + (nvec_max + 3) / 4 * 4;
   if (tail < (size_t)p.cluster * 512 * 4) tail = (size_t)p.cluster * 512 * 4;
-  const size_t smem = p.smem + (nvec_max * 2 + 15) / 16 * 16 + tail;
+  const size_t smem = p.smem / 2 + (nvec_max * 2 + 15) / 16 * 16 + tail;  // the teacher's slice only
   cudaError_t e = cudaFuncSetAttribute(kl_topk_row_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
