@@ -217,13 +217,14 @@ struct KlSliceGeom {
 };
 
 // Stages the slice [v0, v0 + n) of row `row` of the teacher and the student
-// into st / ss (the teacher only when ss is null): the 16-byte-aligned
-// interior by TMA bulk copies (completion on `bar`, bounded wait; *s_ok = 0
-// if it expired), the head and tail by plain loads.  Called by every thread
-// of the CTA (contains barriers).
+// into st / ss (the teacher only when ss is null; then, on request, the
+// student's interior is prefetched into L2): the 16-byte-aligned interior by
+// TMA bulk copies (completion on `bar`, bounded wait; *s_ok = 0 if it
+// expired), the head and tail by plain loads.  Called by every thread of the
+// CTA (contains barriers).
 template <typename T, int NT = kKlThreads>
 NVFP4_DEV KlSliceGeom kl_stage_slice(const KlArgs& args, int64_t row, int64_t v0, int n, T* st, T* ss,
-                                     uint64_t* bar_, int* s_ok_) {
+                                     uint64_t* bar_, int* s_ok_, bool prefetch_student = false) {
   using E = KlElem<T>;
   constexpr int V8 = E::kVec;
   constexpr int ESZ = (int)sizeof(T);
@@ -254,6 +255,7 @@ NVFP4_DEV KlSliceGeom kl_stage_slice(const KlArgs& args, int64_t row, int64_t v0
     mbar_expect_tx(&bar, (uint32_t)((ss != nullptr ? 2 : 1) * nint * ESZ));
     bulk_g2s(st + off + head, gt + head, (uint32_t)(nint * ESZ), &bar);
     if (ss != nullptr) bulk_g2s(ss + off + head, gs + head, (uint32_t)(nint * ESZ), &bar);
+    if (ss == nullptr && prefetch_student) bulk_prefetch_l2(gs + head, (uint32_t)(nint * ESZ));
   }
   // head and tail logits with plain loads, pad slots with the pad value; all
   // disjoint from the bulk-copied interior [off + head, off + tail0)
@@ -289,7 +291,7 @@ NVFP4_DEV KlSliceGeom kl_stage_slice(const KlArgs& args, int64_t row, int64_t v0
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
+__global__ void __launch_bounds__(kKlThreads, 6) kl_row_kernel(KlArgs args) {
   using E = KlElem<T>;
   constexpr int V8 = E::kVec;        // elements per 16-byte vector
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -308,14 +310,31 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
   if (v1 > args.vocab) v1 = args.vocab;
   const int n = v1 > v0 ? (int)(v1 - v0) : 0;
 
+  // The teacher slice is staged in shared memory; the student slice is
+  // prefetched into L2 and read from global memory in both passes (slot j
+  // holds logit v0 + j - off of the row), which halves the shared memory of
+  // a CTA and so doubles the CTAs an SM holds.
   T* st = reinterpret_cast<T*>(smem_raw);
-  T* ss = st + args.slice + 2 * V8;
-  const KlSliceGeom geo = kl_stage_slice<T>(args, row, v0, n, st, ss, &bar, &s_ok);
+  const T* gs = reinterpret_cast<const T*>(args.student) + row * args.ld + v0;
+  const KlSliceGeom geo = kl_stage_slice<T>(args, row, v0, n, st, nullptr, &bar, &s_ok, true);
   const int off = geo.off, nslots = geo.nslots, nvec = geo.nvec;
   const bool ok = s_ok != 0;
+  const int kfirst = (off + V8 - 1) / V8;  // vectors [kfirst, klast) hold no pad slot
+  const int klast = nslots / V8;
 
   const uint4* vt = reinterpret_cast<const uint4*>(st);
-  const uint4* vs = reinterpret_cast<const uint4*>(ss);
+  // the student's vector k, pad value outside the slice; interior vectors are
+  // 16-byte aligned in global memory as in shared memory
+  auto svec = [&](int k) -> uint4 {
+    if (k >= kfirst && k < klast) return __ldg(reinterpret_cast<const uint4*>(gs + (k * V8 - off)));
+    float z[V8];
+#pragma unroll
+    for (int e = 0; e < V8; ++e) {
+      const int j = k * V8 + e;
+      z[e] = (j >= off && j < nslots) ? E::load1(gs + (j - off)) : kPadLogit;
+    }
+    return E::pack(z);
+  };
   const float a = args.a;  // log2(e) / T > 0
 
   // ---- online statistics over this thread's vectors; the running maxima are
@@ -326,7 +345,7 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
   float zmt = kPadLogit, zms = kPadLogit;  // running max of the raw logits
   if (ok) {
     for (int k = threadIdx.x; k < nvec; k += kKlThreads) {
-      const uint4 rt = vt[k], rs = vs[k];
+      const uint4 rt = vt[k], rs = svec(k);
       const float lt = E::vmax(rt), ls = E::vmax(rs);
       if (lt > zmt || ls > zms) {
         zmt = fmaxf(zmt, lt);
@@ -443,12 +462,10 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
     const float gm = fold ? 1.0f : g;
     T* gout = reinterpret_cast<T*>(args.dlogits) + row * args.ld_grad + v0 - off;  // slot j -> gout[j]
     const bool vec_ok = (((uintptr_t)gout) & 15u) == 0;
-    const int kfirst = (off + V8 - 1) / V8;          // first vector with no leading pad
-    const int klast = nslots / V8;                   // vectors [kfirst, klast) are all real
     for (int k = threadIdx.x; k < nvec; k += kKlThreads) {
       float o[V8];
       if constexpr (sizeof(T) == 2) {
-        const uint4 rt = vt[k], rs = vs[k];
+        const uint4 rt = vt[k], rs = svec(k);
         const uint32_t wt[4] = {rt.x, rt.y, rt.z, rt.w}, ws[4] = {rs.x, rs.y, rs.z, rs.w};
         const f32x2 A = pair(a, a), NLt = pair(-Lt, -Lt), NLs = pair(-Ls, -Ls), G = pair(gm, gm);
 #pragma unroll
@@ -463,7 +480,7 @@ __global__ void __launch_bounds__(kKlThreads) kl_row_kernel(KlArgs args) {
       } else {
         float zt[V8], zs[V8];
         E::unpack(vt[k], zt);
-        E::unpack(vs[k], zs);
+        E::unpack(svec(k), zs);
 #pragma unroll
         for (int j = 0; j < V8; ++j) {
           const float pt = exp2_poly(fmaf(zt[j], a, -Lt));
@@ -1025,12 +1042,13 @@ static bool kl_plan(int64_t vocab, int esz, KlPlan& p) {
 
 template <typename T>
 static cudaError_t launch_kl(const KlArgs& a, const KlPlan& p, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(kl_row_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+  const size_t smem = p.smem / 2;  // the teacher's slice only
+  cudaError_t e = cudaFuncSetAttribute(kl_row_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(a.rows * p.cluster));
   cfg.blockDim = dim3(kKlThreads);
-  cfg.dynamicSmemBytes = p.smem;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;

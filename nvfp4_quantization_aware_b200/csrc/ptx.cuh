@@ -81,6 +81,12 @@ NVFP4_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* ba
       : "memory");
 }
 
+// Bulk prefetch of global memory into L2 (no completion to wait for);
+// address 16-byte aligned, size a multiple of 16.
+NVFP4_DEV void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // 3-D tiled tensor store from this CTA's shared memory (bulk-group
 // completion).  Coordinates must be non-negative; x * element size a
 // multiple of 16 bytes.  Out-of-range parts of the box are not written.
