@@ -307,32 +307,13 @@ def run_ours(args, world, rank, local):
 def run_e2e(Q, xs, dev, stream, K, world):
     """Same metric through the public API with pinned host buffers: per step
     the inputs are copied host -> device, both passes run, and the frozen
-    codes + block scales + tensor scales are copied back."""
+    codes + block scales + tensor scales are copied back.  The library's
+    HostGroupedQuantizer overlaps the copies of one chunk of tensors with the
+    kernels of the next (three streams)."""
     hx = [x.cpu().pin_memory() for x in xs]
-    n = len(xs)
-    ts = torch.zeros(n, dtype=torch.float32, device=dev)
-    dx = [torch.empty_like(x) for x in xs]
-    sbs = [torch.empty(x.shape[0], x.shape[1] // 16, dtype=torch.uint8, device=dev) for x in xs]
-    cd = [torch.empty(x.shape[0], x.shape[1] // 2, dtype=torch.uint8, device=dev) for x in xs]
-    cf = [torch.empty_like(c) for c in cd]
-    hc = [torch.empty(c.shape, dtype=torch.uint8).pin_memory() for c in cd]
-    hs = [torch.empty(s.shape, dtype=torch.uint8).pin_memory() for s in sbs]
-    hts = torch.empty(n, dtype=torch.float32).pin_memory()
-    ws = torch.empty(int(Q.lib().nvfp4_grouped_workspace_size(Q.DYNAMIC)), dtype=torch.uint8, device=dev)
-
-    def step():
-        for d, h in zip(dx, hx):
-            d.copy_(h, non_blocking=True)
-        Q.nvfp4_quantize_grouped(dx, Q.DYNAMIC, tensor_scales=ts, block_scales=sbs, codes=cd, workspace=ws)
-        Q.nvfp4_quantize_grouped(dx, Q.FROZEN_ALL, tensor_scales=ts, block_scales=sbs, codes=cf)
-        for h, c in zip(hc, cf):
-            h.copy_(c, non_blocking=True)
-        for h, s in zip(hs, sbs):
-            h.copy_(s, non_blocking=True)
-        hts.copy_(ts, non_blocking=True)
-
+    hq = Q.HostGroupedQuantizer(hx, dev, passes=(Q.DYNAMIC, Q.FROZEN_ALL))
     with torch.cuda.stream(stream):
-        step()
+        hq.run(stream)
         stream.synchronize()
         start = torch.cuda.Event(enable_timing=True)
         end = torch.cuda.Event(enable_timing=True)
@@ -340,17 +321,16 @@ def run_e2e(Q, xs, dev, stream, K, world):
         torch.cuda.synchronize(dev)
         start.record(stream)
         for _ in range(K):
-            step()
+            hq.run(stream)
         end.record(stream)
         torch.cuda.synchronize(dev)
         barrier(world)
     ms = max_over_ranks(start.elapsed_time(end), world) / K
     n_elem = sum(x.numel() for x in xs)
     units = sum_over_ranks(float(n_elem), world)
-    h2d = sum(x.numel() * x.element_size() for x in xs)
-    d2h = sum(c.numel() for c in cf) + sum(s.numel() for s in sbs) + 4 * n
     return {"value": round(units * 2 * BYTES_PER_ELEM / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3), "steps": K}
+            "h2d_bytes_per_step": hq.h2d_bytes, "d2h_bytes_per_step": hq.d2h_bytes, "ms_per_step": round(ms, 3),
+            "steps": K, "chunks": len(hq.chunks)}
 
 
 def flush_l2(buf):

@@ -55,3 +55,4 @@ from .binding import (  # noqa: F401
     nvfp4_calibrate_mse_grouped,
 )
 from .autograd import FakeQuantSTE, KLDistillLoss, fake_quant_ste, kl_distill_loss  # noqa: F401
+from .hostio import HostGroupedQuantizer  # noqa: F401
