@@ -686,6 +686,36 @@ nvfp4_status qad_kl_topk_fwd_bwd(const void* teacher, const void* student, nvfp4
                                  float grad_scale, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Top-p KL distillation loss (Qwen3.6-35B-A3B W4A4 tutorial, section "5.
+ * 评估": its recommendation for the next QAD run, after the runs that hit the
+ * output-length cap, is to select the teacher's top-p entries instead of the
+ * top-k ones).  Per row, S = the shortest prefix of the teacher's entries in
+ * decreasing logit order (equal logits: smaller vocabulary index first) whose
+ * teacher probability softmax(z_t / T) sums to at least top_p; top_p >= 1
+ * selects the whole row.  The loss and gradient over S are those of
+ * qad_kl_topk_fwd_bwd with k = |S|.
+ * Arguments as qad_kl_topk_fwd_bwd with top_p (> 0, NVFP4_ERR_ARG otherwise)
+ * in place of k, plus:
+ *   row_k       device int64 [rows] or NULL: receives |S| of every row
+ *   workspace   >= qad_kl_topp_workspace_size(rows, vocab, dtype) bytes,
+ *               16-byte aligned
+ * The probabilities are summed in 64-bit fixed point (the largest logit of a
+ * row weighs 2^40; exponentials from the hardware ex2), so |S| does not
+ * depend on the order of the additions; against a float64 computation it can
+ * differ only where the cumulative probability lies within ~1e-6 of top_p.
+ * Two launches more than the top-k loss' first one: a pass over the teacher
+ * logits that finds |S| (a radix select whose buckets hold probability mass),
+ * then the top-k loss with a k per row.
+ * ------------------------------------------------------------------------ */
+size_t qad_kl_topp_workspace_size(int64_t rows, int64_t vocab, nvfp4_dtype dtype);
+
+nvfp4_status qad_kl_topp_fwd_bwd(const void* teacher, const void* student, nvfp4_dtype dtype,
+                                 int64_t rows, int64_t vocab, int64_t ld, float top_p, float temperature,
+                                 float* loss, float* row_kl, void* dlogits, int64_t ld_grad,
+                                 float grad_scale, int64_t* row_k, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/* ------------------------------------------------------------------------
  * qad_kl_fwd_bwd without a workspace argument, for callers that cannot
  * allocate device memory when they compute the loss (a framework whose
  * caching allocator holds the device budget, a fixed pre-planned memory

@@ -51,6 +51,7 @@ from .binding import (  # noqa: F401
     nvfp4_selftest_division,
     qad_kl_fwd_bwd,
     qad_kl_topk_fwd_bwd,
+    qad_kl_topp_fwd_bwd,
     nvfp4_calibrate_mse,
     nvfp4_calibrate_mse_grouped,
 )

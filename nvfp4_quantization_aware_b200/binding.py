@@ -156,6 +156,10 @@ def lib() -> ctypes.CDLL:
     L.qad_kl_fwd_bwd.restype = i32
     L.qad_kl_topk_fwd_bwd.argtypes = [p, p, i32, i64, i64, i64, i64, f32, p, p, p, i64, f32, p, sz, p]
     L.qad_kl_topk_fwd_bwd.restype = i32
+    L.qad_kl_topp_workspace_size.argtypes = [i64, i64, i32]
+    L.qad_kl_topp_workspace_size.restype = sz
+    L.qad_kl_topp_fwd_bwd.argtypes = [p, p, i32, i64, i64, i64, f32, f32, p, p, p, i64, f32, p, p, sz, p]
+    L.qad_kl_topp_fwd_bwd.restype = i32
     # MoE layer step
     L.nvfp4_moe_rows_capacity.argtypes = [i32, i32, i32]
     L.nvfp4_moe_rows_capacity.restype = i64
@@ -751,6 +755,41 @@ def qad_kl_topk_fwd_bwd(teacher: torch.Tensor, student: torch.Tensor, k: int, te
                                0 if workspace is None else workspace.numel(), _stream(dev))
     _check(st, "qad_kl_topk_fwd_bwd")
     return loss, row_kl, dlogits
+
+
+def qad_kl_topp_fwd_bwd(teacher: torch.Tensor, student: torch.Tensor, p: float, temperature: float = 1.0,
+                        want_grad: bool = True, grad_scale: float | None = None, want_row_kl: bool = False,
+                        want_row_k: bool = False, dlogits: torch.Tensor | None = None,
+                        workspace: torch.Tensor | None = None):
+    """KL over the teacher's top-p set of each row (the shortest prefix of the
+    top-k order whose teacher probability reaches p; p >= 1: the whole row).
+    Returns (loss f32 [1], row_kl f32 [rows] or None, dlogits or None,
+    row_k int64 [rows] (|S| per row) or None)."""
+    _cuda2d(teacher, "teacher")
+    _cuda2d(student, "student")
+    if teacher.shape != student.shape or teacher.dtype != student.dtype or teacher.stride() != student.stride():
+        raise ValueError("teacher and student must have the same shape, dtype and strides")
+    L = lib()
+    rows, V = teacher.shape
+    dev = teacher.device
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    row_kl = torch.empty(rows, dtype=torch.float32, device=dev) if want_row_kl else None
+    row_k = torch.empty(rows, dtype=torch.int64, device=dev) if want_row_k else None
+    if want_grad and dlogits is None:
+        dlogits = torch.empty_like(student)
+    if not want_grad:
+        dlogits = None
+    if grad_scale is None:
+        grad_scale = 1.0 / rows if rows > 0 else 1.0
+    need = int(L.qad_kl_topp_workspace_size(rows, V, _dtype_code(teacher)))
+    if workspace is None:
+        workspace = _workspace(need, dev)
+    st = L.qad_kl_topp_fwd_bwd(_ptr(teacher), _ptr(student), _dtype_code(teacher), rows, V, teacher.stride(0),
+                               float(p), float(temperature), _ptr(loss), _ptr(row_kl), _ptr(dlogits),
+                               dlogits.stride(0) if dlogits is not None else V, float(grad_scale), _ptr(row_k),
+                               _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(dev))
+    _check(st, "qad_kl_topp_fwd_bwd")
+    return loss, row_kl, dlogits, row_k
 
 
 # ------------------------------------------------------------------ MSE calibration

@@ -199,6 +199,7 @@ struct KlArgs {
   void* dlogits;          // may be NULL
   int64_t ld_grad;
   int64_t topk;           // top-k kernel: entries of the teacher's top set per row
+  const int64_t* topk_rows = nullptr;  // top-k kernel: a k per row instead (device), when set
 };
 
 // Stand-in for positions of the shared-memory slice that hold no logit (the
@@ -741,7 +742,9 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topk_row_kernel(KlArgs args) 
   const int kw0 = wid * W;
 
   // ---- radix select of the k-th largest key over the row
-  const uint32_t kk = (uint32_t)(args.topk < args.vocab ? args.topk : args.vocab);
+  int64_t kreq = args.topk_rows != nullptr ? args.topk_rows[row] : args.topk;
+  if (kreq < 1) kreq = 1;
+  const uint32_t kk = (uint32_t)(kreq < args.vocab ? kreq : args.vocab);
   uint32_t prefix = 0, remaining = kk;
   for (int p = 0; p < PASSES; ++p) {
     // digit p: bf16 bits [15:7] then [6:0]; f32 8 bits at a time from the top
@@ -992,6 +995,261 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topk_row_kernel(KlArgs args) 
   }
 }
 
+// ------------------------------------------------------------------ top-p set size
+//
+// The Qwen3.6-35B-A3B W4A4 tutorial (section "5. 评估", on the runs that hit
+// the output-length cap) suggests selecting the teacher's top-p entries
+// instead of the top-k ones.  Per row, S is the shortest prefix of the top-k
+// order (decreasing teacher logit, equal logits by smaller index) whose
+// teacher probability at temperature T reaches p; the loss over S is the
+// top-k loss with k = |S|.  kl_topp_count_kernel finds |S| for every row with
+// the top-k kernel's cluster layout (teacher slice staged; the student is not
+// read) and a radix select over the same keys in which a bucket counts
+// teacher probability mass instead of entries.  The mass of a logit is
+// 2^((z - max z) a) in fixed point (2^40 for the largest logit), summed as
+// integers, so that the sums, and therefore the chosen set, do not depend on
+// the order of the additions.  A CTA's bucket sums are kept as two 32-bit
+// words (low word by a 32-bit atomic that returns the old value, the carry
+// and the high bits of the mass by a second, rare one); the cluster sums are
+// 64-bit.
+
+constexpr float kToppScale = 0x1p40f;
+
+// the logit whose order-preserving key is `key` (inverse of KlKey<T>::key)
+template <typename T>
+NVFP4_DEV float topp_key_value(uint32_t key);
+template <>
+NVFP4_DEV float topp_key_value<__nv_bfloat16>(uint32_t key) {
+  const uint32_t u = (key & 0x8000u) ? (key & 0x7FFFu) : (~key & 0xFFFFu);
+  return __uint_as_float(u << 16);
+}
+template <>
+NVFP4_DEV float topp_key_value<float>(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// fixed-point teacher mass of a logit, mw = a * (largest logit)
+NVFP4_DEV unsigned long long topp_mass(float z, float a, float mw) {
+  return (unsigned long long)__float2ull_rn(ex2(fmaf(z, a, -mw)) * kToppScale);
+}
+
+// The bucket (largest digit first) in which the cumulative mass reaches
+// `need` >= 1: thread t owns bins / kTopkThreads buckets (or one) from the
+// top; returns through s_* the digit, the mass and the count of the buckets
+// above it, and s_found = 0 when the buckets together hold less than `need`.
+NVFP4_DEV void topp_find_bucket(const unsigned long long* hm, const unsigned* hc, int bins,
+                                unsigned long long need, unsigned long long* warp_m, unsigned* warp_c,
+                                unsigned* s_digit, unsigned long long* s_before_m, unsigned* s_before_c,
+                                int* s_found) {
+  const int t = (int)threadIdx.x, lane = t & 31, wid = t >> 5;
+  const int per = bins > kTopkThreads ? bins / kTopkThreads : 1;
+  const int b_hi = bins - 1 - t * per;
+  unsigned long long mine_m = 0ull;
+  unsigned mine_c = 0u;
+  if (b_hi >= 0)
+    for (int i = 0; i < per; ++i) {
+      mine_m += hm[b_hi - i];
+      mine_c += hc[b_hi - i];
+    }
+  unsigned long long xm = mine_m;
+  unsigned xc = mine_c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long ym = __shfl_up_sync(0xFFFFFFFFu, xm, o);
+    const unsigned yc = __shfl_up_sync(0xFFFFFFFFu, xc, o);
+    if (lane >= o) {
+      xm += ym;
+      xc += yc;
+    }
+  }
+  if (lane == 31) {
+    warp_m[wid] = xm;
+    warp_c[wid] = xc;
+  }
+  if (t == 0) *s_found = 0;
+  __syncthreads();
+  unsigned long long before_m = xm - mine_m;
+  unsigned before_c = xc - mine_c;
+  for (int w = 0; w < wid; ++w) {
+    before_m += warp_m[w];
+    before_c += warp_c[w];
+  }
+  if (b_hi >= 0 && before_m < need && need <= before_m + mine_m) {
+    unsigned long long cm = before_m;
+    unsigned cc = before_c;
+    for (int i = 0; i < per; ++i) {
+      const int b = b_hi - i;
+      if (cm + hm[b] >= need) {
+        *s_digit = (unsigned)b;
+        *s_before_m = cm;
+        *s_before_c = cc;
+        *s_found = 1;
+        break;
+      }
+      cm += hm[b];
+      cc += hc[b];
+    }
+  }
+  __syncthreads();
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args, float top_p, int64_t* row_k) {
+  using E = KlElem<T>;
+  using Kf = KlKey<T>;
+  constexpr int V8 = E::kVec;
+  constexpr bool BF = sizeof(T) == 2;
+  constexpr int PASSES = BF ? 2 : 4;
+  constexpr int WPV = 4;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  __shared__ uint64_t bar;
+  __shared__ int s_ok, s_found;
+  __shared__ unsigned long long hist_m[512];  // cluster sums
+  __shared__ unsigned hist_lo[512], hist_hi[512], hist_c[512];
+  __shared__ unsigned recv_max[kKlMaxCluster];
+  __shared__ unsigned warp_max[kTopkWarps];
+  __shared__ unsigned long long warp_m[kTopkWarps];
+  __shared__ unsigned warp_c[kTopkWarps];
+  __shared__ unsigned s_digit, s_before_c;
+  __shared__ unsigned long long s_before_m, s_P;
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int csize = (int)cluster.num_blocks();
+  const int crank = (int)cluster.block_rank();
+  const int64_t row = blockIdx.x / csize;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t v0 = (int64_t)crank * args.slice;
+  int64_t v1 = v0 + args.slice;
+  if (v1 > args.vocab) v1 = args.vocab;
+  const int n = v1 > v0 ? (int)(v1 - v0) : 0;
+
+  T* st = reinterpret_cast<T*>(smem_raw);
+  // cluster exchange of the CTA histograms: low and high mass words and
+  // counts, [csize][512] each
+  unsigned* recv_lo = reinterpret_cast<unsigned*>(st + args.slice + 2 * V8);
+  unsigned* recv_hi = recv_lo + csize * 512;
+  unsigned* recv_c = recv_hi + csize * 512;
+  const KlSliceGeom geo = kl_stage_slice<T, kTopkThreads>(args, row, v0, n, st, nullptr, &bar, &s_ok);
+  const int off = geo.off, nslots = geo.nslots, nvec = geo.nvec;
+  const bool ok = s_ok != 0;
+  const uint32_t* wt = reinterpret_cast<const uint32_t*>(st);
+  const float a = args.a;
+
+  // ---- largest key of the row
+  uint32_t mk = 0u;
+  if (ok)
+    for (int k = (int)threadIdx.x; k < nvec; k += kTopkThreads)
+#pragma unroll
+      for (int q = 0; q < WPV; ++q) {
+        const uint32_t w = wt[k * WPV + q];
+#pragma unroll
+        for (int h = 0; h < Kf::kPerWord; ++h) {
+          const int j = k * V8 + q * Kf::kPerWord + h;
+          if (j >= off && j < nslots) mk = max(mk, Kf::key(w, h));
+        }
+      }
+  mk = __reduce_max_sync(0xFFFFFFFFu, mk);
+  if (lane == 0) warp_max[wid] = mk;
+  __syncthreads();
+  if ((int)threadIdx.x < csize) {
+    uint32_t c = warp_max[0];
+    for (int w = 1; w < kTopkWarps; ++w) c = max(c, warp_max[w]);
+    cluster.map_shared_rank(recv_max, (int)threadIdx.x)[crank] = c;
+  }
+  cluster.sync();
+  uint32_t kmax = recv_max[0];
+  for (int r = 1; r < csize; ++r) kmax = max(kmax, recv_max[r]);
+  const float mw = topp_key_value<T>(kmax) * a;
+
+  // ---- radix select on mass: the key tau at which the cumulative mass from
+  // the top reaches P = ceil(p * total mass)
+  uint32_t prefix = 0u;
+  unsigned long long above_m = 0ull, P = 0ull;
+  unsigned above_c = 0u, n_tau = 0u;
+  bool found = true;
+  for (int p = 0; p < PASSES && found; ++p) {
+    const int dbits = BF ? (p == 0 ? 9 : 7) : 8;
+    const int shift = BF ? (p == 0 ? 7 : 0) : Kf::kBits - 8 * (p + 1);
+    const int bins = 1 << dbits;
+    for (int b = (int)threadIdx.x; b < bins; b += kTopkThreads) {
+      hist_lo[b] = 0u;
+      hist_hi[b] = 0u;
+      hist_c[b] = 0u;
+    }
+    __syncthreads();
+    if (ok)
+      for (int k = (int)threadIdx.x; k < nvec; k += kTopkThreads)
+#pragma unroll
+        for (int q = 0; q < WPV; ++q) {
+          const uint32_t w = wt[k * WPV + q];
+#pragma unroll
+          for (int h = 0; h < Kf::kPerWord; ++h) {
+            const int j = k * V8 + q * Kf::kPerWord + h;
+            const uint32_t key = Kf::key(w, h);
+            if (j >= off && j < nslots && (p == 0 || (key >> (shift + dbits)) == prefix)) {
+              const unsigned b = (key >> shift) & (uint32_t)(bins - 1);
+              const unsigned long long q = topp_mass(topp_key_value<T>(key), a, mw);
+              const unsigned qlo = (unsigned)q, qhi = (unsigned)(q >> 32);
+              const unsigned old = atomicAdd(&hist_lo[b], qlo);
+              const unsigned up = qhi + (old + qlo < old ? 1u : 0u);  // high bits + carry
+              if (up != 0u) atomicAdd(&hist_hi[b], up);
+              atomicAdd(&hist_c[b], 1u);
+            }
+          }
+        }
+    __syncthreads();
+    for (int i = (int)threadIdx.x; i < csize * bins; i += kTopkThreads) {
+      const int r = i / bins, b = i - r * bins;
+      cluster.map_shared_rank(recv_lo, r)[crank * 512 + b] = hist_lo[b];
+      cluster.map_shared_rank(recv_hi, r)[crank * 512 + b] = hist_hi[b];
+      cluster.map_shared_rank(recv_c, r)[crank * 512 + b] = hist_c[b];
+    }
+    cluster.sync();
+    for (int b = (int)threadIdx.x; b < bins; b += kTopkThreads) {
+      unsigned long long tm = 0ull;
+      unsigned tc = 0u;
+      for (int r = 0; r < csize; ++r) {
+        tm += ((unsigned long long)recv_hi[r * 512 + b] << 32) | recv_lo[r * 512 + b];
+        tc += recv_c[r * 512 + b];
+      }
+      hist_m[b] = tm;
+      hist_c[b] = tc;
+    }
+    cluster.sync();  // every CTA has read its buffers before a peer writes the next digit's rows
+    if (p == 0) {
+      if (threadIdx.x == 0) {
+        unsigned long long tot = 0ull;
+        for (int b = 0; b < bins; ++b) tot += hist_m[b];
+        const unsigned long long need = (unsigned long long)ceil((double)top_p * (double)tot);
+        s_P = need > 0ull ? need : 1ull;
+      }
+      __syncthreads();
+      P = s_P;
+    }
+    topp_find_bucket(hist_m, hist_c, bins, P - above_m, warp_m, warp_c, &s_digit, &s_before_m, &s_before_c,
+                     &s_found);
+    found = s_found != 0;
+    if (found) {
+      above_m += s_before_m;
+      above_c += s_before_c;
+      prefix = (prefix << dbits) | s_digit;
+      n_tau = hist_c[s_digit];
+    }
+    __syncthreads();  // hist_*, s_* are rewritten by the next digit
+  }
+  if (crank == 0 && threadIdx.x == 0) {
+    int64_t m = args.vocab;
+    if (found && ok) {
+      const unsigned long long q_tau = topp_mass(topp_key_value<T>(prefix), a, mw);
+      unsigned long long r = q_tau > 0ull ? (P - above_m + q_tau - 1ull) / q_tau : (unsigned long long)n_tau;
+      if (r < 1ull) r = 1ull;
+      if (r > n_tau) r = n_tau;
+      m = (int64_t)above_c + (int64_t)r;
+    }
+    row_k[row] = m;
+  }
+}
+
 // loss = mean of row_kl in a fixed order (double accumulation); optionally
 // copies the per-row values to the caller's buffer.
 __global__ void __launch_bounds__(1024) kl_mean_kernel(const float* __restrict__ row_kl, int64_t rows,
@@ -1085,6 +1343,35 @@ static cudaError_t launch_kl_topk(const KlArgs& a, const KlPlan& p, cudaStream_t
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kl_topk_row_kernel<T>, a);
+}
+
+template <typename T>
+static cudaError_t launch_kl_topp_count(const KlArgs& a, const KlPlan& p, float top_p, int64_t* row_k,
+                                        cudaStream_t s) {
+  // the teacher slice, then the mass (u64) and count (u32) exchange buffers
+  const size_t smem = p.smem / 2 + (size_t)p.cluster * 512 * 12;
+  cudaError_t e =
+      cudaFuncSetAttribute(kl_topp_count_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(a.rows * p.cluster));
+  cfg.blockDim = dim3(kTopkThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kl_topp_count_kernel<T>, a, top_p, row_k);
+}
+
+// every entry of k[0..n) = v
+__global__ void fill_i64_kernel(int64_t* k, int64_t n, int64_t v) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    k[i] = v;
 }
 
 }  // namespace nvfp4
@@ -1182,6 +1469,67 @@ nvfp4_status qad_kl_topk_fwd_bwd(const void* teacher, const void* student, nvfp4
   if (e != cudaSuccess) return NVFP4_ERR_CUDA;
   kl_mean_kernel<<<1, 1024, 0, s>>>(args.row_kl, rows, loss, row_kl);
   count_launches(2);
+  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+size_t qad_kl_topp_workspace_size(int64_t rows, int64_t vocab, nvfp4_dtype dtype) {
+  return rows > 0 ? qad_kl_workspace_size(rows, vocab, dtype) + (size_t)rows * sizeof(int64_t) : 0;
+}
+
+nvfp4_status qad_kl_topp_fwd_bwd(const void* teacher, const void* student, nvfp4_dtype dtype, int64_t rows,
+                                 int64_t vocab, int64_t ld, float top_p, float temperature, float* loss,
+                                 float* row_kl, void* dlogits, int64_t ld_grad, float grad_scale, int64_t* row_k,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  NVFP4_ENTRY("qad_kl_topp_fwd_bwd");
+  if (dtype != NVFP4_BF16 && dtype != NVFP4_F32) return NVFP4_ERR_DTYPE;
+  if (!(temperature > 0.0f) || !loss || !(top_p > 0.0f)) return NVFP4_ERR_ARG;
+  if (rows < 0 || vocab <= 0 || ld < vocab) return NVFP4_ERR_SHAPE;
+  if (dlogits && ld_grad < vocab) return NVFP4_ERR_SHAPE;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (rows == 0) return cudaMemsetAsync(loss, 0, sizeof(float), s) == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+  if (!teacher || !student) return NVFP4_ERR_ARG;
+  if (rows > 0x7FFFFFFFll / kKlMaxCluster) return NVFP4_ERR_SHAPE;
+  const int esz = dtype == NVFP4_BF16 ? 2 : 4;
+  if (((uintptr_t)teacher ^ (uintptr_t)student) & 15u) return NVFP4_ERR_ALIGN;
+  if (((uintptr_t)teacher | (uintptr_t)student) % esz) return NVFP4_ERR_ALIGN;
+  if (dlogits && ((uintptr_t)dlogits % esz)) return NVFP4_ERR_ALIGN;
+  if (row_k && ((uintptr_t)row_k % sizeof(int64_t))) return NVFP4_ERR_ALIGN;
+  const size_t need = qad_kl_topp_workspace_size(rows, vocab, dtype);
+  if (!workspace || workspace_bytes < need) return NVFP4_ERR_WORKSPACE;
+  if (((uintptr_t)workspace & 15u) != 0) return NVFP4_ERR_ALIGN;
+  KlPlan plan;
+  if (!kl_plan(vocab, esz, plan)) return NVFP4_ERR_UNSUPPORTED;
+  KlArgs args;
+  args.teacher = teacher;
+  args.student = student;
+  args.rows = rows;
+  args.vocab = vocab;
+  args.ld = ld;
+  args.slice = plan.slice;
+  args.a = 1.4426950408889634f / temperature;
+  args.gscale = grad_scale / temperature;
+  args.row_kl = reinterpret_cast<float*>(workspace);
+  args.dlogits = dlogits;
+  args.ld_grad = ld_grad;
+  args.topk = vocab;
+  int64_t* ks = row_k ? row_k
+                      : reinterpret_cast<int64_t*>(static_cast<uint8_t*>(workspace) +
+                                                   qad_kl_workspace_size(rows, vocab, dtype));
+  cudaError_t e;
+  if (top_p >= 1.0f) {  // the whole row
+    const int64_t blocks = (rows + 255) / 256 < 1024 ? (rows + 255) / 256 : 1024;
+    fill_i64_kernel<<<(unsigned)blocks, 256, 0, s>>>(ks, rows, vocab);
+    e = cudaGetLastError();
+  } else {
+    e = dtype == NVFP4_BF16 ? launch_kl_topp_count<__nv_bfloat16>(args, plan, top_p, ks, s)
+                            : launch_kl_topp_count<float>(args, plan, top_p, ks, s);
+  }
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  args.topk_rows = ks;
+  e = dtype == NVFP4_BF16 ? launch_kl_topk<__nv_bfloat16>(args, plan, s) : launch_kl_topk<float>(args, plan, s);
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  kl_mean_kernel<<<1, 1024, 0, s>>>(args.row_kl, rows, loss, row_kl);
+  count_launches(3);
   return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 

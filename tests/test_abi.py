@@ -116,3 +116,23 @@ def test_timeout_selftest_rejects_unbounded_limits(lib):
     lib.nvfp4_selftest_timeout.argtypes = [ctypes.c_int64, ctypes.c_void_p]
     assert lib.nvfp4_selftest_timeout(0, None) == 1
     assert lib.nvfp4_selftest_timeout((1 << 32) + 1, None) == 1
+
+
+def test_topp_validates_before_any_launch(lib):
+    """Argument checks of qad_kl_topp_fwd_bwd return before touching the GPU."""
+    import nvfp4_quantization_aware_b200 as Q
+    L = Q.lib()
+    p = ctypes.c_void_p(64)
+    ws = ctypes.c_void_p(256)
+    need = L.qad_kl_topp_workspace_size(4, 100, 0)
+    assert need == L.qad_kl_workspace_size(4, 100, 0) + 4 * 8
+    assert L.qad_kl_topp_workspace_size(0, 100, 0) == 0
+    call = lambda top_p, T=1.0, row_k=None, wsb=need, dtype=0: L.qad_kl_topp_fwd_bwd(
+        p, p, dtype, 4, 100, 100, top_p, T, p, None, None, 100, 1.0, row_k, ws, wsb, None)
+    assert call(0.0) == 1                      # top_p must be > 0
+    assert call(-0.5) == 1
+    assert call(float("nan")) == 1
+    assert call(0.9, T=0.0) == 1               # temperature > 0
+    assert call(0.9, dtype=7) == 4             # dtype
+    assert call(0.9, wsb=need - 1) == 8        # workspace too small
+    assert call(0.9, row_k=ctypes.c_void_p(68)) == 3  # row_k not 8-byte aligned
