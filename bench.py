@@ -950,6 +950,10 @@ def run_profile_case(case: str):
         d = S.distill_logits(seed=0, device=dev, rows=2048)
         for _ in range(5):
             Q.qad_kl_topk_fwd_bwd(d["teacher"], d["student"], 4096)
+    elif case == "kl_topp":
+        d = S.distill_logits(seed=0, device=dev, rows=2048)
+        for _ in range(5):
+            Q.qad_kl_topp_fwd_bwd(d["teacher"], d["student"], 0.95)
     elif case == "w4a16":
         w = S.weights(4096, 4096, seed=1, device=dev)
         x = S.channel_scaled_activations(8192, 4096, seed=0, device=dev)
@@ -974,7 +978,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-secondary", action="store_true", help="skip the GEMM and KL measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["quant", "gemm", "gemm_small", "kl", "kl_topk", "w4a16", "calibrate", "moe"],
+    ap.add_argument("--profile", choices=["quant", "gemm", "gemm_small", "kl", "kl_topk", "kl_topp", "w4a16", "calibrate",
+                             "moe"],
                     default=None,
                     help="run one small single-kernel case (for ncu captures) and exit")
     args = ap.parse_args()

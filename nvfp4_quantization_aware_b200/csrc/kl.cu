@@ -1035,59 +1035,39 @@ NVFP4_DEV unsigned long long topp_mass(float z, float a, float mw) {
 
 // The bucket (largest digit first) in which the cumulative mass reaches
 // `need` >= 1: thread t owns bins / kTopkThreads buckets (or one) from the
-// top; returns through s_* the digit, the mass and the count of the buckets
-// above it, and s_found = 0 when the buckets together hold less than `need`.
-NVFP4_DEV void topp_find_bucket(const unsigned long long* hm, const unsigned* hc, int bins,
-                                unsigned long long need, unsigned long long* warp_m, unsigned* warp_c,
-                                unsigned* s_digit, unsigned long long* s_before_m, unsigned* s_before_c,
+// top; returns through s_* the digit and the mass of the buckets above it,
+// and s_found = 0 when the buckets together hold less than `need`.
+NVFP4_DEV void topp_find_bucket(const unsigned long long* hm, int bins, unsigned long long need,
+                                unsigned long long* warp_m, unsigned* s_digit, unsigned long long* s_before_m,
                                 int* s_found) {
   const int t = (int)threadIdx.x, lane = t & 31, wid = t >> 5;
   const int per = bins > kTopkThreads ? bins / kTopkThreads : 1;
   const int b_hi = bins - 1 - t * per;
-  unsigned long long mine_m = 0ull;
-  unsigned mine_c = 0u;
+  unsigned long long mine = 0ull;
   if (b_hi >= 0)
-    for (int i = 0; i < per; ++i) {
-      mine_m += hm[b_hi - i];
-      mine_c += hc[b_hi - i];
-    }
-  unsigned long long xm = mine_m;
-  unsigned xc = mine_c;
+    for (int i = 0; i < per; ++i) mine += hm[b_hi - i];
+  unsigned long long x = mine;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const unsigned long long ym = __shfl_up_sync(0xFFFFFFFFu, xm, o);
-    const unsigned yc = __shfl_up_sync(0xFFFFFFFFu, xc, o);
-    if (lane >= o) {
-      xm += ym;
-      xc += yc;
-    }
+    const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
   }
-  if (lane == 31) {
-    warp_m[wid] = xm;
-    warp_c[wid] = xc;
-  }
+  if (lane == 31) warp_m[wid] = x;
   if (t == 0) *s_found = 0;
   __syncthreads();
-  unsigned long long before_m = xm - mine_m;
-  unsigned before_c = xc - mine_c;
-  for (int w = 0; w < wid; ++w) {
-    before_m += warp_m[w];
-    before_c += warp_c[w];
-  }
-  if (b_hi >= 0 && before_m < need && need <= before_m + mine_m) {
-    unsigned long long cm = before_m;
-    unsigned cc = before_c;
+  unsigned long long before = x - mine;
+  for (int w = 0; w < wid; ++w) before += warp_m[w];
+  if (b_hi >= 0 && before < need && need <= before + mine) {
+    unsigned long long cm = before;
     for (int i = 0; i < per; ++i) {
       const int b = b_hi - i;
       if (cm + hm[b] >= need) {
         *s_digit = (unsigned)b;
         *s_before_m = cm;
-        *s_before_c = cc;
         *s_found = 1;
         break;
       }
       cm += hm[b];
-      cc += hc[b];
     }
   }
   __syncthreads();
@@ -1104,13 +1084,12 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ uint64_t bar;
   __shared__ int s_ok, s_found;
-  __shared__ unsigned long long hist_m[512];  // cluster sums
-  __shared__ unsigned hist_lo[512], hist_hi[512], hist_c[512];
+  __shared__ unsigned long long hist_m[512];   // cluster sums
+  __shared__ unsigned hist_lo[512], hist_hi[512];  // this CTA's sums: low word, high bits and carries
   __shared__ unsigned recv_max[kKlMaxCluster];
-  __shared__ unsigned warp_max[kTopkWarps];
+  __shared__ unsigned warp_u[2][kTopkWarps];
   __shared__ unsigned long long warp_m[kTopkWarps];
-  __shared__ unsigned warp_c[kTopkWarps];
-  __shared__ unsigned s_digit, s_before_c;
+  __shared__ unsigned s_digit;
   __shared__ unsigned long long s_before_m, s_P;
 
   cg::cluster_group cluster = cg::this_cluster();
@@ -1124,36 +1103,46 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
   const int n = v1 > v0 ? (int)(v1 - v0) : 0;
 
   T* st = reinterpret_cast<T*>(smem_raw);
-  // cluster exchange of the CTA histograms: low and high mass words and
-  // counts, [csize][512] each
-  unsigned* recv_lo = reinterpret_cast<unsigned*>(st + args.slice + 2 * V8);
+  const int nvec_max = (int)((args.slice + 2 * V8) / V8);
+  // bf16: high byte of each vector's largest valid key (0 when it has none)
+  uint8_t* vtop = reinterpret_cast<uint8_t*>(st + args.slice + 2 * V8);
+  // cluster exchange of the CTA histograms ([csize][512] low words, then
+  // [csize][512] high words), later of the CTA counts; then the warps'
+  // vector lists ([nvec_max])
+  unsigned* recv_lo = reinterpret_cast<unsigned*>(vtop + (nvec_max + 15) / 16 * 16);
   unsigned* recv_hi = recv_lo + csize * 512;
-  unsigned* recv_c = recv_hi + csize * 512;
+  unsigned* vlist = recv_hi + csize * 512;
   const KlSliceGeom geo = kl_stage_slice<T, kTopkThreads>(args, row, v0, n, st, nullptr, &bar, &s_ok);
   const int off = geo.off, nslots = geo.nslots, nvec = geo.nvec;
   const bool ok = s_ok != 0;
   const uint32_t* wt = reinterpret_cast<const uint32_t*>(st);
   const float a = args.a;
+  const int W = ((nvec + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;  // warp w lists vectors [w W, (w+1) W)
+  const int kw0 = wid * W;
 
-  // ---- largest key of the row
+  // ---- largest key of the row (and of every vector)
   uint32_t mk = 0u;
   if (ok)
-    for (int k = (int)threadIdx.x; k < nvec; k += kTopkThreads)
+    for (int k = (int)threadIdx.x; k < nvec; k += kTopkThreads) {
+      uint32_t vm = 0u;
 #pragma unroll
       for (int q = 0; q < WPV; ++q) {
         const uint32_t w = wt[k * WPV + q];
 #pragma unroll
         for (int h = 0; h < Kf::kPerWord; ++h) {
           const int j = k * V8 + q * Kf::kPerWord + h;
-          if (j >= off && j < nslots) mk = max(mk, Kf::key(w, h));
+          if (j >= off && j < nslots) vm = max(vm, Kf::key(w, h));
         }
       }
+      mk = max(mk, vm);
+      if (BF) vtop[k] = (uint8_t)(vm >> 8);
+    }
   mk = __reduce_max_sync(0xFFFFFFFFu, mk);
-  if (lane == 0) warp_max[wid] = mk;
+  if (lane == 0) warp_u[0][wid] = mk;
   __syncthreads();
   if ((int)threadIdx.x < csize) {
-    uint32_t c = warp_max[0];
-    for (int w = 1; w < kTopkWarps; ++w) c = max(c, warp_max[w]);
+    uint32_t c = warp_u[0][0];
+    for (int w = 1; w < kTopkWarps; ++w) c = max(c, warp_u[0][w]);
     cluster.map_shared_rank(recv_max, (int)threadIdx.x)[crank] = c;
   }
   cluster.sync();
@@ -1165,7 +1154,6 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
   // the top reaches P = ceil(p * total mass)
   uint32_t prefix = 0u;
   unsigned long long above_m = 0ull, P = 0ull;
-  unsigned above_c = 0u, n_tau = 0u;
   bool found = true;
   for (int p = 0; p < PASSES && found; ++p) {
     const int dbits = BF ? (p == 0 ? 9 : 7) : 8;
@@ -1174,48 +1162,52 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
     for (int b = (int)threadIdx.x; b < bins; b += kTopkThreads) {
       hist_lo[b] = 0u;
       hist_hi[b] = 0u;
-      hist_c[b] = 0u;
     }
     __syncthreads();
-    if (ok)
-      for (int k = (int)threadIdx.x; k < nvec; k += kTopkThreads)
+    auto add_key = [&](uint32_t key) {
+      const unsigned b = (key >> shift) & (uint32_t)(bins - 1);
+      const unsigned long long q = topp_mass(topp_key_value<T>(key), a, mw);
+      const unsigned qlo = (unsigned)q, qhi = (unsigned)(q >> 32);
+      const unsigned old = atomicAdd(&hist_lo[b], qlo);
+      const unsigned up = qhi + (old + qlo < old ? 1u : 0u);  // high bits + carry
+      if (up != 0u) atomicAdd(&hist_hi[b], up);
+    };
+    auto vector_keys = [&](int k, bool match) {
 #pragma unroll
-        for (int q = 0; q < WPV; ++q) {
-          const uint32_t w = wt[k * WPV + q];
+      for (int q = 0; q < WPV; ++q) {
+        const uint32_t w = wt[k * WPV + q];
 #pragma unroll
-          for (int h = 0; h < Kf::kPerWord; ++h) {
-            const int j = k * V8 + q * Kf::kPerWord + h;
-            const uint32_t key = Kf::key(w, h);
-            if (j >= off && j < nslots && (p == 0 || (key >> (shift + dbits)) == prefix)) {
-              const unsigned b = (key >> shift) & (uint32_t)(bins - 1);
-              const unsigned long long q = topp_mass(topp_key_value<T>(key), a, mw);
-              const unsigned qlo = (unsigned)q, qhi = (unsigned)(q >> 32);
-              const unsigned old = atomicAdd(&hist_lo[b], qlo);
-              const unsigned up = qhi + (old + qlo < old ? 1u : 0u);  // high bits + carry
-              if (up != 0u) atomicAdd(&hist_hi[b], up);
-              atomicAdd(&hist_c[b], 1u);
-            }
-          }
+        for (int h = 0; h < Kf::kPerWord; ++h) {
+          const int j = k * V8 + q * Kf::kPerWord + h;
+          const uint32_t key = Kf::key(w, h);
+          if (j >= off && j < nslots && (!match || (key >> (shift + dbits)) == prefix)) add_key(key);
         }
+      }
+    };
+    if (ok) {
+      if (BF && p == 1) {
+        // only the vectors whose largest key can lie in bucket `prefix`
+        const uint32_t top = prefix >> 1;
+        const unsigned len =
+            topk_warp_list(vlist, kw0, W, nvec, [&](int k) { return (uint32_t)vtop[k] >= top; });
+        for (unsigned i = lane; i < len; i += 32) vector_keys((int)vlist[kw0 + i], true);
+      } else {
+        for (int k = (int)threadIdx.x; k < nvec; k += kTopkThreads) vector_keys(k, p > 0);
+      }
+    }
     __syncthreads();
     for (int i = (int)threadIdx.x; i < csize * bins; i += kTopkThreads) {
       const int r = i / bins, b = i - r * bins;
       cluster.map_shared_rank(recv_lo, r)[crank * 512 + b] = hist_lo[b];
       cluster.map_shared_rank(recv_hi, r)[crank * 512 + b] = hist_hi[b];
-      cluster.map_shared_rank(recv_c, r)[crank * 512 + b] = hist_c[b];
     }
     cluster.sync();
     for (int b = (int)threadIdx.x; b < bins; b += kTopkThreads) {
       unsigned long long tm = 0ull;
-      unsigned tc = 0u;
-      for (int r = 0; r < csize; ++r) {
-        tm += ((unsigned long long)recv_hi[r * 512 + b] << 32) | recv_lo[r * 512 + b];
-        tc += recv_c[r * 512 + b];
-      }
+      for (int r = 0; r < csize; ++r) tm += ((unsigned long long)recv_hi[r * 512 + b] << 32) | recv_lo[r * 512 + b];
       hist_m[b] = tm;
-      hist_c[b] = tc;
     }
-    cluster.sync();  // every CTA has read its buffers before a peer writes the next digit's rows
+    cluster.sync();  // every CTA has read its buffers before a peer writes them again
     if (p == 0) {
       if (threadIdx.x == 0) {
         unsigned long long tot = 0ull;
@@ -1226,25 +1218,66 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
       __syncthreads();
       P = s_P;
     }
-    topp_find_bucket(hist_m, hist_c, bins, P - above_m, warp_m, warp_c, &s_digit, &s_before_m, &s_before_c,
-                     &s_found);
+    topp_find_bucket(hist_m, bins, P - above_m, warp_m, &s_digit, &s_before_m, &s_found);
     found = s_found != 0;
     if (found) {
       above_m += s_before_m;
-      above_c += s_before_c;
       prefix = (prefix << dbits) | s_digit;
-      n_tau = hist_c[s_digit];
     }
     __syncthreads();  // hist_*, s_* are rewritten by the next digit
+  }
+  // ---- keys above tau and equal to tau, counted over the row (found is the
+  // same in every CTA of the cluster)
+  unsigned n_gt = 0u, n_eq = 0u;
+  if (found) {
+    const uint32_t tau = prefix;
+    unsigned c_gt = 0u, c_eq = 0u;
+    if (ok)
+      for (int k = (int)threadIdx.x; k < nvec; k += kTopkThreads) {
+        if (BF && (uint32_t)vtop[k] < (tau >> 8)) continue;  // no key of this vector reaches tau
+#pragma unroll
+        for (int q = 0; q < WPV; ++q) {
+          const uint32_t w = wt[k * WPV + q];
+#pragma unroll
+          for (int h = 0; h < Kf::kPerWord; ++h) {
+            const int j = k * V8 + q * Kf::kPerWord + h;
+            const uint32_t key = Kf::key(w, h);
+            const bool in = j >= off && j < nslots;
+            c_gt += (in && key > tau) ? 1u : 0u;
+            c_eq += (in && key == tau) ? 1u : 0u;
+          }
+        }
+      }
+    c_gt = __reduce_add_sync(0xFFFFFFFFu, c_gt);
+    c_eq = __reduce_add_sync(0xFFFFFFFFu, c_eq);
+    if (lane == 0) {
+      warp_u[0][wid] = c_gt;
+      warp_u[1][wid] = c_eq;
+    }
+    __syncthreads();
+    if ((int)threadIdx.x < csize) {
+      unsigned g = 0u, e = 0u;
+      for (int w = 0; w < kTopkWarps; ++w) {
+        g += warp_u[0][w];
+        e += warp_u[1][w];
+      }
+      cluster.map_shared_rank(recv_lo, (int)threadIdx.x)[crank] = g;
+      cluster.map_shared_rank(recv_hi, (int)threadIdx.x)[crank] = e;
+    }
+    cluster.sync();
+    for (int r = 0; r < csize; ++r) {
+      n_gt += recv_lo[r];
+      n_eq += recv_hi[r];
+    }
   }
   if (crank == 0 && threadIdx.x == 0) {
     int64_t m = args.vocab;
     if (found && ok) {
       const unsigned long long q_tau = topp_mass(topp_key_value<T>(prefix), a, mw);
-      unsigned long long r = q_tau > 0ull ? (P - above_m + q_tau - 1ull) / q_tau : (unsigned long long)n_tau;
+      unsigned long long r = q_tau > 0ull ? (P - above_m + q_tau - 1ull) / q_tau : (unsigned long long)n_eq;
       if (r < 1ull) r = 1ull;
-      if (r > n_tau) r = n_tau;
-      m = (int64_t)above_c + (int64_t)r;
+      if (r > n_eq) r = n_eq;
+      m = (int64_t)n_gt + (int64_t)r;
     }
     row_k[row] = m;
   }
@@ -1348,8 +1381,11 @@ static cudaError_t launch_kl_topk(const KlArgs& a, const KlPlan& p, cudaStream_t
 template <typename T>
 static cudaError_t launch_kl_topp_count(const KlArgs& a, const KlPlan& p, float top_p, int64_t* row_k,
                                         cudaStream_t s) {
-  // the teacher slice, then the mass (u64) and count (u32) exchange buffers
-  const size_t smem = p.smem / 2 + (size_t)p.cluster * 512 * 12;
+  // the teacher slice, the vector tops (u8), the two exchange buffers
+  // ([cluster][512] u32 each) and the vector lists (u32)
+  const int vec = 16 / (int)sizeof(T);
+  const size_t nvec_max = (size_t)((p.slice + 2 * vec) / vec);
+  const size_t smem = p.smem / 2 + (nvec_max + 15) / 16 * 16 + (size_t)p.cluster * 512 * 8 + nvec_max * 4;
   cudaError_t e =
       cudaFuncSetAttribute(kl_topp_count_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
