@@ -1116,6 +1116,9 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
   const int off = geo.off, nslots = geo.nslots, nvec = geo.nvec;
   const bool ok = s_ok != 0;
   const uint32_t* wt = reinterpret_cast<const uint32_t*>(st);
+  const uint4* vt = reinterpret_cast<const uint4*>(st);
+  const int kfirst = (off + V8 - 1) / V8;  // vectors [kfirst, klast) hold no pad slot
+  const int klast = nslots / V8;
   const float a = args.a;
   const int W = ((nvec + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;  // warp w lists vectors [w W, (w+1) W)
   const int kw0 = wid * W;
@@ -1125,6 +1128,15 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
   if (ok)
     for (int k = (int)threadIdx.x; k < nvec; k += kTopkThreads) {
       uint32_t vm = 0u;
+      if (BF && k >= kfirst && k < klast) {  // interior bf16 vector: keys two at a time
+        const uint4 v = vt[k];
+        const uint32_t m2 = __vmaxu2(__vmaxu2(bf16x2_keys(v.x), bf16x2_keys(v.y)),
+                                     __vmaxu2(bf16x2_keys(v.z), bf16x2_keys(v.w)));
+        vm = max(m2 & 0xFFFFu, m2 >> 16);
+        mk = max(mk, vm);
+        vtop[k] = (uint8_t)(vm >> 8);
+        continue;
+      }
 #pragma unroll
       for (int q = 0; q < WPV; ++q) {
         const uint32_t w = wt[k * WPV + q];
@@ -1164,14 +1176,14 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
       hist_hi[b] = 0u;
     }
     __syncthreads();
-    auto add_key = [&](uint32_t key) {
-      const unsigned b = (key >> shift) & (uint32_t)(bins - 1);
-      const unsigned long long q = topp_mass(topp_key_value<T>(key), a, mw);
+    auto add_mass = [&](unsigned b, float z) {
+      const unsigned long long q = topp_mass(z, a, mw);
       const unsigned qlo = (unsigned)q, qhi = (unsigned)(q >> 32);
       const unsigned old = atomicAdd(&hist_lo[b], qlo);
       const unsigned up = qhi + (old + qlo < old ? 1u : 0u);  // high bits + carry
       if (up != 0u) atomicAdd(&hist_hi[b], up);
     };
+    auto add_key = [&](uint32_t key) { add_mass((key >> shift) & (uint32_t)(bins - 1), topp_key_value<T>(key)); };
     auto vector_keys = [&](int k, bool match) {
 #pragma unroll
       for (int q = 0; q < WPV; ++q) {
@@ -1192,7 +1204,20 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
             topk_warp_list(vlist, kw0, W, nvec, [&](int k) { return (uint32_t)vtop[k] >= top; });
         for (unsigned i = lane; i < len; i += 32) vector_keys((int)vlist[kw0 + i], true);
       } else {
-        for (int k = (int)threadIdx.x; k < nvec; k += kTopkThreads) vector_keys(k, p > 0);
+        for (int k = (int)threadIdx.x; k < nvec; k += kTopkThreads) {
+          if (BF && p == 0 && k >= kfirst && k < klast) {  // interior bf16 vector, first digit
+            const uint4 v = vt[k];
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t k2 = bf16x2_keys(w4[q]);
+              add_mass((k2 & 0xFFFFu) >> 7, __uint_as_float(w4[q] << 16));
+              add_mass(k2 >> 23, __uint_as_float(w4[q] & 0xFFFF0000u));
+            }
+            continue;
+          }
+          vector_keys(k, p > 0);
+        }
       }
     }
     __syncthreads();
