@@ -1033,15 +1033,18 @@ NVFP4_DEV unsigned long long topp_mass(float z, float a, float mw) {
   return (unsigned long long)__float2ull_rn(ex2(fmaf(z, a, -mw)) * kToppScale);
 }
 
+constexpr int kToppThreads = 512;  // two CTAs of 16 warps per SM (64 registers a thread)
+constexpr int kToppWarps = kToppThreads / 32;
+
 // The bucket (largest digit first) in which the cumulative mass reaches
-// `need` >= 1: thread t owns bins / kTopkThreads buckets (or one) from the
+// `need` >= 1: thread t owns bins / kToppThreads buckets (or one) from the
 // top; returns through s_* the digit and the mass of the buckets above it,
 // and s_found = 0 when the buckets together hold less than `need`.
 NVFP4_DEV void topp_find_bucket(const unsigned long long* hm, int bins, unsigned long long need,
                                 unsigned long long* warp_m, unsigned* s_digit, unsigned long long* s_before_m,
                                 int* s_found) {
   const int t = (int)threadIdx.x, lane = t & 31, wid = t >> 5;
-  const int per = bins > kTopkThreads ? bins / kTopkThreads : 1;
+  const int per = bins > kToppThreads ? bins / kToppThreads : 1;
   const int b_hi = bins - 1 - t * per;
   unsigned long long mine = 0ull;
   if (b_hi >= 0)
@@ -1074,7 +1077,7 @@ NVFP4_DEV void topp_find_bucket(const unsigned long long* hm, int bins, unsigned
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args, float top_p, int64_t* row_k) {
+__global__ void __launch_bounds__(kToppThreads, 2) kl_topp_count_kernel(KlArgs args, float top_p, int64_t* row_k) {
   using E = KlElem<T>;
   using Kf = KlKey<T>;
   constexpr int V8 = E::kVec;
@@ -1087,8 +1090,8 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
   __shared__ unsigned long long hist_m[512];   // cluster sums
   __shared__ unsigned hist_lo[512], hist_hi[512];  // this CTA's sums: low word, high bits and carries
   __shared__ unsigned recv_max[kKlMaxCluster];
-  __shared__ unsigned warp_u[2][kTopkWarps];
-  __shared__ unsigned long long warp_m[kTopkWarps];
+  __shared__ unsigned warp_u[2][kToppWarps];
+  __shared__ unsigned long long warp_m[kToppWarps];
   __shared__ unsigned s_digit;
   __shared__ unsigned long long s_before_m, s_P;
 
@@ -1112,7 +1115,7 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
   unsigned* recv_lo = reinterpret_cast<unsigned*>(vtop + (nvec_max + 15) / 16 * 16);
   unsigned* recv_hi = recv_lo + csize * 512;
   unsigned* vlist = recv_hi + csize * 512;
-  const KlSliceGeom geo = kl_stage_slice<T, kTopkThreads>(args, row, v0, n, st, nullptr, &bar, &s_ok);
+  const KlSliceGeom geo = kl_stage_slice<T, kToppThreads>(args, row, v0, n, st, nullptr, &bar, &s_ok);
   const int off = geo.off, nslots = geo.nslots, nvec = geo.nvec;
   const bool ok = s_ok != 0;
   const uint32_t* wt = reinterpret_cast<const uint32_t*>(st);
@@ -1120,13 +1123,13 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
   const int kfirst = (off + V8 - 1) / V8;  // vectors [kfirst, klast) hold no pad slot
   const int klast = nslots / V8;
   const float a = args.a;
-  const int W = ((nvec + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;  // warp w lists vectors [w W, (w+1) W)
+  const int W = ((nvec + kToppWarps - 1) / kToppWarps + 31) / 32 * 32;  // warp w lists vectors [w W, (w+1) W)
   const int kw0 = wid * W;
 
   // ---- largest key of the row (and of every vector)
   uint32_t mk = 0u;
   if (ok)
-    for (int k = (int)threadIdx.x; k < nvec; k += kTopkThreads) {
+    for (int k = (int)threadIdx.x; k < nvec; k += kToppThreads) {
       uint32_t vm = 0u;
       if (BF && k >= kfirst && k < klast) {  // interior bf16 vector: keys two at a time
         const uint4 v = vt[k];
@@ -1154,7 +1157,7 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
   __syncthreads();
   if ((int)threadIdx.x < csize) {
     uint32_t c = warp_u[0][0];
-    for (int w = 1; w < kTopkWarps; ++w) c = max(c, warp_u[0][w]);
+    for (int w = 1; w < kToppWarps; ++w) c = max(c, warp_u[0][w]);
     cluster.map_shared_rank(recv_max, (int)threadIdx.x)[crank] = c;
   }
   cluster.sync();
@@ -1171,7 +1174,7 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
     const int dbits = BF ? (p == 0 ? 9 : 7) : 8;
     const int shift = BF ? (p == 0 ? 7 : 0) : Kf::kBits - 8 * (p + 1);
     const int bins = 1 << dbits;
-    for (int b = (int)threadIdx.x; b < bins; b += kTopkThreads) {
+    for (int b = (int)threadIdx.x; b < bins; b += kToppThreads) {
       hist_lo[b] = 0u;
       hist_hi[b] = 0u;
     }
@@ -1204,7 +1207,7 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
             topk_warp_list(vlist, kw0, W, nvec, [&](int k) { return (uint32_t)vtop[k] >= top; });
         for (unsigned i = lane; i < len; i += 32) vector_keys((int)vlist[kw0 + i], true);
       } else {
-        for (int k = (int)threadIdx.x; k < nvec; k += kTopkThreads) {
+        for (int k = (int)threadIdx.x; k < nvec; k += kToppThreads) {
           if (BF && p == 0 && k >= kfirst && k < klast) {  // interior bf16 vector, first digit
             const uint4 v = vt[k];
             const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
@@ -1221,13 +1224,13 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
       }
     }
     __syncthreads();
-    for (int i = (int)threadIdx.x; i < csize * bins; i += kTopkThreads) {
+    for (int i = (int)threadIdx.x; i < csize * bins; i += kToppThreads) {
       const int r = i / bins, b = i - r * bins;
       cluster.map_shared_rank(recv_lo, r)[crank * 512 + b] = hist_lo[b];
       cluster.map_shared_rank(recv_hi, r)[crank * 512 + b] = hist_hi[b];
     }
     cluster.sync();
-    for (int b = (int)threadIdx.x; b < bins; b += kTopkThreads) {
+    for (int b = (int)threadIdx.x; b < bins; b += kToppThreads) {
       unsigned long long tm = 0ull;
       for (int r = 0; r < csize; ++r) tm += ((unsigned long long)recv_hi[r * 512 + b] << 32) | recv_lo[r * 512 + b];
       hist_m[b] = tm;
@@ -1258,7 +1261,7 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
     const uint32_t tau = prefix;
     unsigned c_gt = 0u, c_eq = 0u;
     if (ok)
-      for (int k = (int)threadIdx.x; k < nvec; k += kTopkThreads) {
+      for (int k = (int)threadIdx.x; k < nvec; k += kToppThreads) {
         if (BF && (uint32_t)vtop[k] < (tau >> 8)) continue;  // no key of this vector reaches tau
 #pragma unroll
         for (int q = 0; q < WPV; ++q) {
@@ -1282,7 +1285,7 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topp_count_kernel(KlArgs args
     __syncthreads();
     if ((int)threadIdx.x < csize) {
       unsigned g = 0u, e = 0u;
-      for (int w = 0; w < kTopkWarps; ++w) {
+      for (int w = 0; w < kToppWarps; ++w) {
         g += warp_u[0][w];
         e += warp_u[1][w];
       }
@@ -1416,7 +1419,7 @@ static cudaError_t launch_kl_topp_count(const KlArgs& a, const KlPlan& p, float 
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(a.rows * p.cluster));
-  cfg.blockDim = dim3(kTopkThreads);
+  cfg.blockDim = dim3(kToppThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
