@@ -271,7 +271,7 @@ def run_ours(args, world, rank, local):
         secondary["w4a16"] = bench_w4a16(Q, dev, stream, P, max(3, min(K, 20)))
         secondary["kl"] = bench_kl(Q, dev, stream, P, max(3, min(K, 10)))
         secondary["kl_topk"] = bench_kl_topk(Q, dev, stream, P, max(3, min(K, 10)))
-        secondary["kl_topp"] = bench_kl_topp(Q, dev, stream, max(3, min(K, 5)))
+        secondary["kl_topp"] = bench_kl_topp(Q, dev, stream, P, max(3, min(K, 5)))
         secondary["calibrate_mse"] = bench_calibrate(Q, dev, stream, xs, 3)
         secondary["moe_step"] = bench_moe(Q, dev, stream, P, max(3, min(K, 10)))
         # the FP4 probe runs last: its sustained launch (~70 ms at full tensor
@@ -803,7 +803,7 @@ def bench_kl_topk(Q, dev, stream, P, K, k=4096):
             "config": "distillation logits 16384 x 131072 bf16 (as kl), KL over the teacher's top-4096 per row"}
 
 
-def bench_kl_topp(Q, dev, stream, K, p=0.95):
+def bench_kl_topp(Q, dev, stream, P, K, p=0.95):
     """Top-p KL (the pages' suggested replacement for top-k) on the same
     distillation logits: tokens per second; also the mean set size."""
     from nvfp4_quantization_aware_b200 import synthetic as S
@@ -827,7 +827,13 @@ def bench_kl_topp(Q, dev, stream, K, p=0.95):
     ms = e0.elapsed_time(e1) / K
     del t, s, grad, d
     torch.cuda.empty_cache()
-    return {"tokens_per_s": round(rows / (ms * 1e-3), 1), "ms": round(ms, 4), "p": p, "mean_set_size": round(mean_k, 1),
+    gbs = 6.0 * rows * V / (ms * 1e-3) / 1e9
+    return {"tokens_per_s": round(rows / (ms * 1e-3), 1), "ms": round(ms, 4), "gbs": round(gbs, 1), "p": p,
+            "mean_set_size": round(mean_k, 1),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": P["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / P["hbm_gbs"], 4),
+                         "kernel": "kl_topp_count_kernel<bf16> + kl_topk_row_kernel<bf16> (whole loss)",
+                         "algorithmic_bytes_per_launch": 6 * rows * V},
             "config": "distillation logits 16384 x 131072 bf16 (as kl), KL over the teacher's top-p set per row "
                       "(set size kernel + top-k kernel with a k per row)"}
 
