@@ -728,7 +728,9 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topk_row_kernel(KlArgs args) 
   unsigned* vlist = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(vmax) + (nvec_max * 2 + 15) / 16 * 16);
   uint8_t* sel_mask = reinterpret_cast<uint8_t*>(vlist + nvec_max);  // bit e: element e of the vector is in S
   unsigned* recv_a = vlist;                                          // [csize][512], first digit only
-  const KlSliceGeom geo = kl_stage_slice<T, kTopkThreads>(args, row, v0, n, st, nullptr, &bar, &s_ok);
+  // the student's slice is prefetched into L2: the statistics and gradient
+  // passes read the vectors holding members of S, which cover most of its lines
+  const KlSliceGeom geo = kl_stage_slice<T, kTopkThreads>(args, row, v0, n, st, nullptr, &bar, &s_ok, true);
   const int off = geo.off, nslots = geo.nslots, nvec = geo.nvec;
   const int kfirst = (off + V8 - 1) / V8;  // vectors [kfirst, klast) hold no pad slot
   const int klast = nslots / V8;
