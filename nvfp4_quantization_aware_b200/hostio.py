@@ -83,6 +83,11 @@ class HostGroupedQuantizer:
         nc = len(self.chunks)
         self.ev_in = [torch.cuda.Event() for _ in range(nc)]
         self.ev_comp = [torch.cuda.Event() for _ in range(nc)]
+        # the device buffers are used on the side streams: when they are freed,
+        # the caching allocator waits for the work queued there
+        for t in [*self.dx, *self.d_codes, *self.d_sb, self.d_ts, self.workspace]:
+            for st in (self.s_in, self.s_comp, self.s_out):
+                t.record_stream(st)
 
     @property
     def h2d_bytes(self) -> int:
