@@ -632,60 +632,6 @@ NVFP4_DEV unsigned topk_warp_list(unsigned* list, int kw0, int W, int nvec, P pr
   return len;
 }
 
-// The largest slot index among the first `take` (in index order) keys equal
-// to tau of this CTA's slice, 0 < take < the CTA's count, where every such
-// key lies in a vector of the warps' lists (each list in index order, the
-// warps' ranges in index order): lanes own contiguous runs of their warp's
-// list, count their ties, scan the counts over the CTA, and the lane holding
-// the take-th tie finds its slot.  Writes *s_thr.
-template <typename T>
-NVFP4_DEV void topk_rank_ties(const uint32_t* wt, const unsigned* list, unsigned len, int kw0, int off, int nslots,
-                              uint32_t tau, unsigned take, unsigned* warp_tot, int* s_thr) {
-  using Kf = KlKey<T>;
-  constexpr int V8 = KlElem<T>::kVec;
-  constexpr int WPV = 4;
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const unsigned run = (len + 31u) / 32u;
-  const unsigned i0 = min((unsigned)lane * run, len), i1 = min(i0 + run, len);
-  unsigned c = 0u;
-  for (unsigned i = i0; i < i1; ++i) {
-    const int k = (int)list[kw0 + i];
-#pragma unroll
-    for (int q = 0; q < WPV; ++q) {
-      const uint32_t w = wt[k * WPV + q];
-#pragma unroll
-      for (int h = 0; h < Kf::kPerWord; ++h) {
-        const int j = k * V8 + q * Kf::kPerWord + h;
-        c += (j >= off && j < nslots && Kf::key(w, h) == tau) ? 1u : 0u;
-      }
-    }
-  }
-  unsigned x = c;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned y = __shfl_up_sync(0xFFFFFFFFu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) warp_tot[wid] = x;
-  __syncthreads();
-  unsigned before = x - c;
-  for (int w = 0; w < wid; ++w) before += warp_tot[w];
-  if (before < take && take <= before + c) {
-    unsigned seen = before;
-    for (unsigned i = i0; i < i1; ++i) {
-      const int k = (int)list[kw0 + i];
-      for (int q = 0; q < WPV; ++q) {
-        const uint32_t w = wt[k * WPV + q];
-        for (int h = 0; h < Kf::kPerWord; ++h) {
-          const int j = k * V8 + q * Kf::kPerWord + h;
-          if (j >= off && j < nslots && Kf::key(w, h) == tau && ++seen == take) *s_thr = j;
-        }
-      }
-    }
-  }
-  __syncthreads();
-}
-
 template <typename T>
 __global__ void __launch_bounds__(kTopkThreads) kl_topk_row_kernel(KlArgs args) {
   using E = KlElem<T>;
@@ -704,7 +650,6 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topk_row_kernel(KlArgs args) 
   __shared__ __align__(16) unsigned recv_b[kKlMaxCluster][256];
   __shared__ unsigned warp_sum[kTopkWarps];
   __shared__ unsigned s_digit, s_remaining, s_count;
-  __shared__ int s_thr;
   __shared__ KlStats warp_stats[kTopkWarps];
   __shared__ KlStats peer_stats[kKlMaxCluster];
 
@@ -841,20 +786,22 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topk_row_kernel(KlArgs args) 
     sel_mask[k] = 0u;
     return ok && (!BF || (uint32_t)vmax[k] >= tau);
   });
-  // slots j with key == tau belong to S iff j <= thr
-  int thr = take == n_mine ? 0x7FFFFFFF : -1;
-  if (take != 0u && take != n_mine) {  // CTA-uniform: this CTA holds the boundary among the ties
-    topk_rank_ties<T>(wt, vlist, len, kw0, off, nslots, tau, take, warp_sum, &s_thr);
-    thr = s_thr;
-  }
-  // ---- their selection masks; the list keeps (in place, in order) the
-  // vectors with a selected element
+  // ---- their selection masks.  Keys above tau are in S; keys equal to tau
+  // are when this CTA takes all of its ties, none when it takes none, and in
+  // the one CTA that takes some of them (CTA-uniform), the first `take` in
+  // index order: a first pass keeps each listed vector's tie bits in its list
+  // entry (bits 24..31; vector indices stay below 2^16), a scan over the warps
+  // gives each warp's first rank, and a second pass adds the ties below
+  // `take`.  Either way the list ends up holding (in place, in order) the
+  // vectors with a selected element.
+  const bool split_ties = take != 0u && take != n_mine;
+  const bool all_ties = take == n_mine;
   const unsigned lt_mask = (1u << lane) - 1u;
-  unsigned list_len = 0u;
+  unsigned list_len = 0u, ties_before = 0u;
   for (unsigned ib = 0; ib < len; ib += 32) {  // warp-uniform trip count
     const unsigned i = ib + lane;
     const int k = i < len ? (int)vlist[kw0 + i] : -1;
-    unsigned mask = 0u;
+    unsigned gt = 0u, eq = 0u;
     if (k >= 0) {
       const uint4 v = vt[k];
       const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
@@ -862,10 +809,9 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topk_row_kernel(KlArgs args) 
 #pragma unroll
         for (int q = 0; q < WPV; ++q) {
           const uint32_t k2 = bf16x2_keys(w4[q]);
-          const int j0 = k * V8 + 2 * q;
           const uint32_t k0 = k2 & 0xFFFFu, k1 = k2 >> 16;
-          mask |= (k0 > tau || (k0 == tau && j0 <= thr) ? 1u : 0u) << (2 * q);
-          mask |= (k1 > tau || (k1 == tau && j0 + 1 <= thr) ? 1u : 0u) << (2 * q + 1);
+          gt |= ((k0 > tau ? 1u : 0u) | (k1 > tau ? 2u : 0u)) << (2 * q);
+          eq |= ((k0 == tau ? 1u : 0u) | (k1 == tau ? 2u : 0u)) << (2 * q);
         }
       } else {
 #pragma unroll
@@ -875,15 +821,58 @@ __global__ void __launch_bounds__(kTopkThreads) kl_topk_row_kernel(KlArgs args) 
             const int e = q * Kf::kPerWord + h;
             const int j = k * V8 + e;
             const uint32_t key = Kf::key(w4[q], h);
-            const bool in = j >= off && j < nslots && (key > tau || (key == tau && j <= thr));
-            mask |= (in ? 1u : 0u) << e;
+            const bool valid = j >= off && j < nslots;
+            gt |= (valid && key > tau ? 1u : 0u) << e;
+            eq |= (valid && key == tau ? 1u : 0u) << e;
           }
       }
-      sel_mask[k] = (uint8_t)mask;
     }
-    const unsigned b = __ballot_sync(0xFFFFFFFFu, mask != 0u);  // every lane has read its entry
-    if (mask != 0u) vlist[kw0 + list_len + __popc(b & lt_mask)] = (unsigned)k;
-    list_len += __popc(b);
+    if (split_ties) {
+      if (k >= 0) {
+        sel_mask[k] = (uint8_t)gt;
+        vlist[kw0 + i] = (unsigned)k | (eq << 24);
+      }
+      ties_before += __reduce_add_sync(0xFFFFFFFFu, (unsigned)__popc(eq));
+    } else {
+      const unsigned mask = gt | (all_ties ? eq : 0u);
+      if (k >= 0) sel_mask[k] = (uint8_t)mask;
+      const unsigned b = __ballot_sync(0xFFFFFFFFu, mask != 0u);  // every lane has read its entry
+      if (mask != 0u) vlist[kw0 + list_len + __popc(b & lt_mask)] = (unsigned)k;
+      list_len += __popc(b);
+    }
+  }
+  if (split_ties) {  // CTA-uniform
+    if (lane == 0) warp_sum[wid] = ties_before;
+    __syncthreads();
+    unsigned rank = 0u;  // ties of this CTA in the warps before this one
+    for (int w = 0; w < wid; ++w) rank += warp_sum[w];
+    for (unsigned ib = 0; ib < len; ib += 32) {
+      const unsigned i = ib + lane;
+      const unsigned entry = i < len ? vlist[kw0 + i] : 0u;
+      const int k = i < len ? (int)(entry & 0xFFFFFFu) : -1;
+      unsigned eq = entry >> 24;
+      const unsigned c = (unsigned)__popc(eq);
+      unsigned x = c;  // inclusive scan of the tie counts over the lanes
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+        if (lane >= o) x += y;
+      }
+      const unsigned first = rank + x - c;  // rank of this vector's first tie
+      unsigned mask = 0u;
+      if (k >= 0) {
+        mask = sel_mask[k];
+        for (unsigned r = first; r < take && eq != 0u; ++r) {  // its ties ranked below `take`
+          mask |= eq & (0u - eq);
+          eq &= eq - 1u;
+        }
+        sel_mask[k] = (uint8_t)mask;
+      }
+      rank += __shfl_sync(0xFFFFFFFFu, x, 31);
+      const unsigned b = __ballot_sync(0xFFFFFFFFu, mask != 0u);  // every lane has read its entry
+      if (mask != 0u) vlist[kw0 + list_len + __popc(b & lt_mask)] = (unsigned)k;
+      list_len += __popc(b);
+    }
   }
   unsigned* sel_list = vlist;
   __syncthreads();
