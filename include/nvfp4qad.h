@@ -703,9 +703,9 @@ nvfp4_status qad_kl_topk_fwd_bwd(const void* teacher, const void* student, nvfp4
  * row weighs 2^40; exponentials from the hardware ex2), so |S| does not
  * depend on the order of the additions; against a float64 computation it can
  * differ only where the cumulative probability lies within ~1e-6 of top_p.
- * Two launches more than the top-k loss' first one: a pass over the teacher
- * logits that finds |S| (a radix select whose buckets hold probability mass),
- * then the top-k loss with a k per row.
+ * Three launches: a pass over the teacher logits that finds |S| (a radix
+ * select whose buckets hold probability mass; for top_p >= 1 a fill), the
+ * top-k loss kernel with that k per row, and the mean over the rows.
  * ------------------------------------------------------------------------ */
 size_t qad_kl_topp_workspace_size(int64_t rows, int64_t vocab, nvfp4_dtype dtype);
 
