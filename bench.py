@@ -16,6 +16,7 @@ Also measured in the same run and reported under "gemm" and "kl":
   * KL distillation loss + dLogits over 16384 x 131072 bf16 teacher/student
     logits -- tokens/s and GB/s (6 B per logit);
   * the top-k KL loss (key "kl_topk"): the same logits, k = 4096 per row;
+  * the top-p KL loss (key "kl_topp"): the same logits, p = 0.95;
   * weight-only NVFP4 (key "w4a16"): the same GEMM shapes with bf16
     activations, the weights dequantized in the main loop, beside W4A4 and
     the BF16 GEMM of the dequantized weights;
@@ -32,7 +33,13 @@ Timing: device time with CUDA events on the launching stream; the K timed
 steps are one CUDA-graph replay of K consecutive steps, bracketed by a
 barrier and synchronize; the maximum over ranks is reported.  Inputs are
 larger than L2 (1.07 GB), so no flush is needed between steps; the GEMM
-(25 MB of operands) is timed with an L2 flush before every launch.
+(25 MB of operands) cycles through copies of its weights (and, at M = 8192,
+of its activations) totalling more than twice the L2, so every launch reads
+its operands from HBM.
+
+"e2e" repeats the headline step through the public API from pinned host
+memory (HostGroupedQuantizer: host-to-device copies, both passes, and the
+codes and scales copied back, overlapped chunk by chunk).
 
 --impl reference times the CPU oracle (oracle/, test infrastructure) on the
 host cores on a bounded sample of the same workload.
