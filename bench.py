@@ -498,12 +498,29 @@ def bench_gemm(Q, dev, stream, P, K, probe=None):
             stream.synchronize()
             q_ms = statistics.mean(evs[k][0].elapsed_time(evs[k][1]) for k in range(steps))
             g_ms = statistics.mean(evs[k][1].elapsed_time(evs[k][2]) for k in range(steps))
+            del g
+            # the same quantize + GEMM pairs with no timing events between them
+            # (an event between two launches also keeps the second from starting
+            # early): one event pair around all steps
+            e0 = torch.cuda.Event(enable_timing=True, external=True)
+            e1 = torch.cuda.Event(enable_timing=True, external=True)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                e0.record(stream)
+                for k in range(steps):
+                    step(k)
+                    Q.nvfp4_gemm_w4a4(xc, xsf, xts, *ws[k % nw], out=c)
+                e1.record(stream)
+            g.replay()
+            stream.synchronize()
+            pair_ms = e0.elapsed_time(e1) / steps
             del g, xs
             flops = 2.0 * M * 4096 * 4096
             tflops = flops / (g_ms * 1e-3) / 1e12
             gemm_bytes = 4096 * 4096 * 0.5625 + M * 4096 * 0.5625 + M * 4096 * 2
             out[f"M{M}"] = {"tflops": round(tflops, 1), "gemm_ms": round(g_ms, 5), "x_quant_ms": round(q_ms, 5),
                             "end_to_end_tflops": round(flops / ((q_ms + g_ms) * 1e-3) / 1e12, 1),
+                            "x_quant_plus_gemm_ms": round(pair_ms, 5),
                             "gemm_gbs": round(gemm_bytes / (g_ms * 1e-3) / 1e9, 1),
                             "weight_copies": nw, "activation_copies": nx, "steps": steps,
                             "roofline": {"bound": "tensor" if M >= 1024 else "hbm",
