@@ -1196,7 +1196,21 @@ __global__ void __launch_bounds__(kToppThreads, 2) kl_topp_count_kernel(KlArgs a
         const uint32_t top = prefix >> 1;
         const unsigned len =
             topk_warp_list(vlist, kw0, W, nvec, [&](int k) { return (uint32_t)vtop[k] >= top; });
-        for (unsigned i = lane; i < len; i += 32) vector_keys((int)vlist[kw0 + i], true);
+        for (unsigned i = lane; i < len; i += 32) {
+          const int k = (int)vlist[kw0 + i];
+          if (BF && k >= kfirst && k < klast) {  // interior bf16 vector: two keys at a time
+            const uint4 v = vt[k];
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t k2 = bf16x2_keys(w4[q]);
+              if (((k2 & 0xFFFFu) >> 7) == prefix) add_mass(k2 & 0x7Fu, __uint_as_float(w4[q] << 16));
+              if ((k2 >> 23) == prefix) add_mass((k2 >> 16) & 0x7Fu, __uint_as_float(w4[q] & 0xFFFF0000u));
+            }
+            continue;
+          }
+          vector_keys(k, true);
+        }
       } else {
         for (int k = (int)threadIdx.x; k < nvec; k += kToppThreads) {
           if (BF && p == 0 && k >= kfirst && k < klast) {  // interior bf16 vector, first digit
@@ -1254,6 +1268,18 @@ __global__ void __launch_bounds__(kToppThreads, 2) kl_topp_count_kernel(KlArgs a
     if (ok)
       for (int k = (int)threadIdx.x; k < nvec; k += kToppThreads) {
         if (BF && (uint32_t)vtop[k] < (tau >> 8)) continue;  // no key of this vector reaches tau
+        if (BF && k >= kfirst && k < klast) {  // interior bf16 vector: two keys at a time
+          const uint4 v = vt[k];
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t k2 = bf16x2_keys(w4[q]);
+            const uint32_t k0 = k2 & 0xFFFFu, k1 = k2 >> 16;
+            c_gt += (k0 > tau ? 1u : 0u) + (k1 > tau ? 1u : 0u);
+            c_eq += (k0 == tau ? 1u : 0u) + (k1 == tau ? 1u : 0u);
+          }
+          continue;
+        }
 #pragma unroll
         for (int q = 0; q < WPV; ++q) {
           const uint32_t w = wt[k * WPV + q];
